@@ -1,0 +1,228 @@
+"""CPU oracle for the zero-computation-expert MoE layer.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` are the only callers.  Nothing in the product
+package imports this module, and this module imports nothing from the product.
+
+The arithmetic lives in ``zcmoe_oracle.c`` (plain C, fp64, plus an fp32 replica
+of the routing rule); this file builds it with gcc and wraps it with ctypes.
+Python here only marshals arrays, except ``layer_outputs`` which sums the
+per-expert fp64 results in numpy and ``brute_force_topk`` which enumerates
+subsets with itertools (tiny inputs only).
+
+Parity status: every function is pinned by tests under ``tests/`` (see
+test_oracle_pins.py) except the bias controller's convergence rate, which is
+"parity unpinned": the pages give no gains and no trajectory.
+"""
+from __future__ import annotations
+
+import ctypes
+import itertools
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "zcmoe_oracle.c")
+_SO = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+F32P = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
+F64P = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+I32P = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+I64P = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2 -ffp-contract=off, OpenMP)."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
+               "-fvisibility=hidden", "-o", _SO, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _SO
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_SO)
+        vp, i64, i32, f32, f64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_double
+        L.zo_router_logits.argtypes = [vp, i32, vp, i32, vp, i64, i32, i32, F64P]
+        L.zo_router_logits.restype = None
+        L.zo_softmax_f64.argtypes = [F64P, i64, i32, F64P]
+        L.zo_softmax_f64.restype = None
+        L.zo_topk_f64.argtypes = [F64P, vp, i64, i32, i32, f64, I32P, F64P, vp]
+        L.zo_topk_f64.restype = None
+        L.zo_zexp.argtypes = [f32]
+        L.zo_zexp.restype = f32
+        L.zo_route_replica_f32.argtypes = [F32P, vp, i64, i32, i32, f32, vp, I32P, F32P]
+        L.zo_route_replica_f32.restype = None
+        L.zo_integer_stage.argtypes = [I32P, i64, i32, i32, i32, I32P, I32P, I32P, I32P]
+        L.zo_integer_stage.restype = i64
+        L.zo_ffn_f64.argtypes = [vp, i32, i64, vp, vp, vp, i32, i32, i32, F64P]
+        L.zo_ffn_f64.restype = None
+        L.zo_layer_f64.argtypes = [vp, i32, i64, I32P, F64P, i32, i32, vp, vp, vp, i32, i32, i32, F64P]
+        L.zo_layer_f64.restype = None
+        L.zo_update_bias.argtypes = [I64P, I64P, i32, i32, i32, f32, f32, f32, f32, f32, F32P, F32P, F32P,
+                                     F32P, F32P]
+        L.zo_update_bias.restype = None
+        _lib = L
+    return _lib
+
+
+def _arr(a):
+    """(pointer, dtype code) for a float32 array or a uint16 bf16-bits array."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return a, 1
+    if a.dtype != np.float32:
+        raise TypeError(f"oracle inputs are float32 or bf16 bits (uint16), got {a.dtype}")
+    return a, 0
+
+
+def router_logits(x, wr, offset=None):
+    """fp64 logits l = x W_r^T + o.  x [T,d], wr [E,d] (float32 or bf16 bits)."""
+    x, xd = _arr(x)
+    wr, wd = _arr(wr)
+    T, d = x.shape
+    E = wr.shape[0]
+    out = np.empty((T, E), dtype=np.float64)
+    off = None if offset is None else np.ascontiguousarray(offset, dtype=np.float32)
+    lib().zo_router_logits(x.ctypes.data, xd, wr.ctypes.data, wd, None if off is None else off.ctypes.data,
+                           T, d, E, out)
+    return out
+
+
+def softmax(logits):
+    l = np.ascontiguousarray(logits, dtype=np.float64)
+    T, E = l.shape
+    out = np.empty_like(l)
+    lib().zo_softmax_f64(l, T, E, out)
+    return out
+
+
+def topk(scores, bias, k, scale=1.0):
+    """fp64 bias-shifted top-k.  Returns idx [T,k] int32, gate [T,k] f64, margin [T] f64."""
+    s = np.ascontiguousarray(scores, dtype=np.float64)
+    T, E = s.shape
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float64)
+    idx = np.empty((T, k), dtype=np.int32)
+    gate = np.empty((T, k), dtype=np.float64)
+    margin = np.empty(T, dtype=np.float64)
+    lib().zo_topk_f64(s, None if b is None else b.ctypes.data, T, E, k, float(scale), idx, gate, margin.ctypes.data)
+    return idx, gate, margin
+
+
+def zexp(x: float) -> float:
+    return float(lib().zo_zexp(float(x)))
+
+
+def route_replica_f32(logits_f32, bias_f32, k, scale=1.0, want_scores=False):
+    """fp32 replica of the routing rule, fed fp32 logits.  Returns (idx, gate, scores|None)."""
+    l = np.ascontiguousarray(logits_f32, dtype=np.float32)
+    T, E = l.shape
+    b = None if bias_f32 is None else np.ascontiguousarray(bias_f32, dtype=np.float32)
+    idx = np.empty((T, k), dtype=np.int32)
+    gate = np.empty((T, k), dtype=np.float32)
+    scores = np.empty((T, E), dtype=np.float32) if want_scores else None
+    lib().zo_route_replica_f32(l, None if b is None else b.ctypes.data, T, E, k, float(scale),
+                               None if scores is None else scores.ctypes.data, idx, gate)
+    return idx, gate, scores
+
+
+def integer_stage(idx, N, E):
+    """counts [E], offsets [N+1], perm [P] (entries t*k+j), pos [T,k] (-1 for zero slots)."""
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    T, k = idx.shape
+    counts = np.empty(E, dtype=np.int32)
+    offsets = np.empty(N + 1, dtype=np.int32)
+    perm = np.empty(max(T * k, 1), dtype=np.int32)
+    pos = np.empty((T, k), dtype=np.int32)
+    P = lib().zo_integer_stage(idx, T, k, N, E, counts, offsets, perm, pos)
+    return counts, offsets, perm[:P].copy(), pos
+
+
+def ffn(xs, wg, wu, wd):
+    """fp64 SwiGLU expert on rows xs [n,d]; wg,wu [inter,d], wd [d,inter]."""
+    xs, xd = _arr(xs)
+    wg, gd = _arr(wg)
+    wu, _ = _arr(wu)
+    wd_, _ = _arr(wd)
+    n, d = xs.shape
+    inter = wg.shape[0]
+    out = np.empty((n, d), dtype=np.float64)
+    lib().zo_ffn_f64(xs.ctypes.data, xd, n, wg.ctypes.data, wu.ctypes.data, wd_.ctypes.data, gd, d, inter, out)
+    return out
+
+
+def layer(x, idx, gate, N, wg, wu, wd):
+    """fp64 layer output for all tokens, all weights in memory."""
+    x, xd = _arr(x)
+    wg, gd = _arr(wg)
+    wu, _ = _arr(wu)
+    wd_, _ = _arr(wd)
+    T, d = x.shape
+    k = idx.shape[1]
+    inter = wg.shape[1]
+    y = np.empty((T, d), dtype=np.float64)
+    lib().zo_layer_f64(x.ctypes.data, xd, T, np.ascontiguousarray(idx, dtype=np.int32),
+                       np.ascontiguousarray(gate, dtype=np.float64), k, N, wg.ctypes.data, wu.ctypes.data,
+                       wd_.ctypes.data, gd, d, inter, y)
+    return y
+
+
+def layer_outputs(x_rows, idx, gate, N, expert_weights):
+    """fp64 layer output for a few tokens when the expert weights are fetched one
+    expert at a time.  ``expert_weights(e) -> (wg, wu, wd)``.  Sums
+    g * F_e(x) over the token's FFN slots plus (sum of zero-slot gates) * x."""
+    x_rows = np.ascontiguousarray(x_rows)
+    n, d = x_rows.shape
+    xf = x_rows.astype(np.float64) if x_rows.dtype == np.float32 else \
+        (x_rows.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    y = np.zeros((n, d), dtype=np.float64)
+    zsum = np.zeros(n, dtype=np.float64)
+    users = {}
+    for r in range(n):
+        for j in range(idx.shape[1]):
+            e = int(idx[r, j])
+            if e >= N:
+                zsum[r] += float(gate[r, j])
+            else:
+                users.setdefault(e, []).append((r, j))
+    for e in sorted(users):
+        wg, wu, wd = expert_weights(e)
+        rows = [r for r, _ in users[e]]
+        f = ffn(x_rows[rows], wg, wu, wd)
+        for i, (r, j) in enumerate(users[e]):
+            y[r] += float(gate[r, j]) * f[i]
+    y += zsum[:, None] * xf
+    return y
+
+
+def update_bias(counts, tokens, N, Z, k, gains, b0, state):
+    """One controller step in place.  counts int64 [E], tokens int64 [1];
+    gains = (kp, ki, kd, decay, target_ffn); state = dict(eta [1], integ [E], eprev [E], bias [E])."""
+    kp, ki, kd, decay, target = gains
+    lib().zo_update_bias(counts, tokens, N, Z, k, kp, ki, kd, decay, target, np.ascontiguousarray(b0, np.float32),
+                         state["eta"], state["integ"], state["eprev"], state["bias"])
+
+
+def new_controller_state(b0):
+    E = len(b0)
+    return {"eta": np.ones(1, np.float32), "integ": np.zeros(E, np.float32), "eprev": np.zeros(E, np.float32),
+            "bias": np.array(b0, dtype=np.float32)}
+
+
+def brute_force_topk(v, k):
+    """Enumerate all k-subsets of v (tiny E only); the chosen set maximises sum(v)
+    with ties broken towards the lexicographically smaller sorted index tuple.
+    Returns the indices ordered by v descending, then index ascending."""
+    E = len(v)
+    best, best_sum = None, None
+    for comb in itertools.combinations(range(E), k):
+        s = sum(float(v[i]) for i in comb)
+        if best is None or s > best_sum:
+            best, best_sum = comb, s
+    return sorted(best, key=lambda i: (-float(v[i]), i))

@@ -1,0 +1,348 @@
+/*
+ * Oracle for the zero-computation-expert MoE layer forward pass.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU-baseline
+ * leg of the benchmark may load this library.  It shares no code, header or
+ * constant table with the CUDA library; the two are written separately from the
+ * same definitions.
+ *
+ * Plain, slow, obviously correct C.  Floating point is fp64 unless a function
+ * says it replicates the fp32 routing rule.  Built with -O2 -ffp-contract=off
+ * (no fused multiply-add except where fma() is written out) and no fast-math.
+ *
+ * Sources (page title, section):
+ *  - LongCat-Flash technical summary (zhangjingwei.cn), section 二 架構, part 1
+ *    "零計算專家": Z zero-computation experts that only return their input; an
+ *    expert-specific bias, driven by a PID controller, shifts the routing scores
+ *    to keep the FFN/zero selection ratio near a target; corpus-level balance.
+ *  - same page, 模型配置: 512 FFN experts + 256 zero experts, 12 activated per
+ *    token, hidden 6144, expert intermediate 2048.
+ *  - LongCat-Flash tech-report thread (web3.cnouyi.fund): the bias works like
+ *    DeepSeek-V3's auxiliary-loss-free balancing (bias in selection only) with a
+ *    decay schedule on its update.
+ *  - LongCat-Flash-Lite N-gram article (onthewifi.com), part 02: the router is a
+ *    fused "softmax + top-k + scaling" step.
+ *
+ * Readings where the pages are silent (each is listed with its reason in the
+ * design notes): softmax over all N+Z experts; top-k on score+bias, ties to the
+ * lower expert index, slots ordered by biased score then index; gate = scale *
+ * unbiased score, no renormalisation; zero expert output = its input; FFN expert
+ * = SwiGLU, W_d (silu(W_g x) * (W_u x)), no biases; FFN experts are ids 0..N-1,
+ * zero experts N..N+Z-1; positional PID on the per-expert load error.
+ *
+ * Parity status of each function is stated beside it; pins live in tests/.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ZO_EXPORT __attribute__((visibility("default")))
+
+/* ------------------------------------------------------------------------- */
+/* Input element access: dtype 0 = float32, 1 = bf16 bit patterns (uint16).   */
+/* bf16 -> float is exact (the 16 bits become the high half of the float).   */
+/* ------------------------------------------------------------------------- */
+static double elem(const void *p, int dtype, int64_t i) {
+  if (dtype == 1) {
+    uint32_t u = ((uint32_t)((const uint16_t *)p)[i]) << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+  }
+  return (double)((const float *)p)[i];
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 1: router logits  l[t,e] = sum_c x[t,c] W_r[e,c] + o[e]   (fp64)      */
+/* Page: onthewifi.com part 02 (router logits feed softmax+top-k);            */
+/* zhangjingwei.cn 二.1 (routing scores).  Pinned: tests/test_oracle_pins.py  */
+/* ------------------------------------------------------------------------- */
+ZO_EXPORT void zo_router_logits(const void *x, int x_dtype, const void *wr, int w_dtype,
+                                const float *offset, int64_t T, int d, int E, double *logits) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int c = 0; c < d; ++c) acc += elem(x, x_dtype, t * d + c) * elem(wr, w_dtype, (int64_t)e * d + c);
+      if (offset) acc += (double)offset[e];
+      logits[t * E + e] = acc;
+    }
+  }
+}
+
+/* Step 2: s = softmax(l) over all E experts, fp64. */
+ZO_EXPORT void zo_softmax_f64(const double *l, int64_t T, int E, double *s) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    const double *lt = l + t * E;
+    double m = lt[0];
+    for (int e = 1; e < E; ++e)
+      if (lt[e] > m) m = lt[e];
+    double sum = 0.0;
+    for (int e = 0; e < E; ++e) sum += exp(lt[e] - m);
+    for (int e = 0; e < E; ++e) s[t * E + e] = exp(lt[e] - m) / sum;
+  }
+}
+
+/* Steps 3-5 (fp64): v = s + b; S = the k largest v, ties to the lower index,
+ * slot order v descending then index ascending; gate = scale * s (bias never in
+ * the gate, no renormalisation).  margin[t] = v_(k) - v_(k+1) (+inf if k == E),
+ * used to exclude near-ties from index comparison.
+ * Page: web3.cnouyi.fund (DSv3-like bias in selection); zhangjingwei.cn 二.1. */
+ZO_EXPORT void zo_topk_f64(const double *s, const double *bias, int64_t T, int E, int k, double scale,
+                           int32_t *idx, double *gate, double *margin) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    const double *st = s + t * E;
+    unsigned char *taken = (unsigned char *)calloc((size_t)E, 1);
+    double last = 0.0;
+    for (int j = 0; j < k; ++j) {
+      int best = -1;
+      double bv = 0.0;
+      for (int e = 0; e < E; ++e) {
+        if (taken[e]) continue;
+        double v = st[e] + (bias ? bias[e] : 0.0);
+        if (best < 0 || v > bv) { best = e; bv = v; } /* strict '>' keeps the lower index on ties */
+      }
+      taken[best] = 1;
+      idx[t * k + j] = best;
+      gate[t * k + j] = scale * st[best];
+      last = bv;
+    }
+    if (margin) {
+      double next = -INFINITY;
+      int found = 0;
+      for (int e = 0; e < E; ++e) {
+        if (taken[e]) continue;
+        double v = st[e] + (bias ? bias[e] : 0.0);
+        if (!found || v > next) { next = v; found = 1; }
+      }
+      margin[t] = found ? last - next : INFINITY;
+    }
+    free(taken);
+  }
+}
+
+/* ------------------------------------------------------------------------- */
+/* fp32 routing replica.                                                     */
+/*                                                                           */
+/* Integer results (indices, counts, permutation) are decided by fp32        */
+/* comparisons, so this replica takes the same decisions in the same         */
+/* precision as the device kernel, from the same written rule:               */
+/*   m = max_e l_e;  u_e = zexp(l_e - m)                                     */
+/*   sum: 32 partials, partial[p] = sum over e = p, p+32, ... (ascending);   */
+/*        then for w = 16,8,4,2,1: partial[p] = partial[p] + partial[p^w]    */
+/*   s_e = u_e / partial[0];  v_e = s_e + b_e;  top-k as in zo_topk_f64;     */
+/*   gate = scale * s.   Every operation rounds once to fp32.                */
+/* zexp: Cody-Waite reduction with ln2 split into C1 (ln2 truncated to 16    */
+/* significant bits, so n*C1 is exact for |n| < 256) and C2 = fl32(ln2-C1),  */
+/* n = rint(x * fl32(1/ln2)); degree-7 Taylor polynomial (coefficients       */
+/* fl32(1/i!)) in Horner form with explicit fma; scaled by 2^n through the   */
+/* exponent bits; results below 2^-125 flush to zero.  Pinned against libm   */
+/* exp to <= 2 ulp in tests.                                                 */
+/* ------------------------------------------------------------------------- */
+ZO_EXPORT float zo_zexp(float x) {
+  const float L2E = 0x1.715476p+0f;
+  const float C1 = 0x1.62e4p-1f;
+  const float C2 = 0x1.7f7d1cp-20f;
+  if (!(x > -88.0f)) return 0.0f;
+  float n = rintf(x * L2E);
+  if (n < -125.0f) return 0.0f;
+  if (n > 127.0f) return INFINITY;
+  float r = fmaf(-n, C1, x);
+  r = fmaf(-n, C2, r);
+  float p = 0x1.a01a02p-13f;    /* 1/7! */
+  p = fmaf(p, r, 0x1.6c16c2p-10f); /* 1/6! */
+  p = fmaf(p, r, 0x1.111112p-7f);  /* 1/5! */
+  p = fmaf(p, r, 0x1.555556p-5f);  /* 1/4! */
+  p = fmaf(p, r, 0x1.555556p-3f);  /* 1/3! */
+  p = fmaf(p, r, 0.5f);
+  p = fmaf(p, r, 1.0f);
+  p = fmaf(p, r, 1.0f);
+  int ni = (int)n;
+  uint32_t bits = (uint32_t)(ni + 127) << 23;
+  float scale;
+  memcpy(&scale, &bits, 4);
+  return p * scale;
+}
+
+ZO_EXPORT void zo_route_replica_f32(const float *logits, const float *bias, int64_t T, int E, int k,
+                                    float scale, float *scores, int32_t *idx, float *gate) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    const float *lt = logits + t * E;
+    float *u = (float *)malloc(sizeof(float) * (size_t)E);
+    unsigned char *taken = (unsigned char *)calloc((size_t)E, 1);
+    float m = lt[0];
+    for (int e = 1; e < E; ++e)
+      if (lt[e] > m) m = lt[e];
+    for (int e = 0; e < E; ++e) u[e] = zo_zexp(lt[e] - m);
+    float part[32];
+    for (int p = 0; p < 32; ++p) {
+      float acc = 0.0f;
+      for (int e = p; e < E; e += 32) acc = acc + u[e];
+      part[p] = acc;
+    }
+    for (int w = 16; w >= 1; w >>= 1) {
+      float nxt[32];
+      for (int p = 0; p < 32; ++p) nxt[p] = part[p] + part[p ^ w];
+      memcpy(part, nxt, sizeof(part));
+    }
+    const float sum = part[0];
+    for (int e = 0; e < E; ++e) u[e] = u[e] / sum; /* u now holds s */
+    if (scores)
+      for (int e = 0; e < E; ++e) scores[t * E + e] = u[e];
+    for (int j = 0; j < k; ++j) {
+      int best = -1;
+      float bv = 0.0f;
+      for (int e = 0; e < E; ++e) {
+        if (taken[e]) continue;
+        float v = u[e] + (bias ? bias[e] : 0.0f);
+        if (best < 0 || v > bv) { best = e; bv = v; }
+      }
+      taken[best] = 1;
+      idx[t * k + j] = best;
+      gate[t * k + j] = scale * u[best];
+    }
+    free(taken);
+    free(u);
+  }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Integer stage (exact).  counts[e] over all E experts; offsets = exclusive */
+/* scan over FFN experts 0..N-1 (offsets[N] = P, the FFN pairs); perm lists  */
+/* the FFN pairs ordered by (expert asc, token asc), each entry t*k + j;     */
+/* pos[t*k+j] = its place in perm, or -1 for a zero-expert slot.             */
+/* Zero experts are routed to no expert computation at all (they cost        */
+/* nothing, zhangjingwei.cn 二.1), so only FFN pairs enter the permutation.  */
+/* ------------------------------------------------------------------------- */
+ZO_EXPORT int64_t zo_integer_stage(const int32_t *idx, int64_t T, int k, int N, int E, int32_t *counts,
+                                   int32_t *offsets, int32_t *perm, int32_t *pos) {
+  for (int e = 0; e < E; ++e) counts[e] = 0;
+  for (int64_t i = 0; i < T * k; ++i) counts[idx[i]]++;
+  offsets[0] = 0;
+  for (int e = 0; e < N; ++e) offsets[e + 1] = offsets[e] + counts[e];
+  int32_t *fill = (int32_t *)calloc((size_t)N, sizeof(int32_t));
+  for (int64_t t = 0; t < T; ++t) {
+    for (int j = 0; j < k; ++j) {
+      int e = idx[t * k + j];
+      if (e < N) {
+        int32_t p = offsets[e] + fill[e]++;
+        perm[p] = (int32_t)(t * k + j);
+        pos[t * k + j] = p;
+      } else {
+        pos[t * k + j] = -1;
+      }
+    }
+  }
+  free(fill);
+  return offsets[N];
+}
+
+/* ------------------------------------------------------------------------- */
+/* FFN expert (SwiGLU), fp64:  F(x) = W_d (silu(W_g x) * (W_u x)),           */
+/* silu(z) = z / (1 + exp(-z)).  W_g, W_u are [inter, d]; W_d is [d, inter]. */
+/* out[r, :] = F(xs[r, :]) for n rows.                                        */
+/* ------------------------------------------------------------------------- */
+ZO_EXPORT void zo_ffn_f64(const void *xs, int x_dtype, int64_t n, const void *wg, const void *wu,
+                          const void *wd, int w_dtype, int d, int inter, double *out) {
+#pragma omp parallel for schedule(dynamic)
+  for (int64_t r = 0; r < n; ++r) {
+    double *h = (double *)malloc(sizeof(double) * (size_t)inter);
+    for (int i = 0; i < inter; ++i) {
+      double g = 0.0, u = 0.0;
+      for (int c = 0; c < d; ++c) {
+        const double xv = elem(xs, x_dtype, r * d + c);
+        g += elem(wg, w_dtype, (int64_t)i * d + c) * xv;
+        u += elem(wu, w_dtype, (int64_t)i * d + c) * xv;
+      }
+      h[i] = g / (1.0 + exp(-g)) * u;
+    }
+    for (int c = 0; c < d; ++c) {
+      double acc = 0.0;
+      for (int i = 0; i < inter; ++i) acc += elem(wd, w_dtype, (int64_t)c * inter + i) * h[i];
+      out[r * d + c] = acc;
+    }
+    free(h);
+  }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Whole layer output for tokens with all weights in memory (small configs): */
+/* y_t = sum_{j: e_j < N} g_j F_{e_j}(x_t) + (sum_{j: e_j >= N} g_j) x_t.     */
+/* Zero experts return x unchanged (zhangjingwei.cn 二.1).                    */
+/* wg/wu: [N, inter, d], wd: [N, d, inter].                                  */
+/* ------------------------------------------------------------------------- */
+ZO_EXPORT void zo_layer_f64(const void *x, int x_dtype, int64_t T, const int32_t *idx, const double *gate,
+                            int k, int N, const void *wg, const void *wu, const void *wd, int w_dtype, int d,
+                            int inter, double *y) {
+  const int64_t wsz = (int64_t)inter * d;
+  const size_t esz = (w_dtype == 1) ? 2 : 4;
+  const size_t xsz = (x_dtype == 1) ? 2 : 4;
+  for (int64_t t = 0; t < T; ++t) {
+    double *yt = y + t * d;
+    for (int c = 0; c < d; ++c) yt[c] = 0.0;
+    double zsum = 0.0;
+    double *f = (double *)malloc(sizeof(double) * (size_t)d);
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[t * k + j];
+      const double g = gate[t * k + j];
+      if (e >= N) {
+        zsum += g;
+        continue;
+      }
+      zo_ffn_f64((const char *)x + (size_t)(t * d) * xsz, x_dtype, 1, (const char *)wg + (size_t)(e * wsz) * esz,
+                 (const char *)wu + (size_t)(e * wsz) * esz, (const char *)wd + (size_t)(e * wsz) * esz, w_dtype,
+                 d, inter, f);
+      for (int c = 0; c < d; ++c) yt[c] += g * f[c];
+    }
+    for (int c = 0; c < d; ++c) yt[c] += zsum * elem(x, x_dtype, t * d + c);
+    free(f);
+  }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Bias controller (fp32, every operation rounded once, no fma).             */
+/* zhangjingwei.cn 二.1: a PID controller sets expert-specific bias terms so  */
+/* the FFN/zero selection ratio stays near its target; corpus-level balance; */
+/* web3.cnouyi.fund: a decay schedule on the bias update.  Reading:          */
+/*   load  l_i = fl32(c_i) / fl32(T_acc)                                     */
+/*   target tau_i = K/N (FFN) or (k-K)/Z (zero), K = target FFN picks/token   */
+/*   error e_i = tau_i - l_i;  eta <- eta*decay                               */
+/*   I_i <- I_i + eta*e_i                                                     */
+/*   b_i <- ((kp*eta*e_i + ki*I_i) + kd*eta*(e_i - eprev_i)) + b0_i           */
+/*   eprev_i <- e_i;  counts and T_acc reset to zero.                         */
+/* state: eta[1], integ[E], eprev[E]; b0 = initial bias.  No-op if T_acc==0.  */
+/* Convergence rate: parity unpinned (the pages give no gains).              */
+/* ------------------------------------------------------------------------- */
+ZO_EXPORT void zo_update_bias(int64_t *counts, int64_t *tokens, int N, int Z, int k, float kp, float ki, float kd,
+                              float decay, float target_ffn, const float *b0, float *eta, float *integ,
+                              float *eprev, float *bias) {
+  const int E = N + Z;
+  if (*tokens <= 0) return;
+  const float tf = (float)*tokens;
+  const float tau_f = target_ffn / (float)N;
+  const float tau_z = Z > 0 ? ((float)k - target_ffn) / (float)Z : 0.0f;
+  const float et = *eta * decay;
+  *eta = et;
+  const float kpe = kp * et;
+  const float kde = kd * et;
+  for (int i = 0; i < E; ++i) {
+    const float load = (float)counts[i] / tf;
+    const float tau = i < N ? tau_f : tau_z;
+    const float err = tau - load;
+    const float step = et * err;
+    integ[i] = integ[i] + step;
+    const float p = kpe * err;
+    const float q = ki * integ[i];
+    const float dd = kde * (err - eprev[i]);
+    const float s1 = p + q;
+    const float s2 = s1 + dd;
+    bias[i] = s2 + b0[i];
+    eprev[i] = err;
+    counts[i] = 0;
+  }
+  *tokens = 0;
+}

@@ -1,0 +1,381 @@
+"""Pins for the CPU oracle: each check ties the oracle to something other than
+itself (closed forms, brute force, invariants the pages fix, library routines
+for special cases), chosen so that a dropped term, a wrong sign or index, or a
+transposed operand fails at least one of them.  CPU only."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from mixture_experts_layer_shifted_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- generator
+def test_philox_known_answers():
+    # Known-answer vectors of Philox4x32-10 (Random123 distribution, kat_vectors).
+    cases = [
+        ((0, 0, 0, 0), (0, 0), (0x6627e8d5, 0xe169c58d, 0xbc57ac4c, 0x9b00dbd8)),
+        ((0xffffffff,) * 4, (0xffffffff, 0xffffffff), (0x408f276d, 0x41c83b0e, 0xa20bc7c6, 0x6d5451fd)),
+        ((0x243f6a88, 0x85a308d3, 0x13198a2e, 0x03707344), (0xa4093822, 0x299f31d0),
+         (0xd16cfe09, 0x94fdcceb, 0x5001e420, 0x24126ea1)),
+    ]
+    for c, k, want in cases:
+        got = synth.philox4x32_10(*c, *k)
+        assert tuple(int(v) for v in got) == want
+
+
+def test_generator_recipes():
+    v = synth.normal_f32(np.arange(200000, dtype=np.uint64), synth.TID_X, 0, 1.0)
+    assert abs(v.mean()) < 0.01 and abs(v.var() - 1.0) < 0.01
+    assert v.min() >= -6.0 and v.max() <= 6.0
+    # the Irwin-Hall value is exact: z * 65536 is an integer
+    assert np.all((v * 65536.0) == np.round(v * 65536.0))
+    u = synth.uniform_f32(np.arange(100000, dtype=np.uint64), synth.TID_BIAS, 0, -0.2, 0.2)
+    assert u.min() > -0.2 and u.max() < 0.2 and abs(u.mean()) < 0.005
+    # bf16 rounding: nearest-even on hand-made bit patterns
+    f = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9, -2.5], dtype=np.float32)
+    got = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(f))
+    assert got.tolist() == [1.0, 1.0, 1.0 + 4 * 2 ** -8, 1.0, -2.5]
+    o = synth.zipf_logit_offsets(16)
+    assert sorted(np.round(np.exp(-o / 1.1)).astype(int).tolist()) == list(range(1, 17))
+
+
+# ---------------------------------------------------------------- exp
+def test_zexp_accuracy_and_special_values():
+    assert oracle.zexp(0.0) == 1.0
+    assert oracle.zexp(-200.0) == 0.0
+    xs = np.concatenate([np.linspace(-86.0, 0.0, 20011), -np.logspace(-8, 1.9, 4001)]).astype(np.float32)
+    worst = 0.0
+    for x in xs:
+        z = oracle.zexp(float(x))
+        ref = math.exp(float(x))
+        worst = max(worst, abs(z - ref) / float(np.spacing(np.float32(ref))))
+    assert worst <= 2.0, worst
+    # at fp32 inputs next to n ln 2 the result is 2**n times exp of the input's rounding error
+    for n in range(-100, 1):
+        x = np.float32(n * math.log(2))
+        want = 2.0 ** n * math.exp(float(x) - n * math.log(2))
+        assert oracle.zexp(x) == pytest.approx(want, rel=2.5e-7)
+
+
+# ---------------------------------------------------------------- router
+def test_router_logits_against_library_matmul():
+    x = synth.normal((7, 33), synth.TID_X, 3, 1.0, "bf16")
+    wr = synth.normal((5, 33), synth.TID_WR, 3, 0.5, "bf16")
+    off = np.array([0.0, 1.0, -2.0, 0.5, 0.25], np.float32)
+    got = oracle.router_logits(x, wr, off)
+    ref = synth.bf16_bits_to_f32(x).astype(np.float64) @ synth.bf16_bits_to_f32(wr).astype(np.float64).T + off
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    # operand order matters: a transposed weight would change the shape or values
+    assert got.shape == (7, 5)
+
+
+def test_softmax_closed_forms():
+    l = np.array([[0.3, -1.2], [5.0, 5.0], [1000.0, 999.0]])
+    s = oracle.softmax(l)
+    assert s[0, 0] == pytest.approx(1.0 / (1.0 + math.exp(-1.5)), rel=1e-15)
+    assert s[1, 0] == s[1, 1] == 0.5
+    assert s[2, 0] == pytest.approx(1.0 / (1.0 + math.exp(-1.0)), rel=1e-15)
+    r = _rng(1).normal(size=(9, 24))
+    s = oracle.softmax(r)
+    np.testing.assert_allclose(s.sum(1), 1.0, rtol=1e-14)
+    np.testing.assert_allclose(oracle.softmax(r + 7.0), s, rtol=1e-13)  # shift invariance
+    np.testing.assert_allclose(s[:, 3] / s[:, 5], np.exp(r[:, 3] - r[:, 5]), rtol=1e-12)
+
+
+# ---------------------------------------------------------------- top-k
+def test_topk_brute_force_tiny_config():
+    # tiny layer shape: E = 16 FFN + 8 zero experts, k = 4, bias ~ U(-0.1, 0.1)
+    T, E, k = 12, 24, 4
+    s = oracle.softmax(_rng(2).normal(size=(T, E)))
+    b = _rng(3).uniform(-0.1, 0.1, size=E)
+    idx, gate, margin = oracle.topk(s, b, k, scale=1.0)
+    for t in range(T):
+        v = s[t] + b
+        assert list(idx[t]) == oracle.brute_force_topk(v, k)
+        np.testing.assert_array_equal(gate[t], s[t, idx[t]])
+        assert margin[t] > 0
+
+
+def test_topk_ties_and_order():
+    s = np.array([[0.1, 0.3, 0.3, 0.2, 0.1]])
+    idx, gate, margin = oracle.topk(s, None, 3)
+    assert idx[0].tolist() == [1, 2, 3]
+    assert margin[0] == pytest.approx(0.1)
+    idx, _, margin = oracle.topk(s, None, 4)
+    assert idx[0].tolist() == [1, 2, 3, 0]  # tie between experts 0 and 4 goes to 0
+    assert margin[0] == 0.0
+    # bias reorders selection, gate stays the unbiased score times the scale
+    b = np.array([0.0, 0.0, 0.0, 0.0, 0.5])
+    idx, gate, _ = oracle.topk(s, b, 2, scale=2.5)
+    assert idx[0].tolist() == [4, 1]
+    assert gate[0].tolist() == [2.5 * 0.1, 2.5 * 0.3]
+
+
+def test_topk_unbiased_equals_topk_of_logits():
+    l = _rng(4).normal(size=(20, 24))
+    idx, _, _ = oracle.topk(oracle.softmax(l), None, 6)
+    ref = np.argsort(-l, axis=1, kind="stable")[:, :6]
+    np.testing.assert_array_equal(idx, ref)
+
+
+def test_bias_changes_selection_never_gates():
+    T, E, k = 64, 24, 4
+    s = oracle.softmax(_rng(5).normal(size=(T, E)))
+    b = _rng(6).uniform(-0.1, 0.1, size=E)
+    i0, g0, _ = oracle.topk(s, None, k, 1.5)
+    i1, g1, _ = oracle.topk(s, b, k, 1.5)
+    assert (i0 != i1).any()  # the bias does change selection here
+    for t in range(T):
+        for j in range(k):
+            assert g1[t, j] == 1.5 * s[t, i1[t, j]]
+        common = set(i0[t]) & set(i1[t])
+        for e in common:
+            assert g0[t, list(i0[t]).index(e)] == g1[t, list(i1[t]).index(e)]
+
+
+def test_raising_zero_bias_never_lowers_zero_picks():
+    T, N, Z, k = 128, 16, 8, 4
+    s = oracle.softmax(_rng(7).normal(size=(T, N + Z)))
+    prev = -1
+    for beta in [0.0, 0.01, 0.03, 0.1, 0.3, 1.0]:
+        b = np.concatenate([np.zeros(N), np.full(Z, beta)])
+        idx, _, _ = oracle.topk(s, b, k)
+        zero_picks = int((idx >= N).sum())
+        assert zero_picks >= prev
+        prev = zero_picks
+        ffn_per_token = (idx < N).sum(1)
+        assert ffn_per_token.min() >= 0 and ffn_per_token.max() <= k
+    assert prev == T * min(k, Z)
+
+
+def test_replica_matches_fp64_routing_away_from_ties():
+    T, E, k = 256, 96, 8
+    l = _rng(8).normal(size=(T, E)).astype(np.float32) * 3
+    b = _rng(9).uniform(-0.2, 0.2, size=E).astype(np.float32)
+    i32, g32, s32 = oracle.route_replica_f32(l, b, k, 1.0, want_scores=True)
+    s64 = oracle.softmax(l.astype(np.float64))
+    np.testing.assert_allclose(s32, s64, rtol=4e-6, atol=1e-30)
+    i64, g64, margin = oracle.topk(s64, b.astype(np.float64), k)
+    ok = margin > 1e-5
+    assert ok.mean() > 0.9
+    np.testing.assert_array_equal(i32[ok], i64[ok])
+    np.testing.assert_allclose(g32, s32[np.arange(T)[:, None], i32], rtol=0)
+    # the 32-way summation rule gives a sum of exactly 1 +- a few ulp
+    np.testing.assert_allclose(s32.astype(np.float64).sum(1), 1.0, atol=5e-6)
+
+
+# ---------------------------------------------------------------- integer stage
+def test_integer_stage_against_stable_sort():
+    T, N, Z, k = 300, 16, 8, 4
+    s = oracle.softmax(_rng(10).normal(size=(T, N + Z)))
+    idx, _, _ = oracle.topk(s, None, k)
+    counts, offsets, perm, pos = oracle.integer_stage(idx, N, N + Z)
+    assert counts.sum() == T * k
+    np.testing.assert_array_equal(counts, np.bincount(idx.ravel(), minlength=N + Z))
+    assert offsets[0] == 0 and np.all(np.diff(offsets) >= 0) and offsets[N] == (idx < N).sum()
+    flat = idx.ravel()
+    pairs = np.nonzero(flat < N)[0]
+    key = flat[pairs].astype(np.int64) * (T * k) + pairs
+    ref = pairs[np.argsort(key, kind="stable")]
+    np.testing.assert_array_equal(perm, ref)
+    assert len(set(perm.tolist())) == len(perm)  # bijection onto the FFN pairs
+    pf = pos.ravel()
+    assert np.all(pf[flat >= N] == -1)
+    np.testing.assert_array_equal(perm[pf[flat < N]], np.nonzero(flat < N)[0])
+
+
+# ---------------------------------------------------------------- expert math
+def _silu(z):
+    return z / (1.0 + math.exp(-z))
+
+
+def test_ffn_scalar_closed_form():
+    for xg, wg, wu, wd in [(1.5, 0.7, -2.0, 0.3), (-0.4, 2.0, 1.0, -1.5)]:
+        x = np.array([[xg]], np.float32)
+        got = oracle.ffn(x, np.array([[wg]], np.float32), np.array([[wu]], np.float32), np.array([[wd]], np.float32))
+        a, b, c, xv = (float(np.float32(v)) for v in (wg, wu, wd, xg))
+        assert got[0, 0] == pytest.approx(c * _silu(a * xv) * (b * xv), rel=1e-15)
+
+
+def test_ffn_against_library_matmul():
+    d, inter, n = 40, 24, 5
+    x = synth.normal((n, d), 11, 0, 1.0)
+    wg = synth.normal((inter, d), 12, 0, 0.2)
+    wu = synth.normal((inter, d), 13, 0, 0.2)
+    wd = synth.normal((d, inter), 14, 0, 0.2)
+    got = oracle.ffn(x, wg, wu, wd)
+    x64 = x.astype(np.float64)
+    g = x64 @ wg.astype(np.float64).T
+    u = x64 @ wu.astype(np.float64).T
+    ref = (g / (1.0 + np.exp(-g)) * u) @ wd.astype(np.float64).T
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+    # gate and up are not interchangeable: swapping them changes the result
+    assert not np.allclose(oracle.ffn(x, wu, wg, wd), got)
+
+
+def _tiny_layer(seed=0, T=16, d=32, N=6, Z=3, inter=8, k=3):
+    x = synth.normal((T, d), synth.TID_X, seed, 1.0)
+    wg = synth.normal((N, inter, d), synth.TID_WG, seed, 0.2)
+    wu = synth.normal((N, inter, d), synth.TID_WU, seed, 0.2)
+    wd = synth.normal((N, d, inter), synth.TID_WD, seed, 0.2)
+    return x, wg, wu, wd
+
+
+def test_layer_dense_masked_formulation():
+    T, d, N, Z, inter, k = 16, 32, 6, 3, 8, 3
+    x, wg, wu, wd = _tiny_layer(T=T, d=d, N=N, Z=Z, inter=inter, k=k)
+    s = oracle.softmax(_rng(12).normal(size=(T, N + Z)))
+    idx, gate, _ = oracle.topk(s, None, k, 0.75)
+    y = oracle.layer(x, idx, gate, N, wg, wu, wd)
+    # dense: every FFN expert on every token, then a gate mask
+    F = np.stack([oracle.ffn(x, wg[e], wu[e], wd[e]) for e in range(N)], 1)  # [T, N, d]
+    G = np.zeros((T, N + Z))
+    np.put_along_axis(G, idx.astype(np.int64), gate, 1)
+    ref = np.einsum("te,ted->td", G[:, :N], F) + G[:, N:].sum(1, keepdims=True) * x.astype(np.float64)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-14)
+    # the per-expert fetch path gives the same numbers
+    y2 = oracle.layer_outputs(x, idx, gate, N, lambda e: (wg[e], wu[e], wd[e]))
+    np.testing.assert_allclose(y2, y, rtol=1e-12, atol=1e-14)
+
+
+def test_layer_identical_experts_closed_form():
+    T, d, N, Z, inter, k = 10, 16, 4, 4, 8, 4
+    x, wg, wu, wd = _tiny_layer(T=T, d=d, N=N, Z=Z, inter=inter, k=k)
+    wg[:] = wg[0]
+    wu[:] = wu[0]
+    wd[:] = wd[0]
+    s = oracle.softmax(_rng(13).normal(size=(T, N + Z)))
+    idx, gate, _ = oracle.topk(s, None, k)
+    y = oracle.layer(x, idx, gate, N, wg, wu, wd)
+    F = oracle.ffn(x, wg[0], wu[0], wd[0])
+    gf = np.where(idx < N, gate, 0).sum(1, keepdims=True)
+    gz = np.where(idx >= N, gate, 0).sum(1, keepdims=True)
+    np.testing.assert_allclose(y, gf * F + gz * x.astype(np.float64), rtol=1e-12, atol=1e-14)
+
+
+def test_zero_only_tokens_return_weighted_input_exactly():
+    T, d, N, Z, k = 8, 16, 4, 4, 3
+    x, wg, wu, wd = _tiny_layer(T=T, d=d, N=N, Z=Z, inter=8, k=k)
+    s = oracle.softmax(_rng(14).normal(size=(T, N + Z)))
+    b = np.concatenate([np.zeros(N), np.full(Z, 0.5)])  # +0.5 on zero experts: every pick is a zero expert
+    idx, gate, _ = oracle.topk(s, b, k)
+    assert np.all(idx >= N)
+    y = oracle.layer(x, idx, gate, N, wg, wu, wd)
+    zsum = np.zeros(T)
+    for j in range(k):
+        zsum += gate[:, j]
+    np.testing.assert_array_equal(y, zsum[:, None] * x.astype(np.float64))
+
+
+def test_all_experts_chosen_when_k_equals_E():
+    T, d, N, Z, inter = 6, 16, 3, 2, 8
+    x, wg, wu, wd = _tiny_layer(T=T, d=d, N=N, Z=Z, inter=inter, k=N + Z)
+    s = oracle.softmax(_rng(15).normal(size=(T, N + Z)))
+    idx, gate, margin = oracle.topk(s, None, N + Z)
+    assert np.all(np.sort(idx, 1) == np.arange(N + Z))
+    assert np.all(np.isinf(margin))
+    y = oracle.layer(x, idx, gate, N, wg, wu, wd)
+    ref = sum(s[:, e:e + 1] * oracle.ffn(x, wg[e], wu[e], wd[e]) for e in range(N)) + \
+        s[:, N:].sum(1, keepdims=True) * x.astype(np.float64)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------- controller
+def test_update_bias_hand_worked_step():
+    N, Z, k = 2, 1, 2
+    counts = np.array([3, 1, 4], np.int64)  # 4 tokens x k=2 = 8 picks
+    tokens = np.array([4], np.int64)
+    b0 = np.array([0.0, 0.1, -0.1], np.float32)
+    st = oracle.new_controller_state(b0)
+    kp, ki, kd, decay, K = 0.5, 0.25, 2.0, 0.5, 1.5
+    oracle.update_bias(counts, tokens, N, Z, k, (kp, ki, kd, decay, K), b0, st)
+    eta = 0.5
+    tau = [K / N, K / N, (k - K) / Z]
+    load = [3 / 4, 1 / 4, 4 / 4]
+    for i in range(3):
+        e = tau[i] - load[i]
+        integ = eta * e
+        want = kp * eta * e + ki * integ + kd * eta * (e - 0.0) + float(b0[i])
+        assert st["bias"][i] == pytest.approx(want, abs=2e-7)
+        assert st["integ"][i] == pytest.approx(integ, abs=1e-7)
+        assert st["eprev"][i] == pytest.approx(e, abs=1e-7)
+    assert st["eta"][0] == 0.5
+    assert counts.tolist() == [0, 0, 0] and tokens[0] == 0
+    # errors sum to zero: sum(load) == sum(tau) == k
+    assert abs(float(st["eprev"].astype(np.float64).sum())) < 1e-6
+    # an underloaded expert gains bias, an overloaded one loses it
+    assert st["bias"][1] > b0[1] and st["bias"][2] < b0[2]
+
+
+def test_update_bias_fixed_point_and_incremental_form():
+    N, Z, k = 4, 4, 4
+    b0 = np.full(N + Z, 0.01, np.float32)
+    st = oracle.new_controller_state(b0)
+    # loads exactly on target (K = 2): FFN 2/4 = 0.5 per expert, zero 2/4 = 0.5
+    for _ in range(3):
+        counts = np.full(N + Z, 8, np.int64)
+        tokens = np.array([16], np.int64)
+        oracle.update_bias(counts, tokens, N, Z, k, (0.0, 0.1, 0.0, 1.0, 2.0), b0, st)
+    np.testing.assert_array_equal(st["bias"], b0)
+    # kp = kd = 0: the positional form equals incremental b += ki * eta * e
+    st = oracle.new_controller_state(b0)
+    ref = b0.astype(np.float64).copy()
+    eta = 1.0
+    rng = _rng(16)
+    for _ in range(5):
+        c = rng.multinomial(64, [1 / 8] * 8).astype(np.int64)
+        tokens = np.array([16], np.int64)
+        load = c / 16.0
+        eta *= 0.9
+        tau = np.array([2 / 4] * 4 + [2 / 4] * 4)
+        ref += 0.1 * eta * (tau - load)
+        oracle.update_bias(c, tokens, N, Z, k, (0.0, 0.1, 0.0, 0.9, 2.0), b0, st)
+    np.testing.assert_allclose(st["bias"], ref, atol=2e-6)
+    assert st["eta"][0] == pytest.approx(0.9 ** 5, rel=1e-6)
+    # nothing accumulated: no change at all
+    before = st["bias"].copy()
+    oracle.update_bias(np.zeros(8, np.int64), np.zeros(1, np.int64), N, Z, k, (1, 1, 1, 1, 2.0), b0, st)
+    np.testing.assert_array_equal(st["bias"], before)
+
+
+def test_controller_moves_ffn_share_towards_target():
+    # closed loop on the oracle alone: router + top-k + counts + controller
+    T, N, Z, k = 512, 16, 8, 4
+    rng = _rng(17)
+    l = rng.normal(size=(T, N + Z)) * 0.5
+    s = oracle.softmax(l)
+    b0 = np.zeros(N + Z, np.float32)
+    st = oracle.new_controller_state(b0)
+    K = 3.0
+    first = None
+    for step in range(30):
+        idx, _, _ = oracle.topk(s, st["bias"].astype(np.float64), k)
+        ffn = float((idx < N).sum()) / T
+        first = ffn if first is None else first
+        c = np.bincount(idx.ravel(), minlength=N + Z).astype(np.int64)
+        oracle.update_bias(c, np.array([T], np.int64), N, Z, k, (0.0, 0.05, 0.0, 1.0, K), b0, st)
+    assert abs(ffn - K) < abs(first - K)
+
+
+# ---------------------------------------------------------------- the pages' layer shape
+def test_page_layer_shape_is_consistent():
+    cfg = json.load(open(os.path.join(GOLDEN, "longcat_flash_layer.json")))
+    per_layer = cfg["n_ffn"] * 3 * cfg["hidden"] * cfg["expert_inter"]
+    total = per_layer * cfg["layers"]
+    # the FFN experts alone are ~97% of the stated 560B parameters
+    assert 0.9 * cfg["total_params_billion"] * 1e9 < total < cfg["total_params_billion"] * 1e9
+    # uniform routing over 512 + 256 experts picks k * N / E = 8 FFN experts per token,
+    # inside the range the thread reports for realised experts per token
+    expect = cfg["top_k"] * cfg["n_ffn"] / (cfg["n_ffn"] + cfg["n_zero"])
+    lo, hi = min(cfg["realised_ffn_per_token"].values()), max(cfg["realised_ffn_per_token"].values())
+    assert lo <= expect <= hi
