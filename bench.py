@@ -1,0 +1,380 @@
+"""Benchmark of the zero-computation-expert MoE layer forward on B200.
+
+One step = one pass of the whole hot path over one batch: router GEMM +
+softmax/top-k + integer stage + gather + grouped gate/up GEMM + grouped down
+GEMM + combine (zcmoe_forward), then the bias controller step
+(zcmoe_update_bias; with N > 1 ranks the selection counts are summed over the
+ranks with one NCCL all-reduce first, so every replica takes the same step).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl zcmoe|reference]
+
+Prints one JSON line (rank 0).  Inputs are seeded synthetic tensors made on the
+device; the weights (tens of GB) and the token batch are far larger than the
+126 MB L2, so no flush is needed between steps.  ``--impl reference`` times the
+CPU oracle on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ZC-MoE layer tokens/s on 1 B200; % of BF16 tensor / HBM roofline"
+DEFAULT_WORKLOAD = "prefill_560b"
+GAINS = dict(kp=0.0, ki=0.02, kd=0.0, decay=1.0)
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [v.strip() for v in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+        return dist, dist.get_rank(), ws, local
+    return None, 0, 1, 0
+
+
+def algorithmic_work(wl, P, distinct):
+    """FLOPs and bytes per forward from the realised routing: P FFN pairs and
+    `distinct` FFN experts hit.  F = 2 T d E + 6 d inter P;
+    B = distinct * 3 d inter * 2 + E d * 2 + 2 T d * 2 (bf16)."""
+    esz = 2 if wl.dtype == "bf16" else 4
+    F = 2.0 * wl.T * wl.d * wl.E + 6.0 * wl.d * wl.inter * P
+    B = distinct * 3.0 * wl.d * wl.inter * esz + wl.E * wl.d * esz + 2.0 * wl.T * wl.d * esz
+    return F, B
+
+
+def to_host_bits(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    return t.contiguous().cpu().numpy()
+
+
+def cpu_oracle_sample(wl, weights, x, bias, offset, n_tokens, budget_s=20.0):
+    """Times the oracle on the first tokens of the batch (router, routing, experts,
+    combine) with the weights it needs already on the host.  Returns (tokens, seconds, cores)."""
+    import oracle
+    import torch
+    cores = len(os.sched_getaffinity(0))
+    xs = to_host_bits(x[:n_tokens])
+    wr = to_host_bits(weights[0])
+    # routing first (cheap) to learn which experts the sample needs; fetch them before timing
+    l = oracle.router_logits(xs, wr, offset)
+    idx, gate, _ = oracle.topk(oracle.softmax(l), bias.astype(np.float64), wl.top_k)
+    need = sorted({int(e) for e in idx.ravel() if e < wl.n_ffn})
+    cache = {e: tuple(to_host_bits(w[e]) for w in weights[1:]) for e in need}
+    done = 0
+    t0 = time.perf_counter()
+    for t in range(n_tokens):
+        l = oracle.router_logits(xs[t:t + 1], wr, offset)
+        i1, g1, _ = oracle.topk(oracle.softmax(l), bias.astype(np.float64), wl.top_k)
+        oracle.layer_outputs(xs[t:t + 1], i1, g1, wl.n_ffn, lambda e: cache[e])
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    del cache
+    torch.cuda.empty_cache()
+    return done, dt, cores
+
+
+def run_reference(args, wl, rank, ws):
+    """Reference arm: the CPU oracle, timed on the host cores on a bounded sample per step."""
+    if rank != 0:
+        return
+    import torch
+    from mixture_experts_layer_shifted_b200 import configs
+    weights = configs.device_weights(wl)
+    x = configs.device_tokens(wl)
+    bias = configs.bias_vector(wl)
+    offset = configs.logit_offsets(wl)
+    per_step = 4 if wl.d >= 4096 else 16
+    for _ in range(args.warmup):
+        cpu_oracle_sample(wl, weights, x, bias, offset, 1, budget_s=5.0)
+    tot_tok, tot_s, cores = 0, 0.0, 1
+    for _ in range(args.steps):
+        n, s, cores = cpu_oracle_sample(wl, weights, x, bias, offset, per_step, budget_s=15.0)
+        tot_tok += n
+        tot_s += s
+    v = tot_tok / tot_s
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "n_ffn": wl.n_ffn, "n_zero": wl.n_zero,
+                       "inter": wl.inter, "top_k": wl.top_k, "parallelism": "dp1"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{per_step} tokens per step of the {wl.name} batch, full layer in fp64"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="zcmoe", choices=["zcmoe", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    import torch
+    from mixture_experts_layer_shifted_b200 import configs
+    from mixture_experts_layer_shifted_b200.zcmoe import LayerShape, ZcMoE
+
+    dist, rank, ws, local = _dist()
+    wl = configs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl, rank, ws)
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    peaks = _peaks()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    weights = configs.device_weights(wl)
+    xs = [configs.device_tokens(wl, step=rank * 4 + i) for i in range(2)]
+    bias = configs.bias_vector(wl)
+    offset = configs.logit_offsets(wl)
+    shape = LayerShape(wl.d, wl.n_ffn, wl.n_zero, wl.inter, wl.top_k, wl.dtype)
+    layer = ZcMoE(shape, *weights, max_tokens=wl.T, init_bias=bias, logit_offset=offset)
+    y = torch.empty_like(xs[0])
+    counts_buf = torch.empty(wl.E + 1, dtype=torch.int64, device=dev)
+    target = wl.target_ffn if wl.target_ffn is not None else wl.top_k * wl.n_ffn / wl.E
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        layer.forward(xs[i % 2], y)
+        if dist:
+            layer.read_counts(counts_buf)
+            dist.all_reduce(counts_buf)
+            layer.write_counts(counts_buf)
+        layer.update_bias(target_ffn_per_token=target, **GAINS)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    layer.check()
+
+    # ---------------------------------------------------------------- timed region (device time)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = ev0.elapsed_time(ev1)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    layer.check()
+    tokens = wl.T * ws * args.steps
+    value = tokens / (ms / 1e3)
+
+    # ---------------------------------------------------------------- realised routing of one batch
+    E, k = wl.E, wl.top_k
+    idx = torch.empty((wl.T, k), dtype=torch.int32, device=dev)
+    offs = torch.empty((wl.n_ffn + 1,), dtype=torch.int32, device=dev)
+    layer.forward(xs[0], y, debug={"idx": idx, "offsets": offs})
+    torch.cuda.synchronize()
+    cnt = np.diff(offs.cpu().numpy())
+    P = int(cnt.sum())
+    distinct = int((cnt > 0).sum())
+    F, B = algorithmic_work(wl, P, distinct)
+
+    # ---------------------------------------------------------------- per-stage device time (events on the launch stream)
+    layer.profile_begin()
+    nprof = max(3, min(args.steps, 10))
+    for i in range(nprof):
+        layer.forward(xs[i % 2], y)
+    stage_ms, nf = layer.profile_end()
+    stage_avg = {s: v / nf for s, v in stage_ms.items()}
+    gu_ms = stage_avg["gate_up"]
+    gu_flops = 4.0 * wl.d * wl.inter * P
+    tensor_peak = peaks["bf16_tflops_sustained"]
+    achieved = gu_flops / (gu_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "grouped gate/up GEMM + SwiGLU (k_tc_gemm<1>)", "achieved": achieved,
+                "peak": tensor_peak, "unit": "TFLOP/s", "frac": achieved / tensor_peak, "traffic": None,
+                "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
+                "per_launch": {"flops": gu_flops, "ms": gu_ms, "units": f"{P} FFN (token, expert) pairs x 4 d inter"}}
+    fwd_ms = sum(stage_avg.values())
+    t_roof = max(F / (peaks["bf16_tflops_sustained"] * 1e12), B / (peaks["hbm_gbs"] * 1e9))
+    layer_roof = {"forward_ms": fwd_ms, "roofline_ms": 1e3 * t_roof, "frac": 1e3 * t_roof / fwd_ms,
+                  "flops": F, "bytes": B, "stage_ms": stage_avg,
+                  "down": {"ms": stage_avg["down"],
+                           "tflops": 2.0 * wl.d * wl.inter * P / (stage_avg["down"] * 1e-3) / 1e12}}
+
+    # ---------------------------------------------------------------- e2e through host buffers (C ABI, pinned)
+    xh = xs[0].cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    for _ in range(2):
+        layer.forward_host(xh, yh)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, min(args.steps, 10))
+    e0.record(stream)
+    for _ in range(n_e2e):
+        layer.forward_host(xh, yh)
+        layer.update_bias(target_ffn_per_token=target, **GAINS)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    io_bytes = xh.numel() * xh.element_size()
+    e2e = {"value": wl.T * ws / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
+           "d2h_bytes_per_step": io_bytes, "ms_per_step": e2e_ms}
+
+    # ---------------------------------------------------------------- CPU oracle baseline (rank 0, N = 1)
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        n_tok = 8 if wl.d >= 4096 else 64
+        n, s, cores = cpu_oracle_sample(wl, weights, xs[0], bias, offset, n_tok, budget_s=20.0)
+        cpu = {"value": n / s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"first {n} tokens of the {wl.name} batch: fp64 router, routing, experts and combine "
+                         f"({s:.1f} s); the needed expert weights copied to the host beforehand, not timed"}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded Philox, random-init weights)",
+            "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "n_ffn": wl.n_ffn, "n_zero": wl.n_zero,
+                       "inter": wl.inter, "top_k": wl.top_k, "parallelism": f"dp{ws}",
+                       "l2": "inputs larger than L2 (weights %.1f GB, x %.0f MB); no flush" %
+                             (wl.weight_bytes() / 1e9, xs[0].numel() * xs[0].element_size() / 1e6),
+                       "realised": {"P": P, "ffn_per_token": P / wl.T, "distinct_experts": distinct,
+                                    "zero_fraction": 1.0 - P / (wl.T * k)}},
+            "roofline": roofline, "layer_roofline": layer_roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 10 * args.steps, "clocks": clocks, "peaks": peaks}
+
+    # secondary workload (decode): reported beside the headline, not as the headline
+    if rank == 0 and ws == 1 and not args.no_secondary and wl.name == "prefill_560b":
+        wd = configs.WORKLOADS["decode_560b"]
+        xd = configs.device_tokens(wd)
+        layer2 = ZcMoE(LayerShape(wd.d, wd.n_ffn, wd.n_zero, wd.inter, wd.top_k, wd.dtype), *weights,
+                       max_tokens=wd.T, init_bias=configs.bias_vector(wd))
+        yd = torch.empty_like(xd)
+        for _ in range(5):
+            layer2.forward(xd, yd)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nd = 20
+        a.record(stream)
+        for _ in range(nd):
+            layer2.forward(xd, yd)
+        b.record(stream)
+        torch.cuda.synchronize()
+        dms = a.elapsed_time(b) / nd
+        offs2 = torch.empty((wd.n_ffn + 1,), dtype=torch.int32, device=dev)
+        layer2.forward(xd, yd, debug={"offsets": offs2})
+        cnt2 = np.diff(offs2.cpu().numpy())
+        F2, B2 = algorithmic_work(wd, int(cnt2.sum()), int((cnt2 > 0).sum()))
+        hbm = B2 / (dms * 1e-3) / 1e9
+        line["decode"] = {"workload": wd.name, "tokens_per_s": wd.T / (dms * 1e-3), "ms_per_forward": dms,
+                          "hbm_gbs": hbm, "hbm_frac": hbm / peaks["hbm_gbs"], "bytes": B2,
+                          "P": int(cnt2.sum()), "distinct_experts": int((cnt2 > 0).sum())}
+        layer2.close()
+
+    layer.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,181 @@
+/*
+ * zcmoe — forward pass of a mixture-of-experts layer with zero-computation
+ * experts, for NVIDIA B200 (sm_100a).  C ABI of libzcmoe.so.
+ *
+ * The layer (LongCat-Flash technical summary, zhangjingwei.cn, section 二 架構,
+ * part 1 "零計算專家", and 模型配置):
+ *   - N FFN experts (ids 0..N-1) and Z zero-computation experts (ids N..N+Z-1);
+ *     a zero expert returns its input and costs nothing;
+ *   - router logits over all E = N+Z experts are softmaxed (LongCat-Flash-Lite
+ *     N-gram article, onthewifi.com, part 02: fused "softmax + top-k + scaling");
+ *   - top-k is taken on score + per-expert bias; the bias only selects
+ *     (LongCat-Flash tech-report thread, web3.cnouyi.fund: DeepSeek-V3-style
+ *     auxiliary-loss-free bias, with a decay schedule on its update);
+ *   - the gate of a chosen expert is routed_scale * its unbiased score;
+ *   - chosen FFN experts apply a SwiGLU FFN, W_d (silu(W_g x) * (W_u x));
+ *   - the output is the gate-weighted sum;
+ *   - a PID controller moves the bias so the FFN/zero selection ratio tracks a
+ *     target (zhangjingwei.cn, 二.1, "計算預算控制").
+ *
+ * Conventions for every entry point:
+ *   - Return 0 (ZCMOE_OK) or a negative ZCMOE_E* code; zcmoe_last_error() then
+ *     holds a message (thread-local).  Nothing aborts, traps or exits.
+ *   - "device" pointers are CUDA device memory of the current device; "host"
+ *     pointers are ordinary CPU memory.  All tensors are dense row-major.
+ *   - zcmoe_forward and zcmoe_update_bias only enqueue work on `stream` and do
+ *     not synchronise the host; the caller orders calls on one handle (one
+ *     stream at a time; concurrent calls on one handle are undefined).
+ */
+#ifndef ZCMOE_H
+#define ZCMOE_H
+
+#include <stdint.h>
+#include <cuda_runtime.h>
+
+#if defined(__GNUC__)
+#define ZCMOE_API __attribute__((visibility("default")))
+#else
+#define ZCMOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ZCMOE_OK 0
+#define ZCMOE_EINVAL (-1)       /* null pointer, bad shape, misaligned pointer or size    */
+#define ZCMOE_ERANGE (-2)       /* T < 0 or T > max_tokens                                 */
+#define ZCMOE_ENOMEM (-3)       /* device or host allocation failed                        */
+#define ZCMOE_ECUDA (-4)        /* a CUDA runtime/driver call or launch failed             */
+#define ZCMOE_EUNSUPPORTED (-5) /* device is not sm_100, or dtype/shape has no kernel      */
+#define ZCMOE_ETIMEOUT (-6)     /* a device-side wait gave up (reported by zcmoe_check)    */
+
+typedef struct zcmoe_s *zcmoe_t;
+
+typedef enum { ZCMOE_F32 = 0, ZCMOE_BF16 = 1 } zcmoe_dtype;
+
+/* Layer shape and routing constants.  Sizes are element counts.
+ * Limits: 1 <= n_ffn, 0 <= n_zero, E = n_ffn + n_zero <= 1024, 1 <= top_k <= min(E, 32),
+ * d and inter multiples of 64, 1 <= max_tokens <= 2^20.
+ * dtype: ZCMOE_BF16 -> x, y, all weights bf16, fp32 accumulation (tensor cores);
+ *        ZCMOE_F32  -> everything fp32 with fp32 CUDA-core arithmetic (no TF32). */
+typedef struct {
+  int32_t d;            /* hidden size                                   */
+  int32_t n_ffn;        /* N, FFN experts                                */
+  int32_t n_zero;       /* Z, zero-computation experts                   */
+  int32_t inter;        /* FFN expert intermediate size                  */
+  int32_t top_k;        /* experts chosen per token                      */
+  int32_t max_tokens;   /* largest T accepted by zcmoe_forward           */
+  int32_t dtype;        /* zcmoe_dtype                                   */
+  float routed_scale;   /* gate = routed_scale * score (the "scaling" of the fused router); 1.0 if unsure */
+  const float *init_bias;    /* host [E] or NULL (zeros); copied at create; also the controller's b0 */
+  const float *logit_offset; /* host [E] or NULL; copied; added to every token's logits before softmax */
+} zcmoe_config;
+
+/* Device weight pointers, BORROWED: the caller keeps them alive and unchanged
+ * until zcmoe_destroy.  Element type = config dtype.  16-byte aligned.
+ *   w_router [E, d]; w_gate [N, inter, d]; w_up [N, inter, d]; w_down [N, d, inter]. */
+typedef struct {
+  const void *w_router;
+  const void *w_gate;
+  const void *w_up;
+  const void *w_down;
+} zcmoe_weights;
+
+/* Controller gains (the pages give none; see zcmoe_update_bias). */
+typedef struct {
+  float kp, ki, kd;
+  float decay;                /* eta <- eta * decay before every step (eta starts at 1) */
+  float target_ffn_per_token; /* K: target mean number of FFN experts per token, 0 <= K <= top_k */
+} zcmoe_gains;
+
+/* Optional device outputs of one forward, for tests and inspection; any field
+ * may be NULL.  Shapes: logits/scores [T, E] fp32, idx [T, k] int32 (expert id,
+ * slot order = biased score descending then id ascending), gate [T, k] fp32,
+ * counts [E] int32, offsets [N+1] int32 (exclusive scan of FFN counts; offsets[N] = P),
+ * perm [T*k] int32 (first P entries valid: FFN pairs t*k+j ordered by expert then
+ * token), pos [T, k] int32 (row of pair (t,j) in the permuted order, -1 for zero experts),
+ * expert_out [T*k, d] config dtype (first P rows valid: the FFN expert outputs F_e(x_t),
+ * one row per pair in the permuted order, before gating). */
+typedef struct {
+  float *logits;
+  float *scores;
+  int32_t *idx;
+  float *gate;
+  int32_t *counts;
+  int32_t *offsets;
+  int32_t *perm;
+  int32_t *pos;
+  void *expert_out;
+} zcmoe_debug;
+
+/* Creates a layer handle: validates shapes and alignment, allocates the handle's
+ * device state (bias, controller state and accumulators, workspace for
+ * max_tokens), and builds the TMA descriptors of the weights.  Requires the
+ * current device to be sm_100.  On error *out is left NULL. */
+ZCMOE_API int zcmoe_create(const zcmoe_config *cfg, const zcmoe_weights *w, zcmoe_t *out);
+
+/* One forward pass over T tokens (zhangjingwei.cn 二.1; onthewifi.com part 02):
+ * x [T, d] device (config dtype) -> y [T, d] device (config dtype), y must not
+ * overlap x.  Also adds this batch's per-expert selection counts and T to the
+ * controller accumulators.  T == 0 is a no-op.  Asynchronous on `stream`. */
+ZCMOE_API int zcmoe_forward(zcmoe_t h, const void *x, int64_t T, void *y, cudaStream_t stream, const zcmoe_debug *dbg);
+
+/* The same forward pass from and to HOST memory: copies x [T, d] (host) into a
+ * handle-owned device staging buffer, runs zcmoe_forward, and copies y [T, d]
+ * back to host memory, all enqueued on `stream`.  The staging buffers (2 x
+ * max_tokens x d elements) are allocated on the first call.  Use page-locked
+ * host buffers so the copies are asynchronous; keep both alive and read y only
+ * after the stream has been synchronised. */
+ZCMOE_API int zcmoe_forward_host(zcmoe_t h, const void *x_host, int64_t T, void *y_host, cudaStream_t stream);
+
+/* One bias-controller step (zhangjingwei.cn 二.1 "PID controller"; web3.cnouyi.fund
+ * "decay schedule"), fp32 with every operation rounded once:
+ *   load l_i = c_i / T_acc from the accumulated counts; target tau_i = K/N for FFN
+ *   experts, (k-K)/Z for zero experts; e_i = tau_i - l_i; eta <- eta*decay;
+ *   I_i <- I_i + eta*e_i; b_i <- ((kp*eta*e_i + ki*I_i) + kd*eta*(e_i - e_prev_i)) + b0_i;
+ *   e_prev_i <- e_i; the accumulators are reset.  No-op while T_acc == 0.
+ * Asynchronous on `stream`. */
+ZCMOE_API int zcmoe_update_bias(zcmoe_t h, const zcmoe_gains *g, cudaStream_t stream);
+
+/* Data-parallel exchange of the accumulators.  read: copies the handle's
+ * accumulators into dst [E+1] int64 device (counts, then T_acc); write: replaces
+ * them with src [E+1].  A replica group sums the read buffers (all-reduce) and
+ * writes the sum back before zcmoe_update_bias, so every replica takes the same
+ * bit-exact controller step.  Asynchronous on `stream`. */
+ZCMOE_API int zcmoe_read_counts(zcmoe_t h, int64_t *dst, cudaStream_t stream);
+ZCMOE_API int zcmoe_write_counts(zcmoe_t h, const int64_t *src, cudaStream_t stream);
+
+/* Host copies of the controller state (any pointer may be NULL): bias [E] fp32,
+ * accumulated counts [E] int64, accumulated tokens [1] int64, eta [1] fp32.
+ * Synchronises the device. */
+ZCMOE_API int zcmoe_get_state(zcmoe_t h, float *bias, int64_t *counts, int64_t *tokens, float *eta);
+
+/* Replaces the bias (host [E] fp32).  Does not change b0 or the controller state.  Synchronous. */
+ZCMOE_API int zcmoe_set_bias(zcmoe_t h, const float *bias);
+
+/* Synchronises the device and reports a device-side timeout (ZCMOE_ETIMEOUT) if a
+ * kernel's bounded wait gave up since the last check; clears the flag. */
+ZCMOE_API int zcmoe_check(zcmoe_t h);
+
+/* Stage timing for measurement.  zcmoe_profile_begin starts recording CUDA
+ * events between the stages of every later zcmoe_forward on this handle;
+ * zcmoe_profile_end synchronises, writes per-stage device time summed over the
+ * recorded forwards into ms[ZCMOE_NUM_STAGES] (host) and the number of forwards
+ * into *n_forwards, and stops recording.  Stages, in order: router GEMM,
+ * softmax/top-k, integer stage, row gather, gate/up GEMM, down GEMM, combine. */
+#define ZCMOE_NUM_STAGES 7
+ZCMOE_API int zcmoe_profile_begin(zcmoe_t h);
+ZCMOE_API int zcmoe_profile_end(zcmoe_t h, float *ms, int32_t *n_forwards);
+
+/* Frees the handle's own memory; never touches the borrowed weights.  NULL is a no-op. */
+ZCMOE_API int zcmoe_destroy(zcmoe_t h);
+
+/* Message for the last failing call on this thread ("" if none). */
+ZCMOE_API const char *zcmoe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZCMOE_H */

@@ -1,0 +1,476 @@
+// Routing, integer stage, row gather, combine and bias controller kernels.
+//
+// Sources (page title, section):
+//  - LongCat-Flash technical summary (zhangjingwei.cn), 二 架構, part 1
+//    "零計算專家": zero experts return the input at no cost; an expert-specific
+//    bias shifts the routing scores; a PID controller keeps the FFN/zero
+//    selection ratio near a target.
+//  - LongCat-Flash tech-report thread (web3.cnouyi.fund): DeepSeek-V3-like
+//    auxiliary-loss-free bias (selection only) with a decay schedule.
+//  - LongCat-Flash-Lite N-gram article (onthewifi.com), part 02: the router is a
+//    fused softmax + top-k + scaling step.
+//
+// Every floating-point operation that can change an integer decision (softmax,
+// biased score, comparison) is written with an explicit rounding intrinsic so
+// that the compiler cannot contract or reorder it; the rule it follows is:
+//   m = max_e l_e;  u_e = zexp(l_e - m);
+//   per lane p (e = p, p+32, ...): partial sums in ascending e; then a
+//   butterfly over lane distance 16, 8, 4, 2, 1: partial += partner;
+//   s_e = u_e / sum;  v_e = s_e + b_e;  top-k on v, ties to the lower id;
+//   gate = scale * s.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "zc_internal.h"
+
+namespace zc {
+namespace {
+
+// exp for x <= 0 (the softmax only needs that range; larger x is still handled
+// up to overflow).  Cody-Waite reduction: n = rint(x * fl32(1/ln2)),
+// r = (x - n*C1) - n*C2 with C1 = ln2 truncated to 16 significant bits (n*C1 is
+// exact for |n| < 256) and C2 = fl32(ln2 - C1); degree-7 Taylor polynomial of
+// e^r with coefficients fl32(1/i!) in Horner form with fused multiply-adds;
+// scaled by 2^n built in the exponent field; results under 2^-125 flush to 0.
+__device__ __forceinline__ float zexp(float x) {
+  if (!(x > -88.0f)) return 0.0f;
+  const float n = rintf(__fmul_rn(x, 0x1.715476p+0f));
+  if (n < -125.0f) return 0.0f;
+  if (n > 127.0f) return __int_as_float(0x7f800000);
+  float r = __fmaf_rn(-n, 0x1.62e4p-1f, x);
+  r = __fmaf_rn(-n, 0x1.7f7d1cp-20f, r);
+  float p = 0x1.a01a02p-13f;
+  p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);
+  p = __fmaf_rn(p, r, 0x1.111112p-7f);
+  p = __fmaf_rn(p, r, 0x1.555556p-5f);
+  p = __fmaf_rn(p, r, 0x1.555556p-3f);
+  p = __fmaf_rn(p, r, 0.5f);
+  p = __fmaf_rn(p, r, 1.0f);
+  p = __fmaf_rn(p, r, 1.0f);
+  const float scale = __int_as_float(((int)n + 127) << 23);
+  return __fmul_rn(p, scale);
+}
+
+__device__ __forceinline__ bool better(float va, int ea, float vb, int eb) {
+  return va > vb || (va == vb && ea < eb);
+}
+
+// One warp per token.  EPL = experts held per lane (E <= 32 * EPL).
+template <int EPL>
+__global__ void __launch_bounds__(256) k_softmax_topk(const float* __restrict__ logits, const float* __restrict__ bias,
+                                                      int T, int E, int k, float scale, int32_t* __restrict__ idx,
+                                                      float* __restrict__ gate, float* __restrict__ scores) {
+  const int lane = threadIdx.x & 31;
+  const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
+  float b[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    b[i] = e < E ? bias[e] : 0.0f;
+  }
+  for (int t = warp; t < T; t += nwarps) {
+    const float* lt = logits + (int64_t)t * E;
+    float l[EPL];
+    float m = -__int_as_float(0x7f800000);
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      l[i] = e < E ? lt[e] : -__int_as_float(0x7f800000);
+      m = fmaxf(m, l[i]);
+    }
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, w));
+    float u[EPL];
+    float acc = 0.0f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      u[i] = 0.0f;
+      if (e < E) {
+        u[i] = zexp(__fsub_rn(l[i], m));
+        acc = __fadd_rn(acc, u[i]);
+      }
+    }
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, w));
+    float v[EPL];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      u[i] = __fdiv_rn(u[i], acc);  // u now holds the score s
+      v[i] = __fadd_rn(u[i], b[i]);
+      if (e >= E) taken |= 1u << i;
+      else if (scores) scores[(int64_t)t * E + e] = u[i];
+    }
+    int my_idx = 0;
+    float my_gate = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      float bv = -__int_as_float(0x7f800000);
+      int be = 0x7fffffff;
+      float bs = 0.0f;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (!((taken >> i) & 1u) && better(v[i], e, bv, be)) {
+          bv = v[i];
+          be = e;
+          bs = u[i];
+        }
+      }
+#pragma unroll
+      for (int w = 16; w >= 1; w >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, w);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, w);
+        const float os = __shfl_xor_sync(0xffffffffu, bs, w);
+        if (better(ov, oe, bv, be)) {
+          bv = ov;
+          be = oe;
+          bs = os;
+        }
+      }
+      if (lane == (be & 31)) taken |= 1u << (be >> 5);
+      if (lane == j) {
+        my_idx = be;
+        my_gate = __fmul_rn(scale, bs);
+      }
+    }
+    if (lane < k) {
+      idx[(int64_t)t * k + lane] = my_idx;
+      gate[(int64_t)t * k + lane] = my_gate;
+    }
+  }
+}
+
+// Integer stage, part 1: per block of 256 tokens, one 32-bit token mask per
+// (warp, expert) in shared memory; writes the block's per-expert counts.
+__global__ void __launch_bounds__(kChunk) k_route_count(const int32_t* __restrict__ idx, int T, int k, int E,
+                                                        int32_t* __restrict__ chunk_cnt) {
+  extern __shared__ uint32_t smask[];  // [8][E]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < 8 * E; i += kChunk) smask[i] = 0u;
+  __syncthreads();
+  const int t = blockIdx.x * kChunk + tid;
+  if (t < T)
+    for (int j = 0; j < k; ++j) atomicOr(&smask[warp * E + idx[(int64_t)t * k + j]], 1u << lane);
+  __syncthreads();
+  for (int e = tid; e < E; e += kChunk) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) c += __popc(smask[w * E + e]);
+    chunk_cnt[(int64_t)blockIdx.x * E + e] = c;
+  }
+}
+
+// Block-wide exclusive scan of two ints (1024 threads).
+__device__ __forceinline__ int2 block_exclusive_scan2(int2 v, int2* warp_tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int2 inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, inc.x, o);
+    const int b = __shfl_up_sync(0xffffffffu, inc.y, o);
+    if (lane >= o) {
+      inc.x += a;
+      inc.y += b;
+    }
+  }
+  if (lane == 31) warp_tot[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int2 w = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : make_int2(0, 0);
+    int2 wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, wi.x, o);
+      const int b = __shfl_up_sync(0xffffffffu, wi.y, o);
+      if (lane >= o) {
+        wi.x += a;
+        wi.y += b;
+      }
+    }
+    warp_tot[lane] = make_int2(wi.x - w.x, wi.y - w.y);
+  }
+  __syncthreads();
+  const int2 base = warp_tot[warp];
+  return make_int2(base.x + inc.x - v.x, base.y + inc.y - v.y);
+}
+
+// Integer stage, part 2 (one block of 1024 threads, thread = expert): totals,
+// controller accumulation, exclusive scans over FFN experts of the counts and
+// of their 128-row block counts, and the first permuted row of every
+// (token block, expert) pair, written over chunk_cnt.
+__global__ void __launch_bounds__(1024) k_route_scan(int32_t* __restrict__ chunk_cnt, int nchunks, int T, int N, int E,
+                                                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                     int32_t* __restrict__ mb_off, int32_t* __restrict__ scal,
+                                                     int64_t* __restrict__ acc_counts, int64_t* __restrict__ acc_tokens) {
+  __shared__ int2 warp_tot[32];
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E) {
+#pragma unroll 8
+    for (int c = 0; c < nchunks; ++c) total += chunk_cnt[(int64_t)c * E + e];
+    counts[e] = total;
+    acc_counts[e] += total;
+  }
+  const int2 v = (e < N) ? make_int2(total, (total + kBM - 1) / kBM) : make_int2(0, 0);
+  const int2 ex = block_exclusive_scan2(v, warp_tot);
+  if (e < N) {
+    offsets[e] = ex.x;
+    mb_off[e] = ex.y;
+    if (e == N - 1) {
+      offsets[N] = ex.x + v.x;
+      mb_off[N] = ex.y + v.y;
+      scal[0] = ex.x + v.x;
+      scal[1] = ex.y + v.y;
+    }
+    int run = ex.x;
+    for (int c = 0; c < nchunks; ++c) {
+      const int64_t i = (int64_t)c * E + e;
+      const int cc = chunk_cnt[i];
+      chunk_cnt[i] = run;
+      run += cc;
+    }
+  }
+  if (e == 0) *acc_tokens += T;
+}
+
+// Integer stage, part 3: the permuted row of every FFN pair.  Within a 256-token
+// block the rank of (t, e) is the number of earlier tokens of the block that
+// chose e (earlier warps' masks, then the lower lanes of its own warp's mask),
+// so the order is ascending token within each expert.
+__global__ void __launch_bounds__(kChunk) k_route_scatter(const int32_t* __restrict__ idx, int T, int k, int N, int E,
+                                                          const int32_t* __restrict__ chunk_base,
+                                                          int32_t* __restrict__ perm, int32_t* __restrict__ pos) {
+  extern __shared__ uint32_t smask[];  // [8][E]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < 8 * E; i += kChunk) smask[i] = 0u;
+  __syncthreads();
+  const int t = blockIdx.x * kChunk + tid;
+  if (t < T)
+    for (int j = 0; j < k; ++j) atomicOr(&smask[warp * E + idx[(int64_t)t * k + j]], 1u << lane);
+  __syncthreads();
+  if (t >= T) return;
+  for (int j = 0; j < k; ++j) {
+    const int64_t pair = (int64_t)t * k + j;
+    const int e = idx[pair];
+    if (e < N) {
+      int r = chunk_base[(int64_t)blockIdx.x * E + e];
+      for (int w = 0; w < warp; ++w) r += __popc(smask[w * E + e]);
+      r += __popc(smask[warp * E + e] & ((1u << lane) - 1u));
+      pos[pair] = r;
+      perm[r] = (int32_t)pair;
+    } else {
+      pos[pair] = -1;
+    }
+  }
+}
+
+// X_perm[p] = x[perm[p] / k] for p < P (P read from the device).
+__global__ void k_gather_rows(const uint4* __restrict__ x, int row_vecs, const int32_t* __restrict__ perm, int k,
+                              const int32_t* __restrict__ scal, uint4* __restrict__ xperm) {
+  const int64_t P = scal[0];
+  const int64_t n = P * row_vecs;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t p = i / row_vecs;
+    const int v = (int)(i - p * row_vecs);
+    const int t = perm[p] / k;
+    xperm[i] = x[(int64_t)t * row_vecs + v];
+  }
+}
+
+// Combine / unpermute (zero experts folded in as identity terms):
+//   y_t = zsum_t * x_t + sum over FFN slots j (in slot order) of g_tj * Y[pos_tj],
+// fp32 accumulation, one rounding to the output type.  A gather per token, no atomics.
+template <typename TIO>
+struct Vec;
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int kN = 8;
+  __device__ static void load(const __nv_bfloat16* p, float* f) {
+    const uint4 r = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 t = __bfloat1622float2(h[i]);
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  }
+  __device__ static void store(__nv_bfloat16* p, const float* f) {
+    uint4 r;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    *reinterpret_cast<uint4*>(p) = r;
+  }
+};
+template <>
+struct Vec<float> {
+  static constexpr int kN = 4;
+  __device__ static void load(const float* p, float* f) {
+    const float4 r = *reinterpret_cast<const float4*>(p);
+    f[0] = r.x;
+    f[1] = r.y;
+    f[2] = r.z;
+    f[3] = r.w;
+  }
+  __device__ static void store(float* p, const float* f) { *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]); }
+};
+
+template <typename TIO>
+__global__ void __launch_bounds__(128) k_combine(const TIO* __restrict__ x, const TIO* __restrict__ Y,
+                                                 const float* __restrict__ gate, const int32_t* __restrict__ pos, int T,
+                                                 int k, int d, TIO* __restrict__ y) {
+  constexpr int V = Vec<TIO>::kN;
+  __shared__ float sg[32];
+  __shared__ int32_t sp[32];
+  __shared__ float szsum;
+  const int nv = d / V;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    if (threadIdx.x < k) {
+      sg[threadIdx.x] = gate[(int64_t)t * k + threadIdx.x];
+      sp[threadIdx.x] = pos[(int64_t)t * k + threadIdx.x];
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float z = 0.0f;
+      for (int j = 0; j < k; ++j)
+        if (sp[j] < 0) z = __fadd_rn(z, sg[j]);
+      szsum = z;
+    }
+    __syncthreads();
+    const float zsum = szsum;
+    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+      float acc[V], a[V];
+      Vec<TIO>::load(x + (int64_t)t * d + v * V, a);
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[i] = __fmul_rn(zsum, a[i]);
+      for (int j = 0; j < k; ++j) {
+        const int p = sp[j];
+        if (p < 0) continue;
+        Vec<TIO>::load(Y + (int64_t)p * d + v * V, a);
+        const float g = sg[j];
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] = __fmaf_rn(g, a[i], acc[i]);
+      }
+      Vec<TIO>::store(y + (int64_t)t * d + v * V, acc);
+    }
+    __syncthreads();
+  }
+}
+
+// Bias controller step; one block, thread = expert.  Every operation rounds
+// once and none is fused, in the order of the rule in the header.
+__global__ void __launch_bounds__(1024) k_update_bias(int64_t* __restrict__ counts, int64_t* __restrict__ tokens, int N,
+                                                      int Z, int k, float kp, float ki, float kd, float decay,
+                                                      float target, const float* __restrict__ b0,
+                                                      float* __restrict__ eta, float* __restrict__ integ,
+                                                      float* __restrict__ eprev, float* __restrict__ bias) {
+  const int64_t tok = *tokens;
+  const float eta0 = *eta;
+  __syncthreads();
+  if (tok <= 0) return;
+  const int E = N + Z;
+  const float tf = __ll2float_rn(tok);
+  const float tau_f = __fdiv_rn(target, __int2float_rn(N));
+  const float tau_z = Z > 0 ? __fdiv_rn(__fsub_rn(__int2float_rn(k), target), __int2float_rn(Z)) : 0.0f;
+  const float et = __fmul_rn(eta0, decay);
+  const float kpe = __fmul_rn(kp, et);
+  const float kde = __fmul_rn(kd, et);
+  for (int i = threadIdx.x; i < E; i += blockDim.x) {
+    const float load = __fdiv_rn(__ll2float_rn(counts[i]), tf);
+    const float tau = i < N ? tau_f : tau_z;
+    const float err = __fsub_rn(tau, load);
+    const float step = __fmul_rn(et, err);
+    const float in = __fadd_rn(integ[i], step);
+    integ[i] = in;
+    const float p = __fmul_rn(kpe, err);
+    const float q = __fmul_rn(ki, in);
+    const float dd = __fmul_rn(kde, __fsub_rn(err, eprev[i]));
+    bias[i] = __fadd_rn(__fadd_rn(__fadd_rn(p, q), dd), b0[i]);
+    eprev[i] = err;
+    counts[i] = 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    *eta = et;
+    *tokens = 0;
+  }
+}
+
+int grid_cap(int want, int cap) { return want < 1 ? 1 : (want < cap ? want : cap); }
+
+}  // namespace
+
+cudaError_t launch_softmax_topk(const float* logits, const float* bias, int T, int E, int k, float scale, int32_t* idx,
+                                float* gate, float* scores, int sms, cudaStream_t s) {
+  const int grid = grid_cap((T + 7) / 8, sms * 16);
+  const int epl = (E + 31) / 32;
+#define ZC_TOPK(n)                                                                                   \
+  case n:                                                                                            \
+    k_softmax_topk<n><<<grid, 256, 0, s>>>(logits, bias, T, E, k, scale, idx, gate, scores); \
+    break;
+  switch (epl) {
+    ZC_TOPK(1) ZC_TOPK(2) ZC_TOPK(3) ZC_TOPK(4) ZC_TOPK(5) ZC_TOPK(6) ZC_TOPK(7) ZC_TOPK(8)
+    ZC_TOPK(9) ZC_TOPK(10) ZC_TOPK(11) ZC_TOPK(12) ZC_TOPK(13) ZC_TOPK(14) ZC_TOPK(15) ZC_TOPK(16)
+    ZC_TOPK(17) ZC_TOPK(18) ZC_TOPK(19) ZC_TOPK(20) ZC_TOPK(21) ZC_TOPK(22) ZC_TOPK(23) ZC_TOPK(24)
+    ZC_TOPK(25) ZC_TOPK(26) ZC_TOPK(27) ZC_TOPK(28) ZC_TOPK(29) ZC_TOPK(30) ZC_TOPK(31) ZC_TOPK(32)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef ZC_TOPK
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int32_t* chunk_cnt, cudaStream_t s) {
+  const int nchunks = (T + kChunk - 1) / kChunk;
+  k_route_count<<<nchunks, kChunk, 8 * E * sizeof(uint32_t), s>>>(idx, T, k, E, chunk_cnt);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_scan(int32_t* chunk_cnt, int nchunks, int T, int N, int E, int32_t* counts, int32_t* offsets,
+                              int32_t* mb_off, int32_t* scal, int64_t* acc_counts, int64_t* acc_tokens, cudaStream_t s) {
+  k_route_scan<<<1, 1024, 0, s>>>(chunk_cnt, nchunks, T, N, E, counts, offsets, mb_off, scal, acc_counts, acc_tokens);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_scatter(const int32_t* idx, int T, int k, int N, int E, const int32_t* chunk_base,
+                                 int32_t* perm, int32_t* pos, cudaStream_t s) {
+  const int nchunks = (T + kChunk - 1) / kChunk;
+  k_route_scatter<<<nchunks, kChunk, 8 * E * sizeof(uint32_t), s>>>(idx, T, k, N, E, chunk_base, perm, pos);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const void* x, int row_bytes, const int32_t* perm, int k, const int32_t* scal,
+                               void* xperm, int sms, cudaStream_t s) {
+  k_gather_rows<<<sms * 8, 256, 0, s>>>(static_cast<const uint4*>(x), row_bytes / 16, perm, k, scal,
+                                        static_cast<uint4*>(xperm));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(int bf16, const void* x, const void* Y, const int32_t* idx, const float* gate,
+                           const int32_t* pos, int T, int k, int N, int d, void* y, int sms, cudaStream_t s) {
+  (void)idx;
+  (void)N;
+  const int grid = grid_cap(T, sms * 16);
+  if (bf16)
+    k_combine<__nv_bfloat16><<<grid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
+                                                  static_cast<const __nv_bfloat16*>(Y), gate, pos, T, k, d,
+                                                  static_cast<__nv_bfloat16*>(y));
+  else
+    k_combine<float><<<grid, 128, 0, s>>>(static_cast<const float*>(x), static_cast<const float*>(Y), gate, pos, T, k,
+                                          d, static_cast<float*>(y));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_update_bias(int64_t* counts, int64_t* tokens, int N, int Z, int k, float kp, float ki, float kd,
+                               float decay, float target, const float* b0, float* eta, float* integ, float* eprev,
+                               float* bias, cudaStream_t s) {
+  k_update_bias<<<1, 1024, 0, s>>>(counts, tokens, N, Z, k, kp, ki, kd, decay, target, b0, eta, integ, eprev, bias);
+  return cudaGetLastError();
+}
+
+}  // namespace zc

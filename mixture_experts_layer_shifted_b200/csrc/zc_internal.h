@@ -1,0 +1,72 @@
+// Internal interfaces between the C-ABI layer (zcmoe.cu) and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace zc {
+
+// Rows of one tensor-core output tile; also the m-block granularity of the
+// expert offsets produced by the integer stage.
+constexpr int kBM = 128;
+// Tokens per block of the integer stage (8 warps x 32 lanes, one token per thread).
+constexpr int kChunk = 256;
+
+// ------------------------------------------------------------- routing (route.cu)
+cudaError_t launch_softmax_topk(const float* logits, const float* bias, int T, int E, int k, float scale, int32_t* idx,
+                                float* gate, float* scores, int sms, cudaStream_t s);
+cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int32_t* chunk_cnt, cudaStream_t s);
+cudaError_t launch_route_scan(int32_t* chunk_cnt, int nchunks, int T, int N, int E, int32_t* counts, int32_t* offsets,
+                              int32_t* mb_off, int32_t* scal, int64_t* acc_counts, int64_t* acc_tokens, cudaStream_t s);
+cudaError_t launch_route_scatter(const int32_t* idx, int T, int k, int N, int E, const int32_t* chunk_base,
+                                 int32_t* perm, int32_t* pos, cudaStream_t s);
+cudaError_t launch_gather_rows(const void* x, int row_bytes, const int32_t* perm, int k, const int32_t* scal,
+                               void* xperm, int sms, cudaStream_t s);
+cudaError_t launch_combine(int bf16, const void* x, const void* Y, const int32_t* idx, const float* gate,
+                           const int32_t* pos, int T, int k, int N, int d, void* y, int sms, cudaStream_t s);
+cudaError_t launch_update_bias(int64_t* counts, int64_t* tokens, int N, int Z, int k, float kp, float ki, float kd,
+                               float decay, float target, const float* b0, float* eta, float* integ, float* eprev,
+                               float* bias, cudaStream_t s);
+
+// ------------------------------------------------------------- tensor-core GEMM (gemm_tc.cu)
+enum TcMode { kRouter = 0, kGateUp = 1, kDown = 2 };
+
+struct TcArgs {
+  int K;                    // reduction length (elements)
+  int n_out;                // valid output columns
+  int nblocks;              // output column tiles
+  int ngroups;              // experts (router: 1)
+  const int32_t* row_off;   // [ngroups+1] first permuted row of each expert (router: unused)
+  const int32_t* mb_off;    // [ngroups+1] first m-block of each expert (router: unused)
+  int M;                    // router: token rows
+  int b_rows_per_group;     // rows of the B tensor per expert (gate/up: inter, down: d)
+  void* out;                // output matrix
+  int64_t ldo;              // its row stride (elements)
+  const float* col_add;     // router: per-column offset added to the logits (or null)
+  int* err;                 // device error word (bounded waits)
+};
+
+int tc_smem_bytes();
+int tc_block_n(int mode);
+cudaError_t launch_tc_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                           const TcArgs& args, int grid, cudaStream_t s);
+
+// ------------------------------------------------------------- fp32 CUDA-core GEMM (gemm_simt.cu)
+struct SimtArgs {
+  const float* A;
+  const float* B0;
+  const float* B1;
+  int K;
+  int n_out;
+  int ngroups;
+  const int32_t* row_off;
+  const int32_t* mb_off;
+  int M;
+  int b_rows_per_group;
+  float* out;
+  int64_t ldo;
+  const float* col_add;
+};
+cudaError_t launch_simt_gemm(int mode, const SimtArgs& args, int max_mblocks, cudaStream_t s);
+
+}  // namespace zc

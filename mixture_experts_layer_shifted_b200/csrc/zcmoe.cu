@@ -1,0 +1,567 @@
+// C ABI of the zero-computation-expert MoE layer (declared in include/zcmoe.h).
+//
+// A forward pass is a fixed sequence of kernels on the caller's stream, with no
+// host synchronisation and no host-visible intermediate:
+//   router GEMM (+ logit offset)      -> logits [T, E] fp32
+//   softmax + bias-shifted top-k      -> idx, gate [T, k]
+//   integer stage (count, scan, scatter) -> counts, offsets, row blocks, perm, pos
+//   row gather                        -> X_perm [P, d]
+//   grouped gate/up GEMM + SwiGLU     -> H [P, inter]
+//   grouped down GEMM                 -> Y [P, d]
+//   combine (zero experts as identity terms) -> y [T, d]
+// Every size that depends on the routing (P, row blocks) stays on the device;
+// the persistent GEMM kernels read it there.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <cstdarg>
+#include <mutex>
+#include <new>
+#include <unordered_set>
+#include <vector>
+
+#include "../../include/zcmoe.h"
+#include "zc_internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+// Live handles, so that a destroyed or foreign handle is rejected instead of
+// being dereferenced.
+std::mutex g_live_mu;
+std::unordered_set<const void*> g_live;
+
+bool is_live(const void* h) {
+  std::lock_guard<std::mutex> lk(g_live_mu);
+  return h && g_live.count(h) != 0;
+}
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+#define ZC_CUDA(call)                                                                               \
+  do {                                                                                             \
+    cudaError_t e_ = (call);                                                                       \
+    if (e_ != cudaSuccess) return fail(ZCMOE_ECUDA, "%s: %s (%s:%d)", #call, cudaGetErrorString(e_), \
+                                       __FILE__, __LINE__);                                       \
+  } while (0)
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] (inner contiguous), box [box_outer, 64], 128-byte swizzle.
+int make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(ZCMOE_ECUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0) return fail(ZCMOE_EINVAL, "tensor base not 16-byte aligned");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ZCMOE_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return ZCMOE_OK;
+}
+
+template <typename T>
+int dalloc(T** p, size_t n) {
+  *p = nullptr;
+  if (n == 0) n = 1;
+  cudaError_t e = cudaMalloc(reinterpret_cast<void**>(p), n * sizeof(T));
+  if (e != cudaSuccess) {
+    *p = nullptr;
+    cudaGetLastError();
+    return fail(ZCMOE_ENOMEM, "cudaMalloc(%zu bytes) failed: %s", n * sizeof(T), cudaGetErrorString(e));
+  }
+  return ZCMOE_OK;
+}
+
+}  // namespace
+
+struct zcmoe_s {
+  zcmoe_config cfg;
+  int E, N, Z, k, d, inter, max_T, bf16, sms, device;
+  int max_chunks, max_pairs, max_mblocks;
+  zcmoe_weights w;
+  // controller state
+  float *bias, *b0, *offset, *eta, *integ, *eprev;
+  int64_t *acc_counts, *acc_tokens;  // acc_tokens = acc_counts + E (one buffer, E+1 entries)
+  int* err;
+  // workspace
+  float *logits, *gate;
+  int32_t *idx, *pos, *counts, *offsets, *mb_off, *scal, *chunk, *perm;
+  void *xperm, *H, *Y;
+  void *stage_x, *stage_y;  // device staging for zcmoe_forward_host (allocated on first use)
+  // stage timing (zcmoe_profile_begin/end): ZCMOE_NUM_STAGES + 1 events per forward
+  bool profiling;
+  std::vector<cudaEvent_t>* events;
+  // tensor maps of fixed buffers
+  CUtensorMap tm_wr, tm_wg, tm_wu, tm_wd, tm_xperm, tm_h;
+  bool alive;
+};
+
+static void release(zcmoe_s* h) {
+  void* ptrs[] = {h->bias,  h->b0,     h->offset, h->eta,   h->integ,   h->eprev,  h->acc_counts,
+                  h->err,   h->logits, h->gate,   h->idx,   h->pos,     h->counts, h->offsets,
+                  h->mb_off, h->scal,  h->chunk,  h->perm,  h->xperm,   h->H,      h->Y,
+                  h->stage_x, h->stage_y};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  if (h->events) {
+    for (cudaEvent_t e : *h->events) cudaEventDestroy(e);
+    delete h->events;
+    h->events = nullptr;
+  }
+}
+
+extern "C" {
+
+const char* zcmoe_last_error(void) { return g_err; }
+
+int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) {
+  g_err[0] = 0;
+  if (!out) return fail(ZCMOE_EINVAL, "out is NULL");
+  *out = nullptr;
+  if (!cfg || !w) return fail(ZCMOE_EINVAL, "cfg or weights is NULL");
+  const int N = cfg->n_ffn, Z = cfg->n_zero, E = N + Z, k = cfg->top_k;
+  if (N < 1 || Z < 0 || E > 1024) return fail(ZCMOE_EINVAL, "need 1 <= n_ffn and n_ffn + n_zero <= 1024");
+  if (k < 1 || k > E || k > 32) return fail(ZCMOE_EINVAL, "need 1 <= top_k <= min(E, 32)");
+  if (cfg->d < 64 || cfg->d % 64 || cfg->inter < 64 || cfg->inter % 64)
+    return fail(ZCMOE_EINVAL, "d and inter must be positive multiples of 64");
+  if (cfg->max_tokens < 1 || cfg->max_tokens > (1 << 20)) return fail(ZCMOE_EINVAL, "need 1 <= max_tokens <= 2^20");
+  if (cfg->dtype != ZCMOE_F32 && cfg->dtype != ZCMOE_BF16) return fail(ZCMOE_EINVAL, "unknown dtype");
+  if (!w->w_router || !w->w_gate || !w->w_up || !w->w_down) return fail(ZCMOE_EINVAL, "a weight pointer is NULL");
+  const void* wp[4] = {w->w_router, w->w_gate, w->w_up, w->w_down};
+  for (const void* p : wp)
+    if (reinterpret_cast<uintptr_t>(p) & 15u) return fail(ZCMOE_EINVAL, "weight pointers must be 16-byte aligned");
+  if ((int64_t)cfg->max_tokens * k >= (int64_t)1 << 31) return fail(ZCMOE_EINVAL, "max_tokens * top_k too large");
+
+  int dev = 0;
+  ZC_CUDA(cudaGetDevice(&dev));
+  cudaDeviceProp prop;
+  ZC_CUDA(cudaGetDeviceProperties(&prop, dev));
+  if (prop.major != 10) return fail(ZCMOE_EUNSUPPORTED, "device %d is sm_%d%d; this library targets sm_100a", dev,
+                                    prop.major, prop.minor);
+  if (cfg->dtype == ZCMOE_BF16 && prop.sharedMemPerBlockOptin < (size_t)zc::tc_smem_bytes())
+    return fail(ZCMOE_EUNSUPPORTED, "not enough shared memory per block");
+
+  zcmoe_s* h = new (std::nothrow) zcmoe_s();
+  if (!h) return fail(ZCMOE_ENOMEM, "host allocation failed");
+  memset(h, 0, sizeof(*h));
+  h->cfg = *cfg;
+  h->cfg.init_bias = nullptr;
+  h->cfg.logit_offset = nullptr;
+  h->E = E;
+  h->N = N;
+  h->Z = Z;
+  h->k = k;
+  h->d = cfg->d;
+  h->inter = cfg->inter;
+  h->max_T = cfg->max_tokens;
+  h->bf16 = cfg->dtype == ZCMOE_BF16;
+  h->sms = prop.multiProcessorCount;
+  h->device = dev;
+  h->w = *w;
+  h->max_chunks = (h->max_T + zc::kChunk - 1) / zc::kChunk;
+  h->max_pairs = h->max_T * k;
+  h->max_mblocks = (h->max_pairs + zc::kBM - 1) / zc::kBM + N;
+  const size_t esz = h->bf16 ? 2 : 4;
+
+  int rc = ZCMOE_OK;
+#define ZC_ALLOC(p, n)                     \
+  if (rc == ZCMOE_OK) rc = dalloc(&(p), (n));
+  ZC_ALLOC(h->bias, E);
+  ZC_ALLOC(h->b0, E);
+  if (cfg->logit_offset) ZC_ALLOC(h->offset, E);
+  ZC_ALLOC(h->eta, 1);
+  ZC_ALLOC(h->integ, E);
+  ZC_ALLOC(h->eprev, E);
+  ZC_ALLOC(h->acc_counts, E + 1);
+  ZC_ALLOC(h->err, 1);
+  ZC_ALLOC(h->logits, (size_t)h->max_T * E);
+  ZC_ALLOC(h->gate, (size_t)h->max_pairs);
+  ZC_ALLOC(h->idx, (size_t)h->max_pairs);
+  ZC_ALLOC(h->pos, (size_t)h->max_pairs);
+  ZC_ALLOC(h->counts, E);
+  ZC_ALLOC(h->offsets, N + 1);
+  ZC_ALLOC(h->mb_off, N + 1);
+  ZC_ALLOC(h->scal, 4);
+  ZC_ALLOC(h->chunk, (size_t)h->max_chunks * E);
+  ZC_ALLOC(h->perm, (size_t)h->max_pairs);
+  {
+    uint8_t *xp = nullptr, *hh = nullptr, *yy = nullptr;
+    ZC_ALLOC(xp, (size_t)h->max_pairs * h->d * esz);
+    ZC_ALLOC(hh, (size_t)h->max_pairs * h->inter * esz);
+    ZC_ALLOC(yy, (size_t)h->max_pairs * h->d * esz);
+    h->xperm = xp;
+    h->H = hh;
+    h->Y = yy;
+  }
+#undef ZC_ALLOC
+  if (rc != ZCMOE_OK) {
+    release(h);
+    delete h;
+    return rc;
+  }
+  h->acc_tokens = h->acc_counts + E;
+
+  // initial state: bias = b0 = init_bias (or 0), eta = 1, integral/previous error = 0
+  {
+    float* hb = new (std::nothrow) float[E];
+    if (!hb) {
+      release(h);
+      delete h;
+      return fail(ZCMOE_ENOMEM, "host allocation failed");
+    }
+    for (int i = 0; i < E; ++i) hb[i] = cfg->init_bias ? cfg->init_bias[i] : 0.0f;
+    const float one = 1.0f;
+    cudaError_t e = cudaMemcpy(h->bias, hb, E * sizeof(float), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(h->b0, hb, E * sizeof(float), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && cfg->logit_offset)
+      e = cudaMemcpy(h->offset, cfg->logit_offset, E * sizeof(float), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(h->eta, &one, sizeof(float), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemset(h->integ, 0, E * sizeof(float));
+    if (e == cudaSuccess) e = cudaMemset(h->eprev, 0, E * sizeof(float));
+    if (e == cudaSuccess) e = cudaMemset(h->acc_counts, 0, (E + 1) * sizeof(int64_t));
+    if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(h->xperm, 0, (size_t)h->max_pairs * h->d * esz);
+    if (e == cudaSuccess) e = cudaMemset(h->H, 0, (size_t)h->max_pairs * h->inter * esz);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    delete[] hb;
+    if (e != cudaSuccess) {
+      release(h);
+      delete h;
+      return fail(ZCMOE_ECUDA, "initialising state: %s", cudaGetErrorString(e));
+    }
+  }
+
+  if (h->bf16) {
+    const uint64_t d = h->d, inter = h->inter;
+    rc = make_tmap(&h->tm_wr, w->w_router, d, (uint64_t)E, 256);
+    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wg, w->w_gate, d, (uint64_t)N * inter, 128);
+    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wu, w->w_up, d, (uint64_t)N * inter, 128);
+    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wd, w->w_down, inter, (uint64_t)N * d, 256);
+    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_xperm, h->xperm, d, (uint64_t)h->max_pairs, 128);
+    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_h, h->H, inter, (uint64_t)h->max_pairs, 128);
+    if (rc != ZCMOE_OK) {
+      release(h);
+      delete h;
+      return rc;
+    }
+  }
+  h->alive = true;
+  {
+    std::lock_guard<std::mutex> lk(g_live_mu);
+    g_live.insert(h);
+  }
+  *out = h;
+  return ZCMOE_OK;
+}
+
+int zcmoe_forward(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream_t s, const zcmoe_debug* dbg) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (T < 0 || T > h->max_T) return fail(ZCMOE_ERANGE, "T=%lld outside [0, %d]", (long long)T, h->max_T);
+  if (T == 0) return ZCMOE_OK;
+  if (!x || !y) return fail(ZCMOE_EINVAL, "x or y is NULL");
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(y) & 15u))
+    return fail(ZCMOE_EINVAL, "x and y must be 16-byte aligned");
+  const size_t esz = h->bf16 ? 2 : 4;
+  const size_t xbytes = (size_t)T * h->d * esz;
+  const uintptr_t xa = reinterpret_cast<uintptr_t>(x), ya = reinterpret_cast<uintptr_t>(y);
+  if (xa < ya + xbytes && ya < xa + xbytes) return fail(ZCMOE_EINVAL, "y overlaps x");
+
+  const int Ti = (int)T, E = h->E, N = h->N, k = h->k, d = h->d, inter = h->inter;
+  const int nchunks = (Ti + zc::kChunk - 1) / zc::kChunk;
+  auto mark = [&]() -> cudaError_t {
+    if (!h->profiling) return cudaSuccess;
+    cudaEvent_t ev;
+    cudaError_t e = cudaEventCreate(&ev);
+    if (e != cudaSuccess) return e;
+    h->events->push_back(ev);
+    return cudaEventRecord(ev, s);
+  };
+  ZC_CUDA(mark());
+
+  // 1. router logits
+  if (h->bf16) {
+    CUtensorMap tm_x;
+    int rc = make_tmap(&tm_x, x, (uint64_t)d, (uint64_t)T, 128);
+    if (rc != ZCMOE_OK) return rc;
+    zc::TcArgs a{};
+    a.K = d;
+    a.n_out = E;
+    a.nblocks = (E + zc::tc_block_n(zc::kRouter) - 1) / zc::tc_block_n(zc::kRouter);
+    a.ngroups = 1;
+    a.M = Ti;
+    a.out = h->logits;
+    a.ldo = E;
+    a.col_add = h->offset;
+    a.err = h->err;
+    const int tiles = ((Ti + zc::kBM - 1) / zc::kBM) * a.nblocks;
+    ZC_CUDA(zc::launch_tc_gemm(zc::kRouter, tm_x, h->tm_wr, h->tm_wr, a, tiles < h->sms ? tiles : h->sms, s));
+  } else {
+    zc::SimtArgs a{};
+    a.A = static_cast<const float*>(x);
+    a.B0 = static_cast<const float*>(h->w.w_router);
+    a.K = d;
+    a.n_out = E;
+    a.ngroups = 1;
+    a.M = Ti;
+    a.out = h->logits;
+    a.ldo = E;
+    a.col_add = h->offset;
+    ZC_CUDA(zc::launch_simt_gemm(zc::kRouter, a, (Ti + zc::kBM - 1) / zc::kBM, s));
+  }
+  ZC_CUDA(mark());
+  // 2. softmax + bias-shifted top-k
+  ZC_CUDA(zc::launch_softmax_topk(h->logits, h->bias, Ti, E, k, h->cfg.routed_scale, h->idx, h->gate,
+                                  dbg ? dbg->scores : nullptr, h->sms, s));
+  ZC_CUDA(mark());
+  // 3. integer stage
+  ZC_CUDA(zc::launch_route_count(h->idx, Ti, k, E, h->chunk, s));
+  ZC_CUDA(zc::launch_route_scan(h->chunk, nchunks, Ti, N, E, h->counts, h->offsets, h->mb_off, h->scal,
+                                h->acc_counts, h->acc_tokens, s));
+  ZC_CUDA(zc::launch_route_scatter(h->idx, Ti, k, N, E, h->chunk, h->perm, h->pos, s));
+  ZC_CUDA(mark());
+  // 4. gather the FFN pairs' rows
+  ZC_CUDA(zc::launch_gather_rows(x, (int)(d * esz), h->perm, k, h->scal, h->xperm, h->sms, s));
+  ZC_CUDA(mark());
+  // 5./6. expert GEMMs
+  const int max_mb = (Ti * k + zc::kBM - 1) / zc::kBM + N;
+  if (h->bf16) {
+    zc::TcArgs a{};
+    a.K = d;
+    a.n_out = inter;
+    a.nblocks = (inter + zc::tc_block_n(zc::kGateUp) - 1) / zc::tc_block_n(zc::kGateUp);
+    a.ngroups = N;
+    a.row_off = h->offsets;
+    a.mb_off = h->mb_off;
+    a.b_rows_per_group = inter;
+    a.out = h->H;
+    a.ldo = inter;
+    a.err = h->err;
+    int bound = max_mb * a.nblocks;
+    ZC_CUDA(zc::launch_tc_gemm(zc::kGateUp, h->tm_xperm, h->tm_wg, h->tm_wu, a, bound < h->sms ? bound : h->sms, s));
+    ZC_CUDA(mark());
+    zc::TcArgs b{};
+    b.K = inter;
+    b.n_out = d;
+    b.nblocks = (d + zc::tc_block_n(zc::kDown) - 1) / zc::tc_block_n(zc::kDown);
+    b.ngroups = N;
+    b.row_off = h->offsets;
+    b.mb_off = h->mb_off;
+    b.b_rows_per_group = d;
+    b.out = h->Y;
+    b.ldo = d;
+    b.err = h->err;
+    bound = max_mb * b.nblocks;
+    ZC_CUDA(zc::launch_tc_gemm(zc::kDown, h->tm_h, h->tm_wd, h->tm_wd, b, bound < h->sms ? bound : h->sms, s));
+  } else {
+    zc::SimtArgs a{};
+    a.A = static_cast<const float*>(h->xperm);
+    a.B0 = static_cast<const float*>(h->w.w_gate);
+    a.B1 = static_cast<const float*>(h->w.w_up);
+    a.K = d;
+    a.n_out = inter;
+    a.ngroups = N;
+    a.row_off = h->offsets;
+    a.mb_off = h->mb_off;
+    a.b_rows_per_group = inter;
+    a.out = static_cast<float*>(h->H);
+    a.ldo = inter;
+    ZC_CUDA(zc::launch_simt_gemm(zc::kGateUp, a, max_mb, s));
+    ZC_CUDA(mark());
+    zc::SimtArgs b{};
+    b.A = static_cast<const float*>(h->H);
+    b.B0 = static_cast<const float*>(h->w.w_down);
+    b.K = inter;
+    b.n_out = d;
+    b.ngroups = N;
+    b.row_off = h->offsets;
+    b.mb_off = h->mb_off;
+    b.b_rows_per_group = d;
+    b.out = static_cast<float*>(h->Y);
+    b.ldo = d;
+    ZC_CUDA(zc::launch_simt_gemm(zc::kDown, b, max_mb, s));
+  }
+  ZC_CUDA(mark());
+  // 7. combine
+  ZC_CUDA(zc::launch_combine(h->bf16, x, h->Y, h->idx, h->gate, h->pos, Ti, k, N, d, y, h->sms, s));
+  ZC_CUDA(mark());
+
+  if (dbg) {
+    if (dbg->logits) ZC_CUDA(cudaMemcpyAsync(dbg->logits, h->logits, (size_t)T * E * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->idx) ZC_CUDA(cudaMemcpyAsync(dbg->idx, h->idx, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->gate) ZC_CUDA(cudaMemcpyAsync(dbg->gate, h->gate, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->counts) ZC_CUDA(cudaMemcpyAsync(dbg->counts, h->counts, (size_t)E * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->offsets)
+      ZC_CUDA(cudaMemcpyAsync(dbg->offsets, h->offsets, (size_t)(N + 1) * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->perm) ZC_CUDA(cudaMemcpyAsync(dbg->perm, h->perm, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->pos) ZC_CUDA(cudaMemcpyAsync(dbg->pos, h->pos, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->expert_out)
+      ZC_CUDA(cudaMemcpyAsync(dbg->expert_out, h->Y, (size_t)T * k * d * esz, cudaMemcpyDeviceToDevice, s));
+  }
+  return ZCMOE_OK;
+}
+
+int zcmoe_forward_host(zcmoe_t h, const void* x_host, int64_t T, void* y_host, cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (T < 0 || T > h->max_T) return fail(ZCMOE_ERANGE, "T=%lld outside [0, %d]", (long long)T, h->max_T);
+  if (T == 0) return ZCMOE_OK;
+  if (!x_host || !y_host) return fail(ZCMOE_EINVAL, "x or y is NULL");
+  const size_t bytes_max = (size_t)h->max_T * h->d * (h->bf16 ? 2 : 4);
+  if (!h->stage_x) {
+    uint8_t *a = nullptr, *b = nullptr;
+    int rc = dalloc(&a, bytes_max);
+    if (rc == ZCMOE_OK) rc = dalloc(&b, bytes_max);
+    if (rc != ZCMOE_OK) {
+      if (a) cudaFree(a);
+      return rc;
+    }
+    h->stage_x = a;
+    h->stage_y = b;
+  }
+  const size_t bytes = (size_t)T * h->d * (h->bf16 ? 2 : 4);
+  ZC_CUDA(cudaMemcpyAsync(h->stage_x, x_host, bytes, cudaMemcpyHostToDevice, s));
+  int rc = zcmoe_forward(h, h->stage_x, T, h->stage_y, s, nullptr);
+  if (rc != ZCMOE_OK) return rc;
+  ZC_CUDA(cudaMemcpyAsync(y_host, h->stage_y, bytes, cudaMemcpyDeviceToHost, s));
+  return ZCMOE_OK;
+}
+
+int zcmoe_update_bias(zcmoe_t h, const zcmoe_gains* g, cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (!g) return fail(ZCMOE_EINVAL, "gains is NULL");
+  if (!(g->target_ffn_per_token >= 0.0f && g->target_ffn_per_token <= (float)h->k))
+    return fail(ZCMOE_EINVAL, "target_ffn_per_token must lie in [0, top_k]");
+  if (h->Z == 0 && g->target_ffn_per_token != (float)h->k)
+    return fail(ZCMOE_EINVAL, "without zero experts the FFN target must equal top_k");
+  ZC_CUDA(zc::launch_update_bias(h->acc_counts, h->acc_tokens, h->N, h->Z, h->k, g->kp, g->ki, g->kd, g->decay,
+                                 g->target_ffn_per_token, h->b0, h->eta, h->integ, h->eprev, h->bias, s));
+  return ZCMOE_OK;
+}
+
+int zcmoe_read_counts(zcmoe_t h, int64_t* dst, cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (!dst) return fail(ZCMOE_EINVAL, "dst is NULL");
+  ZC_CUDA(cudaMemcpyAsync(dst, h->acc_counts, (size_t)(h->E + 1) * sizeof(int64_t), cudaMemcpyDeviceToDevice, s));
+  return ZCMOE_OK;
+}
+
+int zcmoe_write_counts(zcmoe_t h, const int64_t* src, cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (!src) return fail(ZCMOE_EINVAL, "src is NULL");
+  ZC_CUDA(cudaMemcpyAsync(h->acc_counts, src, (size_t)(h->E + 1) * sizeof(int64_t), cudaMemcpyDeviceToDevice, s));
+  return ZCMOE_OK;
+}
+
+int zcmoe_get_state(zcmoe_t h, float* bias, int64_t* counts, int64_t* tokens, float* eta) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  ZC_CUDA(cudaDeviceSynchronize());
+  if (bias) ZC_CUDA(cudaMemcpy(bias, h->bias, h->E * sizeof(float), cudaMemcpyDeviceToHost));
+  if (counts) ZC_CUDA(cudaMemcpy(counts, h->acc_counts, h->E * sizeof(int64_t), cudaMemcpyDeviceToHost));
+  if (tokens) ZC_CUDA(cudaMemcpy(tokens, h->acc_tokens, sizeof(int64_t), cudaMemcpyDeviceToHost));
+  if (eta) ZC_CUDA(cudaMemcpy(eta, h->eta, sizeof(float), cudaMemcpyDeviceToHost));
+  return ZCMOE_OK;
+}
+
+int zcmoe_set_bias(zcmoe_t h, const float* bias) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (!bias) return fail(ZCMOE_EINVAL, "bias is NULL");
+  ZC_CUDA(cudaDeviceSynchronize());
+  ZC_CUDA(cudaMemcpy(h->bias, bias, h->E * sizeof(float), cudaMemcpyHostToDevice));
+  return ZCMOE_OK;
+}
+
+int zcmoe_check(zcmoe_t h) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  ZC_CUDA(cudaDeviceSynchronize());
+  int code = 0;
+  ZC_CUDA(cudaMemcpy(&code, h->err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (code) {
+    ZC_CUDA(cudaMemset(h->err, 0, sizeof(int)));
+    return fail(ZCMOE_ETIMEOUT, "a device-side wait timed out (site %d)", code);
+  }
+  return ZCMOE_OK;
+}
+
+int zcmoe_profile_begin(zcmoe_t h) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (!h->events) h->events = new (std::nothrow) std::vector<cudaEvent_t>();
+  if (!h->events) return fail(ZCMOE_ENOMEM, "host allocation failed");
+  for (cudaEvent_t e : *h->events) cudaEventDestroy(e);
+  h->events->clear();
+  h->profiling = true;
+  return ZCMOE_OK;
+}
+
+int zcmoe_profile_end(zcmoe_t h, float* ms, int32_t* n_forwards) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (!h->profiling || !h->events) return fail(ZCMOE_EINVAL, "profiling was not started");
+  h->profiling = false;
+  ZC_CUDA(cudaDeviceSynchronize());
+  const size_t per = ZCMOE_NUM_STAGES + 1;
+  const size_t n = h->events->size() / per;
+  for (int i = 0; i < ZCMOE_NUM_STAGES; ++i) ms[i] = 0.0f;
+  for (size_t f = 0; f < n; ++f) {
+    for (int i = 0; i < ZCMOE_NUM_STAGES; ++i) {
+      float t = 0.0f;
+      ZC_CUDA(cudaEventElapsedTime(&t, (*h->events)[f * per + i], (*h->events)[f * per + i + 1]));
+      ms[i] += t;
+    }
+  }
+  if (n_forwards) *n_forwards = (int32_t)n;
+  for (cudaEvent_t e : *h->events) cudaEventDestroy(e);
+  h->events->clear();
+  return ZCMOE_OK;
+}
+
+int zcmoe_destroy(zcmoe_t h) {
+  g_err[0] = 0;
+  if (!h) return ZCMOE_OK;
+  {
+    std::lock_guard<std::mutex> lk(g_live_mu);
+    if (!g_live.erase(h)) return fail(ZCMOE_EINVAL, "invalid or already destroyed handle");
+  }
+  h->alive = false;
+  cudaDeviceSynchronize();
+  release(h);
+  delete h;
+  return ZCMOE_OK;
+}
+
+}  // extern "C"

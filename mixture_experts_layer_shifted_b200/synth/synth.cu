@@ -67,14 +67,14 @@ extern "C" {
 
 // Fills dst[0..n) (device, float32 if bf16 == 0 else bfloat16) with the normal recipe.
 // Returns 0 or the cudaError_t of the launch.
-int zcsynth_normal(void* dst, int64_t n, int bf16, uint32_t tid, uint64_t seed, float stdv, cudaStream_t stream) {
+__attribute__((visibility("default"))) int zcsynth_normal(void* dst, int64_t n, int bf16, uint32_t tid, uint64_t seed, float stdv, cudaStream_t stream) {
   if (n <= 0) return 0;
   k_normal<<<grid_for(n), 256, 0, stream>>>(dst, n, bf16, tid, seed, stdv);
   return (int)cudaGetLastError();
 }
 
 // Fills dst[0..n) (device float32) with the uniform recipe on (lo, hi).
-int zcsynth_uniform(float* dst, int64_t n, uint32_t tid, uint64_t seed, float lo, float hi, cudaStream_t stream) {
+__attribute__((visibility("default"))) int zcsynth_uniform(float* dst, int64_t n, uint32_t tid, uint64_t seed, float lo, float hi, cudaStream_t stream) {
   if (n <= 0) return 0;
   k_uniform<<<grid_for(n), 256, 0, stream>>>(dst, n, tid, seed, lo, hi);
   return (int)cudaGetLastError();

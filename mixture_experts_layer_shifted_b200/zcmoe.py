@@ -1,0 +1,275 @@
+"""ctypes binding of libzcmoe.so (C ABI in include/zcmoe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch supplies device memory and streams.  There is no fallback:
+if the library is missing or the device is not an sm_100 part, calls fail.
+
+The functions carry the C names; ``ZcMoE`` is a small owner object that keeps
+the weight tensors alive for the handle's lifetime.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch  # noqa: F401  (loads the CUDA runtime the library links against)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzcmoe.so")
+
+ZCMOE_OK = 0
+ZCMOE_EINVAL = -1
+ZCMOE_ERANGE = -2
+ZCMOE_ENOMEM = -3
+ZCMOE_ECUDA = -4
+ZCMOE_EUNSUPPORTED = -5
+ZCMOE_ETIMEOUT = -6
+ZCMOE_F32 = 0
+ZCMOE_BF16 = 1
+
+EXPORTED = ("zcmoe_create", "zcmoe_forward", "zcmoe_forward_host", "zcmoe_update_bias", "zcmoe_read_counts",
+            "zcmoe_write_counts", "zcmoe_get_state", "zcmoe_set_bias", "zcmoe_check", "zcmoe_profile_begin",
+            "zcmoe_profile_end", "zcmoe_destroy", "zcmoe_last_error")
+STAGES = ("router", "softmax_topk", "integer", "gather", "gate_up", "down", "combine")
+
+
+class ZcmoeError(RuntimeError):
+    def __init__(self, code, where, msg):
+        super().__init__(f"{where} failed with code {code}: {msg}")
+        self.code = code
+
+
+class zcmoe_config(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("n_ffn", ctypes.c_int32), ("n_zero", ctypes.c_int32),
+                ("inter", ctypes.c_int32), ("top_k", ctypes.c_int32), ("max_tokens", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("routed_scale", ctypes.c_float),
+                ("init_bias", ctypes.POINTER(ctypes.c_float)), ("logit_offset", ctypes.POINTER(ctypes.c_float))]
+
+
+class zcmoe_weights(ctypes.Structure):
+    _fields_ = [("w_router", ctypes.c_void_p), ("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p),
+                ("w_down", ctypes.c_void_p)]
+
+
+class zcmoe_gains(ctypes.Structure):
+    _fields_ = [("kp", ctypes.c_float), ("ki", ctypes.c_float), ("kd", ctypes.c_float), ("decay", ctypes.c_float),
+                ("target_ffn_per_token", ctypes.c_float)]
+
+
+class zcmoe_debug(ctypes.Structure):
+    _fields_ = [("logits", ctypes.c_void_p), ("scores", ctypes.c_void_p), ("idx", ctypes.c_void_p),
+                ("gate", ctypes.c_void_p), ("counts", ctypes.c_void_p), ("offsets", ctypes.c_void_p),
+                ("perm", ctypes.c_void_p), ("pos", ctypes.c_void_p), ("expert_out", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """Loads libzcmoe.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.zcmoe_create.argtypes = [ctypes.POINTER(zcmoe_config), ctypes.POINTER(zcmoe_weights), ctypes.POINTER(vp)]
+        L.zcmoe_forward.argtypes = [vp, vp, i64, vp, vp, ctypes.POINTER(zcmoe_debug)]
+        L.zcmoe_forward_host.argtypes = [vp, vp, i64, vp, vp]
+        L.zcmoe_update_bias.argtypes = [vp, ctypes.POINTER(zcmoe_gains), vp]
+        L.zcmoe_read_counts.argtypes = [vp, vp, vp]
+        L.zcmoe_write_counts.argtypes = [vp, vp, vp]
+        L.zcmoe_get_state.argtypes = [vp, vp, vp, vp, vp]
+        L.zcmoe_set_bias.argtypes = [vp, vp]
+        L.zcmoe_check.argtypes = [vp]
+        L.zcmoe_destroy.argtypes = [vp]
+        L.zcmoe_profile_begin.argtypes = [vp]
+        L.zcmoe_profile_end.argtypes = [vp, vp, vp]
+        for f in EXPORTED[:-1]:
+            getattr(L, f).restype = i32
+        L.zcmoe_last_error.argtypes = []
+        L.zcmoe_last_error.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(rc, where):
+    if rc != ZCMOE_OK:
+        raise ZcmoeError(rc, where, lib().zcmoe_last_error().decode(errors="replace"))
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+# ----------------------------------------------------------------- C names
+def zcmoe_create(cfg: zcmoe_config, w: zcmoe_weights) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(lib().zcmoe_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)), "zcmoe_create")
+    return h
+
+
+def zcmoe_forward(h, x_ptr, T, y_ptr, stream=None, dbg: zcmoe_debug | None = None):
+    _check(lib().zcmoe_forward(h, x_ptr, T, y_ptr, _stream(stream), ctypes.byref(dbg) if dbg is not None else None),
+           "zcmoe_forward")
+
+
+def zcmoe_forward_host(h, x_host_ptr, T, y_host_ptr, stream=None):
+    _check(lib().zcmoe_forward_host(h, x_host_ptr, T, y_host_ptr, _stream(stream)), "zcmoe_forward_host")
+
+
+def zcmoe_update_bias(h, gains: zcmoe_gains, stream=None):
+    _check(lib().zcmoe_update_bias(h, ctypes.byref(gains), _stream(stream)), "zcmoe_update_bias")
+
+
+def zcmoe_read_counts(h, dst_ptr, stream=None):
+    _check(lib().zcmoe_read_counts(h, dst_ptr, _stream(stream)), "zcmoe_read_counts")
+
+
+def zcmoe_write_counts(h, src_ptr, stream=None):
+    _check(lib().zcmoe_write_counts(h, src_ptr, _stream(stream)), "zcmoe_write_counts")
+
+
+def zcmoe_get_state(h, bias_ptr=None, counts_ptr=None, tokens_ptr=None, eta_ptr=None):
+    _check(lib().zcmoe_get_state(h, bias_ptr, counts_ptr, tokens_ptr, eta_ptr), "zcmoe_get_state")
+
+
+def zcmoe_set_bias(h, bias_ptr):
+    _check(lib().zcmoe_set_bias(h, bias_ptr), "zcmoe_set_bias")
+
+
+def zcmoe_check(h):
+    _check(lib().zcmoe_check(h), "zcmoe_check")
+
+
+def zcmoe_profile_begin(h):
+    _check(lib().zcmoe_profile_begin(h), "zcmoe_profile_begin")
+
+
+def zcmoe_profile_end(h):
+    """Returns ({stage: total ms}, number of forwards recorded)."""
+    ms = (ctypes.c_float * len(STAGES))()
+    n = ctypes.c_int32()
+    _check(lib().zcmoe_profile_end(h, ms, ctypes.byref(n)), "zcmoe_profile_end")
+    return dict(zip(STAGES, [float(v) for v in ms])), int(n.value)
+
+
+def zcmoe_destroy(h):
+    _check(lib().zcmoe_destroy(h), "zcmoe_destroy")
+
+
+def zcmoe_last_error() -> str:
+    return lib().zcmoe_last_error().decode(errors="replace")
+
+
+# ----------------------------------------------------------------- owner object
+@dataclass
+class LayerShape:
+    d: int
+    n_ffn: int
+    n_zero: int
+    inter: int
+    top_k: int
+    dtype: str = "bf16"  # "bf16" or "f32"
+    routed_scale: float = 1.0
+
+    @property
+    def E(self):
+        return self.n_ffn + self.n_zero
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+
+class ZcMoE:
+    """Owns a handle plus references to its (borrowed) device weights."""
+
+    def __init__(self, shape: LayerShape, w_router, w_gate, w_up, w_down, max_tokens: int, init_bias=None,
+                 logit_offset=None):
+        import numpy as np
+        self.shape = shape
+        self.weights = (w_router, w_gate, w_up, w_down)
+        E = shape.E
+        for t, want in zip(self.weights, [(E, shape.d), (shape.n_ffn, shape.inter, shape.d),
+                                          (shape.n_ffn, shape.inter, shape.d), (shape.n_ffn, shape.d, shape.inter)]):
+            if tuple(t.shape) != want or t.dtype != shape.torch_dtype or not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"weight of shape {tuple(t.shape)} {t.dtype}; expected {want} {shape.torch_dtype}")
+        self._bias0 = None if init_bias is None else np.ascontiguousarray(init_bias, dtype=np.float32)
+        self._offset = None if logit_offset is None else np.ascontiguousarray(logit_offset, dtype=np.float32)
+        fp = ctypes.POINTER(ctypes.c_float)
+        cfg = zcmoe_config(shape.d, shape.n_ffn, shape.n_zero, shape.inter, shape.top_k, max_tokens,
+                           ZCMOE_BF16 if shape.dtype == "bf16" else ZCMOE_F32, shape.routed_scale,
+                           None if self._bias0 is None else self._bias0.ctypes.data_as(fp),
+                           None if self._offset is None else self._offset.ctypes.data_as(fp))
+        w = zcmoe_weights(w_router.data_ptr(), w_gate.data_ptr(), w_up.data_ptr(), w_down.data_ptr())
+        self.max_tokens = max_tokens
+        self.h = zcmoe_create(cfg, w)
+
+    def forward(self, x, y=None, stream=None, debug: dict | None = None):
+        """y = layer(x); ``debug`` maps zcmoe_debug field names to device tensors to fill."""
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty_like(x)
+        dbg = None
+        if debug:
+            dbg = zcmoe_debug(**{k: v.data_ptr() for k, v in debug.items()})
+        zcmoe_forward(self.h, ctypes.c_void_p(x.data_ptr()), T, ctypes.c_void_p(y.data_ptr()), stream, dbg)
+        return y
+
+    def forward_host(self, x_host, y_host, stream=None):
+        zcmoe_forward_host(self.h, ctypes.c_void_p(x_host.data_ptr()), x_host.shape[0],
+                           ctypes.c_void_p(y_host.data_ptr()), stream)
+        return y_host
+
+    def update_bias(self, kp=0.0, ki=0.0, kd=0.0, decay=1.0, target_ffn_per_token=None, stream=None):
+        K = float(self.shape.top_k if target_ffn_per_token is None else target_ffn_per_token)
+        zcmoe_update_bias(self.h, zcmoe_gains(kp, ki, kd, decay, K), stream)
+
+    def read_counts(self, dst, stream=None):
+        zcmoe_read_counts(self.h, ctypes.c_void_p(dst.data_ptr()), stream)
+
+    def write_counts(self, src, stream=None):
+        zcmoe_write_counts(self.h, ctypes.c_void_p(src.data_ptr()), stream)
+
+    def state(self):
+        import numpy as np
+        E = self.shape.E
+        bias = np.empty(E, np.float32)
+        counts = np.empty(E, np.int64)
+        tokens = np.empty(1, np.int64)
+        eta = np.empty(1, np.float32)
+        zcmoe_get_state(self.h, bias.ctypes.data, counts.ctypes.data, tokens.ctypes.data, eta.ctypes.data)
+        return {"bias": bias, "counts": counts, "tokens": int(tokens[0]), "eta": float(eta[0])}
+
+    def set_bias(self, bias):
+        import numpy as np
+        b = np.ascontiguousarray(bias, dtype=np.float32)
+        zcmoe_set_bias(self.h, b.ctypes.data)
+
+    def check(self):
+        zcmoe_check(self.h)
+
+    def profile_begin(self):
+        zcmoe_profile_begin(self.h)
+
+    def profile_end(self):
+        return zcmoe_profile_end(self.h)
+
+    def close(self):
+        if self.h is not None:
+            zcmoe_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -248,9 +248,9 @@ ZO_EXPORT int64_t zo_integer_stage(const int32_t *idx, int64_t T, int k, int N, 
 /* ------------------------------------------------------------------------- */
 ZO_EXPORT void zo_ffn_f64(const void *xs, int x_dtype, int64_t n, const void *wg, const void *wu,
                           const void *wd, int w_dtype, int d, int inter, double *out) {
-#pragma omp parallel for schedule(dynamic)
+  double *h = (double *)malloc(sizeof(double) * (size_t)inter);
   for (int64_t r = 0; r < n; ++r) {
-    double *h = (double *)malloc(sizeof(double) * (size_t)inter);
+#pragma omp parallel for schedule(static)
     for (int i = 0; i < inter; ++i) {
       double g = 0.0, u = 0.0;
       for (int c = 0; c < d; ++c) {
@@ -260,13 +260,14 @@ ZO_EXPORT void zo_ffn_f64(const void *xs, int x_dtype, int64_t n, const void *wg
       }
       h[i] = g / (1.0 + exp(-g)) * u;
     }
+#pragma omp parallel for schedule(static)
     for (int c = 0; c < d; ++c) {
       double acc = 0.0;
       for (int i = 0; i < inter; ++i) acc += elem(wd, w_dtype, (int64_t)c * inter + i) * h[i];
       out[r * d + c] = acc;
     }
-    free(h);
   }
+  free(h);
 }
 
 /* ------------------------------------------------------------------------- */

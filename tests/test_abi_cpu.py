@@ -1,0 +1,85 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point the header declares, and rejects bad arguments before it
+touches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "zcmoe.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"ZCMOE_API\s+[\w\s\*]+?\b(zcmoe_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def zc():
+    from mixture_experts_layer_shifted_b200 import build
+    build.build()
+    from mixture_experts_layer_shifted_b200 import zcmoe
+    return zcmoe
+
+
+def test_header_declares_the_four_calls():
+    names = _declared()
+    for n in ("zcmoe_create", "zcmoe_forward", "zcmoe_update_bias", "zcmoe_destroy"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(zc):
+    lib = zc.lib()
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert sorted(zc.EXPORTED) == _declared()
+
+
+def test_synth_library_exports():
+    from mixture_experts_layer_shifted_b200 import build, synth
+    build.build()
+    lib = synth.device_lib()
+    assert hasattr(lib, "zcsynth_normal") and hasattr(lib, "zcsynth_uniform")
+
+
+def test_bad_arguments_are_rejected_on_the_host(zc):
+    lib = zc.lib()
+    h = ctypes.c_void_p()
+    cfg = zc.zcmoe_config(256, 16, 8, 128, 4, 64, zc.ZCMOE_F32, 1.0, None, None)
+    w = zc.zcmoe_weights(16, 16, 16, 16)
+    assert lib.zcmoe_create(None, ctypes.byref(w), ctypes.byref(h)) == zc.ZCMOE_EINVAL
+    assert lib.zcmoe_create(ctypes.byref(cfg), ctypes.byref(w), None) == zc.ZCMOE_EINVAL
+    for bad in [dict(d=100), dict(inter=0), dict(top_k=0), dict(top_k=33), dict(n_ffn=0), dict(n_zero=2000),
+                dict(max_tokens=0), dict(dtype=7)]:
+        c = zc.zcmoe_config(256, 16, 8, 128, 4, 64, zc.ZCMOE_F32, 1.0, None, None)
+        for k_, v in bad.items():
+            setattr(c, k_, v)
+        assert lib.zcmoe_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(h)) == zc.ZCMOE_EINVAL, bad
+        assert h.value is None
+        assert zc.zcmoe_last_error() != ""
+    w_bad = zc.zcmoe_weights(16, 17, 16, 16)  # misaligned
+    assert lib.zcmoe_create(ctypes.byref(cfg), ctypes.byref(w_bad), ctypes.byref(h)) == zc.ZCMOE_EINVAL
+    w_null = zc.zcmoe_weights(16, None, 16, 16)
+    assert lib.zcmoe_create(ctypes.byref(cfg), ctypes.byref(w_null), ctypes.byref(h)) == zc.ZCMOE_EINVAL
+    # handles that were never created are refused, not dereferenced
+    fake = ctypes.c_void_p(0x1000)
+    assert lib.zcmoe_forward(fake, None, 1, None, None, None) == zc.ZCMOE_EINVAL
+    assert lib.zcmoe_update_bias(fake, None, None) == zc.ZCMOE_EINVAL
+    assert lib.zcmoe_check(fake) == zc.ZCMOE_EINVAL
+    assert lib.zcmoe_destroy(fake) == zc.ZCMOE_EINVAL
+    assert lib.zcmoe_destroy(None) == zc.ZCMOE_OK
+
+
+def test_create_without_a_device_fails_cleanly(zc):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    lib = zc.lib()
+    h = ctypes.c_void_p()
+    cfg = zc.zcmoe_config(256, 16, 8, 128, 4, 64, zc.ZCMOE_F32, 1.0, None, None)
+    w = zc.zcmoe_weights(16, 16, 16, 16)
+    rc = lib.zcmoe_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h))
+    assert rc in (zc.ZCMOE_ECUDA, zc.ZCMOE_EUNSUPPORTED)
+    assert h.value is None
