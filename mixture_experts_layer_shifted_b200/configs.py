@@ -63,6 +63,10 @@ WORKLOADS = {
                                       notes="literal +0.5 on zero experts: every pick is a zero expert"),
     "skewed_4096": Workload("skewed_4096", T=32768, d=4096, n_ffn=256, inter=1024, n_zero=128, top_k=8, dtype="bf16",
                             w_std=0.02, bias=("zero",), zipf_s=1.1, steps=100, target_ffn=6.0),
+    # small case of the prefill kernels for profiler captures: a few GB on the device,
+    # inputs still larger than L2
+    "prefill_probe": Workload("prefill_probe", T=2048, d=6144, n_ffn=32, inter=2048, n_zero=16, top_k=12,
+                              dtype="bf16", w_std=0.006, bias=("zero",)),
 }
 
 

@@ -57,6 +57,7 @@ class Run:
         self.layer = ZcMoE(self.shape, *self.weights, max_tokens=max_tokens or max(self.T, 1), init_bias=self.bias,
                            logit_offset=self.offset)
         self.x = configs.device_tokens(w, self.T) if x is None else x
+        self.cur_bias = self.bias  # the bias the layer routes with now (changes with update_bias)
 
     def forward(self, debug=True):
         T, E, k, d = self.T, self.w.E, self.w.top_k, self.w.d
@@ -103,7 +104,7 @@ class Run:
         GPU's indices must reproduce every integer and every fp32 value."""
         d = self.dbg
         k = self.w.top_k
-        idx, gate, scores = oracle.route_replica_f32(d["logits"], self.bias, k, self.shape.routed_scale,
+        idx, gate, scores = oracle.route_replica_f32(d["logits"], self.cur_bias, k, self.shape.routed_scale,
                                                      want_scores=True)
         np.testing.assert_array_equal(d["scores"].view(np.uint32), scores.view(np.uint32))
         np.testing.assert_array_equal(d["idx"], idx)
@@ -129,7 +130,7 @@ class Run:
         bound = self.w.d * 2.0 ** -23 * (xs @ ws.T) + 1e-6
         assert np.all(np.abs(got - ref) <= bound)
         s = oracle.softmax(ref)
-        idx, gate, margin = oracle.topk(s, self.bias.astype(np.float64), self.w.top_k, self.shape.routed_scale)
+        idx, gate, margin = oracle.topk(s, self.cur_bias.astype(np.float64), self.w.top_k, self.shape.routed_scale)
         ok = margin >= TIE_MARGIN
         np.testing.assert_array_equal(self.dbg["idx"][rows][ok], idx[ok])
         np.testing.assert_allclose(self.dbg["gate"][rows][ok], gate[ok], rtol=1e-4, atol=1e-9)
