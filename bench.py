@@ -200,6 +200,7 @@ def main():
 
     import torch
     from mixture_experts_layer_shifted_b200 import configs
+    from mixture_experts_layer_shifted_b200.dp import controller_step
     from mixture_experts_layer_shifted_b200.zcmoe import LayerShape, ZcMoE
 
     dist, rank, ws, local = _dist()
@@ -228,10 +229,9 @@ def main():
     def step(i):
         layer.forward(xs[i % 2], y)
         if dist:
-            layer.read_counts(counts_buf)
-            dist.all_reduce(counts_buf)
-            layer.write_counts(counts_buf)
-        layer.update_bias(target_ffn_per_token=target, **GAINS)
+            controller_step(layer, counts_buf, target_ffn_per_token=target, **GAINS)
+        else:
+            layer.update_bias(target_ffn_per_token=target, **GAINS)
 
     for i in range(args.warmup):
         step(i)
