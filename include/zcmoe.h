@@ -168,6 +168,37 @@ ZCMOE_API int zcmoe_check(zcmoe_t h);
 ZCMOE_API int zcmoe_profile_begin(zcmoe_t h);
 ZCMOE_API int zcmoe_profile_end(zcmoe_t h, float *ms, int32_t *n_forwards);
 
+/* Routing stage without any device allocation (the pages have no counterpart:
+ * this is an interface for callers, not a step of the method).
+ *
+ * For callers that cannot call cudaMalloc: code running inside a framework's
+ * memory pool or under a fixed device-memory budget, where a raw allocation
+ * would bypass the pool or exceed the budget, and latency-critical loops where
+ * cudaMalloc/cudaFree could synchronise the device.  No handle is needed.
+ *
+ * Computes, from caller-owned device buffers, exactly what zcmoe_forward's
+ * routing stage computes: scores = softmax(logits) over E = n_ffn + n_zero
+ * experts, top-k on score + bias (ties to the lower id), gate = routed_scale *
+ * score, then counts [E], offsets [n_ffn+1], perm [T*k] (first offsets[n_ffn]
+ * entries valid) and pos [T, k], with the layouts of zcmoe_debug.
+ *   logits [T, E] fp32, bias [E] fp32 (inputs); idx, gate [T, k]; counts,
+ *   offsets, perm, pos (outputs).  All device pointers, all caller-owned.
+ *
+ * Its only scratch is one fixed 1 MiB device array inside the library
+ * (reserved on every GPU that loads it, until the process exits).  A call needs
+ * ceil(T/256) * E * 4 + (E+1) * 8 + (n_ffn+5) * 4 bytes of it; larger requests
+ * return ZCMOE_ERANGE with the limit in zcmoe_last_error() (E = 768 allows
+ * T <= 87,040; E = 96 allows about 695,000).  The first call on each device
+ * looks up the array's device address (with that device current); make that
+ * first call before any stream capture.  All calls share the array and it keeps
+ * the previous call's contents (whatever must start at zero is cleared on each
+ * call), so calls whose executions can overlap on the GPU (for example on two
+ * streams) race with each other: order them on one stream or synchronise
+ * between them.  Asynchronous on `stream`. */
+ZCMOE_API int zcmoe_route_noalloc(const float *logits, const float *bias, int64_t T, int32_t n_ffn, int32_t n_zero,
+                                  int32_t top_k, float routed_scale, int32_t *idx, float *gate, int32_t *counts,
+                                  int32_t *offsets, int32_t *perm, int32_t *pos, cudaStream_t stream);
+
 /* Frees the handle's own memory; never touches the borrowed weights.  NULL is a no-op. */
 ZCMOE_API int zcmoe_destroy(zcmoe_t h);
 

@@ -12,6 +12,9 @@ constexpr int kBM = 128;
 // Tokens per block of the integer stage (8 warps x 32 lanes, one token per thread).
 constexpr int kChunk = 256;
 
+// Copies msg into the calling thread's zcmoe_last_error() slot (zcmoe.cu).
+void set_last_error(const char* msg);
+
 // ------------------------------------------------------------- routing (route.cu)
 cudaError_t launch_softmax_topk(const float* logits, const float* bias, int T, int E, int k, float scale, int32_t* idx,
                                 float* gate, float* scores, int sms, cudaStream_t s);

@@ -102,6 +102,10 @@ int dalloc(T** p, size_t n) {
 
 }  // namespace
 
+namespace zc {
+void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+}  // namespace zc
+
 struct zcmoe_s {
   zcmoe_config cfg;
   int E, N, Z, k, d, inter, max_T, bf16, sms, device;
