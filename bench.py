@@ -108,6 +108,22 @@ def _dist():
     return None, 0, 1, 0
 
 
+def recorded_traffic(workload, kernel):
+    """DRAM bytes per launch from the committed ncu capture, or None when the
+    GEMM source changed since the capture (the counters no longer apply)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"gemm_dram_traffic_{workload}.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path))
+    h = hashlib.sha256()
+    for f in ("gemm_tc.cu", "zc_ptx.cuh"):
+        h.update(open(os.path.join(ROOT, "mixture_experts_layer_shifted_b200", "csrc", f), "rb").read())
+    if rec.get("kernel_source_sha256") != h.hexdigest() or kernel not in rec:
+        return None
+    return rec[kernel]["dram_read_bytes"] + rec[kernel]["dram_write_bytes"]
+
+
 def algorithmic_work(wl, P, distinct):
     """FLOPs and bytes per forward from the realised routing: P FFN pairs and
     `distinct` FFN experts hit.  F = 2 T d E + 6 d inter P;
@@ -286,7 +302,7 @@ def main():
     tensor_peak = peaks["bf16_tflops_sustained"]
     achieved = gu_flops / (gu_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "kernel": "grouped gate/up GEMM + SwiGLU (k_tc_gemm<1>)", "achieved": achieved,
-                "peak": tensor_peak, "unit": "TFLOP/s", "frac": achieved / tensor_peak, "traffic": None,
+                "peak": tensor_peak, "unit": "TFLOP/s", "frac": achieved / tensor_peak, "traffic": recorded_traffic(wl.name, "gate_up"),
                 "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
                 "per_launch": {"flops": gu_flops, "ms": gu_ms, "units": f"{P} FFN (token, expert) pairs x 4 d inter"}}
     fwd_ms = sum(stage_avg.values())
