@@ -268,16 +268,26 @@ __global__ void __launch_bounds__(kChunk) k_route_scatter(const int32_t* __restr
   }
 }
 
-// X_perm[p] = x[perm[p] / k] for p < P (P read from the device).
-__global__ void k_gather_rows(const uint4* __restrict__ x, int row_vecs, const int32_t* __restrict__ perm, int k,
-                              const int32_t* __restrict__ scal, uint4* __restrict__ xperm) {
-  const int64_t P = scal[0];
-  const int64_t n = P * row_vecs;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t p = i / row_vecs;
-    const int v = (int)(i - p * row_vecs);
-    const int t = perm[p] / k;
-    xperm[i] = x[(int64_t)t * row_vecs + v];
+// X_perm[p] = x[perm[p] / k] for p < P (P read from the device).  One warp per
+// row, 16-byte vectors, four loads in flight per lane.
+__global__ void __launch_bounds__(256) k_gather_rows(const uint4* __restrict__ x, int row_vecs,
+                                                     const int32_t* __restrict__ perm, int k,
+                                                     const int32_t* __restrict__ scal, uint4* __restrict__ xperm) {
+  const int P = scal[0];
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
+  for (int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); p < P; p += nwarps) {
+    const uint4* src = x + (int64_t)(perm[p] / k) * row_vecs;
+    uint4* dst = xperm + (int64_t)p * row_vecs;
+    int v = lane;
+    for (; v + 96 < row_vecs; v += 128) {
+      const uint4 a = src[v], b = src[v + 32], c = src[v + 64], d = src[v + 96];
+      dst[v] = a;
+      dst[v + 32] = b;
+      dst[v + 64] = c;
+      dst[v + 96] = d;
+    }
+    for (; v < row_vecs; v += 32) dst[v] = src[v];
   }
 }
 
@@ -320,14 +330,16 @@ struct Vec<float> {
   __device__ static void store(float* p, const float* f) { *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]); }
 };
 
-template <typename TIO>
+// One block per token (grid-stride); the token's gates and positions are read
+// once into registers, and the slot loop is unrolled so that all of a vector's
+// k + 1 loads are in flight together.
+template <typename TIO, int KMAX>
 __global__ void __launch_bounds__(128) k_combine(const TIO* __restrict__ x, const TIO* __restrict__ Y,
                                                  const float* __restrict__ gate, const int32_t* __restrict__ pos, int T,
                                                  int k, int d, TIO* __restrict__ y) {
   constexpr int V = Vec<TIO>::kN;
-  __shared__ float sg[32];
-  __shared__ int32_t sp[32];
-  __shared__ float szsum;
+  __shared__ float sg[KMAX];
+  __shared__ int32_t sp[KMAX];
   const int nv = d / V;
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
     if (threadIdx.x < k) {
@@ -335,30 +347,31 @@ __global__ void __launch_bounds__(128) k_combine(const TIO* __restrict__ x, cons
       sp[threadIdx.x] = pos[(int64_t)t * k + threadIdx.x];
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      float z = 0.0f;
-      for (int j = 0; j < k; ++j)
-        if (sp[j] < 0) z = __fadd_rn(z, sg[j]);
-      szsum = z;
+    float g[KMAX];
+    int32_t p[KMAX];
+    float zsum = 0.0f;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      g[j] = j < k ? sg[j] : 0.0f;
+      p[j] = j < k ? sp[j] : -2;  // -2: no slot
+      if (p[j] == -1) zsum = __fadd_rn(zsum, g[j]);
     }
     __syncthreads();
-    const float zsum = szsum;
     for (int v = threadIdx.x; v < nv; v += blockDim.x) {
       float acc[V], a[V];
       Vec<TIO>::load(x + (int64_t)t * d + v * V, a);
 #pragma unroll
       for (int i = 0; i < V; ++i) acc[i] = __fmul_rn(zsum, a[i]);
-      for (int j = 0; j < k; ++j) {
-        const int p = sp[j];
-        if (p < 0) continue;
-        Vec<TIO>::load(Y + (int64_t)p * d + v * V, a);
-        const float g = sg[j];
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] = __fmaf_rn(g, a[i], acc[i]);
+      for (int j = 0; j < KMAX; ++j) {
+        if (p[j] >= 0) {
+          Vec<TIO>::load(Y + (int64_t)p[j] * d + v * V, a);
+#pragma unroll
+          for (int i = 0; i < V; ++i) acc[i] = __fmaf_rn(g[j], a[i], acc[i]);
+        }
       }
       Vec<TIO>::store(y + (int64_t)t * d + v * V, acc);
     }
-    __syncthreads();
   }
 }
 
@@ -456,13 +469,22 @@ cudaError_t launch_combine(int bf16, const void* x, const void* Y, const int32_t
   (void)idx;
   (void)N;
   const int grid = grid_cap(T, sms * 16);
-  if (bf16)
-    k_combine<__nv_bfloat16><<<grid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
-                                                  static_cast<const __nv_bfloat16*>(Y), gate, pos, T, k, d,
-                                                  static_cast<__nv_bfloat16*>(y));
-  else
-    k_combine<float><<<grid, 128, 0, s>>>(static_cast<const float*>(x), static_cast<const float*>(Y), gate, pos, T, k,
-                                          d, static_cast<float*>(y));
+#define ZC_COMBINE(KM)                                                                                        \
+  if (bf16)                                                                                                   \
+    k_combine<__nv_bfloat16, KM><<<grid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(x),                   \
+                                                      static_cast<const __nv_bfloat16*>(Y), gate, pos, T, k, d, \
+                                                      static_cast<__nv_bfloat16*>(y));                        \
+  else                                                                                                        \
+    k_combine<float, KM><<<grid, 128, 0, s>>>(static_cast<const float*>(x), static_cast<const float*>(Y), gate, \
+                                              pos, T, k, d, static_cast<float*>(y));
+  if (k <= 8) {
+    ZC_COMBINE(8)
+  } else if (k <= 16) {
+    ZC_COMBINE(16)
+  } else {
+    ZC_COMBINE(32)
+  }
+#undef ZC_COMBINE
   return cudaGetLastError();
 }
 

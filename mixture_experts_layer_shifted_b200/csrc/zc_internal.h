@@ -1,6 +1,7 @@
 // Internal interfaces between the C-ABI layer (zcmoe.cu) and the kernels.
 #pragma once
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 

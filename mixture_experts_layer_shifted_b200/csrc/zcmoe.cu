@@ -170,7 +170,8 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
   ZC_CUDA(cudaGetDeviceProperties(&prop, dev));
   if (prop.major != 10) return fail(ZCMOE_EUNSUPPORTED, "device %d is sm_%d%d; this library targets sm_100a", dev,
                                     prop.major, prop.minor);
-  if (cfg->dtype == ZCMOE_BF16 && prop.sharedMemPerBlockOptin < (size_t)zc::tc_smem_bytes())
+  if (cfg->dtype == ZCMOE_BF16 &&
+      prop.sharedMemPerBlockOptin < (size_t)zc::tc_smem_bytes())
     return fail(ZCMOE_EUNSUPPORTED, "not enough shared memory per block");
 
   zcmoe_s* h = new (std::nothrow) zcmoe_s();
@@ -357,6 +358,7 @@ int zcmoe_forward(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream_t s, 
   ZC_CUDA(mark());
   // 5./6. expert GEMMs
   const int max_mb = (Ti * k + zc::kBM - 1) / zc::kBM + N;
+  // Swapped tiles (weights x tokens) unless fixed otherwise: they need no row padding.
   if (h->bf16) {
     zc::TcArgs a{};
     a.K = d;

@@ -142,11 +142,13 @@ def test_small_zero_only_tokens_return_weighted_input(small):
 
 
 # ---------------------------------------------------------------- ragged shapes and edge cases
+
 @pytest.mark.parametrize("T,d,N,inter,Z,k", [
     (1, 256, 8, 128, 4, 3),          # one token
     (1000, 320, 40, 192, 24, 6),     # d and inter not multiples of the column tiles; ragged T
     (300, 512, 33, 64, 0, 5),        # no zero experts
     (257, 192, 4, 256, 60, 32),      # k = 32, most picks zero experts
+    (2000, 256, 3, 128, 1, 2),       # > 256 tokens per expert: several token tiles
 ])
 def test_ragged_bf16(cuda_ok, T, d, N, inter, Z, k):
     w = configs.Workload("ragged", T=T, d=d, n_ffn=N, inter=inter, n_zero=Z, top_k=k, dtype="bf16", w_std=0.05,
