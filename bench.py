@@ -210,6 +210,8 @@ def main():
     ap.add_argument("--impl", default="zcmoe", choices=["zcmoe", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every step eagerly instead of replaying one captured CUDA graph (N=1)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -253,6 +255,20 @@ def main():
         step(i)
     torch.cuda.synchronize()
     layer.check()
+    use_graph = not dist and not args.eager
+    if use_graph:
+        # one step (forward on each of the two batches + bias update) captured once;
+        # replays launch the same kernels with no host work in between
+        graphs = []
+        for i in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(i)
+            graphs.append(g)
+        torch.cuda.synchronize()
+
+        def step(i):  # noqa: F811
+            graphs[i % 2].replay()
 
     # ---------------------------------------------------------------- timed region (device time)
     sampler = ClockSampler(local)
@@ -357,7 +373,8 @@ def main():
                        "realised": {"P": P, "ffn_per_token": P / wl.T, "distinct_experts": distinct,
                                     "zero_fraction": 1.0 - P / (wl.T * k)}},
             "roofline": roofline, "layer_roofline": layer_roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": 10 * args.steps, "clocks": clocks, "peaks": peaks}
+            "gpu_launches": 10 * args.steps, "clocks": clocks, "peaks": peaks,
+            "launch": "cuda graph per step" if use_graph else "eager"}
 
     # secondary workload (decode): reported beside the headline, not as the headline
     if rank == 0 and ws == 1 and not args.no_secondary and wl.name == "prefill_560b":

@@ -158,6 +158,13 @@ ZCMOE_API int zcmoe_set_bias(zcmoe_t h, const float *bias);
  * kernel's bounded wait gave up since the last check; clears the flag. */
 ZCMOE_API int zcmoe_check(zcmoe_t h);
 
+/* Failure-detection self-test: launches one kernel that waits, through the same
+ * bounded-wait routine the pipelined kernels use, on a barrier that nothing
+ * releases, so the wait gives up after limit_ns (1e3 .. 1e9) and records a
+ * timeout.  A later zcmoe_check then returns ZCMOE_ETIMEOUT (site 99) and the
+ * context stays usable.  Asynchronous on `stream`. */
+ZCMOE_API int zcmoe_selftest_wait(zcmoe_t h, int64_t limit_ns, cudaStream_t stream);
+
 /* Stage timing for measurement.  zcmoe_profile_begin starts recording CUDA
  * events between the stages of every later zcmoe_forward on this handle;
  * zcmoe_profile_end synchronises, writes per-stage device time summed over the

@@ -556,6 +556,14 @@ int zcmoe_profile_end(zcmoe_t h, float* ms, int32_t* n_forwards) {
   return ZCMOE_OK;
 }
 
+int zcmoe_selftest_wait(zcmoe_t h, int64_t limit_ns, cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (limit_ns < 1000 || limit_ns > 1000000000LL) return fail(ZCMOE_EINVAL, "limit_ns must lie in [1e3, 1e9]");
+  ZC_CUDA(zc::launch_selftest_wait(h->err, (uint64_t)limit_ns, s));
+  return ZCMOE_OK;
+}
+
 int zcmoe_destroy(zcmoe_t h) {
   g_err[0] = 0;
   if (!h) return ZCMOE_OK;

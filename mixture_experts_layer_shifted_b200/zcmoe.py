@@ -30,7 +30,7 @@ ZCMOE_BF16 = 1
 
 EXPORTED = ("zcmoe_create", "zcmoe_forward", "zcmoe_forward_host", "zcmoe_update_bias", "zcmoe_read_counts",
             "zcmoe_write_counts", "zcmoe_get_state", "zcmoe_set_bias", "zcmoe_check", "zcmoe_profile_begin",
-            "zcmoe_profile_end", "zcmoe_route_noalloc", "zcmoe_destroy", "zcmoe_last_error")
+            "zcmoe_profile_end", "zcmoe_selftest_wait", "zcmoe_route_noalloc", "zcmoe_destroy", "zcmoe_last_error")
 STAGES = ("router", "softmax_topk", "integer", "gather", "gate_up", "down", "combine")
 
 
@@ -86,6 +86,7 @@ def lib():
         L.zcmoe_destroy.argtypes = [vp]
         L.zcmoe_profile_begin.argtypes = [vp]
         L.zcmoe_profile_end.argtypes = [vp, vp, vp]
+        L.zcmoe_selftest_wait.argtypes = [vp, i64, vp]
         L.zcmoe_route_noalloc.argtypes = [vp, vp, i64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
                                           vp, vp, vp, vp, vp, vp, vp]
         for f in EXPORTED[:-1]:
@@ -161,6 +162,10 @@ def zcmoe_profile_end(h):
     n = ctypes.c_int32()
     _check(lib().zcmoe_profile_end(h, ms, ctypes.byref(n)), "zcmoe_profile_end")
     return dict(zip(STAGES, [float(v) for v in ms])), int(n.value)
+
+
+def zcmoe_selftest_wait(h, limit_ns, stream=None):
+    _check(lib().zcmoe_selftest_wait(h, int(limit_ns), _stream(stream)), "zcmoe_selftest_wait")
 
 
 def zcmoe_route_noalloc(logits, bias, T, n_ffn, n_zero, top_k, routed_scale, idx, gate, counts, offsets, perm, pos,
