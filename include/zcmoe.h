@@ -121,12 +121,14 @@ ZCMOE_API int zcmoe_create(const zcmoe_config *cfg, const zcmoe_weights *w, zcmo
  * controller accumulators.  T == 0 is a no-op.  Asynchronous on `stream`. */
 ZCMOE_API int zcmoe_forward(zcmoe_t h, const void *x, int64_t T, void *y, cudaStream_t stream, const zcmoe_debug *dbg);
 
-/* The same forward pass from and to HOST memory: copies x [T, d] (host) into a
- * handle-owned device staging buffer, runs zcmoe_forward, and copies y [T, d]
- * back to host memory, all enqueued on `stream`.  The staging buffers (2 x
- * max_tokens x d elements) are allocated on the first call.  Use page-locked
- * host buffers so the copies are asynchronous; keep both alive and read y only
- * after the stream has been synchronised. */
+/* The same forward pass from and to HOST memory.  x [T, d] (host) is copied into
+ * one of two handle-owned device staging buffers on an internal copy stream (so
+ * the upload for the next call overlaps this call's compute), `stream` waits for
+ * it, runs zcmoe_forward, and copies y [T, d] back to host memory on `stream`.
+ * The staging buffers (3 x max_tokens x d elements) and the copy stream are
+ * created on the first call.  Use page-locked host buffers so the copies are
+ * asynchronous; x_host may be reused once `stream` has passed this call's
+ * forward, and y_host is complete once `stream` has been synchronised. */
 ZCMOE_API int zcmoe_forward_host(zcmoe_t h, const void *x_host, int64_t T, void *y_host, cudaStream_t stream);
 
 /* One bias-controller step (zhangjingwei.cn 二.1 "PID controller"; web3.cnouyi.fund

@@ -119,7 +119,12 @@ struct zcmoe_s {
   float *logits, *gate;
   int32_t *idx, *pos, *counts, *offsets, *mb_off, *scal, *chunk, *perm;
   void *xperm, *H, *Y;
-  void *stage_x, *stage_y;  // device staging for zcmoe_forward_host (allocated on first use)
+  // zcmoe_forward_host: x staged through two device buffers filled on an internal
+  // copy stream, so the next call's upload overlaps this call's compute; y staged once
+  void *stage_x, *stage_x2, *stage_y;
+  cudaStream_t copy_stream;
+  cudaEvent_t ev_in[2], ev_used[2];
+  long long host_calls;
   // stage timing (zcmoe_profile_begin/end): ZCMOE_NUM_STAGES + 1 events per forward
   bool profiling;
   std::vector<cudaEvent_t>* events;
@@ -132,9 +137,14 @@ static void release(zcmoe_s* h) {
   void* ptrs[] = {h->bias,  h->b0,     h->offset, h->eta,   h->integ,   h->eprev,  h->acc_counts,
                   h->err,   h->logits, h->gate,   h->idx,   h->pos,     h->counts, h->offsets,
                   h->mb_off, h->scal,  h->chunk,  h->perm,  h->xperm,   h->H,      h->Y,
-                  h->stage_x, h->stage_y};
+                  h->stage_x, h->stage_x2, h->stage_y};
   for (void* p : ptrs)
     if (p) cudaFree(p);
+  for (int i = 0; i < 2; ++i) {
+    if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+    if (h->ev_used[i]) cudaEventDestroy(h->ev_used[i]);
+  }
+  if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
   if (h->events) {
     for (cudaEvent_t e : *h->events) cudaEventDestroy(e);
     delete h->events;
@@ -443,21 +453,47 @@ int zcmoe_forward_host(zcmoe_t h, const void* x_host, int64_t T, void* y_host, c
   if (!x_host || !y_host) return fail(ZCMOE_EINVAL, "x or y is NULL");
   const size_t bytes_max = (size_t)h->max_T * h->d * (h->bf16 ? 2 : 4);
   if (!h->stage_x) {
-    uint8_t *a = nullptr, *b = nullptr;
+    uint8_t *a = nullptr, *a2 = nullptr, *b = nullptr;
     int rc = dalloc(&a, bytes_max);
+    if (rc == ZCMOE_OK) rc = dalloc(&a2, bytes_max);
     if (rc == ZCMOE_OK) rc = dalloc(&b, bytes_max);
-    if (rc != ZCMOE_OK) {
+    cudaError_t e = cudaSuccess;
+    if (rc == ZCMOE_OK) e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking);
+    for (int i = 0; i < 2 && rc == ZCMOE_OK && e == cudaSuccess; ++i) {
+      e = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_used[i], cudaEventDisableTiming);
+    }
+    if (rc != ZCMOE_OK || e != cudaSuccess) {
       if (a) cudaFree(a);
-      return rc;
+      if (a2) cudaFree(a2);
+      if (b) cudaFree(b);
+      for (int i = 0; i < 2; ++i) {
+        if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+        if (h->ev_used[i]) cudaEventDestroy(h->ev_used[i]);
+        h->ev_in[i] = h->ev_used[i] = nullptr;
+      }
+      if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
+      h->copy_stream = nullptr;
+      if (rc != ZCMOE_OK) return rc;
+      return fail(ZCMOE_ECUDA, "creating the copy stream: %s", cudaGetErrorString(e));
     }
     h->stage_x = a;
+    h->stage_x2 = a2;
     h->stage_y = b;
   }
   const size_t bytes = (size_t)T * h->d * (h->bf16 ? 2 : 4);
-  ZC_CUDA(cudaMemcpyAsync(h->stage_x, x_host, bytes, cudaMemcpyHostToDevice, s));
-  int rc = zcmoe_forward(h, h->stage_x, T, h->stage_y, s, nullptr);
+  const int buf = (int)(h->host_calls & 1);
+  void* sx = buf ? h->stage_x2 : h->stage_x;
+  // the buffer was last read by the forward two calls ago
+  if (h->host_calls >= 2) ZC_CUDA(cudaStreamWaitEvent(h->copy_stream, h->ev_used[buf], 0));
+  ZC_CUDA(cudaMemcpyAsync(sx, x_host, bytes, cudaMemcpyHostToDevice, h->copy_stream));
+  ZC_CUDA(cudaEventRecord(h->ev_in[buf], h->copy_stream));
+  ZC_CUDA(cudaStreamWaitEvent(s, h->ev_in[buf], 0));
+  int rc = zcmoe_forward(h, sx, T, h->stage_y, s, nullptr);
   if (rc != ZCMOE_OK) return rc;
+  ZC_CUDA(cudaEventRecord(h->ev_used[buf], s));
   ZC_CUDA(cudaMemcpyAsync(y_host, h->stage_y, bytes, cudaMemcpyDeviceToHost, s));
+  ++h->host_calls;
   return ZCMOE_OK;
 }
 

@@ -235,3 +235,21 @@ def test_forward_host_matches_device(small):
     small.layer.forward_host(xh, yh)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(yh.view(torch.int16).numpy().view(np.uint16), small.y)
+
+
+def test_forward_host_back_to_back_calls(small):
+    """Several host-buffer calls in flight (uploads double-buffered on the copy
+    stream) each return their own input's output."""
+    xs = [configs.device_tokens(small.w, step=s) for s in (5, 6, 7)]
+    want = []
+    for x in xs:
+        y = small.layer.forward(x)
+        torch.cuda.synchronize()
+        want.append(y.view(torch.int16).cpu().numpy())
+    xh = [x.cpu().pin_memory() for x in xs]
+    yh = [torch.empty_like(x).pin_memory() for x in xh]
+    for a, b in zip(xh, yh):
+        small.layer.forward_host(a, b)
+    torch.cuda.synchronize()
+    for b, w in zip(yh, want):
+        np.testing.assert_array_equal(b.view(torch.int16).numpy(), w)
