@@ -211,6 +211,72 @@ ZCMOE_API int zcmoe_route_noalloc(const float *logits, const float *bias, int64_
 /* Frees the handle's own memory; never touches the borrowed weights.  NULL is a no-op. */
 ZCMOE_API int zcmoe_destroy(zcmoe_t h);
 
+/* ------------------------------------------------------------------------
+ * Dense FFN path and the shortcut-connected overlap (ScMoE).
+ *
+ * LongCat-Flash technical summary (zhangjingwei.cn), 二 架構 part 2 "快捷連接 MoE":
+ * the first MLA block's output goes straight to the MoE block, so the dense FFN
+ * of the preceding block does not wait for the MoE layer and the two can run at
+ * the same time; 五 訓練基礎設施 "ScMoE結構和分塊" and 六 推理與部署 (single-batch
+ * overlap) use that window to hide the MoE's dispatch/combine traffic.  模型配置:
+ * the dense path is 12288 wide on the 6144 hidden size.
+ *
+ * The dense FFN is y = W_down (silu(W_gate x) * (W_up x)), the form of an FFN
+ * expert (the pages do not name the dense path's activation): bf16 operands,
+ * fp32 accumulation on the tensor cores, the SwiGLU product rounded once to
+ * bf16 before the down projection, y rounded once to bf16. */
+typedef struct zcmoe_dense_s *zcmoe_dense_t;
+
+/* d and inter positive multiples of 64; 1 <= max_tokens <= 2^20.  bf16 only. */
+typedef struct {
+  int32_t d;
+  int32_t inter;
+  int32_t max_tokens;
+} zcmoe_dense_config;
+
+/* Device pointers, bf16, 16-byte aligned, borrowed (not copied) until
+ * zcmoe_dense_destroy: w_gate [inter, d], w_up [inter, d], w_down [d, inter]. */
+typedef struct {
+  const void *w_gate;
+  const void *w_up;
+  const void *w_down;
+} zcmoe_dense_weights;
+
+/* Checks the shapes, allocates the intermediate [max_tokens, inter] bf16 and
+ * the internal stream and events that zcmoe_forward_overlap uses, and builds
+ * the weights' TMA descriptors.  Requires sm_100.  On error *out is left NULL. */
+ZCMOE_API int zcmoe_dense_create(const zcmoe_dense_config *cfg, const zcmoe_dense_weights *w, zcmoe_dense_t *out);
+
+/* x [T, d] device bf16 -> y [T, d] device bf16; y must not overlap x.  T == 0 is
+ * a no-op.  Asynchronous on `stream`; one stream at a time per handle. */
+ZCMOE_API int zcmoe_dense_forward(zcmoe_dense_t h, const void *x, int64_t T, void *y, cudaStream_t stream);
+
+/* The MoE layer and the dense FFN over the same T tokens, run concurrently:
+ *   y_moe = zcmoe_forward(moe, x_moe, T),  y_dense = zcmoe_dense_forward(dense, x_dense, T),
+ * with results identical, bit for bit, to the two calls made one after the
+ * other (the MoE's controller accumulators advance exactly as in zcmoe_forward).
+ * The dense FFN runs on the dense handle's internal stream, forked from and
+ * joined back into `stream`: its gate/up GEMM starts when the MoE router GEMM
+ * has finished and runs beside the MoE's memory-bound stages (softmax/top-k,
+ * integer stage, row gather); its down GEMM starts when the MoE down GEMM has
+ * finished and runs beside the combine.  When the call returns, all the work of
+ * both is ordered before anything later enqueued on `stream`, so the call can
+ * be captured into a CUDA graph on `stream`.
+ * Requires: both handles live, the MoE handle bf16, equal d, 0 <= T <= both
+ * max_tokens, 16-byte aligned buffers; y_moe and y_dense overlap neither each
+ * other nor x_moe / x_dense (x_moe == x_dense is allowed). */
+ZCMOE_API int zcmoe_forward_overlap(zcmoe_t moe, zcmoe_dense_t dense, const void *x_moe, const void *x_dense,
+                                    int64_t T, void *y_moe, void *y_dense, cudaStream_t stream);
+
+/* ZCMOE_OK, or ZCMOE_ETIMEOUT if one of the dense handle's kernels gave up a
+ * bounded wait since the last check (the flag is then cleared).  Synchronises
+ * the device. */
+ZCMOE_API int zcmoe_dense_check(zcmoe_dense_t h);
+
+/* Frees the dense handle's own memory and stream; never touches the borrowed
+ * weights.  NULL is a no-op. */
+ZCMOE_API int zcmoe_dense_destroy(zcmoe_dense_t h);
+
 /* Message for the last failing call on this thread ("" if none). */
 ZCMOE_API const char *zcmoe_last_error(void);
 

@@ -32,6 +32,7 @@ class Workload:
     seed: int = 0
     steps: int = 1            # forward (+ bias update) steps of the workload
     target_ffn: float | None = None
+    dense_inter: int = 0      # width of the dense FFN path run beside the layer (ScMoE); 0: none
     notes: str = ""
 
     @property
@@ -52,11 +53,11 @@ WORKLOADS = {
     "tiny_f32": Workload("tiny_f32", T=64, d=256, n_ffn=16, inter=128, n_zero=8, top_k=4, dtype="f32",
                          w_std=0.02, bias=("uniform", -0.1, 0.1)),
     "small_bf16": Workload("small_bf16", T=4096, d=1024, n_ffn=64, inter=512, n_zero=32, top_k=8, dtype="bf16",
-                           w_std=0.02, bias=("uniform", -0.2, 0.2)),
+                           w_std=0.02, bias=("uniform", -0.2, 0.2), dense_inter=3072),
     "prefill_560b": Workload("prefill_560b", T=16384, d=6144, n_ffn=512, inter=2048, n_zero=256, top_k=12,
-                             dtype="bf16", w_std=0.006, bias=("zero",)),
+                             dtype="bf16", w_std=0.006, bias=("zero",), dense_inter=12288),
     "decode_560b": Workload("decode_560b", T=128, d=6144, n_ffn=512, inter=2048, n_zero=256, top_k=12, dtype="bf16",
-                            w_std=0.006, bias=("zero",),
+                            w_std=0.006, bias=("zero",), dense_inter=12288,
                             notes="bias 0: uniform routing already sends 256/768 = 1/3 of picks to zero experts"),
     "decode_560b_zero_bias": Workload("decode_560b_zero_bias", T=128, d=6144, n_ffn=512, inter=2048, n_zero=256,
                                       top_k=12, dtype="bf16", w_std=0.006, bias=("zero_experts", 0.5),
@@ -66,7 +67,7 @@ WORKLOADS = {
     # small case of the prefill kernels for profiler captures: a few GB on the device,
     # inputs still larger than L2
     "prefill_probe": Workload("prefill_probe", T=2048, d=6144, n_ffn=32, inter=2048, n_zero=16, top_k=12,
-                              dtype="bf16", w_std=0.006, bias=("zero",)),
+                              dtype="bf16", w_std=0.006, bias=("zero",), dense_inter=12288),
 }
 
 
@@ -96,6 +97,21 @@ def device_weights(w: Workload, device="cuda"):
     out = []
     for shp, tid in zip(shapes, tids):
         t = torch.empty(shp, dtype=dt, device=device)
+        synth.fill_normal_(t, tid, w.seed, w.w_std)
+        out.append(t)
+    return tuple(out)
+
+
+def device_dense_weights(w: Workload, device="cuda"):
+    """(w_gate [I, d], w_up [I, d], w_down [d, I]) of the dense FFN path, I = w.dense_inter, bf16."""
+    import torch
+    if w.dense_inter <= 0:
+        raise ValueError(f"workload {w.name} has no dense FFN path")
+    shapes = [(w.dense_inter, w.d), (w.dense_inter, w.d), (w.d, w.dense_inter)]
+    tids = [synth.TID_DENSE_G, synth.TID_DENSE_U, synth.TID_DENSE_D]
+    out = []
+    for shp, tid in zip(shapes, tids):
+        t = torch.empty(shp, dtype=torch.bfloat16, device=device)
         synth.fill_normal_(t, tid, w.seed, w.w_std)
         out.append(t)
     return tuple(out)

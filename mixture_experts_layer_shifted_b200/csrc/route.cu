@@ -427,6 +427,17 @@ __global__ void k_selftest_wait(int* err, uint64_t limit_ns) {
 
 int grid_cap(int want, int cap) { return want < 1 ? 1 : (want < cap ? want : cap); }
 
+// One group holding all T rows (the dense FFN through the grouped GEMM):
+// row_off = {0, T}, mb_off = {0, ceil(T / 128)}.
+__global__ void k_single_group(int32_t* row_off, int32_t* mb_off, int T) {
+  if (threadIdx.x == 0) {
+    row_off[0] = 0;
+    row_off[1] = T;
+    mb_off[0] = 0;
+    mb_off[1] = (T + kBM - 1) / kBM;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_softmax_topk(const float* logits, const float* bias, int T, int E, int k, float scale, int32_t* idx,
@@ -492,6 +503,11 @@ cudaError_t launch_combine(int bf16, const void* x, const void* Y, const int32_t
 
 cudaError_t launch_selftest_wait(int* err, uint64_t limit_ns, cudaStream_t s) {
   k_selftest_wait<<<1, 32, 0, s>>>(err, limit_ns);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_single_group(int32_t* row_off, int32_t* mb_off, int T, cudaStream_t s) {
+  k_single_group<<<1, 32, 0, s>>>(row_off, mb_off, T);
   return cudaGetLastError();
 }
 

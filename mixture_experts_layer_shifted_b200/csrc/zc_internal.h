@@ -29,6 +29,7 @@ cudaError_t launch_gather_rows(const void* x, int row_bytes, const int32_t* perm
 cudaError_t launch_combine(int bf16, const void* x, const void* Y, const int32_t* idx, const float* gate,
                            const int32_t* pos, int T, int k, int N, int d, void* y, int sms, cudaStream_t s);
 cudaError_t launch_selftest_wait(int* err, uint64_t limit_ns, cudaStream_t s);
+cudaError_t launch_single_group(int32_t* row_off, int32_t* mb_off, int T, cudaStream_t s);
 cudaError_t launch_update_bias(int64_t* counts, int64_t* tokens, int N, int Z, int k, float kp, float ki, float kd,
                                float decay, float target, const float* b0, float* eta, float* integ, float* eprev,
                                float* bias, cudaStream_t s);

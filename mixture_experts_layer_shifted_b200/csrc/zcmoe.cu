@@ -33,11 +33,21 @@ thread_local char g_err[512] = "";
 // Live handles, so that a destroyed or foreign handle is rejected instead of
 // being dereferenced.
 std::mutex g_live_mu;
-std::unordered_set<const void*> g_live;
+std::unordered_set<const void*> g_live;        // zcmoe_t
+std::unordered_set<const void*> g_live_dense;  // zcmoe_dense_t
 
 bool is_live(const void* h) {
   std::lock_guard<std::mutex> lk(g_live_mu);
   return h && g_live.count(h) != 0;
+}
+bool is_live_dense(const void* h) {
+  std::lock_guard<std::mutex> lk(g_live_mu);
+  return h && g_live_dense.count(h) != 0;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
 }
 
 int fail(int code, const char* fmt, ...) {
@@ -151,6 +161,77 @@ static void release(zcmoe_s* h) {
     h->events = nullptr;
   }
 }
+
+// ---------------------------------------------------------------- dense FFN path
+// y = W_down (silu(W_gate x) * (W_up x)) through the same grouped tensor-core
+// GEMM as the experts, with one group holding all T rows.
+struct zcmoe_dense_s {
+  int d, inter, max_T, sms;
+  zcmoe_dense_weights w;
+  void* H;           // [max_T, inter] bf16
+  int32_t* offs;     // one group: row_off[2], then mb_off[2] (written per call)
+  int* err;          // bounded-wait error word of the dense kernels
+  cudaStream_t side; // zcmoe_forward_overlap enqueues the dense FFN here
+  cudaEvent_t ev_router, ev_down, ev_join;
+  CUtensorMap tm_wg, tm_wu, tm_wd, tm_h;
+};
+
+static void release_dense(zcmoe_dense_s* h) {
+  void* ptrs[] = {h->H, h->offs, h->err};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  cudaEvent_t evs[] = {h->ev_router, h->ev_down, h->ev_join};
+  for (cudaEvent_t e : evs)
+    if (e) cudaEventDestroy(e);
+  if (h->side) cudaStreamDestroy(h->side);
+}
+
+// gate/up GEMM with the SwiGLU epilogue: H[:T] = silu(x W_g^T) * (x W_u^T), bf16
+static int dense_gate_up(zcmoe_dense_s* h, const void* x, int T, cudaStream_t s) {
+  CUtensorMap tm_x;
+  int rc = make_tmap(&tm_x, x, (uint64_t)h->d, (uint64_t)T, 128);
+  if (rc != ZCMOE_OK) return rc;
+  ZC_CUDA(zc::launch_single_group(h->offs, h->offs + 2, T, s));
+  zc::TcArgs a{};
+  a.K = h->d;
+  a.n_out = h->inter;
+  a.nblocks = (h->inter + zc::tc_block_n(zc::kGateUp) - 1) / zc::tc_block_n(zc::kGateUp);
+  a.ngroups = 1;
+  a.row_off = h->offs;
+  a.mb_off = h->offs + 2;
+  a.b_rows_per_group = h->inter;
+  a.out = h->H;
+  a.ldo = h->inter;
+  a.err = h->err;
+  const int tiles = ((T + zc::kBM - 1) / zc::kBM) * a.nblocks;
+  ZC_CUDA(zc::launch_tc_gemm(zc::kGateUp, tm_x, h->tm_wg, h->tm_wu, a, tiles < h->sms ? tiles : h->sms, s));
+  return ZCMOE_OK;
+}
+
+// down GEMM: y = H[:T] W_d^T, bf16
+static int dense_down(zcmoe_dense_s* h, int T, void* y, cudaStream_t s) {
+  zc::TcArgs b{};
+  b.K = h->inter;
+  b.n_out = h->d;
+  b.nblocks = (h->d + zc::tc_block_n(zc::kDown) - 1) / zc::tc_block_n(zc::kDown);
+  b.ngroups = 1;
+  b.row_off = h->offs;
+  b.mb_off = h->offs + 2;
+  b.b_rows_per_group = h->d;
+  b.out = y;
+  b.ldo = h->d;
+  b.err = h->err;
+  const int tiles = ((T + zc::kBM - 1) / zc::kBM) * b.nblocks;
+  ZC_CUDA(zc::launch_tc_gemm(zc::kDown, h->tm_h, h->tm_wd, h->tm_wd, b, tiles < h->sms ? tiles : h->sms, s));
+  return ZCMOE_OK;
+}
+
+// The dense FFN enqueued beside a MoE forward (zcmoe_forward_overlap).
+struct DenseSide {
+  zcmoe_dense_s* dn;
+  const void* x;
+  void* y;
+};
 
 extern "C" {
 
@@ -297,9 +378,11 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
   return ZCMOE_OK;
 }
 
-int zcmoe_forward(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream_t s, const zcmoe_debug* dbg) {
-  g_err[0] = 0;
-  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+// The forward pass; with `side`, the dense FFN's two GEMMs are forked onto its
+// stream after the router GEMM and after the down GEMM, and joined back into
+// `s` after the combine.
+static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream_t s, const zcmoe_debug* dbg,
+                        const DenseSide* side) {
   if (T < 0 || T > h->max_T) return fail(ZCMOE_ERANGE, "T=%lld outside [0, %d]", (long long)T, h->max_T);
   if (T == 0) return ZCMOE_OK;
   if (!x || !y) return fail(ZCMOE_EINVAL, "x or y is NULL");
@@ -353,6 +436,12 @@ int zcmoe_forward(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream_t s, 
     ZC_CUDA(zc::launch_simt_gemm(zc::kRouter, a, (Ti + zc::kBM - 1) / zc::kBM, s));
   }
   ZC_CUDA(mark());
+  if (side) {
+    ZC_CUDA(cudaEventRecord(side->dn->ev_router, s));
+    ZC_CUDA(cudaStreamWaitEvent(side->dn->side, side->dn->ev_router, 0));
+    const int rc = dense_gate_up(side->dn, side->x, Ti, side->dn->side);
+    if (rc != ZCMOE_OK) return rc;
+  }
   // 2. softmax + bias-shifted top-k
   ZC_CUDA(zc::launch_softmax_topk(h->logits, h->bias, Ti, E, k, h->cfg.routed_scale, h->idx, h->gate,
                                   dbg ? dbg->scores : nullptr, h->sms, s));
@@ -426,9 +515,17 @@ int zcmoe_forward(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream_t s, 
     ZC_CUDA(zc::launch_simt_gemm(zc::kDown, b, max_mb, s));
   }
   ZC_CUDA(mark());
+  if (side) {
+    ZC_CUDA(cudaEventRecord(side->dn->ev_down, s));
+    ZC_CUDA(cudaStreamWaitEvent(side->dn->side, side->dn->ev_down, 0));
+    const int rc = dense_down(side->dn, Ti, side->y, side->dn->side);
+    if (rc != ZCMOE_OK) return rc;
+    ZC_CUDA(cudaEventRecord(side->dn->ev_join, side->dn->side));
+  }
   // 7. combine
   ZC_CUDA(zc::launch_combine(h->bf16, x, h->Y, h->idx, h->gate, h->pos, Ti, k, N, d, y, h->sms, s));
   ZC_CUDA(mark());
+  if (side) ZC_CUDA(cudaStreamWaitEvent(s, side->dn->ev_join, 0));
 
   if (dbg) {
     if (dbg->logits) ZC_CUDA(cudaMemcpyAsync(dbg->logits, h->logits, (size_t)T * E * 4, cudaMemcpyDeviceToDevice, s));
@@ -443,6 +540,12 @@ int zcmoe_forward(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream_t s, 
       ZC_CUDA(cudaMemcpyAsync(dbg->expert_out, h->Y, (size_t)T * k * d * esz, cudaMemcpyDeviceToDevice, s));
   }
   return ZCMOE_OK;
+}
+
+int zcmoe_forward(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream_t s, const zcmoe_debug* dbg) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  return forward_impl(h, x, T, y, s, dbg, nullptr);
 }
 
 int zcmoe_forward_host(zcmoe_t h, const void* x_host, int64_t T, void* y_host, cudaStream_t s) {
@@ -610,6 +713,142 @@ int zcmoe_destroy(zcmoe_t h) {
   h->alive = false;
   cudaDeviceSynchronize();
   release(h);
+  delete h;
+  return ZCMOE_OK;
+}
+
+// ---------------------------------------------------------------- dense FFN path and the overlap
+
+int zcmoe_dense_create(const zcmoe_dense_config* cfg, const zcmoe_dense_weights* w, zcmoe_dense_t* out) {
+  g_err[0] = 0;
+  if (!out) return fail(ZCMOE_EINVAL, "out is NULL");
+  *out = nullptr;
+  if (!cfg || !w) return fail(ZCMOE_EINVAL, "cfg or weights is NULL");
+  if (cfg->d < 64 || cfg->d % 64 || cfg->inter < 64 || cfg->inter % 64)
+    return fail(ZCMOE_EINVAL, "d and inter must be positive multiples of 64");
+  if (cfg->max_tokens < 1 || cfg->max_tokens > (1 << 20)) return fail(ZCMOE_EINVAL, "need 1 <= max_tokens <= 2^20");
+  if (!w->w_gate || !w->w_up || !w->w_down) return fail(ZCMOE_EINVAL, "a weight pointer is NULL");
+  const void* wp[3] = {w->w_gate, w->w_up, w->w_down};
+  for (const void* p : wp)
+    if (reinterpret_cast<uintptr_t>(p) & 15u) return fail(ZCMOE_EINVAL, "weight pointers must be 16-byte aligned");
+
+  int dev = 0;
+  ZC_CUDA(cudaGetDevice(&dev));
+  cudaDeviceProp prop;
+  ZC_CUDA(cudaGetDeviceProperties(&prop, dev));
+  if (prop.major != 10) return fail(ZCMOE_EUNSUPPORTED, "device %d is sm_%d%d; this library targets sm_100a", dev,
+                                    prop.major, prop.minor);
+  if (prop.sharedMemPerBlockOptin < (size_t)zc::tc_smem_bytes())
+    return fail(ZCMOE_EUNSUPPORTED, "not enough shared memory per block");
+
+  zcmoe_dense_s* h = new (std::nothrow) zcmoe_dense_s();
+  if (!h) return fail(ZCMOE_ENOMEM, "host allocation failed");
+  memset(h, 0, sizeof(*h));
+  h->d = cfg->d;
+  h->inter = cfg->inter;
+  h->max_T = cfg->max_tokens;
+  h->sms = prop.multiProcessorCount;
+  h->w = *w;
+  const size_t hbytes = (size_t)h->max_T * h->inter * 2;
+  uint8_t* hh = nullptr;
+  int rc = dalloc(&hh, hbytes);
+  h->H = hh;
+  if (rc == ZCMOE_OK) rc = dalloc(&h->offs, 4);
+  if (rc == ZCMOE_OK) rc = dalloc(&h->err, 1);
+  if (rc == ZCMOE_OK) {
+    cudaError_t e = cudaMemset(h->H, 0, hbytes);
+    if (e == cudaSuccess) e = cudaMemset(h->offs, 0, 4 * sizeof(int32_t));
+    if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int));
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_router, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_down, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) rc = fail(ZCMOE_ECUDA, "initialising the dense handle: %s", cudaGetErrorString(e));
+  }
+  if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wg, w->w_gate, (uint64_t)h->d, (uint64_t)h->inter, 128);
+  if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wu, w->w_up, (uint64_t)h->d, (uint64_t)h->inter, 128);
+  if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wd, w->w_down, (uint64_t)h->inter, (uint64_t)h->d, 256);
+  if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_h, h->H, (uint64_t)h->inter, (uint64_t)h->max_T, 128);
+  if (rc != ZCMOE_OK) {
+    release_dense(h);
+    delete h;
+    return rc;
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_live_mu);
+    g_live_dense.insert(h);
+  }
+  *out = h;
+  return ZCMOE_OK;
+}
+
+int zcmoe_dense_forward(zcmoe_dense_t h, const void* x, int64_t T, void* y, cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live_dense(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed dense handle");
+  if (T < 0 || T > h->max_T) return fail(ZCMOE_ERANGE, "T=%lld outside [0, %d]", (long long)T, h->max_T);
+  if (T == 0) return ZCMOE_OK;
+  if (!x || !y) return fail(ZCMOE_EINVAL, "x or y is NULL");
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(y) & 15u))
+    return fail(ZCMOE_EINVAL, "x and y must be 16-byte aligned");
+  const size_t nb = (size_t)T * h->d * 2;
+  if (overlaps(x, nb, y, nb)) return fail(ZCMOE_EINVAL, "y overlaps x");
+  const int rc = dense_gate_up(h, x, (int)T, s);
+  if (rc != ZCMOE_OK) return rc;
+  return dense_down(h, (int)T, y, s);
+}
+
+int zcmoe_forward_overlap(zcmoe_t moe, zcmoe_dense_t dense, const void* x_moe, const void* x_dense, int64_t T,
+                          void* y_moe, void* y_dense, cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live(moe)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (!is_live_dense(dense)) return fail(ZCMOE_EINVAL, "invalid or destroyed dense handle");
+  if (!moe->bf16) return fail(ZCMOE_EUNSUPPORTED, "the overlap needs a bf16 MoE handle");
+  if (moe->d != dense->d) return fail(ZCMOE_EINVAL, "hidden sizes differ (%d vs %d)", moe->d, dense->d);
+  if (T < 0 || T > moe->max_T || T > dense->max_T)
+    return fail(ZCMOE_ERANGE, "T=%lld outside [0, %d]", (long long)T,
+                moe->max_T < dense->max_T ? moe->max_T : dense->max_T);
+  if (T == 0) return ZCMOE_OK;
+  if (!x_moe || !x_dense || !y_moe || !y_dense) return fail(ZCMOE_EINVAL, "a buffer is NULL");
+  const void* bufs[4] = {x_moe, x_dense, y_moe, y_dense};
+  for (const void* p : bufs)
+    if (reinterpret_cast<uintptr_t>(p) & 15u) return fail(ZCMOE_EINVAL, "buffers must be 16-byte aligned");
+  const size_t nb = (size_t)T * moe->d * 2;
+  if (overlaps(y_moe, nb, y_dense, nb) || overlaps(y_moe, nb, x_moe, nb) || overlaps(y_moe, nb, x_dense, nb) ||
+      overlaps(y_dense, nb, x_moe, nb) || overlaps(y_dense, nb, x_dense, nb))
+    return fail(ZCMOE_EINVAL, "an output overlaps another buffer");
+  const DenseSide side{dense, x_dense, y_dense};
+  const int rc = forward_impl(moe, x_moe, T, y_moe, s, nullptr, &side);
+  if (rc != ZCMOE_OK) {
+    // best effort: leave no work of the side stream unjoined
+    if (cudaEventRecord(dense->ev_join, dense->side) == cudaSuccess) cudaStreamWaitEvent(s, dense->ev_join, 0);
+    cudaGetLastError();
+  }
+  return rc;
+}
+
+int zcmoe_dense_check(zcmoe_dense_t h) {
+  g_err[0] = 0;
+  if (!is_live_dense(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed dense handle");
+  ZC_CUDA(cudaDeviceSynchronize());
+  int code = 0;
+  ZC_CUDA(cudaMemcpy(&code, h->err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (code) {
+    ZC_CUDA(cudaMemset(h->err, 0, sizeof(int)));
+    return fail(ZCMOE_ETIMEOUT, "a device-side wait timed out (site %d)", code);
+  }
+  return ZCMOE_OK;
+}
+
+int zcmoe_dense_destroy(zcmoe_dense_t h) {
+  g_err[0] = 0;
+  if (!h) return ZCMOE_OK;
+  {
+    std::lock_guard<std::mutex> lk(g_live_mu);
+    if (!g_live_dense.erase(h)) return fail(ZCMOE_EINVAL, "invalid or already destroyed dense handle");
+  }
+  cudaDeviceSynchronize();
+  release_dense(h);
   delete h;
   return ZCMOE_OK;
 }

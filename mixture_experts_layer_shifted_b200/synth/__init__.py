@@ -46,6 +46,9 @@ TID_WU = 4
 TID_WD = 5
 TID_BIAS = 6
 TID_ZIPF = 7
+TID_DENSE_G = 8   # dense FFN path (ScMoE): W_gate, W_up, W_down
+TID_DENSE_U = 9
+TID_DENSE_D = 10
 
 
 def philox4x32_10(c0, c1, c2, c3, k0, k1):

@@ -30,7 +30,9 @@ ZCMOE_BF16 = 1
 
 EXPORTED = ("zcmoe_create", "zcmoe_forward", "zcmoe_forward_host", "zcmoe_update_bias", "zcmoe_read_counts",
             "zcmoe_write_counts", "zcmoe_get_state", "zcmoe_set_bias", "zcmoe_check", "zcmoe_profile_begin",
-            "zcmoe_profile_end", "zcmoe_selftest_wait", "zcmoe_route_noalloc", "zcmoe_destroy", "zcmoe_last_error")
+            "zcmoe_profile_end", "zcmoe_selftest_wait", "zcmoe_route_noalloc", "zcmoe_destroy",
+            "zcmoe_dense_create", "zcmoe_dense_forward", "zcmoe_forward_overlap", "zcmoe_dense_check",
+            "zcmoe_dense_destroy", "zcmoe_last_error")
 STAGES = ("router", "softmax_topk", "integer", "gather", "gate_up", "down", "combine")
 
 
@@ -63,6 +65,14 @@ class zcmoe_debug(ctypes.Structure):
                 ("perm", ctypes.c_void_p), ("pos", ctypes.c_void_p), ("expert_out", ctypes.c_void_p)]
 
 
+class zcmoe_dense_config(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("inter", ctypes.c_int32), ("max_tokens", ctypes.c_int32)]
+
+
+class zcmoe_dense_weights(ctypes.Structure):
+    _fields_ = [("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p)]
+
+
 _lib = None
 
 
@@ -89,6 +99,12 @@ def lib():
         L.zcmoe_selftest_wait.argtypes = [vp, i64, vp]
         L.zcmoe_route_noalloc.argtypes = [vp, vp, i64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
                                           vp, vp, vp, vp, vp, vp, vp]
+        L.zcmoe_dense_create.argtypes = [ctypes.POINTER(zcmoe_dense_config), ctypes.POINTER(zcmoe_dense_weights),
+                                         ctypes.POINTER(vp)]
+        L.zcmoe_dense_forward.argtypes = [vp, vp, i64, vp, vp]
+        L.zcmoe_forward_overlap.argtypes = [vp, vp, vp, vp, i64, vp, vp, vp]
+        L.zcmoe_dense_check.argtypes = [vp]
+        L.zcmoe_dense_destroy.argtypes = [vp]
         for f in EXPORTED[:-1]:
             getattr(L, f).restype = i32
         L.zcmoe_last_error.argtypes = []
@@ -178,6 +194,29 @@ def zcmoe_route_noalloc(logits, bias, T, n_ffn, n_zero, top_k, routed_scale, idx
 
 def zcmoe_destroy(h):
     _check(lib().zcmoe_destroy(h), "zcmoe_destroy")
+
+
+def zcmoe_dense_create(cfg: zcmoe_dense_config, w: zcmoe_dense_weights) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(lib().zcmoe_dense_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)), "zcmoe_dense_create")
+    return h
+
+
+def zcmoe_dense_forward(h, x_ptr, T, y_ptr, stream=None):
+    _check(lib().zcmoe_dense_forward(h, x_ptr, T, y_ptr, _stream(stream)), "zcmoe_dense_forward")
+
+
+def zcmoe_forward_overlap(moe, dense, x_moe_ptr, x_dense_ptr, T, y_moe_ptr, y_dense_ptr, stream=None):
+    _check(lib().zcmoe_forward_overlap(moe, dense, x_moe_ptr, x_dense_ptr, T, y_moe_ptr, y_dense_ptr, _stream(stream)),
+           "zcmoe_forward_overlap")
+
+
+def zcmoe_dense_check(h):
+    _check(lib().zcmoe_dense_check(h), "zcmoe_dense_check")
+
+
+def zcmoe_dense_destroy(h):
+    _check(lib().zcmoe_dense_destroy(h), "zcmoe_dense_destroy")
 
 
 def zcmoe_last_error() -> str:
@@ -288,3 +327,53 @@ class ZcMoE:
             self.close()
         except Exception:
             pass
+
+
+class ZcDense:
+    """Owns a dense-FFN handle plus references to its (borrowed) bf16 weights:
+    w_gate [inter, d], w_up [inter, d], w_down [d, inter]."""
+
+    def __init__(self, w_gate, w_up, w_down, max_tokens: int):
+        inter, d = w_gate.shape
+        self.d, self.inter, self.max_tokens = d, inter, max_tokens
+        self.weights = (w_gate, w_up, w_down)
+        for t, want in zip(self.weights, [(inter, d), (inter, d), (d, inter)]):
+            if tuple(t.shape) != want or t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"weight of shape {tuple(t.shape)} {t.dtype}; expected {want} bfloat16")
+        cfg = zcmoe_dense_config(d, inter, max_tokens)
+        w = zcmoe_dense_weights(w_gate.data_ptr(), w_up.data_ptr(), w_down.data_ptr())
+        self.h = zcmoe_dense_create(cfg, w)
+
+    def forward(self, x, y=None, stream=None):
+        if y is None:
+            y = torch.empty_like(x)
+        zcmoe_dense_forward(self.h, ctypes.c_void_p(x.data_ptr()), x.shape[0], ctypes.c_void_p(y.data_ptr()), stream)
+        return y
+
+    def check(self):
+        zcmoe_dense_check(self.h)
+
+    def close(self):
+        if self.h is not None:
+            zcmoe_dense_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def forward_overlap(moe: ZcMoE, dense: ZcDense, x_moe, x_dense=None, y_moe=None, y_dense=None, stream=None):
+    """(y_moe, y_dense): the MoE layer and the dense FFN over the same tokens, run
+    concurrently (zcmoe_forward_overlap).  x_dense defaults to x_moe."""
+    x_dense = x_moe if x_dense is None else x_dense
+    if x_dense.shape[0] != x_moe.shape[0]:
+        raise ValueError("x_moe and x_dense must hold the same number of tokens")
+    y_moe = torch.empty_like(x_moe) if y_moe is None else y_moe
+    y_dense = torch.empty_like(x_dense) if y_dense is None else y_dense
+    zcmoe_forward_overlap(moe.h, dense.h, ctypes.c_void_p(x_moe.data_ptr()), ctypes.c_void_p(x_dense.data_ptr()),
+                          x_moe.shape[0], ctypes.c_void_p(y_moe.data_ptr()), ctypes.c_void_p(y_dense.data_ptr()),
+                          stream)
+    return y_moe, y_dense

@@ -83,3 +83,32 @@ def test_create_without_a_device_fails_cleanly(zc):
     rc = lib.zcmoe_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h))
     assert rc in (zc.ZCMOE_ECUDA, zc.ZCMOE_EUNSUPPORTED)
     assert h.value is None
+
+
+def test_dense_and_overlap_arguments_are_rejected_on_the_host(zc):
+    lib = zc.lib()
+    h = ctypes.c_void_p()
+    w = zc.zcmoe_dense_weights(16, 16, 16)
+    cfg = zc.zcmoe_dense_config(256, 384, 64)
+    assert lib.zcmoe_dense_create(None, ctypes.byref(w), ctypes.byref(h)) == zc.ZCMOE_EINVAL
+    assert lib.zcmoe_dense_create(ctypes.byref(cfg), ctypes.byref(w), None) == zc.ZCMOE_EINVAL
+    for bad in [dict(d=100), dict(d=0), dict(inter=32), dict(inter=100), dict(max_tokens=0),
+                dict(max_tokens=(1 << 20) + 1)]:
+        c = zc.zcmoe_dense_config(256, 384, 64)
+        for k_, v in bad.items():
+            setattr(c, k_, v)
+        assert lib.zcmoe_dense_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(h)) == zc.ZCMOE_EINVAL, bad
+        assert h.value is None
+        assert zc.zcmoe_last_error() != ""
+    assert lib.zcmoe_dense_create(ctypes.byref(cfg), ctypes.byref(zc.zcmoe_dense_weights(16, 24, 16)),
+                                  ctypes.byref(h)) == zc.ZCMOE_EINVAL  # misaligned
+    assert lib.zcmoe_dense_create(ctypes.byref(cfg), ctypes.byref(zc.zcmoe_dense_weights(16, 16, None)),
+                                  ctypes.byref(h)) == zc.ZCMOE_EINVAL
+    # handles that were never created are refused, not dereferenced; a MoE handle
+    # is not a dense handle
+    fake = ctypes.c_void_p(0x1000)
+    assert lib.zcmoe_dense_forward(fake, None, 1, None, None) == zc.ZCMOE_EINVAL
+    assert lib.zcmoe_dense_check(fake) == zc.ZCMOE_EINVAL
+    assert lib.zcmoe_dense_destroy(fake) == zc.ZCMOE_EINVAL
+    assert lib.zcmoe_dense_destroy(None) == zc.ZCMOE_OK
+    assert lib.zcmoe_forward_overlap(fake, fake, None, None, 1, None, None, None) == zc.ZCMOE_EINVAL
