@@ -201,6 +201,53 @@ def run_reference(args, wl, rank, ws):
     print(json.dumps(line), flush=True)
 
 
+def measure_overlap(wl, layer, x, stream, peaks, reps=10):
+    """The dense FFN path beside the layer on the same batch (shortcut-connected
+    MoE): device time of the layer alone, the dense FFN alone, the two one after
+    the other, and the two through zcmoe_forward_overlap; each a replayed graph."""
+    import torch
+    from mixture_experts_layer_shifted_b200 import configs
+    from mixture_experts_layer_shifted_b200.zcmoe import ZcDense, forward_overlap
+
+    dense = ZcDense(*configs.device_dense_weights(wl), max_tokens=wl.T)
+    y, yd = torch.empty_like(x), torch.empty_like(x)
+    variants = {
+        "moe": lambda: layer.forward(x, y),
+        "dense": lambda: dense.forward(x, yd),
+        "sequential": lambda: (layer.forward(x, y), dense.forward(x, yd)),
+        "overlap": lambda: forward_overlap(layer, dense, x, y_moe=y, y_dense=yd),
+    }
+    ms = {}
+    for name, fn in variants.items():
+        fn()  # first calls outside the capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms[name] = a.elapsed_time(b) / reps
+        del g
+    dense.check()
+    layer.check()
+    dense.close()
+    f_dense = 6.0 * wl.T * wl.d * wl.dense_inter
+    hidden = ms["sequential"] - ms["overlap"]
+    tflops = f_dense / (ms["dense"] * 1e-3) / 1e12
+    return {"dense_inter": wl.dense_inter, "ms_moe": ms["moe"], "ms_dense": ms["dense"],
+            "ms_sequential": ms["sequential"], "ms_overlap": ms["overlap"], "hidden_ms": hidden,
+            "hidden_frac_of_dense": hidden / ms["dense"], "speedup": ms["sequential"] / ms["overlap"],
+            "dense_tflops": tflops, "dense_frac": tflops / peaks["bf16_tflops_sustained"],
+            "note": "each variant one replayed CUDA graph, %d replays after 3; same batch for both paths" % reps}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -403,6 +450,10 @@ def main():
                           "hbm_gbs": hbm, "hbm_frac": hbm / peaks["hbm_gbs"], "bytes": B2,
                           "P": int(cnt2.sum()), "distinct_experts": int((cnt2 > 0).sum())}
         layer2.close()
+
+    # secondary: the dense FFN path run beside the layer (shortcut-connected MoE)
+    if rank == 0 and ws == 1 and not args.no_secondary and wl.dense_inter > 0:
+        line["scmoe_overlap"] = measure_overlap(wl, layer, xs[0], stream, peaks)
 
     layer.close()
     if rank == 0:
