@@ -61,6 +61,17 @@ def lib():
         L.zo_route_replica_f32.restype = None
         L.zo_integer_stage.argtypes = [I32P, i64, i32, i32, i32, I32P, I32P, I32P, I32P]
         L.zo_integer_stage.restype = i64
+        U8P = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
+        L.zo_e4m3_encode.argtypes = [f32]
+        L.zo_e4m3_encode.restype = ctypes.c_uint8
+        L.zo_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.zo_e4m3_decode.restype = f64
+        L.zo_e8m0_scale.argtypes = [f32]
+        L.zo_e8m0_scale.restype = ctypes.c_uint8
+        L.zo_quantize_blocks.argtypes = [vp, i32, i64, i64, i32, U8P, U8P]
+        L.zo_quantize_blocks.restype = None
+        L.zo_ffn_fp8_f64.argtypes = [vp, i32, i64, U8P, U8P, U8P, U8P, U8P, U8P, i32, i32, F64P]
+        L.zo_ffn_fp8_f64.restype = None
         L.zo_ffn_f64.argtypes = [vp, i32, i64, vp, vp, vp, i32, i32, i32, F64P]
         L.zo_ffn_f64.restype = None
         L.zo_layer_f64.argtypes = [vp, i32, i64, I32P, F64P, i32, i32, vp, vp, vp, i32, i32, i32, F64P]
@@ -226,3 +237,52 @@ def brute_force_topk(v, k):
         if best is None or s > best_sum:
             best, best_sum = comb, s
     return sorted(best, key=lambda i: (-float(v[i]), i))
+
+
+# ----------------------------------------------------------------- block-scaled FP8
+def e4m3_encode(v: float) -> int:
+    """E4M3 code of v (round to nearest even, saturating at 448)."""
+    return int(lib().zo_e4m3_encode(float(v)))
+
+
+def e4m3_decode(code: int) -> float:
+    return float(lib().zo_e4m3_decode(int(code)))
+
+
+def e8m0_scale(amax: float) -> int:
+    """E8M0 code of the smallest power of two s with amax <= 448 s (127 for amax 0)."""
+    return int(lib().zo_e8m0_scale(float(amax)))
+
+
+def quantize_blocks(src, block_rows):
+    """(codes [rows, cols] uint8, scales [ceil(rows/block_rows), cols/128] uint8) of a
+    2-D fp32 array or bf16 bit array; block_rows 1 or 128."""
+    src, dt = _arr(src)
+    rows, cols = src.shape
+    if cols % 128:
+        raise ValueError("cols must be a multiple of 128")
+    codes = np.empty((rows, cols), np.uint8)
+    scales = np.empty(((rows + block_rows - 1) // block_rows, cols // 128), np.uint8)
+    lib().zo_quantize_blocks(src.ctypes.data, dt, rows, cols, block_rows, codes, scales)
+    return codes, scales
+
+
+def dequantize_blocks(codes, scales, block_rows):
+    """fp64 values codes * 2^(scale - 127) (NaN codes give NaN)."""
+    table = np.array([e4m3_decode(c) for c in range(256)], np.float64)
+    rows, cols = codes.shape
+    sc = np.repeat(np.repeat(scales.astype(np.int64) - 127, block_rows, 0)[:rows], 128, 1)
+    return np.ldexp(table[codes], sc)
+
+
+def ffn_fp8(xs, wq, sq):
+    """fp64 SwiGLU expert on FP8 operands: xs [n, d] (fp32 or bf16 bits) quantized per
+    [1,128] inside; wq = (wg, wu, wd) codes, sq = their [128,128] scales."""
+    xs, xd = _arr(xs)
+    n, d = xs.shape
+    wg, wu, wd = (np.ascontiguousarray(w, np.uint8) for w in wq)
+    sg, su, sd = (np.ascontiguousarray(s_, np.uint8) for s_ in sq)
+    inter = wg.shape[0]
+    out = np.empty((n, d), np.float64)
+    lib().zo_ffn_fp8_f64(xs.ctypes.data, xd, n, wg, sg, wu, su, wd, sd, d, inter, out)
+    return out

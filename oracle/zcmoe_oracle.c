@@ -347,3 +347,141 @@ ZO_EXPORT void zo_update_bias(int64_t *counts, int64_t *tokens, int N, int Z, in
   }
   *tokens = 0;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Block-scaled FP8 experts.                                                  */
+/* LongCat-Flash technical summary (zhangjingwei.cn), 六 推理與部署, 定制內核    */
+/* "量化": the same fine-grained block quantization as DeepSeek-V3, one scale   */
+/* per [1,128] block of activations and per [128,128] block of weights.      */
+/* Readings (the pages fix neither the code nor the scale format):            */
+/*  - codes are FP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa      */
+/*    bits; no infinities; S.1111.111 is NaN; largest finite 448), rounded to  */
+/*    nearest with ties to even, saturating at 448;                            */
+/*  - a block's scale is a power of two stored as E8M0 (value 2^(c-127)): the  */
+/*    smallest 2^E with amax <= 448 * 2^E (code clamped to [0, 254]); an all-  */
+/*    zero block takes 2^0;  q = E4M3(v / 2^E), v ~ q * 2^E.                    */
+/* Parity: pinned against torch's float8_e4m3fn conversion, boundary values   */
+/* and closed forms in tests/test_oracle_pins.py.                             */
+/* ------------------------------------------------------------------------- */
+
+ZO_EXPORT double zo_e4m3_decode(uint8_t c) {
+  const int s = c >> 7, E = (c >> 3) & 15, M = c & 7;
+  if (E == 15 && M == 7) return NAN;
+  const double v = (E == 0) ? ldexp((double)M, -9) : ldexp(8.0 + M, E - 10);
+  return s ? -v : v;
+}
+
+ZO_EXPORT uint8_t zo_e4m3_encode(float v) {
+  if (isnan(v)) return 0x7F;
+  const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  const double a = fabs((double)v);
+  if (a >= 448.0) return sign | 0x7E;
+  /* spacing of representable magnitudes around a: 2^-9 below the smallest
+     normal 2^-6, else 2^(k-3) for a in [2^k, 2^(k+1)) */
+  double q;
+  if (a < ldexp(1.0, -6)) {
+    q = ldexp(1.0, -9);
+  } else {
+    int e;
+    frexp(a, &e); /* a in [2^(e-1), 2^e) */
+    q = ldexp(1.0, e - 1 - 3);
+  }
+  const double n = a / q; /* exact: q is a power of two */
+  double r = floor(n);
+  const double frac = n - r;
+  if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) == 1.0)) r += 1.0;
+  const double val = r * q; /* <= 448 because a < 448 */
+  if (val == 0.0) return sign;
+  if (val < ldexp(1.0, -6)) return sign | (uint8_t)(val / ldexp(1.0, -9)); /* subnormal, M = 1..7 */
+  int ee;
+  const double m = frexp(val, &ee); /* val = m * 2^ee, m in [0.5, 1) */
+  const int E = ee - 1 + 7;
+  const int M = (int)((2.0 * m - 1.0) * 8.0);
+  return sign | (uint8_t)(E << 3) | (uint8_t)M;
+}
+
+ZO_EXPORT uint8_t zo_e8m0_scale(float amax) {
+  if (!(amax > 0.0f)) return 127;
+  int e;
+  frexp((double)amax, &e); /* amax in [2^k, 2^(k+1)), k = e - 1 */
+  const int k = e - 1;
+  const int E = ((double)amax <= 1.75 * ldexp(1.0, k)) ? k - 8 : k - 7; /* 448 = 1.75 * 2^8 */
+  int code = E + 127;
+  if (code < 0) code = 0;
+  if (code > 254) code = 254;
+  return (uint8_t)code;
+}
+
+/* src [rows, cols] (dtype 0 fp32, 1 bf16 bits), cols a multiple of 128;
+   block_rows 1 ([1,128] blocks) or 128 ([128,128] blocks; a last partial row
+   block is allowed).  codes [rows, cols]; scales [ceil(rows/block_rows), cols/128]. */
+ZO_EXPORT void zo_quantize_blocks(const void *src, int dtype, int64_t rows, int64_t cols, int block_rows,
+                                  uint8_t *codes, uint8_t *scales) {
+  const int64_t nrb = (rows + block_rows - 1) / block_rows, ncb = cols / 128;
+  for (int64_t rb = 0; rb < nrb; ++rb) {
+    const int64_t r0 = rb * block_rows, r1 = (r0 + block_rows < rows) ? r0 + block_rows : rows;
+    for (int64_t cb = 0; cb < ncb; ++cb) {
+      double amax = 0.0;
+      for (int64_t r = r0; r < r1; ++r)
+        for (int64_t c = cb * 128; c < cb * 128 + 128; ++c) {
+          const double a = fabs(elem(src, dtype, r * cols + c));
+          if (a > amax) amax = a;
+        }
+      const uint8_t sc = zo_e8m0_scale((float)amax); /* exact: amax is a source value */
+      scales[rb * ncb + cb] = sc;
+      const double inv = ldexp(1.0, 127 - (int)sc);
+      for (int64_t r = r0; r < r1; ++r)
+        for (int64_t c = cb * 128; c < cb * 128 + 128; ++c)
+          codes[r * cols + c] = zo_e4m3_encode((float)(elem(src, dtype, r * cols + c) * inv));
+    }
+  }
+}
+
+/* FFN expert on block-scaled FP8 operands, fp64 arithmetic on the dequantized
+   values.  Each row of xs (dtype as zo_ffn_f64) is quantized per [1,128] here;
+   the weights come as codes with [128,128] scales: wg, wu [inter, d] with
+   scales [inter/128, d/128]; wd [d, inter] with scales [d/128, inter/128].
+   h = silu(g) * u is rounded to fp32 and quantized per [1,128] before the down
+   projection (reading: the kernel quantizes H from its fp32 values, so the
+   quantization decision is taken in that precision).  out [n, d] fp64. */
+ZO_EXPORT void zo_ffn_fp8_f64(const void *xs, int x_dtype, int64_t n, const uint8_t *wg, const uint8_t *sg,
+                              const uint8_t *wu, const uint8_t *su, const uint8_t *wd, const uint8_t *sd, int d,
+                              int inter, double *out) {
+  const size_t xsz = (x_dtype == 1) ? 2 : 4;
+  uint8_t *xq = (uint8_t *)malloc((size_t)d), *xs_sc = (uint8_t *)malloc((size_t)d / 128);
+  uint8_t *hq = (uint8_t *)malloc((size_t)inter), *hs_sc = (uint8_t *)malloc((size_t)inter / 128);
+  double *xv = (double *)malloc(sizeof(double) * (size_t)d);
+  double *hv = (double *)malloc(sizeof(double) * (size_t)inter);
+  float *h32 = (float *)malloc(sizeof(float) * (size_t)inter);
+  const int dkb = d / 128, ikb = inter / 128;
+  for (int64_t r = 0; r < n; ++r) {
+    zo_quantize_blocks((const char *)xs + (size_t)(r * d) * xsz, x_dtype, 1, d, 1, xq, xs_sc);
+    for (int c = 0; c < d; ++c) xv[c] = ldexp(zo_e4m3_decode(xq[c]), (int)xs_sc[c / 128] - 127);
+#pragma omp parallel for schedule(static)
+    for (int i = 0; i < inter; ++i) {
+      double g = 0.0, u = 0.0;
+      for (int c = 0; c < d; ++c) {
+        const int sgi = (int)sg[(i / 128) * dkb + c / 128] - 127, sui = (int)su[(i / 128) * dkb + c / 128] - 127;
+        g += ldexp(zo_e4m3_decode(wg[(int64_t)i * d + c]), sgi) * xv[c];
+        u += ldexp(zo_e4m3_decode(wu[(int64_t)i * d + c]), sui) * xv[c];
+      }
+      h32[i] = (float)(g / (1.0 + exp(-g)) * u);
+    }
+    zo_quantize_blocks(h32, 0, 1, inter, 1, hq, hs_sc);
+    for (int i = 0; i < inter; ++i) hv[i] = ldexp(zo_e4m3_decode(hq[i]), (int)hs_sc[i / 128] - 127);
+#pragma omp parallel for schedule(static)
+    for (int c = 0; c < d; ++c) {
+      double acc = 0.0;
+      for (int i = 0; i < inter; ++i)
+        acc += ldexp(zo_e4m3_decode(wd[(int64_t)c * inter + i]), (int)sd[(c / 128) * ikb + i / 128] - 127) * hv[i];
+      out[r * d + c] = acc;
+    }
+  }
+  free(xq);
+  free(xs_sc);
+  free(hq);
+  free(hs_sc);
+  free(xv);
+  free(hv);
+  free(h32);
+}

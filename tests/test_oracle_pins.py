@@ -379,3 +379,107 @@ def test_page_layer_shape_is_consistent():
     expect = cfg["top_k"] * cfg["n_ffn"] / (cfg["n_ffn"] + cfg["n_zero"])
     lo, hi = min(cfg["realised_ffn_per_token"].values()), max(cfg["realised_ffn_per_token"].values())
     assert lo <= expect <= hi
+
+
+# ---------------------------------------------------------------- block-scaled FP8 (oracle only)
+
+def test_e4m3_decode_all_codes_against_torch():
+    import torch
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float32).numpy().astype(np.float64)
+    got = np.array([oracle.e4m3_decode(c) for c in range(256)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x38] == 1.0 and np.isnan(got[0x7F])
+
+
+def test_e4m3_encode_against_torch():
+    """Round to nearest even on exact values, midpoints (ties) and random values in [-448, 448]."""
+    import torch
+    exact = np.array([oracle.e4m3_decode(c) for c in range(256)])
+    exact = np.unique(exact[~np.isnan(exact)])
+    mids = (exact[1:] + exact[:-1]) / 2.0
+    rng = np.random.default_rng(11)
+    rnd = rng.uniform(-1, 1, 20000) * np.exp2(rng.integers(-12, 9, 20000))
+    vals = np.concatenate([exact, mids, rnd, [-0.0, 448.0, -448.0, 2.0 ** -10, 3 * 2.0 ** -10]]).astype(np.float32)
+    vals = vals[np.abs(vals) <= 448.0]
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(v) for v in vals], np.uint8)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, [(float(vals[i]), int(got[i]), int(ref[i])) for i in bad[:5]]
+    # saturation beyond the largest finite value
+    assert oracle.e4m3_encode(1e6) == 0x7E and oracle.e4m3_encode(-500.0) == 0xFE
+
+
+def test_e8m0_scale_is_the_smallest_sufficient_power_of_two():
+    rng = np.random.default_rng(12)
+    amax = (rng.uniform(0.5, 1.0, 5000) * np.exp2(rng.integers(-100, 100, 5000))).astype(np.float32)
+    for a in amax:
+        c = oracle.e8m0_scale(float(a))
+        assert 0 < c < 254
+        s = 2.0 ** (c - 127)
+        assert a / s <= 448.0 < a / (s / 2), (a, c)
+    assert oracle.e8m0_scale(0.0) == 127
+    assert oracle.e8m0_scale(448.0) == 127 and oracle.e8m0_scale(np.nextafter(np.float32(448), np.float32(1e9))) == 128
+    assert oracle.e8m0_scale(1.75 * 2.0 ** 20) == 127 + 12 and oracle.e8m0_scale(2.0 ** 21) == 127 + 13
+    assert oracle.e8m0_scale(2.0 ** -140) == 0      # clamped: the block quantizes to zeros and small codes
+    assert oracle.e8m0_scale(3e38) == 127 + 120
+
+
+@pytest.mark.parametrize("block_rows,rows", [(1, 7), (128, 300)])
+def test_quantize_blocks_error_bound_and_structure(block_rows, rows):
+    rng = np.random.default_rng(13)
+    cols = 384
+    x = (rng.standard_normal((rows, cols)) * np.exp2(rng.integers(-6, 6, (rows, 1)))).astype(np.float32)
+    codes, scales = oracle.quantize_blocks(x, block_rows)
+    assert scales.shape == ((rows + block_rows - 1) // block_rows, cols // 128)
+    deq = oracle.dequantize_blocks(codes, scales, block_rows)
+    s = np.ldexp(1.0, np.repeat(np.repeat(scales.astype(np.int64) - 127, block_rows, 0)[:rows], 128, 1))
+    v = x.astype(np.float64) / s                         # exact scaled values
+    assert np.abs(v).max() <= 448.0
+    e = np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** -6)))
+    spacing = np.exp2(e - 3)                             # 2^-9 below the smallest normal
+    assert np.all(np.abs(v - deq / s) <= spacing / 2)
+    # each block's scale is minimal: its largest scaled value exceeds 224
+    for rb in range(scales.shape[0]):
+        for cb in range(scales.shape[1]):
+            blk = np.abs(v[rb * block_rows:(rb + 1) * block_rows, cb * 128:(cb + 1) * 128])
+            assert blk.max() > 224.0
+
+
+def test_ffn_fp8_lossless_closed_form():
+    """One token, one active hidden unit, every value exactly representable after
+    quantization: g = 64 (silu(64) rounds to 64 in fp32), u = 1, so y = 64 * W_d[:, 0]
+    exactly.  Swapping gate and up would give silu(1) * 64 instead."""
+    d = inter = 128
+    x = np.zeros((1, d), np.float32)
+    x[0, 0] = 1.0
+    wg = np.zeros((inter, d), np.float32)
+    wu = np.zeros((inter, d), np.float32)
+    wg[0, 0], wu[0, 0] = 64.0, 1.0
+    wd = np.zeros((d, inter), np.float32)
+    wd[:, 0] = ((np.arange(d) % 8) - 4) * 0.25
+    q = [oracle.quantize_blocks(w, 128) for w in (wg, wu, wd)]
+    for (c, s_), w in zip(q, (wg, wu, wd)):
+        assert np.array_equal(oracle.dequantize_blocks(c, s_, 128), w)   # lossless
+    y = oracle.ffn_fp8(x, [c for c, _ in q], [s_ for _, s_ in q])
+    assert np.array_equal(y[0], 64.0 * wd[:, 0].astype(np.float64))
+    y_swapped = oracle.ffn_fp8(x, [q[1][0], q[0][0], q[2][0]], [q[1][1], q[0][1], q[2][1]])
+    assert not np.allclose(y_swapped, y)
+
+
+def test_ffn_fp8_is_close_to_the_unquantized_expert():
+    """The quantization error of the method on random data: a few percent of a row's
+    largest output, far below the difference a wrong operand or scale would make."""
+    rng = np.random.default_rng(14)
+    d, inter = 256, 384
+    x = rng.standard_normal((4, d)).astype(np.float32)
+    wg, wu = (rng.standard_normal((inter, d)) * 0.06).astype(np.float32), (rng.standard_normal((inter, d)) * 0.06).astype(np.float32)
+    wd = (rng.standard_normal((d, inter)) * 0.05).astype(np.float32)
+    q = [oracle.quantize_blocks(w, 128) for w in (wg, wu, wd)]
+    y8 = oracle.ffn_fp8(x, [c for c, _ in q], [s_ for _, s_ in q])
+    y = oracle.ffn(x, wg, wu, wd)
+    rel = np.abs(y8 - y).max(axis=1) / np.abs(y).max(axis=1)
+    assert rel.max() < 0.08, rel
+    assert rel.max() > 1e-4          # it is a lossy path
