@@ -52,13 +52,24 @@ extern "C" {
 
 typedef struct zcmoe_s *zcmoe_t;
 
-typedef enum { ZCMOE_F32 = 0, ZCMOE_BF16 = 1 } zcmoe_dtype;
+typedef enum { ZCMOE_F32 = 0, ZCMOE_BF16 = 1, ZCMOE_FP8 = 2 } zcmoe_dtype;
 
 /* Layer shape and routing constants.  Sizes are element counts.
  * Limits: 1 <= n_ffn, 0 <= n_zero, E = n_ffn + n_zero <= 1024, 1 <= top_k <= min(E, 32),
  * d and inter multiples of 64, 1 <= max_tokens <= 2^20.
  * dtype: ZCMOE_BF16 -> x, y, all weights bf16, fp32 accumulation (tensor cores);
- *        ZCMOE_F32  -> everything fp32 with fp32 CUDA-core arithmetic (no TF32). */
+ *        ZCMOE_F32  -> everything fp32 with fp32 CUDA-core arithmetic (no TF32);
+ *        ZCMOE_FP8  -> x, y and all weights bf16 at the interface, FFN experts on
+ *                      block-scaled FP8 (technical summary, 六 定制內核 "量化": DeepSeek-V3's
+ *                      blocks, one scale per [1,128] of activations and per [128,128]
+ *                      of weights): E4M3 codes, power-of-two E8M0 scales (the
+ *                      smallest 2^E with block max <= 448 * 2^E), fp32 accumulation.
+ *                      zcmoe_create quantizes the expert weights into memory of its
+ *                      own and reads w_gate / w_up / w_down only then; x rows are
+ *                      quantized per [1,128] on the way into the gate/up GEMM and
+ *                      silu(g)*u per [1,128] before the down GEMM; the router, the
+ *                      combine and y stay bf16.  Needs d a multiple of 512 and inter
+ *                      a multiple of 128. */
 typedef struct {
   int32_t d;            /* hidden size                                   */
   int32_t n_ffn;        /* N, FFN experts                                */
@@ -95,7 +106,7 @@ typedef struct {
  * counts [E] int32, offsets [N+1] int32 (exclusive scan of FFN counts; offsets[N] = P),
  * perm [T*k] int32 (first P entries valid: FFN pairs t*k+j ordered by expert then
  * token), pos [T, k] int32 (row of pair (t,j) in the permuted order, -1 for zero experts),
- * expert_out [T*k, d] config dtype (first P rows valid: the FFN expert outputs F_e(x_t),
+ * expert_out [T*k, d] config dtype, bf16 for ZCMOE_FP8 (first P rows valid: the FFN expert outputs F_e(x_t),
  * one row per pair in the permuted order, before gating). */
 typedef struct {
   float *logits;
@@ -210,6 +221,18 @@ ZCMOE_API int zcmoe_route_noalloc(const float *logits, const float *bias, int64_
 
 /* Frees the handle's own memory; never touches the borrowed weights.  NULL is a no-op. */
 ZCMOE_API int zcmoe_destroy(zcmoe_t h);
+
+/* Block quantization to FP8 E4M3 with E8M0 scales, the rule ZCMOE_FP8 layers use
+ * (round to nearest even; scale 2^E the smallest power of two with the block's
+ * largest magnitude <= 448 * 2^E, E + 127 clamped to [0, 254]; an all-zero block
+ * takes 2^0).  No handle needed.
+ *   src [rows, cols] device, ZCMOE_BF16 or ZCMOE_F32 (src_dtype), 16-byte aligned;
+ *   cols a positive multiple of 128; block_rows 1 ([1,128] blocks) or 128
+ *   ([128,128] blocks; the last row block may be partial);
+ *   codes [rows, cols] uint8 device; scales [ceil(rows / block_rows), cols / 128]
+ *   uint8 device (E8M0 bytes).  Asynchronous on `stream`. */
+ZCMOE_API int zcmoe_quantize_e4m3(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, int32_t block_rows,
+                                  uint8_t *codes, uint8_t *scales, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * Dense FFN path and the shortcut-connected overlap (ScMoE).

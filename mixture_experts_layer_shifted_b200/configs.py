@@ -24,7 +24,7 @@ class Workload:
     inter: int
     n_zero: int
     top_k: int
-    dtype: str            # "f32" or "bf16"
+    dtype: str            # "f32", "bf16", or "fp8" (bf16 interface, block-scaled FP8 experts)
     x_std: float = 1.0
     w_std: float = 0.02
     bias: tuple = ("zero",)   # ("zero",) | ("uniform", lo, hi) | ("zero_experts", value)
@@ -40,7 +40,7 @@ class Workload:
         return self.n_ffn + self.n_zero
 
     def weight_bytes(self):
-        esz = 2 if self.dtype == "bf16" else 4
+        esz = 4 if self.dtype == "f32" else 2
         return (3 * self.n_ffn * self.inter * self.d + self.E * self.d) * esz
 
     def with_(self, **kw):
@@ -69,6 +69,10 @@ WORKLOADS = {
     "prefill_probe": Workload("prefill_probe", T=2048, d=6144, n_ffn=32, inter=2048, n_zero=16, top_k=12,
                               dtype="bf16", w_std=0.006, bias=("zero",), dense_inter=12288),
 }
+# the same layers with block-scaled FP8 experts
+for _name in ("small_bf16", "prefill_560b", "decode_560b", "skewed_4096", "prefill_probe"):
+    _fp8 = _name.replace("_bf16", "") + "_fp8"
+    WORKLOADS[_fp8] = WORKLOADS[_name].with_(name=_fp8, dtype="fp8")
 
 
 def bias_vector(w: Workload) -> np.ndarray:
@@ -91,7 +95,7 @@ def logit_offsets(w: Workload):
 def device_weights(w: Workload, device="cuda"):
     """(w_router [E,d], w_gate [N,inter,d], w_up [N,inter,d], w_down [N,d,inter]) on the device."""
     import torch
-    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
     shapes = [(w.E, w.d), (w.n_ffn, w.inter, w.d), (w.n_ffn, w.inter, w.d), (w.n_ffn, w.d, w.inter)]
     tids = [synth.TID_WR, synth.TID_WG, synth.TID_WU, synth.TID_WD]
     out = []
@@ -121,7 +125,7 @@ def device_tokens(w: Workload, T: int | None = None, device="cuda", step: int = 
     """x [T, d] on the device; step > 0 gives a fresh batch of the same distribution."""
     import torch
     T = w.T if T is None else T
-    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
     x = torch.empty((T, w.d), dtype=dt, device=device)
     synth.fill_normal_(x, synth.TID_X + 16 * step, w.seed, w.x_std)
     return x

@@ -1,0 +1,199 @@
+// Block quantizers to FP8 E4M3 with E8M0 power-of-two scales (rule in zc_fp8.cuh):
+//   k_quant_rows  : [1,128] blocks (activations), one warp per block
+//   k_quant_tiles : [128,128] blocks (weights), one CTA per block
+//   k_gather_quant: the FFN pairs' token rows, quantized per [1,128] on the way
+//                   into the expert-sorted operand of the FP8 gate/up GEMM
+// Scales go out either plain ([row blocks, cols/128], for zcmoe_quantize_e4m3)
+// or as the GEMM's scale atoms.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "zc_fp8.cuh"
+#include "zc_internal.h"
+
+namespace zc {
+namespace {
+
+__device__ __forceinline__ float ld_f(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ float ld_f(const float* p) { return *p; }
+
+// four consecutive elements (8- or 16-byte aligned)
+__device__ __forceinline__ void ld4(const __nv_bfloat16* p, float* v) {
+  const uint2 r = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+  v[0] = a.x;
+  v[1] = a.y;
+  v[2] = b.x;
+  v[3] = b.y;
+}
+__device__ __forceinline__ void ld4(const float* p, float* v) {
+  const float4 r = *reinterpret_cast<const float4*>(p);
+  v[0] = r.x;
+  v[1] = r.y;
+  v[2] = r.z;
+  v[3] = r.w;
+}
+
+__device__ __forceinline__ float warp_max(float a) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  return a;
+}
+
+template <typename TIN, bool ATOM>
+__global__ void __launch_bounds__(256) k_quant_rows(const TIN* __restrict__ src, int64_t rows, int cols,
+                                                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                    int groups) {
+  const int lane = threadIdx.x & 31;
+  const int ncb = cols >> 7;
+  const int64_t nblk = rows * ncb;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < nblk; i += nwarps) {
+    const int64_t r = i / ncb;
+    const int cb = (int)(i - r * ncb);
+    const int64_t off = r * cols + cb * 128 + lane * 4;
+    float v[4];
+    ld4(src + off, v);
+    const float amax = warp_max(fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
+    const uint32_t code = e8m0_code(amax);
+    const float inv = e8m0_inverse(code);
+    *reinterpret_cast<uint32_t*>(codes + off) = pack_e4m3x4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);
+    if (lane == 0) scales[ATOM ? atom_offset(r, cb, groups) : r * ncb + cb] = (uint8_t)code;
+  }
+}
+
+template <typename TIN, bool ATOM>
+__global__ void __launch_bounds__(128) k_quant_tiles(const TIN* __restrict__ src, int64_t rows, int cols,
+                                                     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                     int groups) {
+  __shared__ float part[4];
+  const int cb = blockIdx.x;
+  const int64_t r0 = (int64_t)blockIdx.y * 128;
+  const int nr = (int)(rows - r0 < 128 ? rows - r0 : 128);
+  const int c = cb * 128 + threadIdx.x;
+  float amax = 0.0f;
+  for (int r = 0; r < nr; ++r) amax = fmaxf(amax, fabsf(ld_f(src + (r0 + r) * cols + c)));
+  amax = warp_max(amax);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = fmaxf(fmaxf(part[0], part[1]), fmaxf(part[2], part[3]));
+  const uint32_t code = e8m0_code(amax);
+  const float inv = e8m0_inverse(code);
+  for (int r = 0; r < nr; ++r)
+    codes[(r0 + r) * cols + c] = (uint8_t)(pack_e4m3x4(ld_f(src + (r0 + r) * cols + c) * inv, 0.f, 0.f, 0.f) & 0xFFu);
+  if (ATOM) {
+    if ((int)threadIdx.x < nr) scales[atom_offset(r0 + threadIdx.x, cb, groups)] = (uint8_t)code;
+  } else if (threadIdx.x == 0) {
+    scales[blockIdx.y * (cols >> 7) + cb] = (uint8_t)code;
+  }
+}
+
+// FFN pair p (expert e, token t = perm[p] / k) goes to padded row
+// p - offsets[e] + 128 * mb_off[e], so every expert's rows start a 128-row block.
+__global__ void __launch_bounds__(256) k_gather_quant(const __nv_bfloat16* __restrict__ x, int d,
+                                                      const int32_t* __restrict__ perm,
+                                                      const int32_t* __restrict__ idx, int k,
+                                                      const int32_t* __restrict__ offsets,
+                                                      const int32_t* __restrict__ mb_off,
+                                                      const int32_t* __restrict__ scal, uint8_t* __restrict__ x8,
+                                                      uint8_t* __restrict__ sx, int groups) {
+  const int P = scal[0];
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
+  for (int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); p < P; p += nwarps) {
+    const int pair = perm[p];
+    const int e = idx[pair];
+    const int64_t pad = (int64_t)(p - offsets[e]) + (int64_t)mb_off[e] * 128;
+    const __nv_bfloat16* src = x + (int64_t)(pair / k) * d;
+    uint8_t* dst = x8 + pad * d;
+    for (int c0 = 0; c0 < d; c0 += 512) {  // d is a multiple of 512
+      // four 128-column blocks in flight per lane
+      float v[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) ld4(src + c0 + 128 * u + lane * 4, v[u]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float amax =
+            warp_max(fmaxf(fmaxf(fabsf(v[u][0]), fabsf(v[u][1])), fmaxf(fabsf(v[u][2]), fabsf(v[u][3]))));
+        const uint32_t code = e8m0_code(amax);
+        const float inv = e8m0_inverse(code);
+        *reinterpret_cast<uint32_t*>(dst + c0 + 128 * u + lane * 4) =
+            pack_e4m3x4(v[u][0] * inv, v[u][1] * inv, v[u][2] * inv, v[u][3] * inv);
+        if (lane == 0) sx[atom_offset(pad, (c0 >> 7) + u, groups)] = (uint8_t)code;
+      }
+    }
+  }
+}
+
+// Debug copy: pair p's expert output from its padded row to row p.
+__global__ void __launch_bounds__(256) k_unpad_rows(const uint4* __restrict__ ypad, int row_vecs,
+                                                    const int32_t* __restrict__ perm, const int32_t* __restrict__ idx,
+                                                    const int32_t* __restrict__ offsets,
+                                                    const int32_t* __restrict__ mb_off,
+                                                    const int32_t* __restrict__ scal, uint4* __restrict__ out) {
+  const int P = scal[0];
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
+  for (int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); p < P; p += nwarps) {
+    const int e = idx[perm[p]];
+    const int64_t pad = (int64_t)(p - offsets[e]) + (int64_t)mb_off[e] * 128;
+    for (int v = lane; v < row_vecs; v += 32) out[(int64_t)p * row_vecs + v] = ypad[pad * row_vecs + v];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_unpad_rows(const void* ypad, int row_bytes, const int32_t* perm, const int32_t* idx,
+                              const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, void* out, int sms,
+                              cudaStream_t s) {
+  k_unpad_rows<<<sms * 4, 256, 0, s>>>(static_cast<const uint4*>(ypad), row_bytes / 16, perm, idx, offsets, mb_off,
+                                        scal, static_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows(int bf16, const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
+                              int atom_groups, int sms, cudaStream_t s) {
+  const int64_t warps = rows * (cols / 128);
+  int64_t blocks = (warps + 7) / 8;
+  if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+  if (blocks < 1) blocks = 1;
+  const bool atom = atom_groups > 0;
+  if (bf16) {
+    auto src_ = static_cast<const __nv_bfloat16*>(src);
+    if (atom) k_quant_rows<__nv_bfloat16, true><<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, atom_groups);
+    else k_quant_rows<__nv_bfloat16, false><<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, 0);
+  } else {
+    auto src_ = static_cast<const float*>(src);
+    if (atom) k_quant_rows<float, true><<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, atom_groups);
+    else k_quant_rows<float, false><<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, 0);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_tiles(int bf16, const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
+                               int atom_groups, cudaStream_t s) {
+  const dim3 grid(cols / 128, (unsigned)((rows + 127) / 128));
+  const bool atom = atom_groups > 0;
+  if (bf16) {
+    auto src_ = static_cast<const __nv_bfloat16*>(src);
+    if (atom) k_quant_tiles<__nv_bfloat16, true><<<grid, 128, 0, s>>>(src_, rows, cols, codes, scales, atom_groups);
+    else k_quant_tiles<__nv_bfloat16, false><<<grid, 128, 0, s>>>(src_, rows, cols, codes, scales, 0);
+  } else {
+    auto src_ = static_cast<const float*>(src);
+    if (atom) k_quant_tiles<float, true><<<grid, 128, 0, s>>>(src_, rows, cols, codes, scales, atom_groups);
+    else k_quant_tiles<float, false><<<grid, 128, 0, s>>>(src_, rows, cols, codes, scales, 0);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_quant(const void* x, int d, const int32_t* perm, const int32_t* idx, int k,
+                                const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x8,
+                                uint8_t* sx, int groups, int sms, cudaStream_t s) {
+  k_gather_quant<<<sms * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), d, perm, idx, k, offsets, mb_off, scal,
+                                          x8, sx, groups);
+  return cudaGetLastError();
+}
+
+}  // namespace zc

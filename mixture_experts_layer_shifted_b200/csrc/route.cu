@@ -334,10 +334,14 @@ struct Vec<float> {
 // One block per token.  Measured on B200 against variants with the slot loop
 // unrolled or several vectors per thread: this plain form keeps the most loads
 // in flight (many resident blocks) and reaches ~91% of the HBM copy rate.
+// With offsets / mb_off (FP8 layers), Y holds expert e's pairs from padded row
+// 128 mb_off[e] on, so a pair's row is pos - offsets[e] + 128 mb_off[e].
 template <typename TIO>
 __global__ void __launch_bounds__(128) k_combine(const TIO* __restrict__ x, const TIO* __restrict__ Y,
                                                  const float* __restrict__ gate, const int32_t* __restrict__ pos, int T,
-                                                 int k, int d, TIO* __restrict__ y) {
+                                                 int k, int d, TIO* __restrict__ y, const int32_t* __restrict__ idx,
+                                                 const int32_t* __restrict__ offsets,
+                                                 const int32_t* __restrict__ mb_off) {
   constexpr int V = Vec<TIO>::kN;
   __shared__ float sg[32];
   __shared__ int32_t sp[32];
@@ -346,7 +350,12 @@ __global__ void __launch_bounds__(128) k_combine(const TIO* __restrict__ x, cons
   const int t = blockIdx.x;
   if (threadIdx.x < k) {
     sg[threadIdx.x] = gate[(int64_t)t * k + threadIdx.x];
-    sp[threadIdx.x] = pos[(int64_t)t * k + threadIdx.x];
+    int p = pos[(int64_t)t * k + threadIdx.x];
+    if (offsets && p >= 0) {
+      const int e = idx[(int64_t)t * k + threadIdx.x];
+      p = p - offsets[e] + 128 * mb_off[e];
+    }
+    sp[threadIdx.x] = p;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -487,17 +496,17 @@ cudaError_t launch_gather_rows(const void* x, int row_bytes, const int32_t* perm
 }
 
 cudaError_t launch_combine(int bf16, const void* x, const void* Y, const int32_t* idx, const float* gate,
-                           const int32_t* pos, int T, int k, int N, int d, void* y, int sms, cudaStream_t s) {
-  (void)idx;
+                           const int32_t* pos, int T, int k, int N, int d, void* y, int sms, cudaStream_t s,
+                           const int32_t* offsets, const int32_t* mb_off) {
   (void)N;
   (void)sms;
   if (bf16)
     k_combine<__nv_bfloat16><<<T, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
                                                static_cast<const __nv_bfloat16*>(Y), gate, pos, T, k, d,
-                                               static_cast<__nv_bfloat16*>(y));
+                                               static_cast<__nv_bfloat16*>(y), idx, offsets, mb_off);
   else
     k_combine<float><<<T, 128, 0, s>>>(static_cast<const float*>(x), static_cast<const float*>(Y), gate, pos, T, k, d,
-                                       static_cast<float*>(y));
+                                       static_cast<float*>(y), idx, offsets, mb_off);
   return cudaGetLastError();
 }
 

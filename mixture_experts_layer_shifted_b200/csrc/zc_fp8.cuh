@@ -1,0 +1,57 @@
+// Block-scaled FP8 helpers shared by the quantizers and the FP8 GEMM.
+//
+// LongCat-Flash technical summary (zhangjingwei.cn), 六 推理與部署, 定制內核
+// "量化": DeepSeek-V3's fine-grained block quantization, one scale per [1,128]
+// block of activations and per [128,128] block of weights.  Codes are FP8 E4M3
+// (round to nearest even, saturating at 448); a block's scale is the smallest
+// power of two 2^E with amax <= 448 * 2^E, stored as the E8M0 byte E + 127
+// (clamped to [0, 254]; an all-zero block takes 2^0), which is the scale format
+// the tensor cores' block-scaled MMA reads.
+//
+// Scale atoms.  The block-scaled MMA takes its scales from tensor memory, one
+// byte per operand row per 32-deep K slice; tcgen05.cp (32x128b, broadcast to
+// the four lane quarters) fills them from a 512-byte shared-memory atom that
+// holds 128 operand rows x 4 K-blocks: byte 16*(r%32) + 4*(r/32) + j is the
+// scale of row r in the j-th 128-deep K-block of the atom.  Scales are stored in
+// global memory as these atoms, atom (R, G) covering rows [128R, 128R+128) and
+// K-blocks [4G, 4G+4), at byte offset (R * groups + G) * 512.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace zc {
+
+constexpr int kAtomBytes = 512;
+
+// E8M0 code of a block's largest magnitude (amax >= 0, finite).
+__device__ __forceinline__ uint32_t e8m0_code(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  if (b == 0u) return 127u;
+  const int ef = (int)(b >> 23);
+  if (ef == 0) return 0u;  // subnormal block maximum: the smallest scale suffices
+  const int k = ef - 127;  // amax in [2^k, 2^(k+1))
+  // 448 = 1.75 * 2^8: amax <= 1.75 * 2^k  <=>  mantissa fraction <= 0.75
+  const int E = ((b & 0x7FFFFFu) <= 0x600000u) ? k - 8 : k - 7;
+  const int c = E + 127;
+  return (uint32_t)(c < 0 ? 0 : (c > 254 ? 254 : c));
+}
+
+// 2^(127 - code) as fp32 (code <= 253).
+__device__ __forceinline__ float e8m0_inverse(uint32_t code) { return __uint_as_float((254u - code) << 23); }
+
+// Four E4M3 codes packed little-endian (byte i = code of v_i).
+__device__ __forceinline__ uint32_t pack_e4m3x4(float v0, float v1, float v2, float v3) {
+  uint16_t lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(v1), "f"(v0));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(v3), "f"(v2));
+  return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+// Byte offset of (row, K-block) in a scale-atom array with `groups` atoms per 128 rows.
+__host__ __device__ __forceinline__ int64_t atom_offset(int64_t row, int kb, int groups) {
+  const int64_t R = row >> 7;
+  const int r = (int)(row & 127);
+  return (R * groups + (kb >> 2)) * kAtomBytes + 16 * (r & 31) + 4 * (r >> 5) + (kb & 3);
+}
+
+}  // namespace zc

@@ -26,8 +26,10 @@ cudaError_t launch_route_scatter(const int32_t* idx, int T, int k, int N, int E,
                                  int32_t* perm, int32_t* pos, cudaStream_t s);
 cudaError_t launch_gather_rows(const void* x, int row_bytes, const int32_t* perm, int k, const int32_t* scal,
                                void* xperm, int sms, cudaStream_t s);
+// offsets / mb_off non-null: Y rows are padded (FP8 layers), see k_combine.
 cudaError_t launch_combine(int bf16, const void* x, const void* Y, const int32_t* idx, const float* gate,
-                           const int32_t* pos, int T, int k, int N, int d, void* y, int sms, cudaStream_t s);
+                           const int32_t* pos, int T, int k, int N, int d, void* y, int sms, cudaStream_t s,
+                           const int32_t* offsets = nullptr, const int32_t* mb_off = nullptr);
 cudaError_t launch_selftest_wait(int* err, uint64_t limit_ns, cudaStream_t s);
 cudaError_t launch_single_group(int32_t* row_off, int32_t* mb_off, int T, cudaStream_t s);
 cudaError_t launch_update_bias(int64_t* counts, int64_t* tokens, int N, int Z, int k, float kp, float ki, float kd,
@@ -56,6 +58,44 @@ int tc_smem_bytes();
 int tc_block_n(int mode);
 cudaError_t launch_tc_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                            const TcArgs& args, int grid, cudaStream_t s);
+
+// ------------------------------------------------------------- block-scaled FP8 (fp8_quant.cu, gemm_fp8.cu)
+// atom_groups > 0: scales written as scale atoms with that many atoms per 128
+// rows; 0: plain [row blocks, cols/128].
+cudaError_t launch_quant_rows(int bf16, const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
+                              int atom_groups, int sms, cudaStream_t s);
+cudaError_t launch_quant_tiles(int bf16, const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
+                               int atom_groups, cudaStream_t s);
+cudaError_t launch_gather_quant(const void* x, int d, const int32_t* perm, const int32_t* idx, int k,
+                                const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x8,
+                                uint8_t* sx, int groups, int sms, cudaStream_t s);
+
+cudaError_t launch_unpad_rows(const void* ypad, int row_bytes, const int32_t* perm, const int32_t* idx,
+                              const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, void* out, int sms,
+                              cudaStream_t s);
+
+struct Fp8Args {
+  int K;                   // reduction length (a multiple of 128)
+  int n_out;               // valid output columns
+  int nblocks;             // output column tiles
+  int ngroups;             // experts
+  const int32_t* row_off;  // [ngroups+1] pair offsets (the counts' exclusive scan)
+  const int32_t* mb_off;   // [ngroups+1] row-block offsets: expert g's rows start at padded row 128 mb_off[g]
+  int b_rows_per_group;    // rows of the B tensor per expert (gate/up: inter, down: d)
+  const uint8_t* sfa;      // A scale atoms
+  const uint8_t* sfb0;     // B scale atoms (gate/up: W_g, down: W_d)
+  const uint8_t* sfb1;     // gate/up: W_u scale atoms
+  int groups_k;            // scale atoms per 128 rows of A and B = ceil(K / 512)
+  void* out;               // gate/up: H codes [padded rows, n_out]; down: Y bf16 [padded rows, n_out]
+  int64_t ldo;             // its row stride (elements)
+  uint8_t* out_sf;         // gate/up: H scale atoms, out_groups per 128 rows
+  int out_groups;
+  int* err;                // device error word (bounded waits)
+};
+int fp8_smem_bytes();
+int fp8_block_n(int mode);
+cudaError_t launch_fp8_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                            const Fp8Args& args, int grid, cudaStream_t s);
 
 // ------------------------------------------------------------- fp32 CUDA-core GEMM (gemm_simt.cu)
 struct SimtArgs {

@@ -24,6 +24,7 @@
 #include <vector>
 
 #include "../../include/zcmoe.h"
+#include "zc_fp8.cuh"
 #include "zc_internal.h"
 
 namespace {
@@ -81,20 +82,24 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [outer, inner] (inner contiguous), box [box_outer, 64], 128-byte swizzle.
-int make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+// 2-D tensor [outer, inner] (inner contiguous) of bf16 (esz 2) or FP8 codes
+// (esz 1); box [box_outer, 128 bytes], 128-byte swizzle.
+int make_tmap_esz(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer, int esz) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(ZCMOE_ECUDA, "cuTensorMapEncodeTiled entry point unavailable");
   if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0) return fail(ZCMOE_EINVAL, "tensor base not 16-byte aligned");
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {64, box_outer};
+  cuuint64_t strides[1] = {inner * (uint64_t)esz};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esz), box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(tm, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(ZCMOE_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return ZCMOE_OK;
+}
+int make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+  return make_tmap_esz(tm, base, inner, outer, box_outer, 2);
 }
 
 template <typename T>
@@ -140,6 +145,13 @@ struct zcmoe_s {
   std::vector<cudaEvent_t>* events;
   // tensor maps of fixed buffers
   CUtensorMap tm_wr, tm_wg, tm_wu, tm_wd, tm_xperm, tm_h;
+  // ZCMOE_FP8: expert weights as E4M3 codes + scale atoms (owned), padded
+  // activation operands (expert e's pairs from row 128 mb_off[e] on) with their
+  // scale atoms, padded expert outputs; atoms per 128 rows: gd (K = d), gi (K = inter)
+  int fp8, gd, gi;
+  uint8_t *w8g, *w8u, *w8d, *sfg, *sfu, *sfd, *x8, *sx, *h8, *sh;
+  void* ypad;
+  CUtensorMap tm8_wg, tm8_wu, tm8_wd, tm8_x, tm8_h;
   bool alive;
 };
 
@@ -147,7 +159,8 @@ static void release(zcmoe_s* h) {
   void* ptrs[] = {h->bias,  h->b0,     h->offset, h->eta,   h->integ,   h->eprev,  h->acc_counts,
                   h->err,   h->logits, h->gate,   h->idx,   h->pos,     h->counts, h->offsets,
                   h->mb_off, h->scal,  h->chunk,  h->perm,  h->xperm,   h->H,      h->Y,
-                  h->stage_x, h->stage_x2, h->stage_y};
+                  h->stage_x, h->stage_x2, h->stage_y, h->w8g, h->w8u, h->w8d, h->sfg, h->sfu, h->sfd,
+                  h->x8, h->sx, h->h8, h->sh, h->ypad};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (int i = 0; i < 2; ++i) {
@@ -248,7 +261,10 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
   if (cfg->d < 64 || cfg->d % 64 || cfg->inter < 64 || cfg->inter % 64)
     return fail(ZCMOE_EINVAL, "d and inter must be positive multiples of 64");
   if (cfg->max_tokens < 1 || cfg->max_tokens > (1 << 20)) return fail(ZCMOE_EINVAL, "need 1 <= max_tokens <= 2^20");
-  if (cfg->dtype != ZCMOE_F32 && cfg->dtype != ZCMOE_BF16) return fail(ZCMOE_EINVAL, "unknown dtype");
+  if (cfg->dtype != ZCMOE_F32 && cfg->dtype != ZCMOE_BF16 && cfg->dtype != ZCMOE_FP8)
+    return fail(ZCMOE_EINVAL, "unknown dtype");
+  if (cfg->dtype == ZCMOE_FP8 && (cfg->d % 512 || cfg->inter % 128))
+    return fail(ZCMOE_EINVAL, "FP8 experts need d a multiple of 512 and inter a multiple of 128");
   if (!w->w_router || !w->w_gate || !w->w_up || !w->w_down) return fail(ZCMOE_EINVAL, "a weight pointer is NULL");
   const void* wp[4] = {w->w_router, w->w_gate, w->w_up, w->w_down};
   for (const void* p : wp)
@@ -261,8 +277,9 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
   ZC_CUDA(cudaGetDeviceProperties(&prop, dev));
   if (prop.major != 10) return fail(ZCMOE_EUNSUPPORTED, "device %d is sm_%d%d; this library targets sm_100a", dev,
                                     prop.major, prop.minor);
-  if (cfg->dtype == ZCMOE_BF16 &&
-      prop.sharedMemPerBlockOptin < (size_t)zc::tc_smem_bytes())
+  if (cfg->dtype != ZCMOE_F32 &&
+      prop.sharedMemPerBlockOptin < (size_t)(zc::tc_smem_bytes() > zc::fp8_smem_bytes() ? zc::tc_smem_bytes()
+                                                                                         : zc::fp8_smem_bytes()))
     return fail(ZCMOE_EUNSUPPORTED, "not enough shared memory per block");
 
   zcmoe_s* h = new (std::nothrow) zcmoe_s();
@@ -278,7 +295,8 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
   h->d = cfg->d;
   h->inter = cfg->inter;
   h->max_T = cfg->max_tokens;
-  h->bf16 = cfg->dtype == ZCMOE_BF16;
+  h->bf16 = cfg->dtype != ZCMOE_F32;  // ZCMOE_FP8 layers are bf16 at the interface
+  h->fp8 = cfg->dtype == ZCMOE_FP8;
   h->sms = prop.multiProcessorCount;
   h->device = dev;
   h->w = *w;
@@ -310,12 +328,32 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
   ZC_ALLOC(h->perm, (size_t)h->max_pairs);
   {
     uint8_t *xp = nullptr, *hh = nullptr, *yy = nullptr;
-    ZC_ALLOC(xp, (size_t)h->max_pairs * h->d * esz);
-    ZC_ALLOC(hh, (size_t)h->max_pairs * h->inter * esz);
-    ZC_ALLOC(yy, (size_t)h->max_pairs * h->d * esz);
+    // FP8 layers use the padded FP8 operands below instead
+    ZC_ALLOC(xp, h->fp8 ? 0 : (size_t)h->max_pairs * h->d * esz);
+    ZC_ALLOC(hh, h->fp8 ? 0 : (size_t)h->max_pairs * h->inter * esz);
+    ZC_ALLOC(yy, h->fp8 ? 0 : (size_t)h->max_pairs * h->d * esz);
     h->xperm = xp;
     h->H = hh;
     h->Y = yy;
+  }
+  if (h->fp8) {
+    const size_t prow = (size_t)h->max_mblocks * zc::kBM;  // padded rows
+    h->gd = (h->d / 128 + 3) / 4;
+    h->gi = (h->inter / 128 + 3) / 4;
+    const size_t wn = (size_t)N * h->inter * h->d;
+    ZC_ALLOC(h->w8g, wn);
+    ZC_ALLOC(h->w8u, wn);
+    ZC_ALLOC(h->w8d, wn);
+    ZC_ALLOC(h->sfg, (size_t)N * (h->inter / 128) * h->gd * zc::kAtomBytes);
+    ZC_ALLOC(h->sfu, (size_t)N * (h->inter / 128) * h->gd * zc::kAtomBytes);
+    ZC_ALLOC(h->sfd, (size_t)N * (h->d / 128) * h->gi * zc::kAtomBytes);
+    ZC_ALLOC(h->x8, prow * h->d);
+    ZC_ALLOC(h->sx, (size_t)h->max_mblocks * h->gd * zc::kAtomBytes);
+    ZC_ALLOC(h->h8, prow * h->inter);
+    ZC_ALLOC(h->sh, (size_t)h->max_mblocks * h->gi * zc::kAtomBytes);
+    uint8_t* yp = nullptr;
+    ZC_ALLOC(yp, prow * h->d * 2);
+    h->ypad = yp;
   }
 #undef ZC_ALLOC
   if (rc != ZCMOE_OK) {
@@ -344,8 +382,21 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
     if (e == cudaSuccess) e = cudaMemset(h->eprev, 0, E * sizeof(float));
     if (e == cudaSuccess) e = cudaMemset(h->acc_counts, 0, (E + 1) * sizeof(int64_t));
     if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int));
-    if (e == cudaSuccess) e = cudaMemset(h->xperm, 0, (size_t)h->max_pairs * h->d * esz);
-    if (e == cudaSuccess) e = cudaMemset(h->H, 0, (size_t)h->max_pairs * h->inter * esz);
+    if (e == cudaSuccess && !h->fp8) e = cudaMemset(h->xperm, 0, (size_t)h->max_pairs * h->d * esz);
+    if (e == cudaSuccess && !h->fp8) e = cudaMemset(h->H, 0, (size_t)h->max_pairs * h->inter * esz);
+    if (h->fp8) {
+      // padded operand rows that no pair fills read as zeros
+      const size_t prow = (size_t)h->max_mblocks * zc::kBM;
+      if (e == cudaSuccess) e = cudaMemset(h->x8, 0, prow * h->d);
+      if (e == cudaSuccess) e = cudaMemset(h->h8, 0, prow * h->inter);
+      if (e == cudaSuccess) e = cudaMemset(h->sx, 0, (size_t)h->max_mblocks * h->gd * zc::kAtomBytes);
+      if (e == cudaSuccess) e = cudaMemset(h->sh, 0, (size_t)h->max_mblocks * h->gi * zc::kAtomBytes);
+      // the expert weights, quantized per [128,128] into scale atoms
+      const int64_t ri = (int64_t)N * h->inter, rd = (int64_t)N * h->d;
+      if (e == cudaSuccess) e = zc::launch_quant_tiles(1, w->w_gate, ri, h->d, h->w8g, h->sfg, h->gd, 0);
+      if (e == cudaSuccess) e = zc::launch_quant_tiles(1, w->w_up, ri, h->d, h->w8u, h->sfu, h->gd, 0);
+      if (e == cudaSuccess) e = zc::launch_quant_tiles(1, w->w_down, rd, h->inter, h->w8d, h->sfd, h->gi, 0);
+    }
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     delete[] hb;
     if (e != cudaSuccess) {
@@ -361,8 +412,16 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
     if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wg, w->w_gate, d, (uint64_t)N * inter, 128);
     if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wu, w->w_up, d, (uint64_t)N * inter, 128);
     if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wd, w->w_down, inter, (uint64_t)N * d, 256);
-    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_xperm, h->xperm, d, (uint64_t)h->max_pairs, 128);
-    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_h, h->H, inter, (uint64_t)h->max_pairs, 128);
+    if (rc == ZCMOE_OK && !h->fp8) rc = make_tmap(&h->tm_xperm, h->xperm, d, (uint64_t)h->max_pairs, 128);
+    if (rc == ZCMOE_OK && !h->fp8) rc = make_tmap(&h->tm_h, h->H, inter, (uint64_t)h->max_pairs, 128);
+    if (h->fp8) {
+      const uint64_t prow = (uint64_t)h->max_mblocks * zc::kBM;
+      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_wg, h->w8g, d, (uint64_t)N * inter, 128, 1);
+      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_wu, h->w8u, d, (uint64_t)N * inter, 128, 1);
+      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_wd, h->w8d, inter, (uint64_t)N * d, 256, 1);
+      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_x, h->x8, d, prow, 128, 1);
+      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_h, h->h8, inter, prow, 128, 1);
+    }
     if (rc != ZCMOE_OK) {
       release(h);
       delete h;
@@ -452,13 +511,54 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
                                 h->acc_counts, h->acc_tokens, s));
   ZC_CUDA(zc::launch_route_scatter(h->idx, Ti, k, N, E, h->chunk, h->perm, h->pos, s));
   ZC_CUDA(mark());
-  // 4. gather the FFN pairs' rows
-  ZC_CUDA(zc::launch_gather_rows(x, (int)(d * esz), h->perm, k, h->scal, h->xperm, h->sms, s));
+  // 4. gather the FFN pairs' rows (FP8 layers: quantized per [1,128] into padded rows)
+  if (h->fp8)
+    ZC_CUDA(zc::launch_gather_quant(x, d, h->perm, h->idx, k, h->offsets, h->mb_off, h->scal, h->x8, h->sx, h->gd,
+                                    h->sms, s));
+  else
+    ZC_CUDA(zc::launch_gather_rows(x, (int)(d * esz), h->perm, k, h->scal, h->xperm, h->sms, s));
   ZC_CUDA(mark());
   // 5./6. expert GEMMs
   const int max_mb = (Ti * k + zc::kBM - 1) / zc::kBM + N;
-  // Swapped tiles (weights x tokens) unless fixed otherwise: they need no row padding.
-  if (h->bf16) {
+  if (h->fp8) {
+    zc::Fp8Args a{};
+    a.K = d;
+    a.n_out = inter;
+    a.nblocks = inter / zc::fp8_block_n(zc::kGateUp);
+    a.ngroups = N;
+    a.row_off = h->offsets;
+    a.mb_off = h->mb_off;
+    a.b_rows_per_group = inter;
+    a.sfa = h->sx;
+    a.sfb0 = h->sfg;
+    a.sfb1 = h->sfu;
+    a.groups_k = h->gd;
+    a.out = h->h8;
+    a.ldo = inter;
+    a.out_sf = h->sh;
+    a.out_groups = h->gi;
+    a.err = h->err;
+    int bound = max_mb * a.nblocks;
+    ZC_CUDA(zc::launch_fp8_gemm(zc::kGateUp, h->tm8_x, h->tm8_wg, h->tm8_wu, a, bound < h->sms ? bound : h->sms, s));
+    ZC_CUDA(mark());
+    zc::Fp8Args b{};
+    b.K = inter;
+    b.n_out = d;
+    b.nblocks = (d + zc::fp8_block_n(zc::kDown) - 1) / zc::fp8_block_n(zc::kDown);
+    b.ngroups = N;
+    b.row_off = h->offsets;
+    b.mb_off = h->mb_off;
+    b.b_rows_per_group = d;
+    b.sfa = h->sh;
+    b.sfb0 = h->sfd;
+    b.sfb1 = nullptr;
+    b.groups_k = h->gi;
+    b.out = h->ypad;
+    b.ldo = d;
+    b.err = h->err;
+    bound = max_mb * b.nblocks;
+    ZC_CUDA(zc::launch_fp8_gemm(zc::kDown, h->tm8_h, h->tm8_wd, h->tm8_wd, b, bound < h->sms ? bound : h->sms, s));
+  } else if (h->bf16) {
     zc::TcArgs a{};
     a.K = d;
     a.n_out = inter;
@@ -523,7 +623,11 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     ZC_CUDA(cudaEventRecord(side->dn->ev_join, side->dn->side));
   }
   // 7. combine
-  ZC_CUDA(zc::launch_combine(h->bf16, x, h->Y, h->idx, h->gate, h->pos, Ti, k, N, d, y, h->sms, s));
+  if (h->fp8)
+    ZC_CUDA(zc::launch_combine(1, x, h->ypad, h->idx, h->gate, h->pos, Ti, k, N, d, y, h->sms, s, h->offsets,
+                               h->mb_off));
+  else
+    ZC_CUDA(zc::launch_combine(h->bf16, x, h->Y, h->idx, h->gate, h->pos, Ti, k, N, d, y, h->sms, s));
   ZC_CUDA(mark());
   if (side) ZC_CUDA(cudaStreamWaitEvent(s, side->dn->ev_join, 0));
 
@@ -536,7 +640,10 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
       ZC_CUDA(cudaMemcpyAsync(dbg->offsets, h->offsets, (size_t)(N + 1) * 4, cudaMemcpyDeviceToDevice, s));
     if (dbg->perm) ZC_CUDA(cudaMemcpyAsync(dbg->perm, h->perm, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
     if (dbg->pos) ZC_CUDA(cudaMemcpyAsync(dbg->pos, h->pos, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
-    if (dbg->expert_out)
+    if (dbg->expert_out && h->fp8)
+      ZC_CUDA(zc::launch_unpad_rows(h->ypad, d * 2, h->perm, h->idx, h->offsets, h->mb_off, h->scal, dbg->expert_out,
+                                    h->sms, s));
+    else if (dbg->expert_out)
       ZC_CUDA(cudaMemcpyAsync(dbg->expert_out, h->Y, (size_t)T * k * d * esz, cudaMemcpyDeviceToDevice, s));
   }
   return ZCMOE_OK;
@@ -714,6 +821,28 @@ int zcmoe_destroy(zcmoe_t h) {
   cudaDeviceSynchronize();
   release(h);
   delete h;
+  return ZCMOE_OK;
+}
+
+int zcmoe_quantize_e4m3(const void* src, int32_t src_dtype, int64_t rows, int64_t cols, int32_t block_rows,
+                        uint8_t* codes, uint8_t* scales, cudaStream_t s) {
+  g_err[0] = 0;
+  if (src_dtype != ZCMOE_BF16 && src_dtype != ZCMOE_F32) return fail(ZCMOE_EINVAL, "src_dtype must be BF16 or F32");
+  if (block_rows != 1 && block_rows != 128) return fail(ZCMOE_EINVAL, "block_rows must be 1 or 128");
+  if (rows < 0 || cols <= 0 || cols % 128 || cols > (1 << 30)) return fail(ZCMOE_EINVAL, "bad rows / cols");
+  if (rows == 0) return ZCMOE_OK;
+  if (block_rows == 128 && (rows + 127) / 128 > 65535) return fail(ZCMOE_ERANGE, "too many row blocks");
+  if (!src || !codes || !scales) return fail(ZCMOE_EINVAL, "a pointer is NULL");
+  if ((reinterpret_cast<uintptr_t>(src) & 15u) || (reinterpret_cast<uintptr_t>(codes) & 15u))
+    return fail(ZCMOE_EINVAL, "src and codes must be 16-byte aligned");
+  int dev = 0, sms = 0;
+  ZC_CUDA(cudaGetDevice(&dev));
+  ZC_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const int bf16 = src_dtype == ZCMOE_BF16;
+  if (block_rows == 1)
+    ZC_CUDA(zc::launch_quant_rows(bf16, src, rows, (int)cols, codes, scales, 0, sms, s));
+  else
+    ZC_CUDA(zc::launch_quant_tiles(bf16, src, rows, (int)cols, codes, scales, 0, s));
   return ZCMOE_OK;
 }
 

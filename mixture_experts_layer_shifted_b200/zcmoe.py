@@ -27,12 +27,14 @@ ZCMOE_EUNSUPPORTED = -5
 ZCMOE_ETIMEOUT = -6
 ZCMOE_F32 = 0
 ZCMOE_BF16 = 1
+ZCMOE_FP8 = 2
+_DTYPES = {"f32": ZCMOE_F32, "bf16": ZCMOE_BF16, "fp8": ZCMOE_FP8}
 
 EXPORTED = ("zcmoe_create", "zcmoe_forward", "zcmoe_forward_host", "zcmoe_update_bias", "zcmoe_read_counts",
             "zcmoe_write_counts", "zcmoe_get_state", "zcmoe_set_bias", "zcmoe_check", "zcmoe_profile_begin",
             "zcmoe_profile_end", "zcmoe_selftest_wait", "zcmoe_route_noalloc", "zcmoe_destroy",
             "zcmoe_dense_create", "zcmoe_dense_forward", "zcmoe_forward_overlap", "zcmoe_dense_check",
-            "zcmoe_dense_destroy", "zcmoe_last_error")
+            "zcmoe_dense_destroy", "zcmoe_quantize_e4m3", "zcmoe_last_error")
 STAGES = ("router", "softmax_topk", "integer", "gather", "gate_up", "down", "combine")
 
 
@@ -104,6 +106,7 @@ def lib():
         L.zcmoe_dense_forward.argtypes = [vp, vp, i64, vp, vp]
         L.zcmoe_forward_overlap.argtypes = [vp, vp, vp, vp, i64, vp, vp, vp]
         L.zcmoe_dense_check.argtypes = [vp]
+        L.zcmoe_quantize_e4m3.argtypes = [vp, ctypes.c_int32, i64, i64, ctypes.c_int32, vp, vp, vp]
         L.zcmoe_dense_destroy.argtypes = [vp]
         for f in EXPORTED[:-1]:
             getattr(L, f).restype = i32
@@ -219,6 +222,23 @@ def zcmoe_dense_destroy(h):
     _check(lib().zcmoe_dense_destroy(h), "zcmoe_dense_destroy")
 
 
+def zcmoe_quantize_e4m3(src_ptr, src_dtype, rows, cols, block_rows, codes_ptr, scales_ptr, stream=None):
+    _check(lib().zcmoe_quantize_e4m3(src_ptr, src_dtype, rows, cols, block_rows, codes_ptr, scales_ptr,
+                                     _stream(stream)), "zcmoe_quantize_e4m3")
+
+
+def quantize_e4m3(src, block_rows, stream=None):
+    """(codes uint8 [rows, cols], scales uint8 [ceil(rows/block_rows), cols/128]) of a
+    2-D bf16 or fp32 device tensor (block-scaled FP8, the rule of ZCMOE_FP8 layers)."""
+    rows, cols = src.shape
+    codes = torch.empty((rows, cols), dtype=torch.uint8, device=src.device)
+    scales = torch.empty(((rows + block_rows - 1) // block_rows, cols // 128), dtype=torch.uint8, device=src.device)
+    dt = ZCMOE_BF16 if src.dtype == torch.bfloat16 else ZCMOE_F32
+    zcmoe_quantize_e4m3(ctypes.c_void_p(src.data_ptr()), dt, rows, cols, block_rows, ctypes.c_void_p(codes.data_ptr()),
+                        ctypes.c_void_p(scales.data_ptr()), stream)
+    return codes, scales
+
+
 def zcmoe_last_error() -> str:
     return lib().zcmoe_last_error().decode(errors="replace")
 
@@ -231,7 +251,7 @@ class LayerShape:
     n_zero: int
     inter: int
     top_k: int
-    dtype: str = "bf16"  # "bf16" or "f32"
+    dtype: str = "bf16"  # "bf16", "f32", or "fp8" (bf16 interface, block-scaled FP8 experts)
     routed_scale: float = 1.0
 
     @property
@@ -240,7 +260,7 @@ class LayerShape:
 
     @property
     def torch_dtype(self):
-        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
 
 
 class ZcMoE:
@@ -260,7 +280,7 @@ class ZcMoE:
         self._offset = None if logit_offset is None else np.ascontiguousarray(logit_offset, dtype=np.float32)
         fp = ctypes.POINTER(ctypes.c_float)
         cfg = zcmoe_config(shape.d, shape.n_ffn, shape.n_zero, shape.inter, shape.top_k, max_tokens,
-                           ZCMOE_BF16 if shape.dtype == "bf16" else ZCMOE_F32, shape.routed_scale,
+                           _DTYPES[shape.dtype], shape.routed_scale,
                            None if self._bias0 is None else self._bias0.ctypes.data_as(fp),
                            None if self._offset is None else self._offset.ctypes.data_as(fp))
         w = zcmoe_weights(w_router.data_ptr(), w_gate.data_ptr(), w_up.data_ptr(), w_down.data_ptr())

@@ -454,6 +454,8 @@ ZO_EXPORT void zo_ffn_fp8_f64(const void *xs, int x_dtype, int64_t n, const uint
   double *hv = (double *)malloc(sizeof(double) * (size_t)inter);
   float *h32 = (float *)malloc(sizeof(float) * (size_t)inter);
   const int dkb = d / 128, ikb = inter / 128;
+  double tab[256]; /* code -> value; a scale 2^s multiplies exactly */
+  for (int c = 0; c < 256; ++c) tab[c] = zo_e4m3_decode((uint8_t)c);
   for (int64_t r = 0; r < n; ++r) {
     zo_quantize_blocks((const char *)xs + (size_t)(r * d) * xsz, x_dtype, 1, d, 1, xq, xs_sc);
     for (int c = 0; c < d; ++c) xv[c] = ldexp(zo_e4m3_decode(xq[c]), (int)xs_sc[c / 128] - 127);
@@ -461,9 +463,10 @@ ZO_EXPORT void zo_ffn_fp8_f64(const void *xs, int x_dtype, int64_t n, const uint
     for (int i = 0; i < inter; ++i) {
       double g = 0.0, u = 0.0;
       for (int c = 0; c < d; ++c) {
-        const int sgi = (int)sg[(i / 128) * dkb + c / 128] - 127, sui = (int)su[(i / 128) * dkb + c / 128] - 127;
-        g += ldexp(zo_e4m3_decode(wg[(int64_t)i * d + c]), sgi) * xv[c];
-        u += ldexp(zo_e4m3_decode(wu[(int64_t)i * d + c]), sui) * xv[c];
+        const double sgv = ldexp(1.0, (int)sg[(i / 128) * dkb + c / 128] - 127);
+        const double suv = ldexp(1.0, (int)su[(i / 128) * dkb + c / 128] - 127);
+        g += (tab[wg[(int64_t)i * d + c]] * sgv) * xv[c];
+        u += (tab[wu[(int64_t)i * d + c]] * suv) * xv[c];
       }
       h32[i] = (float)(g / (1.0 + exp(-g)) * u);
     }
@@ -473,7 +476,7 @@ ZO_EXPORT void zo_ffn_fp8_f64(const void *xs, int x_dtype, int64_t n, const uint
     for (int c = 0; c < d; ++c) {
       double acc = 0.0;
       for (int i = 0; i < inter; ++i)
-        acc += ldexp(zo_e4m3_decode(wd[(int64_t)c * inter + i]), (int)sd[(c / 128) * ikb + i / 128] - 127) * hv[i];
+        acc += (tab[wd[(int64_t)c * inter + i]] * ldexp(1.0, (int)sd[(c / 128) * ikb + i / 128] - 127)) * hv[i];
       out[r * d + c] = acc;
     }
   }
