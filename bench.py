@@ -127,11 +127,22 @@ def recorded_traffic(workload, kernel):
 def algorithmic_work(wl, P, distinct):
     """FLOPs and bytes per forward from the realised routing: P FFN pairs and
     `distinct` FFN experts hit.  F = 2 T d E + 6 d inter P;
-    B = distinct * 3 d inter * 2 + E d * 2 + 2 T d * 2 (bf16)."""
-    esz = 2 if wl.dtype == "bf16" else 4
+    B = distinct * 3 d inter * w + E d * 2 + 2 T d * 2 (bf16; expert weights w = 2
+    bytes, or 1 for FP8 experts; fp32 layers 4 throughout)."""
+    esz = 4 if wl.dtype == "f32" else 2
+    wsz = 1 if wl.dtype == "fp8" else esz
     F = 2.0 * wl.T * wl.d * wl.E + 6.0 * wl.d * wl.inter * P
-    B = distinct * 3.0 * wl.d * wl.inter * esz + wl.E * wl.d * esz + 2.0 * wl.T * wl.d * esz
+    B = distinct * 3.0 * wl.d * wl.inter * wsz + wl.E * wl.d * esz + 2.0 * wl.T * wl.d * esz
     return F, B
+
+
+def roofline_ms(wl, F, B, peaks):
+    """max(tensor time, HBM time); FP8 experts at twice the measured bf16 rate (the
+    nominal 4.5 / 2.25 PFLOP/s ratio), the router in bf16."""
+    p = peaks["bf16_tflops_sustained"] * 1e12
+    f_router = 2.0 * wl.T * wl.d * wl.E
+    t_tensor = (f_router / p + (F - f_router) / (2 * p)) if wl.dtype == "fp8" else F / p
+    return 1e3 * max(t_tensor, B / (peaks["hbm_gbs"] * 1e9))
 
 
 def to_host_bits(t):
@@ -155,13 +166,17 @@ def cpu_oracle_sample(wl, weights, x, bias, offset, n_tokens, min_s=10.0):
     idx, gate, _ = oracle.topk(oracle.softmax(l), bias.astype(np.float64), wl.top_k)
     need = sorted({int(e) for e in idx.ravel() if e < wl.n_ffn})
     cache = {e: tuple(to_host_bits(w[e]) for w in weights[1:]) for e in need}
+    efn = None
+    if wl.dtype == "fp8":  # weights quantized once, as the layer does at create
+        q8 = {e: [oracle.quantize_blocks(w, 128) for w in cache[e]] for e in need}
+        efn = lambda e, rows: oracle.ffn_fp8(rows, [c for c, _ in q8[e]], [s_ for _, s_ in q8[e]])
     done = 0
     t0 = time.perf_counter()
     while True:  # the sample is processed again until the time budget is spent
         for t in range(n_tokens):
             l = oracle.router_logits(xs[t:t + 1], wr, offset)
             i1, g1, _ = oracle.topk(oracle.softmax(l), bias.astype(np.float64), wl.top_k)
-            oracle.layer_outputs(xs[t:t + 1], i1, g1, wl.n_ffn, lambda e: cache[e])
+            oracle.layer_outputs(xs[t:t + 1], i1, g1, wl.n_ffn, lambda e: cache[e], expert_fn=efn)
             done += 1
         if time.perf_counter() - t0 > min_s:
             break
@@ -246,6 +261,79 @@ def measure_overlap(wl, layer, x, stream, peaks, reps=10):
             "hidden_frac_of_dense": hidden / ms["dense"], "speedup": ms["sequential"] / ms["overlap"],
             "dense_tflops": tflops, "dense_frac": tflops / peaks["bf16_tflops_sustained"],
             "note": "each variant one replayed CUDA graph, %d replays after 3; same batch for both paths" % reps}
+
+
+def graph_ms(fn, stream, reps=10):
+    """Device time of fn() as one replayed CUDA graph (first call outside the capture)."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) / reps
+
+
+def measure_fp8(layer, weights, x, stream, peaks, bias, offset):
+    """The same layer with block-scaled FP8 experts, on the same weights and batch:
+    forward time against the bf16 layer, the FP8 GEMMs against the FP8 peak, and
+    the decode batch against HBM."""
+    import torch
+    from mixture_experts_layer_shifted_b200 import configs
+    from mixture_experts_layer_shifted_b200.zcmoe import LayerShape, ZcMoE
+
+    out = {}
+    for name, layer_b in (("prefill_560b_fp8", layer), ("decode_560b_fp8", None)):
+        wf = configs.WORKLOADS[name]
+        xf = x if layer_b is not None else configs.device_tokens(wf)
+        shp = LayerShape(wf.d, wf.n_ffn, wf.n_zero, wf.inter, wf.top_k, "fp8")
+        l8 = ZcMoE(shp, *weights, max_tokens=wf.T, init_bias=configs.bias_vector(wf),
+                   logit_offset=configs.logit_offsets(wf))
+        lb = layer_b
+        if lb is None:
+            lb = ZcMoE(LayerShape(wf.d, wf.n_ffn, wf.n_zero, wf.inter, wf.top_k, "bf16"), *weights,
+                       max_tokens=wf.T, init_bias=configs.bias_vector(wf), logit_offset=configs.logit_offsets(wf))
+        y8, yb = torch.empty_like(xf), torch.empty_like(xf)
+        ms8 = graph_ms(lambda: l8.forward(xf, y8), stream)
+        msb = graph_ms(lambda: lb.forward(xf, yb), stream)
+        offs = torch.empty((wf.n_ffn + 1,), dtype=torch.int32, device=xf.device)
+        l8.forward(xf, y8, debug={"offsets": offs})
+        torch.cuda.synchronize()
+        cnt = np.diff(offs.cpu().numpy())
+        P, distinct = int(cnt.sum()), int((cnt > 0).sum())
+        F, B = algorithmic_work(wf, P, distinct)
+        l8.profile_begin()
+        for _ in range(5):
+            l8.forward(xf, y8)
+        st, nf = l8.profile_end()
+        st = {k_: v / nf for k_, v in st.items()}
+        p8 = 2 * peaks["bf16_tflops_sustained"]
+        gu = 4.0 * wf.d * wf.inter * P / (st["gate_up"] * 1e-3) / 1e12
+        dn = 2.0 * wf.d * wf.inter * P / (st["down"] * 1e-3) / 1e12
+        rec = {"tokens_per_s": wf.T / (ms8 * 1e-3), "ms_per_forward": ms8, "bf16_ms_per_forward": msb,
+               "speedup_vs_bf16": msb / ms8, "stage_ms": st,
+               "gate_up": {"tflops": gu, "frac_fp8_peak": gu / p8},
+               "down": {"tflops": dn, "frac_fp8_peak": dn / p8},
+               "layer_roofline_ms": roofline_ms(wf, F, B, peaks), "P": P}
+        if layer_b is None:
+            rec["hbm_gbs"] = B / (ms8 * 1e-3) / 1e9
+            rec["hbm_frac"] = rec["hbm_gbs"] / peaks["hbm_gbs"]
+            lb.close()
+        l8.check()
+        l8.close()
+        out[name] = rec
+    out["peak_note"] = "fp8 dense peak = 2 x measured sustained bf16 (nominal 4.5/2.25 PFLOP/s ratio)"
+    return out
 
 
 def main():
@@ -362,15 +450,20 @@ def main():
     stage_avg = {s: v / nf for s, v in stage_ms.items()}
     gu_ms = stage_avg["gate_up"]
     gu_flops = 4.0 * wl.d * wl.inter * P
-    tensor_peak = peaks["bf16_tflops_sustained"]
+    fp8 = wl.dtype == "fp8"
+    tensor_peak = peaks["bf16_tflops_sustained"] * (2 if fp8 else 1)
     achieved = gu_flops / (gu_ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "grouped gate/up GEMM + SwiGLU (k_tc_gemm<1>)", "achieved": achieved,
-                "peak": tensor_peak, "unit": "TFLOP/s", "frac": achieved / tensor_peak, "traffic": recorded_traffic(wl.name, "gate_up"),
-                "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
+    kname = ("grouped FP8 gate/up GEMM + SwiGLU + quantize (k_fp8_gemm<1>)" if fp8
+             else "grouped gate/up GEMM + SwiGLU (k_tc_gemm<1>)")
+    roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved,
+                "peak": tensor_peak, "unit": "TFLOP/s", "frac": achieved / tensor_peak,
+                "traffic": None if fp8 else recorded_traffic(wl.name, "gate_up"),
+                "peak_kind": (f"fp8 dense = 2 x bf16 dense sustained ({peaks['source']}; nominal 4.5/2.25 ratio)" if fp8
+                              else f"bf16 dense, sustained, {peaks['source']}"),
                 "per_launch": {"flops": gu_flops, "ms": gu_ms, "units": f"{P} FFN (token, expert) pairs x 4 d inter"}}
     fwd_ms = sum(stage_avg.values())
-    t_roof = max(F / (peaks["bf16_tflops_sustained"] * 1e12), B / (peaks["hbm_gbs"] * 1e9))
-    layer_roof = {"forward_ms": fwd_ms, "roofline_ms": 1e3 * t_roof, "frac": 1e3 * t_roof / fwd_ms,
+    t_roof_ms = roofline_ms(wl, F, B, peaks)
+    layer_roof = {"forward_ms": fwd_ms, "roofline_ms": t_roof_ms, "frac": t_roof_ms / fwd_ms,
                   "flops": F, "bytes": B, "stage_ms": stage_avg,
                   "down": {"ms": stage_avg["down"],
                            "tflops": 2.0 * wl.d * wl.inter * P / (stage_avg["down"] * 1e-3) / 1e12}}
@@ -450,6 +543,10 @@ def main():
                           "hbm_gbs": hbm, "hbm_frac": hbm / peaks["hbm_gbs"], "bytes": B2,
                           "P": int(cnt2.sum()), "distinct_experts": int((cnt2 > 0).sum())}
         layer2.close()
+
+    # secondary: the same layer with block-scaled FP8 experts (bf16 headline unchanged)
+    if rank == 0 and ws == 1 and not args.no_secondary and wl.name == "prefill_560b":
+        line["fp8"] = measure_fp8(layer, weights, xs[0], stream, peaks, bias, offset)
 
     # secondary: the dense FFN path run beside the layer (shortcut-connected MoE)
     if rank == 0 and ws == 1 and not args.no_secondary and wl.dense_inter > 0:

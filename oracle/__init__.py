@@ -184,12 +184,12 @@ def layer(x, idx, gate, N, wg, wu, wd):
     return y
 
 
-def layer_outputs(x_rows, idx, gate, N, expert_weights, fp8=False):
+def layer_outputs(x_rows, idx, gate, N, expert_weights, fp8=False, expert_fn=None):
     """fp64 layer output for a few tokens when the expert weights are fetched one
     expert at a time.  ``expert_weights(e) -> (wg, wu, wd)``.  Sums
     g * F_e(x) over the token's FFN slots plus (sum of zero-slot gates) * x.
     fp8: F_e is the block-scaled FP8 expert (ffn_fp8) on weights quantized here
-    per [128,128]."""
+    per [128,128].  expert_fn(e, rows) -> F_e(rows), if given, replaces both."""
     x_rows = np.ascontiguousarray(x_rows)
     n, d = x_rows.shape
     xf = x_rows.astype(np.float64) if x_rows.dtype == np.float32 else \
@@ -205,8 +205,13 @@ def layer_outputs(x_rows, idx, gate, N, expert_weights, fp8=False):
             else:
                 users.setdefault(e, []).append((r, j))
     for e in sorted(users):
-        wg, wu, wd = expert_weights(e)
         rows = [r for r, _ in users[e]]
+        if expert_fn is not None:
+            f = expert_fn(e, x_rows[rows])
+            for i, (r, j) in enumerate(users[e]):
+                y[r] += float(gate[r, j]) * f[i]
+            continue
+        wg, wu, wd = expert_weights(e)
         if fp8:
             q = [quantize_blocks(w, 128) for w in (wg, wu, wd)]
             f = ffn_fp8(x_rows[rows], [c for c, _ in q], [s_ for _, s_ in q])
