@@ -72,6 +72,16 @@ def lib():
         L.zo_quantize_blocks.restype = None
         L.zo_ffn_fp8_f64.argtypes = [vp, i32, i64, U8P, U8P, U8P, U8P, U8P, U8P, i32, i32, F64P]
         L.zo_ffn_fp8_f64.restype = None
+        L.zo_e2m1_encode.argtypes = [f32]
+        L.zo_e2m1_encode.restype = ctypes.c_uint8
+        L.zo_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.zo_e2m1_decode.restype = f64
+        L.zo_mx4_scale.argtypes = [f32]
+        L.zo_mx4_scale.restype = ctypes.c_uint8
+        L.zo_quantize_mx4.argtypes = [vp, i32, i64, i64, U8P, U8P]
+        L.zo_quantize_mx4.restype = None
+        L.zo_ffn_fp4_f64.argtypes = [vp, i32, i64, U8P, U8P, U8P, U8P, U8P, U8P, i32, i32, F64P]
+        L.zo_ffn_fp4_f64.restype = None
         L.zo_ffn_f64.argtypes = [vp, i32, i64, vp, vp, vp, i32, i32, i32, F64P]
         L.zo_ffn_f64.restype = None
         L.zo_layer_f64.argtypes = [vp, i32, i64, I32P, F64P, i32, i32, vp, vp, vp, i32, i32, i32, F64P]
@@ -296,4 +306,53 @@ def ffn_fp8(xs, wq, sq):
     inter = wg.shape[0]
     out = np.empty((n, d), np.float64)
     lib().zo_ffn_fp8_f64(xs.ctypes.data, xd, n, wg, sg, wu, su, wd, sd, d, inter, out)
+    return out
+
+
+# ----------------------------------------------------------------- W4A4 (MXFP4)
+def e2m1_encode(v: float) -> int:
+    return int(lib().zo_e2m1_encode(float(v)))
+
+
+def e2m1_decode(code: int) -> float:
+    return float(lib().zo_e2m1_decode(int(code)))
+
+
+def mx4_scale(amax: float) -> int:
+    """E8M0 code of the smallest power of two s with amax <= 6 s (127 for amax 0)."""
+    return int(lib().zo_mx4_scale(float(amax)))
+
+
+def quantize_mx4(src):
+    """(codes [rows, cols/2] uint8, two per byte with the even element low; scales
+    [rows, cols/32] uint8) of a 2-D fp32 array or bf16 bit array."""
+    src, dt = _arr(src)
+    rows, cols = src.shape
+    if cols % 32:
+        raise ValueError("cols must be a multiple of 32")
+    codes = np.empty((rows, cols // 2), np.uint8)
+    scales = np.empty((rows, cols // 32), np.uint8)
+    lib().zo_quantize_mx4(src.ctypes.data, dt, rows, cols, codes, scales)
+    return codes, scales
+
+
+def dequantize_mx4(codes, scales):
+    table = np.array([e2m1_decode(c) for c in range(16)], np.float64)
+    rows = codes.shape[0]
+    nib = np.empty((rows, codes.shape[1] * 2), np.uint8)
+    nib[:, 0::2] = codes & 0xF
+    nib[:, 1::2] = codes >> 4
+    return np.ldexp(table[nib], np.repeat(scales.astype(np.int64) - 127, 32, 1))
+
+
+def ffn_fp4(xs, wq, sq):
+    """fp64 SwiGLU expert on MXFP4 operands: xs [n, d] quantized per [1,32] inside;
+    wq = (wg, wu, wd) packed codes, sq = their [1,32] scales."""
+    xs, xd = _arr(xs)
+    n, d = xs.shape
+    wg, wu, wd = (np.ascontiguousarray(w, np.uint8) for w in wq)
+    sg, su, sd = (np.ascontiguousarray(s_, np.uint8) for s_ in sq)
+    inter = wg.shape[0]
+    out = np.empty((n, d), np.float64)
+    lib().zo_ffn_fp4_f64(xs.ctypes.data, xd, n, wg, sg, wu, su, wd, sd, d, inter, out)
     return out

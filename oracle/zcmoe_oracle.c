@@ -488,3 +488,133 @@ ZO_EXPORT void zo_ffn_fp8_f64(const void *xs, int x_dtype, int64_t n, const uint
   free(hv);
   free(h32);
 }
+
+/* ------------------------------------------------------------------------- */
+/* W4A4 experts.  A LongCat-Flash news page (gate.com post) says the model    */
+/* serves with W4A4: expert weights and activations quantized to 4 bits.      */
+/* The format is not given; reading: MXFP4 (OCP microscaling) -- E2M1 codes    */
+/* (1 sign, 2 exponent bits with bias 1, 1 mantissa bit: 0, 0.5, 1, 1.5, 2, 3, */
+/* 4, 6), round to nearest with ties to even, saturating at 6; one E8M0 scale  */
+/* per 32 consecutive elements along the reduction dimension (every row of x, */
+/* H and each weight matrix), the smallest 2^E with amax <= 6 * 2^E (code      */
+/* clamped to [0, 254], 127 for an all-zero block).  Two codes per byte, the   */
+/* even element in the low nibble.  Pinned in tests/test_oracle_pins.py.      */
+/* ------------------------------------------------------------------------- */
+
+ZO_EXPORT double zo_e2m1_decode(uint8_t c) {
+  const int s = (c >> 3) & 1, E = (c >> 1) & 3, M = c & 1;
+  const double v = (E == 0) ? 0.5 * M : ldexp(1.0 + 0.5 * M, E - 1);
+  return s ? -v : v;
+}
+
+ZO_EXPORT uint8_t zo_e2m1_encode(float v) {
+  const uint8_t sign = signbit(v) ? 0x8 : 0x0;
+  const double a = fabs((double)v);
+  if (!(a < 6.0)) return sign | 0x7; /* saturate (NaN included) */
+  double q;                          /* spacing of representable magnitudes around a */
+  if (a < 1.0) {
+    q = 0.5;
+  } else {
+    int e;
+    frexp(a, &e); /* a in [2^(e-1), 2^e) */
+    q = ldexp(1.0, e - 1 - 1);
+  }
+  const double n = a / q;
+  double r = floor(n);
+  const double frac = n - r;
+  if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) == 1.0)) r += 1.0;
+  const double val = r * q;
+  if (val < 1.0) return sign | (uint8_t)(val / 0.5); /* 0 or 0.5 */
+  int ee;
+  const double m = frexp(val, &ee); /* val = m * 2^ee, m in [0.5, 1) */
+  const int E = ee - 1 + 1;
+  const int M = (int)((2.0 * m - 1.0) * 2.0);
+  return sign | (uint8_t)(E << 1) | (uint8_t)M;
+}
+
+ZO_EXPORT uint8_t zo_mx4_scale(float amax) {
+  if (!(amax > 0.0f)) return 127;
+  int e;
+  frexp((double)amax, &e);
+  const int k = e - 1; /* amax in [2^k, 2^(k+1)) */
+  const int E = ((double)amax <= 1.5 * ldexp(1.0, k)) ? k - 2 : k - 1; /* 6 = 1.5 * 2^2 */
+  int code = E + 127;
+  if (code < 0) code = 0;
+  if (code > 254) code = 254;
+  return (uint8_t)code;
+}
+
+/* src [rows, cols] (dtype 0 fp32, 1 bf16 bits), cols a multiple of 32.
+   codes [rows, cols/2] (two per byte, even element low); scales [rows, cols/32]. */
+ZO_EXPORT void zo_quantize_mx4(const void *src, int dtype, int64_t rows, int64_t cols, uint8_t *codes,
+                               uint8_t *scales) {
+  const int64_t nb = cols / 32;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < nb; ++b) {
+      double amax = 0.0;
+      for (int64_t c = b * 32; c < b * 32 + 32; ++c) {
+        const double a = fabs(elem(src, dtype, r * cols + c));
+        if (a > amax) amax = a;
+      }
+      const uint8_t sc = zo_mx4_scale((float)amax);
+      scales[r * nb + b] = sc;
+      const double inv = ldexp(1.0, 127 - (int)sc);
+      for (int64_t c = b * 32; c < b * 32 + 32; c += 2) {
+        const uint8_t lo = zo_e2m1_encode((float)(elem(src, dtype, r * cols + c) * inv));
+        const uint8_t hi = zo_e2m1_encode((float)(elem(src, dtype, r * cols + c + 1) * inv));
+        codes[r * (cols / 2) + c / 2] = (uint8_t)(lo | (hi << 4));
+      }
+    }
+}
+
+static double mx4_value(const uint8_t *codes, const uint8_t *scales, int64_t cols, int64_t r, int64_t c,
+                        const double *tab) {
+  const uint8_t byte = codes[r * (cols / 2) + c / 2];
+  const uint8_t code = (c & 1) ? (byte >> 4) : (byte & 0xF);
+  return tab[code] * ldexp(1.0, (int)scales[r * (cols / 32) + c / 32] - 127);
+}
+
+/* FFN expert on MXFP4 operands, fp64 arithmetic on the dequantized values.
+   Each row of xs is quantized per [1,32] here; wg, wu [inter, d] and wd [d, inter]
+   come as codes + scales ([1,32] along each row).  h = silu(g) * u is rounded to
+   fp32 and quantized per [1,32] before the down projection (the kernel's
+   precision, as for the FP8 expert).  out [n, d] fp64. */
+ZO_EXPORT void zo_ffn_fp4_f64(const void *xs, int x_dtype, int64_t n, const uint8_t *wg, const uint8_t *sg,
+                              const uint8_t *wu, const uint8_t *su, const uint8_t *wd, const uint8_t *sd, int d,
+                              int inter, double *out) {
+  const size_t xsz = (x_dtype == 1) ? 2 : 4;
+  double tab[16];
+  for (int c = 0; c < 16; ++c) tab[c] = zo_e2m1_decode((uint8_t)c);
+  uint8_t *xq = (uint8_t *)malloc((size_t)d / 2), *xsc = (uint8_t *)malloc((size_t)d / 32);
+  uint8_t *hq = (uint8_t *)malloc((size_t)inter / 2), *hsc = (uint8_t *)malloc((size_t)inter / 32);
+  double *xv = (double *)malloc(sizeof(double) * (size_t)d), *hv = (double *)malloc(sizeof(double) * (size_t)inter);
+  float *h32 = (float *)malloc(sizeof(float) * (size_t)inter);
+  for (int64_t r = 0; r < n; ++r) {
+    zo_quantize_mx4((const char *)xs + (size_t)(r * d) * xsz, x_dtype, 1, d, xq, xsc);
+    for (int c = 0; c < d; ++c) xv[c] = mx4_value(xq, xsc, d, 0, c, tab);
+#pragma omp parallel for schedule(static)
+    for (int i = 0; i < inter; ++i) {
+      double g = 0.0, u = 0.0;
+      for (int c = 0; c < d; ++c) {
+        g += mx4_value(wg, sg, d, i, c, tab) * xv[c];
+        u += mx4_value(wu, su, d, i, c, tab) * xv[c];
+      }
+      h32[i] = (float)(g / (1.0 + exp(-g)) * u);
+    }
+    zo_quantize_mx4(h32, 0, 1, inter, hq, hsc);
+    for (int i = 0; i < inter; ++i) hv[i] = mx4_value(hq, hsc, inter, 0, i, tab);
+#pragma omp parallel for schedule(static)
+    for (int c = 0; c < d; ++c) {
+      double acc = 0.0;
+      for (int i = 0; i < inter; ++i) acc += mx4_value(wd, sd, inter, c, i, tab) * hv[i];
+      out[r * d + c] = acc;
+    }
+  }
+  free(xq);
+  free(xsc);
+  free(hq);
+  free(hsc);
+  free(xv);
+  free(hv);
+  free(h32);
+}

@@ -483,3 +483,92 @@ def test_ffn_fp8_is_close_to_the_unquantized_expert():
     rel = np.abs(y8 - y).max(axis=1) / np.abs(y).max(axis=1)
     assert rel.max() < 0.08, rel
     assert rel.max() > 1e-4          # it is a lossy path
+
+
+# ---------------------------------------------------------------- W4A4 (MXFP4, oracle only)
+
+# E2M1 magnitudes of the OCP Microscaling Formats (MX) v1.0 specification (FP4 E2M1 element).
+E2M1_VALUES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_e2m1_decode_is_the_mx_value_set():
+    got = [oracle.e2m1_decode(c) for c in range(16)]
+    assert got[:8] == E2M1_VALUES
+    assert [-v for v in got[8:]] == E2M1_VALUES and np.signbit(got[8])
+    assert all(oracle.e2m1_encode(got[c]) == c for c in range(16))   # round trip
+
+
+def test_e2m1_encode_against_brute_force():
+    """Nearest representable magnitude, ties to the even code (mantissa bit 0), saturating at 6."""
+    mags = np.array(E2M1_VALUES)
+    rng = np.random.default_rng(21)
+    vals = np.concatenate([np.arange(-7.0, 7.0, 1 / 64), (mags[1:] + mags[:-1]) / 2, rng.uniform(-8, 8, 3000)])
+    for v in vals.astype(np.float32):
+        a = min(abs(float(v)), 6.0)
+        dist = np.abs(mags - a)
+        best = np.flatnonzero(dist == dist.min())
+        code = int(best[0]) if len(best) == 1 else int([b for b in best if b % 2 == 0][0])
+        want = code | (8 if np.signbit(v) else 0)
+        assert oracle.e2m1_encode(v) == want, (float(v), oracle.e2m1_encode(v), want)
+
+
+def test_mx4_scale_is_the_smallest_sufficient_power_of_two():
+    rng = np.random.default_rng(22)
+    amax = (rng.uniform(0.5, 1.0, 3000) * np.exp2(rng.integers(-100, 100, 3000))).astype(np.float32)
+    for a in amax:
+        c = oracle.mx4_scale(float(a))
+        s = 2.0 ** (c - 127)
+        assert a / s <= 6.0 < a / (s / 2), (a, c)
+    assert oracle.mx4_scale(0.0) == 127 and oracle.mx4_scale(6.0) == 127 and oracle.mx4_scale(1.0) == 125
+    assert oracle.mx4_scale(np.nextafter(np.float32(6), np.float32(10))) == 128
+
+
+def test_quantize_mx4_bound_and_packing():
+    rng = np.random.default_rng(23)
+    x = (rng.standard_normal((5, 96)) * np.exp2(rng.integers(-8, 8, (5, 1)))).astype(np.float32)
+    codes, scales = oracle.quantize_mx4(x)
+    assert codes.shape == (5, 48) and scales.shape == (5, 3)
+    deq = oracle.dequantize_mx4(codes, scales)
+    s = np.ldexp(1.0, np.repeat(scales.astype(np.int64) - 127, 32, 1))
+    v = x.astype(np.float64) / s
+    assert np.abs(v).max() <= 6.0
+    spacing = np.where(np.abs(v) < 1.0, 0.5, np.exp2(np.floor(np.log2(np.maximum(np.abs(v), 1.0))) - 1))
+    assert np.all(np.abs(v - deq / s) <= spacing / 2)
+    # even element in the low nibble
+    y = np.zeros((1, 32), np.float32)
+    y[0, :2] = [6.0, 1.0]
+    c, sc = oracle.quantize_mx4(y)
+    assert sc[0, 0] == 127 and c[0, 0] == (0x7 | (0x2 << 4))
+
+
+def test_ffn_fp4_lossless_closed_form():
+    """As the FP8 closed form: g = 64, u = 1 on one active unit, every value exactly
+    representable after MXFP4 quantization, so y = 64 * W_d[:, 0] exactly."""
+    d = inter = 64
+    x = np.zeros((1, d), np.float32)
+    x[0, 0] = 1.0
+    wg = np.zeros((inter, d), np.float32)
+    wu = np.zeros((inter, d), np.float32)
+    wg[0, 0], wu[0, 0] = 64.0, 1.0
+    wd = np.zeros((d, inter), np.float32)
+    wd[:, 0] = ((np.arange(d) % 8) - 4) * 0.25
+    q = [oracle.quantize_mx4(w) for w in (wg, wu, wd)]
+    for (c, s_), w in zip(q, (wg, wu, wd)):
+        assert np.array_equal(oracle.dequantize_mx4(c, s_), w)
+    y = oracle.ffn_fp4(x, [c for c, _ in q], [s_ for _, s_ in q])
+    assert np.array_equal(y[0], 64.0 * wd[:, 0].astype(np.float64))
+    y_swapped = oracle.ffn_fp4(x, [q[1][0], q[0][0], q[2][0]], [q[1][1], q[0][1], q[2][1]])
+    assert not np.allclose(y_swapped, y)
+
+
+def test_ffn_fp4_is_close_to_the_unquantized_expert():
+    rng = np.random.default_rng(24)
+    d, inter = 256, 384
+    x = rng.standard_normal((4, d)).astype(np.float32)
+    wg, wu = (rng.standard_normal((inter, d)) * 0.06).astype(np.float32), (rng.standard_normal((inter, d)) * 0.06).astype(np.float32)
+    wd = (rng.standard_normal((d, inter)) * 0.05).astype(np.float32)
+    q = [oracle.quantize_mx4(w) for w in (wg, wu, wd)]
+    y4 = oracle.ffn_fp4(x, [c for c, _ in q], [s_ for _, s_ in q])
+    y = oracle.ffn(x, wg, wu, wd)
+    rel = np.abs(y4 - y).max(axis=1) / np.abs(y).max(axis=1)
+    assert 1e-3 < rel.max() < 0.35, rel
