@@ -52,7 +52,7 @@ extern "C" {
 
 typedef struct zcmoe_s *zcmoe_t;
 
-typedef enum { ZCMOE_F32 = 0, ZCMOE_BF16 = 1, ZCMOE_FP8 = 2 } zcmoe_dtype;
+typedef enum { ZCMOE_F32 = 0, ZCMOE_BF16 = 1, ZCMOE_FP8 = 2, ZCMOE_FP4 = 3 } zcmoe_dtype;
 
 /* Layer shape and routing constants.  Sizes are element counts.
  * Limits: 1 <= n_ffn, 0 <= n_zero, E = n_ffn + n_zero <= 1024, 1 <= top_k <= min(E, 32),
@@ -69,7 +69,13 @@ typedef enum { ZCMOE_F32 = 0, ZCMOE_BF16 = 1, ZCMOE_FP8 = 2 } zcmoe_dtype;
  *                      quantized per [1,128] on the way into the gate/up GEMM and
  *                      silu(g)*u per [1,128] before the down GEMM; the router, the
  *                      combine and y stay bf16.  Needs d a multiple of 512 and inter
- *                      a multiple of 128. */
+ *                      a multiple of 128;
+ *        ZCMOE_FP4  -> as ZCMOE_FP8 with W4A4 experts (a LongCat-Flash news page,
+ *                      gate.com post: expert weights and activations in 4 bits; the
+ *                      format is not named): MXFP4, E2M1 codes with one E8M0 scale
+ *                      (the smallest 2^E with block max <= 6 * 2^E) per 32 elements
+ *                      along the reduction dimension of x, silu(g)*u and every weight
+ *                      row.  Needs d a multiple of 512 and inter a multiple of 256. */
 typedef struct {
   int32_t d;            /* hidden size                                   */
   int32_t n_ffn;        /* N, FFN experts                                */
@@ -106,7 +112,7 @@ typedef struct {
  * counts [E] int32, offsets [N+1] int32 (exclusive scan of FFN counts; offsets[N] = P),
  * perm [T*k] int32 (first P entries valid: FFN pairs t*k+j ordered by expert then
  * token), pos [T, k] int32 (row of pair (t,j) in the permuted order, -1 for zero experts),
- * expert_out [T*k, d] config dtype, bf16 for ZCMOE_FP8 (first P rows valid: the FFN expert outputs F_e(x_t),
+ * expert_out [T*k, d] config dtype, bf16 for ZCMOE_FP8 / ZCMOE_FP4 (first P rows valid: the FFN expert outputs F_e(x_t),
  * one row per pair in the permuted order, before gating). */
 typedef struct {
   float *logits;
@@ -233,6 +239,18 @@ ZCMOE_API int zcmoe_destroy(zcmoe_t h);
  *   uint8 device (E8M0 bytes).  Asynchronous on `stream`. */
 ZCMOE_API int zcmoe_quantize_e4m3(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, int32_t block_rows,
                                   uint8_t *codes, uint8_t *scales, cudaStream_t stream);
+
+/* MXFP4 quantization, the rule ZCMOE_FP4 layers use: E2M1 codes (0, 0.5, 1, 1.5, 2,
+ * 3, 4, 6), round to nearest even, saturating at 6; one E8M0 scale per 32
+ * consecutive elements of a row, the smallest power of two 2^E with the block's
+ * largest magnitude <= 6 * 2^E (E + 127 clamped to [0, 254]; 2^0 for an all-zero
+ * block).  No handle needed.
+ *   src [rows, cols] device, ZCMOE_BF16 or ZCMOE_F32, 16-byte aligned; cols a
+ *   positive multiple of 256; codes [rows, cols / 2] uint8 device, two codes per
+ *   byte with the even element in the low nibble; scales [rows, cols / 32] uint8
+ *   device.  Asynchronous on `stream`. */
+ZCMOE_API int zcmoe_quantize_mx4(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, uint8_t *codes,
+                                 uint8_t *scales, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * Dense FFN path and the shortcut-connected overlap (ScMoE).

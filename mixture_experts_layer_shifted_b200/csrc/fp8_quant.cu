@@ -127,6 +127,88 @@ __global__ void __launch_bounds__(256) k_gather_quant(const __nv_bfloat16* __res
   }
 }
 
+// ---------------------------------------------------------------- MXFP4 ([1,32] blocks)
+// eight consecutive elements (16- or 32-byte aligned)
+__device__ __forceinline__ void ld8(const __nv_bfloat16* p, float* v) {
+  const uint4 r = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void ld8(const float* p, float* v) {
+  ld4(p, v);
+  ld4(p + 4, v + 4);
+}
+
+// The eight values of one lane, its 32-element block spread over four lanes:
+// the lane's packed codes (x) and the block's scale code (y, shared by the four lanes).
+__device__ __forceinline__ uint2 quant8_mx4(const float* v) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  const uint32_t code = mx4_code(a);
+  return make_uint2(pack_e2m1x8(v, e8m0_inverse(code)), code);
+}
+
+// src [rows, cols] -> codes [rows, cols/2], scales plain [rows, cols/32] or atoms
+// (groups = ceil(cols/128)).  cols a multiple of 256; one warp per 256 elements.
+template <typename TIN, bool ATOM>
+__global__ void __launch_bounds__(256) k_quant_mx4(const TIN* __restrict__ src, int64_t rows, int cols,
+                                                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                   int groups) {
+  const int lane = threadIdx.x & 31;
+  const int nch = cols >> 8;
+  const int64_t nwork = rows * nch;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < nwork; i += nwarps) {
+    const int64_t r = i / nch;
+    const int c = (int)(i - r * nch) * 256 + lane * 8;
+    float v[8];
+    ld8(src + r * cols + c, v);
+    const uint2 q = quant8_mx4(v);
+    *reinterpret_cast<uint32_t*>(codes + r * (cols >> 1) + (c >> 1)) = q.x;
+    if ((lane & 3) == 0) scales[ATOM ? atom_offset(r, c >> 5, groups) : r * (cols >> 5) + (c >> 5)] = (uint8_t)q.y;
+  }
+}
+
+// MXFP4 form of k_gather_quant (same padded rows); d a multiple of 512.
+__global__ void __launch_bounds__(256) k_gather_quant4(const __nv_bfloat16* __restrict__ x, int d,
+                                                       const int32_t* __restrict__ perm,
+                                                       const int32_t* __restrict__ idx, int k,
+                                                       const int32_t* __restrict__ offsets,
+                                                       const int32_t* __restrict__ mb_off,
+                                                       const int32_t* __restrict__ scal, uint8_t* __restrict__ x4,
+                                                       uint8_t* __restrict__ sx, int groups) {
+  const int P = scal[0];
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
+  for (int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); p < P; p += nwarps) {
+    const int pair = perm[p];
+    const int e = idx[pair];
+    const int64_t pad = (int64_t)(p - offsets[e]) + (int64_t)mb_off[e] * 128;
+    const __nv_bfloat16* src = x + (int64_t)(pair / k) * d;
+    uint8_t* dst = x4 + pad * (d >> 1);
+    for (int c0 = 0; c0 < d; c0 += 512) {
+      float v[2][8];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) ld8(src + c0 + 256 * u + lane * 8, v[u]);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int c = c0 + 256 * u + lane * 8;
+        const uint2 q = quant8_mx4(v[u]);
+        *reinterpret_cast<uint32_t*>(dst + (c >> 1)) = q.x;
+        if ((lane & 3) == 0) sx[atom_offset(pad, c >> 5, groups)] = (uint8_t)q.y;
+      }
+    }
+  }
+}
+
 // Debug copy: pair p's expert output from its padded row to row p.
 __global__ void __launch_bounds__(256) k_unpad_rows(const uint4* __restrict__ ypad, int row_vecs,
                                                     const int32_t* __restrict__ perm, const int32_t* __restrict__ idx,
@@ -169,6 +251,33 @@ cudaError_t launch_quant_rows(int bf16, const void* src, int64_t rows, int cols,
     if (atom) k_quant_rows<float, true><<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, atom_groups);
     else k_quant_rows<float, false><<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, 0);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_mx4(int bf16, const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
+                             int atom_groups, int sms, cudaStream_t s) {
+  const int64_t warps = rows * (cols / 256);
+  int64_t blocks = (warps + 7) / 8;
+  if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+  if (blocks < 1) blocks = 1;
+  const bool atom = atom_groups > 0;
+  if (bf16) {
+    auto src_ = static_cast<const __nv_bfloat16*>(src);
+    if (atom) k_quant_mx4<__nv_bfloat16, true><<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, atom_groups);
+    else k_quant_mx4<__nv_bfloat16, false><<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, 0);
+  } else {
+    auto src_ = static_cast<const float*>(src);
+    if (atom) k_quant_mx4<float, true><<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, atom_groups);
+    else k_quant_mx4<float, false><<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, 0);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_quant4(const void* x, int d, const int32_t* perm, const int32_t* idx, int k,
+                                 const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x4,
+                                 uint8_t* sx, int groups, int sms, cudaStream_t s) {
+  k_gather_quant4<<<sms * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), d, perm, idx, k, offsets, mb_off, scal,
+                                           x4, sx, groups);
   return cudaGetLastError();
 }
 

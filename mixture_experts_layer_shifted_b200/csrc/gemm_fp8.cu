@@ -34,12 +34,12 @@ namespace {
 constexpr int BM = 128, BN = 256, BK = 128, STAGES = 4;
 constexpr uint32_t A_BYTES = BM * BK;              // 16 KB
 constexpr uint32_t B_BYTES = BN * BK;              // 32 KB
-constexpr uint32_t SF_BYTES = 3 * kAtomBytes;      // A atom + two B atoms
+constexpr uint32_t SF_BYTES = 6 * kAtomBytes;      // per stage: FP8 uses 3 atoms, MXFP4 6
 constexpr uint32_t TILE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 320;
 constexpr int NUM_EPI = 256;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_COL = 256;                   // scale buffers: [256, 280)
+constexpr uint32_t SF_COL = 256;                   // scale buffers: [256, 304)
 constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES + SF_BYTES) + 256 + 2 * 2 * BM * 4;
 
 struct Tile {
@@ -102,6 +102,20 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t tsfa,
+                                            uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+// kind::mxf4 block-scaled: E2M1 A and B (packed, K-major), fp32 D, E8M0 scales, K = 64;
+// each MMA reads two scale bytes per row from byte `sf` (0 or 2).
+__device__ __forceinline__ uint32_t idesc_mxf4(uint32_t sf) {
+  return (sf << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24) |
+         (sf << 29);
+}
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NUM_EPI) : "memory"); }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
@@ -124,7 +138,9 @@ __device__ __forceinline__ bool epi_all(bool ok) {
   return r != 0;
 }
 
-template <int MODE>
+// FMT 0: FP8 E4M3 with [1,128] / [128,128] scales (128 K per k-block, atoms loaded every
+// fourth k-block); FMT 1: MXFP4 with [1,32] scales (256 K per k-block, six atoms every k-block).
+template <int MODE, int FMT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_fp8_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                const __grid_constant__ CUtensorMap tmB1, const Fp8Args args) {
@@ -169,7 +185,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int total = total_tiles(args);
-  const int num_k = args.K / BK;
+  const int num_k = args.K / (FMT ? 2 * BK : BK);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -189,10 +205,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          const bool with_sf = (kb & 3) == 0;
+          const bool with_sf = FMT ? true : (kb & 3) == 0;
           uint8_t* a_dst = sA + stage * A_BYTES;
           uint8_t* b_dst = sB + stage * B_BYTES;
-          mbar_expect_tx(&full[stage], TILE_BYTES + (with_sf ? SF_BYTES : 0u));
+          mbar_expect_tx(&full[stage], TILE_BYTES + (with_sf ? (FMT ? 6u : 3u) * kAtomBytes : 0u));
           tma_load_2d(a_dst, &tmA, kb * BK, (int)ti.a_row, &full[stage]);
           if (MODE == kGateUp) {
             tma_load_2d(b_dst, &tmB0, kb * BK, ti.b_row, &full[stage]);
@@ -200,12 +216,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           } else {
             tma_load_2d(b_dst, &tmB0, kb * BK, ti.b_row, &full[stage]);
           }
-          if (with_sf) {
-            uint8_t* sf_dst = sSF + stage * SF_BYTES;
+          uint8_t* sf_dst = sSF + stage * SF_BYTES;
+          if (FMT == 0 && with_sf) {
             const int64_t g = (int64_t)(kb >> 2) * kAtomBytes;
             bulk_load(sf_dst, sfa + g, kAtomBytes, &full[stage]);
             bulk_load(sf_dst + kAtomBytes, sfb_lo + g, kAtomBytes, &full[stage]);
             bulk_load(sf_dst + 2 * kAtomBytes, sfb_hi + g, kAtomBytes, &full[stage]);
+          } else if (FMT == 1) {
+            // K groups 2kb, 2kb+1: [A g0][A g1][B lo g0][B hi g0][B lo g1][B hi g1]
+            const int64_t g = (int64_t)(2 * kb) * kAtomBytes;
+            bulk_load(sf_dst, sfa + g, kAtomBytes, &full[stage]);
+            bulk_load(sf_dst + kAtomBytes, sfa + g + kAtomBytes, kAtomBytes, &full[stage]);
+            bulk_load(sf_dst + 2 * kAtomBytes, sfb_lo + g, kAtomBytes, &full[stage]);
+            bulk_load(sf_dst + 3 * kAtomBytes, sfb_hi + g, kAtomBytes, &full[stage]);
+            bulk_load(sf_dst + 4 * kAtomBytes, sfb_lo + g + kAtomBytes, kAtomBytes, &full[stage]);
+            bulk_load(sf_dst + 5 * kAtomBytes, sfb_hi + g + kAtomBytes, kAtomBytes, &full[stage]);
           }
           ++fills;
           if (++stage == STAGES) {
@@ -242,21 +267,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sfa_t = tmem_base + SF_COL + 16u * (uint32_t)((kb >> 2) & 1);
-          const uint32_t sfb_t = sfa_t + 4;
-          if ((kb & 3) == 0) {
-            const uint32_t sd = smem_u32(sSF + stage * SF_BYTES);
-            tc_cp_scales(sfa_t, atom_desc(sd));
-            tc_cp_scales(sfb_t, atom_desc(sd + kAtomBytes));
-            tc_cp_scales(sfb_t + 4, atom_desc(sd + 2 * kAtomBytes));
-          }
-          const uint32_t sf = (uint32_t)(kb & 3);
-          const uint32_t idesc = idesc_mxf8(sf);
+          const uint32_t sd = smem_u32(sSF + stage * SF_BYTES);
+          if (FMT == 0) {
+            const uint32_t sfa_t = tmem_base + SF_COL + 16u * (uint32_t)((kb >> 2) & 1);
+            const uint32_t sfb_t = sfa_t + 4;
+            if ((kb & 3) == 0) {
+              tc_cp_scales(sfa_t, atom_desc(sd));
+              tc_cp_scales(sfb_t, atom_desc(sd + kAtomBytes));
+              tc_cp_scales(sfb_t + 4, atom_desc(sd + 2 * kAtomBytes));
+            }
+            const uint32_t sf = (uint32_t)(kb & 3);
+            const uint32_t idesc = idesc_mxf8(sf);
 #pragma unroll
-          for (int kk = 0; kk < BK / 32; ++kk)
-            tc_mma_mxf8(tmem_base, adesc0 + (uint64_t)(stage * (A_BYTES >> 4) + kk * 2),
-                        bdesc0 + (uint64_t)(stage * (B_BYTES >> 4) + kk * 2), idesc, (sf << 30) | sfa_t,
-                        (sf << 30) | sfb_t, (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < BK / 32; ++kk)
+              tc_mma_mxf8(tmem_base, adesc0 + (uint64_t)(stage * (A_BYTES >> 4) + kk * 2),
+                          bdesc0 + (uint64_t)(stage * (B_BYTES >> 4) + kk * 2), idesc, (sf << 30) | sfa_t,
+                          (sf << 30) | sfb_t, (kb | kk) != 0 ? 1u : 0u);
+          } else {
+            // TMEM scales of this k-block: A g0 +0, A g1 +4, B g0 +8 (rows 0..127) / +12 (128..255), B g1 +16 / +20
+            const uint32_t buf = tmem_base + SF_COL + 24u * (uint32_t)(kb & 1);
+#pragma unroll
+            for (int a = 0; a < 6; ++a) tc_cp_scales(buf + 4 * a, atom_desc(sd + a * kAtomBytes));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {  // K = 64 each: 32 bytes of the 128-byte rows
+              const uint32_t sf = (uint32_t)((kk & 1) * 2);
+              const uint32_t g = (uint32_t)(kk >> 1);
+              tc_mma_mxf4(tmem_base, adesc0 + (uint64_t)(stage * (A_BYTES >> 4) + kk * 2),
+                          bdesc0 + (uint64_t)(stage * (B_BYTES >> 4) + kk * 2), idesc_mxf4(sf),
+                          (sf << 30) | (buf + 4 * g), (sf << 30) | (buf + 8 + 8 * g), (kb | kk) != 0 ? 1u : 0u);
+            }
+          }
           tc_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
@@ -282,7 +322,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const Tile ti = decode_tile<MODE>(args, t);
       const bool got = mbar_wait(tfull, acc_phase, err, 15);
-      if (MODE == kGateUp) {
+      if (MODE == kGateUp && FMT == 0) {
         if (!epi_all(got)) break;
       } else if (!got) {
         break;
@@ -300,14 +340,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_wait_ld();
         tc_fence_before();
         mbar_arrive(tempty);  // the accumulator may be overwritten from here on
-        float amax = 0.0f;
+        float amax = 0.0f, am0 = 0.0f, am1 = 0.0f;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const float h0 = silu_mul(__uint_as_float(g0[j]), __uint_as_float(u0[j]));
           const float h1 = silu_mul(__uint_as_float(g1[j]), __uint_as_float(u1[j]));
           g0[j] = __float_as_uint(h0);
           g1[j] = __float_as_uint(h1);
-          amax = fmaxf(amax, fmaxf(fabsf(h0), fabsf(h1)));
+          am0 = fmaxf(am0, fabsf(h0));
+          am1 = fmaxf(am1, fabsf(h1));
+        }
+        amax = fmaxf(am0, am1);
+        if (FMT == 1) {
+          // [1,32] blocks: columns [64 half, +32) and [64 half + 32, +32) of this H block
+          const int col0 = ti.n_blk * (BN / 2) + 64 * half;
+          if (row_ok && col0 < args.n_out) {
+            uint8_t* dst = static_cast<uint8_t*>(args.out) + grow * args.ldo + (col0 >> 1);
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const uint32_t* h = q == 0 ? g0 : g1;
+              const uint32_t code = mx4_code(q == 0 ? am0 : am1);
+              const float inv = e8m0_inverse(code);
+              float f[8];
+              uint4 v;
+              uint32_t* vw = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+              for (int w = 0; w < 4; ++w) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(h[8 * w + i]);
+                vw[w] = pack_e2m1x8(f, inv);
+              }
+              *reinterpret_cast<uint4*>(dst + 16 * q) = v;
+              args.out_sf[atom_offset(grow, (col0 >> 5) + q, args.out_groups)] = (uint8_t)code;
+            }
+          }
+          acc_phase ^= 1u;
+          buf ^= 1;
+          continue;
         }
         // the row's [1,128] block spans both halves: exchange the partial maxima
         amax_s[(buf * 2 + half) * BM + row] = amax;
@@ -373,16 +442,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const Fp8Args& args,
                         int grid, cudaStream_t s) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_fp8_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaError_t e =
+        cudaFuncSetAttribute(k_fp8_gemm<MODE, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k_fp8_gemm<MODE><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, args);
+  k_fp8_gemm<MODE, FMT><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, args);
   return cudaGetLastError();
 }
 
@@ -393,14 +463,11 @@ int fp8_block_n(int mode) { return mode == kGateUp ? BN / 2 : BN; }
 
 cudaError_t launch_fp8_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                             const Fp8Args& args, int grid, cudaStream_t s) {
-  switch (mode) {
-    case kGateUp:
-      return launch_mode<kGateUp>(a, b0, b1, args, grid, s);
-    case kDown:
-      return launch_mode<kDown>(a, b0, b1, args, grid, s);
-    default:
-      return cudaErrorInvalidValue;
-  }
+  if (mode == kGateUp) return args.fmt ? launch_mode<kGateUp, 1>(a, b0, b1, args, grid, s)
+                                       : launch_mode<kGateUp, 0>(a, b0, b1, args, grid, s);
+  if (mode == kDown) return args.fmt ? launch_mode<kDown, 1>(a, b0, b1, args, grid, s)
+                                     : launch_mode<kDown, 0>(a, b0, b1, args, grid, s);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace zc

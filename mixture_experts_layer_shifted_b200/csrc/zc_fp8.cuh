@@ -47,6 +47,42 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float v0, float v1, float v2, fl
   return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
+// ---------------------------------------------------------------- W4A4 (MXFP4)
+// A LongCat-Flash news page (gate.com post) reports W4A4 serving (expert
+// weights and activations in 4 bits) without naming the format; here MXFP4:
+// E2M1 codes (0, 0.5, 1, 1.5, 2, 3, 4, 6), round to nearest even, saturating;
+// one E8M0 scale per 32 elements along K, the smallest 2^E with amax <= 6 * 2^E.
+// Two codes per byte, the even element in the low nibble.  Scale atoms as above
+// with j indexing the 32-element blocks of a 128-element K group (so `kb` in
+// atom_offset is the 32-block index and `groups` = ceil(K / 128)).
+
+__device__ __forceinline__ uint32_t mx4_code(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  if (b == 0u) return 127u;
+  const int ef = (int)(b >> 23);
+  if (ef == 0) return 0u;
+  const int k = ef - 127;
+  // 6 = 1.5 * 2^2: amax <= 1.5 * 2^k  <=>  mantissa fraction <= 0.5
+  const int E = ((b & 0x7FFFFFu) <= 0x400000u) ? k - 2 : k - 1;
+  const int c = E + 127;
+  return (uint32_t)(c < 0 ? 0 : (c > 254 ? 254 : c));
+}
+
+// Two E2M1 codes in one byte: v_lo in bits 0..3, v_hi in bits 4..7.
+__device__ __forceinline__ uint32_t pack_e2m1x2(float v_lo, float v_hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}\n"
+      : "=r"(r)
+      : "f"(v_hi), "f"(v_lo));
+  return r;
+}
+
+// Eight E2M1 codes (v[0] lowest nibble) of v * inv.
+__device__ __forceinline__ uint32_t pack_e2m1x8(const float* v, float inv) {
+  return pack_e2m1x2(v[0] * inv, v[1] * inv) | (pack_e2m1x2(v[2] * inv, v[3] * inv) << 8) |
+         (pack_e2m1x2(v[4] * inv, v[5] * inv) << 16) | (pack_e2m1x2(v[6] * inv, v[7] * inv) << 24);
+}
+
 // Byte offset of (row, K-block) in a scale-atom array with `groups` atoms per 128 rows.
 __host__ __device__ __forceinline__ int64_t atom_offset(int64_t row, int kb, int groups) {
   const int64_t R = row >> 7;

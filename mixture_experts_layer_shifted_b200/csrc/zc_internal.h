@@ -70,12 +70,20 @@ cudaError_t launch_gather_quant(const void* x, int d, const int32_t* perm, const
                                 const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x8,
                                 uint8_t* sx, int groups, int sms, cudaStream_t s);
 
+// MXFP4: [1,32] blocks along each row (cols a multiple of 256), codes two per byte;
+// atom_groups > 0: scale atoms with that many atoms (128 elements each) per 128 rows.
+cudaError_t launch_quant_mx4(int bf16, const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
+                             int atom_groups, int sms, cudaStream_t s);
+cudaError_t launch_gather_quant4(const void* x, int d, const int32_t* perm, const int32_t* idx, int k,
+                                 const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x4,
+                                 uint8_t* sx, int groups, int sms, cudaStream_t s);
 cudaError_t launch_unpad_rows(const void* ypad, int row_bytes, const int32_t* perm, const int32_t* idx,
                               const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, void* out, int sms,
                               cudaStream_t s);
 
 struct Fp8Args {
-  int K;                   // reduction length (a multiple of 128)
+  int fmt;                 // 0: FP8 E4M3, [1,128]/[128,128] scales; 1: MXFP4, [1,32] scales
+  int K;                   // reduction length in elements (FP8: a multiple of 128, MXFP4: of 256)
   int n_out;               // valid output columns
   int nblocks;             // output column tiles
   int ngroups;             // experts
@@ -85,9 +93,9 @@ struct Fp8Args {
   const uint8_t* sfa;      // A scale atoms
   const uint8_t* sfb0;     // B scale atoms (gate/up: W_g, down: W_d)
   const uint8_t* sfb1;     // gate/up: W_u scale atoms
-  int groups_k;            // scale atoms per 128 rows of A and B = ceil(K / 512)
-  void* out;               // gate/up: H codes [padded rows, n_out]; down: Y bf16 [padded rows, n_out]
-  int64_t ldo;             // its row stride (elements)
+  int groups_k;            // scale atoms per 128 rows of A and B: FP8 ceil(K / 512), MXFP4 ceil(K / 128)
+  void* out;               // gate/up: H codes [padded rows, n_out (FP8) or n_out / 2 (MXFP4) bytes]; down: Y bf16
+  int64_t ldo;             // its row stride (gate/up: bytes; down: elements)
   uint8_t* out_sf;         // gate/up: H scale atoms, out_groups per 128 rows
   int out_groups;
   int* err;                // device error word (bounded waits)

@@ -148,7 +148,7 @@ struct zcmoe_s {
   // ZCMOE_FP8: expert weights as E4M3 codes + scale atoms (owned), padded
   // activation operands (expert e's pairs from row 128 mb_off[e] on) with their
   // scale atoms, padded expert outputs; atoms per 128 rows: gd (K = d), gi (K = inter)
-  int fp8, gd, gi;
+  int fp8, fmt, gd, gi;  // fp8: block-scaled experts (ZCMOE_FP8 or ZCMOE_FP4); fmt 1 for MXFP4
   uint8_t *w8g, *w8u, *w8d, *sfg, *sfu, *sfd, *x8, *sx, *h8, *sh;
   void* ypad;
   CUtensorMap tm8_wg, tm8_wu, tm8_wd, tm8_x, tm8_h;
@@ -261,10 +261,12 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
   if (cfg->d < 64 || cfg->d % 64 || cfg->inter < 64 || cfg->inter % 64)
     return fail(ZCMOE_EINVAL, "d and inter must be positive multiples of 64");
   if (cfg->max_tokens < 1 || cfg->max_tokens > (1 << 20)) return fail(ZCMOE_EINVAL, "need 1 <= max_tokens <= 2^20");
-  if (cfg->dtype != ZCMOE_F32 && cfg->dtype != ZCMOE_BF16 && cfg->dtype != ZCMOE_FP8)
+  if (cfg->dtype != ZCMOE_F32 && cfg->dtype != ZCMOE_BF16 && cfg->dtype != ZCMOE_FP8 && cfg->dtype != ZCMOE_FP4)
     return fail(ZCMOE_EINVAL, "unknown dtype");
   if (cfg->dtype == ZCMOE_FP8 && (cfg->d % 512 || cfg->inter % 128))
     return fail(ZCMOE_EINVAL, "FP8 experts need d a multiple of 512 and inter a multiple of 128");
+  if (cfg->dtype == ZCMOE_FP4 && (cfg->d % 512 || cfg->inter % 256))
+    return fail(ZCMOE_EINVAL, "MXFP4 experts need d a multiple of 512 and inter a multiple of 256");
   if (!w->w_router || !w->w_gate || !w->w_up || !w->w_down) return fail(ZCMOE_EINVAL, "a weight pointer is NULL");
   const void* wp[4] = {w->w_router, w->w_gate, w->w_up, w->w_down};
   for (const void* p : wp)
@@ -295,8 +297,9 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
   h->d = cfg->d;
   h->inter = cfg->inter;
   h->max_T = cfg->max_tokens;
-  h->bf16 = cfg->dtype != ZCMOE_F32;  // ZCMOE_FP8 layers are bf16 at the interface
-  h->fp8 = cfg->dtype == ZCMOE_FP8;
+  h->bf16 = cfg->dtype != ZCMOE_F32;  // ZCMOE_FP8 / ZCMOE_FP4 layers are bf16 at the interface
+  h->fp8 = cfg->dtype == ZCMOE_FP8 || cfg->dtype == ZCMOE_FP4;
+  h->fmt = cfg->dtype == ZCMOE_FP4;
   h->sms = prop.multiProcessorCount;
   h->device = dev;
   h->w = *w;
@@ -338,18 +341,19 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
   }
   if (h->fp8) {
     const size_t prow = (size_t)h->max_mblocks * zc::kBM;  // padded rows
-    h->gd = (h->d / 128 + 3) / 4;
-    h->gi = (h->inter / 128 + 3) / 4;
-    const size_t wn = (size_t)N * h->inter * h->d;
+    // scale atoms per 128 rows: an atom covers 512 K elements (FP8) or 128 (MXFP4)
+    h->gd = h->fmt ? (h->d + 127) / 128 : (h->d / 128 + 3) / 4;
+    h->gi = h->fmt ? (h->inter + 127) / 128 : (h->inter / 128 + 3) / 4;
+    const size_t wn = (size_t)N * h->inter * h->d / (h->fmt ? 2 : 1);
     ZC_ALLOC(h->w8g, wn);
     ZC_ALLOC(h->w8u, wn);
     ZC_ALLOC(h->w8d, wn);
     ZC_ALLOC(h->sfg, (size_t)N * (h->inter / 128) * h->gd * zc::kAtomBytes);
     ZC_ALLOC(h->sfu, (size_t)N * (h->inter / 128) * h->gd * zc::kAtomBytes);
     ZC_ALLOC(h->sfd, (size_t)N * (h->d / 128) * h->gi * zc::kAtomBytes);
-    ZC_ALLOC(h->x8, prow * h->d);
+    ZC_ALLOC(h->x8, prow * h->d / (h->fmt ? 2 : 1));
     ZC_ALLOC(h->sx, (size_t)h->max_mblocks * h->gd * zc::kAtomBytes);
-    ZC_ALLOC(h->h8, prow * h->inter);
+    ZC_ALLOC(h->h8, prow * h->inter / (h->fmt ? 2 : 1));
     ZC_ALLOC(h->sh, (size_t)h->max_mblocks * h->gi * zc::kAtomBytes);
     uint8_t* yp = nullptr;
     ZC_ALLOC(yp, prow * h->d * 2);
@@ -387,15 +391,21 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
     if (h->fp8) {
       // padded operand rows that no pair fills read as zeros
       const size_t prow = (size_t)h->max_mblocks * zc::kBM;
-      if (e == cudaSuccess) e = cudaMemset(h->x8, 0, prow * h->d);
-      if (e == cudaSuccess) e = cudaMemset(h->h8, 0, prow * h->inter);
+      if (e == cudaSuccess) e = cudaMemset(h->x8, 0, prow * h->d / (h->fmt ? 2 : 1));
+      if (e == cudaSuccess) e = cudaMemset(h->h8, 0, prow * h->inter / (h->fmt ? 2 : 1));
       if (e == cudaSuccess) e = cudaMemset(h->sx, 0, (size_t)h->max_mblocks * h->gd * zc::kAtomBytes);
       if (e == cudaSuccess) e = cudaMemset(h->sh, 0, (size_t)h->max_mblocks * h->gi * zc::kAtomBytes);
-      // the expert weights, quantized per [128,128] into scale atoms
+      // the expert weights, quantized into scale atoms: FP8 per [128,128], MXFP4 per [1,32]
       const int64_t ri = (int64_t)N * h->inter, rd = (int64_t)N * h->d;
-      if (e == cudaSuccess) e = zc::launch_quant_tiles(1, w->w_gate, ri, h->d, h->w8g, h->sfg, h->gd, 0);
-      if (e == cudaSuccess) e = zc::launch_quant_tiles(1, w->w_up, ri, h->d, h->w8u, h->sfu, h->gd, 0);
-      if (e == cudaSuccess) e = zc::launch_quant_tiles(1, w->w_down, rd, h->inter, h->w8d, h->sfd, h->gi, 0);
+      if (h->fmt) {
+        if (e == cudaSuccess) e = zc::launch_quant_mx4(1, w->w_gate, ri, h->d, h->w8g, h->sfg, h->gd, h->sms, 0);
+        if (e == cudaSuccess) e = zc::launch_quant_mx4(1, w->w_up, ri, h->d, h->w8u, h->sfu, h->gd, h->sms, 0);
+        if (e == cudaSuccess) e = zc::launch_quant_mx4(1, w->w_down, rd, h->inter, h->w8d, h->sfd, h->gi, h->sms, 0);
+      } else {
+        if (e == cudaSuccess) e = zc::launch_quant_tiles(1, w->w_gate, ri, h->d, h->w8g, h->sfg, h->gd, 0);
+        if (e == cudaSuccess) e = zc::launch_quant_tiles(1, w->w_up, ri, h->d, h->w8u, h->sfu, h->gd, 0);
+        if (e == cudaSuccess) e = zc::launch_quant_tiles(1, w->w_down, rd, h->inter, h->w8d, h->sfd, h->gi, 0);
+      }
     }
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     delete[] hb;
@@ -415,12 +425,14 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
     if (rc == ZCMOE_OK && !h->fp8) rc = make_tmap(&h->tm_xperm, h->xperm, d, (uint64_t)h->max_pairs, 128);
     if (rc == ZCMOE_OK && !h->fp8) rc = make_tmap(&h->tm_h, h->H, inter, (uint64_t)h->max_pairs, 128);
     if (h->fp8) {
+      // codes as bytes: the K extent is d or inter bytes (FP8), half that (MXFP4)
       const uint64_t prow = (uint64_t)h->max_mblocks * zc::kBM;
-      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_wg, h->w8g, d, (uint64_t)N * inter, 128, 1);
-      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_wu, h->w8u, d, (uint64_t)N * inter, 128, 1);
-      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_wd, h->w8d, inter, (uint64_t)N * d, 256, 1);
-      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_x, h->x8, d, prow, 128, 1);
-      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_h, h->h8, inter, prow, 128, 1);
+      const uint64_t db = d / (h->fmt ? 2 : 1), ib = inter / (h->fmt ? 2 : 1);
+      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_wg, h->w8g, db, (uint64_t)N * inter, 128, 1);
+      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_wu, h->w8u, db, (uint64_t)N * inter, 128, 1);
+      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_wd, h->w8d, ib, (uint64_t)N * d, 256, 1);
+      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_x, h->x8, db, prow, 128, 1);
+      if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_h, h->h8, ib, prow, 128, 1);
     }
     if (rc != ZCMOE_OK) {
       release(h);
@@ -512,7 +524,10 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
   ZC_CUDA(zc::launch_route_scatter(h->idx, Ti, k, N, E, h->chunk, h->perm, h->pos, s));
   ZC_CUDA(mark());
   // 4. gather the FFN pairs' rows (FP8 layers: quantized per [1,128] into padded rows)
-  if (h->fp8)
+  if (h->fp8 && h->fmt)
+    ZC_CUDA(zc::launch_gather_quant4(x, d, h->perm, h->idx, k, h->offsets, h->mb_off, h->scal, h->x8, h->sx, h->gd,
+                                     h->sms, s));
+  else if (h->fp8)
     ZC_CUDA(zc::launch_gather_quant(x, d, h->perm, h->idx, k, h->offsets, h->mb_off, h->scal, h->x8, h->sx, h->gd,
                                     h->sms, s));
   else
@@ -522,6 +537,7 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
   const int max_mb = (Ti * k + zc::kBM - 1) / zc::kBM + N;
   if (h->fp8) {
     zc::Fp8Args a{};
+    a.fmt = h->fmt;
     a.K = d;
     a.n_out = inter;
     a.nblocks = inter / zc::fp8_block_n(zc::kGateUp);
@@ -534,7 +550,7 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     a.sfb1 = h->sfu;
     a.groups_k = h->gd;
     a.out = h->h8;
-    a.ldo = inter;
+    a.ldo = inter / (h->fmt ? 2 : 1);
     a.out_sf = h->sh;
     a.out_groups = h->gi;
     a.err = h->err;
@@ -542,6 +558,7 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     ZC_CUDA(zc::launch_fp8_gemm(zc::kGateUp, h->tm8_x, h->tm8_wg, h->tm8_wu, a, bound < h->sms ? bound : h->sms, s));
     ZC_CUDA(mark());
     zc::Fp8Args b{};
+    b.fmt = h->fmt;
     b.K = inter;
     b.n_out = d;
     b.nblocks = (d + zc::fp8_block_n(zc::kDown) - 1) / zc::fp8_block_n(zc::kDown);
@@ -843,6 +860,22 @@ int zcmoe_quantize_e4m3(const void* src, int32_t src_dtype, int64_t rows, int64_
     ZC_CUDA(zc::launch_quant_rows(bf16, src, rows, (int)cols, codes, scales, 0, sms, s));
   else
     ZC_CUDA(zc::launch_quant_tiles(bf16, src, rows, (int)cols, codes, scales, 0, s));
+  return ZCMOE_OK;
+}
+
+int zcmoe_quantize_mx4(const void* src, int32_t src_dtype, int64_t rows, int64_t cols, uint8_t* codes,
+                       uint8_t* scales, cudaStream_t s) {
+  g_err[0] = 0;
+  if (src_dtype != ZCMOE_BF16 && src_dtype != ZCMOE_F32) return fail(ZCMOE_EINVAL, "src_dtype must be BF16 or F32");
+  if (rows < 0 || cols <= 0 || cols % 256 || cols > (1 << 30)) return fail(ZCMOE_EINVAL, "bad rows / cols");
+  if (rows == 0) return ZCMOE_OK;
+  if (!src || !codes || !scales) return fail(ZCMOE_EINVAL, "a pointer is NULL");
+  if ((reinterpret_cast<uintptr_t>(src) & 15u) || (reinterpret_cast<uintptr_t>(codes) & 15u))
+    return fail(ZCMOE_EINVAL, "src and codes must be 16-byte aligned");
+  int dev = 0, sms = 0;
+  ZC_CUDA(cudaGetDevice(&dev));
+  ZC_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  ZC_CUDA(zc::launch_quant_mx4(src_dtype == ZCMOE_BF16, src, rows, (int)cols, codes, scales, 0, sms, s));
   return ZCMOE_OK;
 }
 

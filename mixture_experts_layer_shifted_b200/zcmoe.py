@@ -28,13 +28,14 @@ ZCMOE_ETIMEOUT = -6
 ZCMOE_F32 = 0
 ZCMOE_BF16 = 1
 ZCMOE_FP8 = 2
-_DTYPES = {"f32": ZCMOE_F32, "bf16": ZCMOE_BF16, "fp8": ZCMOE_FP8}
+ZCMOE_FP4 = 3
+_DTYPES = {"f32": ZCMOE_F32, "bf16": ZCMOE_BF16, "fp8": ZCMOE_FP8, "fp4": ZCMOE_FP4}
 
 EXPORTED = ("zcmoe_create", "zcmoe_forward", "zcmoe_forward_host", "zcmoe_update_bias", "zcmoe_read_counts",
             "zcmoe_write_counts", "zcmoe_get_state", "zcmoe_set_bias", "zcmoe_check", "zcmoe_profile_begin",
             "zcmoe_profile_end", "zcmoe_selftest_wait", "zcmoe_route_noalloc", "zcmoe_destroy",
             "zcmoe_dense_create", "zcmoe_dense_forward", "zcmoe_forward_overlap", "zcmoe_dense_check",
-            "zcmoe_dense_destroy", "zcmoe_quantize_e4m3", "zcmoe_last_error")
+            "zcmoe_dense_destroy", "zcmoe_quantize_e4m3", "zcmoe_quantize_mx4", "zcmoe_last_error")
 STAGES = ("router", "softmax_topk", "integer", "gather", "gate_up", "down", "combine")
 
 
@@ -107,6 +108,7 @@ def lib():
         L.zcmoe_forward_overlap.argtypes = [vp, vp, vp, vp, i64, vp, vp, vp]
         L.zcmoe_dense_check.argtypes = [vp]
         L.zcmoe_quantize_e4m3.argtypes = [vp, ctypes.c_int32, i64, i64, ctypes.c_int32, vp, vp, vp]
+        L.zcmoe_quantize_mx4.argtypes = [vp, ctypes.c_int32, i64, i64, vp, vp, vp]
         L.zcmoe_dense_destroy.argtypes = [vp]
         for f in EXPORTED[:-1]:
             getattr(L, f).restype = i32
@@ -239,6 +241,23 @@ def quantize_e4m3(src, block_rows, stream=None):
     return codes, scales
 
 
+def zcmoe_quantize_mx4(src_ptr, src_dtype, rows, cols, codes_ptr, scales_ptr, stream=None):
+    _check(lib().zcmoe_quantize_mx4(src_ptr, src_dtype, rows, cols, codes_ptr, scales_ptr, _stream(stream)),
+           "zcmoe_quantize_mx4")
+
+
+def quantize_mx4(src, stream=None):
+    """(codes uint8 [rows, cols/2], scales uint8 [rows, cols/32]) of a 2-D bf16 or fp32
+    device tensor (MXFP4, the rule of ZCMOE_FP4 layers)."""
+    rows, cols = src.shape
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=src.device)
+    scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=src.device)
+    dt = ZCMOE_BF16 if src.dtype == torch.bfloat16 else ZCMOE_F32
+    zcmoe_quantize_mx4(ctypes.c_void_p(src.data_ptr()), dt, rows, cols, ctypes.c_void_p(codes.data_ptr()),
+                       ctypes.c_void_p(scales.data_ptr()), stream)
+    return codes, scales
+
+
 def zcmoe_last_error() -> str:
     return lib().zcmoe_last_error().decode(errors="replace")
 
@@ -251,7 +270,7 @@ class LayerShape:
     n_zero: int
     inter: int
     top_k: int
-    dtype: str = "bf16"  # "bf16", "f32", or "fp8" (bf16 interface, block-scaled FP8 experts)
+    dtype: str = "bf16"  # "bf16", "f32", "fp8" or "fp4" (bf16 interface, block-scaled FP8 / MXFP4 experts)
     routed_scale: float = 1.0
 
     @property

@@ -194,12 +194,13 @@ def layer(x, idx, gate, N, wg, wu, wd):
     return y
 
 
-def layer_outputs(x_rows, idx, gate, N, expert_weights, fp8=False, expert_fn=None):
+def layer_outputs(x_rows, idx, gate, N, expert_weights, fp8=False, expert_fn=None, fp4=False):
     """fp64 layer output for a few tokens when the expert weights are fetched one
     expert at a time.  ``expert_weights(e) -> (wg, wu, wd)``.  Sums
     g * F_e(x) over the token's FFN slots plus (sum of zero-slot gates) * x.
     fp8: F_e is the block-scaled FP8 expert (ffn_fp8) on weights quantized here
-    per [128,128].  expert_fn(e, rows) -> F_e(rows), if given, replaces both."""
+    per [128,128].  fp4: the MXFP4 expert (ffn_fp4) on weights quantized here per
+    [1,32].  expert_fn(e, rows) -> F_e(rows), if given, replaces these."""
     x_rows = np.ascontiguousarray(x_rows)
     n, d = x_rows.shape
     xf = x_rows.astype(np.float64) if x_rows.dtype == np.float32 else \
@@ -222,7 +223,10 @@ def layer_outputs(x_rows, idx, gate, N, expert_weights, fp8=False, expert_fn=Non
                 y[r] += float(gate[r, j]) * f[i]
             continue
         wg, wu, wd = expert_weights(e)
-        if fp8:
+        if fp4:
+            q = [quantize_mx4(w) for w in (wg, wu, wd)]
+            f = ffn_fp4(x_rows[rows], [c for c, _ in q], [s_ for _, s_ in q])
+        elif fp8:
             q = [quantize_blocks(w, 128) for w in (wg, wu, wd)]
             f = ffn_fp8(x_rows[rows], [c for c, _ in q], [s_ for _, s_ in q])
         else:

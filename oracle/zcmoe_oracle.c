@@ -418,6 +418,7 @@ ZO_EXPORT uint8_t zo_e8m0_scale(float amax) {
 ZO_EXPORT void zo_quantize_blocks(const void *src, int dtype, int64_t rows, int64_t cols, int block_rows,
                                   uint8_t *codes, uint8_t *scales) {
   const int64_t nrb = (rows + block_rows - 1) / block_rows, ncb = cols / 128;
+#pragma omp parallel for schedule(dynamic, 1) if (rows * cols > (1 << 20))
   for (int64_t rb = 0; rb < nrb; ++rb) {
     const int64_t r0 = rb * block_rows, r1 = (r0 + block_rows < rows) ? r0 + block_rows : rows;
     for (int64_t cb = 0; cb < ncb; ++cb) {
@@ -549,6 +550,7 @@ ZO_EXPORT uint8_t zo_mx4_scale(float amax) {
 ZO_EXPORT void zo_quantize_mx4(const void *src, int dtype, int64_t rows, int64_t cols, uint8_t *codes,
                                uint8_t *scales) {
   const int64_t nb = cols / 32;
+#pragma omp parallel for schedule(static) if (rows * cols > (1 << 20))
   for (int64_t r = 0; r < rows; ++r)
     for (int64_t b = 0; b < nb; ++b) {
       double amax = 0.0;
@@ -596,8 +598,11 @@ ZO_EXPORT void zo_ffn_fp4_f64(const void *xs, int x_dtype, int64_t n, const uint
     for (int i = 0; i < inter; ++i) {
       double g = 0.0, u = 0.0;
       for (int c = 0; c < d; ++c) {
-        g += mx4_value(wg, sg, d, i, c, tab) * xv[c];
-        u += mx4_value(wu, su, d, i, c, tab) * xv[c];
+        const uint8_t bg = wg[(int64_t)i * (d / 2) + c / 2], bu = wu[(int64_t)i * (d / 2) + c / 2];
+        const double sgv = ldexp(1.0, (int)sg[(int64_t)i * (d / 32) + c / 32] - 127);
+        const double suv = ldexp(1.0, (int)su[(int64_t)i * (d / 32) + c / 32] - 127);
+        g += (tab[(c & 1) ? bg >> 4 : bg & 0xF] * sgv) * xv[c];
+        u += (tab[(c & 1) ? bu >> 4 : bu & 0xF] * suv) * xv[c];
       }
       h32[i] = (float)(g / (1.0 + exp(-g)) * u);
     }

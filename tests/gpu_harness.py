@@ -8,7 +8,7 @@ Tolerances (from the arithmetic; written in each check):
   * fp64-routing comparison: indices equal on tokens whose k-th and (k+1)-th
     biased scores differ by at least 1e-5;
   * layer outputs and expert outputs: max over rows of ||err||_inf / ||ref||_inf
-    <= 2e-2 (bf16 layers; FP8 layers against the FP8 oracle) or 1e-4 (fp32 layer).
+    <= 2e-2 (bf16 layers; FP8 / MXFP4 layers against their oracle) or 1e-4 (fp32 layer).
 """
 from __future__ import annotations
 
@@ -19,7 +19,7 @@ import oracle
 from mixture_experts_layer_shifted_b200 import configs, synth
 from mixture_experts_layer_shifted_b200.zcmoe import LayerShape, ZcMoE
 
-TOL = {"bf16": 2e-2, "f32": 1e-4, "fp8": 2e-2}
+TOL = {"bf16": 2e-2, "f32": 1e-4, "fp8": 2e-2, "fp4": 2e-2}
 TIE_MARGIN = 1e-5
 
 
@@ -150,7 +150,10 @@ class Run:
         for e, lst in sorted(byexp.items()):
             wg, wu, wd = self.expert_weights(e)
             rows = [t for _, t in lst]
-            if self.w.dtype == "fp8":
+            if self.w.dtype == "fp4":
+                q = [oracle.quantize_mx4(w_) for w_ in (wg, wu, wd)]
+                ref = oracle.ffn_fp4(self.x_host(rows), [c for c, _ in q], [s_ for _, s_ in q])
+            elif self.w.dtype == "fp8":
                 q = [oracle.quantize_blocks(w_, 128) for w_ in (wg, wu, wd)]
                 ref = oracle.ffn_fp8(self.x_host(rows), [c for c, _ in q], [s_ for _, s_ in q])
             else:
@@ -168,7 +171,7 @@ class Run:
         idx = self.dbg["idx"][rows]
         gate = self.dbg["gate"][rows].astype(np.float64)
         ref = oracle.layer_outputs(self.x_host(rows), idx, gate, self.w.n_ffn, self.expert_weights,
-                                   fp8=self.w.dtype == "fp8")
+                                   fp8=self.w.dtype == "fp8", fp4=self.w.dtype == "fp4")
         err = row_rel_err(self.y[rows], ref)
         assert float(err.max()) <= tol, float(err.max())
         return float(err.max())
