@@ -130,7 +130,7 @@ def algorithmic_work(wl, P, distinct):
     B = distinct * 3 d inter * w + E d * 2 + 2 T d * 2 (bf16; expert weights w = 2
     bytes, or 1 for FP8 experts; fp32 layers 4 throughout)."""
     esz = 4 if wl.dtype == "f32" else 2
-    wsz = 1 if wl.dtype == "fp8" else esz
+    wsz = {"fp8": 1, "fp4": 0.5}.get(wl.dtype, esz)
     F = 2.0 * wl.T * wl.d * wl.E + 6.0 * wl.d * wl.inter * P
     B = distinct * 3.0 * wl.d * wl.inter * wsz + wl.E * wl.d * esz + 2.0 * wl.T * wl.d * esz
     return F, B
@@ -141,7 +141,8 @@ def roofline_ms(wl, F, B, peaks):
     nominal 4.5 / 2.25 PFLOP/s ratio), the router in bf16."""
     p = peaks["bf16_tflops_sustained"] * 1e12
     f_router = 2.0 * wl.T * wl.d * wl.E
-    t_tensor = (f_router / p + (F - f_router) / (2 * p)) if wl.dtype == "fp8" else F / p
+    mult = {"fp8": 2, "fp4": 4}.get(wl.dtype, 1)
+    t_tensor = f_router / p + (F - f_router) / (mult * p)
     return 1e3 * max(t_tensor, B / (peaks["hbm_gbs"] * 1e9))
 
 
@@ -170,6 +171,9 @@ def cpu_oracle_sample(wl, weights, x, bias, offset, n_tokens, min_s=10.0):
     if wl.dtype == "fp8":  # weights quantized once, as the layer does at create
         q8 = {e: [oracle.quantize_blocks(w, 128) for w in cache[e]] for e in need}
         efn = lambda e, rows: oracle.ffn_fp8(rows, [c for c, _ in q8[e]], [s_ for _, s_ in q8[e]])
+    elif wl.dtype == "fp4":
+        q4 = {e: [oracle.quantize_mx4(w) for w in cache[e]] for e in need}
+        efn = lambda e, rows: oracle.ffn_fp4(rows, [c for c, _ in q4[e]], [s_ for _, s_ in q4[e]])
     done = 0
     t0 = time.perf_counter()
     while True:  # the sample is processed again until the time budget is spent
@@ -284,19 +288,21 @@ def graph_ms(fn, stream, reps=10):
     return a.elapsed_time(b) / reps
 
 
-def measure_fp8(layer, weights, x, stream, peaks, bias, offset):
-    """The same layer with block-scaled FP8 experts, on the same weights and batch:
-    forward time against the bf16 layer, the FP8 GEMMs against the FP8 peak, and
-    the decode batch against HBM."""
+def measure_lowp(layer, weights, x, stream, peaks, fmt="fp8"):
+    """The same layer with block-scaled FP8 or W4A4 (MXFP4) experts, on the same weights
+    and batch: forward time against the bf16 layer, the expert GEMMs against the
+    format's peak (2x or 4x the measured sustained bf16 peak, the nominal 4.5 and
+    9 PFLOP/s against 2.25), and the decode batch against HBM."""
     import torch
     from mixture_experts_layer_shifted_b200 import configs
     from mixture_experts_layer_shifted_b200.zcmoe import LayerShape, ZcMoE
 
     out = {}
-    for name, layer_b in (("prefill_560b_fp8", layer), ("decode_560b_fp8", None)):
+    mult = 2 if fmt == "fp8" else 4
+    for name, layer_b in ((f"prefill_560b_{fmt}", layer), (f"decode_560b_{fmt}", None)):
         wf = configs.WORKLOADS[name]
         xf = x if layer_b is not None else configs.device_tokens(wf)
-        shp = LayerShape(wf.d, wf.n_ffn, wf.n_zero, wf.inter, wf.top_k, "fp8")
+        shp = LayerShape(wf.d, wf.n_ffn, wf.n_zero, wf.inter, wf.top_k, fmt)
         l8 = ZcMoE(shp, *weights, max_tokens=wf.T, init_bias=configs.bias_vector(wf),
                    logit_offset=configs.logit_offsets(wf))
         lb = layer_b
@@ -317,13 +323,13 @@ def measure_fp8(layer, weights, x, stream, peaks, bias, offset):
             l8.forward(xf, y8)
         st, nf = l8.profile_end()
         st = {k_: v / nf for k_, v in st.items()}
-        p8 = 2 * peaks["bf16_tflops_sustained"]
+        p8 = mult * peaks["bf16_tflops_sustained"]
         gu = 4.0 * wf.d * wf.inter * P / (st["gate_up"] * 1e-3) / 1e12
         dn = 2.0 * wf.d * wf.inter * P / (st["down"] * 1e-3) / 1e12
         rec = {"tokens_per_s": wf.T / (ms8 * 1e-3), "ms_per_forward": ms8, "bf16_ms_per_forward": msb,
                "speedup_vs_bf16": msb / ms8, "stage_ms": st,
-               "gate_up": {"tflops": gu, "frac_fp8_peak": gu / p8},
-               "down": {"tflops": dn, "frac_fp8_peak": dn / p8},
+               "gate_up": {"tflops": gu, "frac_peak": gu / p8},
+               "down": {"tflops": dn, "frac_peak": dn / p8},
                "layer_roofline_ms": roofline_ms(wf, F, B, peaks), "P": P}
         if layer_b is None:
             rec["hbm_gbs"] = B / (ms8 * 1e-3) / 1e9
@@ -332,7 +338,8 @@ def measure_fp8(layer, weights, x, stream, peaks, bias, offset):
         l8.check()
         l8.close()
         out[name] = rec
-    out["peak_note"] = "fp8 dense peak = 2 x measured sustained bf16 (nominal 4.5/2.25 PFLOP/s ratio)"
+    out["peak_note"] = (f"{fmt} dense peak = {mult} x measured sustained bf16 "
+                        f"(nominal {'4.5' if mult == 2 else '9'}/2.25 PFLOP/s ratio)")
     return out
 
 
@@ -450,15 +457,16 @@ def main():
     stage_avg = {s: v / nf for s, v in stage_ms.items()}
     gu_ms = stage_avg["gate_up"]
     gu_flops = 4.0 * wl.d * wl.inter * P
-    fp8 = wl.dtype == "fp8"
-    tensor_peak = peaks["bf16_tflops_sustained"] * (2 if fp8 else 1)
+    fp8 = wl.dtype in ("fp8", "fp4")
+    mult = {"fp8": 2, "fp4": 4}.get(wl.dtype, 1)
+    tensor_peak = peaks["bf16_tflops_sustained"] * mult
     achieved = gu_flops / (gu_ms * 1e-3) / 1e12
-    kname = ("grouped FP8 gate/up GEMM + SwiGLU + quantize (k_fp8_gemm<1>)" if fp8
+    kname = (f"grouped {wl.dtype.upper()} gate/up GEMM + SwiGLU + quantize (k_fp8_gemm<1>)" if fp8
              else "grouped gate/up GEMM + SwiGLU (k_tc_gemm<1>)")
     roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved,
                 "peak": tensor_peak, "unit": "TFLOP/s", "frac": achieved / tensor_peak,
                 "traffic": None if fp8 else recorded_traffic(wl.name, "gate_up"),
-                "peak_kind": (f"fp8 dense = 2 x bf16 dense sustained ({peaks['source']}; nominal 4.5/2.25 ratio)" if fp8
+                "peak_kind": (f"{wl.dtype} dense = {mult} x bf16 dense sustained ({peaks['source']}; nominal ratio)" if fp8
                               else f"bf16 dense, sustained, {peaks['source']}"),
                 "per_launch": {"flops": gu_flops, "ms": gu_ms, "units": f"{P} FFN (token, expert) pairs x 4 d inter"}}
     fwd_ms = sum(stage_avg.values())
@@ -546,7 +554,8 @@ def main():
 
     # secondary: the same layer with block-scaled FP8 experts (bf16 headline unchanged)
     if rank == 0 and ws == 1 and not args.no_secondary and wl.name == "prefill_560b":
-        line["fp8"] = measure_fp8(layer, weights, xs[0], stream, peaks, bias, offset)
+        line["fp8"] = measure_lowp(layer, weights, xs[0], stream, peaks, "fp8")
+        line["fp4"] = measure_lowp(layer, weights, xs[0], stream, peaks, "fp4")
 
     # secondary: the dense FFN path run beside the layer (shortcut-connected MoE)
     if rank == 0 and ws == 1 and not args.no_secondary and wl.dense_inter > 0:
