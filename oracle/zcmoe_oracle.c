@@ -623,3 +623,115 @@ ZO_EXPORT void zo_ffn_fp4_f64(const void *xs, int x_dtype, int64_t n, const uint
   free(hv);
   free(h32);
 }
+
+/* ------------------------------------------------------------------------- */
+/* Backward pass (training), fp64.                                            */
+/* LongCat-Flash technical summary (zhangjingwei.cn), 五 訓練基礎設施: the MoE   */
+/* layer trains with a deterministic ScatterAdd and a fused GemmAdd (the fp32  */
+/* gradient addition inside the GEMM epilogue).  The mathematics is the chain  */
+/* rule through the forward above, with the routing decisions (which experts   */
+/* a token picked) held fixed: they are a selection, not a differentiable      */
+/* function.  Reading: the bias enters only the selection, so it receives no   */
+/* gradient and contributes none; the logit offset is a constant.             */
+/*   y_t = sum_j g_tj F_ej(x_t) + (sum over zero slots g_tj) x_t                */
+/*   g_tj = scale * s_ej,  s = softmax(W_r x_t + o)                             */
+/*   F(x) = W_d h,  h = silu(a) * b,  a = W_g x,  b = W_u x                      */
+/* Given dy: dF = g dy;  dg_tj = <dy, F(x)> (FFN) or <dy, x> (zero);            */
+/*   dh = W_d^T dF;  da = dh * b * silu'(a);  db = dh * silu(a);               */
+/*   silu'(a) = sig(a) (1 + a (1 - sig(a)));                                    */
+/*   dW_d += dF h^T;  dW_g += da x^T;  dW_u += db x^T;                           */
+/*   dx += W_g^T da + W_u^T db (FFN slots) + g dy (zero slots);                  */
+/*   ds_e = scale * dg (the slot that picked e);  dl = s * (ds - <s, ds>);      */
+/*   dW_r += dl x^T;  dx += W_r^T dl.                                          */
+/* Pinned by central finite differences in tests/test_oracle_pins.py.         */
+/* Gradients are ADDED into dwr [E,d], dwg [N,inter,d], dwu, dwd [N,d,inter]; */
+/* dx [T,d] is written.  s [T,E] are the softmax scores of the forward.       */
+/* ------------------------------------------------------------------------- */
+ZO_EXPORT void zo_layer_bwd_f64(const void *x, int x_dtype, int64_t T, int d, int E, int N, int k, int inter,
+                                const void *wr, const void *wg, const void *wu, const void *wd, int w_dtype,
+                                const int32_t *idx, const double *s, double scale, const double *dy, double *dx,
+                                double *dwr, double *dwg, double *dwu, double *dwd) {
+  double *xv = (double *)malloc(sizeof(double) * (size_t)d);
+  double *a = (double *)malloc(sizeof(double) * (size_t)inter), *b = (double *)malloc(sizeof(double) * (size_t)inter);
+  double *hh = (double *)malloc(sizeof(double) * (size_t)inter), *dh = (double *)malloc(sizeof(double) * (size_t)inter);
+  double *F = (double *)malloc(sizeof(double) * (size_t)d), *dF = (double *)malloc(sizeof(double) * (size_t)d);
+  double *ds = (double *)malloc(sizeof(double) * (size_t)E), *dl = (double *)malloc(sizeof(double) * (size_t)E);
+  const int64_t wsz = (int64_t)inter * d;
+  for (int64_t t = 0; t < T; ++t) {
+    const double *dyt = dy + t * d;
+    double *dxt = dx + t * d;
+    for (int c = 0; c < d; ++c) {
+      xv[c] = elem(x, x_dtype, t * d + c);
+      dxt[c] = 0.0;
+    }
+    for (int e = 0; e < E; ++e) ds[e] = 0.0;
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[t * k + j];
+      const double g = scale * s[t * E + e];
+      if (e >= N) { /* zero expert: F(x) = x */
+        double dg = 0.0;
+        for (int c = 0; c < d; ++c) {
+          dg += dyt[c] * xv[c];
+          dxt[c] += g * dyt[c];
+        }
+        ds[e] += scale * dg;
+        continue;
+      }
+      const int64_t eo = (int64_t)e * wsz;
+      for (int i = 0; i < inter; ++i) {
+        double av = 0.0, bv = 0.0;
+        for (int c = 0; c < d; ++c) {
+          av += elem(wg, w_dtype, eo + (int64_t)i * d + c) * xv[c];
+          bv += elem(wu, w_dtype, eo + (int64_t)i * d + c) * xv[c];
+        }
+        a[i] = av;
+        b[i] = bv;
+        hh[i] = av / (1.0 + exp(-av)) * bv;
+      }
+      double dg = 0.0;
+      for (int c = 0; c < d; ++c) {
+        double f = 0.0;
+        for (int i = 0; i < inter; ++i) f += elem(wd, w_dtype, eo + (int64_t)c * inter + i) * hh[i];
+        F[c] = f;
+        dg += dyt[c] * f;
+        dF[c] = g * dyt[c];
+      }
+      ds[e] += scale * dg;
+      for (int i = 0; i < inter; ++i) {
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c) acc += elem(wd, w_dtype, eo + (int64_t)c * inter + i) * dF[c];
+        dh[i] = acc;
+      }
+      for (int c = 0; c < d; ++c)
+        for (int i = 0; i < inter; ++i) dwd[eo + (int64_t)c * inter + i] += dF[c] * hh[i];
+      for (int i = 0; i < inter; ++i) {
+        const double sg = 1.0 / (1.0 + exp(-a[i]));
+        const double da = dh[i] * b[i] * sg * (1.0 + a[i] * (1.0 - sg));
+        const double db = dh[i] * a[i] * sg;
+        for (int c = 0; c < d; ++c) {
+          dwg[eo + (int64_t)i * d + c] += da * xv[c];
+          dwu[eo + (int64_t)i * d + c] += db * xv[c];
+          dxt[c] += elem(wg, w_dtype, eo + (int64_t)i * d + c) * da + elem(wu, w_dtype, eo + (int64_t)i * d + c) * db;
+        }
+      }
+    }
+    /* router: softmax Jacobian */
+    double sds = 0.0;
+    for (int e = 0; e < E; ++e) sds += s[t * E + e] * ds[e];
+    for (int e = 0; e < E; ++e) dl[e] = s[t * E + e] * (ds[e] - sds);
+    for (int e = 0; e < E; ++e)
+      for (int c = 0; c < d; ++c) {
+        dwr[(int64_t)e * d + c] += dl[e] * xv[c];
+        dxt[c] += elem(wr, w_dtype, (int64_t)e * d + c) * dl[e];
+      }
+  }
+  free(xv);
+  free(a);
+  free(b);
+  free(hh);
+  free(dh);
+  free(F);
+  free(dF);
+  free(ds);
+  free(dl);
+}

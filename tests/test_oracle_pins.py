@@ -572,3 +572,91 @@ def test_ffn_fp4_is_close_to_the_unquantized_expert():
     y = oracle.ffn(x, wg, wu, wd)
     rel = np.abs(y4 - y).max(axis=1) / np.abs(y).max(axis=1)
     assert 1e-3 < rel.max() < 0.35, rel
+
+
+# ---------------------------------------------------------------- backward (oracle only)
+
+def _tiny_fwd_loss(x, wr, wg, wu, wd, bias, dy, N, k, scale, offset):
+    l = oracle.router_logits(x, wr, offset)
+    s = oracle.softmax(l)
+    idx, gate, _ = oracle.topk(s, bias, k, scale)
+    y = oracle.layer(x, idx, gate, N, wg, wu, wd)
+    return float((y * dy).sum()), idx, s
+
+
+def test_backward_against_central_differences():
+    """Every gradient of the fp64 backward (x, W_r, W_g, W_u, W_d) agrees with central
+    differences of <dy, y(x, W)> on a tiny layer, the routing held by small steps
+    (checked: the same experts are picked on both sides of every step)."""
+    rng = np.random.default_rng(31)
+    T, d, N, Z, k, inter, scale = 5, 16, 3, 2, 3, 8, 1.7
+    E = N + Z
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    wr = (rng.standard_normal((E, d)) * 0.4).astype(np.float32)
+    wg = (rng.standard_normal((N, inter, d)) * 0.3).astype(np.float32)
+    wu = (rng.standard_normal((N, inter, d)) * 0.3).astype(np.float32)
+    wd = (rng.standard_normal((N, d, inter)) * 0.3).astype(np.float32)
+    bias = rng.uniform(-0.05, 0.05, E)
+    offset = rng.uniform(-0.1, 0.1, E).astype(np.float32)
+    dy = rng.standard_normal((T, d))
+    params = {"x": x, "wr": wr, "wg": wg, "wu": wu, "wd": wd}
+    L0, idx0, s0 = _tiny_fwd_loss(x, wr, wg, wu, wd, bias, dy, N, k, scale, offset)
+    grads = dict(zip(params, oracle.layer_backward(x, idx0, s0, scale, dy, N, wr, wg, wu, wd)))
+    checked = 0
+    for name, arr in params.items():
+        flat = arr.reshape(-1)
+        for i in rng.choice(flat.size, size=min(12, flat.size), replace=False):
+            v = float(flat[i])
+            hp, hm = np.float32(v + 1e-2), np.float32(v - 1e-2)
+            flat[i] = hp
+            Lp, idxp, _ = _tiny_fwd_loss(params["x"], params["wr"], params["wg"], params["wu"], params["wd"], bias, dy,
+                                         N, k, scale, offset)
+            flat[i] = hm
+            Lm, idxm, _ = _tiny_fwd_loss(params["x"], params["wr"], params["wg"], params["wu"], params["wd"], bias, dy,
+                                         N, k, scale, offset)
+            flat[i] = np.float32(v)
+            if not (np.array_equal(idxp, idx0) and np.array_equal(idxm, idx0)):
+                continue  # the step changed a selection; this coordinate is not differentiable here
+            fd = (Lp - Lm) / (float(hp) - float(hm))
+            an = float(grads[name].reshape(-1)[i])
+            assert abs(fd - an) <= 2e-4 * max(1.0, abs(an)), (name, int(i), fd, an)
+            checked += 1
+    assert checked >= 50
+
+
+def test_backward_bias_gets_no_gradient_and_zero_experts_pass_dy():
+    """With only zero experts chosen the layer is y = (sum of their gates) x: dx = zsum dy
+    plus the router term; the bias never appears in any gradient formula (it only
+    selects), so moving it without changing the selection changes no gradient."""
+    rng = np.random.default_rng(32)
+    T, d, N, Z, k, inter = 3, 8, 2, 4, 2, 8
+    E = N + Z
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    wr = (rng.standard_normal((E, d)) * 0.3).astype(np.float32)
+    wg = rng.standard_normal((N, inter, d)).astype(np.float32)
+    wu = rng.standard_normal((N, inter, d)).astype(np.float32)
+    wd = rng.standard_normal((N, d, inter)).astype(np.float32)
+    bias = np.zeros(E)
+    bias[N:] = 5.0   # every pick is a zero expert
+    dy = rng.standard_normal((T, d))
+    l = oracle.router_logits(x, wr)
+    s = oracle.softmax(l)
+    idx, gate, _ = oracle.topk(s, bias, k, 1.0)
+    assert (idx >= N).all()
+    g1 = oracle.layer_backward(x, idx, s, 1.0, dy, N, wr, wg, wu, wd)
+    assert not g1[2].any() and not g1[3].any() and not g1[4].any()   # no FFN expert ran
+    zsum = gate.sum(axis=1)
+    dl_part = g1[0] - zsum[:, None] * dy
+    # the remaining dx is the router's W_r^T dl, with dl = s * (ds - <s, ds>), ds_e = <dy, x> on picked e
+    ds = np.zeros((T, E))
+    for t in range(T):
+        for j in range(k):
+            ds[t, idx[t, j]] += float(dy[t] @ x[t].astype(np.float64))
+    dl = s * (ds - (s * ds).sum(axis=1, keepdims=True))
+    assert np.allclose(dl_part, dl @ wr.astype(np.float64), rtol=1e-12, atol=1e-12)
+    bias2 = bias.copy()
+    bias2[N:] = 7.0
+    idx2, _, _ = oracle.topk(s, bias2, k, 1.0)
+    assert np.array_equal(idx2, idx)
+    g2 = oracle.layer_backward(x, idx2, s, 1.0, dy, N, wr, wg, wu, wd)
+    assert all(np.array_equal(a_, b_) for a_, b_ in zip(g1, g2))
