@@ -228,6 +228,27 @@ ZCMOE_API int zcmoe_route_noalloc(const float *logits, const float *bias, int64_
 /* Frees the handle's own memory; never touches the borrowed weights.  NULL is a no-op. */
 ZCMOE_API int zcmoe_destroy(zcmoe_t h);
 
+/* Backward pass of the last zcmoe_forward on this handle (training), bf16 layers.
+ * LongCat-Flash technical summary (zhangjingwei.cn), 五 訓練基礎設施: the weight
+ * gradients use a fused GemmAdd (each GEMM adds its fp32 product into the
+ * gradient accumulator in its epilogue) and the input gradient a deterministic
+ * ScatterAdd (a per-token sum in slot order: the same bits on every run).
+ * The chain rule runs through the forward with its routing held fixed (the
+ * selection is not differentiable); the bias only selects and gets no
+ * gradient, nor does the logit offset.
+ *   x  [T, d] device bf16: the tensor the last forward read, unchanged;
+ *   dy [T, d] device bf16: the gradient of the loss with respect to y;
+ *   dx [T, d] device bf16: written;
+ *   g_router [E, d], g_gate [N, inter, d], g_up [N, inter, d], g_down [N, d, inter]:
+ *      device fp32 accumulators, caller-owned; the gradients are ADDED into them;
+ *      NULL skips that weight gradient.
+ * T must equal the last forward's T.  The first call allocates the backward's
+ * workspace (about (6 d + 4 inter) * 2 bytes per padded row plus [T, E] and
+ * [T, d] buffers).  Returns ZCMOE_EUNSUPPORTED for FP32 / FP8 / FP4 layers.
+ * Asynchronous on `stream`. */
+ZCMOE_API int zcmoe_backward(zcmoe_t h, const void *x, const void *dy, int64_t T, void *dx, float *g_router,
+                             float *g_gate, float *g_up, float *g_down, cudaStream_t stream);
+
 /* Block quantization to FP8 E4M3 with E8M0 scales, the rule ZCMOE_FP8 layers use
  * (round to nearest even; scale 2^E the smallest power of two with the block's
  * largest magnitude <= 448 * 2^E, E + 127 clamped to [0, 254]; an all-zero block

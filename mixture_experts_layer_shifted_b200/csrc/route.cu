@@ -145,6 +145,71 @@ __global__ void __launch_bounds__(256) k_softmax_topk(const float* __restrict__ 
   }
 }
 
+// Router backward, one warp per token: the scores s are recomputed from the
+// saved logits exactly as k_softmax_topk computes them; ds_e = scale * dg of the
+// slot that picked e (0 for experts not picked); dl = s * (ds - <s, ds>), bf16
+// into dl [T, ld].  The bias only selected and gets no gradient.
+template <int EPL>
+__global__ void __launch_bounds__(256) k_router_bwd(const float* __restrict__ logits, int T, int E, int k,
+                                                    float scale, const int32_t* __restrict__ idx,
+                                                    const float* __restrict__ dg, __nv_bfloat16* __restrict__ dl,
+                                                    int ld) {
+  const int lane = threadIdx.x & 31;
+  const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
+  for (int t = warp; t < T; t += nwarps) {
+    const float* lt = logits + (int64_t)t * E;
+    float l[EPL];
+    float m = -__int_as_float(0x7f800000);
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      l[i] = e < E ? lt[e] : -__int_as_float(0x7f800000);
+      m = fmaxf(m, l[i]);
+    }
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, w));
+    float u[EPL];
+    float acc = 0.0f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      u[i] = 0.0f;
+      if (e < E) {
+        u[i] = zexp(__fsub_rn(l[i], m));
+        acc = __fadd_rn(acc, u[i]);
+      }
+    }
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, w));
+    float ds[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      u[i] = __fdiv_rn(u[i], acc);
+      ds[i] = 0.0f;
+    }
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(int64_t)t * k + j];
+      if ((e & 31) == lane) {
+        const float v = scale * dg[(int64_t)t * k + j];
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+          if (i == (e >> 5)) ds[i] = v;
+      }
+    }
+    float dot = 0.0f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) dot = fmaf(u[i], ds[i], dot);
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, w);
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < ld) dl[(int64_t)t * ld + e] = __float2bfloat16_rn(e < E ? u[i] * (ds[i] - dot) : 0.0f);
+    }
+  }
+}
+
 // Integer stage, part 1: per block of 256 tokens, one 32-bit token mask per
 // (warp, expert) in shared memory; writes the block's per-expert counts.
 __global__ void __launch_bounds__(kChunk) k_route_count(const int32_t* __restrict__ idx, int T, int k, int E,
@@ -512,6 +577,21 @@ cudaError_t launch_combine(int bf16, const void* x, const void* Y, const int32_t
 
 cudaError_t launch_selftest_wait(int* err, uint64_t limit_ns, cudaStream_t s) {
   k_selftest_wait<<<1, 32, 0, s>>>(err, limit_ns);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_bwd(const float* logits, int T, int E, int k, float scale, const int32_t* idx,
+                              const float* dg, __nv_bfloat16* dl, int ld, int sms, cudaStream_t s) {
+  const int warps = T;
+  int blocks = (warps + 7) / 8;
+  if (blocks > sms * 16) blocks = sms * 16;
+  if (blocks < 1) blocks = 1;
+  // ld >= E, rounded up to 64; each lane covers experts lane, lane + 32, ... < 32 * EPL
+  if (ld <= 128) k_router_bwd<4><<<blocks, 256, 0, s>>>(logits, T, E, k, scale, idx, dg, dl, ld);
+  else if (ld <= 256) k_router_bwd<8><<<blocks, 256, 0, s>>>(logits, T, E, k, scale, idx, dg, dl, ld);
+  else if (ld <= 512) k_router_bwd<16><<<blocks, 256, 0, s>>>(logits, T, E, k, scale, idx, dg, dl, ld);
+  else if (ld <= 1024) k_router_bwd<32><<<blocks, 256, 0, s>>>(logits, T, E, k, scale, idx, dg, dl, ld);
+  else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 

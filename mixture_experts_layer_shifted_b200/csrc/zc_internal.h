@@ -105,6 +105,47 @@ int fp8_block_n(int mode);
 cudaError_t launch_fp8_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                             const Fp8Args& args, int grid, cudaStream_t s);
 
+// ------------------------------------------------------------- backward data movement (moe_bwd.cu, route.cu)
+cudaError_t launch_router_bwd(const float* logits, int T, int E, int k, float scale, const int32_t* idx,
+                              const float* dg, __nv_bfloat16* dl, int ld, int sms, cudaStream_t s);
+cudaError_t launch_gather_pad(const void* x, int d, const int32_t* perm, int k, const int32_t* row_off,
+                              const int32_t* mb_off, int N, void* xpad, void* dypad, int sms, cudaStream_t s);
+cudaError_t launch_combine_bwd(const void* x, const void* dy, const void* Y, const float* gate, const int32_t* pos,
+                               const int32_t* idx, const int32_t* offsets, const int32_t* mb_off, int T, int k, int d,
+                               void* dypad, float* dg, cudaStream_t s);
+cudaError_t launch_final_dx(const void* dy, const void* dxp, const void* dxr, const float* gate, const int32_t* pos,
+                            const int32_t* idx, const int32_t* offsets, const int32_t* mb_off, int T, int k, int d,
+                            void* dx, cudaStream_t s);
+
+// ------------------------------------------------------------- backward GEMMs (gemm_bwd.cu)
+enum BwdSched { kSchedRows = 0, kSchedWgrad = 1 };
+enum BwdEpi { kEpiBf16 = 0, kEpiSwigluBwd = 1, kEpiAddF32 = 2 };
+enum BwdKind { kBwdRowsMnB = 0, kBwdSwiglu = 1, kBwdWgrad = 2 };
+
+struct BwdArgs {
+  int K;                     // kSchedRows: reduction length (a multiple of 64)
+  int n_out, nblocks;        // output columns, 256-column tiles
+  int m_out, mblocks;        // kSchedWgrad: output rows, 128-row tiles
+  int ngroups;               // experts (1 for the router)
+  const int32_t* row_off;    // [ngroups+1] pair offsets
+  const int32_t* mb_off;     // [ngroups+1] row-block offsets (expert g's rows start at padded row 128 mb_off[g])
+  int a_col0;                // first A column (K offset for K-major A, M offset for MN-major A)
+  int64_t b_row_per_group;   // B row offset per expert (K-major B: rows; MN-major B: K rows)
+  int k_split;               // MN-major B: K rows [0, k_split) from tmB0, the rest from tmB1 (INT_MAX: none)
+  void* out;                 // kEpiBf16: bf16 [padded rows, ldo]
+  int64_t ldo;
+  const __nv_bfloat16* dh;   // kEpiSwigluBwd: dH [padded rows, inter]
+  __nv_bfloat16* dgu;        //   out: [dG | dU] [padded rows, 2 inter]
+  __nv_bfloat16* hpad;       //   out: H [padded rows, inter]
+  int inter;
+  float* acc;                // kEpiAddF32: acc[g * acc_group_stride + m * acc_ld + n] += product
+  int64_t acc_ld, acc_group_stride;
+  int* err;                  // device error word (bounded waits)
+};
+int bwd_smem_bytes();
+cudaError_t launch_bwd_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                            const BwdArgs& args, int grid, cudaStream_t s);
+
 // ------------------------------------------------------------- fp32 CUDA-core GEMM (gemm_simt.cu)
 struct SimtArgs {
   const float* A;

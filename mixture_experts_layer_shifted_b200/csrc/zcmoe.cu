@@ -101,6 +101,20 @@ int make_tmap_esz(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t ou
 int make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
   return make_tmap_esz(tm, base, inner, outer, box_outer, 2);
 }
+// bf16 [outer, inner] with a row stride of ld elements (ld >= inner, ld * 2 a multiple of 16)
+int make_tmap_ld(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer, uint64_t ld) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(ZCMOE_ECUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ZCMOE_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return ZCMOE_OK;
+}
 
 template <typename T>
 int dalloc(T** p, size_t n) {
@@ -152,6 +166,13 @@ struct zcmoe_s {
   uint8_t *w8g, *w8u, *w8d, *sfg, *sfu, *sfd, *x8, *sx, *h8, *sh;
   void* ypad;
   CUtensorMap tm8_wg, tm8_wu, tm8_wd, tm8_x, tm8_h;
+  // zcmoe_backward (allocated on its first call): padded X, dY, dH, [dG|dU], H, dX
+  // rows; dg [T*k]; dl [T, dl_ld] bf16; router dx [T, d]; the router's one-group offsets
+  int last_T;
+  int dl_ld;
+  void *b_xpad, *b_dypad, *b_dh, *b_dgu, *b_hpad, *b_dxp, *b_dl, *b_dxr;
+  float* b_dg;
+  int32_t* b_grp;
   bool alive;
 };
 
@@ -160,7 +181,8 @@ static void release(zcmoe_s* h) {
                   h->err,   h->logits, h->gate,   h->idx,   h->pos,     h->counts, h->offsets,
                   h->mb_off, h->scal,  h->chunk,  h->perm,  h->xperm,   h->H,      h->Y,
                   h->stage_x, h->stage_x2, h->stage_y, h->w8g, h->w8u, h->w8d, h->sfg, h->sfu, h->sfd,
-                  h->x8, h->sx, h->h8, h->sh, h->ypad};
+                  h->x8, h->sx, h->h8, h->sh, h->ypad, h->b_xpad, h->b_dypad, h->b_dh, h->b_dgu, h->b_hpad,
+                  h->b_dxp, h->b_dl, h->b_dxr, h->b_dg, h->b_grp};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (int i = 0; i < 2; ++i) {
@@ -466,6 +488,7 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
 
   const int Ti = (int)T, E = h->E, N = h->N, k = h->k, d = h->d, inter = h->inter;
   const int nchunks = (Ti + zc::kChunk - 1) / zc::kChunk;
+  h->last_T = Ti;
   auto mark = [&]() -> cudaError_t {
     if (!h->profiling) return cudaSuccess;
     cudaEvent_t ev;
@@ -838,6 +861,180 @@ int zcmoe_destroy(zcmoe_t h) {
   cudaDeviceSynchronize();
   release(h);
   delete h;
+  return ZCMOE_OK;
+}
+
+int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx, float* g_router, float* g_gate,
+                   float* g_up, float* g_down, cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (!h->bf16 || h->fp8) return fail(ZCMOE_EUNSUPPORTED, "the backward pass needs a bf16 layer");
+  if (T < 0 || T > h->max_T) return fail(ZCMOE_ERANGE, "T=%lld outside [0, %d]", (long long)T, h->max_T);
+  if (T == 0) return ZCMOE_OK;
+  if (T != h->last_T) return fail(ZCMOE_EINVAL, "T=%lld differs from the last forward's %d", (long long)T, h->last_T);
+  if (!x || !dy || !dx) return fail(ZCMOE_EINVAL, "x, dy or dx is NULL");
+  const void* bufs[3] = {x, dy, dx};
+  for (const void* p : bufs)
+    if (reinterpret_cast<uintptr_t>(p) & 15u) return fail(ZCMOE_EINVAL, "x, dy and dx must be 16-byte aligned");
+  const size_t nb = (size_t)T * h->d * 2;
+  if (overlaps(dx, nb, x, nb) || overlaps(dx, nb, dy, nb)) return fail(ZCMOE_EINVAL, "dx overlaps x or dy");
+  if (h->d > 24576) return fail(ZCMOE_EUNSUPPORTED, "the backward pass supports d <= 24576");
+  const int Ti = (int)T, E = h->E, N = h->N, k = h->k, d = h->d, inter = h->inter;
+  const size_t prow = (size_t)h->max_mblocks * zc::kBM;
+  if (!h->b_xpad) {
+    h->dl_ld = (E + 63) / 64 * 64;
+    int rc = ZCMOE_OK;
+    uint8_t *a = nullptr, *b = nullptr, *c = nullptr, *e2 = nullptr, *f = nullptr, *g = nullptr, *l = nullptr,
+            *r = nullptr;
+    rc = dalloc(&a, prow * d * 2);
+    if (rc == ZCMOE_OK) rc = dalloc(&b, prow * d * 2);
+    if (rc == ZCMOE_OK) rc = dalloc(&c, prow * inter * 2);
+    if (rc == ZCMOE_OK) rc = dalloc(&e2, prow * inter * 4);
+    if (rc == ZCMOE_OK) rc = dalloc(&f, prow * inter * 2);
+    if (rc == ZCMOE_OK) rc = dalloc(&g, prow * d * 2);
+    if (rc == ZCMOE_OK) rc = dalloc(&l, (size_t)h->max_T * h->dl_ld * 2);
+    if (rc == ZCMOE_OK) rc = dalloc(&r, (size_t)h->max_T * d * 2);
+    if (rc == ZCMOE_OK) rc = dalloc(&h->b_dg, (size_t)h->max_pairs);
+    if (rc == ZCMOE_OK) rc = dalloc(&h->b_grp, 4);
+    h->b_xpad = a;
+    h->b_dypad = b;
+    h->b_dh = c;
+    h->b_dgu = e2;
+    h->b_hpad = f;
+    h->b_dxp = g;
+    h->b_dl = l;
+    h->b_dxr = r;
+    if (rc != ZCMOE_OK) {
+      void* ps[] = {h->b_xpad, h->b_dypad, h->b_dh, h->b_dgu, h->b_hpad, h->b_dxp, h->b_dl, h->b_dxr, h->b_dg, h->b_grp};
+      for (void* p : ps)
+        if (p) cudaFree(p);
+      h->b_xpad = h->b_dypad = h->b_dh = h->b_dgu = h->b_hpad = h->b_dxp = h->b_dl = h->b_dxr = nullptr;
+      h->b_dg = nullptr;
+      h->b_grp = nullptr;
+      return rc;
+    }
+  }
+  const uint64_t P = prow;
+  CUtensorMap tm_dy_k, tm_wd_mn, tm_x_k, tm_dgu_k, tm_wg_mn, tm_wu_mn, tm_dl_k, tm_wr_mn;
+  CUtensorMap tm_dy_mn, tm_h_mn, tm_dgu_mn, tm_x_mn, tm_dl_mn, tm_xin_mn;
+  int rc = make_tmap(&tm_dy_k, h->b_dypad, d, P, 128);
+  if (rc == ZCMOE_OK) rc = make_tmap(&tm_wd_mn, h->w.w_down, inter, (uint64_t)N * d, 64);
+  if (rc == ZCMOE_OK) rc = make_tmap(&tm_x_k, h->b_xpad, d, P, 128);
+  if (rc == ZCMOE_OK) rc = make_tmap(&tm_dgu_k, h->b_dgu, 2 * (uint64_t)inter, P, 128);
+  if (rc == ZCMOE_OK) rc = make_tmap(&tm_wg_mn, h->w.w_gate, d, (uint64_t)N * inter, 64);
+  if (rc == ZCMOE_OK) rc = make_tmap(&tm_wu_mn, h->w.w_up, d, (uint64_t)N * inter, 64);
+  if (rc == ZCMOE_OK) rc = make_tmap_ld(&tm_dl_k, h->b_dl, E, T, 128, h->dl_ld);
+  if (rc == ZCMOE_OK) rc = make_tmap(&tm_wr_mn, h->w.w_router, d, E, 64);
+  if (rc == ZCMOE_OK) rc = make_tmap(&tm_dy_mn, h->b_dypad, d, P, 64);
+  if (rc == ZCMOE_OK) rc = make_tmap(&tm_h_mn, h->b_hpad, inter, P, 64);
+  if (rc == ZCMOE_OK) rc = make_tmap(&tm_dgu_mn, h->b_dgu, 2 * (uint64_t)inter, P, 64);
+  if (rc == ZCMOE_OK) rc = make_tmap(&tm_x_mn, h->b_xpad, d, P, 64);
+  if (rc == ZCMOE_OK) rc = make_tmap_ld(&tm_dl_mn, h->b_dl, E, T, 64, h->dl_ld);
+  if (rc == ZCMOE_OK) rc = make_tmap(&tm_xin_mn, x, d, T, 64);
+  if (rc != ZCMOE_OK) return rc;
+  const int max_mb = (Ti * k + zc::kBM - 1) / zc::kBM + N;
+  auto grid_for = [&](int64_t tiles) { return (int)(tiles < h->sms ? (tiles < 1 ? 1 : tiles) : h->sms); };
+  auto rows_args = [&]() {
+    zc::BwdArgs a{};
+    a.ngroups = N;
+    a.row_off = h->offsets;
+    a.mb_off = h->mb_off;
+    a.k_split = 0x7fffffff;
+    a.err = h->err;
+    return a;
+  };
+
+  // routing-side backward and the padded operands
+  ZC_CUDA(zc::launch_single_group(h->b_grp, h->b_grp + 2, Ti, s));
+  ZC_CUDA(zc::launch_gather_pad(x, d, h->perm, k, h->offsets, h->mb_off, N, h->b_xpad, h->b_dypad, h->sms, s));
+  ZC_CUDA(zc::launch_combine_bwd(x, dy, h->Y, h->gate, h->pos, h->idx, h->offsets, h->mb_off, Ti, k, d, h->b_dypad,
+                                 h->b_dg, s));
+  ZC_CUDA(zc::launch_router_bwd(h->logits, Ti, E, k, h->cfg.routed_scale, h->idx, h->b_dg,
+                                static_cast<__nv_bfloat16*>(h->b_dl), h->dl_ld, h->sms, s));
+  // dH = dY W_d
+  {
+    zc::BwdArgs a = rows_args();
+    a.K = d;
+    a.n_out = inter;
+    a.nblocks = (inter + 255) / 256;
+    a.b_row_per_group = d;
+    a.out = h->b_dh;
+    a.ldo = inter;
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dy_k, tm_wd_mn, tm_wd_mn, a, grid_for((int64_t)max_mb * a.nblocks),
+                                s));
+  }
+  // [G|U] recomputed from X; SwiGLU backward -> dG, dU; H
+  {
+    zc::BwdArgs a = rows_args();
+    a.K = d;
+    a.n_out = inter;
+    a.nblocks = (inter + 127) / 128;
+    a.b_row_per_group = inter;
+    a.dh = static_cast<const __nv_bfloat16*>(h->b_dh);
+    a.dgu = static_cast<__nv_bfloat16*>(h->b_dgu);
+    a.hpad = static_cast<__nv_bfloat16*>(h->b_hpad);
+    a.inter = inter;
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdSwiglu, tm_x_k, h->tm_wg, h->tm_wu, a, grid_for((int64_t)max_mb * a.nblocks),
+                                s));
+  }
+  // dX = [dG|dU] [W_g; W_u]
+  {
+    zc::BwdArgs a = rows_args();
+    a.K = 2 * inter;
+    a.k_split = inter;
+    a.n_out = d;
+    a.nblocks = (d + 255) / 256;
+    a.b_row_per_group = inter;
+    a.out = h->b_dxp;
+    a.ldo = d;
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dgu_k, tm_wg_mn, tm_wu_mn, a,
+                                grid_for((int64_t)max_mb * a.nblocks), s));
+  }
+  // router: dx_router = dl W_r
+  {
+    zc::BwdArgs a{};
+    a.ngroups = 1;
+    a.row_off = h->b_grp;
+    a.mb_off = h->b_grp + 2;
+    a.k_split = 0x7fffffff;
+    a.err = h->err;
+    a.K = h->dl_ld;
+    a.n_out = d;
+    a.nblocks = (d + 255) / 256;
+    a.b_row_per_group = 0;
+    a.out = h->b_dxr;
+    a.ldo = d;
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dl_k, tm_wr_mn, tm_wr_mn, a,
+                                grid_for((int64_t)((Ti + 127) / 128) * a.nblocks), s));
+  }
+  // dx: the deterministic ScatterAdd
+  ZC_CUDA(zc::launch_final_dx(dy, h->b_dxp, h->b_dxr, h->gate, h->pos, h->idx, h->offsets, h->mb_off, Ti, k, d, dx, s));
+  // weight gradients, added into the fp32 accumulators in the GEMM epilogue
+  auto wgrad = [&](const CUtensorMap& A, const CUtensorMap& B, int a_col0, int m_out, int n_out, float* acc,
+                   int64_t stride, int groups, const int32_t* row_off, const int32_t* mb_off) -> int {
+    zc::BwdArgs a{};
+    a.ngroups = groups;
+    a.row_off = row_off;
+    a.mb_off = mb_off;
+    a.a_col0 = a_col0;
+    a.m_out = m_out;
+    a.mblocks = (m_out + 127) / 128;
+    a.n_out = n_out;
+    a.nblocks = (n_out + 255) / 256;
+    a.acc = acc;
+    a.acc_ld = n_out;
+    a.acc_group_stride = stride;
+    a.err = h->err;
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdWgrad, A, B, B, a, grid_for((int64_t)groups * a.mblocks * a.nblocks), s));
+    return ZCMOE_OK;
+  };
+  if (g_down && (rc = wgrad(tm_dy_mn, tm_h_mn, 0, d, inter, g_down, (int64_t)d * inter, N, h->offsets, h->mb_off)))
+    return rc;
+  if (g_gate && (rc = wgrad(tm_dgu_mn, tm_x_mn, 0, inter, d, g_gate, (int64_t)inter * d, N, h->offsets, h->mb_off)))
+    return rc;
+  if (g_up && (rc = wgrad(tm_dgu_mn, tm_x_mn, inter, inter, d, g_up, (int64_t)inter * d, N, h->offsets, h->mb_off)))
+    return rc;
+  if (g_router && (rc = wgrad(tm_dl_mn, tm_xin_mn, 0, E, d, g_router, 0, 1, h->b_grp, h->b_grp + 2))) return rc;
   return ZCMOE_OK;
 }
 

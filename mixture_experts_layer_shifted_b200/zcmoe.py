@@ -35,7 +35,7 @@ EXPORTED = ("zcmoe_create", "zcmoe_forward", "zcmoe_forward_host", "zcmoe_update
             "zcmoe_write_counts", "zcmoe_get_state", "zcmoe_set_bias", "zcmoe_check", "zcmoe_profile_begin",
             "zcmoe_profile_end", "zcmoe_selftest_wait", "zcmoe_route_noalloc", "zcmoe_destroy",
             "zcmoe_dense_create", "zcmoe_dense_forward", "zcmoe_forward_overlap", "zcmoe_dense_check",
-            "zcmoe_dense_destroy", "zcmoe_quantize_e4m3", "zcmoe_quantize_mx4", "zcmoe_last_error")
+            "zcmoe_dense_destroy", "zcmoe_quantize_e4m3", "zcmoe_quantize_mx4", "zcmoe_backward", "zcmoe_last_error")
 STAGES = ("router", "softmax_topk", "integer", "gather", "gate_up", "down", "combine")
 
 
@@ -109,6 +109,7 @@ def lib():
         L.zcmoe_dense_check.argtypes = [vp]
         L.zcmoe_quantize_e4m3.argtypes = [vp, ctypes.c_int32, i64, i64, ctypes.c_int32, vp, vp, vp]
         L.zcmoe_quantize_mx4.argtypes = [vp, ctypes.c_int32, i64, i64, vp, vp, vp]
+        L.zcmoe_backward.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, vp, vp]
         L.zcmoe_dense_destroy.argtypes = [vp]
         for f in EXPORTED[:-1]:
             getattr(L, f).restype = i32
@@ -241,6 +242,11 @@ def quantize_e4m3(src, block_rows, stream=None):
     return codes, scales
 
 
+def zcmoe_backward(h, x_ptr, dy_ptr, T, dx_ptr, g_router=None, g_gate=None, g_up=None, g_down=None, stream=None):
+    _check(lib().zcmoe_backward(h, x_ptr, dy_ptr, T, dx_ptr, g_router, g_gate, g_up, g_down, _stream(stream)),
+           "zcmoe_backward")
+
+
 def zcmoe_quantize_mx4(src_ptr, src_dtype, rows, cols, codes_ptr, scales_ptr, stream=None):
     _check(lib().zcmoe_quantize_mx4(src_ptr, src_dtype, rows, cols, codes_ptr, scales_ptr, _stream(stream)),
            "zcmoe_quantize_mx4")
@@ -321,6 +327,16 @@ class ZcMoE:
         zcmoe_forward_host(self.h, ctypes.c_void_p(x_host.data_ptr()), x_host.shape[0],
                            ctypes.c_void_p(y_host.data_ptr()), stream)
         return y_host
+
+    def backward(self, x, dy, dx=None, grads: dict | None = None, stream=None):
+        """dx of the last forward (x must be the tensor it read); adds the weight gradients
+        into the fp32 tensors of ``grads`` (keys router, gate, up, down; missing: skipped)."""
+        dx = torch.empty_like(x) if dx is None else dx
+        g = grads or {}
+        ptr = lambda name: ctypes.c_void_p(g[name].data_ptr()) if name in g else None  # noqa: E731
+        zcmoe_backward(self.h, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(dy.data_ptr()), x.shape[0],
+                       ctypes.c_void_p(dx.data_ptr()), ptr("router"), ptr("gate"), ptr("up"), ptr("down"), stream)
+        return dx
 
     def update_bias(self, kp=0.0, ki=0.0, kd=0.0, decay=1.0, target_ffn_per_token=None, stream=None):
         K = float(self.shape.top_k if target_ffn_per_token is None else target_ffn_per_token)

@@ -83,7 +83,7 @@ def lib():
         L.zo_ffn_fp4_f64.argtypes = [vp, i32, i64, U8P, U8P, U8P, U8P, U8P, U8P, i32, i32, F64P]
         L.zo_ffn_fp4_f64.restype = None
         L.zo_layer_bwd_f64.argtypes = [vp, i32, i64, i32, i32, i32, i32, i32, vp, vp, vp, vp, i32, I32P, F64P, f64,
-                                       F64P, F64P, F64P, F64P, F64P, F64P]
+                                       F64P, F64P, vp, vp, vp, vp]
         L.zo_layer_bwd_f64.restype = None
         L.zo_ffn_f64.argtypes = [vp, i32, i64, vp, vp, vp, i32, i32, i32, F64P]
         L.zo_ffn_f64.restype = None
@@ -366,10 +366,11 @@ def ffn_fp4(xs, wq, sq):
 
 
 # ----------------------------------------------------------------- backward (training)
-def layer_backward(x, idx, scores, scale, dy, N, wr, wg, wu, wd):
+def layer_backward(x, idx, scores, scale, dy, N, wr, wg, wu, wd, weights=True):
     """fp64 gradients of the layer for fixed routing: returns (dx [T,d], dW_r [E,d],
-    dW_g [N,inter,d], dW_u [N,inter,d], dW_d [N,d,inter]).  scores [T,E] are the
-    forward's softmax scores; the bias and the logit offset get no gradient."""
+    dW_g [N,inter,d], dW_u [N,inter,d], dW_d [N,d,inter]); weights=False computes dx
+    only (the others are None).  scores [T,E] are the forward's softmax scores; the
+    bias and the logit offset get no gradient."""
     x, xd = _arr(x)
     wr, gd = _arr(wr)
     wg, _ = _arr(wg)
@@ -379,10 +380,12 @@ def layer_backward(x, idx, scores, scale, dy, N, wr, wg, wu, wd):
     E = wr.shape[0]
     inter = wg.shape[1]
     k = idx.shape[1]
-    out = [np.zeros((T, d)), np.zeros((E, d)), np.zeros((N, inter, d)), np.zeros((N, inter, d)),
-           np.zeros((N, d, inter))]
+    dx = np.zeros((T, d))
+    ws = [np.zeros((E, d)), np.zeros((N, inter, d)), np.zeros((N, inter, d)), np.zeros((N, d, inter))] if weights \
+        else [None] * 4
     lib().zo_layer_bwd_f64(x.ctypes.data, xd, T, d, E, N, k, inter, wr.ctypes.data, wg.ctypes.data, wu.ctypes.data,
                            wd_.ctypes.data, gd, np.ascontiguousarray(idx, np.int32),
                            np.ascontiguousarray(scores, np.float64), float(scale),
-                           np.ascontiguousarray(dy, np.float64), *out)
-    return tuple(out)
+                           np.ascontiguousarray(dy, np.float64), dx,
+                           *[None if w_ is None else w_.ctypes.data for w_ in ws])
+    return (dx, *ws)

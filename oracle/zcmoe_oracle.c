@@ -644,8 +644,9 @@ ZO_EXPORT void zo_ffn_fp4_f64(const void *xs, int x_dtype, int64_t n, const uint
 /*   ds_e = scale * dg (the slot that picked e);  dl = s * (ds - <s, ds>);      */
 /*   dW_r += dl x^T;  dx += W_r^T dl.                                          */
 /* Pinned by central finite differences in tests/test_oracle_pins.py.         */
-/* Gradients are ADDED into dwr [E,d], dwg [N,inter,d], dwu, dwd [N,d,inter]; */
-/* dx [T,d] is written.  s [T,E] are the softmax scores of the forward.       */
+/* Gradients are ADDED into dwr [E,d], dwg [N,inter,d], dwu, dwd [N,d,inter] */
+/* (each may be NULL: skipped); dx [T,d] is written.  s [T,E] are the softmax */
+/* scores of the forward.                                                     */
 /* ------------------------------------------------------------------------- */
 ZO_EXPORT void zo_layer_bwd_f64(const void *x, int x_dtype, int64_t T, int d, int E, int N, int k, int inter,
                                 const void *wr, const void *wg, const void *wu, const void *wd, int w_dtype,
@@ -702,15 +703,16 @@ ZO_EXPORT void zo_layer_bwd_f64(const void *x, int x_dtype, int64_t T, int d, in
         for (int c = 0; c < d; ++c) acc += elem(wd, w_dtype, eo + (int64_t)c * inter + i) * dF[c];
         dh[i] = acc;
       }
-      for (int c = 0; c < d; ++c)
-        for (int i = 0; i < inter; ++i) dwd[eo + (int64_t)c * inter + i] += dF[c] * hh[i];
+      if (dwd)
+        for (int c = 0; c < d; ++c)
+          for (int i = 0; i < inter; ++i) dwd[eo + (int64_t)c * inter + i] += dF[c] * hh[i];
       for (int i = 0; i < inter; ++i) {
         const double sg = 1.0 / (1.0 + exp(-a[i]));
         const double da = dh[i] * b[i] * sg * (1.0 + a[i] * (1.0 - sg));
         const double db = dh[i] * a[i] * sg;
         for (int c = 0; c < d; ++c) {
-          dwg[eo + (int64_t)i * d + c] += da * xv[c];
-          dwu[eo + (int64_t)i * d + c] += db * xv[c];
+          if (dwg) dwg[eo + (int64_t)i * d + c] += da * xv[c];
+          if (dwu) dwu[eo + (int64_t)i * d + c] += db * xv[c];
           dxt[c] += elem(wg, w_dtype, eo + (int64_t)i * d + c) * da + elem(wu, w_dtype, eo + (int64_t)i * d + c) * db;
         }
       }
@@ -721,7 +723,7 @@ ZO_EXPORT void zo_layer_bwd_f64(const void *x, int x_dtype, int64_t T, int d, in
     for (int e = 0; e < E; ++e) dl[e] = s[t * E + e] * (ds[e] - sds);
     for (int e = 0; e < E; ++e)
       for (int c = 0; c < d; ++c) {
-        dwr[(int64_t)e * d + c] += dl[e] * xv[c];
+        if (dwr) dwr[(int64_t)e * d + c] += dl[e] * xv[c];
         dxt[c] += elem(wr, w_dtype, (int64_t)e * d + c) * dl[e];
       }
   }
