@@ -343,6 +343,35 @@ def measure_lowp(layer, weights, x, stream, peaks, fmt="fp8"):
     return out
 
 
+def measure_backward(wl, layer, x, stream, peaks, P):
+    """zcmoe_backward after a forward of the same batch: dx only, and dx plus the four
+    weight gradients added into fp32 accumulators (fused GemmAdd); each a replayed graph."""
+    import torch
+    g = torch.Generator(device=x.device).manual_seed(11)
+    dy = (torch.randn(x.shape, generator=g, device=x.device) * 0.05).to(torch.bfloat16)
+    dx = torch.empty_like(x)
+    y = torch.empty_like(x)
+    grads = {"router": torch.zeros((wl.E, wl.d), device=x.device),
+             "gate": torch.zeros((wl.n_ffn, wl.inter, wl.d), device=x.device),
+             "up": torch.zeros((wl.n_ffn, wl.inter, wl.d), device=x.device),
+             "down": torch.zeros((wl.n_ffn, wl.d, wl.inter), device=x.device)}
+    layer.forward(x, y)
+    ms_dx = graph_ms(lambda: layer.backward(x, dy, dx), stream)
+    ms_full = graph_ms(lambda: layer.backward(x, dy, dx, grads=grads), stream, reps=3)
+    layer.check()
+    ok = all(bool(torch.isfinite(t).all()) for t in grads.values())
+    del grads
+    torch.cuda.empty_cache()
+    dpi = float(wl.d) * wl.inter * P
+    f_dx = 10.0 * dpi + 2.0 * wl.T * wl.E * wl.d      # dH, [G|U] recompute, dX, router dx
+    f_w = 6.0 * dpi + 2.0 * wl.T * wl.E * wl.d        # dW_d, dW_g, dW_u, dW_r
+    acc_bytes = 8.0 * (3 * wl.n_ffn * wl.inter * wl.d + wl.E * wl.d)  # fp32 read + write of the accumulators
+    return {"ms_dx_only": ms_dx, "ms_with_weight_grads": ms_full, "tflops_dx_only": f_dx / (ms_dx * 1e-3) / 1e12,
+            "tflops_total": (f_dx + f_w) / (ms_full * 1e-3) / 1e12, "gemmadd_accumulator_bytes": acc_bytes,
+            "gemmadd_hbm_ms": 1e3 * acc_bytes / (peaks["hbm_gbs"] * 1e9), "finite": ok,
+            "note": "weight gradients added into fp32 accumulators (3 x 25.8 GB + router); each a replayed graph"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -556,6 +585,10 @@ def main():
     if rank == 0 and ws == 1 and not args.no_secondary and wl.name == "prefill_560b":
         line["fp8"] = measure_lowp(layer, weights, xs[0], stream, peaks, "fp8")
         line["fp4"] = measure_lowp(layer, weights, xs[0], stream, peaks, "fp4")
+
+    # secondary: the backward pass (training) of the same batch
+    if rank == 0 and ws == 1 and not args.no_secondary and wl.dtype == "bf16":
+        line["backward"] = measure_backward(wl, layer, xs[0], stream, peaks, P)
 
     # secondary: the dense FFN path run beside the layer (shortcut-connected MoE)
     if rank == 0 and ws == 1 and not args.no_secondary and wl.dense_inter > 0:

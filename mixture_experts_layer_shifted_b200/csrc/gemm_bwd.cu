@@ -41,7 +41,8 @@ constexpr uint32_t B_BYTES = BN * BK * 2;
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr uint32_t STG_BYTES = 32 * 32 * 4;       // GemmAdd staging: 32 rows x 32 fp32 per warp and buffer
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 4 * 2 * STG_BYTES + 256;
 
 struct Tile {
   int64_t a_row;   // SCHED_ROWS: first padded A row; SCHED_WGRAD: first K row (padded token row)
@@ -98,6 +99,19 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr) {
          ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
 }
 
+// TMA reduce-add of a 32 x 32 fp32 box (128-byte swizzled in shared memory) into
+// the accumulator at (n, m, g); completion tracked as a bulk group of this thread.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* tm, const void* src, int n, int m, int g) {
+  asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(smem_u32(src)), "r"(n), "r"(m), "r"(g)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -107,12 +121,14 @@ __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(
 template <int SCHED, bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-               const __grid_constant__ CUtensorMap tmB1, const BwdArgs args) {
+               const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmC,
+               const BwdArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint8_t* sStg = sB + STAGES * B_BYTES;  // 1024-aligned: [warp quarter][buffer] of STG_BYTES
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + 4 * 2 * STG_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -256,6 +272,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
+    int chunk = 0;  // kEpiAddF32: reduce-adds issued by this warp (selects the staging buffer)
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const Tile ti = decode_tile<SCHED>(args, t);
       if (ti.num_k == 0) continue;
@@ -337,32 +354,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       } else {
-        // fused GemmAdd: acc[g][m][n] += product, fp32
-        const int m = ti.m_blk * BM + row;
-        float* base = args.acc + (int64_t)ti.g * args.acc_group_stride + (int64_t)m * args.acc_ld;
+        // fused GemmAdd: acc[g][m][n] += product in fp32, done by TMA reduce-adds of
+        // 32 x 32 boxes (the L2 does the read-modify-write; each element is added once)
+        const int m0 = ti.m_blk * BM + quarter * 32;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t r[32];
           tmem_ld32(tbase + c, r);
           tc_wait_ld();
           const int n0 = ti.n_blk * BN + c;
-          if (m >= args.m_out || n0 >= args.n_out) continue;
-          float* p = base + n0;
-          if (n0 + 32 <= args.n_out) {
+          if (m0 >= args.m_out || n0 >= args.n_out) continue;
+          uint8_t* stg = sStg + (quarter * 2 + (chunk & 1)) * STG_BYTES;
+          if (lane == 0) bulk_wait_read_1();  // the reduce two chunks back has read this buffer
+          __syncwarp();
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              float4 v = reinterpret_cast<float4*>(p)[q];
-              v.x += __uint_as_float(r[4 * q + 0]);
-              v.y += __uint_as_float(r[4 * q + 1]);
-              v.z += __uint_as_float(r[4 * q + 2]);
-              v.w += __uint_as_float(r[4 * q + 3]);
-              reinterpret_cast<float4*>(p)[q] = v;
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (n0 + i < args.n_out) p[i] += __uint_as_float(r[i]);
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_3d(&tmC, stg, n0, m0, ti.g);
+            bulk_commit();
           }
+          ++chunk;
         }
       }
       tc_fence_before();
@@ -372,6 +387,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         acc_phase ^= 1u;
       }
     }
+    if (EPI == kEpiAddF32 && lane == 0) bulk_wait_all();  // every reduce-add complete before exit
   }
 
   tc_fence_before();
@@ -383,8 +399,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 template <int SCHED, bool A_MN, bool B_MN, int EPI>
-cudaError_t launch_variant(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const BwdArgs& args,
-                           int grid, cudaStream_t s) {
+cudaError_t launch_variant(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& c,
+                           const BwdArgs& args, int grid, cudaStream_t s) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(k_bwd_gemm<SCHED, A_MN, B_MN, EPI>,
@@ -392,7 +408,7 @@ cudaError_t launch_variant(const CUtensorMap& a, const CUtensorMap& b0, const CU
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k_bwd_gemm<SCHED, A_MN, B_MN, EPI><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, args);
+  k_bwd_gemm<SCHED, A_MN, B_MN, EPI><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, c, args);
   return cudaGetLastError();
 }
 
@@ -401,14 +417,14 @@ cudaError_t launch_variant(const CUtensorMap& a, const CUtensorMap& b0, const CU
 int bwd_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t launch_bwd_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                            const BwdArgs& args, int grid, cudaStream_t s) {
+                            const CUtensorMap& c, const BwdArgs& args, int grid, cudaStream_t s) {
   switch (kind) {
     case kBwdRowsMnB:  // dH, dX, router dx: A K-major, B MN-major, bf16 out
-      return launch_variant<kSchedRows, false, true, kEpiBf16>(a, b0, b1, args, grid, s);
+      return launch_variant<kSchedRows, false, true, kEpiBf16>(a, b0, b1, c, args, grid, s);
     case kBwdSwiglu:  // gate/up recompute + SwiGLU backward
-      return launch_variant<kSchedRows, false, false, kEpiSwigluBwd>(a, b0, b1, args, grid, s);
+      return launch_variant<kSchedRows, false, false, kEpiSwigluBwd>(a, b0, b1, c, args, grid, s);
     case kBwdWgrad:  // weight gradients, fused GemmAdd
-      return launch_variant<kSchedWgrad, true, true, kEpiAddF32>(a, b0, b1, args, grid, s);
+      return launch_variant<kSchedWgrad, true, true, kEpiAddF32>(a, b0, b1, c, args, grid, s);
     default:
       return cudaErrorInvalidValue;
   }

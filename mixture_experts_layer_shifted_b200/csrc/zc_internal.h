@@ -138,13 +138,15 @@ struct BwdArgs {
   __nv_bfloat16* dgu;        //   out: [dG | dU] [padded rows, 2 inter]
   __nv_bfloat16* hpad;       //   out: H [padded rows, inter]
   int inter;
-  float* acc;                // kEpiAddF32: acc[g * acc_group_stride + m * acc_ld + n] += product
+  float* acc;                // kEpiAddF32: acc[g][m][n] += product (through the tensor map c)
   int64_t acc_ld, acc_group_stride;
   int* err;                  // device error word (bounded waits)
 };
 int bwd_smem_bytes();
+// c: kBwdWgrad only -- the fp32 accumulator as a 3-D tensor [groups][m_out][n_out], box 32 x 32 x 1,
+// 128-byte swizzle (the reduce-add target); other kinds ignore it.
 cudaError_t launch_bwd_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                            const BwdArgs& args, int grid, cudaStream_t s);
+                            const CUtensorMap& c, const BwdArgs& args, int grid, cudaStream_t s);
 
 // ------------------------------------------------------------- fp32 CUDA-core GEMM (gemm_simt.cu)
 struct SimtArgs {

@@ -101,6 +101,22 @@ int make_tmap_esz(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t ou
 int make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
   return make_tmap_esz(tm, base, inner, outer, box_outer, 2);
 }
+// fp32 gradient accumulator [groups][rows][cols] as a 3-D tensor, box 32 x 32 x 1,
+// 128-byte swizzle: the target of the backward's TMA reduce-adds (cols a multiple of 4)
+int make_tmap_acc(CUtensorMap* tm, const float* base, uint64_t cols, uint64_t rows, uint64_t groups) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(ZCMOE_ECUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0) return fail(ZCMOE_EINVAL, "gradient not 16-byte aligned");
+  cuuint64_t dims[3] = {cols, rows, groups};
+  cuuint64_t strides[2] = {cols * 4, cols * rows * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ZCMOE_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return ZCMOE_OK;
+}
 // bf16 [outer, inner] with a row stride of ld elements (ld >= inner, ld * 2 a multiple of 16)
 int make_tmap_ld(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer, uint64_t ld) {
   EncodeTiledFn enc = encode_fn();
@@ -960,7 +976,7 @@ int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx
     a.b_row_per_group = d;
     a.out = h->b_dh;
     a.ldo = inter;
-    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dy_k, tm_wd_mn, tm_wd_mn, a, grid_for((int64_t)max_mb * a.nblocks),
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dy_k, tm_wd_mn, tm_wd_mn, tm_dy_k, a, grid_for((int64_t)max_mb * a.nblocks),
                                 s));
   }
   // [G|U] recomputed from X; SwiGLU backward -> dG, dU; H
@@ -974,7 +990,7 @@ int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx
     a.dgu = static_cast<__nv_bfloat16*>(h->b_dgu);
     a.hpad = static_cast<__nv_bfloat16*>(h->b_hpad);
     a.inter = inter;
-    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdSwiglu, tm_x_k, h->tm_wg, h->tm_wu, a, grid_for((int64_t)max_mb * a.nblocks),
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdSwiglu, tm_x_k, h->tm_wg, h->tm_wu, tm_x_k, a, grid_for((int64_t)max_mb * a.nblocks),
                                 s));
   }
   // dX = [dG|dU] [W_g; W_u]
@@ -987,7 +1003,7 @@ int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx
     a.b_row_per_group = inter;
     a.out = h->b_dxp;
     a.ldo = d;
-    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dgu_k, tm_wg_mn, tm_wu_mn, a,
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dgu_k, tm_wg_mn, tm_wu_mn, tm_dgu_k, a,
                                 grid_for((int64_t)max_mb * a.nblocks), s));
   }
   // router: dx_router = dl W_r
@@ -1004,7 +1020,7 @@ int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx
     a.b_row_per_group = 0;
     a.out = h->b_dxr;
     a.ldo = d;
-    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dl_k, tm_wr_mn, tm_wr_mn, a,
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dl_k, tm_wr_mn, tm_wr_mn, tm_dl_k, a,
                                 grid_for((int64_t)((Ti + 127) / 128) * a.nblocks), s));
   }
   // dx: the deterministic ScatterAdd
@@ -1025,7 +1041,10 @@ int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx
     a.acc_ld = n_out;
     a.acc_group_stride = stride;
     a.err = h->err;
-    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdWgrad, A, B, B, a, grid_for((int64_t)groups * a.mblocks * a.nblocks), s));
+    CUtensorMap tmc;
+    const int rc2 = make_tmap_acc(&tmc, acc, (uint64_t)n_out, (uint64_t)m_out, (uint64_t)groups);
+    if (rc2 != ZCMOE_OK) return rc2;
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdWgrad, A, B, B, tmc, a, grid_for((int64_t)groups * a.mblocks * a.nblocks), s));
     return ZCMOE_OK;
   };
   if (g_down && (rc = wgrad(tm_dy_mn, tm_h_mn, 0, d, inter, g_down, (int64_t)d * inter, N, h->offsets, h->mb_off)))
