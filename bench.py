@@ -381,9 +381,15 @@ def main():
     ap.add_argument("--impl", default="zcmoe", choices=["zcmoe", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--secondary", default="decode,fp8,fp4,backward,overlap",
+                    help="comma list of the secondary measurements to run after the headline")
     ap.add_argument("--eager", action="store_true",
                     help="launch every step eagerly instead of replaying one captured CUDA graph (N=1)")
     args = ap.parse_args()
+    sec = set() if args.no_secondary else {s_.strip() for s_ in args.secondary.split(",") if s_.strip()}
+    unknown = sec - {"decode", "fp8", "fp4", "backward", "overlap"}
+    if unknown:
+        ap.error(f"unknown secondary measurement(s): {sorted(unknown)}")
     if args.warmup < 3:
         args.warmup = 3
 
@@ -554,7 +560,7 @@ def main():
             "launch": "cuda graph per step" if use_graph else "eager"}
 
     # secondary workload (decode): reported beside the headline, not as the headline
-    if rank == 0 and ws == 1 and not args.no_secondary and wl.name == "prefill_560b":
+    if rank == 0 and ws == 1 and "decode" in sec and wl.name == "prefill_560b":
         wd = configs.WORKLOADS["decode_560b"]
         xd = configs.device_tokens(wd)
         layer2 = ZcMoE(LayerShape(wd.d, wd.n_ffn, wd.n_zero, wd.inter, wd.top_k, wd.dtype), *weights,
@@ -582,16 +588,17 @@ def main():
         layer2.close()
 
     # secondary: the same layer with block-scaled FP8 experts (bf16 headline unchanged)
-    if rank == 0 and ws == 1 and not args.no_secondary and wl.name == "prefill_560b":
-        line["fp8"] = measure_lowp(layer, weights, xs[0], stream, peaks, "fp8")
-        line["fp4"] = measure_lowp(layer, weights, xs[0], stream, peaks, "fp4")
+    if rank == 0 and ws == 1 and wl.name == "prefill_560b":
+        for fmt in ("fp8", "fp4"):
+            if fmt in sec:
+                line[fmt] = measure_lowp(layer, weights, xs[0], stream, peaks, fmt)
 
     # secondary: the backward pass (training) of the same batch
-    if rank == 0 and ws == 1 and not args.no_secondary and wl.dtype == "bf16":
+    if rank == 0 and ws == 1 and "backward" in sec and wl.dtype == "bf16":
         line["backward"] = measure_backward(wl, layer, xs[0], stream, peaks, P)
 
     # secondary: the dense FFN path run beside the layer (shortcut-connected MoE)
-    if rank == 0 and ws == 1 and not args.no_secondary and wl.dense_inter > 0:
+    if rank == 0 and ws == 1 and "overlap" in sec and wl.dense_inter > 0:
         line["scmoe_overlap"] = measure_overlap(wl, layer, xs[0], stream, peaks)
 
     layer.close()
