@@ -344,32 +344,42 @@ def measure_lowp(layer, weights, x, stream, peaks, fmt="fp8"):
 
 
 def measure_backward(wl, layer, x, stream, peaks, P):
-    """zcmoe_backward after a forward of the same batch: dx only, and dx plus the four
-    weight gradients added into fp32 accumulators (fused GemmAdd); each a replayed graph."""
+    """zcmoe_backward after a forward of the same batch, in training mode (the forward
+    stores G and U; the backward reads them): dx only, and dx plus the four weight
+    gradients added into fp32 accumulators (fused GemmAdd); each a replayed graph.
+    Also the recomputing backward (training mode off) and the forward's cost of storing."""
     import torch
     g = torch.Generator(device=x.device).manual_seed(11)
     dy = (torch.randn(x.shape, generator=g, device=x.device) * 0.05).to(torch.bfloat16)
     dx = torch.empty_like(x)
     y = torch.empty_like(x)
+    layer.forward(x, y)
+    ms_dx_recompute = graph_ms(lambda: layer.backward(x, dy, dx), stream)
+    ms_fwd = graph_ms(lambda: layer.forward(x, y), stream)
+    layer.save_for_backward(True)
+    ms_fwd_saving = graph_ms(lambda: layer.forward(x, y), stream)
+    layer.forward(x, y)
+    ms_dx = graph_ms(lambda: layer.backward(x, dy, dx), stream)
     grads = {"router": torch.zeros((wl.E, wl.d), device=x.device),
              "gate": torch.zeros((wl.n_ffn, wl.inter, wl.d), device=x.device),
              "up": torch.zeros((wl.n_ffn, wl.inter, wl.d), device=x.device),
              "down": torch.zeros((wl.n_ffn, wl.d, wl.inter), device=x.device)}
-    layer.forward(x, y)
-    ms_dx = graph_ms(lambda: layer.backward(x, dy, dx), stream)
     ms_full = graph_ms(lambda: layer.backward(x, dy, dx, grads=grads), stream, reps=3)
     layer.check()
     ok = all(bool(torch.isfinite(t).all()) for t in grads.values())
     del grads
+    layer.save_for_backward(False)
     torch.cuda.empty_cache()
     dpi = float(wl.d) * wl.inter * P
-    f_dx = 10.0 * dpi + 2.0 * wl.T * wl.E * wl.d      # dH, [G|U] recompute, dX, router dx
+    f_dx = 6.0 * dpi + 2.0 * wl.T * wl.E * wl.d       # dH, dX, router dx
     f_w = 6.0 * dpi + 2.0 * wl.T * wl.E * wl.d        # dW_d, dW_g, dW_u, dW_r
     acc_bytes = 8.0 * (3 * wl.n_ffn * wl.inter * wl.d + wl.E * wl.d)  # fp32 read + write of the accumulators
     return {"ms_dx_only": ms_dx, "ms_with_weight_grads": ms_full, "tflops_dx_only": f_dx / (ms_dx * 1e-3) / 1e12,
             "tflops_total": (f_dx + f_w) / (ms_full * 1e-3) / 1e12, "gemmadd_accumulator_bytes": acc_bytes,
             "gemmadd_hbm_ms": 1e3 * acc_bytes / (peaks["hbm_gbs"] * 1e9), "finite": ok,
-            "note": "weight gradients added into fp32 accumulators (3 x 25.8 GB + router); each a replayed graph"}
+            "ms_dx_only_recompute": ms_dx_recompute, "ms_forward": ms_fwd, "ms_forward_saving_gu": ms_fwd_saving,
+            "note": "training mode (forward stores G, U); weight gradients added into fp32 accumulators "
+                    "(3 x 25.8 GB + router); each a replayed graph"}
 
 
 def main():

@@ -249,6 +249,18 @@ ZCMOE_API int zcmoe_destroy(zcmoe_t h);
 ZCMOE_API int zcmoe_backward(zcmoe_t h, const void *x, const void *dy, int64_t T, void *dx, float *g_router,
                              float *g_gate, float *g_up, float *g_down, cudaStream_t stream);
 
+/* Training mode for zcmoe_backward, bf16 layers.  on = 1: every later forward also
+ * stores the gate/up GEMM's outputs G = X W_g^T and U = X W_u^T of its FFN pairs
+ * (rounded to bf16; 4 * inter bytes per padded pair row, allocated here, about
+ * 2.1 GB at T 16384, k 12, 512 experts, inter 2048), and a backward after such a
+ * forward reads them instead of recomputing them (one GEMM fewer: the SwiGLU
+ * backward runs in the dH GEMM's epilogue).  on = 0: forwards store nothing and
+ * the backward recomputes G and U; the buffer is freed.  Call it outside stream
+ * capture, with no forward or backward of this handle in flight.  Returns
+ * ZCMOE_EUNSUPPORTED for FP32 / FP8 / FP4 layers, ZCMOE_ENOMEM if the buffer
+ * cannot be allocated (training mode then stays off). */
+ZCMOE_API int zcmoe_save_for_backward(zcmoe_t h, int32_t on);
+
 /* Block quantization to FP8 E4M3 with E8M0 scales, the rule ZCMOE_FP8 layers use
  * (round to nearest even; scale 2^E the smallest power of two with the block's
  * largest magnitude <= 448 * 2^E, E + 127 clamped to [0, 254]; an all-zero block

@@ -8,7 +8,8 @@
 // drain TMEM, two 256-column accumulators) serves every contraction:
 //
 //   SCHED_ROWS  (rows of an expert's tokens x output columns, K fixed):
-//     dH  = dY W_d                 A dY (K-major)      B W_d (MN-major)          -> bf16
+//     dH  = dY W_d                 A dY (K-major)      B W_d (MN-major)          -> bf16, or (the forward
+//                                  saved G and U) the SwiGLU backward in the epilogue -> dG, dU, H
 //     [G|U] = X [W_g; W_u]^T       A X  (K-major)      B W_g / W_u (K-major)     -> SwiGLU backward epilogue
 //     dX  = [dG|dU] [W_g; W_u]     A dGU (K-major)     B W_g then W_u (MN-major) -> bf16
 //     dx_router = dl W_r           A dl (K-major)      B W_r (MN-major)          -> bf16
@@ -353,6 +354,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ho[q] = vh;
           }
         }
+      } else if (EPI == kEpiSwigluSaved) {
+        // the accumulator is dH (fp32, 256 columns); g and u are the forward's saved values
+        const bool row_ok = row < ti.rows_valid;
+        const int64_t grow = ti.a_row + row;
+        const int inter = args.inter;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tbase + c, r);
+          tc_wait_ld();
+          const int col0 = ti.n_blk * BN + c;
+          if (col0 >= inter) continue;
+          const uint4* gi = reinterpret_cast<const uint4*>(args.gu + grow * 2 * inter + col0);
+          const uint4* ui = reinterpret_cast<const uint4*>(args.gu + grow * 2 * inter + inter + col0);
+          uint4* dgo = reinterpret_cast<uint4*>(args.dgu + grow * 2 * inter + col0);
+          uint4* duo = reinterpret_cast<uint4*>(args.dgu + grow * 2 * inter + inter + col0);
+          uint4* ho = reinterpret_cast<uint4*>(args.hpad + grow * inter + col0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 vdg = make_uint4(0, 0, 0, 0), vdu = vdg, vh = vdg;
+            if (row_ok) {
+              const uint4 g8 = gi[q], u8 = ui[q];
+              const uint32_t gw[4] = {g8.x, g8.y, g8.z, g8.w}, uw[4] = {u8.x, u8.y, u8.z, u8.w};
+              uint32_t* pdg = &vdg.x;
+              uint32_t* pdu = &vdu.x;
+              uint32_t* ph = &vh.x;
+#pragma unroll
+              for (int w = 0; w < 4; ++w) {
+                const float2 g2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[w]));
+                const float2 u2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uw[w]));
+                float da[2], db[2], hv[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const float gv = e ? g2.y : g2.x, uv = e ? u2.y : u2.x;
+                  const float dhv = __uint_as_float(r[8 * q + 2 * w + e]);
+                  const float sg = __fdividef(1.0f, 1.0f + __expf(-gv));
+                  da[e] = dhv * uv * sg * (1.0f + gv * (1.0f - sg));
+                  db[e] = dhv * gv * sg;
+                  hv[e] = silu_mul(gv, uv);
+                }
+                pdg[w] = pack_bf16(da[0], da[1]);
+                pdu[w] = pack_bf16(db[0], db[1]);
+                ph[w] = pack_bf16(hv[0], hv[1]);
+              }
+            }
+            dgo[q] = vdg;
+            duo[q] = vdu;
+            ho[q] = vh;
+          }
+        }
       } else {
         // fused GemmAdd: acc[g][m][n] += product in fp32, done by TMA reduce-adds of
         // 32 x 32 boxes (the L2 does the read-modify-write; each element is added once)
@@ -425,6 +476,8 @@ cudaError_t launch_bwd_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b
       return launch_variant<kSchedRows, false, false, kEpiSwigluBwd>(a, b0, b1, c, args, grid, s);
     case kBwdWgrad:  // weight gradients, fused GemmAdd
       return launch_variant<kSchedWgrad, true, true, kEpiAddF32>(a, b0, b1, c, args, grid, s);
+    case kBwdDhSwiglu:  // dH = dY W_d with the SwiGLU backward on the forward's saved G, U
+      return launch_variant<kSchedRows, false, true, kEpiSwigluSaved>(a, b0, b1, c, args, grid, s);
     default:
       return cudaErrorInvalidValue;
   }

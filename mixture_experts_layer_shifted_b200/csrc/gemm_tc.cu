@@ -3,6 +3,7 @@
 // One persistent kernel serves the three dense contractions of the layer:
 //   router : logits[T, E]        = x[T, d] . W_r[E, d]^T (+ per-expert logit offset), fp32 out
 //   gate/up: H[p, inter]         = silu(X_e W_g,e^T) * (X_e W_u,e^T) for the rows p of expert e, bf16 out
+//            (training: also G and U themselves, rounded to bf16, for the backward)
 //   down   : Y[p, d]             = H_e W_d,e^T, bf16 out
 // (LongCat-Flash technical summary, zhangjingwei.cn, 二 架構 / 模型配置: each FFN
 // expert is 2048 wide on a 6144 hidden size; the per-expert GEMMs run as one
@@ -45,6 +46,7 @@ struct Tile {
   int rows_valid;  // rows of the tile that belong to it
   int b_row;       // first B row
   int n_blk;       // output column tile
+  int p_row;       // grouped modes: the tile's first row in the padded layout (128 (mb_off[g] + row block))
 };
 
 template <int MODE>
@@ -62,6 +64,7 @@ __device__ __forceinline__ Tile decode_tile(const TcArgs& a, int t) {
     ti.a_row = m_blk * BM;
     ti.rows_valid = min(BM, a.M - ti.a_row);
     ti.b_row = ti.n_blk * BN;
+    ti.p_row = ti.a_row;
     return ti;
   }
   // largest expert g with mb_off[g] * nblocks <= t (it has at least one row block)
@@ -80,6 +83,7 @@ __device__ __forceinline__ Tile decode_tile(const TcArgs& a, int t) {
   const int r0 = a.row_off[g];
   ti.a_row = r0 + m_blk * BM;
   ti.rows_valid = min(BM, a.row_off[g + 1] - ti.a_row);
+  ti.p_row = (mb0 + m_blk) * BM;
   ti.b_row = g * a.b_rows_per_group + ti.n_blk * (MODE == kGateUp ? BN / 2 : BN);
   return ti;
 }
@@ -259,6 +263,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               v.w = pack_bf16(silu_mul(__uint_as_float(g[8 * q + 6]), __uint_as_float(u[8 * q + 6])),
                               silu_mul(__uint_as_float(g[8 * q + 7]), __uint_as_float(u[8 * q + 7])));
               dst[q] = v;
+            }
+            if (args.gu_save) {
+              // training: the pre-activations for the backward, in the padded row layout
+              __nv_bfloat16* gs = static_cast<__nv_bfloat16*>(args.gu_save) +
+                                  ((int64_t)ti.p_row + row_in_tile) * 2 * args.n_out + col0;
+              uint4* gdst = reinterpret_cast<uint4*>(gs);
+              uint4* udst = reinterpret_cast<uint4*>(gs + args.n_out);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                gdst[q] = make_uint4(pack_bf16(__uint_as_float(g[8 * q + 0]), __uint_as_float(g[8 * q + 1])),
+                                     pack_bf16(__uint_as_float(g[8 * q + 2]), __uint_as_float(g[8 * q + 3])),
+                                     pack_bf16(__uint_as_float(g[8 * q + 4]), __uint_as_float(g[8 * q + 5])),
+                                     pack_bf16(__uint_as_float(g[8 * q + 6]), __uint_as_float(g[8 * q + 7])));
+                udst[q] = make_uint4(pack_bf16(__uint_as_float(u[8 * q + 0]), __uint_as_float(u[8 * q + 1])),
+                                     pack_bf16(__uint_as_float(u[8 * q + 2]), __uint_as_float(u[8 * q + 3])),
+                                     pack_bf16(__uint_as_float(u[8 * q + 4]), __uint_as_float(u[8 * q + 5])),
+                                     pack_bf16(__uint_as_float(u[8 * q + 6]), __uint_as_float(u[8 * q + 7])));
+              }
             }
           }
         }

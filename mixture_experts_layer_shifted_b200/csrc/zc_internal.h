@@ -51,6 +51,8 @@ struct TcArgs {
   void* out;                // output matrix
   int64_t ldo;              // its row stride (elements)
   const float* col_add;     // router: per-column offset added to the logits (or null)
+  void* gu_save;            // gate/up, optional: the fp32 accumulators G and U rounded to bf16, stored as
+                            // [G | U] [padded rows, 2 n_out] (expert g's pairs from row 128 mb_off[g] on)
   int* err;                 // device error word (bounded waits)
 };
 
@@ -119,8 +121,8 @@ cudaError_t launch_final_dx(const void* dy, const void* dxp, const void* dxr, co
 
 // ------------------------------------------------------------- backward GEMMs (gemm_bwd.cu)
 enum BwdSched { kSchedRows = 0, kSchedWgrad = 1 };
-enum BwdEpi { kEpiBf16 = 0, kEpiSwigluBwd = 1, kEpiAddF32 = 2 };
-enum BwdKind { kBwdRowsMnB = 0, kBwdSwiglu = 1, kBwdWgrad = 2 };
+enum BwdEpi { kEpiBf16 = 0, kEpiSwigluBwd = 1, kEpiAddF32 = 2, kEpiSwigluSaved = 3 };
+enum BwdKind { kBwdRowsMnB = 0, kBwdSwiglu = 1, kBwdWgrad = 2, kBwdDhSwiglu = 3 };
 
 struct BwdArgs {
   int K;                     // kSchedRows: reduction length (a multiple of 64)
@@ -135,7 +137,8 @@ struct BwdArgs {
   void* out;                 // kEpiBf16: bf16 [padded rows, ldo]
   int64_t ldo;
   const __nv_bfloat16* dh;   // kEpiSwigluBwd: dH [padded rows, inter]
-  __nv_bfloat16* dgu;        //   out: [dG | dU] [padded rows, 2 inter]
+  const __nv_bfloat16* gu;   // kEpiSwigluSaved: the forward's [G | U] [padded rows, 2 inter] (dH is the accumulator)
+  __nv_bfloat16* dgu;        //   out (both SwiGLU epilogues): [dG | dU] [padded rows, 2 inter]
   __nv_bfloat16* hpad;       //   out: H [padded rows, inter]
   int inter;
   float* acc;                // kEpiAddF32: acc[g][m][n] += product (through the tensor map c)

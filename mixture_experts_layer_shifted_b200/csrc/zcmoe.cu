@@ -189,6 +189,10 @@ struct zcmoe_s {
   void *b_xpad, *b_dypad, *b_dh, *b_dgu, *b_hpad, *b_dxp, *b_dl, *b_dxr;
   float* b_dg;
   int32_t* b_grp;
+  // zcmoe_save_for_backward: the forward's [G | U] in padded rows; last_saved tells whether
+  // the last forward wrote it
+  void* b_gu;
+  bool last_saved;
   bool alive;
 };
 
@@ -198,7 +202,7 @@ static void release(zcmoe_s* h) {
                   h->mb_off, h->scal,  h->chunk,  h->perm,  h->xperm,   h->H,      h->Y,
                   h->stage_x, h->stage_x2, h->stage_y, h->w8g, h->w8u, h->w8d, h->sfg, h->sfu, h->sfd,
                   h->x8, h->sx, h->h8, h->sh, h->ypad, h->b_xpad, h->b_dypad, h->b_dh, h->b_dgu, h->b_hpad,
-                  h->b_dxp, h->b_dl, h->b_dxr, h->b_dg, h->b_grp};
+                  h->b_dxp, h->b_dl, h->b_dxr, h->b_dg, h->b_grp, h->b_gu};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (int i = 0; i < 2; ++i) {
@@ -625,7 +629,9 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     a.b_rows_per_group = inter;
     a.out = h->H;
     a.ldo = inter;
+    a.gu_save = h->b_gu;
     a.err = h->err;
+    h->last_saved = h->b_gu != nullptr;
     int bound = max_mb * a.nblocks;
     ZC_CUDA(zc::launch_tc_gemm(zc::kGateUp, h->tm_xperm, h->tm_wg, h->tm_wu, a, bound < h->sms ? bound : h->sms, s));
     ZC_CUDA(mark());
@@ -880,6 +886,27 @@ int zcmoe_destroy(zcmoe_t h) {
   return ZCMOE_OK;
 }
 
+int zcmoe_save_for_backward(zcmoe_t h, int32_t on) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (!h->bf16 || h->fp8) return fail(ZCMOE_EUNSUPPORTED, "training mode needs a bf16 layer");
+  if (!on) {
+    if (h->b_gu) {
+      ZC_CUDA(cudaDeviceSynchronize());
+      cudaFree(h->b_gu);
+      h->b_gu = nullptr;
+    }
+    h->last_saved = false;
+    return ZCMOE_OK;
+  }
+  if (h->b_gu) return ZCMOE_OK;
+  uint8_t* p = nullptr;
+  const int rc = dalloc(&p, (size_t)h->max_mblocks * zc::kBM * h->inter * 4);
+  if (rc != ZCMOE_OK) return rc;
+  h->b_gu = p;
+  return ZCMOE_OK;
+}
+
 int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx, float* g_router, float* g_gate,
                    float* g_up, float* g_down, cudaStream_t s) {
   g_err[0] = 0;
@@ -967,8 +994,22 @@ int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx
                                  h->b_dg, s));
   ZC_CUDA(zc::launch_router_bwd(h->logits, Ti, E, k, h->cfg.routed_scale, h->idx, h->b_dg,
                                 static_cast<__nv_bfloat16*>(h->b_dl), h->dl_ld, h->sms, s));
+  if (h->last_saved) {
+    // dH = dY W_d with the SwiGLU backward in its epilogue, on the forward's G and U
+    zc::BwdArgs a = rows_args();
+    a.K = d;
+    a.n_out = inter;
+    a.nblocks = (inter + 255) / 256;
+    a.b_row_per_group = d;
+    a.gu = static_cast<const __nv_bfloat16*>(h->b_gu);
+    a.dgu = static_cast<__nv_bfloat16*>(h->b_dgu);
+    a.hpad = static_cast<__nv_bfloat16*>(h->b_hpad);
+    a.inter = inter;
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdDhSwiglu, tm_dy_k, tm_wd_mn, tm_wd_mn, tm_dy_k, a,
+                                grid_for((int64_t)max_mb * a.nblocks), s));
+  }
   // dH = dY W_d
-  {
+  if (!h->last_saved) {
     zc::BwdArgs a = rows_args();
     a.K = d;
     a.n_out = inter;
@@ -980,7 +1021,7 @@ int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx
                                 s));
   }
   // [G|U] recomputed from X; SwiGLU backward -> dG, dU; H
-  {
+  if (!h->last_saved) {
     zc::BwdArgs a = rows_args();
     a.K = d;
     a.n_out = inter;

@@ -35,7 +35,8 @@ EXPORTED = ("zcmoe_create", "zcmoe_forward", "zcmoe_forward_host", "zcmoe_update
             "zcmoe_write_counts", "zcmoe_get_state", "zcmoe_set_bias", "zcmoe_check", "zcmoe_profile_begin",
             "zcmoe_profile_end", "zcmoe_selftest_wait", "zcmoe_route_noalloc", "zcmoe_destroy",
             "zcmoe_dense_create", "zcmoe_dense_forward", "zcmoe_forward_overlap", "zcmoe_dense_check",
-            "zcmoe_dense_destroy", "zcmoe_quantize_e4m3", "zcmoe_quantize_mx4", "zcmoe_backward", "zcmoe_last_error")
+            "zcmoe_dense_destroy", "zcmoe_quantize_e4m3", "zcmoe_quantize_mx4", "zcmoe_backward",
+            "zcmoe_save_for_backward", "zcmoe_last_error")
 STAGES = ("router", "softmax_topk", "integer", "gather", "gate_up", "down", "combine")
 
 
@@ -110,6 +111,7 @@ def lib():
         L.zcmoe_quantize_e4m3.argtypes = [vp, ctypes.c_int32, i64, i64, ctypes.c_int32, vp, vp, vp]
         L.zcmoe_quantize_mx4.argtypes = [vp, ctypes.c_int32, i64, i64, vp, vp, vp]
         L.zcmoe_backward.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, vp, vp]
+        L.zcmoe_save_for_backward.argtypes = [vp, ctypes.c_int32]
         L.zcmoe_dense_destroy.argtypes = [vp]
         for f in EXPORTED[:-1]:
             getattr(L, f).restype = i32
@@ -247,6 +249,10 @@ def zcmoe_backward(h, x_ptr, dy_ptr, T, dx_ptr, g_router=None, g_gate=None, g_up
            "zcmoe_backward")
 
 
+def zcmoe_save_for_backward(h, on):
+    _check(lib().zcmoe_save_for_backward(h, 1 if on else 0), "zcmoe_save_for_backward")
+
+
 def zcmoe_quantize_mx4(src_ptr, src_dtype, rows, cols, codes_ptr, scales_ptr, stream=None):
     _check(lib().zcmoe_quantize_mx4(src_ptr, src_dtype, rows, cols, codes_ptr, scales_ptr, _stream(stream)),
            "zcmoe_quantize_mx4")
@@ -337,6 +343,10 @@ class ZcMoE:
         zcmoe_backward(self.h, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(dy.data_ptr()), x.shape[0],
                        ctypes.c_void_p(dx.data_ptr()), ptr("router"), ptr("gate"), ptr("up"), ptr("down"), stream)
         return dx
+
+    def save_for_backward(self, on=True):
+        """Training mode: later forwards store G and U for the backward (no recompute)."""
+        zcmoe_save_for_backward(self.h, on)
 
     def update_bias(self, kp=0.0, ki=0.0, kd=0.0, decay=1.0, target_ffn_per_token=None, stream=None):
         K = float(self.shape.top_k if target_ffn_per_token is None else target_ffn_per_token)

@@ -100,9 +100,11 @@ def _cmp(got, ref, name):
     return float(err.max())
 
 
-def _case(w, T=None, init=0.5):
+def _case(w, T=None, init=0.5, saved=False):
     r = Run(w, T=T, max_tokens=(T or w.T) + 3)
     try:
+        if saved:
+            r.layer.save_for_backward(True)
         r.forward()
         g = torch.Generator(device="cuda").manual_seed(5)
         dy = (torch.randn((r.T, w.d), generator=g, device="cuda") * 0.1).to(torch.bfloat16)
@@ -120,8 +122,9 @@ def _case(w, T=None, init=0.5):
         raise
 
 
-def test_backward_small(cuda_ok):
-    r, _ = _case(W["small_bf16"])
+@pytest.mark.parametrize("saved", [False, True], ids=["recompute", "saved"])
+def test_backward_small(cuda_ok, saved):
+    r, _ = _case(W["small_bf16"], saved=saved)
     r.close()
 
 
@@ -131,18 +134,50 @@ def test_backward_small(cuda_ok):
     (2000, 256, 3, 128, 1, 2),     # several row blocks per expert, partial last block
     (300, 512, 9, 384, 0, 5),      # no zero experts
 ])
-def test_backward_ragged(cuda_ok, T, d, N, inter, Z, k):
+@pytest.mark.parametrize("saved", [False, True], ids=["recompute", "saved"])
+def test_backward_ragged(cuda_ok, T, d, N, inter, Z, k, saved):
     w = configs.Workload("ragged_bwd", T=T, d=d, n_ffn=N, inter=inter, n_zero=Z, top_k=k, dtype="bf16", w_std=0.05,
                          bias=("uniform", -0.05, 0.05), seed=3)
-    r, _ = _case(w)
+    r, _ = _case(w, saved=saved)
     r.close()
 
 
-def test_backward_is_deterministic(cuda_ok):
+def test_saved_activations_leave_the_forward_unchanged(cuda_ok):
+    """Training mode only adds stores: y is bit-identical with and without it, and
+    switching it off again returns to the recomputing backward with the same results
+    within rounding (the saved G and U are bf16, the recomputed ones fp32)."""
+    w = W["small_bf16"]
+    r = Run(w)
+    try:
+        y0 = r.layer.forward(r.x).clone()
+        r.layer.save_for_backward(True)
+        y1 = r.layer.forward(r.x).clone()
+        torch.cuda.synchronize()
+        assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+        dy = (torch.randn((r.T, w.d), device="cuda") * 0.1).to(torch.bfloat16)
+        outs = []
+        for on in (True, False):
+            r.layer.save_for_backward(on)
+            r.layer.forward(r.x)
+            grads = _grads(w, 0.0)
+            dx = _run_backward(r, dy, grads)
+            outs.append((dx.float(), grads))
+        (dx_s, g_s), (dx_r, g_r) = outs
+        assert float((dx_s - dx_r).abs().max()) <= 2e-2 * float(dx_r.abs().max())
+        for k_ in g_s:
+            assert float((g_s[k_] - g_r[k_]).abs().max()) <= 2e-2 * float(g_r[k_].abs().max()), k_
+    finally:
+        r.close()
+
+
+@pytest.mark.parametrize("saved", [False, True], ids=["recompute", "saved"])
+def test_backward_is_deterministic(cuda_ok, saved):
     """Two backward passes of the same forward give the same bits (no atomics anywhere)."""
     w = W["small_bf16"]
     r = Run(w)
     try:
+        if saved:
+            r.layer.save_for_backward(True)
         r.forward(debug=False)
         dy = (torch.randn((r.T, w.d), device="cuda") * 0.1).to(torch.bfloat16)
         outs = []
@@ -162,6 +197,7 @@ def test_backward_prefill_full_size_sampled_rows(cuda_ok):
     w = W["prefill_560b"]
     r = Run(w)
     try:
+        r.layer.save_for_backward(True)  # the configuration the bench times
         r.forward()
         dy = (torch.randn((r.T, w.d), device="cuda") * 0.05).to(torch.bfloat16)
         grads = {"router": torch.zeros((w.E, w.d), device="cuda"),
@@ -195,6 +231,9 @@ def test_backward_argument_checks(cuda_ok):
         f.forward(debug=False)
         with pytest.raises(zcmoe.ZcmoeError) as ei:
             f.layer.backward(f.x, torch.zeros_like(f.x))
+        assert ei.value.code == zcmoe.ZCMOE_EUNSUPPORTED
+        with pytest.raises(zcmoe.ZcmoeError) as ei:
+            f.layer.save_for_backward(True)
         assert ei.value.code == zcmoe.ZCMOE_EUNSUPPORTED
     finally:
         f.close()
