@@ -36,14 +36,24 @@
 namespace zc {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128, BN = 256, BK = 64;
 constexpr uint32_t A_BYTES = BM * BK * 2;
 constexpr uint32_t B_BYTES = BN * BK * 2;
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
-constexpr uint32_t STG_BYTES = 32 * 32 * 4;       // GemmAdd staging: 32 rows x 32 fp32 per warp and buffer
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 4 * 2 * STG_BYTES + 256;
+constexpr uint32_t STG_BYTES = 32 * 32 * 4;  // GemmAdd staging: 32 rows x 32 fp32 per warp and buffer
+
+// Operand stages, and GemmAdd staging buffers per epilogue warp (reduce-adds in flight).
+constexpr int kRowStages = 4;
+constexpr int kWgStages = 4, kWgBufs = 2;
+template <int EPI>
+struct Cfg {
+  static constexpr int kStages = EPI == kEpiAddF32 ? kWgStages : kRowStages;
+  static constexpr int kBufs = EPI == kEpiAddF32 ? kWgBufs : 0;
+  static constexpr int kSmem = 1024 + kStages * STAGE_BYTES + 4 * kBufs * STG_BYTES + 256;
+  static_assert(kSmem <= 232448, "shared memory per block");
+};
 
 struct Tile {
   int64_t a_row;   // SCHED_ROWS: first padded A row; SCHED_WGRAD: first K row (padded token row)
@@ -109,7 +119,10 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* tm, const v
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
@@ -124,12 +137,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_bwd_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmC,
                const BwdArgs args) {
+  constexpr int STAGES = Cfg<EPI>::kStages, NBUF = Cfg<EPI>::kBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
   uint8_t* sStg = sB + STAGES * B_BYTES;  // 1024-aligned: [warp quarter][buffer] of STG_BYTES
-  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + 4 * 2 * STG_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + 4 * NBUF * STG_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -415,8 +429,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_wait_ld();
           const int n0 = ti.n_blk * BN + c;
           if (m0 >= args.m_out || n0 >= args.n_out) continue;
-          uint8_t* stg = sStg + (quarter * 2 + (chunk & 1)) * STG_BYTES;
-          if (lane == 0) bulk_wait_read_1();  // the reduce two chunks back has read this buffer
+          constexpr int NB = NBUF > 0 ? NBUF : 1;  // (NBUF is 0 in the instantiations without GemmAdd)
+          uint8_t* stg = sStg + (quarter * NB + chunk % NB) * STG_BYTES;
+          if (lane == 0) bulk_wait_read<NB - 1>();  // the reduce NB chunks back has read this buffer
           __syncwarp();
 #pragma unroll
           for (int j = 0; j < 8; ++j)
@@ -455,17 +470,17 @@ cudaError_t launch_variant(const CUtensorMap& a, const CUtensorMap& b0, const CU
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(k_bwd_gemm<SCHED, A_MN, B_MN, EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<EPI>::kSmem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k_bwd_gemm<SCHED, A_MN, B_MN, EPI><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, c, args);
+  k_bwd_gemm<SCHED, A_MN, B_MN, EPI><<<grid, NUM_THREADS, Cfg<EPI>::kSmem, s>>>(a, b0, b1, c, args);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-int bwd_smem_bytes() { return SMEM_BYTES; }
+int bwd_smem_bytes() { return Cfg<kEpiAddF32>::kSmem > Cfg<kEpiBf16>::kSmem ? Cfg<kEpiAddF32>::kSmem : Cfg<kEpiBf16>::kSmem; }
 
 cudaError_t launch_bwd_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                             const CUtensorMap& c, const BwdArgs& args, int grid, cudaStream_t s) {

@@ -142,6 +142,28 @@ def test_backward_ragged(cuda_ok, T, d, N, inter, Z, k, saved):
     r.close()
 
 
+@pytest.mark.parametrize("names", [("router",), ("gate", "down"), ()], ids=["router-only", "gate+down", "dx-only"])
+def test_backward_gradient_subsets(cuda_ok, names):
+    """Any subset of the weight gradients (NULL skips one): the requested ones are added,
+    dx is unchanged."""
+    w = W["small_bf16"]
+    r = Run(w)
+    try:
+        r.layer.save_for_backward(True)
+        r.forward()
+        g = torch.Generator(device="cuda").manual_seed(5)
+        dy = (torch.randn((r.T, w.d), generator=g, device="cuda") * 0.1).to(torch.bfloat16)
+        grads = {k_: v for k_, v in _grads(w, 0.0).items() if k_ in names}
+        dx = _run_backward(r, dy, grads)
+        ref = _oracle_backward(r, _bf16_to_f64(to_host_bits(dy)))
+        _cmp(_bf16_to_f64(to_host_bits(dx)), ref[0], "dx")
+        for name, i in (("router", 1), ("gate", 2), ("up", 3), ("down", 4)):
+            if name in grads:
+                _cmp(grads[name].double().cpu().numpy(), ref[i], name)
+    finally:
+        r.close()
+
+
 def test_saved_activations_leave_the_forward_unchanged(cuda_ok):
     """Training mode only adds stores: y is bit-identical with and without it, and
     switching it off again returns to the recomputing backward with the same results
