@@ -261,6 +261,55 @@ ZCMOE_API int zcmoe_backward(zcmoe_t h, const void *x, const void *dy, int64_t T
  * cannot be allocated (training mode then stays off). */
 ZCMOE_API int zcmoe_save_for_backward(zcmoe_t h, int32_t on);
 
+/* ---------------------------------------------------------------- expert parallelism
+ * LongCat-Flash technical summary (zhangjingwei.cn), 五 訓練基礎設施: the FFN layers are
+ * partitioned by expert across an EP group (no tensor parallelism).  Rank r of an EP group of
+ * ep_size ranks holds FFN experts [r * n_local, (r + 1) * n_local), n_local = n_ffn / ep_size;
+ * every rank routes its own tokens over all n_ffn + n_zero experts.  A forward is three calls
+ * with two exchanges between them, which the caller runs (NCCL all-to-all, for example):
+ *   1. zcmoe_ep_dispatch: routing and the gather of the FFN pairs' rows, in expert order,
+ *      so the rows for rank r are the contiguous block of its experts;
+ *   exchange the per-expert counts and the rows (rank r gets its experts' rows);
+ *   2. zcmoe_ep_experts: the local experts on the received rows;
+ *   exchange the outputs back (the reverse of the row exchange);
+ *   3. zcmoe_ep_combine: the gate-weighted sum on the token's rank.
+ * Zero-computation experts need no weights: their picks never leave the token's rank
+ * (the combine adds them from x).  The bias controller counts every rank's own picks
+ * (zcmoe_read_counts / zcmoe_write_counts sum them over the group, as with data
+ * parallelism).  bf16 layers; zcmoe_forward, zcmoe_backward and zcmoe_save_for_backward
+ * return ZCMOE_EUNSUPPORTED on a handle with ep_size > 1. */
+
+/* Like zcmoe_create, for rank ep_rank of an EP group of ep_size ranks: `local` holds the
+ * router's full [E, d] weights and this rank's experts only (w_gate, w_up [n_local, inter, d],
+ * w_down [n_local, d, inter], borrowed).  max_recv_rows bounds the rows one zcmoe_ep_experts
+ * call takes (its workspace is max(max_tokens * top_k, max_recv_rows) rows of d + inter + d
+ * bf16 values).  n_ffn must be a multiple of ep_size; ep_size > 1 needs ZCMOE_BF16. */
+ZCMOE_API int zcmoe_create_ep(const zcmoe_config *cfg, const zcmoe_weights *local, int32_t ep_rank, int32_t ep_size,
+                              int64_t max_recv_rows, zcmoe_t *out);
+
+/* Stage 1.  x [T, d] device bf16.  Writes xsend [T * top_k, d] device bf16 (caller-owned; the
+ * first P rows are the FFN pairs' rows, sorted by expert, then token, then slot) and offsets
+ * [n_ffn + 1] device int32 (expert e's rows are [offsets[e], offsets[e+1]); P = offsets[n_ffn]).
+ * Keeps the routing for zcmoe_ep_combine and adds the counts to the controller's accumulators.
+ * Asynchronous on `stream`. */
+ZCMOE_API int zcmoe_ep_dispatch(zcmoe_t h, const void *x, int64_t T, void *xsend, int32_t *offsets,
+                                cudaStream_t stream);
+
+/* Stage 2.  xrecv [P_recv, d] device bf16: the rows received from the ep_size source ranks in rank
+ * order, each source's rows grouped by this rank's local experts in expert order; counts
+ * [ep_size * n_local] HOST int32: counts[s * n_local + e] = the rows source s sent for local
+ * expert e (they must sum to P_recv <= max(max_tokens * top_k, max_recv_rows)).  Writes yrecv
+ * [P_recv, d] device bf16: row q = the expert's output for row q of xrecv.  Reads `counts` before
+ * returning; the computation is asynchronous on `stream` (the call waits for the previous call's
+ * upload of the row layout). */
+ZCMOE_API int zcmoe_ep_experts(zcmoe_t h, const void *xrecv, const int32_t *counts, int64_t P_recv, void *yrecv,
+                               cudaStream_t stream);
+
+/* Stage 3.  x [T, d] device bf16: the tokens of the last dispatch; yback [P, d] device bf16: the
+ * expert outputs in xsend's row order.  Writes y [T, d] device bf16.  T must equal the last
+ * dispatch's.  Asynchronous on `stream`. */
+ZCMOE_API int zcmoe_ep_combine(zcmoe_t h, const void *x, const void *yback, int64_t T, void *y, cudaStream_t stream);
+
 /* Block quantization to FP8 E4M3 with E8M0 scales, the rule ZCMOE_FP8 layers use
  * (round to nearest even; scale 2^E the smallest power of two with the block's
  * largest magnitude <= 448 * 2^E, E + 127 clamped to [0, 254]; an all-zero block

@@ -22,7 +22,7 @@ COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hi
           "-cudart", "shared", "-Xlinker", "-rpath,/usr/local/cuda/lib64",
           "--expt-relaxed-constexpr"]
 
-LAYER_SOURCES = ["zcmoe.cu", "route.cu", "gemm_tc.cu", "gemm_simt.cu", "route_noalloc.cu", "fp8_quant.cu", "gemm_fp8.cu", "gemm_bwd.cu", "moe_bwd.cu"]
+LAYER_SOURCES = ["zcmoe.cu", "route.cu", "gemm_tc.cu", "gemm_simt.cu", "route_noalloc.cu", "fp8_quant.cu", "gemm_fp8.cu", "gemm_bwd.cu", "moe_bwd.cu", "ep.cu"]
 LAYER_HEADERS = ["zc_internal.h", "zc_ptx.cuh"]
 
 

@@ -124,6 +124,11 @@ enum BwdSched { kSchedRows = 0, kSchedWgrad = 1 };
 enum BwdEpi { kEpiBf16 = 0, kEpiSwigluBwd = 1, kEpiAddF32 = 2, kEpiSwigluSaved = 3 };
 enum BwdKind { kBwdRowsMnB = 0, kBwdSwiglu = 1, kBwdWgrad = 2, kBwdDhSwiglu = 3 };
 
+// ------------------------------------------------------------- expert parallelism (ep.cu)
+// Row q of s-major segment i (rows [seg_src[i], seg_src[i+1])) <-> row seg_dst[i] + q - seg_src[i].
+cudaError_t launch_ep_regroup(const void* src, void* dst, int64_t P, int row_bytes, const int32_t* seg_src,
+                              const int32_t* seg_dst, int nseg, int inverse, int sms, cudaStream_t s);
+
 struct BwdArgs {
   int K;                     // kSchedRows: reduction length (a multiple of 64)
   int n_out, nblocks;        // output columns, 256-column tiles

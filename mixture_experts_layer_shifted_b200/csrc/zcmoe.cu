@@ -193,6 +193,16 @@ struct zcmoe_s {
   // the last forward wrote it
   void* b_gu;
   bool last_saved;
+  // expert parallelism (zcmoe_create_ep): the handle holds FFN experts [ep_rank * n_local,
+  // (ep_rank + 1) * n_local); xperm / H / Y have rows_cap rows (the routed pairs of max_T
+  // tokens, or the rows received from all ranks, whichever is larger).  ep_meta (device) and
+  // ep_meta_host (pinned): seg_src [nseg + 1], seg_dst [nseg], exp_off [n_local + 1],
+  // mb_off [n_local + 1] of the last zcmoe_ep_experts, nseg = ep_size * n_local
+  int ep_rank, ep_size, n_local;
+  int64_t rows_cap;
+  int32_t *ep_meta, *ep_meta_host;
+  cudaEvent_t ep_meta_ev;
+  bool ep_meta_pending;
   bool alive;
 };
 
@@ -202,9 +212,11 @@ static void release(zcmoe_s* h) {
                   h->mb_off, h->scal,  h->chunk,  h->perm,  h->xperm,   h->H,      h->Y,
                   h->stage_x, h->stage_x2, h->stage_y, h->w8g, h->w8u, h->w8d, h->sfg, h->sfu, h->sfd,
                   h->x8, h->sx, h->h8, h->sh, h->ypad, h->b_xpad, h->b_dypad, h->b_dh, h->b_dgu, h->b_hpad,
-                  h->b_dxp, h->b_dl, h->b_dxr, h->b_dg, h->b_grp, h->b_gu};
+                  h->b_dxp, h->b_dl, h->b_dxr, h->b_dg, h->b_grp, h->b_gu, h->ep_meta};
   for (void* p : ptrs)
     if (p) cudaFree(p);
+  if (h->ep_meta_host) cudaFreeHost(h->ep_meta_host);
+  if (h->ep_meta_ev) cudaEventDestroy(h->ep_meta_ev);
   for (int i = 0; i < 2; ++i) {
     if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
     if (h->ev_used[i]) cudaEventDestroy(h->ev_used[i]);
@@ -292,12 +304,18 @@ extern "C" {
 
 const char* zcmoe_last_error(void) { return g_err; }
 
-int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) {
+static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_rank, int ep_size,
+                       int64_t max_recv_rows, zcmoe_t* out) {
   g_err[0] = 0;
   if (!out) return fail(ZCMOE_EINVAL, "out is NULL");
   *out = nullptr;
   if (!cfg || !w) return fail(ZCMOE_EINVAL, "cfg or weights is NULL");
   const int N = cfg->n_ffn, Z = cfg->n_zero, E = N + Z, k = cfg->top_k;
+  if (ep_size < 1 || ep_rank < 0 || ep_rank >= ep_size) return fail(ZCMOE_EINVAL, "need 0 <= ep_rank < ep_size");
+  if (N % ep_size) return fail(ZCMOE_EINVAL, "n_ffn must be a multiple of ep_size");
+  if (ep_size > 1 && cfg->dtype != ZCMOE_BF16) return fail(ZCMOE_EUNSUPPORTED, "expert parallelism needs a bf16 layer");
+  if (max_recv_rows < 0 || max_recv_rows >= (int64_t)1 << 31) return fail(ZCMOE_EINVAL, "bad max_recv_rows");
+  const int NL = N / ep_size;  // FFN experts this handle holds
   if (N < 1 || Z < 0 || E > 1024) return fail(ZCMOE_EINVAL, "need 1 <= n_ffn and n_ffn + n_zero <= 1024");
   if (k < 1 || k > E || k > 32) return fail(ZCMOE_EINVAL, "need 1 <= top_k <= min(E, 32)");
   if (cfg->d < 64 || cfg->d % 64 || cfg->inter < 64 || cfg->inter % 64)
@@ -348,7 +366,12 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
   h->max_chunks = (h->max_T + zc::kChunk - 1) / zc::kChunk;
   h->max_pairs = h->max_T * k;
   h->max_mblocks = (h->max_pairs + zc::kBM - 1) / zc::kBM + N;
+  h->ep_rank = ep_rank;
+  h->ep_size = ep_size;
+  h->n_local = NL;
+  h->rows_cap = max_recv_rows > h->max_pairs ? max_recv_rows : (int64_t)h->max_pairs;
   const size_t esz = h->bf16 ? 2 : 4;
+  const size_t rcap = (size_t)h->rows_cap;
 
   int rc = ZCMOE_OK;
 #define ZC_ALLOC(p, n)                     \
@@ -374,13 +397,14 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
   {
     uint8_t *xp = nullptr, *hh = nullptr, *yy = nullptr;
     // FP8 layers use the padded FP8 operands below instead
-    ZC_ALLOC(xp, h->fp8 ? 0 : (size_t)h->max_pairs * h->d * esz);
-    ZC_ALLOC(hh, h->fp8 ? 0 : (size_t)h->max_pairs * h->inter * esz);
-    ZC_ALLOC(yy, h->fp8 ? 0 : (size_t)h->max_pairs * h->d * esz);
+    ZC_ALLOC(xp, h->fp8 ? 0 : rcap * h->d * esz);
+    ZC_ALLOC(hh, h->fp8 ? 0 : rcap * h->inter * esz);
+    ZC_ALLOC(yy, h->fp8 ? 0 : rcap * h->d * esz);
     h->xperm = xp;
     h->H = hh;
     h->Y = yy;
   }
+  if (ep_size > 1) ZC_ALLOC(h->ep_meta, (size_t)2 * ep_size * NL + 1 + 2 * (NL + 1));
   if (h->fp8) {
     const size_t prow = (size_t)h->max_mblocks * zc::kBM;  // padded rows
     // scale atoms per 128 rows: an atom covers 512 K elements (FP8) or 128 (MXFP4)
@@ -408,6 +432,16 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
     return rc;
   }
   h->acc_tokens = h->acc_counts + E;
+  if (ep_size > 1) {
+    cudaError_t e = cudaHostAlloc(reinterpret_cast<void**>(&h->ep_meta_host),
+                                  ((size_t)2 * ep_size * NL + 1 + 2 * (NL + 1)) * sizeof(int32_t), cudaHostAllocDefault);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ep_meta_ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      release(h);
+      delete h;
+      return fail(ZCMOE_ECUDA, "expert-parallel staging: %s", cudaGetErrorString(e));
+    }
+  }
 
   // initial state: bias = b0 = init_bias (or 0), eta = 1, integral/previous error = 0
   {
@@ -428,8 +462,8 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
     if (e == cudaSuccess) e = cudaMemset(h->eprev, 0, E * sizeof(float));
     if (e == cudaSuccess) e = cudaMemset(h->acc_counts, 0, (E + 1) * sizeof(int64_t));
     if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int));
-    if (e == cudaSuccess && !h->fp8) e = cudaMemset(h->xperm, 0, (size_t)h->max_pairs * h->d * esz);
-    if (e == cudaSuccess && !h->fp8) e = cudaMemset(h->H, 0, (size_t)h->max_pairs * h->inter * esz);
+    if (e == cudaSuccess && !h->fp8) e = cudaMemset(h->xperm, 0, rcap * h->d * esz);
+    if (e == cudaSuccess && !h->fp8) e = cudaMemset(h->H, 0, rcap * h->inter * esz);
     if (h->fp8) {
       // padded operand rows that no pair fills read as zeros
       const size_t prow = (size_t)h->max_mblocks * zc::kBM;
@@ -461,11 +495,11 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
   if (h->bf16) {
     const uint64_t d = h->d, inter = h->inter;
     rc = make_tmap(&h->tm_wr, w->w_router, d, (uint64_t)E, 256);
-    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wg, w->w_gate, d, (uint64_t)N * inter, 128);
-    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wu, w->w_up, d, (uint64_t)N * inter, 128);
-    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wd, w->w_down, inter, (uint64_t)N * d, 256);
-    if (rc == ZCMOE_OK && !h->fp8) rc = make_tmap(&h->tm_xperm, h->xperm, d, (uint64_t)h->max_pairs, 128);
-    if (rc == ZCMOE_OK && !h->fp8) rc = make_tmap(&h->tm_h, h->H, inter, (uint64_t)h->max_pairs, 128);
+    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wg, w->w_gate, d, (uint64_t)NL * inter, 128);
+    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wu, w->w_up, d, (uint64_t)NL * inter, 128);
+    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wd, w->w_down, inter, (uint64_t)NL * d, 256);
+    if (rc == ZCMOE_OK && !h->fp8) rc = make_tmap(&h->tm_xperm, h->xperm, d, (uint64_t)h->rows_cap, 128);
+    if (rc == ZCMOE_OK && !h->fp8) rc = make_tmap(&h->tm_h, h->H, inter, (uint64_t)h->rows_cap, 128);
     if (h->fp8) {
       // codes as bytes: the K extent is d or inter bytes (FP8), half that (MXFP4)
       const uint64_t prow = (uint64_t)h->max_mblocks * zc::kBM;
@@ -491,35 +525,19 @@ int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) 
   return ZCMOE_OK;
 }
 
-// The forward pass; with `side`, the dense FFN's two GEMMs are forked onto its
-// stream after the router GEMM and after the down GEMM, and joined back into
-// `s` after the combine.
-static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream_t s, const zcmoe_debug* dbg,
-                        const DenseSide* side) {
-  if (T < 0 || T > h->max_T) return fail(ZCMOE_ERANGE, "T=%lld outside [0, %d]", (long long)T, h->max_T);
-  if (T == 0) return ZCMOE_OK;
-  if (!x || !y) return fail(ZCMOE_EINVAL, "x or y is NULL");
-  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(y) & 15u))
-    return fail(ZCMOE_EINVAL, "x and y must be 16-byte aligned");
-  const size_t esz = h->bf16 ? 2 : 4;
-  const size_t xbytes = (size_t)T * h->d * esz;
-  const uintptr_t xa = reinterpret_cast<uintptr_t>(x), ya = reinterpret_cast<uintptr_t>(y);
-  if (xa < ya + xbytes && ya < xa + xbytes) return fail(ZCMOE_EINVAL, "y overlaps x");
+int zcmoe_create(const zcmoe_config* cfg, const zcmoe_weights* w, zcmoe_t* out) {
+  return create_impl(cfg, w, 0, 1, 0, out);
+}
 
-  const int Ti = (int)T, E = h->E, N = h->N, k = h->k, d = h->d, inter = h->inter;
-  const int nchunks = (Ti + zc::kChunk - 1) / zc::kChunk;
-  h->last_T = Ti;
-  auto mark = [&]() -> cudaError_t {
-    if (!h->profiling) return cudaSuccess;
-    cudaEvent_t ev;
-    cudaError_t e = cudaEventCreate(&ev);
-    if (e != cudaSuccess) return e;
-    h->events->push_back(ev);
-    return cudaEventRecord(ev, s);
-  };
-  ZC_CUDA(mark());
+int zcmoe_create_ep(const zcmoe_config* cfg, const zcmoe_weights* local, int32_t ep_rank, int32_t ep_size,
+                    int64_t max_recv_rows, zcmoe_t* out) {
+  return create_impl(cfg, local, ep_rank, ep_size, max_recv_rows, out);
+}
 
-  // 1. router logits
+// 1. router logits (+ the logit offset), fp32 [T, E]
+static int router_stage(zcmoe_t h, const void* x, int Ti, cudaStream_t s) {
+  const int E = h->E, d = h->d;
+  const int64_t T = Ti;
   if (h->bf16) {
     CUtensorMap tm_x;
     int rc = make_tmap(&tm_x, x, (uint64_t)d, (uint64_t)T, 128);
@@ -549,6 +567,54 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     a.col_add = h->offset;
     ZC_CUDA(zc::launch_simt_gemm(zc::kRouter, a, (Ti + zc::kBM - 1) / zc::kBM, s));
   }
+  return ZCMOE_OK;
+}
+
+// 3. the integer stage: counts (into the controller's accumulators too), offsets,
+// row-block offsets, the permutation of the FFN pairs, the slot positions
+static int integer_stage(zcmoe_t h, int Ti, cudaStream_t s) {
+  const int E = h->E, N = h->N, k = h->k;
+  const int nchunks = (Ti + zc::kChunk - 1) / zc::kChunk;
+  ZC_CUDA(zc::launch_route_count(h->idx, Ti, k, E, h->chunk, s));
+  ZC_CUDA(zc::launch_route_scan(h->chunk, nchunks, Ti, N, E, h->counts, h->offsets, h->mb_off, h->scal,
+                                h->acc_counts, h->acc_tokens, s));
+  ZC_CUDA(zc::launch_route_scatter(h->idx, Ti, k, N, E, h->chunk, h->perm, h->pos, s));
+  return ZCMOE_OK;
+}
+
+// The forward pass; with `side`, the dense FFN's two GEMMs are forked onto its
+// stream after the router GEMM and after the down GEMM, and joined back into
+// `s` after the combine.
+static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream_t s, const zcmoe_debug* dbg,
+                        const DenseSide* side) {
+  if (h->ep_size > 1) return fail(ZCMOE_EUNSUPPORTED, "an expert-parallel handle runs through zcmoe_ep_*");
+  if (T < 0 || T > h->max_T) return fail(ZCMOE_ERANGE, "T=%lld outside [0, %d]", (long long)T, h->max_T);
+  if (T == 0) return ZCMOE_OK;
+  if (!x || !y) return fail(ZCMOE_EINVAL, "x or y is NULL");
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(y) & 15u))
+    return fail(ZCMOE_EINVAL, "x and y must be 16-byte aligned");
+  const size_t esz = h->bf16 ? 2 : 4;
+  const size_t xbytes = (size_t)T * h->d * esz;
+  const uintptr_t xa = reinterpret_cast<uintptr_t>(x), ya = reinterpret_cast<uintptr_t>(y);
+  if (xa < ya + xbytes && ya < xa + xbytes) return fail(ZCMOE_EINVAL, "y overlaps x");
+
+  const int Ti = (int)T, E = h->E, N = h->N, k = h->k, d = h->d, inter = h->inter;
+  h->last_T = Ti;
+  auto mark = [&]() -> cudaError_t {
+    if (!h->profiling) return cudaSuccess;
+    cudaEvent_t ev;
+    cudaError_t e = cudaEventCreate(&ev);
+    if (e != cudaSuccess) return e;
+    h->events->push_back(ev);
+    return cudaEventRecord(ev, s);
+  };
+  ZC_CUDA(mark());
+
+  // 1. router logits
+  {
+    const int rc = router_stage(h, x, Ti, s);
+    if (rc != ZCMOE_OK) return rc;
+  }
   ZC_CUDA(mark());
   if (side) {
     ZC_CUDA(cudaEventRecord(side->dn->ev_router, s));
@@ -561,10 +627,10 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
                                   dbg ? dbg->scores : nullptr, h->sms, s));
   ZC_CUDA(mark());
   // 3. integer stage
-  ZC_CUDA(zc::launch_route_count(h->idx, Ti, k, E, h->chunk, s));
-  ZC_CUDA(zc::launch_route_scan(h->chunk, nchunks, Ti, N, E, h->counts, h->offsets, h->mb_off, h->scal,
-                                h->acc_counts, h->acc_tokens, s));
-  ZC_CUDA(zc::launch_route_scatter(h->idx, Ti, k, N, E, h->chunk, h->perm, h->pos, s));
+  {
+    const int rc = integer_stage(h, Ti, s);
+    if (rc != ZCMOE_OK) return rc;
+  }
   ZC_CUDA(mark());
   // 4. gather the FFN pairs' rows (FP8 layers: quantized per [1,128] into padded rows)
   if (h->fp8 && h->fmt)
@@ -715,6 +781,187 @@ int zcmoe_forward(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream_t s, 
   g_err[0] = 0;
   if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
   return forward_impl(h, x, T, y, s, dbg, nullptr);
+}
+
+// ---------------------------------------------------------------- expert parallelism
+
+int zcmoe_ep_dispatch(zcmoe_t h, const void* x, int64_t T, void* xsend, int32_t* offsets, cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (!h->bf16 || h->fp8) return fail(ZCMOE_EUNSUPPORTED, "expert parallelism needs a bf16 layer");
+  if (T < 0 || T > h->max_T) return fail(ZCMOE_ERANGE, "T=%lld outside [0, %d]", (long long)T, h->max_T);
+  if (!offsets) return fail(ZCMOE_EINVAL, "offsets is NULL");
+  const int Ti = (int)T;
+  if (T == 0) {  // x and xsend may be NULL (no rows)
+    h->last_T = 0;
+    ZC_CUDA(cudaMemsetAsync(offsets, 0, (size_t)(h->N + 1) * sizeof(int32_t), s));
+    return ZCMOE_OK;
+  }
+  if (!x || !xsend) return fail(ZCMOE_EINVAL, "x or xsend is NULL");
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(xsend) & 15u))
+    return fail(ZCMOE_EINVAL, "x and xsend must be 16-byte aligned");
+  const size_t xb = (size_t)T * h->d * 2, sb = (size_t)T * h->k * h->d * 2;
+  if (overlaps(xsend, sb, x, xb)) return fail(ZCMOE_EINVAL, "xsend overlaps x");
+  h->last_T = Ti;
+  int rc = router_stage(h, x, Ti, s);
+  if (rc != ZCMOE_OK) return rc;
+  ZC_CUDA(zc::launch_softmax_topk(h->logits, h->bias, Ti, h->E, h->k, h->cfg.routed_scale, h->idx, h->gate, nullptr,
+                                  h->sms, s));
+  rc = integer_stage(h, Ti, s);
+  if (rc != ZCMOE_OK) return rc;
+  ZC_CUDA(zc::launch_gather_rows(x, h->d * 2, h->perm, h->k, h->scal, xsend, h->sms, s));
+  ZC_CUDA(cudaMemcpyAsync(offsets, h->offsets, (size_t)(h->N + 1) * sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
+  return ZCMOE_OK;
+}
+
+int zcmoe_ep_experts(zcmoe_t h, const void* xrecv, const int32_t* counts, int64_t P_recv, void* yrecv,
+                     cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (!h->bf16 || h->fp8) return fail(ZCMOE_EUNSUPPORTED, "expert parallelism needs a bf16 layer");
+  if (P_recv < 0 || P_recv > h->rows_cap)
+    return fail(ZCMOE_ERANGE, "P_recv=%lld outside [0, %lld]", (long long)P_recv, (long long)h->rows_cap);
+  if (!counts) return fail(ZCMOE_EINVAL, "counts is NULL");
+  const int R = h->ep_size, NL = h->n_local, nseg = R * NL;
+  int64_t total = 0;
+  for (int i = 0; i < nseg; ++i) {
+    if (counts[i] < 0) return fail(ZCMOE_EINVAL, "counts[%d] is negative", i);
+    total += counts[i];
+  }
+  if (total != P_recv) return fail(ZCMOE_EINVAL, "counts sum to %lld, not P_recv=%lld", (long long)total,
+                                   (long long)P_recv);
+  if (P_recv == 0) return ZCMOE_OK;
+  if (!xrecv || !yrecv) return fail(ZCMOE_EINVAL, "xrecv or yrecv is NULL");
+  if ((reinterpret_cast<uintptr_t>(xrecv) & 15u) || (reinterpret_cast<uintptr_t>(yrecv) & 15u))
+    return fail(ZCMOE_EINVAL, "xrecv and yrecv must be 16-byte aligned");
+  const size_t rb = (size_t)P_recv * h->d * 2;
+  if (overlaps(xrecv, rb, yrecv, rb)) return fail(ZCMOE_EINVAL, "yrecv overlaps xrecv");
+  const int d = h->d, inter = h->inter;
+
+  // row layout: ep_size == 1 needs no regrouping (one source: s-major is e-major)
+  const int32_t* exp_off;
+  const int32_t* mb_off;
+  int mb_total = 0;
+  const void* a_rows = xrecv;
+  void* y_rows = yrecv;
+  if (R > 1) {
+    if (h->ep_meta_pending) {
+      ZC_CUDA(cudaEventSynchronize(h->ep_meta_ev));  // the previous upload has read the staging buffer
+      h->ep_meta_pending = false;
+    }
+    int32_t* m = h->ep_meta_host;
+    int32_t* seg_src = m;
+    int32_t* seg_dst = seg_src + nseg + 1;
+    int32_t* eoff = seg_dst + nseg;
+    int32_t* moff = eoff + NL + 1;
+    seg_src[0] = 0;
+    for (int i = 0; i < nseg; ++i) seg_src[i + 1] = seg_src[i] + counts[i];
+    eoff[0] = 0;
+    moff[0] = 0;
+    for (int e = 0; e < NL; ++e) {
+      int cnt = 0;
+      for (int r = 0; r < R; ++r) {
+        seg_dst[r * NL + e] = eoff[e] + cnt;
+        cnt += counts[r * NL + e];
+      }
+      eoff[e + 1] = eoff[e] + cnt;
+      moff[e + 1] = moff[e] + (cnt + zc::kBM - 1) / zc::kBM;
+    }
+    mb_total = moff[NL];
+    const size_t bytes = ((size_t)2 * nseg + 1 + 2 * (NL + 1)) * sizeof(int32_t);
+    ZC_CUDA(cudaMemcpyAsync(h->ep_meta, m, bytes, cudaMemcpyHostToDevice, s));
+    ZC_CUDA(cudaEventRecord(h->ep_meta_ev, s));
+    h->ep_meta_pending = true;
+    const int32_t* dseg_src = h->ep_meta;
+    const int32_t* dseg_dst = dseg_src + nseg + 1;
+    exp_off = dseg_dst + nseg;
+    mb_off = exp_off + NL + 1;
+    // rows into the e-major layout of xperm; the outputs come back through Y
+    ZC_CUDA(zc::launch_ep_regroup(xrecv, h->xperm, P_recv, d * 2, dseg_src, dseg_dst, nseg, 0, h->sms, s));
+    a_rows = h->xperm;
+    y_rows = h->Y;
+  } else {
+    // one source: the counts are the expert offsets; stage them like the segments
+    if (h->ep_meta_pending) {
+      ZC_CUDA(cudaEventSynchronize(h->ep_meta_ev));
+      h->ep_meta_pending = false;
+    }
+    if (!h->ep_meta) {
+      int rc = dalloc(&h->ep_meta, (size_t)2 * (NL + 1));
+      if (rc != ZCMOE_OK) return rc;
+      cudaError_t e = cudaHostAlloc(reinterpret_cast<void**>(&h->ep_meta_host), (size_t)2 * (NL + 1) * sizeof(int32_t),
+                                    cudaHostAllocDefault);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ep_meta_ev, cudaEventDisableTiming);
+      if (e != cudaSuccess) return fail(ZCMOE_ECUDA, "expert-parallel staging: %s", cudaGetErrorString(e));
+    }
+    int32_t* eoff = h->ep_meta_host;
+    int32_t* moff = eoff + NL + 1;
+    eoff[0] = 0;
+    moff[0] = 0;
+    for (int e = 0; e < NL; ++e) {
+      eoff[e + 1] = eoff[e] + counts[e];
+      moff[e + 1] = moff[e] + (counts[e] + zc::kBM - 1) / zc::kBM;
+    }
+    mb_total = moff[NL];
+    ZC_CUDA(cudaMemcpyAsync(h->ep_meta, eoff, (size_t)2 * (NL + 1) * sizeof(int32_t), cudaMemcpyHostToDevice, s));
+    ZC_CUDA(cudaEventRecord(h->ep_meta_ev, s));
+    h->ep_meta_pending = true;
+    exp_off = h->ep_meta;
+    mb_off = exp_off + NL + 1;
+  }
+  CUtensorMap tm_a, tm_h;
+  int rc = make_tmap(&tm_a, a_rows, (uint64_t)d, (uint64_t)P_recv, 128);
+  if (rc == ZCMOE_OK) rc = make_tmap(&tm_h, h->H, (uint64_t)inter, (uint64_t)P_recv, 128);
+  if (rc != ZCMOE_OK) return rc;
+  // the local experts' grouped GEMMs (the forward's kernels, over the received rows)
+  zc::TcArgs a{};
+  a.K = d;
+  a.n_out = inter;
+  a.nblocks = (inter + zc::tc_block_n(zc::kGateUp) - 1) / zc::tc_block_n(zc::kGateUp);
+  a.ngroups = NL;
+  a.row_off = exp_off;
+  a.mb_off = mb_off;
+  a.b_rows_per_group = inter;
+  a.out = h->H;
+  a.ldo = inter;
+  a.err = h->err;
+  int bound = mb_total * a.nblocks;
+  ZC_CUDA(zc::launch_tc_gemm(zc::kGateUp, tm_a, h->tm_wg, h->tm_wu, a, bound < h->sms ? bound : h->sms, s));
+  zc::TcArgs b{};
+  b.K = inter;
+  b.n_out = d;
+  b.nblocks = (d + zc::tc_block_n(zc::kDown) - 1) / zc::tc_block_n(zc::kDown);
+  b.ngroups = NL;
+  b.row_off = exp_off;
+  b.mb_off = mb_off;
+  b.b_rows_per_group = d;
+  b.out = y_rows;
+  b.ldo = d;
+  b.err = h->err;
+  bound = mb_total * b.nblocks;
+  ZC_CUDA(zc::launch_tc_gemm(zc::kDown, tm_h, h->tm_wd, h->tm_wd, b, bound < h->sms ? bound : h->sms, s));
+  if (R > 1) {
+    const int32_t* dseg_src = h->ep_meta;
+    ZC_CUDA(zc::launch_ep_regroup(h->Y, yrecv, P_recv, d * 2, dseg_src, dseg_src + nseg + 1, nseg, 1, h->sms, s));
+  }
+  return ZCMOE_OK;
+}
+
+int zcmoe_ep_combine(zcmoe_t h, const void* x, const void* yback, int64_t T, void* y, cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (!h->bf16 || h->fp8) return fail(ZCMOE_EUNSUPPORTED, "expert parallelism needs a bf16 layer");
+  if (T < 0 || T > h->max_T) return fail(ZCMOE_ERANGE, "T=%lld outside [0, %d]", (long long)T, h->max_T);
+  if (T != h->last_T) return fail(ZCMOE_EINVAL, "T=%lld differs from the last dispatch's %d", (long long)T, h->last_T);
+  if (T == 0) return ZCMOE_OK;
+  if (!x || !y || !yback) return fail(ZCMOE_EINVAL, "x, yback or y is NULL");
+  const void* ps[3] = {x, yback, y};
+  for (const void* p : ps)
+    if (reinterpret_cast<uintptr_t>(p) & 15u) return fail(ZCMOE_EINVAL, "x, yback and y must be 16-byte aligned");
+  const size_t xb = (size_t)T * h->d * 2;
+  if (overlaps(y, xb, x, xb)) return fail(ZCMOE_EINVAL, "y overlaps x");
+  ZC_CUDA(zc::launch_combine(1, x, yback, h->idx, h->gate, h->pos, (int)T, h->k, h->N, h->d, y, h->sms, s));
+  return ZCMOE_OK;
 }
 
 int zcmoe_forward_host(zcmoe_t h, const void* x_host, int64_t T, void* y_host, cudaStream_t s) {
@@ -890,6 +1137,7 @@ int zcmoe_save_for_backward(zcmoe_t h, int32_t on) {
   g_err[0] = 0;
   if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
   if (!h->bf16 || h->fp8) return fail(ZCMOE_EUNSUPPORTED, "training mode needs a bf16 layer");
+  if (h->ep_size > 1) return fail(ZCMOE_EUNSUPPORTED, "training mode needs a layer that holds all experts");
   if (!on) {
     if (h->b_gu) {
       ZC_CUDA(cudaDeviceSynchronize());
@@ -912,6 +1160,7 @@ int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx
   g_err[0] = 0;
   if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
   if (!h->bf16 || h->fp8) return fail(ZCMOE_EUNSUPPORTED, "the backward pass needs a bf16 layer");
+  if (h->ep_size > 1) return fail(ZCMOE_EUNSUPPORTED, "the backward pass needs a layer that holds all experts");
   if (T < 0 || T > h->max_T) return fail(ZCMOE_ERANGE, "T=%lld outside [0, %d]", (long long)T, h->max_T);
   if (T == 0) return ZCMOE_OK;
   if (T != h->last_T) return fail(ZCMOE_EINVAL, "T=%lld differs from the last forward's %d", (long long)T, h->last_T);

@@ -36,7 +36,8 @@ EXPORTED = ("zcmoe_create", "zcmoe_forward", "zcmoe_forward_host", "zcmoe_update
             "zcmoe_profile_end", "zcmoe_selftest_wait", "zcmoe_route_noalloc", "zcmoe_destroy",
             "zcmoe_dense_create", "zcmoe_dense_forward", "zcmoe_forward_overlap", "zcmoe_dense_check",
             "zcmoe_dense_destroy", "zcmoe_quantize_e4m3", "zcmoe_quantize_mx4", "zcmoe_backward",
-            "zcmoe_save_for_backward", "zcmoe_last_error")
+            "zcmoe_save_for_backward", "zcmoe_create_ep", "zcmoe_ep_dispatch", "zcmoe_ep_experts",
+            "zcmoe_ep_combine", "zcmoe_last_error")
 STAGES = ("router", "softmax_topk", "integer", "gather", "gate_up", "down", "combine")
 
 
@@ -112,6 +113,11 @@ def lib():
         L.zcmoe_quantize_mx4.argtypes = [vp, ctypes.c_int32, i64, i64, vp, vp, vp]
         L.zcmoe_backward.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, vp, vp]
         L.zcmoe_save_for_backward.argtypes = [vp, ctypes.c_int32]
+        L.zcmoe_create_ep.argtypes = [ctypes.POINTER(zcmoe_config), ctypes.POINTER(zcmoe_weights), ctypes.c_int32,
+                                      ctypes.c_int32, i64, ctypes.POINTER(vp)]
+        L.zcmoe_ep_dispatch.argtypes = [vp, vp, i64, vp, vp, vp]
+        L.zcmoe_ep_experts.argtypes = [vp, vp, vp, i64, vp, vp]
+        L.zcmoe_ep_combine.argtypes = [vp, vp, vp, i64, vp, vp]
         L.zcmoe_dense_destroy.argtypes = [vp]
         for f in EXPORTED[:-1]:
             getattr(L, f).restype = i32
@@ -141,6 +147,27 @@ def zcmoe_create(cfg: zcmoe_config, w: zcmoe_weights) -> ctypes.c_void_p:
     h = ctypes.c_void_p()
     _check(lib().zcmoe_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)), "zcmoe_create")
     return h
+
+
+def zcmoe_create_ep(cfg: zcmoe_config, w: zcmoe_weights, ep_rank: int, ep_size: int,
+                    max_recv_rows: int) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(lib().zcmoe_create_ep(ctypes.byref(cfg), ctypes.byref(w), ep_rank, ep_size, max_recv_rows, ctypes.byref(h)),
+           "zcmoe_create_ep")
+    return h
+
+
+def zcmoe_ep_dispatch(h, x_ptr, T, xsend_ptr, offsets_ptr, stream=None):
+    _check(lib().zcmoe_ep_dispatch(h, x_ptr, T, xsend_ptr, offsets_ptr, _stream(stream)), "zcmoe_ep_dispatch")
+
+
+def zcmoe_ep_experts(h, xrecv_ptr, counts_host_ptr, P_recv, yrecv_ptr, stream=None):
+    _check(lib().zcmoe_ep_experts(h, xrecv_ptr, counts_host_ptr, P_recv, yrecv_ptr, _stream(stream)),
+           "zcmoe_ep_experts")
+
+
+def zcmoe_ep_combine(h, x_ptr, yback_ptr, T, y_ptr, stream=None):
+    _check(lib().zcmoe_ep_combine(h, x_ptr, yback_ptr, T, y_ptr, _stream(stream)), "zcmoe_ep_combine")
 
 
 def zcmoe_forward(h, x_ptr, T, y_ptr, stream=None, dbg: zcmoe_debug | None = None):
@@ -298,13 +325,16 @@ class ZcMoE:
     """Owns a handle plus references to its (borrowed) device weights."""
 
     def __init__(self, shape: LayerShape, w_router, w_gate, w_up, w_down, max_tokens: int, init_bias=None,
-                 logit_offset=None):
+                 logit_offset=None, ep_rank: int = 0, ep_size: int = 1, max_recv_rows: int = 0):
+        """ep_size > 1: rank ep_rank of an expert-parallel group; w_gate, w_up, w_down then hold
+        only this rank's n_ffn / ep_size experts (see ep.py for the forward)."""
         import numpy as np
         self.shape = shape
         self.weights = (w_router, w_gate, w_up, w_down)
-        E = shape.E
-        for t, want in zip(self.weights, [(E, shape.d), (shape.n_ffn, shape.inter, shape.d),
-                                          (shape.n_ffn, shape.inter, shape.d), (shape.n_ffn, shape.d, shape.inter)]):
+        self.ep_rank, self.ep_size = ep_rank, ep_size
+        E, NL = shape.E, shape.n_ffn // max(ep_size, 1)
+        for t, want in zip(self.weights, [(E, shape.d), (NL, shape.inter, shape.d),
+                                          (NL, shape.inter, shape.d), (NL, shape.d, shape.inter)]):
             if tuple(t.shape) != want or t.dtype != shape.torch_dtype or not t.is_cuda or not t.is_contiguous():
                 raise ValueError(f"weight of shape {tuple(t.shape)} {t.dtype}; expected {want} {shape.torch_dtype}")
         self._bias0 = None if init_bias is None else np.ascontiguousarray(init_bias, dtype=np.float32)
@@ -316,7 +346,8 @@ class ZcMoE:
                            None if self._offset is None else self._offset.ctypes.data_as(fp))
         w = zcmoe_weights(w_router.data_ptr(), w_gate.data_ptr(), w_up.data_ptr(), w_down.data_ptr())
         self.max_tokens = max_tokens
-        self.h = zcmoe_create(cfg, w)
+        self.h = (zcmoe_create(cfg, w) if ep_size == 1 and max_recv_rows == 0
+                  else zcmoe_create_ep(cfg, w, ep_rank, ep_size, max_recv_rows))
 
     def forward(self, x, y=None, stream=None, debug: dict | None = None):
         """y = layer(x); ``debug`` maps zcmoe_debug field names to device tensors to fill."""
