@@ -382,6 +382,142 @@ def measure_backward(wl, layer, x, stream, peaks, P):
                     "(3 x 25.8 GB + router); each a replayed graph"}
 
 
+def run_ep(args, wl, dist, rank, ws, local, peaks):
+    """--ep: the expert-parallel layer (ep.py): rank r holds FFN experts [r N/ws, (r+1) N/ws)
+    and routes its own batch of wl.T tokens; dispatch and combine are NCCL all-to-alls (one
+    GPU: copies), two token chunks.  A step = forward + the shared controller step.  Eager
+    launches (the all-to-all split sizes go through the host)."""
+    import torch
+    from mixture_experts_layer_shifted_b200 import configs
+    from mixture_experts_layer_shifted_b200.ep import CudaStages, EpMoE, LocalComm, TorchComm
+    from mixture_experts_layer_shifted_b200.zcmoe import LayerShape
+
+    dev = torch.device("cuda", local)
+    shape = LayerShape(wl.d, wl.n_ffn, wl.n_zero, wl.inter, wl.top_k, "bf16")
+    if wl.n_ffn % ws:
+        raise SystemExit(f"--ep needs n_ffn ({wl.n_ffn}) to be a multiple of the GPU count")
+    NL = wl.n_ffn // ws
+    full = configs.device_weights(wl)
+    sl = slice(rank * NL, (rank + 1) * NL)
+    wr = full[0]
+    wg, wu, wd = (t[sl].clone() for t in full[1:])
+    keep_full = ws == 1 and not args.no_cpu_baseline  # the oracle sample reads them
+    if not keep_full:
+        del full
+        torch.cuda.empty_cache()
+    comm = TorchComm() if dist else LocalComm()
+    # rows one chunk's experts call may receive: twice a chunk's own FFN pairs (about 3x the balanced share)
+    nck = max(1, args.ep_chunks)
+    cap = 2 * wl.T * wl.top_k // nck
+    layer = EpMoE(shape, wr, wg, wu, wd, max_tokens=wl.T, comm=comm, chunks=nck, max_recv_rows=cap,
+                  init_bias=configs.bias_vector(wl), logit_offset=configs.logit_offsets(wl))
+    # the expert stage timed with events on the launch stream
+    ev_pairs, recv_rows = [], []
+
+    class TimedStages(CudaStages):
+        def experts(self, xrecv, counts):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            y = super().experts(xrecv, counts)
+            b.record()
+            ev_pairs.append((a, b))
+            recv_rows.append(int(xrecv.shape[0]))
+            return y
+
+    layer.stages = [TimedStages(lay) for lay in layer.layers]
+    xs = [configs.device_tokens(wl, step=rank * 4 + i) for i in range(2)]
+    target = wl.target_ffn if wl.target_ffn is not None else wl.top_k * wl.n_ffn / wl.E
+    red = (lambda t: dist.all_reduce(t, op=dist.ReduceOp.SUM)) if dist else None
+
+    def step(i):
+        y = layer.forward(xs[i % 2])
+        layer.controller_step(all_reduce=red, target_ffn_per_token=target, **GAINS)
+        return y
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    ev_pairs.clear()
+    recv_rows.clear()
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    exp_ms = sum(a.elapsed_time(b) for a, b in ev_pairs) / args.steps
+    exp_rows = sum(recv_rows) / args.steps
+    if dist:
+        t = torch.tensor([ms, exp_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, exp_ms = float(t[0]), float(t[1])
+    value = wl.T * ws * args.steps / (ms / 1e3)
+    # end to end: x from pinned host memory, y back to it, every step
+    xh = xs[0].cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, min(args.steps, 10))
+    a.record(stream)
+    for _ in range(n_e2e):
+        xd = xh.to(dev, non_blocking=True)
+        yh.copy_(layer.forward(xd), non_blocking=True)
+        layer.controller_step(all_reduce=red, target_ffn_per_token=target, **GAINS)
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / n_e2e
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    io = xh.numel() * xh.element_size()
+    flops = 6.0 * wl.d * wl.inter * exp_rows
+    peak = peaks["bf16_tflops_sustained"]
+    achieved = flops / (exp_ms * 1e-3) / 1e12 if exp_ms > 0 else 0.0
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        n_tok = 8 if wl.d >= 4096 else 64
+        n, sec, cores = cpu_oracle_sample(wl, full, xs[0], configs.bias_vector(wl), configs.logit_offsets(wl), n_tok,
+                                          min_s=12.0)
+        cpu = {"value": n / sec, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"first {n_tok} tokens of the {wl.name} batch, {n} tokens in {sec:.1f} s"}
+    for lay in layer.layers:
+        lay.check()
+    layer.close()
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Philox, random-init weights)",
+            "config": {"workload": wl.name, "T_per_rank": wl.T, "d": wl.d, "n_ffn": wl.n_ffn, "n_zero": wl.n_zero,
+                       "inter": wl.inter, "top_k": wl.top_k, "parallelism": f"ep{ws}", "chunks": nck,
+                       "l2": "inputs larger than L2; no flush"},
+            "roofline": {"bound": "tensor", "kernel": "zcmoe_ep_experts (regroup + grouped gate/up + down)",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "traffic": None, "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
+                         "per_launch": {"flops": flops, "ms": exp_ms, "units": f"{exp_rows:.0f} received rows x 6 d inter per step"}},
+            "cpu_baseline": cpu,
+            "e2e": {"value": wl.T * ws / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": io,
+                    "d2h_bytes_per_step": io, "ms_per_step": e2e_ms},
+            # per chunk: router GEMM, softmax/top-k, 3 integer-stage kernels, gather, the two expert
+            # GEMMs (+ 2 regroups with ws > 1), combine; per step one bias update per chunk handle
+            "gpu_launches": args.steps * (nck * (9 + (2 if ws > 1 else 0)) + nck), "clocks": clocks, "peaks": peaks,
+            "launch": "eager (host-side split sizes)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -393,6 +529,9 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--secondary", default="decode,fp8,fp4,backward,overlap",
                     help="comma list of the secondary measurements to run after the headline")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism over the GPUs (ep.py) instead of data-parallel replicas")
+    ap.add_argument("--ep-chunks", type=int, default=2, help="--ep: token chunks per step")
     ap.add_argument("--eager", action="store_true",
                     help="launch every step eagerly instead of replaying one captured CUDA graph (N=1)")
     args = ap.parse_args()
@@ -420,6 +559,12 @@ def main():
     peaks = _peaks()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.ep:
+        run_ep(args, wl, dist, rank, ws, local, peaks)
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     weights = configs.device_weights(wl)
     xs = [configs.device_tokens(wl, step=rank * 4 + i) for i in range(2)]
     bias = configs.bias_vector(wl)

@@ -47,6 +47,17 @@ class TorchComm:
                                            async_op=async_op)
 
 
+class LocalComm:
+    """The one-rank group (every expert local): the exchanges are copies."""
+
+    rank, size = 0, 1
+
+    def all_to_all(self, out, inp, out_splits, in_splits, async_op=False):
+        if out.numel():
+            out.copy_(inp)
+        return None
+
+
 class CudaStages:
     """The three stages of one chunk through the C ABI; `layer` is a ZcMoE created with
     this rank's ep_rank / ep_size (its routing state belongs to this chunk)."""
