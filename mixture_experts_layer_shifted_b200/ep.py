@@ -145,7 +145,10 @@ def ep_forward(stages_per_chunk, comm, x, n_ffn: int):
 
 class EpMoE:
     """The layer on one rank of an expert-parallel group: `chunks` handles over the same
-    (borrowed) weights, one per token chunk."""
+    (borrowed) weights, one per token chunk.  max_recv_rows bounds the rows one chunk may
+    receive (default: the worst case, every token of every rank picking min(top_k, n_local)
+    of this rank's experts; a tighter bound saves workspace, a chunk that exceeds it fails
+    with ZCMOE_ERANGE)."""
 
     def __init__(self, shape: zcmoe.LayerShape, w_router, w_gate_local, w_up_local, w_down_local, max_tokens: int,
                  comm=None, chunks: int = 2, max_recv_rows: int | None = None, init_bias=None, logit_offset=None):
