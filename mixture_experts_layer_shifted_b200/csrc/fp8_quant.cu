@@ -92,6 +92,35 @@ __global__ void __launch_bounds__(128) k_quant_tiles(const TIN* __restrict__ src
 
 // FFN pair p (expert e, token t = perm[p] / k) goes to padded row
 // p - offsets[e] + 128 * mb_off[e], so every expert's rows start a 128-row block.
+// Eight bf16 values per lane per 16-byte load: a warp-wide load covers 256 columns, the
+// two 128-column blocks of lanes 0..15 and 16..31; four loads in flight per lane.
+__device__ __forceinline__ void ld8_bf16(const __nv_bfloat16* p, float* v) {
+  const uint4 r = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ float half_warp_max(float a) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  return a;
+}
+// the lane's eight values of one [1,128] block: codes to dst, the block's scale (lanes 0 and 16)
+__device__ __forceinline__ void quant8_e4m3(const float* v, uint8_t* dst, uint8_t* scale, int lane) {
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+  const uint32_t code = e8m0_code(half_warp_max(m));
+  const float inv = e8m0_inverse(code);
+  *reinterpret_cast<uint2*>(dst) = make_uint2(pack_e4m3x4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv),
+                                              pack_e4m3x4(v[4] * inv, v[5] * inv, v[6] * inv, v[7] * inv));
+  if ((lane & 15) == 0) *scale = (uint8_t)code;
+}
+
 __global__ void __launch_bounds__(256) k_gather_quant(const __nv_bfloat16* __restrict__ x, int d,
                                                       const int32_t* __restrict__ perm,
                                                       const int32_t* __restrict__ idx, int k,
@@ -101,6 +130,7 @@ __global__ void __launch_bounds__(256) k_gather_quant(const __nv_bfloat16* __res
                                                       uint8_t* __restrict__ sx, int groups) {
   const int P = scal[0];
   const int lane = threadIdx.x & 31;
+  const int half = lane >> 4;
   const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
   for (int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); p < P; p += nwarps) {
     const int pair = perm[p];
@@ -108,21 +138,24 @@ __global__ void __launch_bounds__(256) k_gather_quant(const __nv_bfloat16* __res
     const int64_t pad = (int64_t)(p - offsets[e]) + (int64_t)mb_off[e] * 128;
     const __nv_bfloat16* src = x + (int64_t)(pair / k) * d;
     uint8_t* dst = x8 + pad * d;
-    for (int c0 = 0; c0 < d; c0 += 512) {  // d is a multiple of 512
-      // four 128-column blocks in flight per lane
-      float v[4][4];
+    int c0 = 0;
+    for (; c0 + 1024 <= d; c0 += 1024) {
+      float v[4][8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) ld4(src + c0 + 128 * u + lane * 4, v[u]);
+      for (int u = 0; u < 4; ++u) ld8_bf16(src + c0 + 256 * u + lane * 8, v[u]);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float amax =
-            warp_max(fmaxf(fmaxf(fabsf(v[u][0]), fabsf(v[u][1])), fmaxf(fabsf(v[u][2]), fabsf(v[u][3]))));
-        const uint32_t code = e8m0_code(amax);
-        const float inv = e8m0_inverse(code);
-        *reinterpret_cast<uint32_t*>(dst + c0 + 128 * u + lane * 4) =
-            pack_e4m3x4(v[u][0] * inv, v[u][1] * inv, v[u][2] * inv, v[u][3] * inv);
-        if (lane == 0) sx[atom_offset(pad, (c0 >> 7) + u, groups)] = (uint8_t)code;
-      }
+      for (int u = 0; u < 4; ++u)
+        quant8_e4m3(v[u], dst + c0 + 256 * u + lane * 8, sx + atom_offset(pad, ((c0 + 256 * u) >> 7) + half, groups),
+                    lane);
+    }
+    if (c0 < d) {  // d is a multiple of 512: a last 512 columns
+      float v[2][8];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) ld8_bf16(src + c0 + 256 * u + lane * 8, v[u]);
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        quant8_e4m3(v[u], dst + c0 + 256 * u + lane * 8, sx + atom_offset(pad, ((c0 + 256 * u) >> 7) + half, groups),
+                    lane);
     }
   }
 }
@@ -194,7 +227,20 @@ __global__ void __launch_bounds__(256) k_gather_quant4(const __nv_bfloat16* __re
     const int64_t pad = (int64_t)(p - offsets[e]) + (int64_t)mb_off[e] * 128;
     const __nv_bfloat16* src = x + (int64_t)(pair / k) * d;
     uint8_t* dst = x4 + pad * (d >> 1);
-    for (int c0 = 0; c0 < d; c0 += 512) {
+    int c0 = 0;
+    for (; c0 + 1024 <= d; c0 += 1024) {  // four 16-byte loads in flight per lane
+      float v[4][8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) ld8(src + c0 + 256 * u + lane * 8, v[u]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 256 * u + lane * 8;
+        const uint2 q = quant8_mx4(v[u]);
+        *reinterpret_cast<uint32_t*>(dst + (c >> 1)) = q.x;
+        if ((lane & 3) == 0) sx[atom_offset(pad, c >> 5, groups)] = (uint8_t)q.y;
+      }
+    }
+    if (c0 < d) {  // d is a multiple of 512: a last 512 columns
       float v[2][8];
 #pragma unroll
       for (int u = 0; u < 2; ++u) ld8(src + c0 + 256 * u + lane * 8, v[u]);
