@@ -68,6 +68,10 @@ WORKLOADS = {
     # inputs still larger than L2
     "prefill_probe": Workload("prefill_probe", T=2048, d=6144, n_ffn=32, inter=2048, n_zero=16, top_k=12,
                               dtype="bf16", w_std=0.006, bias=("zero",), dense_inter=12288),
+    # the 560B layer's expert shape with 16 experts (1.2 GB of weights): small captures of the
+    # backward kernels, ~512 rows per expert as at prefill
+    "bwd_probe": Workload("bwd_probe", T=1024, d=6144, n_ffn=16, inter=2048, n_zero=8, top_k=12, dtype="bf16",
+                          w_std=0.006, bias=("zero",)),
 }
 # the same layers with block-scaled FP8 and W4A4 (MXFP4) experts
 for _name in ("small_bf16", "prefill_560b", "decode_560b", "skewed_4096", "prefill_probe"):
