@@ -365,6 +365,7 @@ def measure_backward(wl, layer, x, stream, peaks, P):
              "up": torch.zeros((wl.n_ffn, wl.inter, wl.d), device=x.device),
              "down": torch.zeros((wl.n_ffn, wl.d, wl.inter), device=x.device)}
     ms_full = graph_ms(lambda: layer.backward(x, dy, dx, grads=grads), stream, reps=3)
+    ms_full_ow = graph_ms(lambda: layer.backward(x, dy, dx, grads=grads, accumulate=False), stream, reps=3)
     layer.check()
     ok = all(bool(torch.isfinite(t).all()) for t in grads.values())
     del grads
@@ -377,7 +378,7 @@ def measure_backward(wl, layer, x, stream, peaks, P):
     return {"ms_dx_only": ms_dx, "ms_with_weight_grads": ms_full, "tflops_dx_only": f_dx / (ms_dx * 1e-3) / 1e12,
             "tflops_total": (f_dx + f_w) / (ms_full * 1e-3) / 1e12, "gemmadd_accumulator_bytes": acc_bytes,
             "gemmadd_hbm_ms": 1e3 * acc_bytes / (peaks["hbm_gbs"] * 1e9), "finite": ok,
-            "ms_dx_only_recompute": ms_dx_recompute, "ms_forward": ms_fwd, "ms_forward_saving_gu": ms_fwd_saving,
+            "ms_with_weight_grads_overwrite": ms_full_ow, "ms_dx_only_recompute": ms_dx_recompute, "ms_forward": ms_fwd, "ms_forward_saving_gu": ms_fwd_saving,
             "note": "training mode (forward stores G, U); weight gradients added into fp32 accumulators "
                     "(3 x 25.8 GB + router); each a replayed graph"}
 

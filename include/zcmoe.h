@@ -249,6 +249,14 @@ ZCMOE_API int zcmoe_destroy(zcmoe_t h);
 ZCMOE_API int zcmoe_backward(zcmoe_t h, const void *x, const void *dy, int64_t T, void *dx, float *g_router,
                              float *g_gate, float *g_up, float *g_down, cudaStream_t stream);
 
+/* zcmoe_backward with flags.  ZCMOE_GRAD_OVERWRITE: the weight gradients are WRITTEN into
+ * g_router / g_gate / g_up / g_down instead of added (the epilogue stores its product; an expert
+ * that no token picked gets zeros), so the accumulators are not read: half the HBM traffic of the
+ * weight gradients, for the first micro-batch of an accumulation.  Other bits: ZCMOE_EINVAL. */
+#define ZCMOE_GRAD_OVERWRITE 1u
+ZCMOE_API int zcmoe_backward_ex(zcmoe_t h, const void *x, const void *dy, int64_t T, void *dx, float *g_router,
+                                float *g_gate, float *g_up, float *g_down, uint32_t flags, cudaStream_t stream);
+
 /* Training mode for zcmoe_backward, bf16 layers.  on = 1: every later forward also
  * stores the gate/up GEMM's outputs G = X W_g^T and U = X W_u^T of its FFN pairs
  * (rounded to bf16; 4 * inter bytes per padded pair row, allocated here, about

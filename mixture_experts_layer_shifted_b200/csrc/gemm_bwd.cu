@@ -118,6 +118,13 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* tm, const v
                "r"(smem_u32(src)), "r"(n), "r"(m), "r"(g)
                : "memory");
 }
+// TMA store of a 32 x 32 fp32 box (the same staging and tensor map): the overwrite mode.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* tm, const void* src, int n, int m, int g) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(smem_u32(src)), "r"(n), "r"(m), "r"(g)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void bulk_wait_read() {
@@ -290,7 +297,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int chunk = 0;  // kEpiAddF32: reduce-adds issued by this warp (selects the staging buffer)
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const Tile ti = decode_tile<SCHED>(args, t);
-      if (ti.num_k == 0) continue;
+      if (ti.num_k == 0) {
+        if (EPI == kEpiAddF32 && args.overwrite) {
+          // overwrite mode: an expert with no rows has a zero gradient (no MMA, no TMEM)
+          constexpr int NB = NBUF > 0 ? NBUF : 1;
+          const int m0 = ti.m_blk * BM + quarter * 32;
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 32) {
+            const int n0 = ti.n_blk * BN + c;
+            if (m0 >= args.m_out || n0 >= args.n_out) continue;
+            uint8_t* stg = sStg + (quarter * NB + chunk % NB) * STG_BYTES;
+            if (lane == 0) bulk_wait_read<NB - 1>();
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(stg + lane * 128 + j * 16) = make_uint4(0, 0, 0, 0);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tmC, stg, n0, m0, ti.g);
+              bulk_commit();
+            }
+            ++chunk;
+          }
+        }
+        continue;
+      }
       if (!mbar_wait(&tfull[acc], acc_phase, err, 25)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
@@ -420,7 +451,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       } else {
         // fused GemmAdd: acc[g][m][n] += product in fp32, done by TMA reduce-adds of
-        // 32 x 32 boxes (the L2 does the read-modify-write; each element is added once)
+        // 32 x 32 boxes (the L2 does the read-modify-write; each element is added once);
+        // overwrite mode: TMA stores of the same boxes (acc[g][m][n] = product)
         const int m0 = ti.m_blk * BM + quarter * 32;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -440,7 +472,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           fence_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_reduce_add_3d(&tmC, stg, n0, m0, ti.g);
+            if (args.overwrite) tma_store_3d(&tmC, stg, n0, m0, ti.g);
+            else tma_reduce_add_3d(&tmC, stg, n0, m0, ti.g);
             bulk_commit();
           }
           ++chunk;

@@ -147,6 +147,7 @@ struct BwdArgs {
   __nv_bfloat16* hpad;       //   out: H [padded rows, inter]
   int inter;
   float* acc;                // kEpiAddF32: acc[g][m][n] += product (through the tensor map c)
+  int overwrite;             //   1: acc[g][m][n] = product instead (experts with no rows get zeros)
   int64_t acc_ld, acc_group_stride;
   int* err;                  // device error word (bounded waits)
 };

@@ -1155,9 +1155,10 @@ int zcmoe_save_for_backward(zcmoe_t h, int32_t on) {
   return ZCMOE_OK;
 }
 
-int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx, float* g_router, float* g_gate,
-                   float* g_up, float* g_down, cudaStream_t s) {
+int zcmoe_backward_ex(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx, float* g_router, float* g_gate,
+                      float* g_up, float* g_down, uint32_t flags, cudaStream_t s) {
   g_err[0] = 0;
+  if (flags & ~(uint32_t)ZCMOE_GRAD_OVERWRITE) return fail(ZCMOE_EINVAL, "unknown flags 0x%x", flags);
   if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
   if (!h->bf16 || h->fp8) return fail(ZCMOE_EUNSUPPORTED, "the backward pass needs a bf16 layer");
   if (h->ep_size > 1) return fail(ZCMOE_EUNSUPPORTED, "the backward pass needs a layer that holds all experts");
@@ -1328,6 +1329,7 @@ int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx
     a.n_out = n_out;
     a.nblocks = (n_out + 255) / 256;
     a.acc = acc;
+    a.overwrite = (flags & ZCMOE_GRAD_OVERWRITE) ? 1 : 0;
     a.acc_ld = n_out;
     a.acc_group_stride = stride;
     a.err = h->err;
@@ -1345,6 +1347,11 @@ int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx
     return rc;
   if (g_router && (rc = wgrad(tm_dl_mn, tm_xin_mn, 0, E, d, g_router, 0, 1, h->b_grp, h->b_grp + 2))) return rc;
   return ZCMOE_OK;
+}
+
+int zcmoe_backward(zcmoe_t h, const void* x, const void* dy, int64_t T, void* dx, float* g_router, float* g_gate,
+                   float* g_up, float* g_down, cudaStream_t s) {
+  return zcmoe_backward_ex(h, x, dy, T, dx, g_router, g_gate, g_up, g_down, 0u, s);
 }
 
 int zcmoe_quantize_e4m3(const void* src, int32_t src_dtype, int64_t rows, int64_t cols, int32_t block_rows,

@@ -36,7 +36,7 @@ EXPORTED = ("zcmoe_create", "zcmoe_forward", "zcmoe_forward_host", "zcmoe_update
             "zcmoe_profile_end", "zcmoe_selftest_wait", "zcmoe_route_noalloc", "zcmoe_destroy",
             "zcmoe_dense_create", "zcmoe_dense_forward", "zcmoe_forward_overlap", "zcmoe_dense_check",
             "zcmoe_dense_destroy", "zcmoe_quantize_e4m3", "zcmoe_quantize_mx4", "zcmoe_backward",
-            "zcmoe_save_for_backward", "zcmoe_create_ep", "zcmoe_ep_dispatch", "zcmoe_ep_experts",
+            "zcmoe_save_for_backward", "zcmoe_backward_ex", "zcmoe_create_ep", "zcmoe_ep_dispatch", "zcmoe_ep_experts",
             "zcmoe_ep_combine", "zcmoe_last_error")
 STAGES = ("router", "softmax_topk", "integer", "gather", "gate_up", "down", "combine")
 
@@ -112,6 +112,7 @@ def lib():
         L.zcmoe_quantize_e4m3.argtypes = [vp, ctypes.c_int32, i64, i64, ctypes.c_int32, vp, vp, vp]
         L.zcmoe_quantize_mx4.argtypes = [vp, ctypes.c_int32, i64, i64, vp, vp, vp]
         L.zcmoe_backward.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, vp, vp]
+        L.zcmoe_backward_ex.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, vp, ctypes.c_uint32, vp]
         L.zcmoe_save_for_backward.argtypes = [vp, ctypes.c_int32]
         L.zcmoe_create_ep.argtypes = [ctypes.POINTER(zcmoe_config), ctypes.POINTER(zcmoe_weights), ctypes.c_int32,
                                       ctypes.c_int32, i64, ctypes.POINTER(vp)]
@@ -271,9 +272,17 @@ def quantize_e4m3(src, block_rows, stream=None):
     return codes, scales
 
 
-def zcmoe_backward(h, x_ptr, dy_ptr, T, dx_ptr, g_router=None, g_gate=None, g_up=None, g_down=None, stream=None):
-    _check(lib().zcmoe_backward(h, x_ptr, dy_ptr, T, dx_ptr, g_router, g_gate, g_up, g_down, _stream(stream)),
-           "zcmoe_backward")
+ZCMOE_GRAD_OVERWRITE = 1
+
+
+def zcmoe_backward(h, x_ptr, dy_ptr, T, dx_ptr, g_router=None, g_gate=None, g_up=None, g_down=None, stream=None,
+                   flags=0):
+    if flags:
+        _check(lib().zcmoe_backward_ex(h, x_ptr, dy_ptr, T, dx_ptr, g_router, g_gate, g_up, g_down, flags,
+                                       _stream(stream)), "zcmoe_backward_ex")
+    else:
+        _check(lib().zcmoe_backward(h, x_ptr, dy_ptr, T, dx_ptr, g_router, g_gate, g_up, g_down, _stream(stream)),
+               "zcmoe_backward")
 
 
 def zcmoe_save_for_backward(h, on):
@@ -365,14 +374,16 @@ class ZcMoE:
                            ctypes.c_void_p(y_host.data_ptr()), stream)
         return y_host
 
-    def backward(self, x, dy, dx=None, grads: dict | None = None, stream=None):
+    def backward(self, x, dy, dx=None, grads: dict | None = None, stream=None, accumulate=True):
         """dx of the last forward (x must be the tensor it read); adds the weight gradients
-        into the fp32 tensors of ``grads`` (keys router, gate, up, down; missing: skipped)."""
+        into the fp32 tensors of ``grads`` (keys router, gate, up, down; missing: skipped), or
+        writes them there with accumulate=False."""
         dx = torch.empty_like(x) if dx is None else dx
         g = grads or {}
         ptr = lambda name: ctypes.c_void_p(g[name].data_ptr()) if name in g else None  # noqa: E731
         zcmoe_backward(self.h, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(dy.data_ptr()), x.shape[0],
-                       ctypes.c_void_p(dx.data_ptr()), ptr("router"), ptr("gate"), ptr("up"), ptr("down"), stream)
+                       ctypes.c_void_p(dx.data_ptr()), ptr("router"), ptr("gate"), ptr("up"), ptr("down"), stream,
+                       flags=0 if accumulate else ZCMOE_GRAD_OVERWRITE)
         return dx
 
     def save_for_backward(self, on=True):

@@ -42,8 +42,8 @@ def _grads(w, init=0.0, seed=0):
     return {k_: (torch.randn(s_, generator=g, device="cuda") * init) for k_, s_ in shapes.items()}
 
 
-def _run_backward(r, dy, grads):
-    dx = r.layer.backward(r.x, dy, grads=grads)
+def _run_backward(r, dy, grads, accumulate=True):
+    dx = r.layer.backward(r.x, dy, grads=grads, accumulate=accumulate)
     torch.cuda.synchronize()
     r.layer.check()
     return dx
@@ -100,7 +100,7 @@ def _cmp(got, ref, name):
     return float(err.max())
 
 
-def _case(w, T=None, init=0.5, saved=False):
+def _case(w, T=None, init=0.5, saved=False, accumulate=True):
     r = Run(w, T=T, max_tokens=(T or w.T) + 3)
     try:
         if saved:
@@ -110,12 +110,14 @@ def _case(w, T=None, init=0.5, saved=False):
         dy = (torch.randn((r.T, w.d), generator=g, device="cuda") * 0.1).to(torch.bfloat16)
         grads = _grads(w, init)
         before = {k_: v.clone() for k_, v in grads.items()}
-        dx = _run_backward(r, dy, grads)
+        dx = _run_backward(r, dy, grads, accumulate)
         ref = _oracle_backward(r, _bf16_to_f64(to_host_bits(dy)))
         _cmp(_bf16_to_f64(to_host_bits(dx)), ref[0], "dx")
         for name, i in (("router", 1), ("gate", 2), ("up", 3), ("down", 4)):
-            added = (grads[name] - before[name]).double().cpu().numpy()
-            _cmp(added, ref[i], name)
+            # accumulate: what was added; overwrite: what is there (experts no token
+            # picked must then hold exact zeros, whatever the accumulator held before)
+            got = (grads[name] - before[name]) if accumulate else grads[name]
+            _cmp(got.double().cpu().numpy(), ref[i], name)
         return r, dy
     except BaseException:
         r.close()
@@ -125,6 +127,17 @@ def _case(w, T=None, init=0.5, saved=False):
 @pytest.mark.parametrize("saved", [False, True], ids=["recompute", "saved"])
 def test_backward_small(cuda_ok, saved):
     r, _ = _case(W["small_bf16"], saved=saved)
+    r.close()
+
+
+@pytest.mark.parametrize("T,N", [(600, 64), (1, 8)], ids=["600-tokens", "one-token"])
+def test_backward_overwrite_mode(cuda_ok, T, N):
+    """ZCMOE_GRAD_OVERWRITE: the gradients replace the accumulators' contents (non-zero
+    before); with one token most experts get exact zeros."""
+    w = W["small_bf16"] if T > 1 else configs.Workload("one_tok", T=1, d=256, n_ffn=N, inter=128, n_zero=4, top_k=3,
+                                                       dtype="bf16", w_std=0.05, bias=("uniform", -0.05, 0.05),
+                                                       seed=3)
+    r, _ = _case(w, T=T, saved=True, accumulate=False)
     r.close()
 
 
