@@ -715,6 +715,24 @@ def main():
             "gpu_launches": 10 * args.steps, "clocks": clocks, "peaks": peaks,
             "launch": "cuda graph per step" if use_graph else "eager"}
 
+    # the controller over the workload's steps (Zipf-skewed routing): FFN experts per token per
+    # step, from a fresh layer, a batch per step; outside the timed region (reads counts each step)
+    if rank == 0 and ws == 1 and wl.steps > 1:
+        ctl = ZcMoE(shape, *weights, max_tokens=wl.T, init_bias=bias, logit_offset=offset)
+        traj = []
+        yc = torch.empty_like(xs[0])
+        for i in range(wl.steps):
+            ctl.forward(configs.device_tokens(wl, step=i), yc)
+            st = ctl.state()
+            traj.append(float(st["counts"][: wl.n_ffn].sum()) / st["tokens"])
+            ctl.update_bias(target_ffn_per_token=target, **GAINS)
+        ctl.check()
+        ctl.close()
+        line["controller"] = {"target_ffn_per_token": target, "steps": wl.steps, "gains": GAINS,
+                              "ffn_per_token_first": traj[0], "ffn_per_token_last": traj[-1],
+                              "ffn_per_token_mean_last10": float(np.mean(traj[-10:])),
+                              "trajectory_every_10": traj[::10]}
+
     # secondary workload (decode): reported beside the headline, not as the headline
     if rank == 0 and ws == 1 and "decode" in sec and wl.name == "prefill_560b":
         wd = configs.WORKLOADS["decode_560b"]
