@@ -668,19 +668,23 @@ def main():
                            "tflops": 2.0 * wl.d * wl.inter * P / (stage_avg["down"] * 1e-3) / 1e12}}
 
     # ---------------------------------------------------------------- e2e through host buffers (C ABI, pinned)
-    xh = xs[0].cpu().pin_memory()
-    yh = torch.empty_like(xh).pin_memory()
-    for _ in range(2):
-        layer.forward_host(xh, yh)
+    # pipelined: step i's y download and step i+1's x upload run beside the forwards; the
+    # flush before the closing event waits for the last download
+    xh = [x.cpu().pin_memory() for x in xs]
+    yh = [torch.empty_like(xh[0]).pin_memory() for _ in range(2)]
+    for i in range(2):
+        layer.forward_host(xh[i], yh[i], pipelined=True)
+    layer.flush_host()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_e2e = max(3, min(args.steps, 10))
     e0.record(stream)
-    for _ in range(n_e2e):
-        layer.forward_host(xh, yh)
+    for i in range(n_e2e):
+        layer.forward_host(xh[i % 2], yh[i % 2], pipelined=True)
         layer.update_bias(target_ffn_per_token=target, **GAINS)
+    layer.flush_host()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / n_e2e
@@ -688,7 +692,7 @@ def main():
         t = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
-    io_bytes = xh.numel() * xh.element_size()
+    io_bytes = xh[0].numel() * xh[0].element_size()
     e2e = {"value": wl.T * ws / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
            "d2h_bytes_per_step": io_bytes, "ms_per_step": e2e_ms}
 

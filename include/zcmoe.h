@@ -148,6 +148,16 @@ ZCMOE_API int zcmoe_forward(zcmoe_t h, const void *x, int64_t T, void *y, cudaSt
  * forward, and y_host is complete once `stream` has been synchronised. */
 ZCMOE_API int zcmoe_forward_host(zcmoe_t h, const void *x_host, int64_t T, void *y_host, cudaStream_t stream);
 
+/* The same, pipelined over calls: the download of this call's y runs on an internal stream
+ * beside the NEXT call's forward (and its upload beside the previous call's), so a loop of
+ * calls overlaps both copies with the compute.  y_host is complete once `stream` has passed
+ * the next zcmoe_forward_host_async / zcmoe_forward_host on this handle, or a
+ * zcmoe_forward_host_flush; keep it untouched until then.  x_host may be reused once
+ * `stream` has passed this call's forward. */
+ZCMOE_API int zcmoe_forward_host_async(zcmoe_t h, const void *x_host, int64_t T, void *y_host, cudaStream_t stream);
+/* Makes `stream` wait for the download of the last zcmoe_forward_host_async. */
+ZCMOE_API int zcmoe_forward_host_flush(zcmoe_t h, cudaStream_t stream);
+
 /* One bias-controller step (zhangjingwei.cn 二.1 "PID controller"; web3.cnouyi.fund
  * "decay schedule"), fp32 with every operation rounded once:
  *   load l_i = c_i / T_acc from the accumulated counts; target tau_i = K/N for FFN

@@ -166,9 +166,11 @@ struct zcmoe_s {
   void *xperm, *H, *Y;
   // zcmoe_forward_host: x staged through two device buffers filled on an internal
   // copy stream, so the next call's upload overlaps this call's compute; y staged once
-  void *stage_x, *stage_x2, *stage_y;
-  cudaStream_t copy_stream;
-  cudaEvent_t ev_in[2], ev_used[2];
+  // zcmoe_forward_host(_async): x and y staged through two device buffers each; uploads on
+  // copy_stream, downloads on d2h_stream, so a call's copies overlap its neighbours' forwards
+  void *stage_x, *stage_x2, *stage_y, *stage_y2;
+  cudaStream_t copy_stream, d2h_stream;
+  cudaEvent_t ev_in[2], ev_used[2], ev_fwd[2], ev_ydone[2];
   long long host_calls;
   // stage timing (zcmoe_profile_begin/end): ZCMOE_NUM_STAGES + 1 events per forward
   bool profiling;
@@ -210,7 +212,7 @@ static void release(zcmoe_s* h) {
   void* ptrs[] = {h->bias,  h->b0,     h->offset, h->eta,   h->integ,   h->eprev,  h->acc_counts,
                   h->err,   h->logits, h->gate,   h->idx,   h->pos,     h->counts, h->offsets,
                   h->mb_off, h->scal,  h->chunk,  h->perm,  h->xperm,   h->H,      h->Y,
-                  h->stage_x, h->stage_x2, h->stage_y, h->w8g, h->w8u, h->w8d, h->sfg, h->sfu, h->sfd,
+                  h->stage_x, h->stage_x2, h->stage_y, h->stage_y2, h->w8g, h->w8u, h->w8d, h->sfg, h->sfu, h->sfd,
                   h->x8, h->sx, h->h8, h->sh, h->ypad, h->b_xpad, h->b_dypad, h->b_dh, h->b_dgu, h->b_hpad,
                   h->b_dxp, h->b_dl, h->b_dxr, h->b_dg, h->b_grp, h->b_gu, h->ep_meta};
   for (void* p : ptrs)
@@ -218,10 +220,12 @@ static void release(zcmoe_s* h) {
   if (h->ep_meta_host) cudaFreeHost(h->ep_meta_host);
   if (h->ep_meta_ev) cudaEventDestroy(h->ep_meta_ev);
   for (int i = 0; i < 2; ++i) {
-    if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
-    if (h->ev_used[i]) cudaEventDestroy(h->ev_used[i]);
+    cudaEvent_t evs[4] = {h->ev_in[i], h->ev_used[i], h->ev_fwd[i], h->ev_ydone[i]};
+    for (cudaEvent_t e : evs)
+      if (e) cudaEventDestroy(e);
   }
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
+  if (h->d2h_stream) cudaStreamDestroy(h->d2h_stream);
   if (h->events) {
     for (cudaEvent_t e : *h->events) cudaEventDestroy(e);
     delete h->events;
@@ -964,55 +968,91 @@ int zcmoe_ep_combine(zcmoe_t h, const void* x, const void* yback, int64_t T, voi
   return ZCMOE_OK;
 }
 
-int zcmoe_forward_host(zcmoe_t h, const void* x_host, int64_t T, void* y_host, cudaStream_t s) {
-  g_err[0] = 0;
-  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+// Call i uses staging buffers i % 2.  Upload (copy_stream, after forward i-2 has read the
+// buffer) -> forward on `s` (after the upload and after download i-2 has read the y buffer)
+// -> download (d2h_stream, after the forward).  At the end of the call `s` waits for
+// download i-1 (async form) or download i (zcmoe_forward_host): in the async form, forward i
+// runs while download i-1 and upload i+1 move.
+static int forward_host_impl(zcmoe_t h, const void* x_host, int64_t T, void* y_host, cudaStream_t s, bool async) {
   if (T < 0 || T > h->max_T) return fail(ZCMOE_ERANGE, "T=%lld outside [0, %d]", (long long)T, h->max_T);
   if (T == 0) return ZCMOE_OK;
   if (!x_host || !y_host) return fail(ZCMOE_EINVAL, "x or y is NULL");
   const size_t bytes_max = (size_t)h->max_T * h->d * (h->bf16 ? 2 : 4);
   if (!h->stage_x) {
-    uint8_t *a = nullptr, *a2 = nullptr, *b = nullptr;
+    uint8_t *a = nullptr, *a2 = nullptr, *b = nullptr, *b2 = nullptr;
     int rc = dalloc(&a, bytes_max);
     if (rc == ZCMOE_OK) rc = dalloc(&a2, bytes_max);
     if (rc == ZCMOE_OK) rc = dalloc(&b, bytes_max);
+    if (rc == ZCMOE_OK) rc = dalloc(&b2, bytes_max);
     cudaError_t e = cudaSuccess;
     if (rc == ZCMOE_OK) e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking);
+    if (rc == ZCMOE_OK && e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->d2h_stream, cudaStreamNonBlocking);
     for (int i = 0; i < 2 && rc == ZCMOE_OK && e == cudaSuccess; ++i) {
-      e = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming);
-      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_used[i], cudaEventDisableTiming);
+      cudaEvent_t* evs[4] = {&h->ev_in[i], &h->ev_used[i], &h->ev_fwd[i], &h->ev_ydone[i]};
+      for (cudaEvent_t* ev : evs)
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
     }
     if (rc != ZCMOE_OK || e != cudaSuccess) {
-      if (a) cudaFree(a);
-      if (a2) cudaFree(a2);
-      if (b) cudaFree(b);
+      uint8_t* bufs[4] = {a, a2, b, b2};
+      for (uint8_t* p : bufs)
+        if (p) cudaFree(p);
       for (int i = 0; i < 2; ++i) {
-        if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
-        if (h->ev_used[i]) cudaEventDestroy(h->ev_used[i]);
-        h->ev_in[i] = h->ev_used[i] = nullptr;
+        cudaEvent_t* evs[4] = {&h->ev_in[i], &h->ev_used[i], &h->ev_fwd[i], &h->ev_ydone[i]};
+        for (cudaEvent_t* ev : evs) {
+          if (*ev) cudaEventDestroy(*ev);
+          *ev = nullptr;
+        }
       }
       if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
-      h->copy_stream = nullptr;
+      if (h->d2h_stream) cudaStreamDestroy(h->d2h_stream);
+      h->copy_stream = h->d2h_stream = nullptr;
       if (rc != ZCMOE_OK) return rc;
-      return fail(ZCMOE_ECUDA, "creating the copy stream: %s", cudaGetErrorString(e));
+      return fail(ZCMOE_ECUDA, "creating the copy streams: %s", cudaGetErrorString(e));
     }
     h->stage_x = a;
     h->stage_x2 = a2;
     h->stage_y = b;
+    h->stage_y2 = b2;
   }
   const size_t bytes = (size_t)T * h->d * (h->bf16 ? 2 : 4);
   const int buf = (int)(h->host_calls & 1);
   void* sx = buf ? h->stage_x2 : h->stage_x;
-  // the buffer was last read by the forward two calls ago
+  void* sy = buf ? h->stage_y2 : h->stage_y;
   if (h->host_calls >= 2) ZC_CUDA(cudaStreamWaitEvent(h->copy_stream, h->ev_used[buf], 0));
   ZC_CUDA(cudaMemcpyAsync(sx, x_host, bytes, cudaMemcpyHostToDevice, h->copy_stream));
   ZC_CUDA(cudaEventRecord(h->ev_in[buf], h->copy_stream));
   ZC_CUDA(cudaStreamWaitEvent(s, h->ev_in[buf], 0));
-  int rc = zcmoe_forward(h, sx, T, h->stage_y, s, nullptr);
+  if (h->host_calls >= 2) ZC_CUDA(cudaStreamWaitEvent(s, h->ev_ydone[buf], 0));
+  int rc = zcmoe_forward(h, sx, T, sy, s, nullptr);
   if (rc != ZCMOE_OK) return rc;
   ZC_CUDA(cudaEventRecord(h->ev_used[buf], s));
-  ZC_CUDA(cudaMemcpyAsync(y_host, h->stage_y, bytes, cudaMemcpyDeviceToHost, s));
+  ZC_CUDA(cudaEventRecord(h->ev_fwd[buf], s));
+  ZC_CUDA(cudaStreamWaitEvent(h->d2h_stream, h->ev_fwd[buf], 0));
+  ZC_CUDA(cudaMemcpyAsync(y_host, sy, bytes, cudaMemcpyDeviceToHost, h->d2h_stream));
+  ZC_CUDA(cudaEventRecord(h->ev_ydone[buf], h->d2h_stream));
+  if (!async) ZC_CUDA(cudaStreamWaitEvent(s, h->ev_ydone[buf], 0));
+  else if (h->host_calls >= 1) ZC_CUDA(cudaStreamWaitEvent(s, h->ev_ydone[buf ^ 1], 0));
   ++h->host_calls;
+  return ZCMOE_OK;
+}
+
+int zcmoe_forward_host(zcmoe_t h, const void* x_host, int64_t T, void* y_host, cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  return forward_host_impl(h, x_host, T, y_host, s, false);
+}
+
+int zcmoe_forward_host_async(zcmoe_t h, const void* x_host, int64_t T, void* y_host, cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  return forward_host_impl(h, x_host, T, y_host, s, true);
+}
+
+int zcmoe_forward_host_flush(zcmoe_t h, cudaStream_t s) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (h->host_calls == 0) return ZCMOE_OK;
+  ZC_CUDA(cudaStreamWaitEvent(s, h->ev_ydone[(int)((h->host_calls - 1) & 1)], 0));
   return ZCMOE_OK;
 }
 

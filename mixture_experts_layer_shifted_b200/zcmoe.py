@@ -36,7 +36,8 @@ EXPORTED = ("zcmoe_create", "zcmoe_forward", "zcmoe_forward_host", "zcmoe_update
             "zcmoe_profile_end", "zcmoe_selftest_wait", "zcmoe_route_noalloc", "zcmoe_destroy",
             "zcmoe_dense_create", "zcmoe_dense_forward", "zcmoe_forward_overlap", "zcmoe_dense_check",
             "zcmoe_dense_destroy", "zcmoe_quantize_e4m3", "zcmoe_quantize_mx4", "zcmoe_backward",
-            "zcmoe_save_for_backward", "zcmoe_backward_ex", "zcmoe_create_ep", "zcmoe_ep_dispatch", "zcmoe_ep_experts",
+            "zcmoe_save_for_backward", "zcmoe_backward_ex", "zcmoe_forward_host_async",
+            "zcmoe_forward_host_flush", "zcmoe_create_ep", "zcmoe_ep_dispatch", "zcmoe_ep_experts",
             "zcmoe_ep_combine", "zcmoe_last_error")
 STAGES = ("router", "softmax_topk", "integer", "gather", "gate_up", "down", "combine")
 
@@ -92,6 +93,8 @@ def lib():
         L.zcmoe_create.argtypes = [ctypes.POINTER(zcmoe_config), ctypes.POINTER(zcmoe_weights), ctypes.POINTER(vp)]
         L.zcmoe_forward.argtypes = [vp, vp, i64, vp, vp, ctypes.POINTER(zcmoe_debug)]
         L.zcmoe_forward_host.argtypes = [vp, vp, i64, vp, vp]
+        L.zcmoe_forward_host_async.argtypes = [vp, vp, i64, vp, vp]
+        L.zcmoe_forward_host_flush.argtypes = [vp, vp]
         L.zcmoe_update_bias.argtypes = [vp, ctypes.POINTER(zcmoe_gains), vp]
         L.zcmoe_read_counts.argtypes = [vp, vp, vp]
         L.zcmoe_write_counts.argtypes = [vp, vp, vp]
@@ -178,6 +181,14 @@ def zcmoe_forward(h, x_ptr, T, y_ptr, stream=None, dbg: zcmoe_debug | None = Non
 
 def zcmoe_forward_host(h, x_host_ptr, T, y_host_ptr, stream=None):
     _check(lib().zcmoe_forward_host(h, x_host_ptr, T, y_host_ptr, _stream(stream)), "zcmoe_forward_host")
+
+
+def zcmoe_forward_host_async(h, x_host_ptr, T, y_host_ptr, stream=None):
+    _check(lib().zcmoe_forward_host_async(h, x_host_ptr, T, y_host_ptr, _stream(stream)), "zcmoe_forward_host_async")
+
+
+def zcmoe_forward_host_flush(h, stream=None):
+    _check(lib().zcmoe_forward_host_flush(h, _stream(stream)), "zcmoe_forward_host_flush")
 
 
 def zcmoe_update_bias(h, gains: zcmoe_gains, stream=None):
@@ -369,10 +380,15 @@ class ZcMoE:
         zcmoe_forward(self.h, ctypes.c_void_p(x.data_ptr()), T, ctypes.c_void_p(y.data_ptr()), stream, dbg)
         return y
 
-    def forward_host(self, x_host, y_host, stream=None):
-        zcmoe_forward_host(self.h, ctypes.c_void_p(x_host.data_ptr()), x_host.shape[0],
-                           ctypes.c_void_p(y_host.data_ptr()), stream)
+    def forward_host(self, x_host, y_host, stream=None, pipelined=False):
+        """y_host = layer(x_host), both page-locked host tensors.  pipelined: y_host is complete
+        once the stream has passed the next forward_host call or flush_host()."""
+        fn = zcmoe_forward_host_async if pipelined else zcmoe_forward_host
+        fn(self.h, ctypes.c_void_p(x_host.data_ptr()), x_host.shape[0], ctypes.c_void_p(y_host.data_ptr()), stream)
         return y_host
+
+    def flush_host(self, stream=None):
+        zcmoe_forward_host_flush(self.h, stream)
 
     def backward(self, x, dy, dx=None, grads: dict | None = None, stream=None, accumulate=True):
         """dx of the last forward (x must be the tensor it read); adds the weight gradients

@@ -237,6 +237,25 @@ def test_forward_host_matches_device(small):
     np.testing.assert_array_equal(yh.view(torch.int16).numpy().view(np.uint16), small.y)
 
 
+@pytest.mark.parametrize("n", [1, 2, 5])
+def test_forward_host_pipelined(small, n):
+    """The pipelined host-buffer forward: each call's output, complete after the next call
+    (or the flush), equals the device forward of its input; the stream is not synchronised
+    between calls, and a plain zcmoe_forward_host call in between keeps the order."""
+    xs = [configs.device_tokens(small.w, step=s) for s in range(10, 10 + n)]
+    want = []
+    for x in xs:
+        want.append(small.layer.forward(x).view(torch.int16).cpu().numpy())
+    xh = [x.cpu().pin_memory() for x in xs]
+    yh = [torch.empty_like(x).pin_memory() for x in xh]
+    for i, (a, b) in enumerate(zip(xh, yh)):
+        small.layer.forward_host(a, b, pipelined=(i != 2))  # call 2 (if any) is the plain form
+    small.layer.flush_host()
+    torch.cuda.synchronize()
+    for b, w in zip(yh, want):
+        np.testing.assert_array_equal(b.view(torch.int16).numpy(), w)
+
+
 def test_forward_host_back_to_back_calls(small):
     """Several host-buffer calls in flight (uploads double-buffered on the copy
     stream) each return their own input's output."""
