@@ -187,7 +187,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      constexpr uint32_t idesc128 = idesc_bf16_f32(BM, BN);
+      constexpr uint32_t idesc64 = idesc_bf16_f32(64, BN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -197,6 +198,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, err, 2)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        // a tile of at most 64 valid rows (an expert's last row block) runs M = 64 MMAs: the
+        // same issue time as M = 128, about half the energy (a power-capped GPU keeps a higher
+        // clock); its rows land in TMEM lanes 32q + (0..15), q = 0..3
+        const uint32_t idesc = decode_tile<MODE>(args, t).rows_valid <= 64 ? idesc64 : idesc128;
         for (int kb = 0; kb < num_k; ++kb) {
           if (!mbar_wait(&full[stage], phase, err, 3)) {
             ok = false;
@@ -230,7 +235,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter+32)
-    const int row_in_tile = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
@@ -238,6 +242,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait(&tfull[acc], acc_phase, err, 5)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+      // M = 64 tiles (see the MMA issuer): row 16 quarter + lane in lanes 0..15 of the quarter
+      const bool m64 = ti.rows_valid <= 64;
+      const int row_in_tile = m64 ? (lane < 16 ? quarter * 16 + lane : BM) : quarter * 32 + lane;
       const bool row_ok = row_in_tile < ti.rows_valid;
       const int64_t grow = (int64_t)ti.a_row + row_in_tile;
       if (MODE == kGateUp) {
