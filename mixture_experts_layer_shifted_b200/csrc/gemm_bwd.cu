@@ -246,7 +246,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
-      const uint32_t idesc = idesc_bf16_f32(BM, BN) | ((A_MN ? 1u : 0u) << 15) | ((B_MN ? 1u : 0u) << 16);
+      const uint32_t majors = ((A_MN ? 1u : 0u) << 15) | ((B_MN ? 1u : 0u) << 16);
+      const uint32_t idesc128 = idesc_bf16_f32(BM, BN) | majors, idesc64 = idesc_bf16_f32(64, BN) | majors;
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -258,6 +259,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, err, 22)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        // a row tile of at most 64 valid rows runs M = 64 MMAs (same issue time, about half
+        // the energy); its rows land in TMEM lanes 32q + (0..15)
+        const uint32_t idesc = (SCHED == kSchedRows && ti.rows_valid <= 64) ? idesc64 : idesc128;
         for (int kb = 0; kb < ti.num_k; ++kb) {
           if (!mbar_wait(&full[stage], phase, err, 23)) {
             ok = false;
@@ -291,12 +295,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------------------------------------------------------- epilogue (warps 2..5)
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     int chunk = 0;  // kEpiAddF32: reduce-adds issued by this warp (selects the staging buffer)
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const Tile ti = decode_tile<SCHED>(args, t);
+      // the tile row of this thread; M = 64 tiles: lanes 0..15 hold rows 16 quarter + lane and
+      // lanes 16..31 stand for rows 64..127 (no data: padding rows, written as zeros where the
+      // epilogue writes padding)
+      const bool m64 = SCHED == kSchedRows && ti.rows_valid <= 64;
+      const int row = m64 ? (lane < 16 ? quarter * 16 + lane : 64 + quarter * 16 + (lane - 16)) : quarter * 32 + lane;
       if (ti.num_k == 0) {
         if (EPI == kEpiAddF32 && args.overwrite) {
           // overwrite mode: an expert with no rows has a zero gradient (no MMA, no TMEM)
