@@ -39,7 +39,8 @@ constexpr uint32_t B_BYTES = BN * BK * 2;
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr uint32_t STG_BYTES = 32 * 128;  // down epilogue: a 32-row x 64-column bf16 box per warp and buffer
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 4 * 2 * STG_BYTES + 256;
 
 struct Tile {
   int a_row;       // first A row of the tile
@@ -90,6 +91,19 @@ __device__ __forceinline__ Tile decode_tile(const TcArgs& a, int t) {
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
+// TMA store of one staged box (128-byte swizzled in shared memory) at (x, y); completion
+// tracked as a bulk group of this thread.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -98,12 +112,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 template <int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-              const __grid_constant__ CUtensorMap tmB1, const TcArgs args) {
+              const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmC, const TcArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint8_t* sStg = sB + STAGES * B_BYTES;  // 1024-aligned: [warp quarter][buffer] of STG_BYTES
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + 4 * 2 * STG_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -237,6 +252,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter+32)
     int acc = 0;
     uint32_t acc_phase = 0;
+    int chunk = 0;  // down: boxes stored by this warp (selects the staging buffer)
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const Tile ti = decode_tile<MODE>(args, t);
       if (!mbar_wait(&tfull[acc], acc_phase, err, 5)) break;
@@ -291,7 +307,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
+      } else if (MODE == kDown && !m64 && quarter * 32 + 32 <= ti.rows_valid) {
+        // 32 valid rows: coalesced TMA stores of 32 x 64 boxes staged in shared memory (thread
+        // = row, its 64 bf16 values as eight 16-byte chunks, chunk j at j ^ (row & 7): the
+        // 128-byte swizzle of the output tensor map)
+        const int grow0 = ti.a_row + quarter * 32;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 64) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tbase + c, r0);
+          tmem_ld32(tbase + c + 32, r1);
+          tc_wait_ld();
+          const int col0 = ti.n_blk * BN + c;
+          if (col0 >= args.n_out) continue;  // the same for the whole warp
+          uint8_t* stg = sStg + (quarter * 2 + (chunk & 1)) * STG_BYTES;
+          if (lane == 0) bulk_wait_read_1();  // the store two boxes back has read this buffer
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t* v = j < 4 ? r0 + 8 * j : r1 + 8 * (j - 4);
+            *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                           pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                           pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                           pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7])));
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmC, stg, col0, grow0);
+            bulk_commit();
+          }
+          ++chunk;
+        }
       } else if (MODE == kDown) {
+        // a partly valid row group (the rows past it belong to the next expert): row stores
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -339,6 +389,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         acc_phase ^= 1u;
       }
     }
+    if (MODE == kDown && lane == 0) bulk_wait_all();  // every store complete before exit
   }
 
   tc_fence_before();
@@ -350,15 +401,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 template <int MODE>
-cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const TcArgs& args,
-                        int grid, cudaStream_t s) {
+cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& c,
+                        const TcArgs& args, int grid, cudaStream_t s) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k_tc_gemm<MODE><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, args);
+  k_tc_gemm<MODE><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, c, args);
   return cudaGetLastError();
 }
 
@@ -368,14 +419,14 @@ int tc_smem_bytes() { return SMEM_BYTES; }
 int tc_block_n(int mode) { return mode == kGateUp ? BN / 2 : BN; }
 
 cudaError_t launch_tc_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                           const TcArgs& args, int grid, cudaStream_t s) {
+                           const CUtensorMap& c, const TcArgs& args, int grid, cudaStream_t s) {
   switch (mode) {
     case kRouter:
-      return launch_mode<kRouter>(a, b0, b1, args, grid, s);
+      return launch_mode<kRouter>(a, b0, b1, c, args, grid, s);
     case kGateUp:
-      return launch_mode<kGateUp>(a, b0, b1, args, grid, s);
+      return launch_mode<kGateUp>(a, b0, b1, c, args, grid, s);
     case kDown:
-      return launch_mode<kDown>(a, b0, b1, args, grid, s);
+      return launch_mode<kDown>(a, b0, b1, c, args, grid, s);
     default:
       return cudaErrorInvalidValue;
   }

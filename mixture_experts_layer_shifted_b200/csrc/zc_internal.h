@@ -58,8 +58,10 @@ struct TcArgs {
 
 int tc_smem_bytes();
 int tc_block_n(int mode);
+// c: kDown only -- the output as a 2-D bf16 tensor [rows, n_out], box 64 x 32, 128-byte swizzle
+// (its full 32-row groups leave by TMA stores); the other modes ignore it.
 cudaError_t launch_tc_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                           const TcArgs& args, int grid, cudaStream_t s);
+                           const CUtensorMap& c, const TcArgs& args, int grid, cudaStream_t s);
 
 // ------------------------------------------------------------- block-scaled FP8 (fp8_quant.cu, gemm_fp8.cu)
 // atom_groups > 0: scales written as scale atoms with that many atoms per 128

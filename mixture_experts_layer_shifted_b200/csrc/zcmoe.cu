@@ -176,7 +176,7 @@ struct zcmoe_s {
   bool profiling;
   std::vector<cudaEvent_t>* events;
   // tensor maps of fixed buffers
-  CUtensorMap tm_wr, tm_wg, tm_wu, tm_wd, tm_xperm, tm_h;
+  CUtensorMap tm_wr, tm_wg, tm_wu, tm_wd, tm_xperm, tm_h, tm_y;
   // ZCMOE_FP8: expert weights as E4M3 codes + scale atoms (owned), padded
   // activation operands (expert e's pairs from row 128 mb_off[e] on) with their
   // scale atoms, padded expert outputs; atoms per 128 rows: gd (K = d), gi (K = inter)
@@ -275,7 +275,7 @@ static int dense_gate_up(zcmoe_dense_s* h, const void* x, int T, cudaStream_t s)
   a.ldo = h->inter;
   a.err = h->err;
   const int tiles = ((T + zc::kBM - 1) / zc::kBM) * a.nblocks;
-  ZC_CUDA(zc::launch_tc_gemm(zc::kGateUp, tm_x, h->tm_wg, h->tm_wu, a, tiles < h->sms ? tiles : h->sms, s));
+  ZC_CUDA(zc::launch_tc_gemm(zc::kGateUp, tm_x, h->tm_wg, h->tm_wu, h->tm_wu, a, tiles < h->sms ? tiles : h->sms, s));
   return ZCMOE_OK;
 }
 
@@ -293,7 +293,10 @@ static int dense_down(zcmoe_dense_s* h, int T, void* y, cudaStream_t s) {
   b.ldo = h->d;
   b.err = h->err;
   const int tiles = ((T + zc::kBM - 1) / zc::kBM) * b.nblocks;
-  ZC_CUDA(zc::launch_tc_gemm(zc::kDown, h->tm_h, h->tm_wd, h->tm_wd, b, tiles < h->sms ? tiles : h->sms, s));
+  CUtensorMap tm_y;
+  const int rc = make_tmap(&tm_y, y, (uint64_t)h->d, (uint64_t)T, 32);
+  if (rc != ZCMOE_OK) return rc;
+  ZC_CUDA(zc::launch_tc_gemm(zc::kDown, h->tm_h, h->tm_wd, h->tm_wd, tm_y, b, tiles < h->sms ? tiles : h->sms, s));
   return ZCMOE_OK;
 }
 
@@ -504,6 +507,7 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
     if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wd, w->w_down, inter, (uint64_t)NL * d, 256);
     if (rc == ZCMOE_OK && !h->fp8) rc = make_tmap(&h->tm_xperm, h->xperm, d, (uint64_t)h->rows_cap, 128);
     if (rc == ZCMOE_OK && !h->fp8) rc = make_tmap(&h->tm_h, h->H, inter, (uint64_t)h->rows_cap, 128);
+    if (rc == ZCMOE_OK && !h->fp8) rc = make_tmap(&h->tm_y, h->Y, d, (uint64_t)h->rows_cap, 32);  // down output
     if (h->fp8) {
       // codes as bytes: the K extent is d or inter bytes (FP8), half that (MXFP4)
       const uint64_t prow = (uint64_t)h->max_mblocks * zc::kBM;
@@ -557,7 +561,7 @@ static int router_stage(zcmoe_t h, const void* x, int Ti, cudaStream_t s) {
     a.col_add = h->offset;
     a.err = h->err;
     const int tiles = ((Ti + zc::kBM - 1) / zc::kBM) * a.nblocks;
-    ZC_CUDA(zc::launch_tc_gemm(zc::kRouter, tm_x, h->tm_wr, h->tm_wr, a, tiles < h->sms ? tiles : h->sms, s));
+    ZC_CUDA(zc::launch_tc_gemm(zc::kRouter, tm_x, h->tm_wr, h->tm_wr, h->tm_wr, a, tiles < h->sms ? tiles : h->sms, s));
   } else {
     zc::SimtArgs a{};
     a.A = static_cast<const float*>(x);
@@ -703,7 +707,8 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     a.err = h->err;
     h->last_saved = h->b_gu != nullptr;
     int bound = max_mb * a.nblocks;
-    ZC_CUDA(zc::launch_tc_gemm(zc::kGateUp, h->tm_xperm, h->tm_wg, h->tm_wu, a, bound < h->sms ? bound : h->sms, s));
+    ZC_CUDA(zc::launch_tc_gemm(zc::kGateUp, h->tm_xperm, h->tm_wg, h->tm_wu, h->tm_wu, a,
+                               bound < h->sms ? bound : h->sms, s));
     ZC_CUDA(mark());
     zc::TcArgs b{};
     b.K = inter;
@@ -717,7 +722,7 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     b.ldo = d;
     b.err = h->err;
     bound = max_mb * b.nblocks;
-    ZC_CUDA(zc::launch_tc_gemm(zc::kDown, h->tm_h, h->tm_wd, h->tm_wd, b, bound < h->sms ? bound : h->sms, s));
+    ZC_CUDA(zc::launch_tc_gemm(zc::kDown, h->tm_h, h->tm_wd, h->tm_wd, h->tm_y, b, bound < h->sms ? bound : h->sms, s));
   } else {
     zc::SimtArgs a{};
     a.A = static_cast<const float*>(h->xperm);
@@ -930,7 +935,7 @@ int zcmoe_ep_experts(zcmoe_t h, const void* xrecv, const int32_t* counts, int64_
   a.ldo = inter;
   a.err = h->err;
   int bound = mb_total * a.nblocks;
-  ZC_CUDA(zc::launch_tc_gemm(zc::kGateUp, tm_a, h->tm_wg, h->tm_wu, a, bound < h->sms ? bound : h->sms, s));
+  ZC_CUDA(zc::launch_tc_gemm(zc::kGateUp, tm_a, h->tm_wg, h->tm_wu, h->tm_wu, a, bound < h->sms ? bound : h->sms, s));
   zc::TcArgs b{};
   b.K = inter;
   b.n_out = d;
@@ -943,7 +948,10 @@ int zcmoe_ep_experts(zcmoe_t h, const void* xrecv, const int32_t* counts, int64_
   b.ldo = d;
   b.err = h->err;
   bound = mb_total * b.nblocks;
-  ZC_CUDA(zc::launch_tc_gemm(zc::kDown, tm_h, h->tm_wd, h->tm_wd, b, bound < h->sms ? bound : h->sms, s));
+  CUtensorMap tm_yr;
+  rc = make_tmap(&tm_yr, y_rows, (uint64_t)d, (uint64_t)P_recv, 32);
+  if (rc != ZCMOE_OK) return rc;
+  ZC_CUDA(zc::launch_tc_gemm(zc::kDown, tm_h, h->tm_wd, h->tm_wd, tm_yr, b, bound < h->sms ? bound : h->sms, s));
   if (R > 1) {
     const int32_t* dseg_src = h->ep_meta;
     ZC_CUDA(zc::launch_ep_regroup(h->Y, yrecv, P_recv, d * 2, dseg_src, dseg_src + nseg + 1, nseg, 1, h->sms, s));
