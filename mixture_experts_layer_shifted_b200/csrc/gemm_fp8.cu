@@ -40,7 +40,8 @@ constexpr int NUM_THREADS = 320;
 constexpr int NUM_EPI = 256;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL = 256;                   // scale buffers: [256, 304)
-constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES + SF_BYTES) + 256 + 2 * 2 * BM * 4;
+constexpr uint32_t STG_BYTES = 32 * 64;           // down epilogue: a 32-row x 32-column bf16 box per warp
+constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES + SF_BYTES) + 8 * STG_BYTES + 256 + 2 * 2 * BM * 4;
 
 struct Tile {
   int64_t a_row;   // first padded A row (a multiple of 128)
@@ -116,6 +117,17 @@ __device__ __forceinline__ uint32_t idesc_mxf4(uint32_t sf) {
   return (sf << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24) |
          (sf << 29);
 }
+// TMA store of one staged box at (x, y); completion tracked as a bulk group of this thread.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NUM_EPI) : "memory"); }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
@@ -143,13 +155,15 @@ __device__ __forceinline__ bool epi_all(bool ok) {
 template <int MODE, int FMT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_fp8_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-               const __grid_constant__ CUtensorMap tmB1, const Fp8Args args) {
+               const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmC,
+               const Fp8Args args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * A_BYTES;
   uint8_t* sSF = sB + STAGES * B_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSF + STAGES * SF_BYTES);
+  uint8_t* sStg = sSF + STAGES * SF_BYTES;  // [epilogue warp] of STG_BYTES (down)
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + 8 * STG_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 1;
@@ -413,25 +427,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_wait_ld();
         tc_fence_before();
         mbar_arrive(tempty);
+        // a row group whose 32 rows are all valid leaves by TMA stores of 32 x 32 boxes staged
+        // in shared memory; a partly valid group (an expert's last rows: few at decode) by row
+        // stores of its valid rows
         const int col0 = ti.n_blk * BN + 128 * half;
-        if (row_ok && col0 < args.n_out) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + grow * args.ldo + col0);
+        if (col0 < args.n_out && quarter * 32 + 32 > ti.rows_valid) {
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + grow * args.ldo + col0);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 v;
-              v.x = pack_bf16(__uint_as_float(r[i][8 * q + 0]), __uint_as_float(r[i][8 * q + 1]));
-              v.y = pack_bf16(__uint_as_float(r[i][8 * q + 2]), __uint_as_float(r[i][8 * q + 3]));
-              v.z = pack_bf16(__uint_as_float(r[i][8 * q + 4]), __uint_as_float(r[i][8 * q + 5]));
-              v.w = pack_bf16(__uint_as_float(r[i][8 * q + 6]), __uint_as_float(r[i][8 * q + 7]));
-              dst[i * 4 + q] = v;
+              for (int q = 0; q < 4; ++q)
+                dst[i * 4 + q] =
+                    make_uint4(pack_bf16(__uint_as_float(r[i][8 * q + 0]), __uint_as_float(r[i][8 * q + 1])),
+                               pack_bf16(__uint_as_float(r[i][8 * q + 2]), __uint_as_float(r[i][8 * q + 3])),
+                               pack_bf16(__uint_as_float(r[i][8 * q + 4]), __uint_as_float(r[i][8 * q + 5])),
+                               pack_bf16(__uint_as_float(r[i][8 * q + 6]), __uint_as_float(r[i][8 * q + 7])));
+          }
+        } else if (col0 < args.n_out) {  // the same for the whole warp
+          uint8_t* stg = sStg + (warp - 2) * STG_BYTES;
+          const int grow0 = (int)ti.a_row + quarter * 32;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (lane == 0) bulk_wait_read_0();  // the previous box has been read out
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<uint4*>(stg + lane * 64 + q * 16) =
+                  make_uint4(pack_bf16(__uint_as_float(r[i][8 * q + 0]), __uint_as_float(r[i][8 * q + 1])),
+                             pack_bf16(__uint_as_float(r[i][8 * q + 2]), __uint_as_float(r[i][8 * q + 3])),
+                             pack_bf16(__uint_as_float(r[i][8 * q + 4]), __uint_as_float(r[i][8 * q + 5])),
+                             pack_bf16(__uint_as_float(r[i][8 * q + 6]), __uint_as_float(r[i][8 * q + 7])));
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmC, stg, col0 + 32 * i, grow0);
+              bulk_commit();
             }
+          }
         }
       }
       acc_phase ^= 1u;
       buf ^= 1;
     }
+    if (MODE == kDown && lane == 0) bulk_wait_all();  // every store complete before exit
   }
 
   tc_fence_before();
@@ -443,8 +482,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 template <int MODE, int FMT>
-cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const Fp8Args& args,
-                        int grid, cudaStream_t s) {
+cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& c,
+                        const Fp8Args& args, int grid, cudaStream_t s) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e =
@@ -452,7 +491,7 @@ cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUten
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k_fp8_gemm<MODE, FMT><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, args);
+  k_fp8_gemm<MODE, FMT><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, c, args);
   return cudaGetLastError();
 }
 
@@ -462,11 +501,11 @@ int fp8_smem_bytes() { return SMEM_BYTES; }
 int fp8_block_n(int mode) { return mode == kGateUp ? BN / 2 : BN; }
 
 cudaError_t launch_fp8_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                            const Fp8Args& args, int grid, cudaStream_t s) {
-  if (mode == kGateUp) return args.fmt ? launch_mode<kGateUp, 1>(a, b0, b1, args, grid, s)
-                                       : launch_mode<kGateUp, 0>(a, b0, b1, args, grid, s);
-  if (mode == kDown) return args.fmt ? launch_mode<kDown, 1>(a, b0, b1, args, grid, s)
-                                     : launch_mode<kDown, 0>(a, b0, b1, args, grid, s);
+                            const CUtensorMap& c, const Fp8Args& args, int grid, cudaStream_t s) {
+  if (mode == kGateUp) return args.fmt ? launch_mode<kGateUp, 1>(a, b0, b1, c, args, grid, s)
+                                       : launch_mode<kGateUp, 0>(a, b0, b1, c, args, grid, s);
+  if (mode == kDown) return args.fmt ? launch_mode<kDown, 1>(a, b0, b1, c, args, grid, s)
+                                     : launch_mode<kDown, 0>(a, b0, b1, c, args, grid, s);
   return cudaErrorInvalidValue;
 }
 

@@ -106,8 +106,10 @@ struct Fp8Args {
 };
 int fp8_smem_bytes();
 int fp8_block_n(int mode);
+// c: kDown only -- the padded output rows [rows, n_out] bf16, box 32 x 32, no swizzle (whole
+// 32-row groups leave by TMA stores); kGateUp ignores it.
 cudaError_t launch_fp8_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                            const Fp8Args& args, int grid, cudaStream_t s);
+                            const CUtensorMap& c, const Fp8Args& args, int grid, cudaStream_t s);
 
 // ------------------------------------------------------------- backward data movement (moe_bwd.cu, route.cu)
 cudaError_t launch_router_bwd(const float* logits, int T, int E, int k, float scale, const int32_t* idx,

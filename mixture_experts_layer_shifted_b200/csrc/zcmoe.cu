@@ -98,6 +98,21 @@ int make_tmap_esz(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t ou
   if (r != CUDA_SUCCESS) return fail(ZCMOE_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return ZCMOE_OK;
 }
+// bf16 [outer, inner], box 32 x 32, no swizzle: a store target for 32-row x 32-column boxes
+int make_tmap_store32(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(ZCMOE_ECUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0) return fail(ZCMOE_EINVAL, "tensor base not 16-byte aligned");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ZCMOE_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return ZCMOE_OK;
+}
 int make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
   return make_tmap_esz(tm, base, inner, outer, box_outer, 2);
 }
@@ -183,7 +198,7 @@ struct zcmoe_s {
   int fp8, fmt, gd, gi;  // fp8: block-scaled experts (ZCMOE_FP8 or ZCMOE_FP4); fmt 1 for MXFP4
   uint8_t *w8g, *w8u, *w8d, *sfg, *sfu, *sfd, *x8, *sx, *h8, *sh;
   void* ypad;
-  CUtensorMap tm8_wg, tm8_wu, tm8_wd, tm8_x, tm8_h;
+  CUtensorMap tm8_wg, tm8_wu, tm8_wd, tm8_x, tm8_h, tm8_y;  // tm8_y: the down GEMM's store target (ypad)
   // zcmoe_backward (allocated on its first call): padded X, dY, dH, [dG|dU], H, dX
   // rows; dg [T*k]; dl [T, dl_ld] bf16; router dx [T, d]; the router's one-group offsets
   int last_T;
@@ -517,6 +532,7 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
       if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_wd, h->w8d, ib, (uint64_t)N * d, 256, 1);
       if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_x, h->x8, db, prow, 128, 1);
       if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_h, h->h8, ib, prow, 128, 1);
+      if (rc == ZCMOE_OK) rc = make_tmap_store32(&h->tm8_y, h->ypad, d, prow);
     }
     if (rc != ZCMOE_OK) {
       release(h);
@@ -672,7 +688,8 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     a.out_groups = h->gi;
     a.err = h->err;
     int bound = max_mb * a.nblocks;
-    ZC_CUDA(zc::launch_fp8_gemm(zc::kGateUp, h->tm8_x, h->tm8_wg, h->tm8_wu, a, bound < h->sms ? bound : h->sms, s));
+    ZC_CUDA(zc::launch_fp8_gemm(zc::kGateUp, h->tm8_x, h->tm8_wg, h->tm8_wu, h->tm8_wu, a,
+                                bound < h->sms ? bound : h->sms, s));
     ZC_CUDA(mark());
     zc::Fp8Args b{};
     b.fmt = h->fmt;
@@ -691,7 +708,8 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     b.ldo = d;
     b.err = h->err;
     bound = max_mb * b.nblocks;
-    ZC_CUDA(zc::launch_fp8_gemm(zc::kDown, h->tm8_h, h->tm8_wd, h->tm8_wd, b, bound < h->sms ? bound : h->sms, s));
+    ZC_CUDA(zc::launch_fp8_gemm(zc::kDown, h->tm8_h, h->tm8_wd, h->tm8_wd, h->tm8_y, b, bound < h->sms ? bound : h->sms,
+                                s));
   } else if (h->bf16) {
     zc::TcArgs a{};
     a.K = d;
