@@ -50,7 +50,8 @@ constexpr int kWgStages = 4, kWgBufs = 2;
 template <int EPI>
 struct Cfg {
   static constexpr int kStages = EPI == kEpiAddF32 ? kWgStages : kRowStages;
-  static constexpr int kBufs = EPI == kEpiAddF32 ? kWgBufs : 0;
+  // staging buffers per epilogue warp: GemmAdd boxes, or the bf16 outputs' TMA-store boxes
+  static constexpr int kBufs = EPI == kEpiAddF32 ? kWgBufs : (EPI == kEpiBf16 ? 2 : 0);
   static constexpr int kSmem = 1024 + kStages * STAGE_BYTES + 4 * kBufs * STG_BYTES + 256;
   static_assert(kSmem <= 232448, "shared memory per block");
 };
@@ -116,6 +117,13 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* tm, const v
   asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
                    reinterpret_cast<uint64_t>(tm)),
                "r"(smem_u32(src)), "r"(n), "r"(m), "r"(g)
+               : "memory");
+}
+// TMA store of a 32-row x 64-column bf16 box (128-byte swizzled in shared memory) at (x, y).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
                : "memory");
 }
 // TMA store of a 32 x 32 fp32 box (the same staging and tensor map): the overwrite mode.
@@ -333,7 +341,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait(&tfull[acc], acc_phase, err, 25)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-      if (EPI == kEpiBf16) {
+      if (EPI == kEpiBf16 && !m64 && quarter * 32 + 32 <= ti.rows_valid) {
+        // 32 valid rows: coalesced TMA stores of 32 x 64 boxes staged in shared memory (thread =
+        // row, chunk j of its 64 values at j ^ (row & 7): the output map's 128-byte swizzle)
+        constexpr int NB = NBUF > 0 ? NBUF : 1;
+        const int grow0 = (int)ti.a_row + quarter * 32;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 64) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tbase + c, r0);
+          tmem_ld32(tbase + c + 32, r1);
+          tc_wait_ld();
+          const int col0 = ti.n_blk * BN + c;
+          if (col0 >= args.n_out) continue;  // the same for the whole warp
+          uint8_t* stg = sStg + (quarter * NB + chunk % NB) * STG_BYTES;
+          if (lane == 0) bulk_wait_read<NB - 1>();
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t* v = j < 4 ? r0 + 8 * j : r1 + 8 * (j - 4);
+            *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                           pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                           pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                           pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7])));
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmC, stg, col0, grow0);
+            bulk_commit();
+          }
+          ++chunk;
+        }
+      } else if (EPI == kEpiBf16) {
         const bool row_ok = row < ti.rows_valid;
         const int64_t grow = ti.a_row + row;
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
@@ -494,7 +535,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         acc_phase ^= 1u;
       }
     }
-    if (EPI == kEpiAddF32 && lane == 0) bulk_wait_all();  // every reduce-add complete before exit
+    if ((EPI == kEpiAddF32 || EPI == kEpiBf16) && lane == 0) bulk_wait_all();  // every store complete before exit
   }
 
   tc_fence_before();

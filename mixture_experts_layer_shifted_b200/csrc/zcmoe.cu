@@ -1333,8 +1333,10 @@ int zcmoe_backward_ex(zcmoe_t h, const void* x, const void* dy, int64_t T, void*
     a.b_row_per_group = d;
     a.out = h->b_dh;
     a.ldo = inter;
-    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dy_k, tm_wd_mn, tm_wd_mn, tm_dy_k, a, grid_for((int64_t)max_mb * a.nblocks),
-                                s));
+    CUtensorMap tm_dh_st;
+    if ((rc = make_tmap(&tm_dh_st, h->b_dh, (uint64_t)inter, P, 32)) != ZCMOE_OK) return rc;
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dy_k, tm_wd_mn, tm_wd_mn, tm_dh_st, a,
+                                grid_for((int64_t)max_mb * a.nblocks), s));
   }
   // [G|U] recomputed from X; SwiGLU backward -> dG, dU; H
   if (!h->last_saved) {
@@ -1360,7 +1362,9 @@ int zcmoe_backward_ex(zcmoe_t h, const void* x, const void* dy, int64_t T, void*
     a.b_row_per_group = inter;
     a.out = h->b_dxp;
     a.ldo = d;
-    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dgu_k, tm_wg_mn, tm_wu_mn, tm_dgu_k, a,
+    CUtensorMap tm_dxp_st;
+    if ((rc = make_tmap(&tm_dxp_st, h->b_dxp, (uint64_t)d, P, 32)) != ZCMOE_OK) return rc;
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dgu_k, tm_wg_mn, tm_wu_mn, tm_dxp_st, a,
                                 grid_for((int64_t)max_mb * a.nblocks), s));
   }
   // router: dx_router = dl W_r
@@ -1377,7 +1381,9 @@ int zcmoe_backward_ex(zcmoe_t h, const void* x, const void* dy, int64_t T, void*
     a.b_row_per_group = 0;
     a.out = h->b_dxr;
     a.ldo = d;
-    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dl_k, tm_wr_mn, tm_wr_mn, tm_dl_k, a,
+    CUtensorMap tm_dxr_st;
+    if ((rc = make_tmap(&tm_dxr_st, h->b_dxr, (uint64_t)d, (uint64_t)T, 32)) != ZCMOE_OK) return rc;
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdRowsMnB, tm_dl_k, tm_wr_mn, tm_wr_mn, tm_dxr_st, a,
                                 grid_for((int64_t)((Ti + 127) / 128) * a.nblocks), s));
   }
   // dx: the deterministic ScatterAdd
