@@ -51,7 +51,8 @@ template <int EPI>
 struct Cfg {
   static constexpr int kStages = EPI == kEpiAddF32 ? kWgStages : kRowStages;
   // staging buffers per epilogue warp: GemmAdd boxes, or the bf16 outputs' TMA-store boxes
-  static constexpr int kBufs = EPI == kEpiAddF32 ? kWgBufs : (EPI == kEpiBf16 ? 2 : 0);
+  //   (the saved-SwiGLU epilogue uses its warp's two buffers as dG, dU, H boxes of 2 KB each)
+  static constexpr int kBufs = EPI == kEpiAddF32 ? kWgBufs : (EPI == kEpiBf16 || EPI == kEpiSwigluSaved ? 2 : 0);
   static constexpr int kSmem = 1024 + kStages * STAGE_BYTES + 4 * kBufs * STG_BYTES + 256;
   static_assert(kSmem <= 232448, "shared memory per block");
 };
@@ -449,10 +450,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       } else if (EPI == kEpiSwigluSaved) {
-        // the accumulator is dH (fp32, 256 columns); g and u are the forward's saved values
+        // the accumulator is dH (fp32, 256 columns); g and u are the forward's saved values.
+        // The padded rows of an expert's block are its own, so the warp's 32 rows (zeros past
+        // the valid ones) leave as 32 x 32 boxes of dG, dU and H by TMA stores (no swizzle;
+        // tmC: [dG | dU], tmB1: H), except in M = 64 tiles, whose lanes hold rows of two groups.
         const bool row_ok = row < ti.rows_valid;
         const int64_t grow = ti.a_row + row;
         const int inter = args.inter;
+        const bool tma_out = !m64;
+        constexpr int NB = NBUF > 0 ? NBUF : 1;
+        uint8_t* stg = sStg + quarter * NB * STG_BYTES;  // dG +0, dU +2 KB, H +4 KB
+        const int grow0 = (int)ti.a_row + quarter * 32;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t r[32];
@@ -460,6 +468,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_wait_ld();
           const int col0 = ti.n_blk * BN + c;
           if (col0 >= inter) continue;
+          if (tma_out) {
+            if (lane == 0) bulk_wait_read<0>();  // the previous boxes have been read out
+            __syncwarp();
+          }
           const uint4* gi = reinterpret_cast<const uint4*>(args.gu + grow * 2 * inter + col0);
           const uint4* ui = reinterpret_cast<const uint4*>(args.gu + grow * 2 * inter + inter + col0);
           uint4* dgo = reinterpret_cast<uint4*>(args.dgu + grow * 2 * inter + col0);
@@ -493,9 +505,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 ph[w] = pack_bf16(hv[0], hv[1]);
               }
             }
-            dgo[q] = vdg;
-            duo[q] = vdu;
-            ho[q] = vh;
+            if (tma_out) {
+              *reinterpret_cast<uint4*>(stg + lane * 64 + q * 16) = vdg;
+              *reinterpret_cast<uint4*>(stg + 2048 + lane * 64 + q * 16) = vdu;
+              *reinterpret_cast<uint4*>(stg + 4096 + lane * 64 + q * 16) = vh;
+            } else {
+              dgo[q] = vdg;
+              duo[q] = vdu;
+              ho[q] = vh;
+            }
+          }
+          if (tma_out) {
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmC, stg, col0, grow0);
+              tma_store_2d(&tmC, stg + 2048, inter + col0, grow0);
+              tma_store_2d(&tmB1, stg + 4096, col0, grow0);
+              bulk_commit();
+            }
           }
         }
       } else {
@@ -535,7 +563,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         acc_phase ^= 1u;
       }
     }
-    if ((EPI == kEpiAddF32 || EPI == kEpiBf16) && lane == 0) bulk_wait_all();  // every store complete before exit
+    if ((EPI == kEpiAddF32 || EPI == kEpiBf16 || EPI == kEpiSwigluSaved) && lane == 0)
+      bulk_wait_all();  // every store complete before exit
   }
 
   tc_fence_before();

@@ -158,7 +158,9 @@ struct BwdArgs {
 int bwd_smem_bytes();
 // c: kBwdWgrad -- the fp32 accumulator as a 3-D tensor [groups][m_out][n_out], box 32 x 32 x 1,
 // 128-byte swizzle (the reduce-add target); kBwdRowsMnB -- the bf16 output [rows, n_out], box
-// 64 x 32, 128-byte swizzle (full 32-row groups leave by TMA stores); other kinds ignore it.
+// 64 x 32, 128-byte swizzle (full 32-row groups leave by TMA stores); kBwdDhSwiglu -- [dG | dU]
+// [rows, 2 inter] bf16, box 32 x 32, no swizzle, with H [rows, inter] the same way as b1; other
+// kinds ignore it.
 cudaError_t launch_bwd_gemm(int kind, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                             const CUtensorMap& c, const BwdArgs& args, int grid, cudaStream_t s);
 

@@ -1321,7 +1321,10 @@ int zcmoe_backward_ex(zcmoe_t h, const void* x, const void* dy, int64_t T, void*
     a.dgu = static_cast<__nv_bfloat16*>(h->b_dgu);
     a.hpad = static_cast<__nv_bfloat16*>(h->b_hpad);
     a.inter = inter;
-    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdDhSwiglu, tm_dy_k, tm_wd_mn, tm_wd_mn, tm_dy_k, a,
+    CUtensorMap tm_dgu_st, tm_h_st;  // store targets: [dG | dU] (as c) and H (as the unused second B)
+    if ((rc = make_tmap_store32(&tm_dgu_st, h->b_dgu, 2 * (uint64_t)inter, P)) != ZCMOE_OK) return rc;
+    if ((rc = make_tmap_store32(&tm_h_st, h->b_hpad, (uint64_t)inter, P)) != ZCMOE_OK) return rc;
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdDhSwiglu, tm_dy_k, tm_wd_mn, tm_h_st, tm_dgu_st, a,
                                 grid_for((int64_t)max_mb * a.nblocks), s));
   }
   // dH = dY W_d
