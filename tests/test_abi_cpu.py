@@ -112,3 +112,29 @@ def test_dense_and_overlap_arguments_are_rejected_on_the_host(zc):
     assert lib.zcmoe_dense_destroy(fake) == zc.ZCMOE_EINVAL
     assert lib.zcmoe_dense_destroy(None) == zc.ZCMOE_OK
     assert lib.zcmoe_forward_overlap(fake, fake, None, None, 1, None, None, None) == zc.ZCMOE_EINVAL
+
+
+def test_training_ep_and_host_entry_points_refuse_unknown_handles(zc):
+    """The backward, training-mode, expert-parallel and pipelined host entry points check the
+    handle (and their own arguments) on the host before any device work."""
+    lib = zc.lib()
+    fake = ctypes.c_void_p(0x1000)
+    E = zc.ZCMOE_EINVAL
+    assert lib.zcmoe_backward(fake, None, None, 1, None, None, None, None, None, None) == E
+    assert lib.zcmoe_backward_ex(fake, None, None, 1, None, None, None, None, None, 0, None) == E
+    assert lib.zcmoe_save_for_backward(fake, 1) == E
+    assert lib.zcmoe_ep_dispatch(fake, None, 1, None, None, None) == E
+    assert lib.zcmoe_ep_experts(fake, None, None, 0, None, None) == E
+    assert lib.zcmoe_ep_combine(fake, None, None, 1, None, None) == E
+    assert lib.zcmoe_forward_host_async(fake, None, 1, None, None) == E
+    assert lib.zcmoe_forward_host_flush(fake, None) == E
+    # create_ep: the group arguments are checked before the device is touched
+    h = ctypes.c_void_p()
+    cfg = zc.zcmoe_config(256, 16, 8, 128, 4, 64, zc.ZCMOE_BF16, 1.0, None, None)
+    w = zc.zcmoe_weights(16, 16, 16, 16)
+    for rank, size, cap in [(0, 3, 0), (2, 2, 0), (-1, 2, 0), (0, 0, 0), (0, 2, -1)]:
+        assert lib.zcmoe_create_ep(ctypes.byref(cfg), ctypes.byref(w), rank, size, cap, ctypes.byref(h)) == E
+        assert h.value is None
+    cfg32 = zc.zcmoe_config(256, 16, 8, 128, 4, 64, zc.ZCMOE_F32, 1.0, None, None)
+    assert lib.zcmoe_create_ep(ctypes.byref(cfg32), ctypes.byref(w), 0, 2, 0,
+                               ctypes.byref(h)) == zc.ZCMOE_EUNSUPPORTED
