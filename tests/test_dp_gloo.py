@@ -77,7 +77,7 @@ def _free_port():
 
 def test_two_rank_controller_matches_single_process():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     b0, b1 = out[0], out[1]

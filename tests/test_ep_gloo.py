@@ -109,7 +109,7 @@ def _free_port():
     (4, (20, 0, 33, 9), 2),   # a rank with no tokens
 ])
 def test_ep_forward_matches_the_whole_layer(world, sizes, chunks):
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), sizes, chunks, out), nprocs=world, join=True)
     wr, wg, wu, wd, bias = _weights()
