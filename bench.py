@@ -77,22 +77,41 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.thread.join(timeout=2)
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            f = [v.strip() for v in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                smax = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return parse_clock_lines(self.lines)
+
+
+THROTTLE_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def parse_clock_lines(lines):
+    """Summary of nvidia-smi samples in ClockSampler.FIELDS order (csv, no header,
+    no units): median SM clock, the max SM clock, every throttle reason seen
+    active, and `rejected` when the record disqualifies the timed region — a
+    hardware or thermal slowdown, or an SM clock far below its max with no
+    reason active (a clock lock left by someone else).  sw_power_cap is normal
+    for a 1 kW part under dense GEMMs and is only listed."""
+    sm, smax, reasons = [], None, set()
+    names = THROTTLE_REASONS + ("sw_power_cap",)
+    for line in lines:
+        f = [v.strip() for v in line.split(",")]
+        if len(f) < 9:
+            continue
+        try:
+            sm.append(float(f[1]))
+            smax = float(f[2])
+        except ValueError:
+            continue
+        for n, v in zip(names, f[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+           "samples": len(sm)}
+    bad = [r for r in THROTTLE_REASONS if r in reasons]
+    if bad:
+        out["rejected"] = "throttled: " + ", ".join(bad)
+    elif sm and smax and not reasons and out["sm_mhz"] < 0.6 * smax:
+        out["rejected"] = f"SM clock {out['sm_mhz']:.0f} of {smax:.0f} MHz with no reason active"
+    return out
 
 
 def _dist():
