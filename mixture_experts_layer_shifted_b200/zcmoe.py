@@ -146,6 +146,27 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _expect(t, name, shape, dtype, cuda=True):
+    """The library sees only a pointer, so the binding checks what the pointer must
+    hold: a contiguous tensor of exactly `shape` (None matches any extent) and
+    `dtype`, on the GPU (cuda=True) or in host memory.  Raises ValueError."""
+    ok = (t.dim() == len(shape) and all(w is None or int(n) == w for n, w in zip(t.shape, shape))
+          and t.dtype == dtype and t.is_contiguous() and bool(t.is_cuda) == cuda)
+    if not ok:
+        want = "[" + ", ".join("*" if w is None else str(w) for w in shape) + "]"
+        where = "device" if cuda else "host"
+        raise ValueError(f"{name}: expected a contiguous {where} tensor {want} {dtype}, got {list(t.shape)} "
+                         f"{t.dtype} on {t.device}{'' if t.is_contiguous() else ' (not contiguous)'}")
+
+
+def _expect_at_least(t, name, numel, dtype):
+    """A device output buffer the library fills from its start: contiguous, of `dtype`,
+    holding at least `numel` elements."""
+    if t.dtype != dtype or not t.is_contiguous() or not t.is_cuda or t.numel() < numel:
+        raise ValueError(f"{name}: expected a contiguous device {dtype} buffer of at least {numel} elements, got "
+                         f"{list(t.shape)} {t.dtype} on {t.device}")
+
+
 # ----------------------------------------------------------------- C names
 def zcmoe_create(cfg: zcmoe_config, w: zcmoe_weights) -> ctypes.c_void_p:
     h = ctypes.c_void_p()
@@ -371,18 +392,33 @@ class ZcMoE:
 
     def forward(self, x, y=None, stream=None, debug: dict | None = None):
         """y = layer(x); ``debug`` maps zcmoe_debug field names to device tensors to fill."""
+        s = self.shape
+        _expect(x, "x", (None, s.d), s.torch_dtype)
         T = x.shape[0]
         if y is None:
             y = torch.empty_like(x)
+        _expect(y, "y", (T, s.d), s.torch_dtype)
         dbg = None
         if debug:
-            dbg = zcmoe_debug(**{k: v.data_ptr() for k, v in debug.items()})
+            k, E = s.top_k, s.E
+            need = {"logits": (T * E, torch.float32), "scores": (T * E, torch.float32), "idx": (T * k, torch.int32),
+                    "gate": (T * k, torch.float32), "counts": (E, torch.int32), "offsets": (s.n_ffn + 1, torch.int32),
+                    "perm": (T * k, torch.int32), "pos": (T * k, torch.int32),
+                    "expert_out": (T * k * s.d, s.torch_dtype)}
+            for name, t in debug.items():
+                if name not in need:
+                    raise ValueError(f"debug: unknown field {name!r}; fields: {sorted(need)}")
+                _expect_at_least(t, f"debug[{name!r}]", *need[name])
+            dbg = zcmoe_debug(**{k_: v.data_ptr() for k_, v in debug.items()})
         zcmoe_forward(self.h, ctypes.c_void_p(x.data_ptr()), T, ctypes.c_void_p(y.data_ptr()), stream, dbg)
         return y
 
     def forward_host(self, x_host, y_host, stream=None, pipelined=False):
         """y_host = layer(x_host), both page-locked host tensors.  pipelined: y_host is complete
         once the stream has passed the next forward_host call or flush_host()."""
+        s = self.shape
+        _expect(x_host, "x_host", (None, s.d), s.torch_dtype, cuda=False)
+        _expect(y_host, "y_host", (x_host.shape[0], s.d), s.torch_dtype, cuda=False)
         fn = zcmoe_forward_host_async if pipelined else zcmoe_forward_host
         fn(self.h, ctypes.c_void_p(x_host.data_ptr()), x_host.shape[0], ctypes.c_void_p(y_host.data_ptr()), stream)
         return y_host
@@ -394,8 +430,20 @@ class ZcMoE:
         """dx of the last forward (x must be the tensor it read); adds the weight gradients
         into the fp32 tensors of ``grads`` (keys router, gate, up, down; missing: skipped), or
         writes them there with accumulate=False."""
+        s = self.shape
+        _expect(x, "x", (None, s.d), s.torch_dtype)
+        T = x.shape[0]
+        _expect(dy, "dy", (T, s.d), s.torch_dtype)
         dx = torch.empty_like(x) if dx is None else dx
+        _expect(dx, "dx", (T, s.d), s.torch_dtype)
         g = grads or {}
+        NL = s.n_ffn // max(self.ep_size, 1)
+        gshape = {"router": (s.E, s.d), "gate": (NL, s.inter, s.d), "up": (NL, s.inter, s.d),
+                  "down": (NL, s.d, s.inter)}
+        for name, t in g.items():
+            if name not in gshape:
+                raise ValueError(f"grads: unknown key {name!r}; keys: {sorted(gshape)}")
+            _expect(t, f"grads[{name!r}]", gshape[name], torch.float32)
         ptr = lambda name: ctypes.c_void_p(g[name].data_ptr()) if name in g else None  # noqa: E731
         zcmoe_backward(self.h, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(dy.data_ptr()), x.shape[0],
                        ctypes.c_void_p(dx.data_ptr()), ptr("router"), ptr("gate"), ptr("up"), ptr("down"), stream,
@@ -411,9 +459,11 @@ class ZcMoE:
         zcmoe_update_bias(self.h, zcmoe_gains(kp, ki, kd, decay, K), stream)
 
     def read_counts(self, dst, stream=None):
+        _expect(dst, "dst", (self.shape.E + 1,), torch.int64)
         zcmoe_read_counts(self.h, ctypes.c_void_p(dst.data_ptr()), stream)
 
     def write_counts(self, src, stream=None):
+        _expect(src, "src", (self.shape.E + 1,), torch.int64)
         zcmoe_write_counts(self.h, ctypes.c_void_p(src.data_ptr()), stream)
 
     def state(self):
@@ -429,6 +479,8 @@ class ZcMoE:
     def set_bias(self, bias):
         import numpy as np
         b = np.ascontiguousarray(bias, dtype=np.float32)
+        if b.shape != (self.shape.E,):
+            raise ValueError(f"bias: expected {self.shape.E} values, got shape {b.shape}")
         zcmoe_set_bias(self.h, b.ctypes.data)
 
     def check(self):
@@ -468,8 +520,10 @@ class ZcDense:
         self.h = zcmoe_dense_create(cfg, w)
 
     def forward(self, x, y=None, stream=None):
+        _expect(x, "x", (None, self.d), torch.bfloat16)
         if y is None:
             y = torch.empty_like(x)
+        _expect(y, "y", (x.shape[0], self.d), torch.bfloat16)
         zcmoe_dense_forward(self.h, ctypes.c_void_p(x.data_ptr()), x.shape[0], ctypes.c_void_p(y.data_ptr()), stream)
         return y
 
@@ -496,6 +550,11 @@ def forward_overlap(moe: ZcMoE, dense: ZcDense, x_moe, x_dense=None, y_moe=None,
         raise ValueError("x_moe and x_dense must hold the same number of tokens")
     y_moe = torch.empty_like(x_moe) if y_moe is None else y_moe
     y_dense = torch.empty_like(x_dense) if y_dense is None else y_dense
+    # the tensors are checked against the MoE layer's row width and dtype; a dense handle
+    # that does not match the layer is refused by the library
+    s = moe.shape
+    for name, t in (("x_moe", x_moe), ("x_dense", x_dense), ("y_moe", y_moe), ("y_dense", y_dense)):
+        _expect(t, name, (x_moe.shape[0], s.d), s.torch_dtype)
     zcmoe_forward_overlap(moe.h, dense.h, ctypes.c_void_p(x_moe.data_ptr()), ctypes.c_void_p(x_dense.data_ptr()),
                           x_moe.shape[0], ctypes.c_void_p(y_moe.data_ptr()), ctypes.c_void_p(y_dense.data_ptr()),
                           stream)

@@ -138,3 +138,62 @@ def test_training_ep_and_host_entry_points_refuse_unknown_handles(zc):
     cfg32 = zc.zcmoe_config(256, 16, 8, 128, 4, 64, zc.ZCMOE_F32, 1.0, None, None)
     assert lib.zcmoe_create_ep(ctypes.byref(cfg32), ctypes.byref(w), 0, 2, 0,
                                ctypes.byref(h)) == zc.ZCMOE_EUNSUPPORTED
+
+
+def test_binding_tensor_checks(zc):
+    """The binding passes bare pointers, so it checks each tensor's dims, dtype,
+    contiguity and memory kind before the call; a mismatch is a ValueError."""
+    import torch
+    ok = torch.zeros((5, 64), dtype=torch.bfloat16)
+    zc._expect(ok, "x", (None, 64), torch.bfloat16, cuda=False)
+    zc._expect(ok, "x", (5, 64), torch.bfloat16, cuda=False)
+    bad = [
+        (ok, (None, 32), torch.bfloat16, False),            # width
+        (ok, (4, 64), torch.bfloat16, False),               # rows
+        (ok, (None, 64), torch.float32, False),             # dtype
+        (ok, (None, 64), torch.bfloat16, True),             # host memory where device memory is needed
+        (ok.reshape(-1), (None, 64), torch.bfloat16, False),  # dims
+        (torch.zeros((64, 5), dtype=torch.bfloat16).t(), (None, 64), torch.bfloat16, False),  # not contiguous
+    ]
+    for t, shape, dtype, cuda in bad:
+        with pytest.raises(ValueError):
+            zc._expect(t, "x", shape, dtype, cuda=cuda)
+    with pytest.raises(ValueError):
+        zc._expect_at_least(torch.zeros(8, dtype=torch.int32), "perm", 8, torch.int32)   # host buffer
+
+
+def test_layer_methods_check_tensors_before_the_library(zc):
+    """A layer object whose handle is not live: a call that passed the binding's checks
+    would reach the library and fail there with EINVAL, so each ValueError below shows
+    the check ran first, and the ZcmoeError shows well-formed tensors get through."""
+    import numpy as np
+    import torch
+    lay = object.__new__(zc.ZcMoE)
+    lay.shape = zc.LayerShape(64, 4, 2, 32, 2, "bf16")
+    lay.ep_size = 1
+    lay.h = ctypes.c_void_p(0x1000)
+    try:
+        x = torch.zeros((5, 64), dtype=torch.bfloat16)
+        y = torch.zeros((5, 64), dtype=torch.bfloat16)
+        with pytest.raises(ValueError):
+            lay.forward(x, y, stream=0)                     # host tensors for a device call
+        with pytest.raises(ValueError):
+            lay.backward(x, y, y.clone(), stream=0)
+        with pytest.raises(ValueError):
+            lay.read_counts(torch.zeros(7, dtype=torch.int64), stream=0)
+        with pytest.raises(ValueError):
+            lay.set_bias(np.zeros(5, np.float32))           # E = 6 values needed
+        with pytest.raises(ValueError):
+            lay.forward_host(x, torch.zeros((4, 64), dtype=torch.bfloat16), stream=0)   # y rows
+        with pytest.raises(ValueError):
+            lay.forward_host(torch.zeros((5, 32), dtype=torch.bfloat16), y, stream=0)   # width
+        with pytest.raises(ValueError):
+            lay.forward_host(x.float(), y.float(), stream=0)                            # dtype
+        with pytest.raises(zc.ZcmoeError) as ei:
+            lay.forward_host(x, y, stream=0)
+        assert ei.value.code == zc.ZCMOE_EINVAL
+        with pytest.raises(zc.ZcmoeError) as ei:
+            lay.set_bias(np.zeros(6, np.float32))
+        assert ei.value.code == zc.ZCMOE_EINVAL
+    finally:
+        lay.h = None
