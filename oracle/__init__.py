@@ -26,6 +26,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "zcmoe_oracle.c")
 _SO = os.path.join(_HERE, "liboracle.so")
+_PREBUILT = False
 _lib = None
 
 F32P = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
@@ -34,12 +35,26 @@ I32P = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
 I64P = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
 
 
+def compile_command(src: str, out: str) -> list:
+    """gcc -O2 -ffp-contract=off, no fast-math, OpenMP: the one way the oracle is built."""
+    return ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
+            "-fvisibility=hidden", "-o", out, src, "-lm"]
+
+
+def use_library(path: str) -> None:
+    """Load the oracle from `path`, a library built elsewhere with compile_command.
+    The pins' mutation test uses it to run the pins against deliberately broken
+    copies of the source; nothing else calls it."""
+    global _SO, _PREBUILT, _lib
+    _SO, _PREBUILT, _lib = path, True, None
+
+
 def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (-O2 -ffp-contract=off, OpenMP)."""
+    """Compile the oracle (nothing to do after use_library)."""
+    if _PREBUILT:
+        return _SO
     if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
-               "-fvisibility=hidden", "-o", _SO, _SRC, "-lm"]
-        subprocess.run(cmd, check=True)
+        subprocess.run(compile_command(_SRC, _SO), check=True)
     return _SO
 
 

@@ -174,6 +174,38 @@ def test_replica_matches_fp64_routing_away_from_ties():
     np.testing.assert_allclose(s32.astype(np.float64).sum(1), 1.0, atol=5e-6)
 
 
+
+def test_replica_ties_go_to_the_lower_index():
+    """Equal logits give bit-equal fp32 scores, so the replica's tie rule decides:
+    the lower expert index first, as in the fp64 rule."""
+    l = np.array([[1.0, 2.0, 2.0, 0.0, 2.0, 1.0]], np.float32)
+    idx, gate, s = oracle.route_replica_f32(l, None, 4, 1.0, want_scores=True)
+    assert s[0, 1] == s[0, 2] == s[0, 4] and s[0, 0] == s[0, 5]
+    assert idx[0].tolist() == [1, 2, 4, 0]
+    b = np.array([0.0, 0.0, 0.0, 0.0, 0.0, 0.0], np.float32)
+    assert oracle.route_replica_f32(l, b, 4, 1.0)[0][0].tolist() == [1, 2, 4, 0]
+    ref = oracle.brute_force_topk(s[0].astype(np.float64), 4)
+    assert sorted(ref) == sorted(idx[0].tolist())
+
+
+def test_replica_is_shift_invariant_bit_for_bit():
+    """The rule subtracts the largest logit before the exponential.  On logits on a
+    2^-10 grid, adding 128 (or 1024) is exact in fp32 and so is the subtraction, so
+    the scores, indices and gates must come out bit-identical, and finite."""
+    rng = _rng(31)
+    l = (np.round(rng.uniform(-8, 8, size=(64, 96)) * 1024) / 1024).astype(np.float32)
+    b = rng.uniform(-0.01, 0.01, size=96).astype(np.float32)
+    i0, g0, s0 = oracle.route_replica_f32(l, b, 8, 1.0, want_scores=True)
+    for c in (128.0, 1024.0):
+        lc = (l + np.float32(c)).astype(np.float32)
+        assert np.array_equal(lc - np.float32(c), l)   # the shift is exact
+        i1, g1, s1 = oracle.route_replica_f32(lc, b, 8, 1.0, want_scores=True)
+        assert np.isfinite(s1).all()
+        np.testing.assert_array_equal(s1.view(np.uint32), s0.view(np.uint32))
+        np.testing.assert_array_equal(i1, i0)
+        np.testing.assert_array_equal(g1.view(np.uint32), g0.view(np.uint32))
+
+
 # ---------------------------------------------------------------- integer stage
 def test_integer_stage_against_stable_sort():
     T, N, Z, k = 300, 16, 8, 4
@@ -315,6 +347,32 @@ def test_update_bias_hand_worked_step():
     assert abs(float(st["eprev"].astype(np.float64).sum())) < 1e-6
     # an underloaded expert gains bias, an overloaded one loses it
     assert st["bias"][1] > b0[1] and st["bias"][2] < b0[2]
+
+
+
+def test_update_bias_second_step_uses_the_previous_error():
+    """Two hand-worked steps, so the derivative term sees a non-zero previous error
+    and the integral term carries the first step's value."""
+    N, Z, k = 2, 1, 2
+    b0 = np.array([0.0, 0.1, -0.1], np.float32)
+    st = oracle.new_controller_state(b0)
+    kp, ki, kd, decay, K = 0.5, 0.25, 2.0, 0.5, 1.5
+    tau = [K / N, K / N, (k - K) / Z]
+    steps = [[3, 1, 4], [1, 4, 3]]       # 4 tokens x k = 2 picks each step
+    eta, integ, eprev = 1.0, [0.0] * 3, [0.0] * 3
+    for c in steps:
+        counts = np.array(c, np.int64)
+        tokens = np.array([4], np.int64)
+        oracle.update_bias(counts, tokens, N, Z, k, (kp, ki, kd, decay, K), b0, st)
+        eta *= decay
+        for i in range(3):
+            e = tau[i] - c[i] / 4
+            integ[i] += eta * e
+            want = kp * eta * e + ki * integ[i] + kd * eta * (e - eprev[i]) + float(b0[i])
+            assert st["bias"][i] == pytest.approx(want, abs=2e-7), (c, i)
+            eprev[i] = e
+    # the second step's derivative term is kd * eta * (e2 - e1), not its sum
+    assert eprev[0] != 0.0 and abs(kd * 0.25 * (eprev[0] - 0.0)) > 1e-3
 
 
 def test_update_bias_fixed_point_and_incremental_form():
@@ -469,6 +527,63 @@ def test_ffn_fp8_lossless_closed_form():
     assert not np.allclose(y_swapped, y)
 
 
+
+def test_ffn_fp8_quantizes_h_per_block():
+    """Two active hidden units with exact operands: h = silu(64) * 7 = 448 sets the
+    [1,128] block's scale to 2^0, and h = silu(48) * 6.5 = 312 lies between the E4M3
+    values 288 and 320, so it must reach the down projection as 320:
+    y = 448 W_d[:, 0] + 320 W_d[:, 1] exactly (312 would mean H was not quantized)."""
+    d = inter = 128
+    x = np.zeros((1, d), np.float32)
+    x[0, 0] = 1.0
+    wg = np.zeros((inter, d), np.float32)
+    wu = np.zeros((inter, d), np.float32)
+    wg[0, 0], wu[0, 0] = 64.0, 7.0
+    wg[1, 0], wu[1, 0] = 48.0, 6.5
+    wd = np.zeros((d, inter), np.float32)
+    wd[:, 0] = ((np.arange(d) % 8) - 4) * 0.25
+    wd[:, 1] = ((np.arange(d) % 5) - 2) * 0.5
+    q = [oracle.quantize_blocks(w, 128) for w in (wg, wu, wd)]
+    for (c, s_), w in zip(q, (wg, wu, wd)):
+        assert np.array_equal(oracle.dequantize_blocks(c, s_, 128), w)   # lossless
+    y = oracle.ffn_fp8(x, [c for c, _ in q], [s_ for _, s_ in q])
+    want = 448.0 * wd[:, 0].astype(np.float64) + 320.0 * wd[:, 1].astype(np.float64)
+    assert np.array_equal(y[0], want)
+    assert not np.array_equal(y[0], 448.0 * wd[:, 0].astype(np.float64) + 312.0 * wd[:, 1].astype(np.float64))
+
+
+
+def _blocky(rng, rows, cols, block_rows, block_cols, std=1.0):
+    """Normal values whose blocks have different magnitudes (factors 1/4 .. 8), so
+    that neighbouring quantization blocks get different scales."""
+    a = rng.normal(size=(rows, cols)) * std
+    f = np.array([1.0, 8.0, 0.25, 2.0])
+    for rb in range(0, rows, block_rows):
+        for cb in range(0, cols, block_cols):
+            a[rb:rb + block_rows, cb:cb + block_cols] *= f[(rb // block_rows + 2 * (cb // block_cols)) % 4]
+    return a.astype(np.float32)
+
+
+def test_ffn_fp8_equals_matmuls_on_the_quantized_operands():
+    """The FP8 expert restated with library matmuls over the operands as the pinned
+    quantizer leaves them: x per [1,128], the weights per [128,128], and H = silu(g) u
+    rounded to fp32 then quantized per [1,128].  Each block has its own scale."""
+    rng = _rng(41)
+    n, d, inter = 6, 256, 384
+    x = _blocky(rng, n, d, 1, 128)
+    wg, wu = _blocky(rng, inter, d, 128, 128, 0.05), _blocky(rng, inter, d, 128, 128, 0.05)
+    wd = _blocky(rng, d, inter, 128, 128, 0.05)
+    q = [oracle.quantize_blocks(m, 128) for m in (wg, wu, wd)]
+    Wg, Wu, Wd = (oracle.dequantize_blocks(c, s_, 128) for c, s_ in q)
+    assert len(np.unique(q[0][1])) > 1                   # the blocks' scales differ
+    y = oracle.ffn_fp8(x, [c for c, _ in q], [s_ for _, s_ in q])
+    xq = oracle.dequantize_blocks(*oracle.quantize_blocks(x, 1), 1)
+    g, u = xq @ Wg.T, xq @ Wu.T
+    h32 = (g / (1.0 + np.exp(-g)) * u).astype(np.float32)
+    want = oracle.dequantize_blocks(*oracle.quantize_blocks(h32, 1), 1) @ Wd.T
+    np.testing.assert_allclose(y, want, rtol=1e-10, atol=1e-12 * np.abs(want).max())
+
+
 def test_ffn_fp8_is_close_to_the_unquantized_expert():
     """The quantization error of the method on random data: a few percent of a row's
     largest output, far below the difference a wrong operand or scale would make."""
@@ -559,6 +674,48 @@ def test_ffn_fp4_lossless_closed_form():
     assert np.array_equal(y[0], 64.0 * wd[:, 0].astype(np.float64))
     y_swapped = oracle.ffn_fp4(x, [q[1][0], q[0][0], q[2][0]], [q[1][1], q[0][1], q[2][1]])
     assert not np.allclose(y_swapped, y)
+
+
+
+def test_ffn_fp4_quantizes_h_per_block():
+    """The MXFP4 counterpart: h = silu(64) * 6 = 384 sets the [1,32] block's scale to
+    2^6 (384 = 6 * 64), and h = silu(48) * 6 = 288 = 4.5 * 64 lies between the E2M1
+    values 4 and 6, so it reaches the down projection as 4 * 64 = 256."""
+    d = inter = 64
+    x = np.zeros((1, d), np.float32)
+    x[0, 0] = 1.0
+    wg = np.zeros((inter, d), np.float32)
+    wu = np.zeros((inter, d), np.float32)
+    wg[0, 0], wu[0, 0] = 64.0, 6.0
+    wg[1, 0], wu[1, 0] = 48.0, 6.0
+    wd = np.zeros((d, inter), np.float32)
+    wd[:, 0] = np.resize([1.0, -1.0, 0.5, -0.5], d)
+    wd[:, 1] = np.resize([0.5, 1.0, -1.0, 0.0], d)
+    q = [oracle.quantize_mx4(w) for w in (wg, wu, wd)]
+    for (c, s_), w in zip(q, (wg, wu, wd)):
+        assert np.array_equal(oracle.dequantize_mx4(c, s_), w)   # lossless
+    y = oracle.ffn_fp4(x, [c for c, _ in q], [s_ for _, s_ in q])
+    want = 384.0 * wd[:, 0].astype(np.float64) + 256.0 * wd[:, 1].astype(np.float64)
+    assert np.array_equal(y[0], want)
+
+
+
+def test_ffn_fp4_equals_matmuls_on_the_quantized_operands():
+    """The MXFP4 expert restated the same way: every operand row quantized per [1,32],
+    H rounded to fp32 then quantized per [1,32]."""
+    rng = _rng(42)
+    n, d, inter = 6, 128, 192
+    x = _blocky(rng, n, d, 1, 32)
+    wg, wu = _blocky(rng, inter, d, 1, 32, 0.05), _blocky(rng, inter, d, 1, 32, 0.05)
+    wd = _blocky(rng, d, inter, 1, 32, 0.05)
+    q = [oracle.quantize_mx4(m) for m in (wg, wu, wd)]
+    Wg, Wu, Wd = (oracle.dequantize_mx4(c, s_) for c, s_ in q)
+    y = oracle.ffn_fp4(x, [c for c, _ in q], [s_ for _, s_ in q])
+    xq = oracle.dequantize_mx4(*oracle.quantize_mx4(x))
+    g, u = xq @ Wg.T, xq @ Wu.T
+    h32 = (g / (1.0 + np.exp(-g)) * u).astype(np.float32)
+    want = oracle.dequantize_mx4(*oracle.quantize_mx4(h32)) @ Wd.T
+    np.testing.assert_allclose(y, want, rtol=1e-10, atol=1e-12 * np.abs(want).max())
 
 
 def test_ffn_fp4_is_close_to_the_unquantized_expert():
