@@ -110,6 +110,20 @@ MUTANTS = [
      "const double sgv = ldexp(1.0, (int)sg[(i / 128) * dkb] - 127);", 0),
     ("FP4 x not quantized", "for (int c = 0; c < d; ++c) xv[c] = mx4_value(xq, xsc, d, 0, c, tab);",
      "for (int c = 0; c < d; ++c) xv[c] = elem(xs, x_dtype, r * d + c);", 0),
+    ("softmax numerator without the max", "s[t * E + e] = exp(lt[e] - m) / sum;", "s[t * E + e] = exp(lt[e]) / sum;", 0),
+    ("top-k never marks a pick taken", "taken[best] = 1;\n      idx[t * k + j] = best;\n      gate[t * k + j] = scale * st[best];",
+     "taken[best] = 0;\n      idx[t * k + j] = best;\n      gate[t * k + j] = scale * st[best];", 0),
+    ("zero expert returns token 0", "yt[c] += zsum * elem(x, x_dtype, t * d + c);", "yt[c] += zsum * elem(x, x_dtype, c);", 0),
+    ("load per pick instead of per token", "const float tf = (float)*tokens;", "const float tf = (float)(*tokens * k);", 0),
+    ("block amax from the first row only", "for (int64_t r = r0; r < r1; ++r)\n        for (int64_t c = cb * 128; c < cb * 128 + 128; ++c) {\n          const double a",
+     "for (int64_t r = r0; r < r0 + 1; ++r)\n        for (int64_t c = cb * 128; c < cb * 128 + 128; ++c) {\n          const double a", 0),
+    ("FP8 down scale index transposed", "ldexp(1.0, (int)sd[(c / 128) * ikb + i / 128] - 127)",
+     "ldexp(1.0, (int)sd[(i / 128) * dkb + c / 128] - 127)", 0),
+    ("router scale dropped in the backward", "ds[e] += scale * dg;\n      for (int i = 0; i < inter; ++i) {",
+     "ds[e] += dg;\n      for (int i = 0; i < inter; ++i) {", 0),
+    ("softmax Jacobian mean without s", "for (int e = 0; e < E; ++e) sds += s[t * E + e] * ds[e];",
+     "for (int e = 0; e < E; ++e) sds += ds[e];", 0),
+    ("up uses the gate weights", "u += elem(wu, w_dtype, (int64_t)i * d + c) * xv;", "u += elem(wg, w_dtype, (int64_t)i * d + c) * xv;", 0),
     ("FP4 weight scale of the first block only", "const double sgv = ldexp(1.0, (int)sg[(int64_t)i * (d / 32) + c / 32] - 127);",
      "const double sgv = ldexp(1.0, (int)sg[(int64_t)i * (d / 32)] - 127);", 0),
 ]
