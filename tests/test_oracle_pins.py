@@ -280,6 +280,39 @@ def test_layer_dense_masked_formulation():
     np.testing.assert_allclose(y2, y, rtol=1e-12, atol=1e-14)
 
 
+
+def test_layer_outputs_bf16_rows_and_quantized_expert_flags():
+    """The per-expert fetch path on bf16 bit patterns equals the same path on the
+    fp32 values they encode; with fp8 / fp4 it runs the FP8 expert on weights
+    quantized per [128,128], or the MXFP4 expert on weights quantized per [1,32]."""
+    T, d, N, Z, inter, k = 12, 128, 4, 2, 128, 3
+    x, wg, wu, wd = _tiny_layer(T=T, d=d, N=N, Z=Z, inter=inter, k=k)
+    s = oracle.softmax(_rng(17).normal(size=(T, N + Z)))
+    idx, gate, _ = oracle.topk(s, None, k, 1.25)
+    bits = synth.f32_to_bf16_bits(x)
+    xb = synth.bf16_bits_to_f32(bits)
+    fetch = lambda e: (wg[e], wu[e], wd[e])  # noqa: E731
+    np.testing.assert_array_equal(oracle.layer_outputs(bits, idx, gate, N, fetch),
+                                  oracle.layer_outputs(xb, idx, gate, N, fetch))
+    np.testing.assert_allclose(oracle.layer_outputs(xb, idx, gate, N, fetch), oracle.layer(xb, idx, gate, N, wg, wu, wd),
+                               rtol=1e-12, atol=1e-14)   # the same sum, added in another order
+
+    def fp8_expert(e, rows):
+        q = [oracle.quantize_blocks(w, 128) for w in fetch(e)]
+        return oracle.ffn_fp8(rows, [c for c, _ in q], [s_ for _, s_ in q])
+
+    def fp4_expert(e, rows):
+        q = [oracle.quantize_mx4(w) for w in fetch(e)]
+        return oracle.ffn_fp4(rows, [c for c, _ in q], [s_ for _, s_ in q])
+
+    y8 = oracle.layer_outputs(bits, idx, gate, N, fetch, fp8=True)
+    np.testing.assert_array_equal(y8, oracle.layer_outputs(bits, idx, gate, N, None, expert_fn=fp8_expert))
+    y4 = oracle.layer_outputs(bits, idx, gate, N, fetch, fp4=True)
+    np.testing.assert_array_equal(y4, oracle.layer_outputs(bits, idx, gate, N, None, expert_fn=fp4_expert))
+    y = oracle.layer_outputs(bits, idx, gate, N, fetch)
+    assert not np.array_equal(y8, y) and not np.array_equal(y4, y) and not np.array_equal(y8, y4)
+
+
 def test_layer_identical_experts_closed_form():
     T, d, N, Z, inter, k = 10, 16, 4, 4, 8, 4
     x, wg, wu, wd = _tiny_layer(T=T, d=d, N=N, Z=Z, inter=inter, k=k)
