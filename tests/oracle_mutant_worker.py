@@ -1,8 +1,11 @@
 """Runs tests/test_oracle_pins.py once per oracle library named on the command
 line, all in this one process (the imports are paid once), and prints one JSON
-line per library: {"lib": path, "rc": pytest's exit code}.  A helper of
-tests/test_oracle_mutants.py, which builds the libraries from mutated copies of
-the oracle's source; not a test module itself."""
+line per library: {"lib": path, "rc": pytest's exit code}.
+
+With ``--oracle-dir DIR`` first, the oracle package is imported from DIR (a copy
+whose Python glue may carry a planted mistake) instead of the repository's.  A
+helper of tests/test_oracle_mutants.py, which builds the libraries and copies;
+not a test module itself."""
 import json
 import os
 import sys
@@ -11,6 +14,9 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
+if len(sys.argv) > 2 and sys.argv[1] == "--oracle-dir":
+    sys.path.insert(0, sys.argv[2])
+    del sys.argv[1:3]
 
 import oracle  # noqa: E402
 

@@ -7,12 +7,17 @@ operand, a changed rounding or tie rule.  The copy is built the way the oracle
 is built, and tests/test_oracle_pins.py runs against it (oracle.use_library, in
 worker processes that each take a share of the copies).
 
+The second test does the same for the oracle's Python glue (oracle/__init__.py):
+each mistake goes into a copy of the package, which a worker imports in place of
+the repository's.
+
 Every mutant must fail at least one pin.  An unchanged copy built the same way
 must pass them all, so a broken harness cannot pass for a caught mutant.  The
 mistakes live only in the temporary copies, on the CPU."""
 import concurrent.futures
 import json
 import os
+import shutil
 import subprocess
 import sys
 
@@ -20,6 +25,7 @@ import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "zcmoe_oracle.c")
+PY_SRC = os.path.join(ROOT, "oracle", "__init__.py")
 
 # (name, text in the source, replacement, which occurrence)
 MUTANTS = [
@@ -129,6 +135,28 @@ MUTANTS = [
 ]
 
 
+# Mistakes in the Python glue (oracle/__init__.py): each runs against its own copy
+# of the package, with the unchanged C library.
+PY_MUTANTS = [
+    ("layer outputs: zero-expert term dropped", "y += zsum[:, None] * xf", "y += 0.0 * zsum[:, None] * xf", 0),
+    ("layer outputs: expert output not gated", "y[r] += float(gate[r, j]) * f[i]", "y[r] += f[i]", 1),
+    ("layer outputs: bf16 rows decoded with the wrong shift", "(x_rows.astype(np.uint32) << 16)",
+     "(x_rows.astype(np.uint32) << 8)", 0),
+    ("layer outputs: FP8 weights quantized per [1,128]",
+     "q = [quantize_blocks(w, 128) for w in (wg, wu, wd)]\n            f = ffn_fp8",
+     "q = [quantize_blocks(w, 1) for w in (wg, wu, wd)]\n            f = ffn_fp8", 0),
+    ("dequantize: scale ignored", "return np.ldexp(table[codes], sc)", "return table[codes]", 0),
+    ("dequantize MXFP4: nibbles swapped", "nib[:, 0::2] = codes & 0xF\n    nib[:, 1::2] = codes >> 4",
+     "nib[:, 0::2] = codes >> 4\n    nib[:, 1::2] = codes & 0xF", 0),
+    ("router logits: offset not passed", "off = None if offset is None else np.ascontiguousarray(offset, dtype=np.float32)",
+     "off = None", 0),
+    ("top-k: scale not passed", "float(scale), idx, gate, margin.ctypes.data", "1.0, idx, gate, margin.ctypes.data", 0),
+    ("integer stage: the whole perm buffer returned", "perm[:P].copy()", "perm.copy()", 0),
+    ("brute force: ties to the later subset", "if best is None or s > best_sum:", "if best is None or s >= best_sum:", 0),
+    ("controller state: eta starts at 0", '"eta": np.ones(1, np.float32)', '"eta": np.zeros(1, np.float32)', 0),
+]
+
+
 def _mutate(src, old, new, nth):
     start = -1
     for _ in range(nth + 1):
@@ -148,11 +176,13 @@ def _build(job):
     return so_path
 
 
-def _run_worker(paths):
-    """The pins against each library in `paths`, in one worker process."""
+def _run_worker(paths, oracle_dir=None):
+    """The pins against each library in `paths`, in one worker process (importing the
+    oracle package from `oracle_dir` when given)."""
     env = dict(os.environ, OMP_NUM_THREADS="2")
-    r = subprocess.run([sys.executable, os.path.join(ROOT, "tests", "oracle_mutant_worker.py"), *paths], cwd=ROOT,
-                       env=env, capture_output=True, text=True, timeout=1200)
+    pre = ["--oracle-dir", oracle_dir] if oracle_dir else []
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "tests", "oracle_mutant_worker.py"), *pre, *paths],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=1200)
     rcs = {}
     for line in r.stdout.splitlines():
         if line.startswith("ZCMOE-MUTANT "):
@@ -180,4 +210,34 @@ def test_every_planted_mistake_fails_a_pin(tmp_path):
     names = {lib: name for lib, (name, _) in zip(libs, jobs)}
     assert rcs[libs[0]] == 0, "the unchanged copy must pass every pin:\n" + "\n".join(logs)
     survivors = [names[lib] for lib in libs[1:] if rcs[lib] != 1]
+    assert not survivors, f"mistakes that no pin caught (pytest exit code other than 1): {survivors}"
+
+
+def _py_copy(job):
+    """A copy of the oracle package with `text` as its Python glue and the repository's
+    C source and library; returns (package parent dir, library path)."""
+    out_dir, text = job
+    pkg = os.path.join(out_dir, "oracle")
+    os.makedirs(pkg, exist_ok=True)
+    with open(os.path.join(pkg, "__init__.py"), "w") as f:
+        f.write(text)
+    shutil.copy2(SRC, os.path.join(pkg, "zcmoe_oracle.c"))
+    so = os.path.join(pkg, "liboracle.so")
+    shutil.copy2(oracle.build(), so)
+    return out_dir, so
+
+
+def test_every_planted_mistake_in_the_python_glue_fails_a_pin(tmp_path):
+    src = open(PY_SRC).read()
+    jobs = [("control", src)] + [(name, _mutate(src, old, new, nth)) for name, old, new, nth in PY_MUTANTS]
+    for name, text in jobs[1:]:
+        assert text != src, name
+    copies = [_py_copy((str(tmp_path / f"p{i}"), text)) for i, (_, text) in enumerate(jobs)]
+    workers = max(1, min(8, (os.cpu_count() or 2) // 2))
+    with concurrent.futures.ThreadPoolExecutor(workers) as ex:
+        results = list(ex.map(lambda c: _run_worker([c[1]], oracle_dir=c[0]), copies))
+    rcs = [got.get(so) for (got, _), (_, so) in zip(results, copies)]
+    logs = [log for _, log in results]
+    assert rcs[0] == 0, "the unchanged copy must pass every pin:\n" + logs[0]
+    survivors = [name for (name, _), rc in zip(jobs[1:], rcs[1:]) if rc != 1]
     assert not survivors, f"mistakes that no pin caught (pytest exit code other than 1): {survivors}"
