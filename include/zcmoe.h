@@ -183,6 +183,25 @@ ZCMOE_API int zcmoe_get_state(zcmoe_t h, float *bias, int64_t *counts, int64_t *
 /* Replaces the bias (host [E] fp32).  Does not change b0 or the controller state.  Synchronous. */
 ZCMOE_API int zcmoe_set_bias(zcmoe_t h, const float *bias);
 
+/* The whole mutable state of the bias controller, for checkpoint and resume (the
+ * PID of zcmoe_update_bias; LongCat-Flash technical summary, 二.1 "計算預算控制").
+ * All host pointers:
+ *   bias [E] fp32    the current bias;
+ *   integ [E] fp32   the PID's integral I;
+ *   eprev [E] fp32   the previous step's error;
+ *   eta [1] fp32     the decayed step factor;
+ *   counts [E] int64, tokens [1] int64   the selections accumulated since the last step.
+ * zcmoe_get_controller fills every non-NULL pointer; it synchronises the device.
+ * zcmoe_set_controller replaces all six (none may be NULL; counts and tokens must be
+ * >= 0 and eta finite, else ZCMOE_EINVAL with nothing changed); synchronous.
+ * b0, the initial bias the PID adds, is fixed at create from init_bias.  A handle
+ * created with the same init_bias and given another handle's controller state takes
+ * bit-identical controller steps from there on. */
+ZCMOE_API int zcmoe_get_controller(zcmoe_t h, float *bias, float *integ, float *eprev, float *eta, int64_t *counts,
+                                   int64_t *tokens);
+ZCMOE_API int zcmoe_set_controller(zcmoe_t h, const float *bias, const float *integ, const float *eprev,
+                                   const float *eta, const int64_t *counts, const int64_t *tokens);
+
 /* Synchronises the device and reports a device-side timeout (ZCMOE_ETIMEOUT) if a
  * kernel's bounded wait gave up since the last check; clears the flag. */
 ZCMOE_API int zcmoe_check(zcmoe_t h);

@@ -17,6 +17,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <cmath>
 #include <cstdarg>
 #include <mutex>
 #include <new>
@@ -1128,6 +1129,41 @@ int zcmoe_set_bias(zcmoe_t h, const float* bias) {
   if (!bias) return fail(ZCMOE_EINVAL, "bias is NULL");
   ZC_CUDA(cudaDeviceSynchronize());
   ZC_CUDA(cudaMemcpy(h->bias, bias, h->E * sizeof(float), cudaMemcpyHostToDevice));
+  return ZCMOE_OK;
+}
+
+int zcmoe_get_controller(zcmoe_t h, float* bias, float* integ, float* eprev, float* eta, int64_t* counts,
+                         int64_t* tokens) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  ZC_CUDA(cudaDeviceSynchronize());
+  const size_t fE = (size_t)h->E * sizeof(float);
+  if (bias) ZC_CUDA(cudaMemcpy(bias, h->bias, fE, cudaMemcpyDeviceToHost));
+  if (integ) ZC_CUDA(cudaMemcpy(integ, h->integ, fE, cudaMemcpyDeviceToHost));
+  if (eprev) ZC_CUDA(cudaMemcpy(eprev, h->eprev, fE, cudaMemcpyDeviceToHost));
+  if (eta) ZC_CUDA(cudaMemcpy(eta, h->eta, sizeof(float), cudaMemcpyDeviceToHost));
+  if (counts) ZC_CUDA(cudaMemcpy(counts, h->acc_counts, (size_t)h->E * sizeof(int64_t), cudaMemcpyDeviceToHost));
+  if (tokens) ZC_CUDA(cudaMemcpy(tokens, h->acc_tokens, sizeof(int64_t), cudaMemcpyDeviceToHost));
+  return ZCMOE_OK;
+}
+
+int zcmoe_set_controller(zcmoe_t h, const float* bias, const float* integ, const float* eprev, const float* eta,
+                         const int64_t* counts, const int64_t* tokens) {
+  g_err[0] = 0;
+  if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
+  if (!bias || !integ || !eprev || !eta || !counts || !tokens) return fail(ZCMOE_EINVAL, "a state pointer is NULL");
+  if (!std::isfinite(*eta)) return fail(ZCMOE_EINVAL, "eta must be finite");
+  if (*tokens < 0) return fail(ZCMOE_EINVAL, "tokens must be >= 0");
+  for (int i = 0; i < h->E; ++i)
+    if (counts[i] < 0) return fail(ZCMOE_EINVAL, "counts must be >= 0 (expert %d)", i);
+  ZC_CUDA(cudaDeviceSynchronize());
+  const size_t fE = (size_t)h->E * sizeof(float);
+  ZC_CUDA(cudaMemcpy(h->bias, bias, fE, cudaMemcpyHostToDevice));
+  ZC_CUDA(cudaMemcpy(h->integ, integ, fE, cudaMemcpyHostToDevice));
+  ZC_CUDA(cudaMemcpy(h->eprev, eprev, fE, cudaMemcpyHostToDevice));
+  ZC_CUDA(cudaMemcpy(h->eta, eta, sizeof(float), cudaMemcpyHostToDevice));
+  ZC_CUDA(cudaMemcpy(h->acc_counts, counts, (size_t)h->E * sizeof(int64_t), cudaMemcpyHostToDevice));
+  ZC_CUDA(cudaMemcpy(h->acc_tokens, tokens, sizeof(int64_t), cudaMemcpyHostToDevice));
   return ZCMOE_OK;
 }
 

@@ -38,7 +38,7 @@ EXPORTED = ("zcmoe_create", "zcmoe_forward", "zcmoe_forward_host", "zcmoe_update
             "zcmoe_dense_destroy", "zcmoe_quantize_e4m3", "zcmoe_quantize_mx4", "zcmoe_backward",
             "zcmoe_save_for_backward", "zcmoe_backward_ex", "zcmoe_forward_host_async",
             "zcmoe_forward_host_flush", "zcmoe_create_ep", "zcmoe_ep_dispatch", "zcmoe_ep_experts",
-            "zcmoe_ep_combine", "zcmoe_last_error")
+            "zcmoe_ep_combine", "zcmoe_get_controller", "zcmoe_set_controller", "zcmoe_last_error")
 STAGES = ("router", "softmax_topk", "integer", "gather", "gate_up", "down", "combine")
 
 
@@ -100,6 +100,8 @@ def lib():
         L.zcmoe_write_counts.argtypes = [vp, vp, vp]
         L.zcmoe_get_state.argtypes = [vp, vp, vp, vp, vp]
         L.zcmoe_set_bias.argtypes = [vp, vp]
+        L.zcmoe_get_controller.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+        L.zcmoe_set_controller.argtypes = [vp, vp, vp, vp, vp, vp, vp]
         L.zcmoe_check.argtypes = [vp]
         L.zcmoe_destroy.argtypes = [vp]
         L.zcmoe_profile_begin.argtypes = [vp]
@@ -230,6 +232,17 @@ def zcmoe_get_state(h, bias_ptr=None, counts_ptr=None, tokens_ptr=None, eta_ptr=
 
 def zcmoe_set_bias(h, bias_ptr):
     _check(lib().zcmoe_set_bias(h, bias_ptr), "zcmoe_set_bias")
+
+
+def zcmoe_get_controller(h, bias_ptr=None, integ_ptr=None, eprev_ptr=None, eta_ptr=None, counts_ptr=None,
+                         tokens_ptr=None):
+    _check(lib().zcmoe_get_controller(h, bias_ptr, integ_ptr, eprev_ptr, eta_ptr, counts_ptr, tokens_ptr),
+           "zcmoe_get_controller")
+
+
+def zcmoe_set_controller(h, bias_ptr, integ_ptr, eprev_ptr, eta_ptr, counts_ptr, tokens_ptr):
+    _check(lib().zcmoe_set_controller(h, bias_ptr, integ_ptr, eprev_ptr, eta_ptr, counts_ptr, tokens_ptr),
+           "zcmoe_set_controller")
 
 
 def zcmoe_check(h):
@@ -482,6 +495,33 @@ class ZcMoE:
         if b.shape != (self.shape.E,):
             raise ValueError(f"bias: expected {self.shape.E} values, got shape {b.shape}")
         zcmoe_set_bias(self.h, b.ctypes.data)
+
+    CONTROLLER_FIELDS = ("bias", "integ", "eprev", "eta", "counts", "tokens")
+
+    def controller_state(self):
+        """The whole controller state as host arrays (a checkpoint): bias, integ, eprev
+        [E] float32, eta [1] float32, counts [E] int64, tokens [1] int64."""
+        import numpy as np
+        E = self.shape.E
+        st = {"bias": np.empty(E, np.float32), "integ": np.empty(E, np.float32), "eprev": np.empty(E, np.float32),
+              "eta": np.empty(1, np.float32), "counts": np.empty(E, np.int64), "tokens": np.empty(1, np.int64)}
+        zcmoe_get_controller(self.h, *(st[k].ctypes.data for k in self.CONTROLLER_FIELDS))
+        return st
+
+    def load_controller_state(self, st):
+        """Restores a controller_state() checkpoint (the handle must have been created
+        with the same init_bias for the steps to continue identically)."""
+        import numpy as np
+        E = self.shape.E
+        want = {"bias": (E, np.float32), "integ": (E, np.float32), "eprev": (E, np.float32), "eta": (1, np.float32),
+                "counts": (E, np.int64), "tokens": (1, np.int64)}
+        arrs = {}
+        for k, (n, dt) in want.items():
+            a = np.ascontiguousarray(st[k], dtype=dt).reshape(-1)
+            if a.shape != (n,):
+                raise ValueError(f"{k}: expected {n} values, got {a.size}")
+            arrs[k] = a
+        zcmoe_set_controller(self.h, *(arrs[k].ctypes.data for k in self.CONTROLLER_FIELDS))
 
     def check(self):
         zcmoe_check(self.h)

@@ -197,3 +197,29 @@ def test_layer_methods_check_tensors_before_the_library(zc):
         assert ei.value.code == zc.ZCMOE_EINVAL
     finally:
         lay.h = None
+
+
+def test_controller_checkpoint_entry_points_refuse_unknown_handles(zc):
+    lib = zc.lib()
+    fake = ctypes.c_void_p(0x1000)
+    assert lib.zcmoe_get_controller(fake, None, None, None, None, None, None) == zc.ZCMOE_EINVAL
+    assert lib.zcmoe_set_controller(fake, None, None, None, None, None, None) == zc.ZCMOE_EINVAL
+    assert "handle" in zc.zcmoe_last_error()
+
+
+def test_load_controller_state_checks_sizes_before_the_library(zc):
+    import numpy as np
+    lay = object.__new__(zc.ZcMoE)
+    lay.shape = zc.LayerShape(64, 4, 2, 32, 2, "bf16")
+    lay.h = ctypes.c_void_p(0x1000)
+    try:
+        E = lay.shape.E
+        good = {"bias": np.zeros(E), "integ": np.zeros(E), "eprev": np.zeros(E), "eta": [1.0],
+                "counts": np.zeros(E, np.int64), "tokens": [0]}
+        with pytest.raises(ValueError):
+            lay.load_controller_state(dict(good, integ=np.zeros(E - 1)))
+        with pytest.raises(zc.ZcmoeError) as ei:      # well-formed: reaches the library, which refuses the handle
+            lay.load_controller_state(good)
+        assert ei.value.code == zc.ZCMOE_EINVAL
+    finally:
+        lay.h = None

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import oracle
-from mixture_experts_layer_shifted_b200 import configs, synth
+from mixture_experts_layer_shifted_b200 import configs, synth, zcmoe
 from tests.gpu_harness import TOL, Run, row_rel_err
 
 pytestmark = pytest.mark.gpu
@@ -214,6 +214,51 @@ def test_controller_step_bitexact(cuda_ok):
             assert s2["eta"] == float(st_o["eta"][0])
     finally:
         r.close()
+
+
+
+def test_controller_checkpoint_and_resume(cuda_ok):
+    """A checkpoint of the whole controller state (bias, I, e_prev, eta and the counts
+    accumulated since the last step), loaded into a fresh handle made with the same
+    init_bias: both handles then take bit-identical steps, equal to the oracle's."""
+    w = W["small_bf16"]
+    gains = (0.3, 0.05, 0.2, 0.97, 5.0)
+    a = Run(w)
+    b = Run(w, weights=a.weights)
+    try:
+        st_o = oracle.new_controller_state(a.bias)
+        for step in range(3):
+            a.x = configs.device_tokens(w, step=step)
+            a.forward(debug=False)
+            s = a.layer.state()
+            oracle.update_bias(s["counts"].copy(), np.array([s["tokens"]], np.int64), w.n_ffn, w.n_zero, w.top_k,
+                               gains, a.bias, st_o)
+            a.layer.update_bias(*gains[:4], target_ffn_per_token=gains[4])
+        a.x = configs.device_tokens(w, step=3)
+        a.forward(debug=False)                       # counts pending at the checkpoint
+        ck = a.layer.controller_state()
+        np.testing.assert_array_equal(ck["integ"].view(np.uint32), st_o["integ"].view(np.uint32))
+        np.testing.assert_array_equal(ck["eprev"].view(np.uint32), st_o["eprev"].view(np.uint32))
+        assert ck["tokens"][0] == w.T and ck["counts"].sum() == w.T * w.top_k
+        b.layer.load_controller_state(ck)
+        back = b.layer.controller_state()
+        for key in ck:
+            np.testing.assert_array_equal(back[key], ck[key])
+        for step in range(4, 7):
+            for r in (a, b):
+                r.layer.update_bias(*gains[:4], target_ffn_per_token=gains[4])
+                r.x = configs.device_tokens(w, step=step)
+                r.forward(debug=False)
+            sa, sb = a.layer.controller_state(), b.layer.controller_state()
+            for key in sa:
+                np.testing.assert_array_equal(sa[key], sb[key])
+        with pytest.raises(zcmoe.ZcmoeError) as ei:   # negative counts are refused, nothing changed
+            b.layer.load_controller_state(dict(ck, counts=-np.ones(w.E, np.int64)))
+        assert ei.value.code == zcmoe.ZCMOE_EINVAL
+        np.testing.assert_array_equal(b.layer.controller_state()["bias"], sb["bias"])
+    finally:
+        a.close()
+        b.close()
 
 
 def test_counts_exchange_roundtrip(small):
