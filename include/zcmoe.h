@@ -84,7 +84,7 @@ typedef struct {
   int32_t top_k;        /* experts chosen per token                      */
   int32_t max_tokens;   /* largest T accepted by zcmoe_forward           */
   int32_t dtype;        /* zcmoe_dtype                                   */
-  float routed_scale;   /* gate = routed_scale * score (the "scaling" of the fused router); 1.0 if unsure */
+  float routed_scale;   /* gate = routed_scale * score (the "scaling" of the fused router); finite; 1.0 if unsure */
   const float *init_bias;    /* host [E] or NULL (zeros); copied at create; also the controller's b0 */
   const float *logit_offset; /* host [E] or NULL; copied; added to every token's logits before softmax */
 } zcmoe_config;

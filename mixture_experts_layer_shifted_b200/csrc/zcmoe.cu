@@ -355,6 +355,7 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
   for (const void* p : wp)
     if (reinterpret_cast<uintptr_t>(p) & 15u) return fail(ZCMOE_EINVAL, "weight pointers must be 16-byte aligned");
   if ((int64_t)cfg->max_tokens * k >= (int64_t)1 << 31) return fail(ZCMOE_EINVAL, "max_tokens * top_k too large");
+  if (!std::isfinite(cfg->routed_scale)) return fail(ZCMOE_EINVAL, "routed_scale must be finite");
 
   int dev = 0;
   ZC_CUDA(cudaGetDevice(&dev));

@@ -223,3 +223,31 @@ def test_load_controller_state_checks_sizes_before_the_library(zc):
         assert ei.value.code == zc.ZCMOE_EINVAL
     finally:
         lay.h = None
+
+
+def test_create_checks_quantized_shapes_scale_and_group_on_the_host(zc):
+    """Refusals that come before any device call: FP8 / MXFP4 shape rules, a routed
+    scale that is not finite, and expert-parallel group arguments."""
+    import math
+    lib = zc.lib()
+    h = ctypes.c_void_p()
+    w = zc.zcmoe_weights(16, 16, 16, 16)
+
+    def cfg(**kw):
+        c = zc.zcmoe_config(512, 16, 8, 256, 4, 64, zc.ZCMOE_BF16, 1.0, None, None)
+        for k_, v in kw.items():
+            setattr(c, k_, v)
+        return c
+
+    for bad in [dict(dtype=zc.ZCMOE_FP8, d=256), dict(dtype=zc.ZCMOE_FP8, inter=192),
+                dict(dtype=zc.ZCMOE_FP4, d=768), dict(dtype=zc.ZCMOE_FP4, inter=128),
+                dict(routed_scale=math.nan), dict(routed_scale=math.inf)]:
+        assert lib.zcmoe_create(ctypes.byref(cfg(**bad)), ctypes.byref(w), ctypes.byref(h)) == zc.ZCMOE_EINVAL, bad
+        assert h.value is None
+    c = cfg()
+    for rank, size, cap in [(-1, 2, 0), (2, 2, 0), (0, 0, 0), (0, 3, 0), (0, 2, -1), (0, 2, 1 << 31)]:
+        assert lib.zcmoe_create_ep(ctypes.byref(c), ctypes.byref(w), rank, size, cap, ctypes.byref(h)) == \
+            zc.ZCMOE_EINVAL, (rank, size, cap)
+        assert h.value is None
+    assert lib.zcmoe_create_ep(ctypes.byref(cfg(dtype=zc.ZCMOE_FP8)), ctypes.byref(w), 0, 2, 0,
+                               ctypes.byref(h)) == zc.ZCMOE_EUNSUPPORTED
