@@ -164,7 +164,8 @@ ZCMOE_API int zcmoe_forward_host_flush(zcmoe_t h, cudaStream_t stream);
  *   experts, (k-K)/Z for zero experts; e_i = tau_i - l_i; eta <- eta*decay;
  *   I_i <- I_i + eta*e_i; b_i <- ((kp*eta*e_i + ki*I_i) + kd*eta*(e_i - e_prev_i)) + b0_i;
  *   e_prev_i <- e_i; the accumulators are reset.  No-op while T_acc == 0.
- * Asynchronous on `stream`. */
+ * kp, ki, kd and decay must be finite and 0 <= K <= top_k (K = top_k without zero
+ * experts), else ZCMOE_EINVAL with nothing enqueued.  Asynchronous on `stream`. */
 ZCMOE_API int zcmoe_update_bias(zcmoe_t h, const zcmoe_gains *g, cudaStream_t stream);
 
 /* Data-parallel exchange of the accumulators.  read: copies the handle's

@@ -1088,6 +1088,8 @@ int zcmoe_update_bias(zcmoe_t h, const zcmoe_gains* g, cudaStream_t s) {
   g_err[0] = 0;
   if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
   if (!g) return fail(ZCMOE_EINVAL, "gains is NULL");
+  if (!std::isfinite(g->kp) || !std::isfinite(g->ki) || !std::isfinite(g->kd) || !std::isfinite(g->decay))
+    return fail(ZCMOE_EINVAL, "kp, ki, kd and decay must be finite");
   if (!(g->target_ffn_per_token >= 0.0f && g->target_ffn_per_token <= (float)h->k))
     return fail(ZCMOE_EINVAL, "target_ffn_per_token must lie in [0, top_k]");
   if (h->Z == 0 && g->target_ffn_per_token != (float)h->k)

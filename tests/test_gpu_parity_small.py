@@ -261,6 +261,21 @@ def test_controller_checkpoint_and_resume(cuda_ok):
         b.close()
 
 
+
+def test_update_bias_refuses_gains_that_are_not_finite(small):
+    """A NaN or infinite gain would poison the bias and every later routing decision:
+    the step is refused on the host and the controller state stays as it was."""
+    before = small.layer.controller_state()
+    for bad in (dict(kp=float("nan")), dict(ki=float("inf")), dict(kd=-float("inf")), dict(decay=float("nan"))):
+        gains = dict(dict(kp=0.0, ki=0.05, kd=0.0, decay=1.0), **bad)
+        with pytest.raises(zcmoe.ZcmoeError) as ei:
+            small.layer.update_bias(target_ffn_per_token=5.0, **gains)
+        assert ei.value.code == zcmoe.ZCMOE_EINVAL
+    after = small.layer.controller_state()
+    for key in before:
+        np.testing.assert_array_equal(after[key], before[key])
+
+
 def test_counts_exchange_roundtrip(small):
     E = small.w.E
     buf = torch.empty(E + 1, dtype=torch.int64, device="cuda")
