@@ -107,6 +107,7 @@ def _free_port():
     (2, (37, 50), 1),
     (2, (37, 50), 2),
     (4, (20, 0, 33, 9), 2),   # a rank with no tokens
+    (2, (1, 6), 2),           # one token in two chunks: one chunk of that rank is empty
 ])
 def test_ep_forward_matches_the_whole_layer(world, sizes, chunks):
     mgr = mp.get_context("spawn").Manager()
