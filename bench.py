@@ -562,6 +562,18 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
 
+    if args.impl == "reference":
+        # the CPU oracle runs on rank 0 alone; the other ranks exit 0 without work, and no
+        # process group is formed (nothing would be exchanged)
+        rank, ws = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
+        if rank != 0:
+            return
+        import torch
+        from mixture_experts_layer_shifted_b200 import configs
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        run_reference(args, configs.WORKLOADS[args.workload], rank, ws)
+        return
+
     import torch
     from mixture_experts_layer_shifted_b200 import configs
     from mixture_experts_layer_shifted_b200.dp import controller_step
@@ -569,12 +581,6 @@ def main():
 
     dist, rank, ws, local = _dist()
     wl = configs.WORKLOADS[args.workload]
-    if args.impl == "reference":
-        run_reference(args, wl, rank, ws)
-        if dist:
-            dist.barrier()
-            dist.destroy_process_group()
-        return
 
     peaks = _peaks()
     dev = torch.device("cuda", local)

@@ -171,3 +171,16 @@ def test_clock_sampler_with_a_fake_nvidia_smi(tmp_path, monkeypatch):
     c = s.stop()
     assert c["samples"] == 2 and c["sm_mhz"] == 1250 and c["reasons"] == ["sw_power_cap"]
     assert "rejected" not in c
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    """Under torchrun the reference arm runs on rank 0 alone: any other rank exits 0 at
+    once, prints nothing and forms no process group (no rendezvous is reachable here,
+    so joining one would fail or hang)."""
+    import subprocess
+    import sys
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1", MASTER_ADDR="127.0.0.1", MASTER_PORT="9")
+    r = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl", "reference", "--gpus", "2"],
+                       env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
