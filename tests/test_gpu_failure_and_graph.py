@@ -4,7 +4,9 @@
   timeout that zcmoe_check reports, and leaves the context usable.
 * A device allocation failure at create is reported as ZCMOE_ENOMEM and
   leaves nothing behind.
-* A forward captured in a CUDA graph replays to the same bits as eager."""
+* A forward captured in a CUDA graph replays to the same bits as eager.
+* A destroyed handle is refused by every entry point (double destroy, use after
+  destroy) instead of being dereferenced."""
 import ctypes
 
 import numpy as np
@@ -84,3 +86,21 @@ def test_forward_in_cuda_graph_matches_eager(cuda_ok):
         assert r.layer.state()["tokens"] == tok0 + 4 * r.T
     finally:
         r.close()
+
+
+def test_destroyed_handle_is_refused(cuda_ok):
+    r = Run(configs.WORKLOADS["tiny_f32"])
+    raw = r.layer.h
+    lib = Z.lib()
+    y = torch.empty_like(r.x)
+    bias = np.zeros(r.w.E, np.float32)
+    assert lib.zcmoe_destroy(raw) == Z.ZCMOE_OK
+    r.layer.h = None                                    # the owner no longer holds it
+    assert lib.zcmoe_destroy(raw) == Z.ZCMOE_EINVAL      # double destroy
+    xp, yp = ctypes.c_void_p(r.x.data_ptr()), ctypes.c_void_p(y.data_ptr())
+    assert lib.zcmoe_forward(raw, xp, r.x.shape[0], yp, None, None) == Z.ZCMOE_EINVAL
+    gains = Z.zcmoe_gains(0.0, 0.02, 0.0, 1.0, 2.0)
+    assert lib.zcmoe_update_bias(raw, ctypes.byref(gains), None) == Z.ZCMOE_EINVAL
+    assert lib.zcmoe_get_state(raw, bias.ctypes.data, None, None, None) == Z.ZCMOE_EINVAL
+    assert lib.zcmoe_check(raw) == Z.ZCMOE_EINVAL
+    assert "handle" in Z.zcmoe_last_error()
