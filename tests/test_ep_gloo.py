@@ -1,4 +1,5 @@
-"""The expert-parallel protocol (ep.ep_forward) with gloo ranks on CPU.
+"""The expert-parallel protocol (ep.ep_forward, EpMoE.controller_step) with gloo
+ranks on CPU.
 
 The stages run on the oracle here (the CUDA stages are exercised by the GPU tests):
 each rank routes its own tokens in fp64, sends the FFN pairs' rows to the ranks that
@@ -124,3 +125,73 @@ def test_ep_forward_matches_the_whole_layer(world, sizes, chunks):
         want = oracle.layer(x, idx, gate, N, wg, wu, wd)
         err = np.abs(got - want).max() / np.abs(want).max()
         assert err < 1e-6, (r, err)
+
+
+class OracleControllerLayer:
+    """Stands in for one chunk handle in EpMoE.controller_step: its accumulated counts
+    and the oracle's controller state, on the CPU."""
+
+    def __init__(self, counts, tokens, b0):
+        self.acc = torch.tensor(list(counts) + [tokens], dtype=torch.int64)
+        self.b0 = b0
+        self.state = oracle.new_controller_state(b0)
+        self.weights = (torch.zeros(1),)
+
+    def read_counts(self, buf):
+        buf.copy_(self.acc)
+
+    def write_counts(self, buf):
+        self.acc.copy_(buf)
+
+    def update_bias(self, kp, ki, kd, decay, target_ffn_per_token):
+        counts, tokens = self.acc[:-1].numpy().copy(), self.acc[-1:].numpy().copy()
+        oracle.update_bias(counts, tokens, N, Z, K, (kp, ki, kd, decay, target_ffn_per_token), self.b0, self.state)
+        self.acc.zero_()
+
+
+GAINS = dict(kp=0.1, ki=0.05, kd=0.02, decay=0.95, target_ffn_per_token=2.0)
+
+
+def _chunk_counts(rank, chunk):
+    rng = np.random.default_rng(1000 + 10 * rank + chunk)
+    T = 13 + 7 * rank + chunk
+    return rng.multinomial(T * K, [1 / E] * E).astype(np.int64), T
+
+
+def _ctl_worker(rank, world, port, out):
+    from mixture_experts_layer_shifted_b200.ep import EpMoE
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        b0 = np.linspace(-0.01, 0.01, E).astype(np.float32)
+        layer = object.__new__(EpMoE)
+        layer.shape = type("S", (), {"E": E})()
+        layer.layers = [OracleControllerLayer(*_chunk_counts(rank, c), b0) for c in range(2)]
+        layer.controller_step(all_reduce=lambda t: dist.all_reduce(t, op=dist.ReduceOp.SUM), **GAINS)
+        out[rank] = [lay.state["bias"].copy() for lay in layer.layers]
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ep_controller_step_gives_every_handle_the_group_step():
+    """Two gloo ranks with two chunk handles each: after EpMoE.controller_step every
+    handle holds the bias of one controller that saw all four chunks' counts."""
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.spawn(_ctl_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+    total = np.zeros(E, np.int64)
+    tokens = 0
+    for r in range(world):
+        for c in range(2):
+            cnt, T = _chunk_counts(r, c)
+            total += cnt
+            tokens += T
+    b0 = np.linspace(-0.01, 0.01, E).astype(np.float32)
+    st = oracle.new_controller_state(b0)
+    oracle.update_bias(total, np.array([tokens], np.int64), N, Z, K,
+                       tuple(GAINS[k] for k in ("kp", "ki", "kd", "decay", "target_ffn_per_token")), b0, st)
+    for r in range(world):
+        for bias in out[r]:
+            np.testing.assert_array_equal(bias.view(np.uint32), st["bias"].view(np.uint32))
