@@ -16,8 +16,9 @@
 //   m = max_e l_e;  u_e = zexp(l_e - m);
 //   per lane p (e = p, p+32, ...): partial sums in ascending e; then a
 //   butterfly over lane distance 16, 8, 4, 2, 1: partial += partner;
-//   s_e = u_e / sum;  v_e = s_e + b_e;  top-k on v, ties to the lower id;
-//   gate = scale * s.
+//   s_e = u_e / sum;  v_e = s_e + b_e;  top-k on v, ties to the lower id,
+//   a NaN v ranking as -inf;  gate = scale * s.
+// The max skips NaN logits (it starts at -inf and takes fmax).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -56,6 +57,11 @@ __device__ __forceinline__ float zexp(float x) {
 __device__ __forceinline__ bool better(float va, int ea, float vb, int eb) {
   return va > vb || (va == vb && ea < eb);
 }
+
+// Selection key of a biased score: a NaN ranks as -inf (below every number), so a
+// row whose scores are not all numbers still selects k distinct valid experts
+// (the lowest untaken ids among the NaN ones) instead of an id out of range.
+__device__ __forceinline__ float rank_key(float v) { return v == v ? v : -__int_as_float(0x7f800000); }
 
 // One warp per token.  EPL = experts held per lane (E <= 32 * EPL).
 template <int EPL>
@@ -102,7 +108,7 @@ __global__ void __launch_bounds__(256) k_softmax_topk(const float* __restrict__ 
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
       u[i] = __fdiv_rn(u[i], acc);  // u now holds the score s
-      v[i] = __fadd_rn(u[i], b[i]);
+      v[i] = rank_key(__fadd_rn(u[i], b[i]));
       if (e >= E) taken |= 1u << i;
       else if (scores) scores[(int64_t)t * E + e] = u[i];
     }
@@ -220,7 +226,10 @@ __global__ void __launch_bounds__(kChunk) k_route_count(const int32_t* __restric
   __syncthreads();
   const int t = blockIdx.x * kChunk + tid;
   if (t < T)
-    for (int j = 0; j < k; ++j) atomicOr(&smask[warp * E + idx[(int64_t)t * k + j]], 1u << lane);
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(int64_t)t * k + j];
+      if ((unsigned)e < (unsigned)E) atomicOr(&smask[warp * E + e], 1u << lane);  // an id out of range is skipped
+    }
   __syncthreads();
   for (int e = tid; e < E; e += kChunk) {
     int c = 0;
@@ -316,13 +325,16 @@ __global__ void __launch_bounds__(kChunk) k_route_scatter(const int32_t* __restr
   __syncthreads();
   const int t = blockIdx.x * kChunk + tid;
   if (t < T)
-    for (int j = 0; j < k; ++j) atomicOr(&smask[warp * E + idx[(int64_t)t * k + j]], 1u << lane);
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(int64_t)t * k + j];
+      if ((unsigned)e < (unsigned)E) atomicOr(&smask[warp * E + e], 1u << lane);
+    }
   __syncthreads();
   if (t >= T) return;
   for (int j = 0; j < k; ++j) {
     const int64_t pair = (int64_t)t * k + j;
     const int e = idx[pair];
-    if (e < N) {
+    if ((unsigned)e < (unsigned)N) {
       int r = chunk_base[(int64_t)blockIdx.x * E + e];
       for (int w = 0; w < warp; ++w) r += __popc(smask[w * E + e]);
       r += __popc(smask[warp * E + e] & ((1u << lane) - 1u));

@@ -71,19 +71,25 @@ ZO_EXPORT void zo_router_logits(const void *x, int x_dtype, const void *wr, int 
   }
 }
 
-/* Step 2: s = softmax(l) over all E experts, fp64. */
+/* Step 2: s = softmax(l) over all E experts, fp64.  The shift m is the largest
+ * logit that is a number (a NaN logit never compares greater). */
 ZO_EXPORT void zo_softmax_f64(const double *l, int64_t T, int E, double *s) {
 #pragma omp parallel for schedule(static)
   for (int64_t t = 0; t < T; ++t) {
     const double *lt = l + t * E;
-    double m = lt[0];
-    for (int e = 1; e < E; ++e)
+    double m = -INFINITY;
+    for (int e = 0; e < E; ++e)
       if (lt[e] > m) m = lt[e];
     double sum = 0.0;
     for (int e = 0; e < E; ++e) sum += exp(lt[e] - m);
     for (int e = 0; e < E; ++e) s[t * E + e] = exp(lt[e] - m) / sum;
   }
 }
+
+/* Selection key: a biased score that is not a number ranks as -inf, below
+ * every number, so k distinct valid experts are always chosen. */
+static double key64(double v) { return v != v ? -INFINITY : v; }
+static float key32(float v) { return v != v ? -INFINITY : v; }
 
 /* Steps 3-5 (fp64): v = s + b; S = the k largest v, ties to the lower index,
  * slot order v descending then index ascending; gate = scale * s (bias never in
@@ -102,7 +108,7 @@ ZO_EXPORT void zo_topk_f64(const double *s, const double *bias, int64_t T, int E
       double bv = 0.0;
       for (int e = 0; e < E; ++e) {
         if (taken[e]) continue;
-        double v = st[e] + (bias ? bias[e] : 0.0);
+        double v = key64(st[e] + (bias ? bias[e] : 0.0));
         if (best < 0 || v > bv) { best = e; bv = v; } /* strict '>' keeps the lower index on ties */
       }
       taken[best] = 1;
@@ -115,7 +121,7 @@ ZO_EXPORT void zo_topk_f64(const double *s, const double *bias, int64_t T, int E
       int found = 0;
       for (int e = 0; e < E; ++e) {
         if (taken[e]) continue;
-        double v = st[e] + (bias ? bias[e] : 0.0);
+        double v = key64(st[e] + (bias ? bias[e] : 0.0));
         if (!found || v > next) { next = v; found = 1; }
       }
       margin[t] = found ? last - next : INFINITY;
@@ -130,10 +136,12 @@ ZO_EXPORT void zo_topk_f64(const double *s, const double *bias, int64_t T, int E
 /* Integer results (indices, counts, permutation) are decided by fp32        */
 /* comparisons, so this replica takes the same decisions in the same         */
 /* precision as the device kernel, from the same written rule:               */
-/*   m = max_e l_e;  u_e = zexp(l_e - m)                                     */
+/*   m = max_e l_e over the logits that are numbers (-inf if none);          */
+/*   u_e = zexp(l_e - m)                                                     */
 /*   sum: 32 partials, partial[p] = sum over e = p, p+32, ... (ascending);   */
 /*        then for w = 16,8,4,2,1: partial[p] = partial[p] + partial[p^w]    */
-/*   s_e = u_e / partial[0];  v_e = s_e + b_e;  top-k as in zo_topk_f64;     */
+/*   s_e = u_e / partial[0];  v_e = s_e + b_e;  top-k as in zo_topk_f64      */
+/*   (a NaN v ranks as -inf);                                                */
 /*   gate = scale * s.   Every operation rounds once to fp32.                */
 /* zexp: Cody-Waite reduction with ln2 split into C1 (ln2 truncated to 16    */
 /* significant bits, so n*C1 is exact for |n| < 256) and C2 = fl32(ln2-C1),  */
@@ -174,8 +182,8 @@ ZO_EXPORT void zo_route_replica_f32(const float *logits, const float *bias, int6
     const float *lt = logits + t * E;
     float *u = (float *)malloc(sizeof(float) * (size_t)E);
     unsigned char *taken = (unsigned char *)calloc((size_t)E, 1);
-    float m = lt[0];
-    for (int e = 1; e < E; ++e)
+    float m = -INFINITY;
+    for (int e = 0; e < E; ++e)
       if (lt[e] > m) m = lt[e];
     for (int e = 0; e < E; ++e) u[e] = zo_zexp(lt[e] - m);
     float part[32];
@@ -198,7 +206,7 @@ ZO_EXPORT void zo_route_replica_f32(const float *logits, const float *bias, int6
       float bv = 0.0f;
       for (int e = 0; e < E; ++e) {
         if (taken[e]) continue;
-        float v = u[e] + (bias ? bias[e] : 0.0f);
+        float v = key32(u[e] + (bias ? bias[e] : 0.0f));
         if (best < 0 || v > bv) { best = e; bv = v; }
       }
       taken[best] = 1;

@@ -38,12 +38,18 @@ MUTANTS = [
     ("ties to the higher index", "if (best < 0 || v > bv) { best = e; bv = v; } /* strict",
      "if (best < 0 || v >= bv) { best = e; bv = v; } /* strict", 0),
     ("bias in the gate", "gate[t * k + j] = scale * st[best];", "gate[t * k + j] = scale * bv;", 0),
-    ("bias ignored in selection", "double v = st[e] + (bias ? bias[e] : 0.0);\n        if (best < 0",
-     "double v = st[e];\n        if (best < 0", 0),
+    ("bias ignored in selection", "double v = key64(st[e] + (bias ? bias[e] : 0.0));\n        if (best < 0",
+     "double v = key64(st[e]);\n        if (best < 0", 0),
     ("routed scale dropped", "gate[t * k + j] = scale * st[best];", "gate[t * k + j] = st[best];", 0),
     # fp32 replica
-    ("replica ties to the higher index", "float v = u[e] + (bias ? bias[e] : 0.0f);\n        if (best < 0 || v > bv)",
-     "float v = u[e] + (bias ? bias[e] : 0.0f);\n        if (best < 0 || v >= bv)", 0),
+    ("replica ties to the higher index", "float v = key32(u[e] + (bias ? bias[e] : 0.0f));\n        if (best < 0 || v > bv)",
+     "float v = key32(u[e] + (bias ? bias[e] : 0.0f));\n        if (best < 0 || v >= bv)", 0),
+    ("NaN biased score not ranked last (fp64)", "static double key64(double v) { return v != v ? -INFINITY : v; }",
+     "static double key64(double v) { return v; }", 0),
+    ("NaN biased score not ranked last (replica)", "static float key32(float v) { return v != v ? -INFINITY : v; }",
+     "static float key32(float v) { return v; }", 0),
+    ("replica max starts at the first logit", "float m = -INFINITY;\n    for (int e = 0; e < E; ++e)\n      if (lt[e] > m) m = lt[e];",
+     "float m = lt[0];\n    for (int e = 1; e < E; ++e)\n      if (lt[e] > m) m = lt[e];", 0),
     ("replica sum tree reads its own partial", "nxt[p] = part[p] + part[p ^ w];", "nxt[p] = part[p] + part[p];", 0),
     ("replica max not subtracted", "u[e] = zo_zexp(lt[e] - m);", "u[e] = zo_zexp(lt[e]);", 0),
     ("zexp coefficient 1/3! wrong", "0x1.555556p-3f);  /* 1/3! */", "0x1.555556p-2f);  /* 1/3! */", 0),
@@ -102,7 +108,7 @@ MUTANTS = [
      "dxt[c] += 0.0 * elem(wr, w_dtype, (int64_t)e * d + c) * dl[e];", 0),
     # more routing and integer-stage slips
     ("replica gate from the biased score", "gate[t * k + j] = scale * u[best];", "gate[t * k + j] = scale * bv;", 0),
-    ("replica bias ignored", "float v = u[e] + (bias ? bias[e] : 0.0f);", "float v = u[e];", 0),
+    ("replica bias ignored", "float v = key32(u[e] + (bias ? bias[e] : 0.0f));", "float v = key32(u[e]);", 0),
     ("margin sign", "margin[t] = found ? last - next : INFINITY;", "margin[t] = found ? next - last : INFINITY;", 0),
     ("zero experts left out of the counts", "for (int64_t i = 0; i < T * k; ++i) counts[idx[i]]++;",
      "for (int64_t i = 0; i < T * k; ++i) if (idx[i] < N) counts[idx[i]]++;", 0),

@@ -121,6 +121,66 @@ def test_topk_ties_and_order():
     assert gate[0].tolist() == [2.5 * 0.1, 2.5 * 0.3]
 
 
+def test_topk_nan_scores_rank_below_every_number():
+    """A biased score that is not a number ranks as -inf: the numbers are chosen
+    first, in the usual order, then the NaN experts by ascending id; every pick is
+    a distinct valid id.  Reduces to the finite case with those scores at -1e300."""
+    T, E, k = 6, 24, 6
+    s = oracle.softmax(_rng(21).normal(size=(T, E)))
+    b = _rng(22).uniform(-0.1, 0.1, size=E)
+    b[[3, 7, 8]] = np.nan
+    idx, gate, _ = oracle.topk(s, b, k)
+    b_fin = b.copy()
+    b_fin[[3, 7, 8]] = -1e300
+    ref, _, _ = oracle.topk(s, b_fin, k)
+    np.testing.assert_array_equal(idx, ref)
+    # more NaN experts than finite ones left: the remaining picks are the lowest NaN ids
+    b2 = np.full(E, np.nan)
+    b2[[10, 20]] = 0.0
+    idx2, gate2, _ = oracle.topk(s, b2, 5)
+    for t in range(T):
+        first = sorted([10, 20], key=lambda e: (-s[t, e], e))
+        assert idx2[t].tolist() == first + [0, 1, 2]
+        np.testing.assert_array_equal(gate2[t], s[t, idx2[t]])
+
+
+def test_replica_nan_and_inf_logits_pick_valid_distinct_experts():
+    """fp32 replica on rows that are not all finite: a NaN logit is skipped by the
+    max and gets weight zexp(NaN) = 0, so the row equals the same row with that
+    logit at -inf; a +inf logit makes every score NaN and the picks are experts
+    0..k-1 in order; an all -inf row likewise; a NaN bias ranks its expert last."""
+    E, k = 24, 4
+    l = _rng(23).normal(size=(6, E)).astype(np.float32)
+    l[1, 5] = np.nan
+    l[5, 0] = np.nan
+    l[2, 9] = np.inf
+    l[3, :] = -np.inf
+    l[4, :] = np.nan
+    bias = _rng(24).uniform(-0.1, 0.1, size=E).astype(np.float32)
+    idx, gate, sc = oracle.route_replica_f32(l, bias, k, 1.0, want_scores=True)
+    ref_row = l[1].copy()
+    ref_row[5] = -np.inf
+    i1, g1, s1 = oracle.route_replica_f32(ref_row[None], bias, k, 1.0, want_scores=True)
+    np.testing.assert_array_equal(idx[1], i1[0])
+    np.testing.assert_array_equal(sc[1].view(np.uint32), s1[0].view(np.uint32))
+    assert sc[1, 5] == 0.0 and np.isfinite(sc[1]).all()
+    ref_row = l[5].copy()
+    ref_row[0] = -np.inf
+    i5, _, s5 = oracle.route_replica_f32(ref_row[None], bias, k, 1.0, want_scores=True)
+    np.testing.assert_array_equal(idx[5], i5[0])
+    np.testing.assert_array_equal(sc[5].view(np.uint32), s5[0].view(np.uint32))
+    for t in (2, 3, 4):
+        assert np.isnan(sc[t]).all()
+        assert idx[t].tolist() == [0, 1, 2, 3]
+        assert np.isnan(gate[t]).all()
+    b_nan = bias.copy()
+    b_nan[[0, 1]] = np.nan
+    i_nan, _, _ = oracle.route_replica_f32(l[:1], b_nan, k, 1.0)
+    assert 0 not in i_nan[0] and 1 not in i_nan[0]
+    for t in range(6):
+        assert len(set(idx[t].tolist())) == k and idx[t].min() >= 0 and idx[t].max() < E
+
+
 def test_topk_unbiased_equals_topk_of_logits():
     l = _rng(4).normal(size=(20, 24))
     idx, _, _ = oracle.topk(oracle.softmax(l), None, 6)
