@@ -242,11 +242,15 @@ ZCMOE_API int zcmoe_profile_end(zcmoe_t h, float *ms, int32_t *n_forwards);
  *
  * Its only scratch is one fixed 1 MiB device array inside the library
  * (reserved on every GPU that loads it, until the process exits).  A call needs
- * ceil(T/256) * E * 4 + (E+1) * 8 + (n_ffn+5) * 4 bytes of it; larger requests
- * return ZCMOE_ERANGE with the limit in zcmoe_last_error() (E = 768 allows
- * T <= 87,040; E = 96 allows about 695,000).  The first call on each device
- * looks up the array's device address (with that device current); make that
- * first call before any stream capture.  All calls share the array and it keeps
+ * align8(ceil(T/256) * E * 4) + (E+1) * 8 + (n_ffn+5) * 4 bytes of it; larger
+ * requests return ZCMOE_ERANGE with the largest allowed T in zcmoe_last_error()
+ * (E = 768 with 512 FFN experts allows T <= 86,528; E = 96 with 64 FFN experts
+ * allows T <= 698,112).  routed_scale must be finite (ZCMOE_EINVAL otherwise).
+ * Every argument check happens before anything is enqueued.  The first call on
+ * each device looks up the array's device address (with that device current)
+ * and caches it with the device's current context; a call in a new context (for
+ * example after cudaDeviceReset) looks it up again.  Make a device's first call
+ * before any stream capture.  All calls share the array and it keeps
  * the previous call's contents (whatever must start at zero is cleared on each
  * call), so calls whose executions can overlap on the GPU (for example on two
  * streams) race with each other: order them on one stream or synchronise
@@ -329,9 +333,10 @@ ZCMOE_API int zcmoe_create_ep(const zcmoe_config *cfg, const zcmoe_weights *loca
  * first P rows are the FFN pairs' rows, sorted by expert, then token, then slot) and offsets
  * [n_ffn + 1] device int32 (expert e's rows are [offsets[e], offsets[e+1]); P = offsets[n_ffn]).
  * Keeps the routing for zcmoe_ep_combine and adds the counts to the controller's accumulators.
- * Asynchronous on `stream`. */
+ * dbg (nullable) receives this chunk's routing as zcmoe_forward's does (expert_out is not
+ * written).  Asynchronous on `stream`. */
 ZCMOE_API int zcmoe_ep_dispatch(zcmoe_t h, const void *x, int64_t T, void *xsend, int32_t *offsets,
-                                cudaStream_t stream);
+                                cudaStream_t stream, const zcmoe_debug *dbg);
 
 /* Stage 2.  xrecv [P_recv, d] device bf16: the rows received from the ep_size source ranks in rank
  * order, each source's rows grouped by this rank's local experts in expert order; counts

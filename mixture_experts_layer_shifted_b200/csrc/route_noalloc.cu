@@ -11,10 +11,12 @@
 //
 // The regular path (zcmoe_forward) is unchanged and keeps its scratch in the
 // handle's workspace; this file only adds a second way in.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdio.h>
 
+#include <cmath>
 #include <mutex>
 
 #include "../../include/zcmoe.h"
@@ -37,11 +39,20 @@ int report(int code) {
   return code;
 }
 
-// Device address of g_route_scratch for each device, looked up once per device
-// with that device current (the host-side symbol is only a stand-in and must
-// never be handed to a kernel).
+// Device address of g_route_scratch, looked up with the device current (the
+// host-side symbol is only a stand-in and must never be handed to a kernel) and
+// cached per device together with the context it was looked up in.  A new
+// primary context (after cudaDeviceReset) reloads the module, which can move the
+// array, so a changed context triggers a fresh lookup.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
 std::mutex g_mu;
-void* g_addr[128] = {};
+struct ScratchSlot {
+  CUcontext ctx;
+  void* addr;
+};
+ScratchSlot g_slot[128] = {};
+CtxGetCurrentFn g_ctx_fn = nullptr;
+std::once_flag g_ctx_once;
 
 int scratch_address(void** out) {
   int dev = 0;
@@ -54,21 +65,61 @@ int scratch_address(void** out) {
     snprintf(g_msg, sizeof(g_msg), "device ordinal %d out of range", dev);
     return report(ZCMOE_EUNSUPPORTED);
   }
+  std::call_once(g_ctx_once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  if (!g_ctx_fn) {
+    snprintf(g_msg, sizeof(g_msg), "cuCtxGetCurrent entry point unavailable");
+    return report(ZCMOE_ECUDA);
+  }
+  // Before this thread's first runtime call that needs a context there is none
+  // current yet: the lookup below binds the primary context, then it is read.
+  CUcontext ctx = nullptr;
+  if (g_ctx_fn(&ctx) != CUDA_SUCCESS) ctx = nullptr;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_addr[dev]) {
+  if (!ctx || !g_slot[dev].addr || g_slot[dev].ctx != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_route_scratch);
     if (e != cudaSuccess || !p) {
       snprintf(g_msg, sizeof(g_msg), "cudaGetSymbolAddress(route scratch): %s", cudaGetErrorString(e));
       return report(ZCMOE_ECUDA);
     }
-    g_addr[dev] = p;
+    if (g_ctx_fn(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+    g_slot[dev].ctx = ctx;
+    g_slot[dev].addr = p;
   }
-  *out = g_addr[dev];
+  *out = g_slot[dev].addr;
   return ZCMOE_OK;
 }
 
 size_t align8(size_t x) { return (x + 7) & ~size_t(7); }
+
+// Scratch layout of one call: per-block counts, then (8-byte aligned) the count
+// accumulators and token counter, the row-block offsets and four scalars.
+struct Layout {
+  size_t off_acc, off_mb, off_scal, need;
+};
+Layout layout(int nchunks, int N, int E) {
+  Layout l;
+  l.off_acc = align8((size_t)nchunks * E * sizeof(int32_t));
+  l.off_mb = l.off_acc + (size_t)(E + 1) * sizeof(int64_t);
+  l.off_scal = l.off_mb + (size_t)(N + 1) * sizeof(int32_t);
+  l.need = l.off_scal + 4 * sizeof(int32_t);
+  return l;
+}
+
+// The largest T whose layout fits the array (a multiple of the 256-token block).
+int64_t max_tokens(int N, int E) {
+  const Layout l0 = layout(0, N, E);
+  int64_t nb = (int64_t)((kScratchBytes - l0.need) / ((size_t)E * sizeof(int32_t)));
+  // the 8-byte alignment of the first region adds at most 4 bytes: one step back at most
+  for (int i = 0; i < 2 && nb > 0 && layout((int)nb, N, E).need > kScratchBytes; ++i) --nb;
+  return nb * zc::kChunk;
+}
 
 }  // namespace
 
@@ -84,6 +135,10 @@ int zcmoe_route_noalloc(const float* logits, const float* bias, int64_t T, int32
     snprintf(g_msg, sizeof(g_msg), "need 1 <= n_ffn, n_ffn + n_zero <= 1024, 1 <= top_k <= min(E, 32)");
     return report(ZCMOE_EINVAL);
   }
+  if (!std::isfinite(routed_scale)) {
+    snprintf(g_msg, sizeof(g_msg), "routed_scale must be finite");
+    return report(ZCMOE_EINVAL);
+  }
   if (T < 0 || T > (1 << 20)) {
     snprintf(g_msg, sizeof(g_msg), "T=%lld outside [0, 2^20]", (long long)T);
     return report(ZCMOE_ERANGE);
@@ -95,15 +150,12 @@ int zcmoe_route_noalloc(const float* logits, const float* bias, int64_t T, int32
   }
   const int Ti = (int)T;
   const int nchunks = (Ti + zc::kChunk - 1) / zc::kChunk;
-  const size_t off_acc = align8((size_t)nchunks * E * sizeof(int32_t));
-  const size_t off_mb = off_acc + (size_t)(E + 1) * sizeof(int64_t);
-  const size_t off_scal = off_mb + (size_t)(N + 1) * sizeof(int32_t);
-  const size_t need = off_scal + 4 * sizeof(int32_t);
-  if (need > kScratchBytes) {
+  const Layout lay = layout(nchunks, N, E);
+  if (lay.need > kScratchBytes) {
     snprintf(g_msg, sizeof(g_msg),
-             "T=%d with %d experts needs %zu bytes of routing scratch; the fixed scratch holds %zu "
-             "(at most %zu token blocks of 256 x experts)",
-             Ti, E, need, kScratchBytes, (kScratchBytes - 1024) / ((size_t)E * sizeof(int32_t)));
+             "T=%d with %d experts (%d FFN) needs %zu bytes of routing scratch; the fixed scratch holds %zu, "
+             "enough for T <= %lld",
+             Ti, E, N, lay.need, kScratchBytes, (long long)max_tokens(N, E));
     return report(ZCMOE_ERANGE);
   }
   void* base = nullptr;
@@ -111,9 +163,9 @@ int zcmoe_route_noalloc(const float* logits, const float* bias, int64_t T, int32
   if (rc != ZCMOE_OK) return rc;
   unsigned char* s = static_cast<unsigned char*>(base);
   int32_t* chunk = reinterpret_cast<int32_t*>(s);
-  int64_t* acc = reinterpret_cast<int64_t*>(s + off_acc);
-  int32_t* mb_off = reinterpret_cast<int32_t*>(s + off_mb);
-  int32_t* scal = reinterpret_cast<int32_t*>(s + off_scal);
+  int64_t* acc = reinterpret_cast<int64_t*>(s + lay.off_acc);
+  int32_t* mb_off = reinterpret_cast<int32_t*>(s + lay.off_mb);
+  int32_t* scal = reinterpret_cast<int32_t*>(s + lay.off_scal);
 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

@@ -123,7 +123,7 @@ def test_training_ep_and_host_entry_points_refuse_unknown_handles(zc):
     assert lib.zcmoe_backward(fake, None, None, 1, None, None, None, None, None, None) == E
     assert lib.zcmoe_backward_ex(fake, None, None, 1, None, None, None, None, None, 0, None) == E
     assert lib.zcmoe_save_for_backward(fake, 1) == E
-    assert lib.zcmoe_ep_dispatch(fake, None, 1, None, None, None) == E
+    assert lib.zcmoe_ep_dispatch(fake, None, 1, None, None, None, None) == E
     assert lib.zcmoe_ep_experts(fake, None, None, 0, None, None) == E
     assert lib.zcmoe_ep_combine(fake, None, None, 1, None, None) == E
     assert lib.zcmoe_forward_host_async(fake, None, 1, None, None) == E
@@ -251,3 +251,29 @@ def test_create_checks_quantized_shapes_scale_and_group_on_the_host(zc):
         assert h.value is None
     assert lib.zcmoe_create_ep(ctypes.byref(cfg(dtype=zc.ZCMOE_FP8)), ctypes.byref(w), 0, 2, 0,
                                ctypes.byref(h)) == zc.ZCMOE_EUNSUPPORTED
+
+
+def test_noalloc_refuses_on_the_host_at_its_exact_limits(zc):
+    """zcmoe_route_noalloc checks its arguments before it touches the device, so the
+    refusals run without a GPU.  Its scratch layout is align8(ceil(T/256) E 4) +
+    (E+1) 8 + (N+1) 4 + 16 bytes of a 1 MiB array: T = 86,528 fits at E = 768,
+    N = 512 and the next 256-token block does not; a routed scale that is not a
+    finite number is refused like zcmoe_create refuses it."""
+    lib = zc.lib()
+    p = ctypes.c_void_p(16)
+    def call(T, N=512, Z=256, k=12, scale=1.0):
+        return lib.zcmoe_route_noalloc(p, p, T, N, Z, k, scale, p, p, p, p, p, p, None)
+    def need(T, N, E):
+        nb = -(-T // 256)
+        return ((nb * E * 4 + 7) & ~7) + (E + 1) * 8 + (N + 1) * 4 + 16
+    assert need(86_528, 512, 768) <= 1 << 20 < need(86_529, 512, 768)
+    assert call(86_529) == zc.ZCMOE_ERANGE
+    msg = zc.lib().zcmoe_last_error().decode()
+    assert "86528" in msg and "scratch" in msg, msg
+    assert need(698_112, 64, 96) <= 1 << 20 < need(698_113, 64, 96)
+    assert call(698_113, N=64, Z=32, k=8) == zc.ZCMOE_ERANGE
+    assert "698112" in zc.lib().zcmoe_last_error().decode()
+    for bad in (float("nan"), float("inf"), -float("inf")):
+        assert call(1024, scale=bad) == zc.ZCMOE_EINVAL
+    assert call(-1) == zc.ZCMOE_ERANGE
+    assert call(1024, k=0) == zc.ZCMOE_EINVAL
