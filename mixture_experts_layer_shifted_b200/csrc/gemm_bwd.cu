@@ -578,13 +578,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 template <int SCHED, bool A_MN, bool B_MN, int EPI>
 cudaError_t launch_variant(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& c,
                            const BwdArgs& args, int grid, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_bwd_gemm<SCHED, A_MN, B_MN, EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<EPI>::kSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static SmemAttr attr{};
+  const cudaError_t e = ensure_smem_attr(attr, k_bwd_gemm<SCHED, A_MN, B_MN, EPI>, Cfg<EPI>::kSmem);
+  if (e != cudaSuccess) return e;
   k_bwd_gemm<SCHED, A_MN, B_MN, EPI><<<grid, NUM_THREADS, Cfg<EPI>::kSmem, s>>>(a, b0, b1, c, args);
   return cudaGetLastError();
 }

@@ -484,13 +484,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 template <int MODE, int FMT>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& c,
                         const Fp8Args& args, int grid, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(k_fp8_gemm<MODE, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static SmemAttr attr{};
+  const cudaError_t e = ensure_smem_attr(attr, k_fp8_gemm<MODE, FMT>, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
   k_fp8_gemm<MODE, FMT><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, c, args);
   return cudaGetLastError();
 }

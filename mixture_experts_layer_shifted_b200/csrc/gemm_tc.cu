@@ -403,12 +403,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 template <int MODE>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& c,
                         const TcArgs& args, int grid, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static SmemAttr attr{};
+  const cudaError_t e = ensure_smem_attr(attr, k_tc_gemm<MODE>, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
   k_tc_gemm<MODE><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, c, args);
   return cudaGetLastError();
 }

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace zc {
 
 // Rows of one tensor-core output tile; also the m-block granularity of the
@@ -15,6 +17,28 @@ constexpr int kChunk = 256;
 
 // Copies msg into the calling thread's zcmoe_last_error() slot (zcmoe.cu).
 void set_last_error(const char* msg);
+
+// A kernel's dynamic shared-memory limit is a per-device attribute.  Each kernel
+// keeps one SmemAttr: a bit per device ordinal (0..127), set once the attribute has
+// been raised on that device.  Threads may race to set it; the attribute call is
+// idempotent and the bits are atomic.
+struct SmemAttr {
+  std::atomic<uint64_t> done[2];
+};
+template <typename Kernel>
+cudaError_t ensure_smem_attr(SmemAttr& a, Kernel* kernel, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  const uint64_t bit = 1ull << (dev & 63);
+  std::atomic<uint64_t>& word = a.done[dev >> 6];
+  if (word.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  word.fetch_or(bit, std::memory_order_acq_rel);
+  return cudaSuccess;
+}
 
 // ------------------------------------------------------------- routing (route.cu)
 cudaError_t launch_softmax_topk(const float* logits, const float* bias, int T, int E, int k, float scale, int32_t* idx,
