@@ -71,15 +71,18 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once for the process (call_once makes
+// the first lookup safe when several threads create or run layers at once).
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+  });
   return fn;
 }
 
@@ -608,6 +611,21 @@ static int integer_stage(zcmoe_t h, int Ti, cudaStream_t s) {
   return ZCMOE_OK;
 }
 
+// The routing outputs a caller asked for in `dbg` (all but scores, which the
+// top-k kernel writes itself, and expert_out), copied out of the handle's workspace.
+static int copy_routing_debug(zcmoe_t h, int T, const zcmoe_debug* dbg, cudaStream_t s) {
+  const int E = h->E, N = h->N, k = h->k;
+  if (dbg->logits) ZC_CUDA(cudaMemcpyAsync(dbg->logits, h->logits, (size_t)T * E * 4, cudaMemcpyDeviceToDevice, s));
+  if (dbg->idx) ZC_CUDA(cudaMemcpyAsync(dbg->idx, h->idx, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
+  if (dbg->gate) ZC_CUDA(cudaMemcpyAsync(dbg->gate, h->gate, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
+  if (dbg->counts) ZC_CUDA(cudaMemcpyAsync(dbg->counts, h->counts, (size_t)E * 4, cudaMemcpyDeviceToDevice, s));
+  if (dbg->offsets)
+    ZC_CUDA(cudaMemcpyAsync(dbg->offsets, h->offsets, (size_t)(N + 1) * 4, cudaMemcpyDeviceToDevice, s));
+  if (dbg->perm) ZC_CUDA(cudaMemcpyAsync(dbg->perm, h->perm, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
+  if (dbg->pos) ZC_CUDA(cudaMemcpyAsync(dbg->pos, h->pos, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
+  return ZCMOE_OK;
+}
+
 // The forward pass; with `side`, the dense FFN's two GEMMs are forked onto its
 // stream after the router GEMM and after the down GEMM, and joined back into
 // `s` after the combine.
@@ -789,14 +807,8 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
   if (side) ZC_CUDA(cudaStreamWaitEvent(s, side->dn->ev_join, 0));
 
   if (dbg) {
-    if (dbg->logits) ZC_CUDA(cudaMemcpyAsync(dbg->logits, h->logits, (size_t)T * E * 4, cudaMemcpyDeviceToDevice, s));
-    if (dbg->idx) ZC_CUDA(cudaMemcpyAsync(dbg->idx, h->idx, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
-    if (dbg->gate) ZC_CUDA(cudaMemcpyAsync(dbg->gate, h->gate, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
-    if (dbg->counts) ZC_CUDA(cudaMemcpyAsync(dbg->counts, h->counts, (size_t)E * 4, cudaMemcpyDeviceToDevice, s));
-    if (dbg->offsets)
-      ZC_CUDA(cudaMemcpyAsync(dbg->offsets, h->offsets, (size_t)(N + 1) * 4, cudaMemcpyDeviceToDevice, s));
-    if (dbg->perm) ZC_CUDA(cudaMemcpyAsync(dbg->perm, h->perm, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
-    if (dbg->pos) ZC_CUDA(cudaMemcpyAsync(dbg->pos, h->pos, (size_t)T * k * 4, cudaMemcpyDeviceToDevice, s));
+    const int rc = copy_routing_debug(h, Ti, dbg, s);
+    if (rc != ZCMOE_OK) return rc;
     if (dbg->expert_out && h->fp8)
       ZC_CUDA(zc::launch_unpad_rows(h->ypad, d * 2, h->perm, h->idx, h->offsets, h->mb_off, h->scal, dbg->expert_out,
                                     h->sms, s));
@@ -814,7 +826,8 @@ int zcmoe_forward(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream_t s, 
 
 // ---------------------------------------------------------------- expert parallelism
 
-int zcmoe_ep_dispatch(zcmoe_t h, const void* x, int64_t T, void* xsend, int32_t* offsets, cudaStream_t s) {
+int zcmoe_ep_dispatch(zcmoe_t h, const void* x, int64_t T, void* xsend, int32_t* offsets, cudaStream_t s,
+                      const zcmoe_debug* dbg) {
   g_err[0] = 0;
   if (!is_live(h)) return fail(ZCMOE_EINVAL, "invalid or destroyed handle");
   if (!h->bf16 || h->fp8) return fail(ZCMOE_EUNSUPPORTED, "expert parallelism needs a bf16 layer");
@@ -834,12 +847,13 @@ int zcmoe_ep_dispatch(zcmoe_t h, const void* x, int64_t T, void* xsend, int32_t*
   h->last_T = Ti;
   int rc = router_stage(h, x, Ti, s);
   if (rc != ZCMOE_OK) return rc;
-  ZC_CUDA(zc::launch_softmax_topk(h->logits, h->bias, Ti, h->E, h->k, h->cfg.routed_scale, h->idx, h->gate, nullptr,
-                                  h->sms, s));
+  ZC_CUDA(zc::launch_softmax_topk(h->logits, h->bias, Ti, h->E, h->k, h->cfg.routed_scale, h->idx, h->gate,
+                                  dbg ? dbg->scores : nullptr, h->sms, s));
   rc = integer_stage(h, Ti, s);
   if (rc != ZCMOE_OK) return rc;
   ZC_CUDA(zc::launch_gather_rows(x, h->d * 2, h->perm, h->k, h->scal, xsend, h->sms, s));
   ZC_CUDA(cudaMemcpyAsync(offsets, h->offsets, (size_t)(h->N + 1) * sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
+  if (dbg) return copy_routing_debug(h, Ti, dbg, s);
   return ZCMOE_OK;
 }
 

@@ -6,17 +6,21 @@ are partitioned by expert over an EP group, without tensor parallelism; the MoE
 layer is split into two chunks along the token dimension so one chunk's
 dispatch/combine traffic overlaps the other's computation.
 
-Rank r holds FFN experts [r * n_local, (r + 1) * n_local).  Per chunk of tokens:
-  1. dispatch: routing on the token's rank; the FFN pairs' rows in expert order, so
-     the rows for rank r are one contiguous block (zero-expert picks stay local);
-  2. exchange of the per-expert row counts, then of the rows (all-to-all);
-  3. the local experts on the received rows (source-major rows, regrouped by
-     expert inside the library);
-  4. exchange of the outputs back (the reverse all-to-all);
-  5. combine on the token's rank.
-The counts must reach the host (the all-to-all split sizes), so each chunk syncs
-twice; with two chunks, chunk 1's row exchange runs while chunk 0's experts
-compute, and chunk 0's return exchange while chunk 1's experts compute.
+Rank r holds FFN experts [r * n_local, (r + 1) * n_local).  A forward:
+  1. dispatch of every chunk: routing on the token's rank; the FFN pairs' rows in
+     expert order, so the rows for rank r are one contiguous block (zero-expert
+     picks stay local);
+  2. ONE exchange of all chunks' per-expert row counts, read on the host with one
+     synchronisation (the all-to-all split sizes);
+  3. per chunk: the row exchange (asynchronous), the local experts on the received
+     rows (source-major rows, regrouped by expert inside the library), and the
+     return exchange (asynchronous), so chunk 1's rows move while chunk 0's experts
+     compute and chunk 0's outputs return while chunk 1's experts compute;
+  4. combine of every chunk on the token's rank.
+The shortcut-connected dense FFN (same page, 二 part 2 "快捷連接 MoE": the dense
+block's FFN runs while the MoE layer's dispatch and combine traffic is in flight)
+can be handed to forward(): it is enqueued on its own stream right after the
+dispatches, so it overlaps the exchanges and the expert GEMMs.
 
 The stages are an object with dispatch / experts / combine (CudaStages: the C
 ABI on device tensors) and the exchanges a communicator with all_to_all
@@ -66,14 +70,15 @@ class CudaStages:
         self.layer = layer
         self.shape = layer.shape
 
-    def dispatch(self, x):
-        """-> (xsend [T*k, d], offsets as a host int64 array [n_ffn + 1]); syncs on the offsets."""
+    def dispatch(self, x, offsets, debug: dict | None = None):
+        """-> xsend [T*k, d]; fills offsets ([n_ffn + 1] int32 on the device); no host sync.
+        debug: zcmoe_debug field names -> device tensors that receive this chunk's routing."""
         T, s = x.shape[0], self.shape
         xsend = torch.empty((max(T * s.top_k, 1), s.d), dtype=x.dtype, device=x.device)
-        off = torch.empty((s.n_ffn + 1,), dtype=torch.int32, device=x.device)
+        dbg = zcmoe.zcmoe_debug(**{k_: v.data_ptr() for k_, v in debug.items()}) if debug else None
         zcmoe.zcmoe_ep_dispatch(self.layer.h, ctypes.c_void_p(x.data_ptr()), T, ctypes.c_void_p(xsend.data_ptr()),
-                                ctypes.c_void_p(off.data_ptr()))
-        return xsend, off.cpu().numpy().astype(np.int64)
+                                ctypes.c_void_p(offsets.data_ptr()), dbg=dbg)
+        return xsend
 
     def experts(self, xrecv, counts):
         """counts [ep_size, n_local] host ints -> yrecv (rows in xrecv's order)."""
@@ -97,18 +102,29 @@ class _Chunk:
         self.x, self.stages = x, stages
 
 
-def _exchange_counts(comm, send_counts, device):
-    R, NL = send_counts.shape
-    sc = torch.as_tensor(send_counts.reshape(-1), dtype=torch.int32).to(device)
-    rc = torch.empty_like(sc)
-    comm.all_to_all(rc, sc, [NL] * R, [NL] * R)
-    return rc.cpu().numpy().astype(np.int64).reshape(R, NL)
+def _exchange_counts(comm, offsets, R, NL):
+    """offsets: [nck, n_ffn + 1] int32 on the device (each chunk's dispatch offsets).
+    One all-to-all of every chunk's per-expert counts, then one host read of both sides:
+    -> (send_counts [nck, R, NL], recv_counts [nck, R, NL], P [nck]) as host int64."""
+    nck = offsets.shape[0]
+    send = (offsets[:, 1:] - offsets[:, :-1]).reshape(nck, R, NL).transpose(0, 1).contiguous()  # [dst, chunk, e]
+    recv = torch.empty_like(send)                                                                # [src, chunk, e]
+    comm.all_to_all(recv.view(-1), send.view(-1), [nck * NL] * R, [nck * NL] * R)
+    both = torch.cat([send.view(-1), recv.view(-1)]).cpu().numpy().astype(np.int64)
+    half = R * nck * NL
+    send_h = both[:half].reshape(R, nck, NL).transpose(1, 0, 2)
+    recv_h = both[half:].reshape(R, nck, NL).transpose(1, 0, 2)
+    return send_h, recv_h, send_h.sum(axis=(1, 2))
 
 
-def ep_forward(stages_per_chunk, comm, x, n_ffn: int):
+def ep_forward(stages_per_chunk, comm, x, n_ffn: int, dense=None, x_dense=None, y_dense=None, dense_stream=None,
+               debug=None):
     """y = layer(x) with the FFN experts spread over comm's ranks.  stages_per_chunk: one
     stage object per chunk (each keeps its chunk's routing until its combine); x is cut into
-    that many contiguous token chunks."""
+    that many contiguous token chunks.  dense (optional, a ZcDense, CUDA only): y_dense =
+    dense(x_dense) is enqueued on dense_stream after the dispatches and joined before
+    returning, so it runs while the exchanges and the expert GEMMs are in flight.  debug
+    (optional list, one dict per chunk): routing outputs of each chunk."""
     R = comm.size
     if n_ffn % R:
         raise ValueError("n_ffn must be a multiple of the group size")
@@ -117,30 +133,41 @@ def ep_forward(stages_per_chunk, comm, x, n_ffn: int):
     T = x.shape[0]
     bounds = [T * i // nck for i in range(nck + 1)]
     chunks = [_Chunk(x[bounds[i]:bounds[i + 1]], st) for i, st in enumerate(stages_per_chunk)]
-    # 1-2: dispatch and the row exchange, chunk after chunk (each row exchange asynchronous)
-    for c in chunks:
-        c.xsend, off = c.stages.dispatch(c.x)
-        c.send_counts = np.diff(off).reshape(R, NL)
-        c.send_rows = c.send_counts.sum(1)
-        c.P = int(off[-1])
-        c.recv_counts = _exchange_counts(comm, c.send_counts, c.x.device)
+    # 1: every chunk's routing and row gather
+    offs = torch.empty((nck, n_ffn + 1), dtype=torch.int32, device=x.device)
+    for i, c in enumerate(chunks):
+        c.xsend = c.stages.dispatch(c.x, offs[i], debug[i] if debug else None)
+    # the dense FFN on its own stream, concurrent with everything below
+    if dense is not None:
+        main = torch.cuda.current_stream(x.device)
+        dense_stream.wait_stream(main)
+        y_dense = dense.forward(x_dense, y_dense, stream=dense_stream)
+    # 2: one count exchange, one host sync
+    send_counts, recv_counts, P = _exchange_counts(comm, offs, R, NL)
+    for i, c in enumerate(chunks):
+        c.send_rows = send_counts[i].sum(1)
+        c.recv_counts = recv_counts[i]
         c.recv_rows = c.recv_counts.sum(1)
+        c.P = int(P[i])
         c.xrecv = c.x.new_empty((int(c.recv_rows.sum()), c.x.shape[1]))
         c.work = comm.all_to_all(c.xrecv, c.xsend[:c.P], c.recv_rows.tolist(), c.send_rows.tolist(), async_op=True)
-    # 3-4: the local experts, each chunk's return exchange asynchronous
+    # 3: the local experts, each chunk's return exchange asynchronous
     for c in chunks:
         if c.work is not None:
             c.work.wait()
         c.yrecv = c.stages.experts(c.xrecv, c.recv_counts)
         c.yback = c.x.new_empty((c.P, c.x.shape[1]))
         c.work = comm.all_to_all(c.yback, c.yrecv, c.send_rows.tolist(), c.recv_rows.tolist(), async_op=True)
-    # 5: combine
+    # 4: combine
     ys = []
     for c in chunks:
         if c.work is not None:
             c.work.wait()
         ys.append(c.stages.combine(c.x, c.yback))
-    return ys[0] if nck == 1 else torch.cat(ys, 0)
+    if dense is not None:
+        main.wait_stream(dense_stream)
+    y = ys[0] if nck == 1 else torch.cat(ys, 0)
+    return (y, y_dense) if dense is not None else y
 
 
 class EpMoE:
@@ -161,9 +188,24 @@ class EpMoE:
                                    init_bias=init_bias, logit_offset=logit_offset, ep_rank=self.comm.rank, ep_size=R,
                                    max_recv_rows=cap) for _ in range(chunks)]
         self.stages = [CudaStages(layer) for layer in self.layers]
+        self.dense_stream = None
 
-    def forward(self, x):
-        return ep_forward(self.stages, self.comm, x, self.shape.n_ffn)
+    def forward(self, x, dense=None, x_dense=None, y_dense=None, debug=None):
+        """y, or (y, y_dense) when a dense FFN (ZcDense) is given: it runs on its own stream
+        while this layer's exchanges and expert GEMMs are in flight (x_dense defaults to x).
+        debug: a list of one dict per chunk (zcmoe_debug field names -> device tensors)."""
+        if dense is not None:
+            if x_dense is None:
+                x_dense = x
+            if self.dense_stream is None:
+                self.dense_stream = torch.cuda.Stream(device=x.device)
+        return ep_forward(self.stages, self.comm, x, self.shape.n_ffn, dense=dense, x_dense=x_dense,
+                          y_dense=y_dense, dense_stream=self.dense_stream, debug=debug)
+
+    def chunk_bounds(self, T):
+        """The token ranges of the chunks a forward of T tokens is cut into."""
+        n = len(self.stages)
+        return [(T * i // n, T * (i + 1) // n) for i in range(n)]
 
     def controller_step(self, all_reduce=None, **gains):
         """One bias-controller step shared by the chunk handles and the group: the

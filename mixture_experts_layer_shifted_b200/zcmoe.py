@@ -121,7 +121,7 @@ def lib():
         L.zcmoe_save_for_backward.argtypes = [vp, ctypes.c_int32]
         L.zcmoe_create_ep.argtypes = [ctypes.POINTER(zcmoe_config), ctypes.POINTER(zcmoe_weights), ctypes.c_int32,
                                       ctypes.c_int32, i64, ctypes.POINTER(vp)]
-        L.zcmoe_ep_dispatch.argtypes = [vp, vp, i64, vp, vp, vp]
+        L.zcmoe_ep_dispatch.argtypes = [vp, vp, i64, vp, vp, vp, ctypes.POINTER(zcmoe_debug)]
         L.zcmoe_ep_experts.argtypes = [vp, vp, vp, i64, vp, vp]
         L.zcmoe_ep_combine.argtypes = [vp, vp, vp, i64, vp, vp]
         L.zcmoe_dense_destroy.argtypes = [vp]
@@ -184,8 +184,9 @@ def zcmoe_create_ep(cfg: zcmoe_config, w: zcmoe_weights, ep_rank: int, ep_size: 
     return h
 
 
-def zcmoe_ep_dispatch(h, x_ptr, T, xsend_ptr, offsets_ptr, stream=None):
-    _check(lib().zcmoe_ep_dispatch(h, x_ptr, T, xsend_ptr, offsets_ptr, _stream(stream)), "zcmoe_ep_dispatch")
+def zcmoe_ep_dispatch(h, x_ptr, T, xsend_ptr, offsets_ptr, stream=None, dbg=None):
+    _check(lib().zcmoe_ep_dispatch(h, x_ptr, T, xsend_ptr, offsets_ptr, _stream(stream),
+                                   ctypes.byref(dbg) if dbg is not None else None), "zcmoe_ep_dispatch")
 
 
 def zcmoe_ep_experts(h, xrecv_ptr, counts_host_ptr, P_recv, yrecv_ptr, stream=None):

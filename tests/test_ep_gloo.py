@@ -47,7 +47,7 @@ class OracleStages:
         self.wr, self.wg, self.wu, self.wd, self.bias = weights
         self.nl = N // size
 
-    def dispatch(self, x):
+    def dispatch(self, x, offsets_out, debug=None):
         xn = x.numpy()
         T = xn.shape[0]
         self.idx, self.gate = _route(xn, self.wr, self.bias) if T else (np.zeros((0, K), np.int32),
@@ -55,7 +55,8 @@ class OracleStages:
         _, offsets, perm, pos = oracle.integer_stage(self.idx, N, E)
         self.pos = pos
         xsend = torch.from_numpy(np.ascontiguousarray(xn[perm // K])) if T else torch.zeros((0, D))
-        return xsend, offsets.astype(np.int64)
+        offsets_out.copy_(torch.from_numpy(offsets.astype(np.int32)))
+        return xsend
 
     def experts(self, xrecv, counts):
         # rows from the sources in rank order, each source's rows grouped by local expert
