@@ -9,19 +9,34 @@
 // expert is 2048 wide on a 6144 hidden size; the per-expert GEMMs run as one
 // grouped GEMM, 五 訓練基礎設施 "優化的分組GEMM", 六 推理與部署 "MoEGEMM".)
 //
-// Tile: 128 rows (tokens) x 256 columns x 64-deep k-blocks, bf16 operands in
-// 128-byte-swizzled K-major shared-memory tiles, fp32 accumulators in TMEM
-// (two 256-column buffers, so the epilogue of one tile overlaps the MMAs of
-// the next).  For gate/up the 256 B rows are 128 rows of W_g followed by the
-// same 128 rows of W_u, so each thread of the epilogue holds the gate and up
+// Row blocks of 128 tokens x 256 columns x 64-deep k-blocks, bf16 operands in
+// 128-byte-swizzled K-major shared-memory tiles, fp32 accumulators in TMEM (two
+// 256-column slots).  For gate/up the 256 B rows are 128 rows of W_g followed by
+// the same 128 rows of W_u, so each thread of the epilogue holds the gate and up
 // value of the same (row, column) and applies SwiGLU before one bf16 rounding.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
-// issues the MMAs (one thread), warps 2..5 drain TMEM (thread = row).
-// Tiles are walked expert-major, then column tile, then row block, so the row
-// blocks that share a weight tile run on neighbouring SMs at the same time and
-// a weight tile is fetched from HBM about once; an expert's activation rows
-// stay in L2 across its column tiles.
+// Work unit of the grouped modes: one weight tile (an expert's 256 B rows) and
+// up to TWO of that expert's row blocks.  Each k-block stages the weight tile
+// once and both row blocks' activations, and the MMAs of both row blocks read
+// the same staged weights, so every SM keeps twice the distinct weight bytes in
+// flight that one row block per tile would (the expert GEMMs stream 38.6 GB of
+// weights at about 255 tokens per expert, where HBM latency, not the tensor
+// pipe, paced the one-row-block schedule).  A pair fills both TMEM slots; a
+// single row block (an expert's odd last block, or every router tile) takes one,
+// so consecutive singles still overlap the epilogue of one with the MMAs of the
+// next.
+//
+// Scheduling: units are numbered expert-major, then column tile, then row-block
+// pair, and handed out by an atomic counter (pairs cost twice a single, and a
+// static round-robin over the mixed costs left some SMs with 20% more work).
+// Neighbouring units share weight tiles through L2, and an expert's activation
+// rows stay in L2 across its column tiles.  The unit ids travel from the
+// producer to the MMA and epilogue warps through a small ring in shared memory.
+//
+// Warp roles (320 threads): warp 0 takes units and issues TMA loads, warp 1 owns
+// TMEM and issues the MMAs (one elected lane of the converged warp), warps 2..9
+// drain TMEM: two warps per TMEM sub-partition, thread = row, each warp of a
+// pair taking half the columns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -33,60 +48,73 @@
 namespace zc {
 namespace {
 
-constexpr int BM = kBM, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = kBM, BN = 256, BK = 64;
 constexpr uint32_t A_BYTES = BM * BK * 2;
 constexpr uint32_t B_BYTES = BN * BK * 2;
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NUM_THREADS = 192;
+constexpr int EPI_WARPS = 8;
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 2 * BN;
-constexpr uint32_t STG_BYTES = 32 * 128;  // down epilogue: a 32-row x 64-column bf16 box per warp and buffer
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 4 * 2 * STG_BYTES + 256;
+constexpr uint32_t STG_BYTES = 32 * 128;  // down epilogue: a 32-row x 64-column bf16 box per warp
+constexpr int RING = 4;                   // unit ids in flight from the producer to the consumers
 
-struct Tile {
-  int a_row;       // first A row of the tile
-  int rows_valid;  // rows of the tile that belong to it
-  int b_row;       // first B row
-  int n_blk;       // output column tile
-  int p_row;       // grouped modes: the tile's first row in the padded layout (128 (mb_off[g] + row block))
+template <int MODE, bool PAIR>
+struct Cfg {
+  static constexpr bool kPair = PAIR && MODE != kRouter;  // stage two row blocks per weight tile
+  static constexpr int kStages = kPair ? 3 : 4;
+  static constexpr uint32_t kStageBytes = B_BYTES + (kPair ? 2 : 1) * A_BYTES;
+  // stages | staging boxes | barriers, the unit ring and the TMEM address
+  static constexpr int kSmem = 1024 + kStages * kStageBytes + EPI_WARPS * STG_BYTES + 512;
 };
 
-template <int MODE>
-__device__ __forceinline__ int total_tiles(const TcArgs& a) {
+struct Unit {
+  int a_row;    // first A row of the first row block
+  int rows[2];  // valid rows of each row block (rows[1] = 0: one row block)
+  int b_row;    // first B row
+  int n_blk;    // output column tile
+  int p_row;    // grouped modes: padded-layout row of the first row block (128 (mb_off[g] + block))
+};
+
+template <int MODE, bool PAIR>
+__device__ __forceinline__ int total_units(const TcArgs& a) {
   if (MODE == kRouter) return ((a.M + BM - 1) / BM) * a.nblocks;
-  return a.mb_off[a.ngroups] * a.nblocks;
+  return (PAIR ? a.sp_off[a.ngroups] : a.mb_off[a.ngroups]) * a.nblocks;
 }
 
-template <int MODE>
-__device__ __forceinline__ Tile decode_tile(const TcArgs& a, int t) {
-  Tile ti;
+template <int MODE, bool PAIR>
+__device__ __forceinline__ Unit decode_unit(const TcArgs& a, int t) {
+  Unit u;
   if (MODE == kRouter) {
     const int m_blk = t / a.nblocks;
-    ti.n_blk = t - m_blk * a.nblocks;
-    ti.a_row = m_blk * BM;
-    ti.rows_valid = min(BM, a.M - ti.a_row);
-    ti.b_row = ti.n_blk * BN;
-    ti.p_row = ti.a_row;
-    return ti;
+    u.n_blk = t - m_blk * a.nblocks;
+    u.a_row = m_blk * BM;
+    u.rows[0] = min(BM, a.M - u.a_row);
+    u.rows[1] = 0;
+    u.b_row = u.n_blk * BN;
+    u.p_row = u.a_row;
+    return u;
   }
-  // largest expert g with mb_off[g] * nblocks <= t (it has at least one row block)
+  // units per expert and column tile: its row-block pairs (PAIR) or its row blocks; the
+  // largest expert g with off[g] * nblocks <= t (it has at least one unit)
+  const int32_t* off = PAIR ? a.sp_off : a.mb_off;
   int lo = 0, hi = a.ngroups - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (a.mb_off[mid] * a.nblocks <= t) lo = mid;
+    if (off[mid] * a.nblocks <= t) lo = mid;
     else hi = mid - 1;
   }
   const int g = lo;
-  const int mb0 = a.mb_off[g];
-  const int nmb = a.mb_off[g + 1] - mb0;
-  const int local = t - mb0 * a.nblocks;
-  ti.n_blk = local / nmb;
-  const int m_blk = local - ti.n_blk * nmb;
-  const int r0 = a.row_off[g];
-  ti.a_row = r0 + m_blk * BM;
-  ti.rows_valid = min(BM, a.row_off[g + 1] - ti.a_row);
-  ti.p_row = (mb0 + m_blk) * BM;
-  ti.b_row = g * a.b_rows_per_group + ti.n_blk * (MODE == kGateUp ? BN / 2 : BN);
-  return ti;
+  const int u0 = off[g];
+  const int nu = off[g + 1] - u0;
+  const int local = t - u0 * a.nblocks;
+  u.n_blk = local / nu;
+  const int m0 = (PAIR ? 2 : 1) * (local - u.n_blk * nu);
+  const int end = a.row_off[g + 1];
+  u.a_row = a.row_off[g] + m0 * BM;
+  u.rows[0] = min(BM, end - u.a_row);
+  u.rows[1] = PAIR ? max(0, min(BM, end - u.a_row - BM)) : 0;
+  u.p_row = (a.mb_off[g] + m0) * BM;
+  u.b_row = g * a.b_rows_per_group + u.n_blk * (MODE == kGateUp ? BN / 2 : BN);
+  return u;
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
@@ -100,7 +128,7 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, const void* 
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
@@ -109,21 +137,161 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// The whole warp waits (every lane polls the barrier, bounded); true only if every lane saw it.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int* err, int code) {
+  const bool ok = mbar_wait(bar, parity, err, code);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Epilogue of one row block: warp `quarter` drains TMEM lanes [32 quarter, 32 quarter + 32)
+// of the accumulator at tbase; `half` selects which half of the columns this warp takes.
 template <int MODE>
+__device__ __forceinline__ void drain_rows(const TcArgs& args, const CUtensorMap* tmC, uint32_t tbase, int quarter,
+                                           int half, int lane, int a_row, int rows_valid, int p_row, int n_blk,
+                                           uint8_t* stg) {
+  // an M = 64 accumulator holds row 16 quarter + lane in lanes 0..15 of the quarter
+  const bool m64 = rows_valid <= 64;
+  const int row_in_tile = m64 ? (lane < 16 ? quarter * 16 + lane : BM) : quarter * 32 + lane;
+  const bool row_ok = row_in_tile < rows_valid;
+  const int64_t grow = (int64_t)a_row + row_in_tile;
+  if (MODE == kGateUp) {
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
+#pragma unroll 1
+    for (int c = half * (BN / 4); c < (half + 1) * (BN / 4); c += 32) {
+      uint32_t g[32], u[32];
+      tmem_ld32(tbase + c, g);
+      tmem_ld32(tbase + BN / 2 + c, u);
+      tc_wait_ld();
+      const int col0 = n_blk * (BN / 2) + c;
+      if (row_ok && col0 < args.n_out) {
+        uint4* dst = reinterpret_cast<uint4*>(out + grow * args.ldo + col0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 v;
+          v.x = pack_bf16(silu_mul(__uint_as_float(g[8 * q + 0]), __uint_as_float(u[8 * q + 0])),
+                          silu_mul(__uint_as_float(g[8 * q + 1]), __uint_as_float(u[8 * q + 1])));
+          v.y = pack_bf16(silu_mul(__uint_as_float(g[8 * q + 2]), __uint_as_float(u[8 * q + 2])),
+                          silu_mul(__uint_as_float(g[8 * q + 3]), __uint_as_float(u[8 * q + 3])));
+          v.z = pack_bf16(silu_mul(__uint_as_float(g[8 * q + 4]), __uint_as_float(u[8 * q + 4])),
+                          silu_mul(__uint_as_float(g[8 * q + 5]), __uint_as_float(u[8 * q + 5])));
+          v.w = pack_bf16(silu_mul(__uint_as_float(g[8 * q + 6]), __uint_as_float(u[8 * q + 6])),
+                          silu_mul(__uint_as_float(g[8 * q + 7]), __uint_as_float(u[8 * q + 7])));
+          dst[q] = v;
+        }
+        if (args.gu_save) {
+          // training: the pre-activations for the backward, in the padded row layout
+          __nv_bfloat16* gs =
+              static_cast<__nv_bfloat16*>(args.gu_save) + ((int64_t)p_row + row_in_tile) * 2 * args.n_out + col0;
+          uint4* gdst = reinterpret_cast<uint4*>(gs);
+          uint4* udst = reinterpret_cast<uint4*>(gs + args.n_out);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            gdst[q] = make_uint4(pack_bf16(__uint_as_float(g[8 * q + 0]), __uint_as_float(g[8 * q + 1])),
+                                 pack_bf16(__uint_as_float(g[8 * q + 2]), __uint_as_float(g[8 * q + 3])),
+                                 pack_bf16(__uint_as_float(g[8 * q + 4]), __uint_as_float(g[8 * q + 5])),
+                                 pack_bf16(__uint_as_float(g[8 * q + 6]), __uint_as_float(g[8 * q + 7])));
+            udst[q] = make_uint4(pack_bf16(__uint_as_float(u[8 * q + 0]), __uint_as_float(u[8 * q + 1])),
+                                 pack_bf16(__uint_as_float(u[8 * q + 2]), __uint_as_float(u[8 * q + 3])),
+                                 pack_bf16(__uint_as_float(u[8 * q + 4]), __uint_as_float(u[8 * q + 5])),
+                                 pack_bf16(__uint_as_float(u[8 * q + 6]), __uint_as_float(u[8 * q + 7])));
+          }
+        }
+      }
+    }
+  } else if (MODE == kDown && !m64 && quarter * 32 + 32 <= rows_valid) {
+    // 32 valid rows: coalesced TMA stores of 32 x 64 boxes staged in shared memory (thread
+    // = row, its 64 bf16 values as eight 16-byte chunks, chunk j at j ^ (row & 7): the
+    // 128-byte swizzle of the output tensor map)
+    const int grow0 = a_row + quarter * 32;
+#pragma unroll 1
+    for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 64) {
+      uint32_t r0[32], r1[32];
+      tmem_ld32(tbase + c, r0);
+      tmem_ld32(tbase + c + 32, r1);
+      tc_wait_ld();
+      const int col0 = n_blk * BN + c;
+      if (col0 >= args.n_out) continue;  // the same for the whole warp
+      if (lane == 0) bulk_wait_read_0();  // the previous store of this warp has read the buffer
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t* v = j < 4 ? r0 + 8 * j : r1 + 8 * (j - 4);
+        *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+            make_uint4(pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                       pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                       pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                       pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7])));
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmC, stg, col0, grow0);
+        bulk_commit();
+      }
+    }
+  } else if (MODE == kDown) {
+    // a partly valid row group (the rows past it belong to the next expert): row stores
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
+#pragma unroll 1
+    for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+      uint32_t r[32];
+      tmem_ld32(tbase + c, r);
+      tc_wait_ld();
+      const int col0 = n_blk * BN + c;
+      if (row_ok && col0 < args.n_out) {
+        uint4* dst = reinterpret_cast<uint4*>(out + grow * args.ldo + col0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 v;
+          v.x = pack_bf16(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
+          v.y = pack_bf16(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
+          v.z = pack_bf16(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
+          v.w = pack_bf16(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
+          dst[q] = v;
+        }
+      }
+    }
+  } else {
+    float* out = static_cast<float*>(args.out);
+#pragma unroll 1
+    for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+      uint32_t r[32];
+      tmem_ld32(tbase + c, r);
+      tc_wait_ld();
+      const int col0 = n_blk * BN + c;
+      if (row_ok && col0 < args.n_out) {
+        float* dst = out + grow * args.ldo + col0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (col0 + i < args.n_out) {
+            const float add = args.col_add ? args.col_add[col0 + i] : 0.0f;
+            dst[i] = __fadd_rn(__uint_as_float(r[i]), add);
+          }
+        }
+      }
+    }
+  }
+}
+
+template <int MODE, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
               const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmC, const TcArgs args) {
+  using C = Cfg<MODE, PAIR>;
+  constexpr int STAGES = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_BYTES;
-  uint8_t* sStg = sB + STAGES * B_BYTES;  // 1024-aligned: [warp quarter][buffer] of STG_BYTES
-  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + 4 * 2 * STG_BYTES);
+  // stage s: [B: 256 x 64][A0: 128 x 64][A1: 128 x 64 (pairs only)], each 1024-aligned
+  uint8_t* sStg = smem + STAGES * C::kStageBytes;  // [epilogue warp] of STG_BYTES
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + EPI_WARPS * STG_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint64_t* done = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* ufull = tempty + 2;
+  uint64_t* uempty = ufull + RING;
+  uint64_t* done = uempty + RING;
+  volatile int* ring = reinterpret_cast<volatile int*>(done + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(ring) + RING);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* err = args.err;
@@ -135,7 +303,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 32 * EPI_WARPS);
+    }
+    for (int r = 0; r < RING; ++r) {
+      mbar_init(&ufull[r], 1);
+      mbar_init(&uempty[r], 1 + EPI_WARPS);  // the MMA warp and every epilogue warp read the id
     }
     mbar_init(done, 1);
     fence_barrier_init();
@@ -154,33 +326,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int total = total_tiles<MODE>(args);
+  const int total = total_units<MODE, C::kPair>(args);
   const int num_k = (args.K + BK - 1) / BK;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------------------------------------------------------- TMA producer
+      // ---------------------------------------------------------------- scheduler + TMA producer
       int stage = 0;
       uint32_t phase = 0;
       int fills = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile ti = decode_tile<MODE>(args, t);
+      for (int i = 0; i <= total && ok; ++i) {
+        const int rs = i % RING;
+        if (!mbar_wait(&uempty[rs], ((i / RING) & 1) ^ 1u, err, 10)) break;
+        int t = atomicAdd(args.sched, 1);
+        if (t >= total) t = -1;
+        ring[rs] = t;
+        mbar_arrive(&ufull[rs]);
+        if (t < 0) break;
+        const Unit u = decode_unit<MODE, C::kPair>(args, t);
+        const bool two = C::kPair && u.rows[1] > 0;
+        const uint32_t bytes = B_BYTES + (two ? 2u : 1u) * A_BYTES;
         for (int kb = 0; kb < num_k; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, err, 1)) {
             ok = false;
             break;
           }
-          uint8_t* a_dst = sA + stage * A_BYTES;
-          uint8_t* b_dst = sB + stage * B_BYTES;
-          mbar_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_2d(a_dst, &tmA, kb * BK, ti.a_row, &full[stage]);
+          uint8_t* b_dst = smem + stage * C::kStageBytes;
+          uint8_t* a_dst = b_dst + B_BYTES;
+          mbar_expect_tx(&full[stage], bytes);
           if (MODE == kGateUp) {
-            tma_load_2d(b_dst, &tmB0, kb * BK, ti.b_row, &full[stage]);
-            tma_load_2d(b_dst + B_BYTES / 2, &tmB1, kb * BK, ti.b_row, &full[stage]);
+            tma_load_2d(b_dst, &tmB0, kb * BK, u.b_row, &full[stage]);
+            tma_load_2d(b_dst + B_BYTES / 2, &tmB1, kb * BK, u.b_row, &full[stage]);
           } else {
-            tma_load_2d(b_dst, &tmB0, kb * BK, ti.b_row, &full[stage]);
+            tma_load_2d(b_dst, &tmB0, kb * BK, u.b_row, &full[stage]);
           }
+          tma_load_2d(a_dst, &tmA, kb * BK, u.a_row, &full[stage]);
+          if (two) tma_load_2d(a_dst + A_BYTES, &tmA, kb * BK, u.a_row + BM, &full[stage]);
           ++fills;
           if (++stage == STAGES) {
             stage = 0;
@@ -200,194 +382,106 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc128 = idesc_bf16_f32(BM, BN);
-      constexpr uint32_t idesc64 = idesc_bf16_f32(64, BN);
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, err, 2)) break;
+    // ---------------------------------------------------------------- MMA issuer (converged warp)
+    constexpr uint32_t idesc128 = idesc_bf16_f32(BM, BN);
+    constexpr uint32_t idesc64 = idesc_bf16_f32(64, BN);
+    int stage = 0;
+    uint32_t phase = 0;
+    int slot = 0;              // TMEM slot of the next row block
+    uint32_t uses[2] = {0, 0};  // row blocks each slot has held so far
+    bool ok = true;
+    for (int i = 0; i <= total && ok; ++i) {
+      const int rs = i % RING;
+      if (!warp_wait(&ufull[rs], (i / RING) & 1, err, 11)) break;
+      const int t = ring[rs];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&uempty[rs]);
+      if (t < 0) break;
+      const Unit u = decode_unit<MODE, C::kPair>(args, t);
+      const bool two = C::kPair && u.rows[1] > 0;
+      const int s0 = slot, s1 = slot ^ 1;
+      // each slot's accumulator must have been drained by the epilogue of its previous use
+      if (!warp_wait(&tempty[s0], (uses[s0] & 1) ^ 1u, err, 2)) break;
+      if (two && !warp_wait(&tempty[s1], (uses[s1] & 1) ^ 1u, err, 2)) break;
+      tc_fence_after();
+      const uint32_t d0 = tmem_base + (uint32_t)(s0 * BN), d1 = tmem_base + (uint32_t)(s1 * BN);
+      // a row block of at most 64 valid rows runs M = 64 MMAs (about half the energy of
+      // M = 128); its rows land in TMEM lanes 32q + (0..15), q = 0..3
+      const uint32_t id0 = u.rows[0] <= 64 ? idesc64 : idesc128;
+      const uint32_t id1 = u.rows[1] <= 64 ? idesc64 : idesc128;
+      for (int kb = 0; kb < num_k; ++kb) {
+        if (!warp_wait(&full[stage], phase, err, 3)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        // a tile of at most 64 valid rows (an expert's last row block) runs M = 64 MMAs: the
-        // same issue time as M = 128, about half the energy (a power-capped GPU keeps a higher
-        // clock); its rows land in TMEM lanes 32q + (0..15), q = 0..3
-        const uint32_t idesc = decode_tile<MODE>(args, t).rows_valid <= 64 ? idesc64 : idesc128;
-        for (int kb = 0; kb < num_k; ++kb) {
-          if (!mbar_wait(&full[stage], phase, err, 3)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
+        if (elect_one()) {
+          const uint32_t b_addr = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t a_addr = b_addr + B_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            tc_mma_f16(d_tmem, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), idesc,
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_f16(d0, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), id0,
                        (kb | kk) != 0 ? 1u : 0u);
+          if (two) {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              tc_mma_f16(d1, sw128_kmajor_desc(a_addr + A_BYTES + kk * 32), sw128_kmajor_desc(b_addr + kk * 32),
+                         id1, (kb | kk) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
         }
-        if (!ok) break;
-        tc_commit(&tfull[acc]);
-        if (++acc == 2) {
-          acc = 0;
-          acc_phase ^= 1u;
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
-      // every MMA of this CTA has completed before TMEM is released
-      tc_commit(done);
-      mbar_wait(done, 0, err, 4);
+      if (!ok) break;
+      if (elect_one()) {
+        tc_commit(&tfull[s0]);
+        if (two) tc_commit(&tfull[s1]);
+      }
+      __syncwarp();
+      ++uses[s0];
+      if (two) ++uses[s1];
+      else slot ^= 1;
     }
+    // every MMA of this CTA has completed before TMEM is released
+    if (elect_one()) tc_commit(done);
+    __syncwarp();
+    warp_wait(done, 0, err, 4);
   } else {
-    // ---------------------------------------------------------------- epilogue
-    const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter+32)
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    int chunk = 0;  // down: boxes stored by this warp (selects the staging buffer)
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile ti = decode_tile<MODE>(args, t);
-      if (!mbar_wait(&tfull[acc], acc_phase, err, 5)) break;
-      tc_fence_after();
-      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-      // M = 64 tiles (see the MMA issuer): row 16 quarter + lane in lanes 0..15 of the quarter
-      const bool m64 = ti.rows_valid <= 64;
-      const int row_in_tile = m64 ? (lane < 16 ? quarter * 16 + lane : BM) : quarter * 32 + lane;
-      const bool row_ok = row_in_tile < ti.rows_valid;
-      const int64_t grow = (int64_t)ti.a_row + row_in_tile;
-      if (MODE == kGateUp) {
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
-#pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          uint32_t g[32], u[32];
-          tmem_ld32(tbase + c, g);
-          tmem_ld32(tbase + BN / 2 + c, u);
-          tc_wait_ld();
-          const int col0 = ti.n_blk * (BN / 2) + c;
-          if (row_ok && col0 < args.n_out) {
-            uint4* dst = reinterpret_cast<uint4*>(out + grow * args.ldo + col0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 v;
-              v.x = pack_bf16(silu_mul(__uint_as_float(g[8 * q + 0]), __uint_as_float(u[8 * q + 0])),
-                              silu_mul(__uint_as_float(g[8 * q + 1]), __uint_as_float(u[8 * q + 1])));
-              v.y = pack_bf16(silu_mul(__uint_as_float(g[8 * q + 2]), __uint_as_float(u[8 * q + 2])),
-                              silu_mul(__uint_as_float(g[8 * q + 3]), __uint_as_float(u[8 * q + 3])));
-              v.z = pack_bf16(silu_mul(__uint_as_float(g[8 * q + 4]), __uint_as_float(u[8 * q + 4])),
-                              silu_mul(__uint_as_float(g[8 * q + 5]), __uint_as_float(u[8 * q + 5])));
-              v.w = pack_bf16(silu_mul(__uint_as_float(g[8 * q + 6]), __uint_as_float(u[8 * q + 6])),
-                              silu_mul(__uint_as_float(g[8 * q + 7]), __uint_as_float(u[8 * q + 7])));
-              dst[q] = v;
-            }
-            if (args.gu_save) {
-              // training: the pre-activations for the backward, in the padded row layout
-              __nv_bfloat16* gs = static_cast<__nv_bfloat16*>(args.gu_save) +
-                                  ((int64_t)ti.p_row + row_in_tile) * 2 * args.n_out + col0;
-              uint4* gdst = reinterpret_cast<uint4*>(gs);
-              uint4* udst = reinterpret_cast<uint4*>(gs + args.n_out);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                gdst[q] = make_uint4(pack_bf16(__uint_as_float(g[8 * q + 0]), __uint_as_float(g[8 * q + 1])),
-                                     pack_bf16(__uint_as_float(g[8 * q + 2]), __uint_as_float(g[8 * q + 3])),
-                                     pack_bf16(__uint_as_float(g[8 * q + 4]), __uint_as_float(g[8 * q + 5])),
-                                     pack_bf16(__uint_as_float(g[8 * q + 6]), __uint_as_float(g[8 * q + 7])));
-                udst[q] = make_uint4(pack_bf16(__uint_as_float(u[8 * q + 0]), __uint_as_float(u[8 * q + 1])),
-                                     pack_bf16(__uint_as_float(u[8 * q + 2]), __uint_as_float(u[8 * q + 3])),
-                                     pack_bf16(__uint_as_float(u[8 * q + 4]), __uint_as_float(u[8 * q + 5])),
-                                     pack_bf16(__uint_as_float(u[8 * q + 6]), __uint_as_float(u[8 * q + 7])));
-              }
-            }
-          }
+    // ---------------------------------------------------------------- epilogue (8 warps)
+    const int quarter = warp & 3;           // TMEM lanes [32 quarter, 32 quarter + 32)
+    const int half = (warp - 2) >> 2;       // which half of the columns
+    uint8_t* stg = sStg + (warp - 2) * STG_BYTES;
+    int slot = 0;
+    uint32_t uses[2] = {0, 0};
+    bool ok = true;
+    for (int i = 0; i <= total && ok; ++i) {
+      const int rs = i % RING;
+      if (!warp_wait(&ufull[rs], (i / RING) & 1, err, 12)) break;
+      const int t = ring[rs];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&uempty[rs]);
+      if (t < 0) break;
+      const Unit u = decode_unit<MODE, C::kPair>(args, t);
+      const int nrb = (C::kPair && u.rows[1] > 0) ? 2 : 1;
+      for (int r = 0; r < nrb; ++r) {
+        const int s = slot ^ r;
+        if (!warp_wait(&tfull[s], uses[s] & 1, err, 5)) {
+          ok = false;
+          break;
         }
-      } else if (MODE == kDown && !m64 && quarter * 32 + 32 <= ti.rows_valid) {
-        // 32 valid rows: coalesced TMA stores of 32 x 64 boxes staged in shared memory (thread
-        // = row, its 64 bf16 values as eight 16-byte chunks, chunk j at j ^ (row & 7): the
-        // 128-byte swizzle of the output tensor map)
-        const int grow0 = ti.a_row + quarter * 32;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 64) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(tbase + c, r0);
-          tmem_ld32(tbase + c + 32, r1);
-          tc_wait_ld();
-          const int col0 = ti.n_blk * BN + c;
-          if (col0 >= args.n_out) continue;  // the same for the whole warp
-          uint8_t* stg = sStg + (quarter * 2 + (chunk & 1)) * STG_BYTES;
-          if (lane == 0) bulk_wait_read_1();  // the store two boxes back has read this buffer
-          __syncwarp();
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t* v = j < 4 ? r0 + 8 * j : r1 + 8 * (j - 4);
-            *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                make_uint4(pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1])),
-                           pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3])),
-                           pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5])),
-                           pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7])));
-          }
-          fence_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmC, stg, col0, grow0);
-            bulk_commit();
-          }
-          ++chunk;
-        }
-      } else if (MODE == kDown) {
-        // a partly valid row group (the rows past it belong to the next expert): row stores
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(tbase + c, r);
-          tc_wait_ld();
-          const int col0 = ti.n_blk * BN + c;
-          if (row_ok && col0 < args.n_out) {
-            uint4* dst = reinterpret_cast<uint4*>(out + grow * args.ldo + col0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 v;
-              v.x = pack_bf16(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
-              v.y = pack_bf16(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
-              v.z = pack_bf16(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
-              v.w = pack_bf16(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
-              dst[q] = v;
-            }
-          }
-        }
-      } else {
-        float* out = static_cast<float*>(args.out);
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(tbase + c, r);
-          tc_wait_ld();
-          const int col0 = ti.n_blk * BN + c;
-          if (row_ok && col0 < args.n_out) {
-            float* dst = out + grow * args.ldo + col0;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              if (col0 + i < args.n_out) {
-                const float add = args.col_add ? args.col_add[col0 + i] : 0.0f;
-                dst[i] = __fadd_rn(__uint_as_float(r[i]), add);
-              }
-            }
-          }
-        }
+        tc_fence_after();
+        const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * BN);
+        drain_rows<MODE>(args, &tmC, tbase, quarter, half, lane, u.a_row + r * BM, u.rows[r], u.p_row + r * BM,
+                         u.n_blk, stg);
+        tc_fence_before();
+        mbar_arrive(&tempty[s]);
+        ++uses[s];
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
+      if (nrb == 1) slot ^= 1;
     }
     if (MODE == kDown && lane == 0) bulk_wait_all();  // every store complete before exit
   }
@@ -400,30 +494,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int MODE>
+template <int MODE, bool PAIR>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& c,
                         const TcArgs& args, int grid, cudaStream_t s) {
+  using C = Cfg<MODE, PAIR>;
   static SmemAttr attr{};
-  const cudaError_t e = ensure_smem_attr(attr, k_tc_gemm<MODE>, SMEM_BYTES);
+  cudaError_t e = ensure_smem_attr(attr, k_tc_gemm<MODE, PAIR>, C::kSmem);
   if (e != cudaSuccess) return e;
-  k_tc_gemm<MODE><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, c, args);
+  if (!args.sched || (C::kPair && !args.sp_off)) return cudaErrorInvalidValue;
+  e = cudaMemsetAsync(args.sched, 0, sizeof(int), s);  // the scheduler's unit counter starts at 0
+  if (e != cudaSuccess) return e;
+  k_tc_gemm<MODE, PAIR><<<grid, NUM_THREADS, C::kSmem, s>>>(a, b0, b1, c, args);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-int tc_smem_bytes() { return SMEM_BYTES; }
+int tc_smem_bytes() {
+  return Cfg<kGateUp, true>::kSmem > Cfg<kGateUp, false>::kSmem ? Cfg<kGateUp, true>::kSmem
+                                                                : Cfg<kGateUp, false>::kSmem;
+}
 int tc_block_n(int mode) { return mode == kGateUp ? BN / 2 : BN; }
 
 cudaError_t launch_tc_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                            const CUtensorMap& c, const TcArgs& args, int grid, cudaStream_t s) {
   switch (mode) {
     case kRouter:
-      return launch_mode<kRouter>(a, b0, b1, c, args, grid, s);
+      return launch_mode<kRouter, false>(a, b0, b1, c, args, grid, s);
     case kGateUp:
-      return launch_mode<kGateUp>(a, b0, b1, c, args, grid, s);
+      return args.pair ? launch_mode<kGateUp, true>(a, b0, b1, c, args, grid, s)
+                       : launch_mode<kGateUp, false>(a, b0, b1, c, args, grid, s);
     case kDown:
-      return launch_mode<kDown>(a, b0, b1, c, args, grid, s);
+      return args.pair ? launch_mode<kDown, true>(a, b0, b1, c, args, grid, s)
+                       : launch_mode<kDown, false>(a, b0, b1, c, args, grid, s);
     default:
       return cudaErrorInvalidValue;
   }

@@ -54,94 +54,169 @@ __device__ __forceinline__ float zexp(float x) {
   return __fmul_rn(p, scale);
 }
 
-__device__ __forceinline__ bool better(float va, int ea, float vb, int eb) {
-  return va > vb || (va == vb && ea < eb);
-}
-
 // Selection key of a biased score: a NaN ranks as -inf (below every number), so a
 // row whose scores are not all numbers still selects k distinct valid experts
 // (the lowest untaken ids among the NaN ones) instead of an id out of range.
 __device__ __forceinline__ float rank_key(float v) { return v == v ? v : -__int_as_float(0x7f800000); }
 
-// One warp per token.  EPL = experts held per lane (E <= 32 * EPL).
+// Selection key of a biased score: unsigned, ordered like the scores (a NaN ranks
+// as -inf, -0 as +0); 0 lies below every score's key and marks an expert already
+// taken (or a padding slot past E).
+__device__ __forceinline__ uint32_t sel_key(float v) {
+  uint32_t b = __float_as_uint(rank_key(v));
+  if (b == 0x80000000u) b = 0u;  // -0 compares equal to +0
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// (a, ea) ranks before (b, eb): the larger key, or the lower id on equal keys.
+__device__ __forceinline__ bool ranks_before(uint32_t a, uint32_t ea, uint32_t b, uint32_t eb) {
+  return a > b || (a == b && ea < eb);
+}
+
+// One warp per token.  EPL = experts held per lane (E <= 32 * EPL); lane p holds
+// experts p, p + 32, ...  Selection, exact and in two steps:
+//  1. threshold: the k-th largest of the 32 lane maxima (ties counted), tau.  At least
+//     k lanes hold a key >= tau, so every one of the k picks has a key >= tau;
+//  2. the candidates (key >= tau) are compacted into one slot per lane and sorted by
+//     (key descending, id ascending) with a 32-lane bitonic network; lanes 0..k-1 then
+//     hold the picks in slot order.
+// When more than 32 candidates reach tau (ties at the threshold, e.g. a row of NaN
+// scores), the picks are taken one by one instead: a warp max of the lanes' best
+// untaken keys, then a warp min of the ids holding it, the winning lane rescanning.
 template <int EPL>
-__global__ void __launch_bounds__(256) k_softmax_topk(const float* __restrict__ logits, const float* __restrict__ bias,
+__global__ void __launch_bounds__(256, 3) k_softmax_topk(const float* __restrict__ logits, const float* __restrict__ bias,
                                                       int T, int E, int k, float scale, int32_t* __restrict__ idx,
                                                       float* __restrict__ gate, float* __restrict__ scores) {
   const int lane = threadIdx.x & 31;
   const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
-  float b[EPL];
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const int e = lane + 32 * i;
-    b[i] = e < E ? bias[e] : 0.0f;
-  }
   for (int t = warp; t < T; t += nwarps) {
     const float* lt = logits + (int64_t)t * E;
-    float l[EPL];
+    float u[EPL];
     float m = -__int_as_float(0x7f800000);
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
-      l[i] = e < E ? lt[e] : -__int_as_float(0x7f800000);
-      m = fmaxf(m, l[i]);
+      u[i] = e < E ? lt[e] : -__int_as_float(0x7f800000);
+      m = fmaxf(m, u[i]);
     }
 #pragma unroll
     for (int w = 16; w >= 1; w >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, w));
-    float u[EPL];
     float acc = 0.0f;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
-      u[i] = 0.0f;
-      if (e < E) {
-        u[i] = zexp(__fsub_rn(l[i], m));
-        acc = __fadd_rn(acc, u[i]);
-      }
+      u[i] = e < E ? zexp(__fsub_rn(u[i], m)) : 0.0f;
+      if (e < E) acc = __fadd_rn(acc, u[i]);
     }
 #pragma unroll
     for (int w = 16; w >= 1; w >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, w));
-    float v[EPL];
-    uint32_t taken = 0;
+    uint32_t key[EPL];
+    uint32_t lmax = 0;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
       u[i] = __fdiv_rn(u[i], acc);  // u now holds the score s
-      v[i] = rank_key(__fadd_rn(u[i], b[i]));
-      if (e >= E) taken |= 1u << i;
-      else if (scores) scores[(int64_t)t * E + e] = u[i];
+      key[i] = e < E ? sel_key(__fadd_rn(u[i], bias[e])) : 0u;
+      if (e < E && scores) scores[(int64_t)t * E + e] = u[i];
+      lmax = max(lmax, key[i]);
+    }
+    // 1. tau = the k-th largest lane maximum
+    uint32_t tau = 0, act = lmax;
+    int need = k;
+    for (int r = 0; r < k && need > 0; ++r) {
+      const uint32_t g = __reduce_max_sync(0xffffffffu, act);
+      need -= __popc(__ballot_sync(0xffffffffu, act == g));
+      if (act == g) act = 0u;
+      tau = g;
+    }
+    // 2. compaction of the candidates: lane c receives the c-th one (key, id, score)
+    uint32_t ck = 0u, ce = 0xffffffffu;
+    float cs = 0.0f;
+    int count = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const bool c = key[i] >= tau;
+      const uint32_t ballot = __ballot_sync(0xffffffffu, c);
+      const int base = count;
+      count += __popc(ballot);
+      if (ballot == 0u) continue;
+      // the candidates of this row go to slots base, base + 1, ... in lane order: lane L
+      // receives slot L, i.e. the candidate of rank L - base, held by the lane of the
+      // (L - base + 1)-th set bit of the ballot
+      const int rank = lane - base;
+      const bool recv = rank >= 0 && rank < __popc(ballot);
+      const int src = recv ? (int)__fns(ballot, 0, rank + 1) : 0;
+      const uint32_t vk = __shfl_sync(0xffffffffu, key[i], src);
+      const float vs = __shfl_sync(0xffffffffu, u[i], src);
+      if (recv) {
+        ck = vk;
+        ce = (uint32_t)(src + 32 * i);
+        cs = vs;
+      }
     }
     int my_idx = 0;
     float my_gate = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      float bv = -__int_as_float(0x7f800000);
-      int be = 0x7fffffff;
-      float bs = 0.0f;
+    if (count <= 32) {
+      // bitonic sort of the 32 slots, best first (empty slots: key 0, id ~0, last)
+#pragma unroll
+      for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          const uint32_t ok = __shfl_xor_sync(0xffffffffu, ck, stride);
+          const uint32_t oe = __shfl_xor_sync(0xffffffffu, ce, stride);
+          const float os = __shfl_xor_sync(0xffffffffu, cs, stride);
+          const bool lower = (lane & stride) == 0;
+          const bool best_first = (lane & size) == 0;  // this block is sorted best first
+          const bool other_before = ranks_before(ok, oe, ck, ce);
+          // the lower lane of a best-first block keeps the better of the two
+          if (other_before == (lower == best_first)) {
+            ck = ok;
+            ce = oe;
+            cs = os;
+          }
+        }
+      }
+      my_idx = (int)ce;
+      my_gate = __fmul_rn(scale, cs);
+    } else {
+      uint32_t bk = 0;
+      int bi = 0;
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        if (!((taken >> i) & 1u) && better(v[i], e, bv, be)) {
-          bv = v[i];
-          be = e;
-          bs = u[i];
+        if (key[i] > bk) {
+          bk = key[i];
+          bi = i;
         }
       }
+      for (int j = 0; j < k; ++j) {
+        const uint32_t gk = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t ge = __reduce_min_sync(0xffffffffu, bk == gk ? (uint32_t)(lane + 32 * bi) : 0xffffffffu);
+        const int wl = (int)(ge & 31u);
+        float ws = 0.0f;
+        if (lane == wl) {
+          bk = 0;
 #pragma unroll
-      for (int w = 16; w >= 1; w >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, w);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, w);
-        const float os = __shfl_xor_sync(0xffffffffu, bs, w);
-        if (better(ov, oe, bv, be)) {
-          bv = ov;
-          be = oe;
-          bs = os;
+          for (int i = 0; i < EPL; ++i) {
+            if (i == bi) {
+              ws = u[i];
+              key[i] = 0u;
+            }
+          }
+          bi = 0;
+#pragma unroll
+          for (int i = 0; i < EPL; ++i) {
+            if (key[i] > bk) {
+              bk = key[i];
+              bi = i;
+            }
+          }
         }
-      }
-      if (lane == (be & 31)) taken |= 1u << (be >> 5);
-      if (lane == j) {
-        my_idx = be;
-        my_gate = __fmul_rn(scale, bs);
+        ws = __shfl_sync(0xffffffffu, ws, wl);
+        if (lane == j) {
+          my_idx = (int)ge;
+          my_gate = __fmul_rn(scale, ws);
+        }
       }
     }
     if (lane < k) {
@@ -274,14 +349,17 @@ __device__ __forceinline__ int2 block_exclusive_scan2(int2 v, int2* warp_tot) {
 }
 
 // Integer stage, part 2 (one block of 1024 threads, thread = expert): totals,
-// controller accumulation, exclusive scans over FFN experts of the counts and
-// of their 128-row block counts, and the first permuted row of every
-// (token block, expert) pair, written over chunk_cnt.
+// controller accumulation, exclusive scans over FFN experts of the counts, of
+// their 128-row block counts and (sp_off, when asked) of their row-block pairs
+// ceil(blocks / 2), and the first permuted row of every (token block, expert)
+// pair, written over chunk_cnt.
 __global__ void __launch_bounds__(1024) k_route_scan(int32_t* __restrict__ chunk_cnt, int nchunks, int T, int N, int E,
                                                      int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                                      int32_t* __restrict__ mb_off, int32_t* __restrict__ scal,
-                                                     int64_t* __restrict__ acc_counts, int64_t* __restrict__ acc_tokens) {
+                                                     int64_t* __restrict__ acc_counts, int64_t* __restrict__ acc_tokens,
+                                                     int32_t* __restrict__ sp_off) {
   __shared__ int2 warp_tot[32];
+  __shared__ int2 warp_tot2[32];
   const int e = threadIdx.x;
   int total = 0;
   if (e < E) {
@@ -292,12 +370,16 @@ __global__ void __launch_bounds__(1024) k_route_scan(int32_t* __restrict__ chunk
   }
   const int2 v = (e < N) ? make_int2(total, (total + kBM - 1) / kBM) : make_int2(0, 0);
   const int2 ex = block_exclusive_scan2(v, warp_tot);
+  const int2 v2 = make_int2((v.y + 1) / 2, 0);
+  const int2 ex2 = sp_off ? block_exclusive_scan2(v2, warp_tot2) : make_int2(0, 0);
   if (e < N) {
     offsets[e] = ex.x;
     mb_off[e] = ex.y;
+    if (sp_off) sp_off[e] = ex2.x;
     if (e == N - 1) {
       offsets[N] = ex.x + v.x;
       mb_off[N] = ex.y + v.y;
+      if (sp_off) sp_off[N] = ex2.x + v2.x;
       scal[0] = ex.x + v.x;
       scal[1] = ex.y + v.y;
     }
@@ -514,13 +596,18 @@ __global__ void k_selftest_wait(int* err, uint64_t limit_ns) {
 int grid_cap(int want, int cap) { return want < 1 ? 1 : (want < cap ? want : cap); }
 
 // One group holding all T rows (the dense FFN through the grouped GEMM):
-// row_off = {0, T}, mb_off = {0, ceil(T / 128)}.
-__global__ void k_single_group(int32_t* row_off, int32_t* mb_off, int T) {
+// row_off = {0, T}, mb_off = {0, ceil(T / 128)}, sp_off (if given) = {0, ceil(mb / 2)}.
+__global__ void k_single_group(int32_t* row_off, int32_t* mb_off, int32_t* sp_off, int T) {
   if (threadIdx.x == 0) {
+    const int mb = (T + kBM - 1) / kBM;
     row_off[0] = 0;
     row_off[1] = T;
     mb_off[0] = 0;
-    mb_off[1] = (T + kBM - 1) / kBM;
+    mb_off[1] = mb;
+    if (sp_off) {
+      sp_off[0] = 0;
+      sp_off[1] = (mb + 1) / 2;
+    }
   }
 }
 
@@ -553,8 +640,10 @@ cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int32_t*
 }
 
 cudaError_t launch_route_scan(int32_t* chunk_cnt, int nchunks, int T, int N, int E, int32_t* counts, int32_t* offsets,
-                              int32_t* mb_off, int32_t* scal, int64_t* acc_counts, int64_t* acc_tokens, cudaStream_t s) {
-  k_route_scan<<<1, 1024, 0, s>>>(chunk_cnt, nchunks, T, N, E, counts, offsets, mb_off, scal, acc_counts, acc_tokens);
+                              int32_t* mb_off, int32_t* scal, int64_t* acc_counts, int64_t* acc_tokens, cudaStream_t s,
+                              int32_t* sp_off) {
+  k_route_scan<<<1, 1024, 0, s>>>(chunk_cnt, nchunks, T, N, E, counts, offsets, mb_off, scal, acc_counts, acc_tokens,
+                                  sp_off);
   return cudaGetLastError();
 }
 
@@ -607,8 +696,8 @@ cudaError_t launch_router_bwd(const float* logits, int T, int E, int k, float sc
   return cudaGetLastError();
 }
 
-cudaError_t launch_single_group(int32_t* row_off, int32_t* mb_off, int T, cudaStream_t s) {
-  k_single_group<<<1, 32, 0, s>>>(row_off, mb_off, T);
+cudaError_t launch_single_group(int32_t* row_off, int32_t* mb_off, int T, cudaStream_t s, int32_t* sp_off) {
+  k_single_group<<<1, 32, 0, s>>>(row_off, mb_off, sp_off, T);
   return cudaGetLastError();
 }
 

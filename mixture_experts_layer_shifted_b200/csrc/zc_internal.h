@@ -44,8 +44,10 @@ cudaError_t ensure_smem_attr(SmemAttr& a, Kernel* kernel, int bytes) {
 cudaError_t launch_softmax_topk(const float* logits, const float* bias, int T, int E, int k, float scale, int32_t* idx,
                                 float* gate, float* scores, int sms, cudaStream_t s);
 cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int32_t* chunk_cnt, cudaStream_t s);
+// sp_off (nullable): [N+1] prefix of the row-block pairs ceil(mb / 2) (the grouped GEMM's work units)
 cudaError_t launch_route_scan(int32_t* chunk_cnt, int nchunks, int T, int N, int E, int32_t* counts, int32_t* offsets,
-                              int32_t* mb_off, int32_t* scal, int64_t* acc_counts, int64_t* acc_tokens, cudaStream_t s);
+                              int32_t* mb_off, int32_t* scal, int64_t* acc_counts, int64_t* acc_tokens, cudaStream_t s,
+                              int32_t* sp_off = nullptr);
 cudaError_t launch_route_scatter(const int32_t* idx, int T, int k, int N, int E, const int32_t* chunk_base,
                                  int32_t* perm, int32_t* pos, cudaStream_t s);
 cudaError_t launch_gather_rows(const void* x, int row_bytes, const int32_t* perm, int k, const int32_t* scal,
@@ -55,7 +57,7 @@ cudaError_t launch_combine(int bf16, const void* x, const void* Y, const int32_t
                            const int32_t* pos, int T, int k, int N, int d, void* y, int sms, cudaStream_t s,
                            const int32_t* offsets = nullptr, const int32_t* mb_off = nullptr);
 cudaError_t launch_selftest_wait(int* err, uint64_t limit_ns, cudaStream_t s);
-cudaError_t launch_single_group(int32_t* row_off, int32_t* mb_off, int T, cudaStream_t s);
+cudaError_t launch_single_group(int32_t* row_off, int32_t* mb_off, int T, cudaStream_t s, int32_t* sp_off = nullptr);
 cudaError_t launch_update_bias(int64_t* counts, int64_t* tokens, int N, int Z, int k, float kp, float ki, float kd,
                                float decay, float target, const float* b0, float* eta, float* integ, float* eprev,
                                float* bias, cudaStream_t s);
@@ -78,7 +80,18 @@ struct TcArgs {
   void* gu_save;            // gate/up, optional: the fp32 accumulators G and U rounded to bf16, stored as
                             // [G | U] [padded rows, 2 n_out] (expert g's pairs from row 128 mb_off[g] on)
   int* err;                 // device error word (bounded waits)
+  // grouped modes: [ngroups+1] first row-block pair of each expert, prefix of ceil(mb / 2)
+  // over the experts' row blocks (the unit of work that shares one staged weight tile)
+  const int32_t* sp_off;
+  int* sched;               // tile counter of the dynamic scheduler, zeroed by the launcher
+  int pair;                 // grouped modes: 1 = units of two row blocks (the expected rows per
+                            // expert fill two or more blocks), 0 = one row block per unit
 };
+
+// Whether the grouped GEMMs should stage two row blocks per weight tile: when an
+// expert's rows are expected to fill at least 128 rows (rows = expected rows per
+// expert, from the batch size and the routing fan-out, known on the host).
+inline int tc_pair_for_rows(int64_t rows) { return rows >= kBM ? 1 : 0; }
 
 int tc_smem_bytes();
 int tc_block_n(int mode);

@@ -182,6 +182,8 @@ struct zcmoe_s {
   // workspace
   float *logits, *gate;
   int32_t *idx, *pos, *counts, *offsets, *mb_off, *scal, *chunk, *perm;
+  int32_t* sp_off;  // [N+1] row-block pairs per expert, prefix (the grouped GEMM's work units)
+  int* sched;       // [4] unit counters of the tensor-core GEMM launches (router, gate/up, down)
   void *xperm, *H, *Y;
   // zcmoe_forward_host: x staged through two device buffers filled on an internal
   // copy stream, so the next call's upload overlaps this call's compute; y staged once
@@ -218,7 +220,7 @@ struct zcmoe_s {
   // (ep_rank + 1) * n_local); xperm / H / Y have rows_cap rows (the routed pairs of max_T
   // tokens, or the rows received from all ranks, whichever is larger).  ep_meta (device) and
   // ep_meta_host (pinned): seg_src [nseg + 1], seg_dst [nseg], exp_off [n_local + 1],
-  // mb_off [n_local + 1] of the last zcmoe_ep_experts, nseg = ep_size * n_local
+  // mb_off [n_local + 1], sp_off [n_local + 1] of the last zcmoe_ep_experts, nseg = ep_size * n_local
   int ep_rank, ep_size, n_local;
   int64_t rows_cap;
   int32_t *ep_meta, *ep_meta_host;
@@ -230,7 +232,7 @@ struct zcmoe_s {
 static void release(zcmoe_s* h) {
   void* ptrs[] = {h->bias,  h->b0,     h->offset, h->eta,   h->integ,   h->eprev,  h->acc_counts,
                   h->err,   h->logits, h->gate,   h->idx,   h->pos,     h->counts, h->offsets,
-                  h->mb_off, h->scal,  h->chunk,  h->perm,  h->xperm,   h->H,      h->Y,
+                  h->mb_off, h->scal,  h->chunk,  h->perm,  h->xperm,   h->H,      h->Y,  h->sp_off, h->sched,
                   h->stage_x, h->stage_x2, h->stage_y, h->stage_y2, h->w8g, h->w8u, h->w8d, h->sfg, h->sfu, h->sfd,
                   h->x8, h->sx, h->h8, h->sh, h->ypad, h->b_xpad, h->b_dypad, h->b_dh, h->b_dgu, h->b_hpad,
                   h->b_dxp, h->b_dl, h->b_dxr, h->b_dg, h->b_grp, h->b_gu, h->ep_meta};
@@ -259,7 +261,8 @@ struct zcmoe_dense_s {
   int d, inter, max_T, sms;
   zcmoe_dense_weights w;
   void* H;           // [max_T, inter] bf16
-  int32_t* offs;     // one group: row_off[2], then mb_off[2] (written per call)
+  int32_t* offs;     // one group: row_off[2], mb_off[2], sp_off[2] (written per call); then the
+                     // GEMMs' unit counters [2]
   int* err;          // bounded-wait error word of the dense kernels
   cudaStream_t side; // zcmoe_forward_overlap enqueues the dense FFN here
   cudaEvent_t ev_router, ev_down, ev_join;
@@ -281,7 +284,7 @@ static int dense_gate_up(zcmoe_dense_s* h, const void* x, int T, cudaStream_t s)
   CUtensorMap tm_x;
   int rc = make_tmap(&tm_x, x, (uint64_t)h->d, (uint64_t)T, 128);
   if (rc != ZCMOE_OK) return rc;
-  ZC_CUDA(zc::launch_single_group(h->offs, h->offs + 2, T, s));
+  ZC_CUDA(zc::launch_single_group(h->offs, h->offs + 2, T, s, h->offs + 4));
   zc::TcArgs a{};
   a.K = h->d;
   a.n_out = h->inter;
@@ -289,6 +292,9 @@ static int dense_gate_up(zcmoe_dense_s* h, const void* x, int T, cudaStream_t s)
   a.ngroups = 1;
   a.row_off = h->offs;
   a.mb_off = h->offs + 2;
+  a.sp_off = h->offs + 4;
+  a.sched = h->offs + 6;
+  a.pair = zc::tc_pair_for_rows(T);
   a.b_rows_per_group = h->inter;
   a.out = h->H;
   a.ldo = h->inter;
@@ -307,6 +313,9 @@ static int dense_down(zcmoe_dense_s* h, int T, void* y, cudaStream_t s) {
   b.ngroups = 1;
   b.row_off = h->offs;
   b.mb_off = h->offs + 2;
+  b.sp_off = h->offs + 4;
+  b.sched = h->offs + 7;
+  b.pair = zc::tc_pair_for_rows(T);
   b.b_rows_per_group = h->d;
   b.out = y;
   b.ldo = h->d;
@@ -418,6 +427,8 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
   ZC_ALLOC(h->counts, E);
   ZC_ALLOC(h->offsets, N + 1);
   ZC_ALLOC(h->mb_off, N + 1);
+  ZC_ALLOC(h->sp_off, N + 1);
+  ZC_ALLOC(h->sched, 4);
   ZC_ALLOC(h->scal, 4);
   ZC_ALLOC(h->chunk, (size_t)h->max_chunks * E);
   ZC_ALLOC(h->perm, (size_t)h->max_pairs);
@@ -431,7 +442,7 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
     h->H = hh;
     h->Y = yy;
   }
-  if (ep_size > 1) ZC_ALLOC(h->ep_meta, (size_t)2 * ep_size * NL + 1 + 2 * (NL + 1));
+  if (ep_size > 1) ZC_ALLOC(h->ep_meta, (size_t)2 * ep_size * NL + 1 + 3 * (NL + 1));
   if (h->fp8) {
     const size_t prow = (size_t)h->max_mblocks * zc::kBM;  // padded rows
     // scale atoms per 128 rows: an atom covers 512 K elements (FP8) or 128 (MXFP4)
@@ -461,7 +472,7 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
   h->acc_tokens = h->acc_counts + E;
   if (ep_size > 1) {
     cudaError_t e = cudaHostAlloc(reinterpret_cast<void**>(&h->ep_meta_host),
-                                  ((size_t)2 * ep_size * NL + 1 + 2 * (NL + 1)) * sizeof(int32_t), cudaHostAllocDefault);
+                                  ((size_t)2 * ep_size * NL + 1 + 3 * (NL + 1)) * sizeof(int32_t), cudaHostAllocDefault);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ep_meta_ev, cudaEventDisableTiming);
     if (e != cudaSuccess) {
       release(h);
@@ -581,6 +592,7 @@ static int router_stage(zcmoe_t h, const void* x, int Ti, cudaStream_t s) {
     a.ldo = E;
     a.col_add = h->offset;
     a.err = h->err;
+    a.sched = h->sched;
     const int tiles = ((Ti + zc::kBM - 1) / zc::kBM) * a.nblocks;
     ZC_CUDA(zc::launch_tc_gemm(zc::kRouter, tm_x, h->tm_wr, h->tm_wr, h->tm_wr, a, tiles < h->sms ? tiles : h->sms, s));
   } else {
@@ -606,7 +618,7 @@ static int integer_stage(zcmoe_t h, int Ti, cudaStream_t s) {
   const int nchunks = (Ti + zc::kChunk - 1) / zc::kChunk;
   ZC_CUDA(zc::launch_route_count(h->idx, Ti, k, E, h->chunk, s));
   ZC_CUDA(zc::launch_route_scan(h->chunk, nchunks, Ti, N, E, h->counts, h->offsets, h->mb_off, h->scal,
-                                h->acc_counts, h->acc_tokens, s));
+                                h->acc_counts, h->acc_tokens, s, h->sp_off));
   ZC_CUDA(zc::launch_route_scatter(h->idx, Ti, k, N, E, h->chunk, h->perm, h->pos, s));
   return ZCMOE_OK;
 }
@@ -738,6 +750,9 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     a.ngroups = N;
     a.row_off = h->offsets;
     a.mb_off = h->mb_off;
+    a.sp_off = h->sp_off;
+    a.sched = h->sched + 1;
+    a.pair = zc::tc_pair_for_rows((int64_t)Ti * k / E);
     a.b_rows_per_group = inter;
     a.out = h->H;
     a.ldo = inter;
@@ -755,6 +770,9 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     b.ngroups = N;
     b.row_off = h->offsets;
     b.mb_off = h->mb_off;
+    b.sp_off = h->sp_off;
+    b.sched = h->sched + 2;
+    b.pair = a.pair;
     b.b_rows_per_group = d;
     b.out = h->Y;
     b.ldo = d;
@@ -884,6 +902,7 @@ int zcmoe_ep_experts(zcmoe_t h, const void* xrecv, const int32_t* counts, int64_
   // row layout: ep_size == 1 needs no regrouping (one source: s-major is e-major)
   const int32_t* exp_off;
   const int32_t* mb_off;
+  const int32_t* sp_off;
   int mb_total = 0;
   const void* a_rows = xrecv;
   void* y_rows = yrecv;
@@ -897,10 +916,12 @@ int zcmoe_ep_experts(zcmoe_t h, const void* xrecv, const int32_t* counts, int64_
     int32_t* seg_dst = seg_src + nseg + 1;
     int32_t* eoff = seg_dst + nseg;
     int32_t* moff = eoff + NL + 1;
+    int32_t* poff = moff + NL + 1;
     seg_src[0] = 0;
     for (int i = 0; i < nseg; ++i) seg_src[i + 1] = seg_src[i] + counts[i];
     eoff[0] = 0;
     moff[0] = 0;
+    poff[0] = 0;
     for (int e = 0; e < NL; ++e) {
       int cnt = 0;
       for (int r = 0; r < R; ++r) {
@@ -908,10 +929,12 @@ int zcmoe_ep_experts(zcmoe_t h, const void* xrecv, const int32_t* counts, int64_
         cnt += counts[r * NL + e];
       }
       eoff[e + 1] = eoff[e] + cnt;
-      moff[e + 1] = moff[e] + (cnt + zc::kBM - 1) / zc::kBM;
+      const int mb = (cnt + zc::kBM - 1) / zc::kBM;
+      moff[e + 1] = moff[e] + mb;
+      poff[e + 1] = poff[e] + (mb + 1) / 2;
     }
     mb_total = moff[NL];
-    const size_t bytes = ((size_t)2 * nseg + 1 + 2 * (NL + 1)) * sizeof(int32_t);
+    const size_t bytes = ((size_t)2 * nseg + 1 + 3 * (NL + 1)) * sizeof(int32_t);
     ZC_CUDA(cudaMemcpyAsync(h->ep_meta, m, bytes, cudaMemcpyHostToDevice, s));
     ZC_CUDA(cudaEventRecord(h->ep_meta_ev, s));
     h->ep_meta_pending = true;
@@ -919,6 +942,7 @@ int zcmoe_ep_experts(zcmoe_t h, const void* xrecv, const int32_t* counts, int64_
     const int32_t* dseg_dst = dseg_src + nseg + 1;
     exp_off = dseg_dst + nseg;
     mb_off = exp_off + NL + 1;
+    sp_off = mb_off + NL + 1;
     // rows into the e-major layout of xperm; the outputs come back through Y
     ZC_CUDA(zc::launch_ep_regroup(xrecv, h->xperm, P_recv, d * 2, dseg_src, dseg_dst, nseg, 0, h->sms, s));
     a_rows = h->xperm;
@@ -930,27 +954,32 @@ int zcmoe_ep_experts(zcmoe_t h, const void* xrecv, const int32_t* counts, int64_
       h->ep_meta_pending = false;
     }
     if (!h->ep_meta) {
-      int rc = dalloc(&h->ep_meta, (size_t)2 * (NL + 1));
+      int rc = dalloc(&h->ep_meta, (size_t)3 * (NL + 1));
       if (rc != ZCMOE_OK) return rc;
-      cudaError_t e = cudaHostAlloc(reinterpret_cast<void**>(&h->ep_meta_host), (size_t)2 * (NL + 1) * sizeof(int32_t),
+      cudaError_t e = cudaHostAlloc(reinterpret_cast<void**>(&h->ep_meta_host), (size_t)3 * (NL + 1) * sizeof(int32_t),
                                     cudaHostAllocDefault);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ep_meta_ev, cudaEventDisableTiming);
       if (e != cudaSuccess) return fail(ZCMOE_ECUDA, "expert-parallel staging: %s", cudaGetErrorString(e));
     }
     int32_t* eoff = h->ep_meta_host;
     int32_t* moff = eoff + NL + 1;
+    int32_t* poff = moff + NL + 1;
     eoff[0] = 0;
     moff[0] = 0;
+    poff[0] = 0;
     for (int e = 0; e < NL; ++e) {
       eoff[e + 1] = eoff[e] + counts[e];
-      moff[e + 1] = moff[e] + (counts[e] + zc::kBM - 1) / zc::kBM;
+      const int mb = (counts[e] + zc::kBM - 1) / zc::kBM;
+      moff[e + 1] = moff[e] + mb;
+      poff[e + 1] = poff[e] + (mb + 1) / 2;
     }
     mb_total = moff[NL];
-    ZC_CUDA(cudaMemcpyAsync(h->ep_meta, eoff, (size_t)2 * (NL + 1) * sizeof(int32_t), cudaMemcpyHostToDevice, s));
+    ZC_CUDA(cudaMemcpyAsync(h->ep_meta, eoff, (size_t)3 * (NL + 1) * sizeof(int32_t), cudaMemcpyHostToDevice, s));
     ZC_CUDA(cudaEventRecord(h->ep_meta_ev, s));
     h->ep_meta_pending = true;
     exp_off = h->ep_meta;
     mb_off = exp_off + NL + 1;
+    sp_off = mb_off + NL + 1;
   }
   CUtensorMap tm_a, tm_h;
   int rc = make_tmap(&tm_a, a_rows, (uint64_t)d, (uint64_t)P_recv, 128);
@@ -964,6 +993,9 @@ int zcmoe_ep_experts(zcmoe_t h, const void* xrecv, const int32_t* counts, int64_
   a.ngroups = NL;
   a.row_off = exp_off;
   a.mb_off = mb_off;
+  a.sp_off = sp_off;
+  a.sched = h->sched + 1;
+  a.pair = zc::tc_pair_for_rows(P_recv / NL);
   a.b_rows_per_group = inter;
   a.out = h->H;
   a.ldo = inter;
@@ -977,6 +1009,9 @@ int zcmoe_ep_experts(zcmoe_t h, const void* xrecv, const int32_t* counts, int64_
   b.ngroups = NL;
   b.row_off = exp_off;
   b.mb_off = mb_off;
+  b.sp_off = sp_off;
+  b.sched = h->sched + 2;
+  b.pair = a.pair;
   b.b_rows_per_group = d;
   b.out = y_rows;
   b.ldo = d;
@@ -1556,11 +1591,11 @@ int zcmoe_dense_create(const zcmoe_dense_config* cfg, const zcmoe_dense_weights*
   uint8_t* hh = nullptr;
   int rc = dalloc(&hh, hbytes);
   h->H = hh;
-  if (rc == ZCMOE_OK) rc = dalloc(&h->offs, 4);
+  if (rc == ZCMOE_OK) rc = dalloc(&h->offs, 8);
   if (rc == ZCMOE_OK) rc = dalloc(&h->err, 1);
   if (rc == ZCMOE_OK) {
     cudaError_t e = cudaMemset(h->H, 0, hbytes);
-    if (e == cudaSuccess) e = cudaMemset(h->offs, 0, 4 * sizeof(int32_t));
+    if (e == cudaSuccess) e = cudaMemset(h->offs, 0, 8 * sizeof(int32_t));
     if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int));
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_router, cudaEventDisableTiming);

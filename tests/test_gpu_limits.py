@@ -86,3 +86,35 @@ def test_rows_that_are_not_finite(cuda_ok):
         r.check_layer_outputs(good[::7])
     finally:
         r.close()
+
+
+def test_routing_with_many_exact_ties(cuda_ok):
+    """Logits on a coarse grid (multiples of 1/2) and biases on a coarser one make many
+    experts share the same biased score, at and around the k-th place: the picks must
+    follow the oracle's rule (equal scores: the lower id first) bit for bit, whether
+    the selection takes its sorted-candidates path or its one-pick-at-a-time path."""
+    import ctypes
+    from mixture_experts_layer_shifted_b200 import zcmoe as Z
+    N, Zn, k, T = 512, 256, 12, 4096
+    E = N + Zn
+    rng = np.random.default_rng(13)
+    l = (np.round(rng.normal(size=(T, E)) * 2.0) / 2.0).astype(np.float32)
+    l[: T // 4] = np.round(l[: T // 4])          # coarser grid: more ties
+    l[T // 4: T // 4 + 8] = 1.5                  # every expert tied
+    bias = np.zeros(E, np.float32)
+    bias[::7] = np.float32(2.0 ** -20)
+    logits, b = torch.from_numpy(l).cuda(), torch.from_numpy(bias).cuda()
+    out = {"idx": (T * k, torch.int32), "gate": (T * k, torch.float32), "counts": (E, torch.int32),
+           "offsets": (N + 1, torch.int32), "perm": (T * k, torch.int32), "pos": (T * k, torch.int32)}
+    out = {key: torch.full((n,), -7, dtype=dt, device="cuda") for key, (n, dt) in out.items()}
+    p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    Z.zcmoe_route_noalloc(p(logits), p(b), T, N, Zn, k, 1.0, p(out["idx"]), p(out["gate"]), p(out["counts"]),
+                          p(out["offsets"]), p(out["perm"]), p(out["pos"]))
+    torch.cuda.synchronize()
+    idx, gate, _ = oracle.route_replica_f32(l, bias, k, 1.0, want_scores=True)
+    np.testing.assert_array_equal(out["idx"].cpu().numpy().reshape(T, k), idx)
+    np.testing.assert_array_equal(out["gate"].cpu().numpy().reshape(T, k).view(np.uint32), gate.view(np.uint32))
+    counts, offsets, perm, pos = oracle.integer_stage(idx, N, E)
+    np.testing.assert_array_equal(out["counts"].cpu().numpy(), counts)
+    np.testing.assert_array_equal(out["perm"].cpu().numpy()[: int(offsets[-1])], perm)
+    np.testing.assert_array_equal(out["pos"].cpu().numpy().reshape(T, k), pos)
