@@ -23,7 +23,7 @@ COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hi
           "--expt-relaxed-constexpr"]
 
 LAYER_SOURCES = ["zcmoe.cu", "route.cu", "gemm_tc.cu", "gemm_simt.cu", "route_noalloc.cu", "fp8_quant.cu", "gemm_fp8.cu", "gemm_bwd.cu", "moe_bwd.cu", "ep.cu"]
-LAYER_HEADERS = ["zc_internal.h", "zc_ptx.cuh"]
+LAYER_HEADERS = ["zc_internal.h", "zc_ptx.cuh", "zc_route.cuh", "zc_fp8.cuh"]
 
 
 def _stale(target, deps):

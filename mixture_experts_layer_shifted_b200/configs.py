@@ -68,6 +68,11 @@ WORKLOADS = {
     # inputs still larger than L2
     "prefill_probe": Workload("prefill_probe", T=2048, d=6144, n_ffn=32, inter=2048, n_zero=16, top_k=12,
                               dtype="bf16", w_std=0.006, bias=("zero",), dense_inter=12288),
+    # the prefill layer's per-expert shape at one eighth of its size (64 FFN + 32 zero experts,
+    # 2048 tokens, top-12: ~256 rows per expert as at prefill; 4.8 GB of weights): profiler
+    # captures of the expert GEMMs, whose traffic scales to prefill_560b by 8
+    "prefill_probe256": Workload("prefill_probe256", T=2048, d=6144, n_ffn=64, inter=2048, n_zero=32, top_k=12,
+                                 dtype="bf16", w_std=0.006, bias=("zero",)),
     # the 560B layer's expert shape with 16 experts (1.2 GB of weights): small captures of the
     # backward kernels, ~512 rows per expert as at prefill
     "bwd_probe": Workload("bwd_probe", T=1024, d=6144, n_ffn=16, inter=2048, n_zero=8, top_k=12, dtype="bf16",

@@ -24,6 +24,8 @@
 #include <unordered_set>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/zcmoe.h"
 #include "zc_fp8.cuh"
 #include "zc_internal.h"
@@ -656,7 +658,13 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
 
   const int Ti = (int)T, E = h->E, N = h->N, k = h->k, d = h->d, inter = h->inter;
   h->last_T = Ti;
-  auto mark = [&]() -> cudaError_t {
+  // Stage boundaries: an NVTX range per stage around its enqueue on the host (profiler
+  // timelines), and, while profiling, a CUDA event on the stream (per-stage device time).
+  bool nvtx_open = false;
+  auto mark = [&](const char* next) -> cudaError_t {
+    if (nvtx_open) nvtxRangePop();
+    nvtx_open = next != nullptr;
+    if (next) nvtxRangePushA(next);
     if (!h->profiling) return cudaSuccess;
     cudaEvent_t ev;
     cudaError_t e = cudaEventCreate(&ev);
@@ -664,14 +672,21 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     h->events->push_back(ev);
     return cudaEventRecord(ev, s);
   };
-  ZC_CUDA(mark());
+  // an early return leaves no range open
+  struct RangeGuard {
+    bool* open;
+    ~RangeGuard() {
+      if (*open) nvtxRangePop();
+    }
+  } range_guard{&nvtx_open};
+  ZC_CUDA(mark("zcmoe.router"));
 
   // 1. router logits
   {
     const int rc = router_stage(h, x, Ti, s);
     if (rc != ZCMOE_OK) return rc;
   }
-  ZC_CUDA(mark());
+  ZC_CUDA(mark("zcmoe.softmax_topk"));
   if (side) {
     ZC_CUDA(cudaEventRecord(side->dn->ev_router, s));
     ZC_CUDA(cudaStreamWaitEvent(side->dn->side, side->dn->ev_router, 0));
@@ -681,13 +696,13 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
   // 2. softmax + bias-shifted top-k
   ZC_CUDA(zc::launch_softmax_topk(h->logits, h->bias, Ti, E, k, h->cfg.routed_scale, h->idx, h->gate,
                                   dbg ? dbg->scores : nullptr, h->sms, s));
-  ZC_CUDA(mark());
+  ZC_CUDA(mark("zcmoe.integer_stage"));
   // 3. integer stage
   {
     const int rc = integer_stage(h, Ti, s);
     if (rc != ZCMOE_OK) return rc;
   }
-  ZC_CUDA(mark());
+  ZC_CUDA(mark("zcmoe.gather"));
   // 4. gather the FFN pairs' rows (FP8 layers: quantized per [1,128] into padded rows)
   if (h->fp8 && h->fmt)
     ZC_CUDA(zc::launch_gather_quant4(x, d, h->perm, h->idx, k, h->offsets, h->mb_off, h->scal, h->x8, h->sx, h->gd,
@@ -697,7 +712,7 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
                                     h->sms, s));
   else
     ZC_CUDA(zc::launch_gather_rows(x, (int)(d * esz), h->perm, k, h->scal, h->xperm, h->sms, s));
-  ZC_CUDA(mark());
+  ZC_CUDA(mark("zcmoe.gate_up"));
   // 5./6. expert GEMMs
   const int max_mb = (Ti * k + zc::kBM - 1) / zc::kBM + N;
   if (h->fp8) {
@@ -722,7 +737,7 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     int bound = max_mb * a.nblocks;
     ZC_CUDA(zc::launch_fp8_gemm(zc::kGateUp, h->tm8_x, h->tm8_wg, h->tm8_wu, h->tm8_wu, a,
                                 bound < h->sms ? bound : h->sms, s));
-    ZC_CUDA(mark());
+    ZC_CUDA(mark("zcmoe.down"));
     zc::Fp8Args b{};
     b.fmt = h->fmt;
     b.K = inter;
@@ -762,7 +777,7 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     int bound = max_mb * a.nblocks;
     ZC_CUDA(zc::launch_tc_gemm(zc::kGateUp, h->tm_xperm, h->tm_wg, h->tm_wu, h->tm_wu, a,
                                bound < h->sms ? bound : h->sms, s));
-    ZC_CUDA(mark());
+    ZC_CUDA(mark("zcmoe.down"));
     zc::TcArgs b{};
     b.K = inter;
     b.n_out = d;
@@ -793,7 +808,7 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     a.out = static_cast<float*>(h->H);
     a.ldo = inter;
     ZC_CUDA(zc::launch_simt_gemm(zc::kGateUp, a, max_mb, s));
-    ZC_CUDA(mark());
+    ZC_CUDA(mark("zcmoe.down"));
     zc::SimtArgs b{};
     b.A = static_cast<const float*>(h->H);
     b.B0 = static_cast<const float*>(h->w.w_down);
@@ -807,7 +822,7 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     b.ldo = d;
     ZC_CUDA(zc::launch_simt_gemm(zc::kDown, b, max_mb, s));
   }
-  ZC_CUDA(mark());
+  ZC_CUDA(mark("zcmoe.combine"));
   if (side) {
     ZC_CUDA(cudaEventRecord(side->dn->ev_down, s));
     ZC_CUDA(cudaStreamWaitEvent(side->dn->side, side->dn->ev_down, 0));
@@ -821,7 +836,7 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
                                h->mb_off));
   else
     ZC_CUDA(zc::launch_combine(h->bf16, x, h->Y, h->idx, h->gate, h->pos, Ti, k, N, d, y, h->sms, s));
-  ZC_CUDA(mark());
+  ZC_CUDA(mark(nullptr));
   if (side) ZC_CUDA(cudaStreamWaitEvent(s, side->dn->ev_join, 0));
 
   if (dbg) {
