@@ -97,6 +97,14 @@ def lib():
         L.zo_quantize_mx4.restype = None
         L.zo_ffn_fp4_f64.argtypes = [vp, i32, i64, U8P, U8P, U8P, U8P, U8P, U8P, i32, i32, F64P]
         L.zo_ffn_fp4_f64.restype = None
+        L.zo_nv4_global.argtypes = [f32]
+        L.zo_nv4_global.restype = f32
+        L.zo_nv4_scale.argtypes = [f32, f32]
+        L.zo_nv4_scale.restype = ctypes.c_uint8
+        L.zo_quantize_nv4.argtypes = [vp, i32, i64, i64, f32, U8P, U8P]
+        L.zo_quantize_nv4.restype = None
+        L.zo_ffn_nv4_f64.argtypes = [vp, i32, i64, U8P, U8P, f32, U8P, U8P, f32, U8P, U8P, f32, i32, i32, F64P]
+        L.zo_ffn_nv4_f64.restype = None
         L.zo_layer_bwd_f64.argtypes = [vp, i32, i64, i32, i32, i32, i32, i32, vp, vp, vp, vp, i32, I32P, F64P, f64,
                                        F64P, F64P, vp, vp, vp, vp]
         L.zo_layer_bwd_f64.restype = None
@@ -212,13 +220,15 @@ def layer(x, idx, gate, N, wg, wu, wd):
     return y
 
 
-def layer_outputs(x_rows, idx, gate, N, expert_weights, fp8=False, expert_fn=None, fp4=False):
+def layer_outputs(x_rows, idx, gate, N, expert_weights, fp8=False, expert_fn=None, fp4=False, nv4=False):
     """fp64 layer output for a few tokens when the expert weights are fetched one
     expert at a time.  ``expert_weights(e) -> (wg, wu, wd)``.  Sums
     g * F_e(x) over the token's FFN slots plus (sum of zero-slot gates) * x.
     fp8: F_e is the block-scaled FP8 expert (ffn_fp8) on weights quantized here
     per [128,128].  fp4: the MXFP4 expert (ffn_fp4) on weights quantized here per
-    [1,32].  expert_fn(e, rows) -> F_e(rows), if given, replaces these."""
+    [1,32].  nv4: the NVFP4 expert (ffn_nv4) on weights quantized here per [1,16]
+    with one fp32 scale per matrix.  expert_fn(e, rows) -> F_e(rows), if given,
+    replaces these."""
     x_rows = np.ascontiguousarray(x_rows)
     n, d = x_rows.shape
     xf = x_rows.astype(np.float64) if x_rows.dtype == np.float32 else \
@@ -241,7 +251,10 @@ def layer_outputs(x_rows, idx, gate, N, expert_weights, fp8=False, expert_fn=Non
                 y[r] += float(gate[r, j]) * f[i]
             continue
         wg, wu, wd = expert_weights(e)
-        if fp4:
+        if nv4:
+            q = [quantize_weight_nv4(w) for w in (wg, wu, wd)]
+            f = ffn_nv4(x_rows[rows], [c for c, _, _ in q], [s_ for _, s_, _ in q], [g_ for _, _, g_ in q])
+        elif fp4:
             q = [quantize_mx4(w) for w in (wg, wu, wd)]
             f = ffn_fp4(x_rows[rows], [c for c, _ in q], [s_ for _, s_ in q])
         elif fp8:
@@ -377,6 +390,62 @@ def ffn_fp4(xs, wq, sq):
     inter = wg.shape[0]
     out = np.empty((n, d), np.float64)
     lib().zo_ffn_fp4_f64(xs.ctypes.data, xd, n, wg, sg, wu, su, wd, sd, d, inter, out)
+    return out
+
+
+# ----------------------------------------------------------------- W4A4 as NVFP4
+def nv4_global(amax: float) -> float:
+    """fp32 tensor scale of a weight matrix: fl32(amax / (6 * 448)), 1 for amax 0."""
+    return float(lib().zo_nv4_global(float(amax)))
+
+
+def nv4_scale(amax: float, g: float = 1.0) -> int:
+    """UE4M3 code of the smallest block scale s with amax <= 6 s g (decided in fp32)."""
+    return int(lib().zo_nv4_scale(float(amax), float(g)))
+
+
+def quantize_nv4(src, g=1.0):
+    """(codes [rows, cols/2] uint8, two per byte with the even element low; scales
+    [rows, cols/16] uint8 UE4M3) of a 2-D fp32 array or bf16 bit array, tensor scale g."""
+    src, dt = _arr(src)
+    rows, cols = src.shape
+    if cols % 16:
+        raise ValueError("cols must be a multiple of 16")
+    codes = np.empty((rows, cols // 2), np.uint8)
+    scales = np.empty((rows, cols // 16), np.uint8)
+    lib().zo_quantize_nv4(src.ctypes.data, dt, rows, cols, float(g), codes, scales)
+    return codes, scales
+
+
+def dequantize_nv4(codes, scales, g=1.0):
+    table = np.array([e2m1_decode(c) for c in range(16)], np.float64)
+    lo, hi = table[codes & 0xF], table[codes >> 4]
+    vals = np.empty((codes.shape[0], codes.shape[1] * 2), np.float64)
+    vals[:, 0::2], vals[:, 1::2] = lo, hi
+    s = np.array([e4m3_decode(int(c)) for c in range(256)], np.float64)[scales]
+    return vals * np.repeat(s, 16, axis=1) * float(g)
+
+
+def quantize_weight_nv4(w):
+    """A weight matrix's NVFP4 form: (codes, scales, g) with g from its largest magnitude."""
+    w_arr, _ = _arr(w)
+    vals = (w_arr.astype(np.uint32) << 16).view(np.float32) if w_arr.dtype == np.uint16 else w_arr
+    g = nv4_global(float(np.abs(vals).max()) if vals.size else 0.0)
+    codes, scales = quantize_nv4(w, g)
+    return codes, scales, g
+
+
+def ffn_nv4(xs, wq, sq, gq):
+    """fp64 SwiGLU expert on NVFP4 operands: xs [n, d] quantized per [1,16] inside (g = 1);
+    wq = (wg, wu, wd) packed codes, sq = their [1,16] UE4M3 scales, gq = their fp32 scales."""
+    xs, xd = _arr(xs)
+    n, d = xs.shape
+    wg, wu, wd = (np.ascontiguousarray(w, np.uint8) for w in wq)
+    sg, su, sd = (np.ascontiguousarray(s_, np.uint8) for s_ in sq)
+    inter = wg.shape[0]
+    out = np.empty((n, d), np.float64)
+    lib().zo_ffn_nv4_f64(xs.ctypes.data, xd, n, wg, sg, float(gq[0]), wu, su, float(gq[1]), wd, sd, float(gq[2]),
+                         d, inter, out)
     return out
 
 

@@ -633,6 +633,117 @@ ZO_EXPORT void zo_ffn_fp4_f64(const void *xs, int x_dtype, int64_t n, const uint
 }
 
 /* ------------------------------------------------------------------------- */
+/* W4A4 as NVFP4 (the survey's name for the 4-bit format): E2M1 codes as in   */
+/* MXFP4; one scale per 16 consecutive elements along the reduction dimension, */
+/* an unsigned E4M3 value (UE4M3: the positive E4M3 values, 2^-9 .. 448); and  */
+/* one fp32 scale g per tensor.  Reading (the pages name no format):           */
+/*  - block scale: the smallest UE4M3 value s with amax <= 6 s g, decided in   */
+/*    fp32: t = fl32(amax / fl32(6 g)), s = the smallest code value >= t (448  */
+/*    at most); an all-zero block takes 1.0;                                   */
+/*  - codes: e2m1(fl32(x * fl32(1 / fl32(s g)))), round to nearest even,       */
+/*    saturating at 6;                                                         */
+/*  - g: weights, one per expert matrix, fl32(amax(matrix) / 2688) (so the     */
+/*    largest block scale is 448; 1 for an all-zero matrix); activations (x    */
+/*    rows, silu(g)*u rows) g = 1: their magnitudes sit inside UE4M3's range.  */
+/* Value = e2m1 * s * g.  Pinned in tests/test_oracle_pins.py.                 */
+/* ------------------------------------------------------------------------- */
+
+ZO_EXPORT float zo_nv4_global(float amax) {
+  if (!(amax > 0.0f)) return 1.0f;
+  const float r = amax / 2688.0f; /* 6 * 448, one fp32 division */
+  return r;
+}
+
+ZO_EXPORT uint8_t zo_nv4_scale(float amax, float g) {
+  if (!(amax > 0.0f)) return 0x38; /* 1.0 */
+  const float six_g = 6.0f * g;
+  const float t = amax / six_g;
+  for (int c = 1; c <= 0x7E; ++c)
+    if ((float)zo_e4m3_decode((uint8_t)c) >= t) return (uint8_t)c;
+  return 0x7E; /* 448 */
+}
+
+/* src [rows, cols] (dtype 0 fp32, 1 bf16 bits), cols a multiple of 16; g the tensor's
+   fp32 scale.  codes [rows, cols/2] (two per byte, even element low); scales
+   [rows, cols/16] UE4M3 bytes. */
+ZO_EXPORT void zo_quantize_nv4(const void *src, int dtype, int64_t rows, int64_t cols, float g, uint8_t *codes,
+                               uint8_t *scales) {
+  const int64_t nb = cols / 16;
+#pragma omp parallel for schedule(static) if (rows * cols > (1 << 20))
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < nb; ++b) {
+      double amax = 0.0;
+      for (int64_t c = b * 16; c < b * 16 + 16; ++c) {
+        const double a = fabs(elem(src, dtype, r * cols + c));
+        if (a > amax) amax = a;
+      }
+      const uint8_t sc = zo_nv4_scale((float)amax, g);
+      scales[r * nb + b] = sc;
+      const float sg = (float)zo_e4m3_decode(sc) * g;
+      const float inv = 1.0f / sg;
+      for (int64_t c = b * 16; c < b * 16 + 16; c += 2) {
+        const uint8_t lo = zo_e2m1_encode((float)elem(src, dtype, r * cols + c) * inv);
+        const uint8_t hi = zo_e2m1_encode((float)elem(src, dtype, r * cols + c + 1) * inv);
+        codes[r * (cols / 2) + c / 2] = (uint8_t)(lo | (hi << 4));
+      }
+    }
+}
+
+static double nv4_value(const uint8_t *codes, const uint8_t *scales, int64_t cols, int64_t r, int64_t c,
+                        const double *tab) {
+  const uint8_t byte = codes[r * (cols / 2) + c / 2];
+  const uint8_t code = (c & 1) ? (byte >> 4) : (byte & 0xF);
+  return tab[code] * zo_e4m3_decode(scales[r * (cols / 16) + c / 16]);
+}
+
+/* FFN expert on NVFP4 operands, fp64 arithmetic on the dequantized values.  Each
+   row of xs is quantized per [1,16] here with g = 1; wg, wu [inter, d] and wd
+   [d, inter] come as codes + UE4M3 scales ([1,16] along each row) and their
+   matrices' fp32 scales gg, gu, gd.  h = silu(g) * u is rounded to fp32 and
+   quantized per [1,16] (g = 1) before the down projection.  out [n, d] fp64. */
+ZO_EXPORT void zo_ffn_nv4_f64(const void *xs, int x_dtype, int64_t n, const uint8_t *wg, const uint8_t *sg, float gg,
+                              const uint8_t *wu, const uint8_t *su, float gu, const uint8_t *wd, const uint8_t *sd,
+                              float gd, int d, int inter, double *out) {
+  const size_t xsz = (x_dtype == 1) ? 2 : 4;
+  double tab[16];
+  for (int c = 0; c < 16; ++c) tab[c] = zo_e2m1_decode((uint8_t)c);
+  uint8_t *xq = (uint8_t *)malloc((size_t)d / 2), *xsc = (uint8_t *)malloc((size_t)d / 16);
+  uint8_t *hq = (uint8_t *)malloc((size_t)inter / 2), *hsc = (uint8_t *)malloc((size_t)inter / 16);
+  double *xv = (double *)malloc(sizeof(double) * (size_t)d), *hv = (double *)malloc(sizeof(double) * (size_t)inter);
+  float *h32 = (float *)malloc(sizeof(float) * (size_t)inter);
+  for (int64_t r = 0; r < n; ++r) {
+    zo_quantize_nv4((const char *)xs + (size_t)(r * d) * xsz, x_dtype, 1, d, 1.0f, xq, xsc);
+    for (int c = 0; c < d; ++c) xv[c] = nv4_value(xq, xsc, d, 0, c, tab);
+#pragma omp parallel for schedule(static)
+    for (int i = 0; i < inter; ++i) {
+      double g = 0.0, u = 0.0;
+      for (int c = 0; c < d; ++c) {
+        g += nv4_value(wg, sg, d, i, c, tab) * xv[c];
+        u += nv4_value(wu, su, d, i, c, tab) * xv[c];
+      }
+      g *= (double)gg;
+      u *= (double)gu;
+      h32[i] = (float)(g / (1.0 + exp(-g)) * u);
+    }
+    zo_quantize_nv4(h32, 0, 1, inter, 1.0f, hq, hsc);
+    for (int i = 0; i < inter; ++i) hv[i] = nv4_value(hq, hsc, inter, 0, i, tab);
+#pragma omp parallel for schedule(static)
+    for (int c = 0; c < d; ++c) {
+      double acc = 0.0;
+      for (int i = 0; i < inter; ++i) acc += nv4_value(wd, sd, inter, c, i, tab) * hv[i];
+      out[r * d + c] = acc * (double)gd;
+    }
+  }
+  free(xq);
+  free(xsc);
+  free(hq);
+  free(hsc);
+  free(xv);
+  free(hv);
+  free(h32);
+}
+
+/* ------------------------------------------------------------------------- */
 /* Backward pass (training), fp64.                                            */
 /* LongCat-Flash technical summary (zhangjingwei.cn), 五 訓練基礎設施: the MoE   */
 /* layer trains with a deterministic ScatterAdd and a fused GemmAdd (the fp32  */

@@ -50,6 +50,16 @@ MUTANTS = [
      "static float key32(float v) { return v; }", 0),
     ("replica max starts at the first logit", "float m = -INFINITY;\n    for (int e = 0; e < E; ++e)\n      if (lt[e] > m) m = lt[e];",
      "float m = lt[0];\n    for (int e = 1; e < E; ++e)\n      if (lt[e] > m) m = lt[e];", 0),
+    ("NVFP4 block scale rounds past an exact fit", "if ((float)zo_e4m3_decode((uint8_t)c) >= t) return (uint8_t)c;",
+     "if ((float)zo_e4m3_decode((uint8_t)c) > t) return (uint8_t)c;", 0),
+    ("NVFP4 tensor scale for 448 instead of 6 * 448", "const float r = amax / 2688.0f;", "const float r = amax / 448.0f;", 0),
+    ("NVFP4 W_d tensor scale dropped", "out[r * d + c] = acc * (double)gd;", "out[r * d + c] = acc;", 0),
+    ("NVFP4 gate and up tensor scales swapped", "g *= (double)gg;\n      u *= (double)gu;",
+     "g *= (double)gu;\n      u *= (double)gg;", 0),
+    ("NVFP4 scale read for blocks of 32", "return tab[code] * zo_e4m3_decode(scales[r * (cols / 16) + c / 16]);",
+     "return tab[code] * zo_e4m3_decode(scales[r * (cols / 16) + c / 32]);", 0),
+    ("NVFP4 codes scaled without the tensor scale", "const float sg = (float)zo_e4m3_decode(sc) * g;",
+     "const float sg = (float)zo_e4m3_decode(sc);", 0),
     ("replica sum tree reads its own partial", "nxt[p] = part[p] + part[p ^ w];", "nxt[p] = part[p] + part[p];", 0),
     ("replica max not subtracted", "u[e] = zo_zexp(lt[e] - m);", "u[e] = zo_zexp(lt[e]);", 0),
     ("zexp coefficient 1/3! wrong", "0x1.555556p-3f);  /* 1/3! */", "0x1.555556p-2f);  /* 1/3! */", 0),

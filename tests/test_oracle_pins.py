@@ -824,6 +824,124 @@ def test_ffn_fp4_is_close_to_the_unquantized_expert():
     assert 1e-3 < rel.max() < 0.35, rel
 
 
+# ---------------------------------------------------------------- W4A4 as NVFP4
+def _e4m3_round_up(t):
+    """The smallest finite E4M3 value >= t, through torch's float8 conversion (a library
+    routine: round to nearest, then one code up if that fell below t)."""
+    import torch
+    t = np.float32(t)
+    v = torch.tensor([t], dtype=torch.float32).to(torch.float8_e4m3fn)
+    code = int(v.view(torch.uint8).item())
+    if float(v.to(torch.float32).item()) < t:
+        code += 1
+    return min(code, 0x7E)
+
+
+def test_nv4_scale_against_library_e4m3_rounding():
+    """The block scale is the smallest UE4M3 value s with amax <= 6 s g, decided in fp32
+    (t = fl32(amax / fl32(6 g))): the same as rounding t up through torch's float8 E4M3."""
+    rng = np.random.default_rng(61)
+    amax = (rng.uniform(0.5, 1.0, 2000) * np.exp2(rng.integers(-12, 12, 2000))).astype(np.float32)
+    gs = np.concatenate([np.ones(1000, np.float32), (rng.uniform(0.5, 1, 1000) * 2.0 ** -8).astype(np.float32)])
+    for a, g in zip(amax, gs):
+        t = np.float32(a) / (np.float32(6.0) * np.float32(g))
+        want = 0x7E if t > 448 else _e4m3_round_up(t)
+        assert oracle.nv4_scale(float(a), float(g)) == want, (a, g)
+        s = oracle.e4m3_decode(want)
+        if t <= 448:
+            assert a <= 6 * s * g * (1 + 2 ** -20)          # no saturation
+    assert oracle.nv4_scale(0.0, 1.0) == 0x38                   # an all-zero block: 1.0
+    assert oracle.nv4_scale(6.0, 1.0) == 0x38 and oracle.e4m3_decode(0x38) == 1.0
+    assert oracle.nv4_scale(1e9, 1.0) == 0x7E                   # saturates at 448
+
+
+def test_nv4_global_makes_the_largest_block_scale_448():
+    rng = np.random.default_rng(62)
+    for std in (0.006, 0.5, 30.0):
+        w = (rng.standard_normal((8, 64)) * std).astype(np.float32)
+        c, s_, g = oracle.quantize_weight_nv4(w)
+        assert g == np.float32(np.abs(w).max()) / np.float32(2688.0)
+        assert s_.max() == 0x7E                                  # the block holding the matrix amax
+        assert oracle.e4m3_decode(int(s_.max())) == 448.0
+    assert oracle.nv4_global(0.0) == 1.0
+
+
+def test_quantize_nv4_bound_and_packing():
+    rng = np.random.default_rng(63)
+    x = (rng.standard_normal((5, 96)) * np.exp2(rng.integers(-4, 4, (5, 1)))).astype(np.float32)
+    for g in (1.0, 2.0 ** -6):
+        codes, scales = oracle.quantize_nv4(x, g)
+        assert codes.shape == (5, 48) and scales.shape == (5, 6)
+        deq = oracle.dequantize_nv4(codes, scales, g)
+        s = np.repeat(np.array([oracle.e4m3_decode(int(c)) for c in scales.ravel()]).reshape(scales.shape), 16, 1) * g
+        v = x.astype(np.float64) / s
+        assert np.abs(v).max() <= 6.0 * (1 + 2 ** -20)
+        spacing = np.where(np.abs(v) < 1.0, 0.5, np.exp2(np.floor(np.log2(np.maximum(np.abs(v), 1.0))) - 1))
+        assert np.all(np.abs(v - deq / s) <= spacing / 2 * (1 + 2 ** -20) + 2 ** -20)
+    y = np.zeros((1, 16), np.float32)
+    y[0, :2] = [6.0, 1.0]                                        # scale 1.0: codes 6 -> 0x7, 1 -> 0x2
+    c, sc = oracle.quantize_nv4(y)
+    assert sc[0, 0] == 0x38 and c[0, 0] == (0x7 | (0x2 << 4))
+
+
+def test_ffn_nv4_lossless_closed_form():
+    """Values that quantize exactly at tensor scale 1.  A 6 in each block sets its scale
+    to 1.0 (x = [6, 0..]; W_g row 0 = [4, 6, 0..]; W_u row 0 = [1, 6, 0..]; every W_d row
+    = [v, 6, 0..] with v an E2M1 value), so g = 24, u = 6 and h = silu(24) * 6 rounds to
+    144 in fp32; h's block holds 144 alone, its scale 24 is an E4M3 value and its code 6.
+    Then y = 144 * W_d[:, 0] exactly, and a tensor scale on W_d multiplies y."""
+    d = inter = 64
+    x = np.zeros((1, d), np.float32)
+    x[0, 0] = 6.0
+    wg = np.zeros((inter, d), np.float32)
+    wu = np.zeros((inter, d), np.float32)
+    wg[0, :2] = [4.0, 6.0]
+    wu[0, :2] = [1.0, 6.0]
+    wd = np.zeros((d, inter), np.float32)
+    wd[:, 0] = np.resize([6.0, -3.0, 1.5, -0.5, 0.0, 4.0, -2.0, 1.0], d)
+    wd[:, 1] = 6.0
+    q = [oracle.quantize_nv4(w, 1.0) for w in (wg, wu, wd)]
+    for (c, s_), w in zip(q, (wg, wu, wd)):
+        assert np.array_equal(oracle.dequantize_nv4(c, s_, 1.0), w)      # lossless
+    codes, scales = [c for c, _ in q], [s_ for _, s_ in q]
+    y = oracle.ffn_nv4(x, codes, scales, [1.0, 1.0, 1.0])
+    assert np.array_equal(y[0], 144.0 * wd[:, 0].astype(np.float64))
+    assert np.array_equal(oracle.ffn_nv4(x, codes, scales, [1.0, 1.0, 0.5])[0], 72.0 * wd[:, 0].astype(np.float64))
+
+
+def test_ffn_nv4_equals_matmuls_on_the_quantized_operands():
+    """The NVFP4 expert restated with library matmuls over the separately pinned
+    quantizers: operand rows per [1,16] (x and H at g = 1, weights at their matrix
+    scale), H rounded to fp32 first."""
+    rng = _rng(64)
+    n, d, inter = 6, 128, 192
+    x = _blocky(rng, n, d, 1, 16)
+    wg, wu = _blocky(rng, inter, d, 1, 16, 0.05), _blocky(rng, inter, d, 1, 16, 0.05)
+    wd = _blocky(rng, d, inter, 1, 16, 0.05)
+    q = [oracle.quantize_weight_nv4(m) for m in (wg, wu, wd)]
+    Wg, Wu, Wd = (oracle.dequantize_nv4(c, s_, g) for c, s_, g in q)
+    y = oracle.ffn_nv4(x, [c for c, _, _ in q], [s_ for _, s_, _ in q], [g for _, _, g in q])
+    xq = oracle.dequantize_nv4(*oracle.quantize_nv4(x))
+    g_, u = xq @ Wg.T, xq @ Wu.T
+    h32 = (g_ / (1.0 + np.exp(-g_)) * u).astype(np.float32)
+    want = oracle.dequantize_nv4(*oracle.quantize_nv4(h32)) @ Wd.T
+    np.testing.assert_allclose(y, want, rtol=1e-9, atol=1e-12 * np.abs(want).max())
+
+
+def test_ffn_nv4_is_close_to_the_unquantized_expert():
+    rng = np.random.default_rng(65)
+    d, inter = 256, 384
+    x = rng.standard_normal((4, d)).astype(np.float32)
+    wg = (rng.standard_normal((inter, d)) * 0.06).astype(np.float32)
+    wu = (rng.standard_normal((inter, d)) * 0.06).astype(np.float32)
+    wd = (rng.standard_normal((d, inter)) * 0.05).astype(np.float32)
+    q = [oracle.quantize_weight_nv4(w) for w in (wg, wu, wd)]
+    y4 = oracle.ffn_nv4(x, [c for c, _, _ in q], [s_ for _, s_, _ in q], [g for _, _, g in q])
+    y = oracle.ffn(x, wg, wu, wd)
+    rel = np.abs(y4 - y).max(axis=1) / np.abs(y).max(axis=1)
+    assert 1e-3 < rel.max() < 0.45, rel
+
+
 # ---------------------------------------------------------------- backward (oracle only)
 
 def _tiny_fwd_loss(x, wr, wg, wu, wd, bias, dy, N, k, scale, offset):
