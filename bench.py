@@ -147,9 +147,10 @@ def algorithmic_work(wl, P, distinct):
     """FLOPs and bytes per forward from the realised routing: P FFN pairs and
     `distinct` FFN experts hit.  F = 2 T d E + 6 d inter P;
     B = distinct * 3 d inter * w + E d * 2 + 2 T d * 2 (bf16; expert weights w = 2
-    bytes, or 1 for FP8 experts; fp32 layers 4 throughout)."""
+    bytes per element, 1 for FP8 experts, 0.5 + 1/32 for MXFP4 (codes + one scale byte
+    per 32) and 0.5 + 1/16 for NVFP4 (one per 16); fp32 layers 4 throughout)."""
     esz = 4 if wl.dtype == "f32" else 2
-    wsz = {"fp8": 1, "fp4": 0.5}.get(wl.dtype, esz)
+    wsz = {"fp8": 1, "fp4": 0.5 + 1 / 32, "nvfp4": 0.5 + 1 / 16}.get(wl.dtype, esz)
     F = 2.0 * wl.T * wl.d * wl.E + 6.0 * wl.d * wl.inter * P
     B = distinct * 3.0 * wl.d * wl.inter * wsz + wl.E * wl.d * esz + 2.0 * wl.T * wl.d * esz
     return F, B
@@ -160,7 +161,7 @@ def roofline_ms(wl, F, B, peaks):
     nominal 4.5 / 2.25 PFLOP/s ratio), the router in bf16."""
     p = peaks["bf16_tflops_sustained"] * 1e12
     f_router = 2.0 * wl.T * wl.d * wl.E
-    mult = {"fp8": 2, "fp4": 4}.get(wl.dtype, 1)
+    mult = {"fp8": 2, "fp4": 4, "nvfp4": 4}.get(wl.dtype, 1)
     t_tensor = f_router / p + (F - f_router) / (mult * p)
     return 1e3 * max(t_tensor, B / (peaks["hbm_gbs"] * 1e9))
 
@@ -193,6 +194,10 @@ def cpu_oracle_sample(wl, weights, x, bias, offset, n_tokens, min_s=10.0):
     elif wl.dtype == "fp4":
         q4 = {e: [oracle.quantize_mx4(w) for w in cache[e]] for e in need}
         efn = lambda e, rows: oracle.ffn_fp4(rows, [c for c, _ in q4[e]], [s_ for _, s_ in q4[e]])
+    elif wl.dtype == "nvfp4":
+        qn = {e: [oracle.quantize_weight_nv4(w) for w in cache[e]] for e in need}
+        efn = lambda e, rows: oracle.ffn_nv4(rows, [c for c, _, _ in qn[e]], [s_ for _, s_, _ in qn[e]],
+                                             [g_ for _, _, g_ in qn[e]])
     done = 0
     t0 = time.perf_counter()
     while True:  # the sample is processed again until the time budget is spent
@@ -547,7 +552,7 @@ def main():
     ap.add_argument("--impl", default="zcmoe", choices=["zcmoe", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
-    ap.add_argument("--secondary", default="decode,fp8,fp4,backward,overlap",
+    ap.add_argument("--secondary", default="decode,fp8,fp4,nvfp4,backward,overlap",
                     help="comma list of the secondary measurements to run after the headline")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism over the GPUs (ep.py) instead of data-parallel replicas")
@@ -556,7 +561,7 @@ def main():
                     help="launch every step eagerly instead of replaying one captured CUDA graph (N=1)")
     args = ap.parse_args()
     sec = set() if args.no_secondary else {s_.strip() for s_ in args.secondary.split(",") if s_.strip()}
-    unknown = sec - {"decode", "fp8", "fp4", "backward", "overlap"}
+    unknown = sec - {"decode", "fp8", "fp4", "nvfp4", "backward", "overlap"}
     if unknown:
         ap.error(f"unknown secondary measurement(s): {sorted(unknown)}")
     if args.warmup < 3:
@@ -673,8 +678,8 @@ def main():
     stage_avg = {s: v / nf for s, v in stage_ms.items()}
     gu_ms = stage_avg["gate_up"]
     gu_flops = 4.0 * wl.d * wl.inter * P
-    fp8 = wl.dtype in ("fp8", "fp4")
-    mult = {"fp8": 2, "fp4": 4}.get(wl.dtype, 1)
+    fp8 = wl.dtype in ("fp8", "fp4", "nvfp4")
+    mult = {"fp8": 2, "fp4": 4, "nvfp4": 4}.get(wl.dtype, 1)
     tensor_peak = peaks["bf16_tflops_sustained"] * mult
     achieved = gu_flops / (gu_ms * 1e-3) / 1e12
     kname = (f"grouped {wl.dtype.upper()} gate/up GEMM + SwiGLU + quantize (k_fp8_gemm<1>)" if fp8
@@ -792,7 +797,7 @@ def main():
 
     # secondary: the same layer with block-scaled FP8 experts (bf16 headline unchanged)
     if rank == 0 and ws == 1 and wl.name == "prefill_560b":
-        for fmt in ("fp8", "fp4"):
+        for fmt in ("fp8", "fp4", "nvfp4"):
             if fmt in sec:
                 line[fmt] = measure_lowp(layer, weights, xs[0], stream, peaks, fmt)
 

@@ -52,7 +52,7 @@ extern "C" {
 
 typedef struct zcmoe_s *zcmoe_t;
 
-typedef enum { ZCMOE_F32 = 0, ZCMOE_BF16 = 1, ZCMOE_FP8 = 2, ZCMOE_FP4 = 3 } zcmoe_dtype;
+typedef enum { ZCMOE_F32 = 0, ZCMOE_BF16 = 1, ZCMOE_FP8 = 2, ZCMOE_FP4 = 3, ZCMOE_NVFP4 = 4 } zcmoe_dtype;
 
 /* Layer shape and routing constants.  Sizes are element counts.
  * Limits: 1 <= n_ffn, 0 <= n_zero, E = n_ffn + n_zero <= 1024, 1 <= top_k <= min(E, 32),
@@ -75,7 +75,13 @@ typedef enum { ZCMOE_F32 = 0, ZCMOE_BF16 = 1, ZCMOE_FP8 = 2, ZCMOE_FP4 = 3 } zcm
  *                      format is not named): MXFP4, E2M1 codes with one E8M0 scale
  *                      (the smallest 2^E with block max <= 6 * 2^E) per 32 elements
  *                      along the reduction dimension of x, silu(g)*u and every weight
- *                      row.  Needs d a multiple of 512 and inter a multiple of 256. */
+ *                      row.  Needs d a multiple of 512 and inter a multiple of 256;
+ *        ZCMOE_NVFP4 -> the same W4A4 experts in NVFP4: E2M1 codes with one UE4M3
+ *                      scale (an unsigned E4M3 value) per 16 elements along the
+ *                      reduction dimension and one fp32 scale g per tensor
+ *                      (zcmoe_quantize_nv4 gives the rule): g = amax / 2688 for
+ *                      each expert's W_g, W_u and W_d (computed at create), g = 1
+ *                      for x rows and silu(g)*u rows.  Same shape limits as ZCMOE_FP4. */
 typedef struct {
   int32_t d;            /* hidden size                                   */
   int32_t n_ffn;        /* N, FFN experts                                */
@@ -376,6 +382,26 @@ ZCMOE_API int zcmoe_quantize_e4m3(const void *src, int32_t src_dtype, int64_t ro
  *   device.  Asynchronous on `stream`. */
 ZCMOE_API int zcmoe_quantize_mx4(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, uint8_t *codes,
                                  uint8_t *scales, cudaStream_t stream);
+
+/* NVFP4 quantization, the rule ZCMOE_NVFP4 layers use: value = e2m1 * s * g, with E2M1
+ * codes as in zcmoe_quantize_mx4, one UE4M3 block scale s per 16 consecutive elements
+ * of a row and one fp32 tensor scale g.  s is the smallest positive E4M3 value with
+ * the block's largest magnitude amax <= 6 s g, decided in fp32 on
+ * t = fl32(amax / fl32(6 g)) (448 at most; 1.0 for an all-zero block); the codes are
+ * e2m1(fl32(x * fl32(1 / fl32(s g)))), round to nearest even, saturating at 6.
+ * The pages report W4A4 without naming a format; this two-level scale is the
+ * NVFP4 reading, kept beside MXFP4.  No handle needed.
+ *   src [rows, cols] device, ZCMOE_BF16 or ZCMOE_F32, 16-byte aligned; cols a
+ *   positive multiple of 256;
+ *   global_scale: g > 0 (finite) to quantize under that scale (activations use 1);
+ *   0 to derive it as the layer does for a weight matrix, g = fl32(amax(src) / 2688)
+ *   (so the largest block scale is 448; 1 for an all-zero tensor), written to
+ *   global_out (one float, device, required then; ignored otherwise);
+ *   codes [rows, cols / 2] uint8 device, two codes per byte with the even element in
+ *   the low nibble; scales [rows, cols / 16] uint8 device (E4M3 bytes).
+ *   Asynchronous on `stream`. */
+ZCMOE_API int zcmoe_quantize_nv4(const void *src, int32_t src_dtype, int64_t rows, int64_t cols, float global_scale,
+                                 uint8_t *codes, uint8_t *scales, float *global_out, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * Dense FFN path and the shortcut-connected overlap (ScMoE).

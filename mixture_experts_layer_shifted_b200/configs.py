@@ -24,7 +24,7 @@ class Workload:
     inter: int
     n_zero: int
     top_k: int
-    dtype: str            # "f32", "bf16", "fp8" or "fp4" (bf16 interface, block-scaled FP8 / MXFP4 experts)
+    dtype: str            # "f32", "bf16", "fp8", "fp4" or "nvfp4" (bf16 interface; FP8 / MXFP4 / NVFP4 experts)
     x_std: float = 1.0
     w_std: float = 0.02
     bias: tuple = ("zero",)   # ("zero",) | ("uniform", lo, hi) | ("zero_experts", value)
@@ -40,7 +40,7 @@ class Workload:
         return self.n_ffn + self.n_zero
 
     def weight_bytes(self):
-        esz = 4 if self.dtype == "f32" else 2  # the caller's weights (bf16 also for fp8 / fp4 layers)
+        esz = 4 if self.dtype == "f32" else 2  # the caller's weights (bf16 also for fp8 / fp4 / nvfp4 layers)
         return (3 * self.n_ffn * self.inter * self.d + self.E * self.d) * esz
 
     def with_(self, **kw):
@@ -78,9 +78,9 @@ WORKLOADS = {
     "bwd_probe": Workload("bwd_probe", T=1024, d=6144, n_ffn=16, inter=2048, n_zero=8, top_k=12, dtype="bf16",
                           w_std=0.006, bias=("zero",)),
 }
-# the same layers with block-scaled FP8 and W4A4 (MXFP4) experts
+# the same layers with block-scaled FP8 and W4A4 (MXFP4, NVFP4) experts
 for _name in ("small_bf16", "prefill_560b", "decode_560b", "skewed_4096", "prefill_probe"):
-    for _dt in ("fp8", "fp4"):
+    for _dt in ("fp8", "fp4", "nvfp4"):
         _n = _name.replace("_bf16", "") + "_" + _dt
         WORKLOADS[_n] = WORKLOADS[_name].with_(name=_n, dtype=_dt)
 

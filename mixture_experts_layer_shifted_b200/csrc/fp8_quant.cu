@@ -3,6 +3,9 @@
 //   k_quant_tiles : [128,128] blocks (weights), one CTA per block
 //   k_gather_quant: the FFN pairs' token rows, quantized per [1,128] on the way
 //                   into the expert-sorted operand of the FP8 gate/up GEMM
+// and their W4A4 forms: MXFP4 ([1,32] blocks, k_quant_mx4 / k_gather_quant4) and
+// NVFP4 ([1,16] blocks with a tensor scale: k_matrix_amax + k_nv4_global, then
+// k_quant_nv4 / k_gather_quant_nv4).
 // Scales go out either plain ([row blocks, cols/128], for zcmoe_quantize_e4m3)
 // or as the GEMM's scale atoms.
 #include <cuda_bf16.h>
@@ -255,6 +258,120 @@ __global__ void __launch_bounds__(256) k_gather_quant4(const __nv_bfloat16* __re
   }
 }
 
+// ---------------------------------------------------------------- NVFP4 ([1,16] blocks, two-level scale)
+// The eight values of one lane, its 16-element block shared with the neighbouring lane,
+// under tensor scale g: the lane's packed codes (x) and the block's UE4M3 code (y).
+__device__ __forceinline__ uint2 quant8_nv4(const float* v, float g) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  const uint32_t code = nv4_code(a, g);
+  return make_uint2(pack_e2m1x8(v, nv4_inverse(code, g)), code);
+}
+
+// Largest magnitude of each of `nmat` matrices of `mrows` rows x cols (consecutive in src):
+// amax_bits[m] (zeroed by the caller) receives it as fp32 bits.  grid (x, nmat).
+template <typename TIN>
+__global__ void __launch_bounds__(256) k_matrix_amax(const TIN* __restrict__ src, int64_t mrows, int cols,
+                                                     uint32_t* __restrict__ amax_bits) {
+  __shared__ float part[8];
+  const int64_t n = mrows * cols;  // a multiple of 8
+  const TIN* base = src + (int64_t)blockIdx.y * n;
+  float a = 0.0f;
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; i < n; i += (int64_t)gridDim.x * blockDim.x * 8) {
+    float v[8];
+    ld8(base + i, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[j]));
+  }
+  a = warp_max(a);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < 8; ++w) a = fmaxf(a, part[w]);
+    atomicMax(amax_bits + blockIdx.y, __float_as_uint(a));  // non-negative floats order as their bits
+  }
+}
+
+// amax (as bits) -> the tensor scale g = fl32(amax / 2688) (1 for an all-zero matrix), in place.
+__global__ void k_nv4_global(uint32_t* __restrict__ v, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    const float a = __uint_as_float(v[i]);
+    v[i] = __float_as_uint(a > 0.0f ? __fdiv_rn(a, 2688.0f) : 1.0f);
+  }
+}
+
+// src [rows, cols] -> codes [rows, cols/2], scales plain [rows, cols/16] or atoms
+// (groups = ceil(cols/64)); row r takes tensor scale gvec[r / rows_per_g] (g_const when gvec
+// is null).  cols a multiple of 256; one warp per 256 elements.
+template <typename TIN, bool ATOM>
+__global__ void __launch_bounds__(256) k_quant_nv4(const TIN* __restrict__ src, int64_t rows, int cols,
+                                                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                   int groups, const float* __restrict__ gvec, int64_t rows_per_g,
+                                                   float g_const) {
+  const int lane = threadIdx.x & 31;
+  const int nch = cols >> 8;
+  const int64_t nwork = rows * nch;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < nwork; i += nwarps) {
+    const int64_t r = i / nch;
+    const int c = (int)(i - r * nch) * 256 + lane * 8;
+    const float g = gvec ? gvec[r / rows_per_g] : g_const;
+    float v[8];
+    ld8(src + r * cols + c, v);
+    const uint2 q = quant8_nv4(v, g);
+    *reinterpret_cast<uint32_t*>(codes + r * (cols >> 1) + (c >> 1)) = q.x;
+    if ((lane & 1) == 0) scales[ATOM ? atom_offset(r, c >> 4, groups) : r * (cols >> 4) + (c >> 4)] = (uint8_t)q.y;
+  }
+}
+
+// NVFP4 form of k_gather_quant (same padded rows, g = 1); d a multiple of 512.
+__global__ void __launch_bounds__(256) k_gather_quant_nv4(const __nv_bfloat16* __restrict__ x, int d,
+                                                          const int32_t* __restrict__ perm,
+                                                          const int32_t* __restrict__ idx, int k,
+                                                          const int32_t* __restrict__ offsets,
+                                                          const int32_t* __restrict__ mb_off,
+                                                          const int32_t* __restrict__ scal, uint8_t* __restrict__ x4,
+                                                          uint8_t* __restrict__ sx, int groups) {
+  const int P = scal[0];
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
+  for (int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); p < P; p += nwarps) {
+    const int pair = perm[p];
+    const int e = idx[pair];
+    const int64_t pad = (int64_t)(p - offsets[e]) + (int64_t)mb_off[e] * 128;
+    const __nv_bfloat16* src = x + (int64_t)(pair / k) * d;
+    uint8_t* dst = x4 + pad * (d >> 1);
+    int c0 = 0;
+    for (; c0 + 1024 <= d; c0 += 1024) {  // four 16-byte loads in flight per lane
+      float v[4][8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) ld8(src + c0 + 256 * u + lane * 8, v[u]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 256 * u + lane * 8;
+        const uint2 q = quant8_nv4(v[u], 1.0f);
+        *reinterpret_cast<uint32_t*>(dst + (c >> 1)) = q.x;
+        if ((lane & 1) == 0) sx[atom_offset(pad, c >> 4, groups)] = (uint8_t)q.y;
+      }
+    }
+    if (c0 < d) {  // d is a multiple of 512: a last 512 columns
+      float v[2][8];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) ld8(src + c0 + 256 * u + lane * 8, v[u]);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int c = c0 + 256 * u + lane * 8;
+        const uint2 q = quant8_nv4(v[u], 1.0f);
+        *reinterpret_cast<uint32_t*>(dst + (c >> 1)) = q.x;
+        if ((lane & 1) == 0) sx[atom_offset(pad, c >> 4, groups)] = (uint8_t)q.y;
+      }
+    }
+  }
+}
+
 // Debug copy: pair p's expert output from its padded row to row p.
 __global__ void __launch_bounds__(256) k_unpad_rows(const uint4* __restrict__ ypad, int row_vecs,
                                                     const int32_t* __restrict__ perm, const int32_t* __restrict__ idx,
@@ -324,6 +441,56 @@ cudaError_t launch_gather_quant4(const void* x, int d, const int32_t* perm, cons
                                  uint8_t* sx, int groups, int sms, cudaStream_t s) {
   k_gather_quant4<<<sms * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), d, perm, idx, k, offsets, mb_off, scal,
                                            x4, sx, groups);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_nv4_global(int bf16, const void* src, int nmat, int64_t mrows, int cols, float* g,
+                              cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(g, 0, (size_t)nmat * sizeof(float), s);
+  if (e != cudaSuccess) return e;
+  int64_t bx = mrows * cols / (256 * 8 * 16);  // ~16 vectors of 8 per thread
+  if (bx < 1) bx = 1;
+  if (bx > 64) bx = 64;
+  const dim3 grid((unsigned)bx, (unsigned)nmat);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(g);
+  if (bf16) k_matrix_amax<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(src), mrows, cols, bits);
+  else k_matrix_amax<float><<<grid, 256, 0, s>>>(static_cast<const float*>(src), mrows, cols, bits);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_nv4_global<<<(nmat + 255) / 256, 256, 0, s>>>(bits, nmat);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_nv4(int bf16, const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
+                             int atom_groups, const float* gvec, int64_t rows_per_g, float g_const, int sms,
+                             cudaStream_t s) {
+  const int64_t warps = rows * (cols / 256);
+  int64_t blocks = (warps + 7) / 8;
+  if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+  if (blocks < 1) blocks = 1;
+  const bool atom = atom_groups > 0;
+  if (bf16) {
+    auto src_ = static_cast<const __nv_bfloat16*>(src);
+    if (atom)
+      k_quant_nv4<__nv_bfloat16, true>
+          <<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, atom_groups, gvec, rows_per_g, g_const);
+    else
+      k_quant_nv4<__nv_bfloat16, false><<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, 0, gvec, rows_per_g, g_const);
+  } else {
+    auto src_ = static_cast<const float*>(src);
+    if (atom)
+      k_quant_nv4<float, true><<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, atom_groups, gvec, rows_per_g, g_const);
+    else
+      k_quant_nv4<float, false><<<(int)blocks, 256, 0, s>>>(src_, rows, cols, codes, scales, 0, gvec, rows_per_g, g_const);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_quant_nv4(const void* x, int d, const int32_t* perm, const int32_t* idx, int k,
+                                    const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x4,
+                                    uint8_t* sx, int groups, int sms, cudaStream_t s) {
+  k_gather_quant_nv4<<<sms * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), d, perm, idx, k, offsets, mb_off,
+                                              scal, x4, sx, groups);
   return cudaGetLastError();
 }
 

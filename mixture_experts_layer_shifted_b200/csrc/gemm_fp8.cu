@@ -9,6 +9,11 @@
 // "量化" -- DeepSeek-V3's [1,128] activation / [128,128] weight blocks; the
 // experts run as one grouped GEMM, "MoEGEMM".)
 //
+// The same kernel runs the W4A4 formats: MXFP4 (kind::mxf4, E8M0 scales per 32
+// elements) and NVFP4 (kind::mxf4nvf4, UE4M3 scales per 16 elements, the
+// weights' per-expert fp32 tensor scales applied to the accumulators), with
+// 256-element k-blocks of packed E2M1 codes (four K=64 MMAs).
+//
 // Tile: 128 rows x 256 columns x 128-deep k-blocks (four K=32 MMAs); E4M3
 // operands in 128-byte-swizzled K-major tiles; one fp32 accumulator of 256
 // TMEM columns (the rest of TMEM holds the scales), drained by eight epilogue
@@ -31,23 +36,32 @@
 namespace zc {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 128, STAGES = 4;
+constexpr int BM = 128, BN = 256, BK = 128;
 constexpr uint32_t A_BYTES = BM * BK;              // 16 KB
 constexpr uint32_t B_BYTES = BN * BK;              // 32 KB
-constexpr uint32_t SF_BYTES = 6 * kAtomBytes;      // per stage: FP8 uses 3 atoms, MXFP4 6
 constexpr uint32_t TILE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 320;
 constexpr int NUM_EPI = 256;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_COL = 256;                   // scale buffers: [256, 304)
+constexpr uint32_t SF_COL = 256;                   // scale buffers: [256, 304) (FP8, MXFP4), [256, 352) (NVFP4)
 constexpr uint32_t STG_BYTES = 32 * 64;           // down epilogue: a 32-row x 32-column bf16 box per warp
-constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES + SF_BYTES) + 8 * STG_BYTES + 256 + 2 * 2 * BM * 4;
+
+// Per format: pipeline depth and scale bytes per stage (FP8 uses 3 atoms of its 6, MXFP4 6,
+// NVFP4 12: one atom per operand 128 rows per K = 64 MMA).
+template <int FMT>
+struct FmtCfg {
+  static constexpr int kStages = FMT == 2 ? 3 : 4;
+  static constexpr uint32_t kSfBytes = (FMT == 2 ? 12 : 6) * kAtomBytes;
+  static constexpr int kSmem = 1024 + kStages * (A_BYTES + B_BYTES + kSfBytes) + 8 * STG_BYTES + 256 + 2 * 2 * BM * 4;
+};
+constexpr int SMEM_BYTES = FmtCfg<0>::kSmem > FmtCfg<2>::kSmem ? FmtCfg<0>::kSmem : FmtCfg<2>::kSmem;
 
 struct Tile {
   int64_t a_row;   // first padded A row (a multiple of 128)
   int rows_valid;  // rows of the tile that belong to the expert
   int b_row;       // first B row
   int n_blk;       // output column tile
+  int grp;         // expert
 };
 
 __device__ __forceinline__ int total_tiles(const Fp8Args& a) { return a.mb_off[a.ngroups] * a.nblocks; }
@@ -65,6 +79,7 @@ __device__ __forceinline__ Tile decode_tile(const Fp8Args& a, int t) {
   const int nmb = a.mb_off[g + 1] - mb0;
   const int local = t - mb0 * a.nblocks;
   Tile ti;
+  ti.grp = g;
   ti.n_blk = local / nmb;
   const int m_blk = local - ti.n_blk * nmb;
   ti.a_row = (int64_t)(mb0 + m_blk) * BM;
@@ -117,6 +132,19 @@ __device__ __forceinline__ uint32_t idesc_mxf4(uint32_t sf) {
   return (sf << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24) |
          (sf << 29);
 }
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t tsfa,
+                                            uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+// kind::mxf4nvf4 with 16-element blocks: E2M1 A and B (packed, K-major), fp32 D, UE4M3
+// scales (bit 23 clear), K = 64; each MMA reads four scale bytes per row (scale-factor id 0).
+__device__ __forceinline__ uint32_t idesc_nvf4() {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
 // TMA store of one staged box at (x, y); completion tracked as a bulk group of this thread.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, const void* src, int x, int y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
@@ -151,12 +179,16 @@ __device__ __forceinline__ bool epi_all(bool ok) {
 }
 
 // FMT 0: FP8 E4M3 with [1,128] / [128,128] scales (128 K per k-block, atoms loaded every
-// fourth k-block); FMT 1: MXFP4 with [1,32] scales (256 K per k-block, six atoms every k-block).
+// fourth k-block); FMT 1: MXFP4 with [1,32] scales (256 K per k-block, six atoms every k-block);
+// FMT 2: NVFP4 with [1,16] UE4M3 scales (256 K per k-block, twelve atoms every k-block) and the
+// weights' per-expert fp32 scales applied to the accumulators in the epilogue.
 template <int MODE, int FMT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_fp8_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmC,
                const Fp8Args args) {
+  constexpr int STAGES = FmtCfg<FMT>::kStages;
+  constexpr uint32_t SF_BYTES = FmtCfg<FMT>::kSfBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -199,7 +231,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int total = total_tiles(args);
-  const int num_k = args.K / (FMT ? 2 * BK : BK);
+  const int num_k = args.K / (FMT ? 2 * BK : BK);  // FP4 k-blocks hold 256 elements (128 bytes)
 
   if (warp == 0) {
     if (lane == 0) {
@@ -222,7 +254,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const bool with_sf = FMT ? true : (kb & 3) == 0;
           uint8_t* a_dst = sA + stage * A_BYTES;
           uint8_t* b_dst = sB + stage * B_BYTES;
-          mbar_expect_tx(&full[stage], TILE_BYTES + (with_sf ? (FMT ? 6u : 3u) * kAtomBytes : 0u));
+          mbar_expect_tx(&full[stage], TILE_BYTES + (with_sf ? (FMT == 2 ? 12u : FMT ? 6u : 3u) * kAtomBytes : 0u));
           tma_load_2d(a_dst, &tmA, kb * BK, (int)ti.a_row, &full[stage]);
           if (MODE == kGateUp) {
             tma_load_2d(b_dst, &tmB0, kb * BK, ti.b_row, &full[stage]);
@@ -245,6 +277,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             bulk_load(sf_dst + 3 * kAtomBytes, sfb_hi + g, kAtomBytes, &full[stage]);
             bulk_load(sf_dst + 4 * kAtomBytes, sfb_lo + g + kAtomBytes, kAtomBytes, &full[stage]);
             bulk_load(sf_dst + 5 * kAtomBytes, sfb_hi + g + kAtomBytes, kAtomBytes, &full[stage]);
+          } else if (FMT == 2) {
+            // K groups 4kb .. 4kb+3 (one per MMA), consecutive in memory: [A][B lo][B hi] x 4 atoms
+            const int64_t g = (int64_t)(4 * kb) * kAtomBytes;
+            bulk_load(sf_dst, sfa + g, 4 * kAtomBytes, &full[stage]);
+            bulk_load(sf_dst + 4 * kAtomBytes, sfb_lo + g, 4 * kAtomBytes, &full[stage]);
+            bulk_load(sf_dst + 8 * kAtomBytes, sfb_hi + g, 4 * kAtomBytes, &full[stage]);
           }
           ++fills;
           if (++stage == STAGES) {
@@ -297,7 +335,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               tc_mma_mxf8(tmem_base, adesc0 + (uint64_t)(stage * (A_BYTES >> 4) + kk * 2),
                           bdesc0 + (uint64_t)(stage * (B_BYTES >> 4) + kk * 2), idesc, (sf << 30) | sfa_t,
                           (sf << 30) | sfb_t, (kb | kk) != 0 ? 1u : 0u);
-          } else {
+          } else if (FMT == 1) {
             // TMEM scales of this k-block: A g0 +0, A g1 +4, B g0 +8 (rows 0..127) / +12 (128..255), B g1 +16 / +20
             const uint32_t buf = tmem_base + SF_COL + 24u * (uint32_t)(kb & 1);
 #pragma unroll
@@ -310,6 +348,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                           bdesc0 + (uint64_t)(stage * (B_BYTES >> 4) + kk * 2), idesc_mxf4(sf),
                           (sf << 30) | (buf + 4 * g), (sf << 30) | (buf + 8 + 8 * g), (kb | kk) != 0 ? 1u : 0u);
             }
+          } else {
+            // TMEM scales of this k-block, one 4-column group per atom: A for MMA kk at +4kk, B at
+            // +16+8kk (rows 0..127) and +20+8kk (rows 128..255)
+            const uint32_t buf = tmem_base + SF_COL + 48u * (uint32_t)(kb & 1);
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+              tc_cp_scales(buf + 4 * a, atom_desc(sd + a * kAtomBytes));
+              tc_cp_scales(buf + 16 + 8 * a, atom_desc(sd + (4 + a) * kAtomBytes));
+              tc_cp_scales(buf + 20 + 8 * a, atom_desc(sd + (8 + a) * kAtomBytes));
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)  // K = 64 each: 32 bytes of the 128-byte rows
+              tc_mma_nvf4(tmem_base, adesc0 + (uint64_t)(stage * (A_BYTES >> 4) + kk * 2),
+                          bdesc0 + (uint64_t)(stage * (B_BYTES >> 4) + kk * 2), idesc_nvf4(), buf + 4 * kk,
+                          buf + 16 + 8 * kk, (kb | kk) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
           if (++stage == STAGES) {
@@ -335,6 +388,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int buf = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const Tile ti = decode_tile<MODE>(args, t);
+      // NVFP4: the weights' tensor scales (gate/up: W_g's and W_u's; down: W_d's)
+      float s0 = 1.0f, s1 = 1.0f;
+      if (FMT == 2) {
+        s0 = __ldg(args.gsc0 + ti.grp);
+        if (MODE == kGateUp) s1 = __ldg(args.gsc1 + ti.grp);
+      }
       const bool got = mbar_wait(tfull, acc_phase, err, 15);
       if (MODE == kGateUp && FMT == 0) {
         if (!epi_all(got)) break;
@@ -357,8 +416,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         float amax = 0.0f, am0 = 0.0f, am1 = 0.0f;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float h0 = silu_mul(__uint_as_float(g0[j]), __uint_as_float(u0[j]));
-          const float h1 = silu_mul(__uint_as_float(g1[j]), __uint_as_float(u1[j]));
+          const float h0 = FMT == 2 ? silu_mul(__uint_as_float(g0[j]) * s0, __uint_as_float(u0[j]) * s1)
+                                    : silu_mul(__uint_as_float(g0[j]), __uint_as_float(u0[j]));
+          const float h1 = FMT == 2 ? silu_mul(__uint_as_float(g1[j]) * s0, __uint_as_float(u1[j]) * s1)
+                                    : silu_mul(__uint_as_float(g1[j]), __uint_as_float(u1[j]));
           g0[j] = __float_as_uint(h0);
           g1[j] = __float_as_uint(h1);
           am0 = fmaxf(am0, fabsf(h0));
@@ -387,6 +448,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               *reinterpret_cast<uint4*>(dst + 16 * q) = v;
               args.out_sf[atom_offset(grow, (col0 >> 5) + q, args.out_groups)] = (uint8_t)code;
             }
+          }
+          acc_phase ^= 1u;
+          buf ^= 1;
+          continue;
+        }
+        if (FMT == 2) {
+          // [1,16] blocks (g = 1): columns [64 half + 16 q, +16) of this H block, q = 0..3
+          const int col0 = ti.n_blk * (BN / 2) + 64 * half;
+          if (row_ok && col0 < args.n_out) {
+            uint8_t* dst = static_cast<uint8_t*>(args.out) + grow * args.ldo + (col0 >> 1);
+            uint32_t w[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t* h = (q < 2 ? g0 : g1) + 16 * (q & 1);
+              float f[16];
+              float am = 0.0f;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                f[i] = __uint_as_float(h[i]);
+                am = fmaxf(am, fabsf(f[i]));
+              }
+              const uint32_t code = nv4_code(am, 1.0f);
+              const float inv = nv4_inverse(code, 1.0f);
+              w[2 * q] = pack_e2m1x8(f, inv);
+              w[2 * q + 1] = pack_e2m1x8(f + 8, inv);
+              args.out_sf[atom_offset(grow, (col0 >> 4) + q, args.out_groups)] = (uint8_t)code;
+            }
+            *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(dst + 16) = make_uint4(w[4], w[5], w[6], w[7]);
           }
           acc_phase ^= 1u;
           buf ^= 1;
@@ -427,6 +517,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_wait_ld();
         tc_fence_before();
         mbar_arrive(tempty);
+        // NVFP4: W_d's tensor scale on the way out
+        auto f = [s0](uint32_t b) { return FMT == 2 ? __uint_as_float(b) * s0 : __uint_as_float(b); };
         // a row group whose 32 rows are all valid leaves by TMA stores of 32 x 32 boxes staged
         // in shared memory; a partly valid group (an expert's last rows: few at decode) by row
         // stores of its valid rows
@@ -439,10 +531,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int q = 0; q < 4; ++q)
                 dst[i * 4 + q] =
-                    make_uint4(pack_bf16(__uint_as_float(r[i][8 * q + 0]), __uint_as_float(r[i][8 * q + 1])),
-                               pack_bf16(__uint_as_float(r[i][8 * q + 2]), __uint_as_float(r[i][8 * q + 3])),
-                               pack_bf16(__uint_as_float(r[i][8 * q + 4]), __uint_as_float(r[i][8 * q + 5])),
-                               pack_bf16(__uint_as_float(r[i][8 * q + 6]), __uint_as_float(r[i][8 * q + 7])));
+                    make_uint4(pack_bf16(f(r[i][8 * q + 0]), f(r[i][8 * q + 1])),
+                               pack_bf16(f(r[i][8 * q + 2]), f(r[i][8 * q + 3])),
+                               pack_bf16(f(r[i][8 * q + 4]), f(r[i][8 * q + 5])),
+                               pack_bf16(f(r[i][8 * q + 6]), f(r[i][8 * q + 7])));
           }
         } else if (col0 < args.n_out) {  // the same for the whole warp
           uint8_t* stg = sStg + (warp - 2) * STG_BYTES;
@@ -454,10 +546,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               *reinterpret_cast<uint4*>(stg + lane * 64 + q * 16) =
-                  make_uint4(pack_bf16(__uint_as_float(r[i][8 * q + 0]), __uint_as_float(r[i][8 * q + 1])),
-                             pack_bf16(__uint_as_float(r[i][8 * q + 2]), __uint_as_float(r[i][8 * q + 3])),
-                             pack_bf16(__uint_as_float(r[i][8 * q + 4]), __uint_as_float(r[i][8 * q + 5])),
-                             pack_bf16(__uint_as_float(r[i][8 * q + 6]), __uint_as_float(r[i][8 * q + 7])));
+                  make_uint4(pack_bf16(f(r[i][8 * q + 0]), f(r[i][8 * q + 1])),
+                             pack_bf16(f(r[i][8 * q + 2]), f(r[i][8 * q + 3])),
+                             pack_bf16(f(r[i][8 * q + 4]), f(r[i][8 * q + 5])),
+                             pack_bf16(f(r[i][8 * q + 6]), f(r[i][8 * q + 7])));
             fence_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -485,9 +577,9 @@ template <int MODE, int FMT>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& c,
                         const Fp8Args& args, int grid, cudaStream_t s) {
   static SmemAttr attr{};
-  const cudaError_t e = ensure_smem_attr(attr, k_fp8_gemm<MODE, FMT>, SMEM_BYTES);
+  const cudaError_t e = ensure_smem_attr(attr, k_fp8_gemm<MODE, FMT>, FmtCfg<FMT>::kSmem);
   if (e != cudaSuccess) return e;
-  k_fp8_gemm<MODE, FMT><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, c, args);
+  k_fp8_gemm<MODE, FMT><<<grid, NUM_THREADS, FmtCfg<FMT>::kSmem, s>>>(a, b0, b1, c, args);
   return cudaGetLastError();
 }
 
@@ -498,10 +590,18 @@ int fp8_block_n(int mode) { return mode == kGateUp ? BN / 2 : BN; }
 
 cudaError_t launch_fp8_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                             const CUtensorMap& c, const Fp8Args& args, int grid, cudaStream_t s) {
-  if (mode == kGateUp) return args.fmt ? launch_mode<kGateUp, 1>(a, b0, b1, c, args, grid, s)
-                                       : launch_mode<kGateUp, 0>(a, b0, b1, c, args, grid, s);
-  if (mode == kDown) return args.fmt ? launch_mode<kDown, 1>(a, b0, b1, c, args, grid, s)
-                                     : launch_mode<kDown, 0>(a, b0, b1, c, args, grid, s);
+  if (args.fmt < 0 || args.fmt > 2 || (args.fmt == 2 && (!args.gsc0 || (mode == kGateUp && !args.gsc1))))
+    return cudaErrorInvalidValue;
+  if (mode == kGateUp) {
+    if (args.fmt == 2) return launch_mode<kGateUp, 2>(a, b0, b1, c, args, grid, s);
+    return args.fmt ? launch_mode<kGateUp, 1>(a, b0, b1, c, args, grid, s)
+                    : launch_mode<kGateUp, 0>(a, b0, b1, c, args, grid, s);
+  }
+  if (mode == kDown) {
+    if (args.fmt == 2) return launch_mode<kDown, 2>(a, b0, b1, c, args, grid, s);
+    return args.fmt ? launch_mode<kDown, 1>(a, b0, b1, c, args, grid, s)
+                    : launch_mode<kDown, 0>(a, b0, b1, c, args, grid, s);
+  }
   return cudaErrorInvalidValue;
 }
 

@@ -83,6 +83,44 @@ __device__ __forceinline__ uint32_t pack_e2m1x8(const float* v, float inv) {
          (pack_e2m1x2(v[4] * inv, v[5] * inv) << 16) | (pack_e2m1x2(v[6] * inv, v[7] * inv) << 24);
 }
 
+// ---------------------------------------------------------------- W4A4 (NVFP4)
+// The same E2M1 codes with a finer, two-level scale: one unsigned E4M3 value
+// (UE4M3: the positive E4M3 values 2^-9 .. 448) per 16 elements along K and one
+// fp32 scale g per tensor (value = code * s * g).  The block scale is the
+// smallest UE4M3 value s with amax <= 6 s g, decided in fp32 on
+// t = fl32(amax / fl32(6 g)); codes are e2m1(fl32(x * fl32(1 / fl32(s g)))).
+// Weights take g = fl32(amax(matrix) / 2688) (so their largest block scale is
+// 448), activations g = 1.  Scale atoms as above with j indexing the 16-element
+// blocks of a 64-element K group (`groups` = ceil(K / 64)).
+
+// The value of a positive E4M3 code (exact in fp32).
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  const uint32_t e = c >> 3, m = c & 7u;
+  return e == 0 ? (float)m * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// The smallest positive E4M3 value >= t (t > 0), as its code; 0x7E (448) for t > 448.
+__device__ __forceinline__ uint32_t ue4m3_ceil(float t) {
+  if (t > 448.0f) return 0x7Eu;
+  const uint32_t b = __float_as_uint(t);
+  const int ef = (int)(b >> 23);
+  if (ef < 121) return (uint32_t)ceilf(t * 512.0f);  // below 2^-6: multiples of 2^-9 (code 8 is 2^-6)
+  const uint32_t mant = b & 0x7FFFFFu;
+  const uint32_t m3 = (mant >> 20) + ((mant & 0xFFFFFu) != 0u);  // 8 carries into the exponent
+  return ((uint32_t)(ef - 120) << 3) + m3;
+}
+
+// UE4M3 block-scale code for a block maximum amax (finite, >= 0) under tensor scale g.
+__device__ __forceinline__ uint32_t nv4_code(float amax, float g) {
+  if (!(amax > 0.0f)) return 0x38u;  // 1.0
+  return ue4m3_ceil(__fdiv_rn(amax, __fmul_rn(6.0f, g)));
+}
+
+// fl32(1 / fl32(s g)): the multiplier that takes a block's elements to code space.
+__device__ __forceinline__ float nv4_inverse(uint32_t code, float g) {
+  return __frcp_rn(__fmul_rn(e4m3_value(code), g));
+}
+
 // Byte offset of (row, K-block) in a scale-atom array with `groups` atoms per 128 rows.
 __host__ __device__ __forceinline__ int64_t atom_offset(int64_t row, int kb, int groups) {
   const int64_t R = row >> 7;

@@ -118,13 +118,22 @@ cudaError_t launch_quant_mx4(int bf16, const void* src, int64_t rows, int cols, 
 cudaError_t launch_gather_quant4(const void* x, int d, const int32_t* perm, const int32_t* idx, int k,
                                  const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x4,
                                  uint8_t* sx, int groups, int sms, cudaStream_t s);
+// NVFP4: g[m] = the tensor scale of matrix m (nmat matrices of mrows x cols, consecutive);
+// rows of src take gvec[r / rows_per_g] (gvec null: g_const)
+cudaError_t launch_nv4_global(int bf16, const void* src, int nmat, int64_t mrows, int cols, float* g, cudaStream_t s);
+cudaError_t launch_quant_nv4(int bf16, const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
+                             int atom_groups, const float* gvec, int64_t rows_per_g, float g_const, int sms,
+                             cudaStream_t s);
+cudaError_t launch_gather_quant_nv4(const void* x, int d, const int32_t* perm, const int32_t* idx, int k,
+                                    const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x4,
+                                    uint8_t* sx, int groups, int sms, cudaStream_t s);
 cudaError_t launch_unpad_rows(const void* ypad, int row_bytes, const int32_t* perm, const int32_t* idx,
                               const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, void* out, int sms,
                               cudaStream_t s);
 
 struct Fp8Args {
-  int fmt;                 // 0: FP8 E4M3, [1,128]/[128,128] scales; 1: MXFP4, [1,32] scales
-  int K;                   // reduction length in elements (FP8: a multiple of 128, MXFP4: of 256)
+  int fmt;                 // 0: FP8 E4M3, [1,128]/[128,128] scales; 1: MXFP4, [1,32] scales; 2: NVFP4, [1,16]
+  int K;                   // reduction length in elements (FP8: a multiple of 128, MXFP4 / NVFP4: of 256)
   int n_out;               // valid output columns
   int nblocks;             // output column tiles
   int ngroups;             // experts
@@ -134,8 +143,11 @@ struct Fp8Args {
   const uint8_t* sfa;      // A scale atoms
   const uint8_t* sfb0;     // B scale atoms (gate/up: W_g, down: W_d)
   const uint8_t* sfb1;     // gate/up: W_u scale atoms
-  int groups_k;            // scale atoms per 128 rows of A and B: FP8 ceil(K / 512), MXFP4 ceil(K / 128)
-  void* out;               // gate/up: H codes [padded rows, n_out (FP8) or n_out / 2 (MXFP4) bytes]; down: Y bf16
+  int groups_k;            // scale atoms per 128 rows of A and B: FP8 ceil(K / 512), MXFP4 ceil(K / 128),
+                           // NVFP4 K / 64
+  const float* gsc0;       // NVFP4: the B tensors' fp32 scales per expert (gate/up: W_g, down: W_d)
+  const float* gsc1;       // NVFP4 gate/up: W_u's
+  void* out;               // gate/up: H codes [padded rows, n_out (FP8) or n_out / 2 (FP4) bytes]; down: Y bf16
   int64_t ldo;             // its row stride (gate/up: bytes; down: elements)
   uint8_t* out_sf;         // gate/up: H scale atoms, out_groups per 128 rows
   int out_groups;

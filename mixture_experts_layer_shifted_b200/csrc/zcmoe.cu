@@ -203,8 +203,9 @@ struct zcmoe_s {
   // ZCMOE_FP8: expert weights as E4M3 codes + scale atoms (owned), padded
   // activation operands (expert e's pairs from row 128 mb_off[e] on) with their
   // scale atoms, padded expert outputs; atoms per 128 rows: gd (K = d), gi (K = inter)
-  int fp8, fmt, gd, gi;  // fp8: block-scaled experts (ZCMOE_FP8 or ZCMOE_FP4); fmt 1 for MXFP4
+  int fp8, fmt, gd, gi;  // fp8: block-scaled experts (ZCMOE_FP8, _FP4, _NVFP4); fmt 1 MXFP4, 2 NVFP4
   uint8_t *w8g, *w8u, *w8d, *sfg, *sfu, *sfd, *x8, *sx, *h8, *sh;
+  float* gsc;  // NVFP4: the fp32 tensor scales of W_g [N], W_u [N], W_d [N], one per expert matrix
   void* ypad;
   CUtensorMap tm8_wg, tm8_wu, tm8_wd, tm8_x, tm8_h, tm8_y;  // tm8_y: the down GEMM's store target (ypad)
   // zcmoe_backward (allocated on its first call): padded X, dY, dH, [dG|dU], H, dX
@@ -235,7 +236,7 @@ static void release(zcmoe_s* h) {
   void* ptrs[] = {h->bias,  h->b0,     h->offset, h->eta,   h->integ,   h->eprev,  h->acc_counts,
                   h->err,   h->logits, h->gate,   h->idx,   h->pos,     h->counts, h->offsets,
                   h->mb_off, h->scal,  h->chunk,  h->perm,  h->xperm,   h->H,      h->Y,  h->sp_off, h->sched,
-                  h->stage_x, h->stage_x2, h->stage_y, h->stage_y2, h->w8g, h->w8u, h->w8d, h->sfg, h->sfu, h->sfd,
+                  h->stage_x, h->stage_x2, h->stage_y, h->stage_y2, h->w8g, h->w8u, h->w8d, h->sfg, h->sfu, h->sfd, h->gsc,
                   h->x8, h->sx, h->h8, h->sh, h->ypad, h->b_xpad, h->b_dypad, h->b_dh, h->b_dgu, h->b_hpad,
                   h->b_dxp, h->b_dl, h->b_dxr, h->b_dg, h->b_grp, h->b_gu, h->ep_meta};
   for (void* p : ptrs)
@@ -358,12 +359,13 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
   if (cfg->d < 64 || cfg->d % 64 || cfg->inter < 64 || cfg->inter % 64)
     return fail(ZCMOE_EINVAL, "d and inter must be positive multiples of 64");
   if (cfg->max_tokens < 1 || cfg->max_tokens > (1 << 20)) return fail(ZCMOE_EINVAL, "need 1 <= max_tokens <= 2^20");
-  if (cfg->dtype != ZCMOE_F32 && cfg->dtype != ZCMOE_BF16 && cfg->dtype != ZCMOE_FP8 && cfg->dtype != ZCMOE_FP4)
+  if (cfg->dtype != ZCMOE_F32 && cfg->dtype != ZCMOE_BF16 && cfg->dtype != ZCMOE_FP8 && cfg->dtype != ZCMOE_FP4 &&
+      cfg->dtype != ZCMOE_NVFP4)
     return fail(ZCMOE_EINVAL, "unknown dtype");
   if (cfg->dtype == ZCMOE_FP8 && (cfg->d % 512 || cfg->inter % 128))
     return fail(ZCMOE_EINVAL, "FP8 experts need d a multiple of 512 and inter a multiple of 128");
-  if (cfg->dtype == ZCMOE_FP4 && (cfg->d % 512 || cfg->inter % 256))
-    return fail(ZCMOE_EINVAL, "MXFP4 experts need d a multiple of 512 and inter a multiple of 256");
+  if ((cfg->dtype == ZCMOE_FP4 || cfg->dtype == ZCMOE_NVFP4) && (cfg->d % 512 || cfg->inter % 256))
+    return fail(ZCMOE_EINVAL, "W4A4 experts need d a multiple of 512 and inter a multiple of 256");
   if (!w->w_router || !w->w_gate || !w->w_up || !w->w_down) return fail(ZCMOE_EINVAL, "a weight pointer is NULL");
   const void* wp[4] = {w->w_router, w->w_gate, w->w_up, w->w_down};
   for (const void* p : wp)
@@ -395,9 +397,9 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
   h->d = cfg->d;
   h->inter = cfg->inter;
   h->max_T = cfg->max_tokens;
-  h->bf16 = cfg->dtype != ZCMOE_F32;  // ZCMOE_FP8 / ZCMOE_FP4 layers are bf16 at the interface
-  h->fp8 = cfg->dtype == ZCMOE_FP8 || cfg->dtype == ZCMOE_FP4;
-  h->fmt = cfg->dtype == ZCMOE_FP4;
+  h->bf16 = cfg->dtype != ZCMOE_F32;  // ZCMOE_FP8 / _FP4 / _NVFP4 layers are bf16 at the interface
+  h->fp8 = cfg->dtype == ZCMOE_FP8 || cfg->dtype == ZCMOE_FP4 || cfg->dtype == ZCMOE_NVFP4;
+  h->fmt = cfg->dtype == ZCMOE_FP4 ? 1 : cfg->dtype == ZCMOE_NVFP4 ? 2 : 0;
   h->sms = prop.multiProcessorCount;
   h->device = dev;
   h->w = *w;
@@ -447,9 +449,10 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
   if (ep_size > 1) ZC_ALLOC(h->ep_meta, (size_t)2 * ep_size * NL + 1 + 3 * (NL + 1));
   if (h->fp8) {
     const size_t prow = (size_t)h->max_mblocks * zc::kBM;  // padded rows
-    // scale atoms per 128 rows: an atom covers 512 K elements (FP8) or 128 (MXFP4)
-    h->gd = h->fmt ? (h->d + 127) / 128 : (h->d / 128 + 3) / 4;
-    h->gi = h->fmt ? (h->inter + 127) / 128 : (h->inter / 128 + 3) / 4;
+    // scale atoms per 128 rows: an atom covers 512 K elements (FP8), 128 (MXFP4) or 64 (NVFP4)
+    const int akb = h->fmt == 2 ? 64 : h->fmt ? 128 : 512;
+    h->gd = (h->d + akb - 1) / akb;
+    h->gi = (h->inter + akb - 1) / akb;
     const size_t wn = (size_t)N * h->inter * h->d / (h->fmt ? 2 : 1);
     ZC_ALLOC(h->w8g, wn);
     ZC_ALLOC(h->w8u, wn);
@@ -457,6 +460,7 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
     ZC_ALLOC(h->sfg, (size_t)N * (h->inter / 128) * h->gd * zc::kAtomBytes);
     ZC_ALLOC(h->sfu, (size_t)N * (h->inter / 128) * h->gd * zc::kAtomBytes);
     ZC_ALLOC(h->sfd, (size_t)N * (h->d / 128) * h->gi * zc::kAtomBytes);
+    if (h->fmt == 2) ZC_ALLOC(h->gsc, (size_t)3 * N);
     ZC_ALLOC(h->x8, prow * h->d / (h->fmt ? 2 : 1));
     ZC_ALLOC(h->sx, (size_t)h->max_mblocks * h->gd * zc::kAtomBytes);
     ZC_ALLOC(h->h8, prow * h->inter / (h->fmt ? 2 : 1));
@@ -513,7 +517,19 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
       if (e == cudaSuccess) e = cudaMemset(h->sh, 0, (size_t)h->max_mblocks * h->gi * zc::kAtomBytes);
       // the expert weights, quantized into scale atoms: FP8 per [128,128], MXFP4 per [1,32]
       const int64_t ri = (int64_t)N * h->inter, rd = (int64_t)N * h->d;
-      if (h->fmt) {
+      if (h->fmt == 2) {
+        // one fp32 tensor scale per expert matrix, then [1,16] blocks under it
+        float *gg = h->gsc, *gu = h->gsc + N, *gdn = h->gsc + 2 * N;
+        if (e == cudaSuccess) e = zc::launch_nv4_global(1, w->w_gate, N, h->inter, h->d, gg, 0);
+        if (e == cudaSuccess) e = zc::launch_nv4_global(1, w->w_up, N, h->inter, h->d, gu, 0);
+        if (e == cudaSuccess) e = zc::launch_nv4_global(1, w->w_down, N, h->d, h->inter, gdn, 0);
+        if (e == cudaSuccess)
+          e = zc::launch_quant_nv4(1, w->w_gate, ri, h->d, h->w8g, h->sfg, h->gd, gg, h->inter, 1.0f, h->sms, 0);
+        if (e == cudaSuccess)
+          e = zc::launch_quant_nv4(1, w->w_up, ri, h->d, h->w8u, h->sfu, h->gd, gu, h->inter, 1.0f, h->sms, 0);
+        if (e == cudaSuccess)
+          e = zc::launch_quant_nv4(1, w->w_down, rd, h->inter, h->w8d, h->sfd, h->gi, gdn, h->d, 1.0f, h->sms, 0);
+      } else if (h->fmt) {
         if (e == cudaSuccess) e = zc::launch_quant_mx4(1, w->w_gate, ri, h->d, h->w8g, h->sfg, h->gd, h->sms, 0);
         if (e == cudaSuccess) e = zc::launch_quant_mx4(1, w->w_up, ri, h->d, h->w8u, h->sfu, h->gd, h->sms, 0);
         if (e == cudaSuccess) e = zc::launch_quant_mx4(1, w->w_down, rd, h->inter, h->w8d, h->sfd, h->gi, h->sms, 0);
@@ -542,7 +558,7 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
     if (rc == ZCMOE_OK && !h->fp8) rc = make_tmap(&h->tm_h, h->H, inter, (uint64_t)h->rows_cap, 128);
     if (rc == ZCMOE_OK && !h->fp8) rc = make_tmap(&h->tm_y, h->Y, d, (uint64_t)h->rows_cap, 32);  // down output
     if (h->fp8) {
-      // codes as bytes: the K extent is d or inter bytes (FP8), half that (MXFP4)
+      // codes as bytes: the K extent is d or inter bytes (FP8), half that (FP4)
       const uint64_t prow = (uint64_t)h->max_mblocks * zc::kBM;
       const uint64_t db = d / (h->fmt ? 2 : 1), ib = inter / (h->fmt ? 2 : 1);
       if (rc == ZCMOE_OK) rc = make_tmap_esz(&h->tm8_wg, h->w8g, db, (uint64_t)N * inter, 128, 1);
@@ -704,7 +720,10 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
   }
   ZC_CUDA(mark("zcmoe.gather"));
   // 4. gather the FFN pairs' rows (FP8 layers: quantized per [1,128] into padded rows)
-  if (h->fp8 && h->fmt)
+  if (h->fp8 && h->fmt == 2)
+    ZC_CUDA(zc::launch_gather_quant_nv4(x, d, h->perm, h->idx, k, h->offsets, h->mb_off, h->scal, h->x8, h->sx, h->gd,
+                                        h->sms, s));
+  else if (h->fp8 && h->fmt)
     ZC_CUDA(zc::launch_gather_quant4(x, d, h->perm, h->idx, k, h->offsets, h->mb_off, h->scal, h->x8, h->sx, h->gd,
                                      h->sms, s));
   else if (h->fp8)
@@ -733,6 +752,8 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     a.ldo = inter / (h->fmt ? 2 : 1);
     a.out_sf = h->sh;
     a.out_groups = h->gi;
+    a.gsc0 = h->gsc;
+    a.gsc1 = h->gsc ? h->gsc + N : nullptr;
     a.err = h->err;
     int bound = max_mb * a.nblocks;
     ZC_CUDA(zc::launch_fp8_gemm(zc::kGateUp, h->tm8_x, h->tm8_wg, h->tm8_wu, h->tm8_wu, a,
@@ -751,6 +772,7 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     b.sfb0 = h->sfd;
     b.sfb1 = nullptr;
     b.groups_k = h->gi;
+    b.gsc0 = h->gsc ? h->gsc + 2 * N : nullptr;
     b.out = h->ypad;
     b.ldo = d;
     b.err = h->err;
@@ -1567,6 +1589,32 @@ int zcmoe_quantize_mx4(const void* src, int32_t src_dtype, int64_t rows, int64_t
   ZC_CUDA(cudaGetDevice(&dev));
   ZC_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   ZC_CUDA(zc::launch_quant_mx4(src_dtype == ZCMOE_BF16, src, rows, (int)cols, codes, scales, 0, sms, s));
+  return ZCMOE_OK;
+}
+
+int zcmoe_quantize_nv4(const void* src, int32_t src_dtype, int64_t rows, int64_t cols, float global_scale,
+                       uint8_t* codes, uint8_t* scales, float* global_out, cudaStream_t s) {
+  g_err[0] = 0;
+  if (src_dtype != ZCMOE_BF16 && src_dtype != ZCMOE_F32) return fail(ZCMOE_EINVAL, "src_dtype must be BF16 or F32");
+  if (rows < 0 || cols <= 0 || cols % 256 || cols > (1 << 30)) return fail(ZCMOE_EINVAL, "bad rows / cols");
+  if (!(std::isfinite(global_scale) && global_scale >= 0.0f))
+    return fail(ZCMOE_EINVAL, "global_scale must be finite and >= 0 (0: derived from the tensor)");
+  if (global_scale == 0.0f && !global_out) return fail(ZCMOE_EINVAL, "global_out is NULL (needed when global_scale is 0)");
+  if (rows == 0) return ZCMOE_OK;
+  if (!src || !codes || !scales) return fail(ZCMOE_EINVAL, "a pointer is NULL");
+  if ((reinterpret_cast<uintptr_t>(src) & 15u) || (reinterpret_cast<uintptr_t>(codes) & 15u) ||
+      (reinterpret_cast<uintptr_t>(global_out) & 3u))
+    return fail(ZCMOE_EINVAL, "src and codes must be 16-byte aligned, global_out 4-byte aligned");
+  int dev = 0, sms = 0;
+  ZC_CUDA(cudaGetDevice(&dev));
+  ZC_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const int bf16 = src_dtype == ZCMOE_BF16;
+  if (global_scale == 0.0f) {
+    ZC_CUDA(zc::launch_nv4_global(bf16, src, 1, rows, (int)cols, global_out, s));
+    ZC_CUDA(zc::launch_quant_nv4(bf16, src, rows, (int)cols, codes, scales, 0, global_out, rows, 1.0f, sms, s));
+  } else {
+    ZC_CUDA(zc::launch_quant_nv4(bf16, src, rows, (int)cols, codes, scales, 0, nullptr, 1, global_scale, sms, s));
+  }
   return ZCMOE_OK;
 }
 

@@ -29,13 +29,14 @@ ZCMOE_F32 = 0
 ZCMOE_BF16 = 1
 ZCMOE_FP8 = 2
 ZCMOE_FP4 = 3
-_DTYPES = {"f32": ZCMOE_F32, "bf16": ZCMOE_BF16, "fp8": ZCMOE_FP8, "fp4": ZCMOE_FP4}
+ZCMOE_NVFP4 = 4
+_DTYPES = {"f32": ZCMOE_F32, "bf16": ZCMOE_BF16, "fp8": ZCMOE_FP8, "fp4": ZCMOE_FP4, "nvfp4": ZCMOE_NVFP4}
 
 EXPORTED = ("zcmoe_create", "zcmoe_forward", "zcmoe_forward_host", "zcmoe_update_bias", "zcmoe_read_counts",
             "zcmoe_write_counts", "zcmoe_get_state", "zcmoe_set_bias", "zcmoe_check", "zcmoe_profile_begin",
             "zcmoe_profile_end", "zcmoe_selftest_wait", "zcmoe_route_noalloc", "zcmoe_destroy",
             "zcmoe_dense_create", "zcmoe_dense_forward", "zcmoe_forward_overlap", "zcmoe_dense_check",
-            "zcmoe_dense_destroy", "zcmoe_quantize_e4m3", "zcmoe_quantize_mx4", "zcmoe_backward",
+            "zcmoe_dense_destroy", "zcmoe_quantize_e4m3", "zcmoe_quantize_mx4", "zcmoe_quantize_nv4", "zcmoe_backward",
             "zcmoe_save_for_backward", "zcmoe_backward_ex", "zcmoe_forward_host_async",
             "zcmoe_forward_host_flush", "zcmoe_create_ep", "zcmoe_ep_dispatch", "zcmoe_ep_experts",
             "zcmoe_ep_combine", "zcmoe_get_controller", "zcmoe_set_controller", "zcmoe_last_error")
@@ -116,6 +117,7 @@ def lib():
         L.zcmoe_dense_check.argtypes = [vp]
         L.zcmoe_quantize_e4m3.argtypes = [vp, ctypes.c_int32, i64, i64, ctypes.c_int32, vp, vp, vp]
         L.zcmoe_quantize_mx4.argtypes = [vp, ctypes.c_int32, i64, i64, vp, vp, vp]
+        L.zcmoe_quantize_nv4.argtypes = [vp, ctypes.c_int32, i64, i64, ctypes.c_float, vp, vp, vp, vp]
         L.zcmoe_backward.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, vp, vp]
         L.zcmoe_backward_ex.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, vp, ctypes.c_uint32, vp]
         L.zcmoe_save_for_backward.argtypes = [vp, ctypes.c_int32]
@@ -352,6 +354,28 @@ def quantize_mx4(src, stream=None):
     return codes, scales
 
 
+def zcmoe_quantize_nv4(src_ptr, src_dtype, rows, cols, global_scale, codes_ptr, scales_ptr, global_out_ptr,
+                       stream=None):
+    _check(lib().zcmoe_quantize_nv4(src_ptr, src_dtype, rows, cols, global_scale, codes_ptr, scales_ptr,
+                                    global_out_ptr, _stream(stream)), "zcmoe_quantize_nv4")
+
+
+def quantize_nv4(src, global_scale=1.0, stream=None):
+    """(codes uint8 [rows, cols/2], scales uint8 [rows, cols/16], g float32 [1]) of a 2-D
+    bf16 or fp32 device tensor (NVFP4, the rule of ZCMOE_NVFP4 layers).  global_scale
+    g > 0 quantizes under g; 0 derives g from the tensor as the layer does for a weight
+    matrix (amax / 2688)."""
+    rows, cols = src.shape
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=src.device)
+    scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=src.device)
+    g = torch.full((1,), float(global_scale), dtype=torch.float32, device=src.device)
+    dt = ZCMOE_BF16 if src.dtype == torch.bfloat16 else ZCMOE_F32
+    zcmoe_quantize_nv4(ctypes.c_void_p(src.data_ptr()), dt, rows, cols, float(global_scale),
+                       ctypes.c_void_p(codes.data_ptr()), ctypes.c_void_p(scales.data_ptr()),
+                       ctypes.c_void_p(g.data_ptr()), stream)
+    return codes, scales, g
+
+
 def zcmoe_last_error() -> str:
     return lib().zcmoe_last_error().decode(errors="replace")
 
@@ -364,7 +388,7 @@ class LayerShape:
     n_zero: int
     inter: int
     top_k: int
-    dtype: str = "bf16"  # "bf16", "f32", "fp8" or "fp4" (bf16 interface, block-scaled FP8 / MXFP4 experts)
+    dtype: str = "bf16"  # "bf16", "f32", "fp8", "fp4" or "nvfp4" (bf16 interface; FP8 / MXFP4 / NVFP4 experts)
     routed_scale: float = 1.0
 
     @property

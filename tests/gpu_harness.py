@@ -19,7 +19,7 @@ import oracle
 from mixture_experts_layer_shifted_b200 import configs, synth
 from mixture_experts_layer_shifted_b200.zcmoe import LayerShape, ZcMoE
 
-TOL = {"bf16": 2e-2, "f32": 1e-4, "fp8": 2e-2, "fp4": 2e-2}
+TOL = {"bf16": 2e-2, "f32": 1e-4, "fp8": 2e-2, "fp4": 2e-2, "nvfp4": 2e-2}
 TIE_MARGIN = 1e-5
 
 
@@ -150,7 +150,11 @@ class Run:
         for e, lst in sorted(byexp.items()):
             wg, wu, wd = self.expert_weights(e)
             rows = [t for _, t in lst]
-            if self.w.dtype == "fp4":
+            if self.w.dtype == "nvfp4":
+                q = [oracle.quantize_weight_nv4(w_) for w_ in (wg, wu, wd)]
+                ref = oracle.ffn_nv4(self.x_host(rows), [c for c, _, _ in q], [s_ for _, s_, _ in q],
+                                     [g_ for _, _, g_ in q])
+            elif self.w.dtype == "fp4":
                 q = [oracle.quantize_mx4(w_) for w_ in (wg, wu, wd)]
                 ref = oracle.ffn_fp4(self.x_host(rows), [c for c, _ in q], [s_ for _, s_ in q])
             elif self.w.dtype == "fp8":
@@ -171,7 +175,8 @@ class Run:
         idx = self.dbg["idx"][rows]
         gate = self.dbg["gate"][rows].astype(np.float64)
         ref = oracle.layer_outputs(self.x_host(rows), idx, gate, self.w.n_ffn, self.expert_weights,
-                                   fp8=self.w.dtype == "fp8", fp4=self.w.dtype == "fp4")
+                                   fp8=self.w.dtype == "fp8", fp4=self.w.dtype == "fp4",
+                                   nv4=self.w.dtype == "nvfp4")
         err = row_rel_err(self.y[rows], ref)
         assert float(err.max()) <= tol, float(err.max())
         return float(err.max())
