@@ -46,15 +46,21 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL = 256;                   // scale buffers: [256, 304) (FP8, MXFP4), [256, 352) (NVFP4)
 constexpr uint32_t STG_BYTES = 32 * 64;           // down epilogue: a 32-row x 32-column bf16 box per warp
 
-// Per format: pipeline depth and scale bytes per stage (FP8 uses 3 atoms of its 6, MXFP4 6,
-// NVFP4 12: one atom per operand 128 rows per K = 64 MMA).
-template <int FMT>
+// Per mode and format: pipeline depth, scale bytes per stage (FP8 uses 3 atoms of its 6,
+// MXFP4 6, NVFP4 12: one atom per operand 128 rows per K = 64 MMA) and the down epilogue's
+// staging boxes (the gate/up epilogue stores from registers and has none).  The NVFP4 down
+// GEMM keeps three stages: four would not fit beside the staging boxes.
+template <int MODE, int FMT>
 struct FmtCfg {
-  static constexpr int kStages = FMT == 2 ? 3 : 4;
+  static constexpr int kStages = (FMT == 2 && MODE == kDown) ? 3 : 4;
   static constexpr uint32_t kSfBytes = (FMT == 2 ? 12 : 6) * kAtomBytes;
-  static constexpr int kSmem = 1024 + kStages * (A_BYTES + B_BYTES + kSfBytes) + 8 * STG_BYTES + 256 + 2 * 2 * BM * 4;
+  static constexpr uint32_t kStgBytes = MODE == kDown ? 8 * STG_BYTES : 0;
+  static constexpr int kSmem = 1024 + kStages * (A_BYTES + B_BYTES + kSfBytes) + kStgBytes + 256 + 2 * 2 * BM * 4;
 };
-constexpr int SMEM_BYTES = FmtCfg<0>::kSmem > FmtCfg<2>::kSmem ? FmtCfg<0>::kSmem : FmtCfg<2>::kSmem;
+constexpr int cmax(int a, int b) { return a > b ? a : b; }
+constexpr int SMEM_BYTES = cmax(cmax(FmtCfg<kGateUp, 0>::kSmem, FmtCfg<kDown, 0>::kSmem),
+                                cmax(FmtCfg<kGateUp, 2>::kSmem, FmtCfg<kDown, 2>::kSmem));
+static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 
 struct Tile {
   int64_t a_row;   // first padded A row (a multiple of 128)
@@ -187,15 +193,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_fp8_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmC,
                const Fp8Args args) {
-  constexpr int STAGES = FmtCfg<FMT>::kStages;
-  constexpr uint32_t SF_BYTES = FmtCfg<FMT>::kSfBytes;
+  constexpr int STAGES = FmtCfg<MODE, FMT>::kStages;
+  constexpr uint32_t SF_BYTES = FmtCfg<MODE, FMT>::kSfBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * A_BYTES;
   uint8_t* sSF = sB + STAGES * B_BYTES;
   uint8_t* sStg = sSF + STAGES * SF_BYTES;  // [epilogue warp] of STG_BYTES (down)
-  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + 8 * STG_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + FmtCfg<MODE, FMT>::kStgBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 1;
@@ -577,9 +583,10 @@ template <int MODE, int FMT>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& c,
                         const Fp8Args& args, int grid, cudaStream_t s) {
   static SmemAttr attr{};
-  const cudaError_t e = ensure_smem_attr(attr, k_fp8_gemm<MODE, FMT>, FmtCfg<FMT>::kSmem);
+  constexpr int smem = FmtCfg<MODE, FMT>::kSmem;
+  const cudaError_t e = ensure_smem_attr(attr, k_fp8_gemm<MODE, FMT>, smem);
   if (e != cudaSuccess) return e;
-  k_fp8_gemm<MODE, FMT><<<grid, NUM_THREADS, FmtCfg<FMT>::kSmem, s>>>(a, b0, b1, c, args);
+  k_fp8_gemm<MODE, FMT><<<grid, NUM_THREADS, smem, s>>>(a, b0, b1, c, args);
   return cudaGetLastError();
 }
 

@@ -50,18 +50,26 @@ namespace {
 
 constexpr int BM = kBM, BN = 256, BK = 64;
 constexpr uint32_t A_BYTES = BM * BK * 2;
-constexpr uint32_t B_BYTES = BN * BK * 2;
 constexpr int EPI_WARPS = 8;
 constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
-constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint32_t STG_BYTES = 32 * 128;  // down epilogue: a 32-row x 64-column bf16 box per warp
 constexpr int RING = 4;                   // unit ids in flight from the producer to the consumers
+constexpr int BN_NARROW = kRouterNarrowN;
+
+// Columns per tile: 256, or 32 for the narrow router (a batch of one or a few row blocks,
+// where 256-column tiles would leave most SMs idle; every logit still sums the same
+// K = 16 MMA steps in the same order, so the tile width does not change its value).
+template <int MODE>
+constexpr int block_n() { return MODE == kRouterNarrow ? BN_NARROW : BN; }
 
 template <int MODE, bool PAIR>
 struct Cfg {
-  static constexpr bool kPair = PAIR && MODE != kRouter;  // stage two row blocks per weight tile
-  static constexpr int kStages = kPair ? 3 : 4;
-  static constexpr uint32_t kStageBytes = B_BYTES + (kPair ? 2 : 1) * A_BYTES;
+  static constexpr bool kPair = PAIR && MODE != kRouter && MODE != kRouterNarrow;  // two row blocks per weight tile
+  static constexpr int kBN = block_n<MODE>();
+  static constexpr uint32_t kBBytes = kBN * BK * 2;
+  static constexpr int kStages = MODE == kRouterNarrow ? 8 : kPair ? 3 : 4;
+  static constexpr uint32_t kStageBytes = kBBytes + (kPair ? 2 : 1) * A_BYTES;
+  static constexpr uint32_t kTmemCols = 2 * kBN;  // two accumulator slots
   // stages | staging boxes | barriers, the unit ring and the TMEM address
   static constexpr int kSmem = 1024 + kStages * kStageBytes + EPI_WARPS * STG_BYTES + 512;
 };
@@ -76,20 +84,20 @@ struct Unit {
 
 template <int MODE, bool PAIR>
 __device__ __forceinline__ int total_units(const TcArgs& a) {
-  if (MODE == kRouter) return ((a.M + BM - 1) / BM) * a.nblocks;
+  if (MODE == kRouter || MODE == kRouterNarrow) return ((a.M + BM - 1) / BM) * a.nblocks;
   return (PAIR ? a.sp_off[a.ngroups] : a.mb_off[a.ngroups]) * a.nblocks;
 }
 
 template <int MODE, bool PAIR>
 __device__ __forceinline__ Unit decode_unit(const TcArgs& a, int t) {
   Unit u;
-  if (MODE == kRouter) {
+  if (MODE == kRouter || MODE == kRouterNarrow) {
     const int m_blk = t / a.nblocks;
     u.n_blk = t - m_blk * a.nblocks;
     u.a_row = m_blk * BM;
     u.rows[0] = min(BM, a.M - u.a_row);
     u.rows[1] = 0;
-    u.b_row = u.n_blk * BN;
+    u.b_row = u.n_blk * block_n<MODE>();
     u.p_row = u.a_row;
     return u;
   }
@@ -252,13 +260,17 @@ __device__ __forceinline__ void drain_rows(const TcArgs& args, const CUtensorMap
       }
     }
   } else {
+    // router: fp32 logits (+ the logit offset); a 32-column tile is drained by the first
+    // warp of each lane quarter alone
+    constexpr int bn = block_n<MODE>();
+    constexpr int cw = bn >= 64 ? bn / 2 : bn;
     float* out = static_cast<float*>(args.out);
 #pragma unroll 1
-    for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+    for (int c = half * cw; c < (half + 1) * cw && c < bn; c += 32) {
       uint32_t r[32];
       tmem_ld32(tbase + c, r);
       tc_wait_ld();
-      const int col0 = n_blk * BN + c;
+      const int col0 = n_blk * bn + c;
       if (row_ok && col0 < args.n_out) {
         float* dst = out + grow * args.ldo + col0;
 #pragma unroll
@@ -318,7 +330,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (MODE == kGateUp) tma_prefetch(&tmB1);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -346,18 +358,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (t < 0) break;
         const Unit u = decode_unit<MODE, C::kPair>(args, t);
         const bool two = C::kPair && u.rows[1] > 0;
-        const uint32_t bytes = B_BYTES + (two ? 2u : 1u) * A_BYTES;
+        const uint32_t bytes = C::kBBytes + (two ? 2u : 1u) * A_BYTES;
         for (int kb = 0; kb < num_k; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, err, 1)) {
             ok = false;
             break;
           }
           uint8_t* b_dst = smem + stage * C::kStageBytes;
-          uint8_t* a_dst = b_dst + B_BYTES;
+          uint8_t* a_dst = b_dst + C::kBBytes;
           mbar_expect_tx(&full[stage], bytes);
           if (MODE == kGateUp) {
             tma_load_2d(b_dst, &tmB0, kb * BK, u.b_row, &full[stage]);
-            tma_load_2d(b_dst + B_BYTES / 2, &tmB1, kb * BK, u.b_row, &full[stage]);
+            tma_load_2d(b_dst + C::kBBytes / 2, &tmB1, kb * BK, u.b_row, &full[stage]);
           } else {
             tma_load_2d(b_dst, &tmB0, kb * BK, u.b_row, &full[stage]);
           }
@@ -383,8 +395,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (converged warp)
-    constexpr uint32_t idesc128 = idesc_bf16_f32(BM, BN);
-    constexpr uint32_t idesc64 = idesc_bf16_f32(64, BN);
+    constexpr uint32_t idesc128 = idesc_bf16_f32(BM, C::kBN);
+    constexpr uint32_t idesc64 = idesc_bf16_f32(64, C::kBN);
     int stage = 0;
     uint32_t phase = 0;
     int slot = 0;              // TMEM slot of the next row block
@@ -404,7 +416,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!warp_wait(&tempty[s0], (uses[s0] & 1) ^ 1u, err, 2)) break;
       if (two && !warp_wait(&tempty[s1], (uses[s1] & 1) ^ 1u, err, 2)) break;
       tc_fence_after();
-      const uint32_t d0 = tmem_base + (uint32_t)(s0 * BN), d1 = tmem_base + (uint32_t)(s1 * BN);
+      const uint32_t d0 = tmem_base + (uint32_t)(s0 * C::kBN), d1 = tmem_base + (uint32_t)(s1 * C::kBN);
       // a row block of at most 64 valid rows runs M = 64 MMAs (about half the energy of
       // M = 128); its rows land in TMEM lanes 32q + (0..15), q = 0..3
       const uint32_t id0 = u.rows[0] <= 64 ? idesc64 : idesc128;
@@ -417,7 +429,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         if (elect_one()) {
           const uint32_t b_addr = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t a_addr = b_addr + B_BYTES;
+          const uint32_t a_addr = b_addr + C::kBBytes;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             tc_mma_f16(d0, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), id0,
@@ -474,7 +486,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * BN);
+        const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * C::kBN);
         drain_rows<MODE>(args, &tmC, tbase, quarter, half, lane, u.a_row + r * BM, u.rows[r], u.p_row + r * BM,
                          u.n_blk, stg);
         tc_fence_before();
@@ -490,7 +502,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
@@ -514,13 +526,15 @@ int tc_smem_bytes() {
   return Cfg<kGateUp, true>::kSmem > Cfg<kGateUp, false>::kSmem ? Cfg<kGateUp, true>::kSmem
                                                                 : Cfg<kGateUp, false>::kSmem;
 }
-int tc_block_n(int mode) { return mode == kGateUp ? BN / 2 : BN; }
+int tc_block_n(int mode) { return mode == kGateUp ? BN / 2 : mode == kRouterNarrow ? BN_NARROW : BN; }
 
 cudaError_t launch_tc_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                            const CUtensorMap& c, const TcArgs& args, int grid, cudaStream_t s) {
   switch (mode) {
     case kRouter:
       return launch_mode<kRouter, false>(a, b0, b1, c, args, grid, s);
+    case kRouterNarrow:
+      return launch_mode<kRouterNarrow, false>(a, b0, b1, c, args, grid, s);
     case kGateUp:
       return args.pair ? launch_mode<kGateUp, true>(a, b0, b1, c, args, grid, s)
                        : launch_mode<kGateUp, false>(a, b0, b1, c, args, grid, s);

@@ -63,7 +63,8 @@ cudaError_t launch_update_bias(int64_t* counts, int64_t* tokens, int N, int Z, i
                                float* bias, cudaStream_t s);
 
 // ------------------------------------------------------------- tensor-core GEMM (gemm_tc.cu)
-enum TcMode { kRouter = 0, kGateUp = 1, kDown = 2 };
+enum TcMode { kRouter = 0, kGateUp = 1, kDown = 2, kRouterNarrow = 3 };
+constexpr int kRouterNarrowN = 32;  // columns per tile of the narrow router (its W_r tensor map's box)
 
 struct TcArgs {
   int K;                    // reduction length (elements)

@@ -199,7 +199,7 @@ struct zcmoe_s {
   bool profiling;
   std::vector<cudaEvent_t>* events;
   // tensor maps of fixed buffers
-  CUtensorMap tm_wr, tm_wg, tm_wu, tm_wd, tm_xperm, tm_h, tm_y;
+  CUtensorMap tm_wr, tm_wr_n, tm_wg, tm_wu, tm_wd, tm_xperm, tm_h, tm_y;  // tm_wr_n: W_r in 32-row boxes
   // ZCMOE_FP8: expert weights as E4M3 codes + scale atoms (owned), padded
   // activation operands (expert e's pairs from row 128 mb_off[e] on) with their
   // scale atoms, padded expert outputs; atoms per 128 rows: gd (K = d), gi (K = inter)
@@ -551,6 +551,7 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
   if (h->bf16) {
     const uint64_t d = h->d, inter = h->inter;
     rc = make_tmap(&h->tm_wr, w->w_router, d, (uint64_t)E, 256);
+    if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wr_n, w->w_router, d, (uint64_t)E, zc::kRouterNarrowN);
     if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wg, w->w_gate, d, (uint64_t)NL * inter, 128);
     if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wu, w->w_up, d, (uint64_t)NL * inter, 128);
     if (rc == ZCMOE_OK) rc = make_tmap(&h->tm_wd, w->w_down, inter, (uint64_t)NL * d, 256);
@@ -600,10 +601,15 @@ static int router_stage(zcmoe_t h, const void* x, int Ti, cudaStream_t s) {
     CUtensorMap tm_x;
     int rc = make_tmap(&tm_x, x, (uint64_t)d, (uint64_t)T, 128);
     if (rc != ZCMOE_OK) return rc;
+    // a batch of a few row blocks takes 32-column tiles, so that more SMs share its
+    // W_r and x bytes (the same logits either way)
+    const int mblocks = (Ti + zc::kBM - 1) / zc::kBM;
+    const int mode = mblocks * ((E + zc::kRouterNarrowN - 1) / zc::kRouterNarrowN) <= h->sms ? zc::kRouterNarrow
+                                                                                               : zc::kRouter;
     zc::TcArgs a{};
     a.K = d;
     a.n_out = E;
-    a.nblocks = (E + zc::tc_block_n(zc::kRouter) - 1) / zc::tc_block_n(zc::kRouter);
+    a.nblocks = (E + zc::tc_block_n(mode) - 1) / zc::tc_block_n(mode);
     a.ngroups = 1;
     a.M = Ti;
     a.out = h->logits;
@@ -611,8 +617,9 @@ static int router_stage(zcmoe_t h, const void* x, int Ti, cudaStream_t s) {
     a.col_add = h->offset;
     a.err = h->err;
     a.sched = h->sched;
-    const int tiles = ((Ti + zc::kBM - 1) / zc::kBM) * a.nblocks;
-    ZC_CUDA(zc::launch_tc_gemm(zc::kRouter, tm_x, h->tm_wr, h->tm_wr, h->tm_wr, a, tiles < h->sms ? tiles : h->sms, s));
+    const int tiles = mblocks * a.nblocks;
+    const CUtensorMap& tm_b = mode == zc::kRouterNarrow ? h->tm_wr_n : h->tm_wr;
+    ZC_CUDA(zc::launch_tc_gemm(mode, tm_x, tm_b, tm_b, tm_b, a, tiles < h->sms ? tiles : h->sms, s));
   } else {
     zc::SimtArgs a{};
     a.A = static_cast<const float*>(x);
