@@ -205,6 +205,73 @@ __global__ void __launch_bounds__(1024) k_route_scan(int32_t* __restrict__ chunk
   if (e == 0) *acc_tokens += T;
 }
 
+// Integer stage of a small batch (T <= 1024, decode) in one block of 1024 threads, one
+// token per thread: the work of the three kernels above in one launch.  One 32-bit token
+// mask per (warp, expert) covers the whole batch, so the counts, the offsets and the
+// order (ascending token within each expert) are the same.
+constexpr int kSmallT = 1024;
+__global__ void __launch_bounds__(1024) k_route_small(const int32_t* __restrict__ idx, int T, int k, int N, int E,
+                                                      int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                      int32_t* __restrict__ mb_off, int32_t* __restrict__ scal,
+                                                      int64_t* __restrict__ acc_counts,
+                                                      int64_t* __restrict__ acc_tokens, int32_t* __restrict__ sp_off,
+                                                      int32_t* __restrict__ perm, int32_t* __restrict__ pos) {
+  extern __shared__ uint32_t smask[];  // [32][E]
+  __shared__ int2 warp_tot[32];
+  __shared__ int2 warp_tot2[32];
+  __shared__ int32_t base[1024];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < 32 * E; i += 1024) smask[i] = 0u;
+  __syncthreads();
+  if (tid < T)
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(int64_t)tid * k + j];
+      if ((unsigned)e < (unsigned)E) atomicOr(&smask[warp * E + e], 1u << lane);  // an id out of range is skipped
+    }
+  __syncthreads();
+  const int e = tid;  // thread = expert
+  int total = 0;
+  if (e < E) {
+#pragma unroll 8
+    for (int w = 0; w < 32; ++w) total += __popc(smask[w * E + e]);
+    counts[e] = total;
+    acc_counts[e] += total;
+  }
+  const int2 v = (e < N) ? make_int2(total, (total + kBM - 1) / kBM) : make_int2(0, 0);
+  const int2 ex = block_exclusive_scan2(v, warp_tot);
+  const int2 v2 = make_int2((v.y + 1) / 2, 0);
+  const int2 ex2 = sp_off ? block_exclusive_scan2(v2, warp_tot2) : make_int2(0, 0);
+  if (e < N) {
+    offsets[e] = ex.x;
+    mb_off[e] = ex.y;
+    base[e] = ex.x;
+    if (sp_off) sp_off[e] = ex2.x;
+    if (e == N - 1) {
+      offsets[N] = ex.x + v.x;
+      mb_off[N] = ex.y + v.y;
+      if (sp_off) sp_off[N] = ex2.x + v2.x;
+      scal[0] = ex.x + v.x;
+      scal[1] = ex.y + v.y;
+    }
+  }
+  if (e == 0) *acc_tokens += T;
+  __syncthreads();
+  if (tid >= T) return;
+  for (int j = 0; j < k; ++j) {
+    const int64_t pair = (int64_t)tid * k + j;
+    const int ej = idx[pair];
+    if ((unsigned)ej < (unsigned)N) {
+      int r = base[ej];
+      for (int w = 0; w < warp; ++w) r += __popc(smask[w * E + ej]);
+      r += __popc(smask[warp * E + ej] & ((1u << lane) - 1u));
+      pos[pair] = r;
+      perm[r] = (int32_t)pair;
+    } else {
+      pos[pair] = -1;
+    }
+  }
+}
+
 // Integer stage, part 3: the permuted row of every FFN pair.  Within a 256-token
 // block the rank of (t, e) is the number of earlier tokens of the block that
 // chose e (earlier warps' masks, then the lower lanes of its own warp's mask),
@@ -301,12 +368,16 @@ struct Vec<float> {
   __device__ static void store(float* p, const float* f) { *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]); }
 };
 
-// One block per token.  Measured on B200 against variants with the slot loop
-// unrolled or several vectors per thread: this plain form keeps the most loads
-// in flight (many resident blocks) and reaches ~91% of the HBM copy rate.
+// Large batches: one block per token, its threads striding over the row's vectors, one
+// slot's load at a time (G = 1) -- many resident blocks keep the most loads in flight
+// (~91% of the HBM copy rate measured on B200).  Small batches (decode): one block per
+// (token, 128 vectors), and G = 8 slots' loads issued together before their products
+// are added, since the blocks are few and each thread's loads would otherwise wait one
+// after another.  The products are added in slot order either way, so the result is the
+// same.
 // With offsets / mb_off (FP8 layers), Y holds expert e's pairs from padded row
 // 128 mb_off[e] on, so a pair's row is pos - offsets[e] + 128 mb_off[e].
-template <typename TIO>
+template <typename TIO, int G>
 __global__ void __launch_bounds__(128) k_combine(const TIO* __restrict__ x, const TIO* __restrict__ Y,
                                                  const float* __restrict__ gate, const int32_t* __restrict__ pos, int T,
                                                  int k, int d, TIO* __restrict__ y, const int32_t* __restrict__ idx,
@@ -336,18 +407,27 @@ __global__ void __launch_bounds__(128) k_combine(const TIO* __restrict__ x, cons
   }
   __syncthreads();
   const float zsum = szsum;
-  for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+  for (int v = blockIdx.y * blockDim.x + threadIdx.x; v < nv; v += gridDim.y * blockDim.x) {
     float acc[V], a[V];
     Vec<TIO>::load(x + (int64_t)t * d + v * V, a);
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = __fmul_rn(zsum, a[i]);
-    for (int j = 0; j < k; ++j) {
-      const int p = sp[j];
-      if (p < 0) continue;
-      Vec<TIO>::load(Y + (int64_t)p * d + v * V, a);
-      const float g = sg[j];
+    for (int j0 = 0; j0 < k; j0 += G) {
+      float b[G][V];
 #pragma unroll
-      for (int i = 0; i < V; ++i) acc[i] = __fmaf_rn(g, a[i], acc[i]);
+      for (int jj = 0; jj < G; ++jj) {
+        const int j = j0 + jj;
+        if (j < k && sp[j] >= 0) Vec<TIO>::load(Y + (int64_t)sp[j] * d + v * V, b[jj]);
+      }
+#pragma unroll
+      for (int jj = 0; jj < G; ++jj) {
+        const int j = j0 + jj;
+        if (j < k && sp[j] >= 0) {
+          const float g = sg[j];
+#pragma unroll
+          for (int i = 0; i < V; ++i) acc[i] = __fmaf_rn(g, b[jj][i], acc[i]);
+        }
+      }
     }
     Vec<TIO>::store(y + (int64_t)t * d + v * V, acc);
   }
@@ -458,6 +538,20 @@ cudaError_t launch_route_scan(int32_t* chunk_cnt, int nchunks, int T, int N, int
   return cudaGetLastError();
 }
 
+int route_small_max_tokens() { return kSmallT; }
+
+cudaError_t launch_route_small(const int32_t* idx, int T, int k, int N, int E, int32_t* counts, int32_t* offsets,
+                               int32_t* mb_off, int32_t* scal, int64_t* acc_counts, int64_t* acc_tokens,
+                               int32_t* sp_off, int32_t* perm, int32_t* pos, cudaStream_t s) {
+  if (T < 1 || T > kSmallT || E > 1024) return cudaErrorInvalidValue;
+  static SmemAttr attr{};
+  const cudaError_t e = ensure_smem_attr(attr, k_route_small, 32 * 1024 * (int)sizeof(uint32_t));
+  if (e != cudaSuccess) return e;
+  k_route_small<<<1, 1024, 32 * E * sizeof(uint32_t), s>>>(idx, T, k, N, E, counts, offsets, mb_off, scal, acc_counts,
+                                                          acc_tokens, sp_off, perm, pos);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_route_scatter(const int32_t* idx, int T, int k, int N, int E, const int32_t* chunk_base,
                                  int32_t* perm, int32_t* pos, cudaStream_t s) {
   const int nchunks = (T + kChunk - 1) / kChunk;
@@ -476,14 +570,22 @@ cudaError_t launch_combine(int bf16, const void* x, const void* Y, const int32_t
                            const int32_t* pos, int T, int k, int N, int d, void* y, int sms, cudaStream_t s,
                            const int32_t* offsets, const int32_t* mb_off) {
   (void)N;
-  (void)sms;
-  if (bf16)
-    k_combine<__nv_bfloat16><<<T, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
-                                               static_cast<const __nv_bfloat16*>(Y), gate, pos, T, k, d,
-                                               static_cast<__nv_bfloat16*>(y), idx, offsets, mb_off);
-  else
-    k_combine<float><<<T, 128, 0, s>>>(static_cast<const float*>(x), static_cast<const float*>(Y), gate, pos, T, k, d,
-                                       static_cast<float*>(y), idx, offsets, mb_off);
+  const int nv = d / (bf16 ? 8 : 4);
+  const bool small = T < sms * 16;  // fewer tokens than 16 blocks per SM
+  const dim3 grid((unsigned)T, small ? (unsigned)((nv + 127) / 128) : 1u);
+  if (bf16) {
+    auto x_ = static_cast<const __nv_bfloat16*>(x);
+    auto Y_ = static_cast<const __nv_bfloat16*>(Y);
+    auto y_ = static_cast<__nv_bfloat16*>(y);
+    if (small) k_combine<__nv_bfloat16, 8><<<grid, 128, 0, s>>>(x_, Y_, gate, pos, T, k, d, y_, idx, offsets, mb_off);
+    else k_combine<__nv_bfloat16, 1><<<grid, 128, 0, s>>>(x_, Y_, gate, pos, T, k, d, y_, idx, offsets, mb_off);
+  } else {
+    auto x_ = static_cast<const float*>(x);
+    auto Y_ = static_cast<const float*>(Y);
+    auto y_ = static_cast<float*>(y);
+    if (small) k_combine<float, 8><<<grid, 128, 0, s>>>(x_, Y_, gate, pos, T, k, d, y_, idx, offsets, mb_off);
+    else k_combine<float, 1><<<grid, 128, 0, s>>>(x_, Y_, gate, pos, T, k, d, y_, idx, offsets, mb_off);
+  }
   return cudaGetLastError();
 }
 

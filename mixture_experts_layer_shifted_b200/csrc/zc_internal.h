@@ -48,6 +48,11 @@ cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int32_t*
 cudaError_t launch_route_scan(int32_t* chunk_cnt, int nchunks, int T, int N, int E, int32_t* counts, int32_t* offsets,
                               int32_t* mb_off, int32_t* scal, int64_t* acc_counts, int64_t* acc_tokens, cudaStream_t s,
                               int32_t* sp_off = nullptr);
+// The three integer-stage kernels in one block for T <= route_small_max_tokens() (same results).
+int route_small_max_tokens();
+cudaError_t launch_route_small(const int32_t* idx, int T, int k, int N, int E, int32_t* counts, int32_t* offsets,
+                               int32_t* mb_off, int32_t* scal, int64_t* acc_counts, int64_t* acc_tokens,
+                               int32_t* sp_off, int32_t* perm, int32_t* pos, cudaStream_t s);
 cudaError_t launch_route_scatter(const int32_t* idx, int T, int k, int N, int E, const int32_t* chunk_base,
                                  int32_t* perm, int32_t* pos, cudaStream_t s);
 cudaError_t launch_gather_rows(const void* x, int row_bytes, const int32_t* perm, int k, const int32_t* scal,

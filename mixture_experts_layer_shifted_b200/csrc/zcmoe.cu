@@ -640,6 +640,11 @@ static int router_stage(zcmoe_t h, const void* x, int Ti, cudaStream_t s) {
 // row-block offsets, the permutation of the FFN pairs, the slot positions
 static int integer_stage(zcmoe_t h, int Ti, cudaStream_t s) {
   const int E = h->E, N = h->N, k = h->k;
+  if (Ti <= zc::route_small_max_tokens()) {  // one launch for a small batch
+    ZC_CUDA(zc::launch_route_small(h->idx, Ti, k, N, E, h->counts, h->offsets, h->mb_off, h->scal, h->acc_counts,
+                                   h->acc_tokens, h->sp_off, h->perm, h->pos, s));
+    return ZCMOE_OK;
+  }
   const int nchunks = (Ti + zc::kChunk - 1) / zc::kChunk;
   ZC_CUDA(zc::launch_route_count(h->idx, Ti, k, E, h->chunk, s));
   ZC_CUDA(zc::launch_route_scan(h->chunk, nchunks, Ti, N, E, h->counts, h->offsets, h->mb_off, h->scal,
