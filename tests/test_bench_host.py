@@ -68,10 +68,11 @@ def test_roofline_picks_the_slower_side():
     assert bench.roofline_ms(wl, F, B, PEAKS) == pytest.approx(1e3 * B / (PEAKS["hbm_gbs"] * 1e9), rel=1e-12)
 
 
-@pytest.mark.parametrize("fmt,wbytes,mult", [("fp8", 1, 2), ("fp4", 0.5, 4)])
+@pytest.mark.parametrize("fmt,wbytes,mult", [("fp8", 1, 2), ("fp4", 0.5 + 1 / 32, 4), ("nvfp4", 0.5 + 1 / 16, 4)])
 def test_low_precision_experts(fmt, wbytes, mult):
-    """FP8 / MXFP4 experts: weights stream at 1 / 0.5 bytes per element, the router
-    and x, y stay bf16, and the expert GEMMs run at 2x / 4x the bf16 rate."""
+    """FP8 / MXFP4 / NVFP4 experts: weights stream at 1 / 0.5 bytes per element (codes)
+    plus one scale byte per 32 (MXFP4) or 16 (NVFP4) elements, the router and x, y stay
+    bf16, and the expert GEMMs run at 2x / 4x / 4x the bf16 rate."""
     wl = W[f"prefill_560b_{fmt}"]
     P, distinct = 131072, 512
     F, B = bench.algorithmic_work(wl, P, distinct)
