@@ -319,6 +319,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // overwrite mode: an expert with no rows has a zero gradient (no MMA, no TMEM)
           constexpr int NB = NBUF > 0 ? NBUF : 1;
           const int m0 = ti.m_blk * BM + quarter * 32;
+          // rows from m_split on belong to the second accumulator (tensor map b1)
+          const bool second = args.m_split > 0 && m0 >= args.m_split;
+          const CUtensorMap* tc = second ? &tmB1 : &tmC;
+          const int mc = second ? m0 - args.m_split : m0;
 #pragma unroll 1
           for (int c = 0; c < BN; c += 32) {
             const int n0 = ti.n_blk * BN + c;
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             fence_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_3d(&tmC, stg, n0, m0, ti.g);
+              tma_store_3d(tc, stg, n0, mc, ti.g);
               bulk_commit();
             }
             ++chunk;
@@ -529,8 +533,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else {
         // fused GemmAdd: acc[g][m][n] += product in fp32, done by TMA reduce-adds of
         // 32 x 32 boxes (the L2 does the read-modify-write; each element is added once);
-        // overwrite mode: TMA stores of the same boxes (acc[g][m][n] = product)
+        // overwrite mode: TMA stores of the same boxes (acc[g][m][n] = product).  With m_split,
+        // one launch serves two accumulators (dW_g and dW_u over [dG | dU]): rows from m_split
+        // on go to the second one (tensor map b1) at row - m_split
         const int m0 = ti.m_blk * BM + quarter * 32;
+        const bool second = args.m_split > 0 && m0 >= args.m_split;
+        const CUtensorMap* tc = second ? &tmB1 : &tmC;
+        const int mc = second ? m0 - args.m_split : m0;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t r[32];
@@ -549,8 +558,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           fence_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (args.overwrite) tma_store_3d(&tmC, stg, n0, m0, ti.g);
-            else tma_reduce_add_3d(&tmC, stg, n0, m0, ti.g);
+            if (args.overwrite) tma_store_3d(tc, stg, n0, mc, ti.g);
+            else tma_reduce_add_3d(tc, stg, n0, mc, ti.g);
             bulk_commit();
           }
           ++chunk;

@@ -208,11 +208,14 @@ struct BwdArgs {
   float* acc;                // kEpiAddF32: acc[g][m][n] += product (through the tensor map c)
   int overwrite;             //   1: acc[g][m][n] = product instead (experts with no rows get zeros)
   int64_t acc_ld, acc_group_stride;
+  int m_split;               //   > 0: output rows >= m_split go to a second accumulator (tensor map b1) at
+                             //   row - m_split (a multiple of 32), so dW_g and dW_u come from one launch
   int* err;                  // device error word (bounded waits)
 };
 int bwd_smem_bytes();
 // c: kBwdWgrad -- the fp32 accumulator as a 3-D tensor [groups][m_out][n_out], box 32 x 32 x 1,
-// 128-byte swizzle (the reduce-add target); kBwdRowsMnB -- the bf16 output [rows, n_out], box
+// 128-byte swizzle (the reduce-add target; with m_split, b1 is the second accumulator's map);
+// kBwdRowsMnB -- the bf16 output [rows, n_out], box
 // 64 x 32, 128-byte swizzle (full 32-row groups leave by TMA stores); kBwdDhSwiglu -- [dG | dU]
 // [rows, 2 inter] bf16, box 32 x 32, no swizzle, with H [rows, inter] the same way as b1; other
 // kinds ignore it.

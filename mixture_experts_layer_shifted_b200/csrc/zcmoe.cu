@@ -1529,15 +1529,19 @@ int zcmoe_backward_ex(zcmoe_t h, const void* x, const void* dy, int64_t T, void*
   // dx: the deterministic ScatterAdd
   ZC_CUDA(zc::launch_final_dx(dy, h->b_dxp, h->b_dxr, h->gate, h->pos, h->idx, h->offsets, h->mb_off, Ti, k, d, dx, s));
   // weight gradients, added into the fp32 accumulators in the GEMM epilogue
+  // acc2 (optional): a second accumulator of the same shape for A's next m_out columns, so that
+  // one launch reads B once for both (dW_g and dW_u over [dG | dU] and X)
   auto wgrad = [&](const CUtensorMap& A, const CUtensorMap& B, int a_col0, int m_out, int n_out, float* acc,
-                   int64_t stride, int groups, const int32_t* row_off, const int32_t* mb_off) -> int {
+                   int64_t stride, int groups, const int32_t* row_off, const int32_t* mb_off,
+                   float* acc2 = nullptr) -> int {
     zc::BwdArgs a{};
     a.ngroups = groups;
     a.row_off = row_off;
     a.mb_off = mb_off;
     a.a_col0 = a_col0;
-    a.m_out = m_out;
-    a.mblocks = (m_out + 127) / 128;
+    a.m_out = acc2 ? 2 * m_out : m_out;
+    a.m_split = acc2 ? m_out : 0;
+    a.mblocks = (a.m_out + 127) / 128;
     a.n_out = n_out;
     a.nblocks = (n_out + 255) / 256;
     a.acc = acc;
@@ -1545,18 +1549,25 @@ int zcmoe_backward_ex(zcmoe_t h, const void* x, const void* dy, int64_t T, void*
     a.acc_ld = n_out;
     a.acc_group_stride = stride;
     a.err = h->err;
-    CUtensorMap tmc;
-    const int rc2 = make_tmap_acc(&tmc, acc, (uint64_t)n_out, (uint64_t)m_out, (uint64_t)groups);
+    CUtensorMap tmc, tmc2;
+    int rc2 = make_tmap_acc(&tmc, acc, (uint64_t)n_out, (uint64_t)m_out, (uint64_t)groups);
+    if (rc2 == ZCMOE_OK && acc2) rc2 = make_tmap_acc(&tmc2, acc2, (uint64_t)n_out, (uint64_t)m_out, (uint64_t)groups);
     if (rc2 != ZCMOE_OK) return rc2;
-    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdWgrad, A, B, B, tmc, a, grid_for((int64_t)groups * a.mblocks * a.nblocks), s));
+    ZC_CUDA(zc::launch_bwd_gemm(zc::kBwdWgrad, A, B, acc2 ? tmc2 : B, tmc, a,
+                                grid_for((int64_t)groups * a.mblocks * a.nblocks), s));
     return ZCMOE_OK;
   };
   if (g_down && (rc = wgrad(tm_dy_mn, tm_h_mn, 0, d, inter, g_down, (int64_t)d * inter, N, h->offsets, h->mb_off)))
     return rc;
-  if (g_gate && (rc = wgrad(tm_dgu_mn, tm_x_mn, 0, inter, d, g_gate, (int64_t)inter * d, N, h->offsets, h->mb_off)))
-    return rc;
-  if (g_up && (rc = wgrad(tm_dgu_mn, tm_x_mn, inter, inter, d, g_up, (int64_t)inter * d, N, h->offsets, h->mb_off)))
-    return rc;
+  if (g_gate && g_up) {  // both from one launch over [dG | dU]: X is read once
+    if ((rc = wgrad(tm_dgu_mn, tm_x_mn, 0, inter, d, g_gate, (int64_t)inter * d, N, h->offsets, h->mb_off, g_up)))
+      return rc;
+  } else {
+    if (g_gate && (rc = wgrad(tm_dgu_mn, tm_x_mn, 0, inter, d, g_gate, (int64_t)inter * d, N, h->offsets, h->mb_off)))
+      return rc;
+    if (g_up && (rc = wgrad(tm_dgu_mn, tm_x_mn, inter, inter, d, g_up, (int64_t)inter * d, N, h->offsets, h->mb_off)))
+      return rc;
+  }
   if (g_router && (rc = wgrad(tm_dl_mn, tm_xin_mn, 0, E, d, g_router, 0, 1, h->b_grp, h->b_grp + 2))) return rc;
   return ZCMOE_OK;
 }

@@ -155,10 +155,12 @@ def test_backward_ragged(cuda_ok, T, d, N, inter, Z, k, saved):
     r.close()
 
 
-@pytest.mark.parametrize("names", [("router",), ("gate", "down"), ()], ids=["router-only", "gate+down", "dx-only"])
+@pytest.mark.parametrize("names", [("router",), ("gate", "down"), ("up",), ("gate", "up"), ()],
+                         ids=["router-only", "gate+down", "up-only", "gate+up", "dx-only"])
 def test_backward_gradient_subsets(cuda_ok, names):
     """Any subset of the weight gradients (NULL skips one): the requested ones are added,
-    dx is unchanged."""
+    dx is unchanged.  dW_g and dW_u together come from one launch over [dG | dU] (two
+    accumulators); either alone from a launch of its own."""
     w = W["small_bf16"]
     r = Run(w)
     try:
