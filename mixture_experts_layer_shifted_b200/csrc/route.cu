@@ -370,11 +370,12 @@ struct Vec<float> {
 
 // Large batches: one block per token, its threads striding over the row's vectors, one
 // slot's load at a time (G = 1) -- many resident blocks keep the most loads in flight
-// (~91% of the HBM copy rate measured on B200).  Small batches (decode): one block per
-// (token, 128 vectors), and G = 8 slots' loads issued together before their products
-// are added, since the blocks are few and each thread's loads would otherwise wait one
+// (~91% of the HBM copy rate measured on B200).  Smaller batches: one block per (token,
+// 128 vectors); and when even those blocks are few (decode), G = 8 slots' loads issued
+// together before their products are added, so that a thread's loads do not wait one
 // after another.  The products are added in slot order either way, so the result is the
-// same.
+// same.  (At 2048 tokens the G = 8 form took twice the time of the one-block-per-token form,
+// 118 against 56 us, hence the thresholds.)
 // With offsets / mb_off (FP8 layers), Y holds expert e's pairs from padded row
 // 128 mb_off[e] on, so a pair's row is pos - offsets[e] + 128 mb_off[e].
 template <typename TIO, int G>
@@ -571,8 +572,10 @@ cudaError_t launch_combine(int bf16, const void* x, const void* Y, const int32_t
                            const int32_t* offsets, const int32_t* mb_off) {
   (void)N;
   const int nv = d / (bf16 ? 8 : 4);
-  const bool small = T < sms * 16;  // fewer tokens than 16 blocks per SM
-  const dim3 grid((unsigned)T, small ? (unsigned)((nv + 127) / 128) : 1u);
+  const int split = (nv + 127) / 128;
+  const bool wide = T < sms * 8;                                 // < 8 token blocks per SM: split the rows
+  const bool small = wide && (int64_t)T * split <= (int64_t)sms * 8;  // still < 8 blocks per SM: G = 8
+  const dim3 grid((unsigned)T, wide ? (unsigned)split : 1u);
   if (bf16) {
     auto x_ = static_cast<const __nv_bfloat16*>(x);
     auto Y_ = static_cast<const __nv_bfloat16*>(Y);
