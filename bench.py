@@ -1,7 +1,7 @@
 """Benchmark of the zero-computation-expert MoE layer forward on B200.
 
 One step = one pass of the whole hot path over one batch: router GEMM +
-softmax/top-k + integer stage + gather + grouped gate/up GEMM + grouped down
+softmax/top-k + integer stage + row scatter + grouped gate/up GEMM + grouped down
 GEMM + combine (zcmoe_forward), then the bias controller step
 (zcmoe_update_bias; with N > 1 ranks the selection counts are summed over the
 ranks with one NCCL all-reduce first, so every replica takes the same step).
@@ -535,9 +535,11 @@ def run_ep(args, wl, dist, rank, ws, local, peaks):
             "cpu_baseline": cpu,
             "e2e": {"value": wl.T * ws / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": io,
                     "d2h_bytes_per_step": io, "ms_per_step": e2e_ms},
-            # per chunk: router GEMM, softmax/top-k, 3 integer-stage kernels, gather, the two expert
-            # GEMMs (+ 2 regroups with ws > 1), combine; per step one bias update per chunk handle
-            "gpu_launches": args.steps * (nck * (9 + (2 if ws > 1 else 0)) + nck), "clocks": clocks, "peaks": peaks,
+            # per chunk: router GEMM, softmax/top-k, the integer stage (one kernel up to 1024 tokens,
+            # else three), the row scatter, the two expert GEMMs (+ 2 regroups with ws > 1), combine;
+            # per step one bias update per chunk handle
+            "gpu_launches": args.steps * (nck * (6 + (1 if wl.T // nck <= 1024 else 3) + (2 if ws > 1 else 0)) + nck),
+            "clocks": clocks, "peaks": peaks,
             "launch": "eager (host-side split sizes)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -746,7 +748,9 @@ def main():
                        "realised": {"P": P, "ffn_per_token": P / wl.T, "distinct_experts": distinct,
                                     "zero_fraction": 1.0 - P / (wl.T * k)}},
             "roofline": roofline, "layer_roofline": layer_roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": 10 * args.steps, "clocks": clocks, "peaks": peaks,
+            # router GEMM, softmax/top-k, the integer stage (one kernel up to 1024 tokens, else
+            # three), the row scatter (or quantizing gather), gate/up, down, combine, bias update
+            "gpu_launches": (7 + (1 if wl.T <= 1024 else 3)) * args.steps, "clocks": clocks, "peaks": peaks,
             "launch": "cuda graph per step" if use_graph else "eager"}
 
     # the controller over the workload's steps (Zipf-skewed routing): FFN experts per token per

@@ -306,26 +306,38 @@ __global__ void __launch_bounds__(kChunk) k_route_scatter(const int32_t* __restr
   }
 }
 
-// X_perm[p] = x[perm[p] / k] for p < P (P read from the device).  One warp per
-// row, 16-byte vectors, four loads in flight per lane.
-__global__ void __launch_bounds__(256) k_gather_rows(const uint4* __restrict__ x, int row_vecs,
-                                                     const int32_t* __restrict__ perm, int k,
-                                                     const int32_t* __restrict__ scal, uint4* __restrict__ xperm) {
-  const int P = scal[0];
+// X_perm[pos[t, j]] = x[t] for every FFN slot of every token: the FFN pairs' rows in
+// expert order, written from the token side.  One warp per token reads its row once, four
+// 16-byte vectors per lane per round, and writes each round to all of the token's FFN rows.
+// (Reading per pair instead -- X_perm[p] = x[token of p], one warp per row -- fetched each
+// token's row up to k times, about twice its bytes from DRAM, and took 0.50 against 0.36-0.39
+// ms at prefill_560b.)
+__global__ void __launch_bounds__(256) k_scatter_rows(const uint4* __restrict__ x, int row_vecs,
+                                                      const int32_t* __restrict__ pos, int T, int k,
+                                                      uint4* __restrict__ xperm) {
   const int lane = threadIdx.x & 31;
   const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
-  for (int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); p < P; p += nwarps) {
-    const uint4* src = x + (int64_t)(perm[p] / k) * row_vecs;
-    uint4* dst = xperm + (int64_t)p * row_vecs;
-    int v = lane;
-    for (; v + 96 < row_vecs; v += 128) {
-      const uint4 a = src[v], b = src[v + 32], c = src[v + 64], d = src[v + 96];
-      dst[v] = a;
-      dst[v + 32] = b;
-      dst[v + 64] = c;
-      dst[v + 96] = d;
+  for (int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); t < T; t += nwarps) {
+    const int my_p = lane < k ? pos[(int64_t)t * k + lane] : -1;  // slot `lane`'s FFN row (-1: zero expert)
+    const uint4* src = x + (int64_t)t * row_vecs;
+    for (int v0 = 0; v0 < row_vecs; v0 += 128) {
+      uint4 a[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + 32 * u + lane;
+        if (v < row_vecs) a[u] = src[v];
+      }
+      for (int j = 0; j < k; ++j) {
+        const int p = __shfl_sync(0xffffffffu, my_p, j);
+        if (p < 0) continue;
+        uint4* dst = xperm + (int64_t)p * row_vecs;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int v = v0 + 32 * u + lane;
+          if (v < row_vecs) dst[v] = a[u];
+        }
+      }
     }
-    for (; v < row_vecs; v += 32) dst[v] = src[v];
   }
 }
 
@@ -560,10 +572,13 @@ cudaError_t launch_route_scatter(const int32_t* idx, int T, int k, int N, int E,
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather_rows(const void* x, int row_bytes, const int32_t* perm, int k, const int32_t* scal,
-                               void* xperm, int sms, cudaStream_t s) {
-  k_gather_rows<<<sms * 8, 256, 0, s>>>(static_cast<const uint4*>(x), row_bytes / 16, perm, k, scal,
-                                        static_cast<uint4*>(xperm));
+cudaError_t launch_scatter_rows(const void* x, int row_bytes, const int32_t* pos, int T, int k, void* xperm, int sms,
+                                cudaStream_t s) {
+  int64_t blocks = ((int64_t)T + 7) / 8;
+  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+  if (blocks < 1) blocks = 1;
+  k_scatter_rows<<<(int)blocks, 256, 0, s>>>(static_cast<const uint4*>(x), row_bytes / 16, pos, T, k,
+                                             static_cast<uint4*>(xperm));
   return cudaGetLastError();
 }
 

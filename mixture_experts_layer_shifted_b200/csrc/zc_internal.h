@@ -55,8 +55,9 @@ cudaError_t launch_route_small(const int32_t* idx, int T, int k, int N, int E, i
                                int32_t* sp_off, int32_t* perm, int32_t* pos, cudaStream_t s);
 cudaError_t launch_route_scatter(const int32_t* idx, int T, int k, int N, int E, const int32_t* chunk_base,
                                  int32_t* perm, int32_t* pos, cudaStream_t s);
-cudaError_t launch_gather_rows(const void* x, int row_bytes, const int32_t* perm, int k, const int32_t* scal,
-                               void* xperm, int sms, cudaStream_t s);
+// X_perm[pos[t, j]] = x[t] for every FFN slot (pos >= 0): the pairs' rows in expert order
+cudaError_t launch_scatter_rows(const void* x, int row_bytes, const int32_t* pos, int T, int k, void* xperm, int sms,
+                                cudaStream_t s);
 // offsets / mb_off non-null: Y rows are padded (FP8 layers), see k_combine.
 cudaError_t launch_combine(int bf16, const void* x, const void* Y, const int32_t* idx, const float* gate,
                            const int32_t* pos, int T, int k, int N, int d, void* y, int sms, cudaStream_t s,

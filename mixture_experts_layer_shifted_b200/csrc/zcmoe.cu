@@ -742,7 +742,7 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     ZC_CUDA(zc::launch_gather_quant(x, d, h->perm, h->idx, k, h->offsets, h->mb_off, h->scal, h->x8, h->sx, h->gd,
                                     h->sms, s));
   else
-    ZC_CUDA(zc::launch_gather_rows(x, (int)(d * esz), h->perm, k, h->scal, h->xperm, h->sms, s));
+    ZC_CUDA(zc::launch_scatter_rows(x, (int)(d * esz), h->pos, Ti, k, h->xperm, h->sms, s));
   ZC_CUDA(mark("zcmoe.gate_up"));
   // 5./6. expert GEMMs
   const int max_mb = (Ti * k + zc::kBM - 1) / zc::kBM + N;
@@ -918,7 +918,7 @@ int zcmoe_ep_dispatch(zcmoe_t h, const void* x, int64_t T, void* xsend, int32_t*
                                   dbg ? dbg->scores : nullptr, h->sms, s));
   rc = integer_stage(h, Ti, s);
   if (rc != ZCMOE_OK) return rc;
-  ZC_CUDA(zc::launch_gather_rows(x, h->d * 2, h->perm, h->k, h->scal, xsend, h->sms, s));
+  ZC_CUDA(zc::launch_scatter_rows(x, h->d * 2, h->pos, Ti, h->k, xsend, h->sms, s));
   ZC_CUDA(cudaMemcpyAsync(offsets, h->offsets, (size_t)(h->N + 1) * sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
   if (dbg) return copy_routing_debug(h, Ti, dbg, s);
   return ZCMOE_OK;
