@@ -1,11 +1,10 @@
 // Block quantizers to FP8 E4M3 with E8M0 power-of-two scales (rule in zc_fp8.cuh):
 //   k_quant_rows  : [1,128] blocks (activations), one warp per block
 //   k_quant_tiles : [128,128] blocks (weights), one CTA per block
-//   k_gather_quant: the FFN pairs' token rows, quantized per [1,128] on the way
-//                   into the expert-sorted operand of the FP8 gate/up GEMM
-// and their W4A4 forms: MXFP4 ([1,32] blocks, k_quant_mx4 / k_gather_quant4) and
-// NVFP4 ([1,16] blocks with a tensor scale: k_matrix_amax + k_nv4_global, then
-// k_quant_nv4 / k_gather_quant_nv4).
+//   k_scatter_quant: the FFN pairs' token rows, quantized on the way into the padded,
+//                   expert-sorted operand of the block-scaled gate/up GEMM (all formats)
+// and their W4A4 forms: MXFP4 ([1,32] blocks, k_quant_mx4) and NVFP4 ([1,16] blocks with a
+// tensor scale: k_matrix_amax + k_nv4_global, then k_quant_nv4).
 // Scales go out either plain ([row blocks, cols/128], for zcmoe_quantize_e4m3)
 // or as the GEMM's scale atoms.
 #include <cuda_bf16.h>
@@ -93,74 +92,11 @@ __global__ void __launch_bounds__(128) k_quant_tiles(const TIN* __restrict__ src
   }
 }
 
-// FFN pair p (expert e, token t = perm[p] / k) goes to padded row
-// p - offsets[e] + 128 * mb_off[e], so every expert's rows start a 128-row block.
-// Eight bf16 values per lane per 16-byte load: a warp-wide load covers 256 columns, the
-// two 128-column blocks of lanes 0..15 and 16..31; four loads in flight per lane.
-__device__ __forceinline__ void ld8_bf16(const __nv_bfloat16* p, float* v) {
-  const uint4 r = *reinterpret_cast<const uint4*>(p);
-  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-    v[2 * i] = f.x;
-    v[2 * i + 1] = f.y;
-  }
-}
+// Largest value over the 16 lanes of a half warp: an FP8 [1,128] block, eight elements a lane.
 __device__ __forceinline__ float half_warp_max(float a) {
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
   return a;
-}
-// the lane's eight values of one [1,128] block: codes to dst, the block's scale (lanes 0 and 16)
-__device__ __forceinline__ void quant8_e4m3(const float* v, uint8_t* dst, uint8_t* scale, int lane) {
-  float m = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
-  const uint32_t code = e8m0_code(half_warp_max(m));
-  const float inv = e8m0_inverse(code);
-  *reinterpret_cast<uint2*>(dst) = make_uint2(pack_e4m3x4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv),
-                                              pack_e4m3x4(v[4] * inv, v[5] * inv, v[6] * inv, v[7] * inv));
-  if ((lane & 15) == 0) *scale = (uint8_t)code;
-}
-
-__global__ void __launch_bounds__(256) k_gather_quant(const __nv_bfloat16* __restrict__ x, int d,
-                                                      const int32_t* __restrict__ perm,
-                                                      const int32_t* __restrict__ idx, int k,
-                                                      const int32_t* __restrict__ offsets,
-                                                      const int32_t* __restrict__ mb_off,
-                                                      const int32_t* __restrict__ scal, uint8_t* __restrict__ x8,
-                                                      uint8_t* __restrict__ sx, int groups) {
-  const int P = scal[0];
-  const int lane = threadIdx.x & 31;
-  const int half = lane >> 4;
-  const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
-  for (int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); p < P; p += nwarps) {
-    const int pair = perm[p];
-    const int e = idx[pair];
-    const int64_t pad = (int64_t)(p - offsets[e]) + (int64_t)mb_off[e] * 128;
-    const __nv_bfloat16* src = x + (int64_t)(pair / k) * d;
-    uint8_t* dst = x8 + pad * d;
-    int c0 = 0;
-    for (; c0 + 1024 <= d; c0 += 1024) {
-      float v[4][8];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) ld8_bf16(src + c0 + 256 * u + lane * 8, v[u]);
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        quant8_e4m3(v[u], dst + c0 + 256 * u + lane * 8, sx + atom_offset(pad, ((c0 + 256 * u) >> 7) + half, groups),
-                    lane);
-    }
-    if (c0 < d) {  // d is a multiple of 512: a last 512 columns
-      float v[2][8];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) ld8_bf16(src + c0 + 256 * u + lane * 8, v[u]);
-#pragma unroll
-      for (int u = 0; u < 2; ++u)
-        quant8_e4m3(v[u], dst + c0 + 256 * u + lane * 8, sx + atom_offset(pad, ((c0 + 256 * u) >> 7) + half, groups),
-                    lane);
-    }
-  }
 }
 
 // ---------------------------------------------------------------- MXFP4 ([1,32] blocks)
@@ -210,51 +146,6 @@ __global__ void __launch_bounds__(256) k_quant_mx4(const TIN* __restrict__ src, 
     const uint2 q = quant8_mx4(v);
     *reinterpret_cast<uint32_t*>(codes + r * (cols >> 1) + (c >> 1)) = q.x;
     if ((lane & 3) == 0) scales[ATOM ? atom_offset(r, c >> 5, groups) : r * (cols >> 5) + (c >> 5)] = (uint8_t)q.y;
-  }
-}
-
-// MXFP4 form of k_gather_quant (same padded rows); d a multiple of 512.
-__global__ void __launch_bounds__(256) k_gather_quant4(const __nv_bfloat16* __restrict__ x, int d,
-                                                       const int32_t* __restrict__ perm,
-                                                       const int32_t* __restrict__ idx, int k,
-                                                       const int32_t* __restrict__ offsets,
-                                                       const int32_t* __restrict__ mb_off,
-                                                       const int32_t* __restrict__ scal, uint8_t* __restrict__ x4,
-                                                       uint8_t* __restrict__ sx, int groups) {
-  const int P = scal[0];
-  const int lane = threadIdx.x & 31;
-  const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
-  for (int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); p < P; p += nwarps) {
-    const int pair = perm[p];
-    const int e = idx[pair];
-    const int64_t pad = (int64_t)(p - offsets[e]) + (int64_t)mb_off[e] * 128;
-    const __nv_bfloat16* src = x + (int64_t)(pair / k) * d;
-    uint8_t* dst = x4 + pad * (d >> 1);
-    int c0 = 0;
-    for (; c0 + 1024 <= d; c0 += 1024) {  // four 16-byte loads in flight per lane
-      float v[4][8];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) ld8(src + c0 + 256 * u + lane * 8, v[u]);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = c0 + 256 * u + lane * 8;
-        const uint2 q = quant8_mx4(v[u]);
-        *reinterpret_cast<uint32_t*>(dst + (c >> 1)) = q.x;
-        if ((lane & 3) == 0) sx[atom_offset(pad, c >> 5, groups)] = (uint8_t)q.y;
-      }
-    }
-    if (c0 < d) {  // d is a multiple of 512: a last 512 columns
-      float v[2][8];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) ld8(src + c0 + 256 * u + lane * 8, v[u]);
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int c = c0 + 256 * u + lane * 8;
-        const uint2 q = quant8_mx4(v[u]);
-        *reinterpret_cast<uint32_t*>(dst + (c >> 1)) = q.x;
-        if ((lane & 3) == 0) sx[atom_offset(pad, c >> 5, groups)] = (uint8_t)q.y;
-      }
-    }
   }
 }
 
@@ -327,46 +218,78 @@ __global__ void __launch_bounds__(256) k_quant_nv4(const TIN* __restrict__ src, 
   }
 }
 
-// NVFP4 form of k_gather_quant (same padded rows, g = 1); d a multiple of 512.
-__global__ void __launch_bounds__(256) k_gather_quant_nv4(const __nv_bfloat16* __restrict__ x, int d,
-                                                          const int32_t* __restrict__ perm,
-                                                          const int32_t* __restrict__ idx, int k,
-                                                          const int32_t* __restrict__ offsets,
-                                                          const int32_t* __restrict__ mb_off,
-                                                          const int32_t* __restrict__ scal, uint8_t* __restrict__ x4,
-                                                          uint8_t* __restrict__ sx, int groups) {
-  const int P = scal[0];
+// ---------------------------------------------------------------- the FFN pairs' rows, quantized
+// The x rows of the FFN pairs into the padded expert-order operand (pair p of expert e at row
+// p - offsets[e] + 128 mb_off[e]), written from the token side: a warp takes one (token, 1024
+// columns) item at a time, reads and quantizes it once (the codes and scales depend only on
+// the row), then writes them to each of the token's FFN rows.  FMT 0: FP8 E4M3 per [1,128];
+// 1: MXFP4 per [1,32]; 2: NVFP4 per [1,16] (g = 1).  d a multiple of 512 (a last item may hold
+// 512 columns); lanes hold eight consecutive elements, a warp-wide load 256 columns.
+template <int FMT>
+__global__ void __launch_bounds__(256) k_scatter_quant(const __nv_bfloat16* __restrict__ x, int d,
+                                                       const int32_t* __restrict__ pos,
+                                                       const int32_t* __restrict__ idx, int T, int k,
+                                                       const int32_t* __restrict__ offsets,
+                                                       const int32_t* __restrict__ mb_off,
+                                                       uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                       int groups) {
   const int lane = threadIdx.x & 31;
   const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
-  for (int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); p < P; p += nwarps) {
-    const int pair = perm[p];
-    const int e = idx[pair];
-    const int64_t pad = (int64_t)(p - offsets[e]) + (int64_t)mb_off[e] * 128;
-    const __nv_bfloat16* src = x + (int64_t)(pair / k) * d;
-    uint8_t* dst = x4 + pad * (d >> 1);
-    int c0 = 0;
-    for (; c0 + 1024 <= d; c0 += 1024) {  // four 16-byte loads in flight per lane
-      float v[4][8];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) ld8(src + c0 + 256 * u + lane * 8, v[u]);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = c0 + 256 * u + lane * 8;
-        const uint2 q = quant8_nv4(v[u], 1.0f);
-        *reinterpret_cast<uint32_t*>(dst + (c >> 1)) = q.x;
-        if ((lane & 1) == 0) sx[atom_offset(pad, c >> 4, groups)] = (uint8_t)q.y;
+  const int64_t row_bytes = FMT == 0 ? d : d / 2;
+  const int nchunks = (d + 1023) / 1024;
+  const int64_t items = (int64_t)T * nchunks;
+  for (int64_t it = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
+    const int t = (int)(it / nchunks);
+    const int c0 = (int)(it - (int64_t)t * nchunks) * 1024;
+    int my_pad = -1;  // lane j < k: the padded row of the token's slot j (-1: a zero expert)
+    if (lane < k) {
+      const int p = pos[(int64_t)t * k + lane];
+      if (p >= 0) {
+        const int e = idx[(int64_t)t * k + lane];
+        my_pad = p - offsets[e] + mb_off[e] * 128;
       }
     }
-    if (c0 < d) {  // d is a multiple of 512: a last 512 columns
-      float v[2][8];
+    const __nv_bfloat16* src = x + (int64_t)t * d;
+    {
+      const int nu = d - c0 >= 1024 ? 4 : 2;  // d is a multiple of 512: a last 512 columns
+      float v[4][8];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) ld8(src + c0 + 256 * u + lane * 8, v[u]);
+      for (int u = 0; u < 4; ++u)
+        if (u < nu) ld8(src + c0 + 256 * u + lane * 8, v[u]);
+      uint2 q[4];       // the lane's codes: FMT 0 eight E4M3 bytes; FP4 eight E2M1 nibbles in x
+      uint32_t sc[4];   // the scale code of the lane's block
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int c = c0 + 256 * u + lane * 8;
-        const uint2 q = quant8_nv4(v[u], 1.0f);
-        *reinterpret_cast<uint32_t*>(dst + (c >> 1)) = q.x;
-        if ((lane & 1) == 0) sx[atom_offset(pad, c >> 4, groups)] = (uint8_t)q.y;
+      for (int u = 0; u < 4; ++u) {
+        if (u >= nu) break;
+        if (FMT == 0) {
+          float m = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[u][i]));
+          sc[u] = e8m0_code(half_warp_max(m));
+          const float inv = e8m0_inverse(sc[u]);
+          q[u] = make_uint2(pack_e4m3x4(v[u][0] * inv, v[u][1] * inv, v[u][2] * inv, v[u][3] * inv),
+                            pack_e4m3x4(v[u][4] * inv, v[u][5] * inv, v[u][6] * inv, v[u][7] * inv));
+        } else {
+          q[u] = FMT == 1 ? quant8_mx4(v[u]) : quant8_nv4(v[u], 1.0f);
+          sc[u] = q[u].y;
+        }
+      }
+      for (int j = 0; j < k; ++j) {
+        const int pad = __shfl_sync(0xffffffffu, my_pad, j);
+        if (pad < 0) continue;
+        uint8_t* dst = codes + (int64_t)pad * row_bytes;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (u >= nu) break;
+          const int c = c0 + 256 * u + lane * 8;
+          if (FMT == 0) {
+            *reinterpret_cast<uint2*>(dst + c) = q[u];
+            if ((lane & 15) == 0) scales[atom_offset(pad, c >> 7, groups)] = (uint8_t)sc[u];
+          } else {
+            *reinterpret_cast<uint32_t*>(dst + (c >> 1)) = q[u].x;
+            if ((lane & (FMT == 1 ? 3 : 1)) == 0) scales[atom_offset(pad, c >> (FMT == 1 ? 5 : 4), groups)] = (uint8_t)sc[u];
+          }
+        }
       }
     }
   }
@@ -436,11 +359,22 @@ cudaError_t launch_quant_mx4(int bf16, const void* src, int64_t rows, int cols, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather_quant4(const void* x, int d, const int32_t* perm, const int32_t* idx, int k,
-                                 const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x4,
-                                 uint8_t* sx, int groups, int sms, cudaStream_t s) {
-  k_gather_quant4<<<sms * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), d, perm, idx, k, offsets, mb_off, scal,
-                                           x4, sx, groups);
+cudaError_t launch_scatter_quant(int fmt, const void* x, int d, const int32_t* pos, const int32_t* idx, int T, int k,
+                                 const int32_t* offsets, const int32_t* mb_off, uint8_t* codes, uint8_t* scales,
+                                 int groups, int sms, cudaStream_t s) {
+  const int64_t items = (int64_t)T * ((d + 1023) / 1024);  // one warp per (token, 1024 columns)
+  int64_t blocks = (items + 7) / 8;
+  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+  if (blocks < 1) blocks = 1;
+  auto x_ = static_cast<const __nv_bfloat16*>(x);
+  if (fmt == 0)
+    k_scatter_quant<0><<<(int)blocks, 256, 0, s>>>(x_, d, pos, idx, T, k, offsets, mb_off, codes, scales, groups);
+  else if (fmt == 1)
+    k_scatter_quant<1><<<(int)blocks, 256, 0, s>>>(x_, d, pos, idx, T, k, offsets, mb_off, codes, scales, groups);
+  else if (fmt == 2)
+    k_scatter_quant<2><<<(int)blocks, 256, 0, s>>>(x_, d, pos, idx, T, k, offsets, mb_off, codes, scales, groups);
+  else
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
@@ -486,14 +420,6 @@ cudaError_t launch_quant_nv4(int bf16, const void* src, int64_t rows, int cols, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather_quant_nv4(const void* x, int d, const int32_t* perm, const int32_t* idx, int k,
-                                    const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x4,
-                                    uint8_t* sx, int groups, int sms, cudaStream_t s) {
-  k_gather_quant_nv4<<<sms * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), d, perm, idx, k, offsets, mb_off,
-                                              scal, x4, sx, groups);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_quant_tiles(int bf16, const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
                                int atom_groups, cudaStream_t s) {
   const dim3 grid(cols / 128, (unsigned)((rows + 127) / 128));
@@ -507,14 +433,6 @@ cudaError_t launch_quant_tiles(int bf16, const void* src, int64_t rows, int cols
     if (atom) k_quant_tiles<float, true><<<grid, 128, 0, s>>>(src_, rows, cols, codes, scales, atom_groups);
     else k_quant_tiles<float, false><<<grid, 128, 0, s>>>(src_, rows, cols, codes, scales, 0);
   }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_gather_quant(const void* x, int d, const int32_t* perm, const int32_t* idx, int k,
-                                const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x8,
-                                uint8_t* sx, int groups, int sms, cudaStream_t s) {
-  k_gather_quant<<<sms * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), d, perm, idx, k, offsets, mb_off, scal,
-                                          x8, sx, groups);
   return cudaGetLastError();
 }
 

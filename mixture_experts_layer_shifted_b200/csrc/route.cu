@@ -307,35 +307,37 @@ __global__ void __launch_bounds__(kChunk) k_route_scatter(const int32_t* __restr
 }
 
 // X_perm[pos[t, j]] = x[t] for every FFN slot of every token: the FFN pairs' rows in
-// expert order, written from the token side.  One warp per token reads its row once, four
-// 16-byte vectors per lane per round, and writes each round to all of the token's FFN rows.
-// (Reading per pair instead -- X_perm[p] = x[token of p], one warp per row -- fetched each
-// token's row up to k times, about twice its bytes from DRAM, and took 0.50 against 0.36-0.39
-// ms at prefill_560b.)
+// expert order, written from the token side.  A warp takes one (token, 2 KB column chunk)
+// item at a time: it reads the chunk once, four 16-byte vectors per lane, and writes it to
+// all of the token's FFN rows.  (Reading per pair instead -- X_perm[p] = x[token of p], one
+// warp per row -- fetched each token's row up to k times, about twice its bytes from DRAM, and
+// took 0.50 against 0.36-0.39 ms at prefill_560b.)
 __global__ void __launch_bounds__(256) k_scatter_rows(const uint4* __restrict__ x, int row_vecs,
                                                       const int32_t* __restrict__ pos, int T, int k,
                                                       uint4* __restrict__ xperm) {
   const int lane = threadIdx.x & 31;
   const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
-  for (int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); t < T; t += nwarps) {
+  const int nchunks = (row_vecs + 127) / 128;
+  const int64_t items = (int64_t)T * nchunks;
+  for (int64_t it = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
+    const int t = (int)(it / nchunks);
+    const int v0 = (int)(it - (int64_t)t * nchunks) * 128;
     const int my_p = lane < k ? pos[(int64_t)t * k + lane] : -1;  // slot `lane`'s FFN row (-1: zero expert)
     const uint4* src = x + (int64_t)t * row_vecs;
-    for (int v0 = 0; v0 < row_vecs; v0 += 128) {
-      uint4 a[4];
+    uint4 a[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int v = v0 + 32 * u + lane;
+      if (v < row_vecs) a[u] = src[v];
+    }
+    for (int j = 0; j < k; ++j) {
+      const int p = __shfl_sync(0xffffffffu, my_p, j);
+      if (p < 0) continue;
+      uint4* dst = xperm + (int64_t)p * row_vecs;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int v = v0 + 32 * u + lane;
-        if (v < row_vecs) a[u] = src[v];
-      }
-      for (int j = 0; j < k; ++j) {
-        const int p = __shfl_sync(0xffffffffu, my_p, j);
-        if (p < 0) continue;
-        uint4* dst = xperm + (int64_t)p * row_vecs;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int v = v0 + 32 * u + lane;
-          if (v < row_vecs) dst[v] = a[u];
-        }
+        if (v < row_vecs) dst[v] = a[u];
       }
     }
   }
@@ -574,7 +576,8 @@ cudaError_t launch_route_scatter(const int32_t* idx, int T, int k, int N, int E,
 
 cudaError_t launch_scatter_rows(const void* x, int row_bytes, const int32_t* pos, int T, int k, void* xperm, int sms,
                                 cudaStream_t s) {
-  int64_t blocks = ((int64_t)T + 7) / 8;
+  const int64_t items = (int64_t)T * ((row_bytes / 16 + 127) / 128);  // one warp per (token, 2 KB chunk)
+  int64_t blocks = (items + 7) / 8;
   if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
   if (blocks < 1) blocks = 1;
   k_scatter_rows<<<(int)blocks, 256, 0, s>>>(static_cast<const uint4*>(x), row_bytes / 16, pos, T, k,

@@ -114,26 +114,21 @@ cudaError_t launch_quant_rows(int bf16, const void* src, int64_t rows, int cols,
                               int atom_groups, int sms, cudaStream_t s);
 cudaError_t launch_quant_tiles(int bf16, const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
                                int atom_groups, cudaStream_t s);
-cudaError_t launch_gather_quant(const void* x, int d, const int32_t* perm, const int32_t* idx, int k,
-                                const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x8,
-                                uint8_t* sx, int groups, int sms, cudaStream_t s);
-
 // MXFP4: [1,32] blocks along each row (cols a multiple of 256), codes two per byte;
 // atom_groups > 0: scale atoms with that many atoms (128 elements each) per 128 rows.
 cudaError_t launch_quant_mx4(int bf16, const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
                              int atom_groups, int sms, cudaStream_t s);
-cudaError_t launch_gather_quant4(const void* x, int d, const int32_t* perm, const int32_t* idx, int k,
-                                 const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x4,
-                                 uint8_t* sx, int groups, int sms, cudaStream_t s);
 // NVFP4: g[m] = the tensor scale of matrix m (nmat matrices of mrows x cols, consecutive);
 // rows of src take gvec[r / rows_per_g] (gvec null: g_const)
 cudaError_t launch_nv4_global(int bf16, const void* src, int nmat, int64_t mrows, int cols, float* g, cudaStream_t s);
 cudaError_t launch_quant_nv4(int bf16, const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
                              int atom_groups, const float* gvec, int64_t rows_per_g, float g_const, int sms,
                              cudaStream_t s);
-cudaError_t launch_gather_quant_nv4(const void* x, int d, const int32_t* perm, const int32_t* idx, int k,
-                                    const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, uint8_t* x4,
-                                    uint8_t* sx, int groups, int sms, cudaStream_t s);
+// The FFN pairs' x rows quantized into the padded expert-order operand of the block-scaled
+// GEMM, one warp per token: fmt 0 FP8 [1,128], 1 MXFP4 [1,32], 2 NVFP4 [1,16] (g = 1)
+cudaError_t launch_scatter_quant(int fmt, const void* x, int d, const int32_t* pos, const int32_t* idx, int T, int k,
+                                 const int32_t* offsets, const int32_t* mb_off, uint8_t* codes, uint8_t* scales,
+                                 int groups, int sms, cudaStream_t s);
 cudaError_t launch_unpad_rows(const void* ypad, int row_bytes, const int32_t* perm, const int32_t* idx,
                               const int32_t* offsets, const int32_t* mb_off, const int32_t* scal, void* out, int sms,
                               cudaStream_t s);

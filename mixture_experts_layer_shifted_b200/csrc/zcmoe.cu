@@ -731,16 +731,11 @@ static int forward_impl(zcmoe_t h, const void* x, int64_t T, void* y, cudaStream
     if (rc != ZCMOE_OK) return rc;
   }
   ZC_CUDA(mark("zcmoe.gather"));
-  // 4. gather the FFN pairs' rows (FP8 layers: quantized per [1,128] into padded rows)
-  if (h->fp8 && h->fmt == 2)
-    ZC_CUDA(zc::launch_gather_quant_nv4(x, d, h->perm, h->idx, k, h->offsets, h->mb_off, h->scal, h->x8, h->sx, h->gd,
-                                        h->sms, s));
-  else if (h->fp8 && h->fmt)
-    ZC_CUDA(zc::launch_gather_quant4(x, d, h->perm, h->idx, k, h->offsets, h->mb_off, h->scal, h->x8, h->sx, h->gd,
+  // 4. the FFN pairs' rows in expert order, each token's row read once (FP8 / FP4 layers:
+  // quantized once per token into every padded row of it)
+  if (h->fp8)
+    ZC_CUDA(zc::launch_scatter_quant(h->fmt, x, d, h->pos, h->idx, Ti, k, h->offsets, h->mb_off, h->x8, h->sx, h->gd,
                                      h->sms, s));
-  else if (h->fp8)
-    ZC_CUDA(zc::launch_gather_quant(x, d, h->perm, h->idx, k, h->offsets, h->mb_off, h->scal, h->x8, h->sx, h->gd,
-                                    h->sms, s));
   else
     ZC_CUDA(zc::launch_scatter_rows(x, (int)(d * esz), h->pos, Ti, k, h->xperm, h->sms, s));
   ZC_CUDA(mark("zcmoe.gate_up"));
