@@ -412,21 +412,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const Unit u = decode_unit<MODE, C::kPair>(args, t);
       const bool two = C::kPair && u.rows[1] > 0;
       const int s0 = slot, s1 = slot ^ 1;
-      // each slot's accumulator must have been drained by the epilogue of its previous use
+      // Each slot's accumulator must have been drained by the epilogue of its previous use.  The
+      // epilogue frees a pair's slots in order, s0 first, so a pair's first row block starts on
+      // the staged k-blocks as soon as s0 is free; the second row block's MMAs on those k-blocks
+      // (which keep their stages until then) follow once s1 is free too.
       if (!warp_wait(&tempty[s0], (uses[s0] & 1) ^ 1u, err, 2)) break;
-      if (two && !warp_wait(&tempty[s1], (uses[s1] & 1) ^ 1u, err, 2)) break;
       tc_fence_after();
       const uint32_t d0 = tmem_base + (uint32_t)(s0 * C::kBN), d1 = tmem_base + (uint32_t)(s1 * C::kBN);
       // a row block of at most 64 valid rows runs M = 64 MMAs (about half the energy of
       // M = 128); its rows land in TMEM lanes 32q + (0..15), q = 0..3
       const uint32_t id0 = u.rows[0] <= 64 ? idesc64 : idesc128;
       const uint32_t id1 = u.rows[1] <= 64 ? idesc64 : idesc128;
+      const uint32_t par1 = (uses[s1] & 1) ^ 1u;
+      bool ready1 = !two;        // s1 free (or not needed)
+      int held = 0;              // leading k-blocks whose second-row-block MMAs wait for s1
+      const int stage0 = stage;  // the stage of the unit's first k-block
+      // second row block's MMAs of k-block kb staged at st, then release the stage (elected lane)
+      auto mma_second = [&](int kb, int st) {
+        const uint32_t b_addr = smem_u32(smem + st * C::kStageBytes);
+        const uint32_t a_addr = b_addr + C::kBBytes + A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          tc_mma_f16(d1, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), id1,
+                     (kb | kk) != 0 ? 1u : 0u);
+        tc_commit(&empty[st]);
+      };
       for (int kb = 0; kb < num_k; ++kb) {
+        if (!ready1 && held == STAGES) {  // every stage is held: wait for s1 now
+          if (!warp_wait(&tempty[s1], par1, err, 2)) {
+            ok = false;
+            break;
+          }
+          ready1 = true;
+          tc_fence_after();
+          if (elect_one())
+            for (int j = 0; j < held; ++j) mma_second(j, (stage0 + j) % STAGES);
+          __syncwarp();
+          held = 0;
+        }
         if (!warp_wait(&full[stage], phase, err, 3)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        if (!ready1) {
+          int r = 0;
+          if (lane == 0) r = mbar_try_wait(&tempty[s1], par1) ? 1 : 0;
+          ready1 = __shfl_sync(0xffffffffu, r, 0) != 0;
+          if (ready1) tc_fence_after();
+        }
         if (elect_one()) {
           const uint32_t b_addr = smem_u32(smem + stage * C::kStageBytes);
           const uint32_t a_addr = b_addr + C::kBBytes;
@@ -434,19 +468,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int kk = 0; kk < BK / 16; ++kk)
             tc_mma_f16(d0, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), id0,
                        (kb | kk) != 0 ? 1u : 0u);
-          if (two) {
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              tc_mma_f16(d1, sw128_kmajor_desc(a_addr + A_BYTES + kk * 32), sw128_kmajor_desc(b_addr + kk * 32),
-                         id1, (kb | kk) != 0 ? 1u : 0u);
+          if (!two) {
+            tc_commit(&empty[stage]);
+          } else if (ready1) {
+            for (int j = 0; j < held; ++j) mma_second(j, (stage0 + j) % STAGES);
+            mma_second(kb, stage);
           }
-          tc_commit(&empty[stage]);
         }
         __syncwarp();
+        if (two) held = ready1 ? 0 : held + 1;
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
         }
+      }
+      if (ok && !ready1) {  // a unit shorter than the held stages: s1 before the accumulators close
+        if (!warp_wait(&tempty[s1], par1, err, 2)) break;
+        tc_fence_after();
+        if (elect_one())
+          for (int j = 0; j < held; ++j) mma_second(j, (stage0 + j) % STAGES);
+        __syncwarp();
       }
       if (!ok) break;
       if (elect_one()) {
