@@ -80,6 +80,8 @@ struct Unit {
   int b_row;    // first B row
   int n_blk;    // output column tile
   int p_row;    // grouped modes: padded-layout row of the first row block (128 (mb_off[g] + block))
+  int keep_b;   // 1: an expert's odd last row block beside its pairs -- it streams the same weight tile
+                // ahead of them, so its weight lines are loaded with the L2 evict-last priority
 };
 
 template <int MODE, bool PAIR>
@@ -98,6 +100,7 @@ __device__ __forceinline__ Unit decode_unit(const TcArgs& a, int t) {
     u.rows[0] = min(BM, a.M - u.a_row);
     u.rows[1] = 0;
     u.b_row = u.n_blk * block_n<MODE>();
+    u.keep_b = 0;
     u.p_row = u.a_row;
     return u;
   }
@@ -121,6 +124,7 @@ __device__ __forceinline__ Unit decode_unit(const TcArgs& a, int t) {
   u.rows[0] = min(BM, end - u.a_row);
   u.rows[1] = PAIR ? max(0, min(BM, end - u.a_row - BM)) : 0;
   u.p_row = (a.mb_off[g] + m0) * BM;
+  u.keep_b = PAIR && u.rows[1] == 0 && nu > 1;
   u.b_row = g * a.b_rows_per_group + u.n_blk * (MODE == kGateUp ? BN / 2 : BN);
   return u;
 }
@@ -348,6 +352,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       int fills = 0;
       bool ok = true;
+      const uint64_t keep_policy = l2_policy_evict_last();
       for (int i = 0; i <= total && ok; ++i) {
         const int rs = i % RING;
         if (!mbar_wait(&uempty[rs], ((i / RING) & 1) ^ 1u, err, 10)) break;
@@ -367,11 +372,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint8_t* b_dst = smem + stage * C::kStageBytes;
           uint8_t* a_dst = b_dst + C::kBBytes;
           mbar_expect_tx(&full[stage], bytes);
-          if (MODE == kGateUp) {
-            tma_load_2d(b_dst, &tmB0, kb * BK, u.b_row, &full[stage]);
-            tma_load_2d(b_dst + C::kBBytes / 2, &tmB1, kb * BK, u.b_row, &full[stage]);
+          if (u.keep_b) {
+            tma_load_2d_hint(b_dst, &tmB0, kb * BK, u.b_row, &full[stage], keep_policy);
+            if (MODE == kGateUp)
+              tma_load_2d_hint(b_dst + C::kBBytes / 2, &tmB1, kb * BK, u.b_row, &full[stage], keep_policy);
           } else {
             tma_load_2d(b_dst, &tmB0, kb * BK, u.b_row, &full[stage]);
+            if (MODE == kGateUp) tma_load_2d(b_dst + C::kBBytes / 2, &tmB1, kb * BK, u.b_row, &full[stage]);
           }
           tma_load_2d(a_dst, &tmA, kb * BK, u.a_row, &full[stage]);
           if (two) tma_load_2d(a_dst + A_BYTES, &tmA, kb * BK, u.a_row + BM, &full[stage]);
