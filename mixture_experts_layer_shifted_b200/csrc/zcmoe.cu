@@ -515,7 +515,7 @@ static int create_impl(const zcmoe_config* cfg, const zcmoe_weights* w, int ep_r
       if (e == cudaSuccess) e = cudaMemset(h->h8, 0, prow * h->inter / (h->fmt ? 2 : 1));
       if (e == cudaSuccess) e = cudaMemset(h->sx, 0, (size_t)h->max_mblocks * h->gd * zc::kAtomBytes);
       if (e == cudaSuccess) e = cudaMemset(h->sh, 0, (size_t)h->max_mblocks * h->gi * zc::kAtomBytes);
-      // the expert weights, quantized into scale atoms: FP8 per [128,128], MXFP4 per [1,32]
+      // the expert weights, quantized into scale atoms: FP8 per [128,128], MXFP4 per [1,32], NVFP4 per [1,16]
       const int64_t ri = (int64_t)N * h->inter, rd = (int64_t)N * h->d;
       if (h->fmt == 2) {
         // one fp32 tensor scale per expert matrix, then [1,16] blocks under it
