@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         if (!ready1) {
           int r = 0;
-          if (lane == 0) r = mbar_try_wait(&tempty[s1], par1) ? 1 : 0;
+          if (lane == 0) r = mbar_poll(&tempty[s1], par1) ? 1 : 0;
           ready1 = __shfl_sync(0xffffffffu, r, 0) != 0;
           if (ready1) tc_fence_after();
         }

@@ -62,6 +62,9 @@ __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int code) {
   return mbar_wait_limit(bar, parity, err, code, kWaitLimitNs);
 }
+// One poll, no loop: whether the phase with the given parity has completed by now (a caller
+// that must have it waits with mbar_wait).
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity) { return mbar_try_wait(bar, parity); }
 
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* tm) {
