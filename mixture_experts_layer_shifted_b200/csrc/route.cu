@@ -29,12 +29,13 @@ template <int EPL>
 __global__ void __launch_bounds__(256, 3) k_softmax_topk(const float* __restrict__ logits, const float* __restrict__ bias,
                                                          int T, int E, int k, float scale, int32_t* __restrict__ idx,
                                                          float* __restrict__ gate, float* __restrict__ scores) {
+  __shared__ uint32_t slots[8][96];  // per warp: the candidates' keys, ids and scores
   const int lane = threadIdx.x & 31;
   const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
   for (int t = warp; t < T; t += nwarps)
     route_token<EPL>(logits + (int64_t)t * E, bias, E, k, scale, idx + (int64_t)t * k, gate + (int64_t)t * k,
-                     scores ? scores + (int64_t)t * E : nullptr, lane);
+                     scores ? scores + (int64_t)t * E : nullptr, lane, slots[threadIdx.x >> 5]);
 }
 
 // Router backward, one warp per token: the scores s are recomputed from the

@@ -70,20 +70,21 @@ __device__ __forceinline__ bool ranks_before(uint32_t a, uint32_t ea, uint32_t b
 
 // One token, one warp (all 32 lanes call it).  EPL = experts held per lane (E <= 32 EPL);
 // lane p holds experts p, p + 32, ...  lt: the token's E logits; writes idx_row[0..k),
-// gate_row[0..k) and, if scores_row is not null, its E scores.  Selection, exact, in
-// two steps:
+// gate_row[0..k) and, if scores_row is not null, its E scores.  slots: this warp's 96 words
+// of shared memory.  Selection, exact, in two steps:
 //  1. threshold: the k-th largest of the 32 lane maxima (ties counted), tau.  At least
 //     k lanes hold a key >= tau, so every one of the k picks has a key >= tau;
-//  2. the candidates (key >= tau) are compacted into one slot per lane and sorted by
-//     (key descending, id ascending) with a 32-lane bitonic network; lanes 0..k-1 then
-//     hold the picks in slot order.
+//  2. the candidates (key >= tau) are compacted into one slot per lane -- each lane writes
+//     its own at the prefix of the lanes' counts -- and sorted by (key descending, id
+//     ascending) with a 32-lane bitonic network; lanes 0..k-1 then hold the picks in slot
+//     order (the sort makes the order of the slots before it irrelevant).
 // When more than 32 candidates reach tau (ties at the threshold, e.g. a row of NaN
 // scores), the picks are taken one by one instead: a warp max of the lanes' best
 // untaken keys, then a warp min of the ids holding it, the winning lane rescanning.
 template <int EPL>
 __device__ __forceinline__ void route_token(const float* __restrict__ lt, const float* __restrict__ bias, int E, int k,
                                             float scale, int32_t* __restrict__ idx_row, float* __restrict__ gate_row,
-                                            float* __restrict__ scores_row, int lane) {
+                                            float* __restrict__ scores_row, int lane, uint32_t* __restrict__ slots) {
   float u[EPL];
   float m = -__int_as_float(0x7f800000);
 #pragma unroll
@@ -123,29 +124,36 @@ __device__ __forceinline__ void route_token(const float* __restrict__ lt, const 
     tau = g;
   }
   // 2. compaction of the candidates: lane c receives the c-th one (key, id, score)
+  int mine = 0;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) mine += key[i] >= tau ? 1 : 0;
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int count = __shfl_sync(0xffffffffu, incl, 31);
   uint32_t ck = 0u, ce = 0xffffffffu;
   float cs = 0.0f;
-  int count = 0;
+  if (count <= 32) {
+    int at = incl - mine;  // this lane's first slot
 #pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const bool c = key[i] >= tau;
-    const uint32_t ballot = __ballot_sync(0xffffffffu, c);
-    const int base = count;
-    count += __popc(ballot);
-    if (ballot == 0u) continue;
-    // the candidates of this row go to slots base, base + 1, ... in lane order: lane L
-    // receives slot L, i.e. the candidate of rank L - base, held by the lane of the
-    // (L - base + 1)-th set bit of the ballot
-    const int rank = lane - base;
-    const bool recv = rank >= 0 && rank < __popc(ballot);
-    const int src = recv ? (int)__fns(ballot, 0, rank + 1) : 0;
-    const uint32_t vk = __shfl_sync(0xffffffffu, key[i], src);
-    const float vs = __shfl_sync(0xffffffffu, u[i], src);
-    if (recv) {
-      ck = vk;
-      ce = (uint32_t)(src + 32 * i);
-      cs = vs;
+    for (int i = 0; i < EPL; ++i) {
+      if (key[i] >= tau) {
+        slots[at] = key[i];
+        slots[32 + at] = (uint32_t)(lane + 32 * i);
+        slots[64 + at] = __float_as_uint(u[i]);
+        ++at;
+      }
     }
+    __syncwarp();
+    if (lane < count) {
+      ck = slots[lane];
+      ce = slots[32 + lane];
+      cs = __uint_as_float(slots[64 + lane]);
+    }
+    __syncwarp();  // every lane has read its slot before the warp's next token writes them
   }
   int my_idx = 0;
   float my_gate = 0.0f;
