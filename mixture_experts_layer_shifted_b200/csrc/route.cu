@@ -11,7 +11,7 @@
 //    fused softmax + top-k + scaling step.
 //
 // The routing of a token (softmax, bias-shifted top-k, gates) and its written
-// fp32 rule live in zc_route.cuh, shared with the router GEMM's fused epilogue.
+// fp32 rule live in zc_route.cuh.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>

@@ -1,6 +1,7 @@
 // Routing of one token by one warp: softmax over the router logits, top-k on the
-// bias-shifted scores, the gates.  Shared by the stand-alone routing kernel and the
-// router GEMM, which runs it in its epilogue warps (the routing fused into the GEMM).
+// bias-shifted scores, the gates.  Run by the routing kernel (k_softmax_topk); it is kept in
+// a header of its own so that any kernel that routes (a router GEMM epilogue was one such
+// variant, measured slower) follows the same rule.
 //
 // Sources (page title, section):
 //  - LongCat-Flash technical summary (zhangjingwei.cn), 二 架構, part 1
