@@ -225,7 +225,8 @@ ZCMOE_API int zcmoe_selftest_wait(zcmoe_t h, int64_t limit_ns, cudaStream_t stre
  * zcmoe_profile_end synchronises, writes per-stage device time summed over the
  * recorded forwards into ms[ZCMOE_NUM_STAGES] (host) and the number of forwards
  * into *n_forwards, and stops recording.  Stages, in order: router GEMM,
- * softmax/top-k, integer stage, row gather, gate/up GEMM, down GEMM, combine. */
+ * softmax/top-k, integer stage, the copy of the FFN pairs' rows into expert order
+ * (quantized for FP8 / FP4 layers), gate/up GEMM, down GEMM, combine. */
 #define ZCMOE_NUM_STAGES 7
 ZCMOE_API int zcmoe_profile_begin(zcmoe_t h);
 ZCMOE_API int zcmoe_profile_end(zcmoe_t h, float *ms, int32_t *n_forwards);
@@ -315,7 +316,7 @@ ZCMOE_API int zcmoe_save_for_backward(zcmoe_t h, int32_t on);
  * ep_size ranks holds FFN experts [r * n_local, (r + 1) * n_local), n_local = n_ffn / ep_size;
  * every rank routes its own tokens over all n_ffn + n_zero experts.  A forward is three calls
  * with two exchanges between them, which the caller runs (NCCL all-to-all, for example):
- *   1. zcmoe_ep_dispatch: routing and the gather of the FFN pairs' rows, in expert order,
+ *   1. zcmoe_ep_dispatch: routing and the copy of the FFN pairs' rows into expert order,
  *      so the rows for rank r are the contiguous block of its experts;
  *   exchange the per-expert counts and the rows (rank r gets its experts' rows);
  *   2. zcmoe_ep_experts: the local experts on the received rows;
@@ -450,7 +451,7 @@ ZCMOE_API int zcmoe_dense_forward(zcmoe_dense_t h, const void *x, int64_t T, voi
  * The dense FFN runs on the dense handle's internal stream, forked from and
  * joined back into `stream`: its gate/up GEMM starts when the MoE router GEMM
  * has finished and runs beside the MoE's memory-bound stages (softmax/top-k,
- * integer stage, row gather); its down GEMM starts when the MoE down GEMM has
+ * integer stage, row copy); its down GEMM starts when the MoE down GEMM has
  * finished and runs beside the combine.  When the call returns, all the work of
  * both is ordered before anything later enqueued on `stream`, so the call can
  * be captured into a CUDA graph on `stream`.

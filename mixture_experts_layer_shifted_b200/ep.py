@@ -133,7 +133,7 @@ def ep_forward(stages_per_chunk, comm, x, n_ffn: int, dense=None, x_dense=None, 
     T = x.shape[0]
     bounds = [T * i // nck for i in range(nck + 1)]
     chunks = [_Chunk(x[bounds[i]:bounds[i + 1]], st) for i, st in enumerate(stages_per_chunk)]
-    # 1: every chunk's routing and row gather
+    # 1: every chunk's routing and the copy of its FFN pairs' rows into expert order
     offs = torch.empty((nck, n_ffn + 1), dtype=torch.int32, device=x.device)
     for i, c in enumerate(chunks):
         c.xsend = c.stages.dispatch(c.x, offs[i], debug[i] if debug else None)
