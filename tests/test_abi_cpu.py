@@ -241,6 +241,7 @@ def test_create_checks_quantized_shapes_scale_and_group_on_the_host(zc):
 
     for bad in [dict(dtype=zc.ZCMOE_FP8, d=256), dict(dtype=zc.ZCMOE_FP8, inter=192),
                 dict(dtype=zc.ZCMOE_FP4, d=768), dict(dtype=zc.ZCMOE_FP4, inter=128),
+                dict(dtype=zc.ZCMOE_NVFP4, d=768), dict(dtype=zc.ZCMOE_NVFP4, inter=128),
                 dict(routed_scale=math.nan), dict(routed_scale=math.inf)]:
         assert lib.zcmoe_create(ctypes.byref(cfg(**bad)), ctypes.byref(w), ctypes.byref(h)) == zc.ZCMOE_EINVAL, bad
         assert h.value is None
@@ -249,8 +250,42 @@ def test_create_checks_quantized_shapes_scale_and_group_on_the_host(zc):
         assert lib.zcmoe_create_ep(ctypes.byref(c), ctypes.byref(w), rank, size, cap, ctypes.byref(h)) == \
             zc.ZCMOE_EINVAL, (rank, size, cap)
         assert h.value is None
-    assert lib.zcmoe_create_ep(ctypes.byref(cfg(dtype=zc.ZCMOE_FP8)), ctypes.byref(w), 0, 2, 0,
-                               ctypes.byref(h)) == zc.ZCMOE_EUNSUPPORTED
+    for dt in (zc.ZCMOE_FP8, zc.ZCMOE_FP4, zc.ZCMOE_NVFP4):
+        assert lib.zcmoe_create_ep(ctypes.byref(cfg(dtype=dt)), ctypes.byref(w), 0, 2, 0,
+                                   ctypes.byref(h)) == zc.ZCMOE_EUNSUPPORTED
+
+
+def test_quantizers_refuse_bad_arguments_on_the_host(zc):
+    """zcmoe_quantize_e4m3 / _mx4 / _nv4 check dtype, shape, pointers, alignment and (NVFP4) the
+    tensor scale before they touch the device; zero rows is a no-op."""
+    import math
+    lib = zc.lib()
+    p16 = ctypes.c_void_p(0x10000)   # never dereferenced: every call below is refused first
+    p_odd = ctypes.c_void_p(0x10008)
+    BF16, F32 = zc.ZCMOE_BF16, zc.ZCMOE_F32
+    E = zc.ZCMOE_EINVAL
+    # E4M3: cols a multiple of 128, block_rows 1 or 128
+    assert lib.zcmoe_quantize_e4m3(p16, 7, 4, 128, 1, p16, p16, None) == E
+    assert lib.zcmoe_quantize_e4m3(p16, BF16, 4, 100, 1, p16, p16, None) == E
+    assert lib.zcmoe_quantize_e4m3(p16, BF16, 4, 128, 64, p16, p16, None) == E
+    assert lib.zcmoe_quantize_e4m3(None, BF16, 4, 128, 1, p16, p16, None) == E
+    assert lib.zcmoe_quantize_e4m3(p_odd, BF16, 4, 128, 1, p16, p16, None) == E
+    assert lib.zcmoe_quantize_e4m3(None, BF16, 0, 128, 1, None, None, None) == zc.ZCMOE_OK
+    # MXFP4: cols a multiple of 256
+    assert lib.zcmoe_quantize_mx4(p16, F32, 4, 128, p16, p16, None) == E
+    assert lib.zcmoe_quantize_mx4(p16, 3, 4, 256, p16, p16, None) == E
+    assert lib.zcmoe_quantize_mx4(p16, BF16, 4, 256, None, p16, None) == E
+    assert lib.zcmoe_quantize_mx4(p16, BF16, 4, 256, p_odd, p16, None) == E
+    assert lib.zcmoe_quantize_mx4(None, BF16, 0, 256, None, None, None) == zc.ZCMOE_OK
+    # NVFP4: cols a multiple of 256; the tensor scale finite and >= 0; 0 derives it and needs global_out
+    assert lib.zcmoe_quantize_nv4(p16, BF16, 4, 128, 1.0, p16, p16, None, None) == E
+    for g in (-1.0, math.nan, math.inf):
+        assert lib.zcmoe_quantize_nv4(p16, BF16, 4, 256, g, p16, p16, p16, None) == E, g
+    assert lib.zcmoe_quantize_nv4(p16, BF16, 4, 256, 0.0, p16, p16, None, None) == E
+    assert lib.zcmoe_quantize_nv4(p16, BF16, 4, 256, 0.0, p16, p16, ctypes.c_void_p(0x10002), None) == E
+    assert lib.zcmoe_quantize_nv4(p16, 5, 4, 256, 1.0, p16, p16, None, None) == E
+    assert lib.zcmoe_quantize_nv4(p_odd, BF16, 4, 256, 1.0, p16, p16, None, None) == E
+    assert lib.zcmoe_quantize_nv4(None, BF16, 0, 256, 1.0, None, None, None, None) == zc.ZCMOE_OK
 
 
 def test_noalloc_refuses_on_the_host_at_its_exact_limits(zc):
