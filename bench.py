@@ -432,7 +432,9 @@ def run_ep(args, wl, dist, rank, ws, local, peaks):
         torch.cuda.empty_cache()
     comm = TorchComm() if dist else LocalComm()
     # rows one chunk's experts call may receive: twice a chunk's own FFN pairs (about 3x the balanced share)
-    nck = max(1, args.ep_chunks)
+    # chunks per step: the pages cut the layer in two so that one chunk's exchange overlaps the
+    # other's experts; a one-rank group has no exchange to hide, so it runs one chunk unless asked
+    nck = max(1, args.ep_chunks if args.ep_chunks > 0 else (2 if ws > 1 else 1))
     cap = 2 * wl.T * wl.top_k // nck
     layer = EpMoE(shape, wr, wg, wu, wd, max_tokens=wl.T, comm=comm, chunks=nck, max_recv_rows=cap,
                   init_bias=configs.bias_vector(wl), logit_offset=configs.logit_offsets(wl))
@@ -558,7 +560,8 @@ def main():
                     help="comma list of the secondary measurements to run after the headline")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism over the GPUs (ep.py) instead of data-parallel replicas")
-    ap.add_argument("--ep-chunks", type=int, default=2, help="--ep: token chunks per step")
+    ap.add_argument("--ep-chunks", type=int, default=0,
+                    help="--ep: token chunks per step (default: 2 with more than one rank, 1 with one)")
     ap.add_argument("--eager", action="store_true",
                     help="launch every step eagerly instead of replaying one captured CUDA graph (N=1)")
     args = ap.parse_args()
