@@ -81,7 +81,8 @@ struct Unit {
   int n_blk;    // output column tile
   int p_row;    // grouped modes: padded-layout row of the first row block (128 (mb_off[g] + block))
   int keep_b;   // 1: an expert's odd last row block beside its pairs -- it streams the same weight tile
-                // ahead of them, so its weight lines are loaded with the L2 evict-last priority
+                // ahead of them, so its weight lines are loaded with the L2 evict-last priority;
+                // 2: a pair of such an expert -- the last reader of those lines, so evict-first
 };
 
 template <int MODE, bool PAIR>
@@ -124,7 +125,8 @@ __device__ __forceinline__ Unit decode_unit(const TcArgs& a, int t) {
   u.rows[0] = min(BM, end - u.a_row);
   u.rows[1] = PAIR ? max(0, min(BM, end - u.a_row - BM)) : 0;
   u.p_row = (a.mb_off[g] + m0) * BM;
-  u.keep_b = PAIR && u.rows[1] == 0 && nu > 1;
+  const int mb = a.mb_off[g + 1] - a.mb_off[g];
+  u.keep_b = !PAIR || (mb & 1) == 0 || mb < 3 ? 0 : (u.rows[1] == 0 ? 1 : 2);
   u.b_row = g * a.b_rows_per_group + u.n_blk * (MODE == kGateUp ? BN / 2 : BN);
   return u;
 }
@@ -352,7 +354,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       int fills = 0;
       bool ok = true;
-      const uint64_t keep_policy = l2_policy_evict_last();
+      const uint64_t keep_policy = l2_policy_evict_last(), drop_policy = l2_policy_evict_first();
       for (int i = 0; i <= total && ok; ++i) {
         const int rs = i % RING;
         if (!mbar_wait(&uempty[rs], ((i / RING) & 1) ^ 1u, err, 10)) break;
@@ -373,9 +375,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint8_t* a_dst = b_dst + C::kBBytes;
           mbar_expect_tx(&full[stage], bytes);
           if (u.keep_b) {
-            tma_load_2d_hint(b_dst, &tmB0, kb * BK, u.b_row, &full[stage], keep_policy);
-            if (MODE == kGateUp)
-              tma_load_2d_hint(b_dst + C::kBBytes / 2, &tmB1, kb * BK, u.b_row, &full[stage], keep_policy);
+            const uint64_t pol = u.keep_b == 1 ? keep_policy : drop_policy;
+            tma_load_2d_hint(b_dst, &tmB0, kb * BK, u.b_row, &full[stage], pol);
+            if (MODE == kGateUp) tma_load_2d_hint(b_dst + C::kBBytes / 2, &tmB1, kb * BK, u.b_row, &full[stage], pol);
           } else {
             tma_load_2d(b_dst, &tmB0, kb * BK, u.b_row, &full[stage]);
             if (MODE == kGateUp) tma_load_2d(b_dst + C::kBBytes / 2, &tmB1, kb * BK, u.b_row, &full[stage]);
